@@ -1,0 +1,401 @@
+"""Benchmark of the GDN-2 chunkwise recurrence on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline: forward tokens/s on the single-layer workload of the pages' 1.3B
+model (B=8, H=16, T=4096, d_k=d_v=128, bf16 inputs, fp32 log-decay and state;
+a token covers all 16 heads).  A step is one gdn2_chunk_fwd call over the
+batch, inputs resident in HBM (1.09 GB per step, larger than the 126 MB L2, so
+no flush is needed).  The same line carries the forward+backward figure on the
+same batch (`fwd_bwd`), the decode figure (`decode`, 256 sequences, 1024
+steps) and the roofline fraction of each, plus:
+
+* `e2e`: the same forward through the public binding with host buffers:
+  pinned-host inputs copied in and o/S_T copied out inside the timed region;
+* `cpu_baseline`: the fp64 oracle timed on a bounded sample on the host cores;
+* `clocks`: SM clock and throttle reasons sampled during the timed regions.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+independent (batch, head) sequences; there is no collective on the data path
+(weak scaling).  Timing is by CUDA events, max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this method
+has: the pages publish no code) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic_inputs import DECODE_WORKLOAD, WORKLOADS, DecodeStream, make_inputs  # noqa: E402
+
+METRIC = "GDN-2 fwd/fwd+bwd tokens/s (H=16,d=128,T=4K); decode steps/s; % of roofline"
+CHUNK = 64
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------ peaks / roofline
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def fwd_bytes(B, T, H, D):
+    """Algorithmic bytes of one forward: per token-head q,k,v,b,w (bf16) + log alpha (fp32)
+    read and o (bf16) written = 2048 B at D=128; plus S0 read and S_T written (fp32)."""
+    per_tok_head = 5 * 2 * D + 4 * D + 2 * D
+    return B * T * H * per_tok_head + B * H * 2 * D * D * 4
+
+
+def bwd_bytes(B, T, H, D):
+    """Per token-head: q,k,v,b,w,do read and dq,dk,dv,db,dw written (bf16), log alpha read
+    and its gradient written (fp32); plus S0 read and dS0 written (dS_T = 0 is not read)."""
+    per_tok_head = 11 * 2 * D + 2 * 4 * D
+    return B * T * H * per_tok_head + B * H * 2 * D * D * 4
+
+
+def decode_bytes(N, H, D):
+    """State read + written (fp32), q,k,v,b,w read and o written (bf16), log alpha (fp32)."""
+    return N * H * (2 * D * D * 4 + 6 * 2 * D + 4 * D)
+
+
+def fwd_flops(B, T, H, D, C=CHUNK):
+    """Dense-tile flops per token-head: 5 C x C x d products (A, W, U, P, P U~) and
+    3 C x d x d products (W S, Q~ S, K^^T U~) per chunk = 10 C d + 6 d^2."""
+    return B * T * H * (10 * C * D + 6 * D * D)
+
+
+def kernel_traffic(kernel_src: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of the kernel (same SHA-256), else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", kernel_src)
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    e = d.get(kernel_src)
+    if not e or e.get("sha256") != h:
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.dev = device_index
+
+    def _gpu_id(self):
+        try:
+            u = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return str(self.dev)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self._gpu_id()],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines += [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        busy = [x for x in sm if x > 0.5 * (smax or max(sm))] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ timing helpers
+def time_region(fn, steps, warmup, stream):
+    for _ in range(warmup):
+        fn()
+    stream.synchronize()
+    if torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if torch.distributed.is_initialized():
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    return ms
+
+
+def roofline(bytes_per_launch, ms_per_launch, pk, traffic=None, bound="hbm"):
+    achieved = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+            "algorithmic_bytes": bytes_per_launch, "peak_source": pk["source"] + " (burst copy)"}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_baseline(w, target_s=12.0, seed=0):
+    """Time the fp64 oracle forward on a bounded sample of (batch, head) sequences of the
+    workload (full length T), sized for about `target_s` seconds of host work."""
+    import oracle  # test infrastructure: only this leg of the benchmark runs it
+    cores = oracle.default_threads()
+    T, D = w["T"], w["Dk"]
+    one = make_inputs(1, T, 1, D, D, dtype=w["dtype"], seed=seed)
+    t0 = time.perf_counter()
+    oracle.ref_fwd(one["q"], one["k"], one["v"], one["log_alpha"], one["b"], one["w"], one["S0"], nthreads=1)
+    per_seq = time.perf_counter() - t0
+    nseq = max(cores, min(w["B"] * w["H"], int(target_s * cores / max(per_seq, 1e-3))))
+    nseq = (nseq // cores) * cores or cores
+    x = make_inputs(1, T, nseq, D, D, dtype=w["dtype"], seed=seed + 1)
+    t0 = time.perf_counter()
+    oracle.ref_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], nthreads=cores)
+    dt = time.perf_counter() - t0
+    tokens = nseq * T / w["H"]  # a token covers all H heads
+    return {"value": round(tokens / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 token-recurrence forward of {nseq} (batch, head) sequences of "
+                      f"T={T}, d={D} ({nseq / w['H']:.2f} batch rows of H={w['H']}), {dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = dict(WORKLOADS[args.workload])
+    cores = oracle.default_threads()
+    T, D, H = w["T"], w["Dk"], w["H"]
+    # one step = one batch row of the workload (all H heads, full length T)
+    x = make_inputs(1, T, H, D, D, dtype=w["dtype"], seed=0)
+    arg = (x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    for _ in range(args.warmup):
+        oracle.ref_fwd(*arg, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.ref_fwd(*arg, nthreads=cores)
+    dt = time.perf_counter() - t0
+    value = args.steps * T / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "B_per_step": 1, "T": T, "H": H, "d": D,
+                       "note": "each step is one batch row (all heads) of the workload"},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps x 1 batch row (H={H}, T={T}, d={D})"},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import gated_delta_rule_78_b200 as g
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    g.load()
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    w = dict(WORKLOADS[args.workload])
+    B, T, H, D = w["B"], w["T"], w["H"], w["Dk"]
+    tokens = B * T  # per rank
+    clocks = ClockSampler(dev.index)
+
+    # ---- forward (headline)
+    x = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=1234 + rank, device=str(dev), with_do=True)
+    o = torch.empty_like(x["v"])
+    ST = torch.empty_like(x["S0"])
+
+    def fwd():
+        g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], o=o, S_T=ST)
+
+    clocks.start()
+    ms_fwd = time_region(fwd, args.steps, args.warmup, stream) / args.steps
+    assert g.gdn2_sync_status() == 0, "a kernel reported a timeout"
+    fb = fwd_bytes(B, T, H, D)
+    value = world * tokens / (ms_fwd * 1e-3)
+
+    # ---- forward + backward on the same batch
+    extras = {}
+    if not args.fwd_only:
+        nws = g.gdn2_workspace_size(1, x["q"].dtype, B, T, H, D, D)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+        grads = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
+                 "dlog_alpha": torch.empty_like(x["log_alpha"]), "db": torch.empty_like(x["b"]),
+                 "dw": torch.empty_like(x["w"]), "dS0": torch.empty_like(x["S0"])}
+
+        def bwd():
+            g.gdn2_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], x["do"],
+                             None, workspace=ws, out=grads)
+
+        ksteps = max(3, args.steps // 4)
+        ms_bwd = time_region(bwd, ksteps, max(3, args.warmup // 2), stream) / ksteps
+        assert g.gdn2_sync_status() == 0
+        bb = bwd_bytes(B, T, H, D)
+        ms_fb = ms_fwd + ms_bwd
+        extras["fwd_bwd"] = {
+            "value": round(world * tokens / (ms_fb * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms_fb, 4), "bwd_ms": round(ms_bwd, 4), "steps": ksteps,
+            "roofline": roofline(fb + bb, ms_fb, pk), "bwd_roofline": roofline(bb, ms_bwd, pk),
+            "launches_per_step": 1 + 3}
+        del ws, grads
+
+        # ---- decode: 256 sequences, 1024 steps, per-step inputs resident
+        dw = DECODE_WORKLOAD
+        N, Hd, Dd, nsteps = dw["N"], dw["H"], dw["Dk"], dw["steps"]
+        ds = DecodeStream(N, Hd, Dd, Dd, dtype=dw["dtype"], seed=99 + rank, device=str(dev))
+        S = ds.S0
+        steps_in = [ds.step() for _ in range(nsteps)]
+        od = torch.empty(N, Hd, Dd, dtype=torch.bfloat16, device=dev)
+        it = {"i": 0}
+
+        def dec():
+            s = steps_in[it["i"] % nsteps]
+            it["i"] += 1
+            g.gdn2_decode_step(s["q"], s["k"], s["v"], s["log_alpha"], s["b"], s["w"], S, o=od)
+
+        ms_all = time_region(dec, nsteps, 16, stream)
+        assert g.gdn2_sync_status() == 0
+        ms_dec = ms_all / nsteps
+        extras["decode"] = {
+            "value": round(world * 1e3 / ms_dec, 1), "unit": "steps/s",
+            "tokens_per_s": round(world * N * 1e3 / ms_dec, 1), "us_per_step": round(ms_dec * 1e3, 3),
+            "steps": nsteps, "workload": f"N={N}, H={Hd}, d={Dd}, fp32 state in place",
+            "roofline": roofline(decode_bytes(N, Hd, Dd), ms_dec, pk, kernel_traffic("decode.cu")),
+            "launches_per_step": 1}
+        del steps_in
+    clocks.stop()
+
+    # ---- end to end through the binding with host buffers
+    hx = {n: t.to("cpu").pin_memory() for n, t in x.items() if n != "do"}
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hS = torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True)
+    dx = {n: torch.empty_like(t) for n, t in x.items() if n != "do"}
+
+    def e2e():
+        for n in dx:
+            dx[n].copy_(hx[n], non_blocking=True)
+        g.gdn2_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["log_alpha"], dx["b"], dx["w"], dx["S0"], o=o, S_T=ST)
+        ho.copy_(o, non_blocking=True)
+        hS.copy_(ST, non_blocking=True)
+
+    ke = max(3, args.steps // 4)
+    ms_e2e = time_region(e2e, ke, 2, stream) / ke
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = o.numel() * o.element_size() + ST.numel() * ST.element_size()
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_fwd, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "T": T, "H": H, "d_k": D, "d_v": D, "chunk": CHUNK,
+                   "inputs": "bf16 q,k,v,b,w; fp32 log alpha and state; S0 ~ N(0, 0.02)",
+                   "l2": f"inputs exceed L2 ({fb / 1e9:.2f} GB per step vs 126 MB): no flush",
+                   "parallelism": f"dp{world}: independent (batch, head) sequences per rank, no collective"},
+        "e2e": {"value": round(world * tokens / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3)},
+        "gpu_launches": args.steps,
+        "roofline": roofline(fb, ms_fwd, pk, kernel_traffic("fwd_tc.cu")),
+        "flops_per_step": fwd_flops(B, T, H, D),
+        "tensor_frac": round(fwd_flops(B, T, H, D) / (ms_fwd * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+        "clocks": clocks.summary(),
+    }
+    line.update(extras)
+    if world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="layer_4k", choices=sorted(WORKLOADS))
+    ap.add_argument("--fwd-only", action="store_true", help="skip the fwd+bwd and decode figures")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    args.steps = max(1, args.steps)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

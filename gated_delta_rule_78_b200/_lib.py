@@ -1,0 +1,177 @@
+"""ctypes binding of libgdn2.so: argument marshalling only.
+
+Every function here takes torch CUDA tensors, checks dtypes/devices, turns
+them into raw pointers and calls the C entry point of the same name.  All
+arithmetic runs in the library's CUDA kernels; nothing here computes.  If the
+library cannot be loaded, every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+
+GDN2_OK = 0
+STATUS_NAMES = {0: "GDN2_OK", -1: "GDN2_ERR_NULL", -2: "GDN2_ERR_SHAPE", -3: "GDN2_ERR_DTYPE",
+                -4: "GDN2_ERR_ALIGN", -5: "GDN2_ERR_WORKSPACE", -6: "GDN2_ERR_CUDA",
+                -7: "GDN2_ERR_TIMEOUT", -8: "GDN2_ERR_UNSUPPORTED"}
+GDN2_F32, GDN2_BF16 = 0, 1
+EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
+           "gdn2_strerror", "gdn2_sync_status")
+
+_lib = None
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = raw().gdn2_strerror(status).decode() if _lib is not None else ""
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+def load(path: str | None = None):
+    """Load libgdn2.so (raises OSError if it is missing: build it first)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise OSError(f"{path} not found: run gated_delta_rule_78_b200/build.py (or __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gdn2_chunk_fwd.argtypes = [i] * 6 + [vp] * 10 + [sz, vp]
+    lib.gdn2_chunk_fwd.restype = i
+    lib.gdn2_decode_step.argtypes = [i] * 5 + [vp] * 8 + [vp]
+    lib.gdn2_decode_step.restype = i
+    lib.gdn2_chunk_bwd.argtypes = [i] * 6 + [vp] * 17 + [sz, vp]
+    lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_workspace_size.argtypes = [i] * 7
+    lib.gdn2_workspace_size.restype = sz
+    lib.gdn2_strerror.argtypes = [i]
+    lib.gdn2_strerror.restype = ctypes.c_char_p
+    lib.gdn2_sync_status.argtypes = [vp]
+    lib.gdn2_sync_status.restype = i
+    _lib = lib
+    return lib
+
+
+def raw():
+    """The loaded ctypes library object (C names, raw pointers)."""
+    return load()
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN2_F32
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _check(fn: str, st: int):
+    if st != GDN2_OK:
+        raise Gdn2Error(fn, st)
+
+
+def _cuda_contig(name, t, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def gdn2_workspace_size(which: int, dtype: torch.dtype, B: int, T: int, H: int, Dk: int, Dv: int) -> int:
+    dt = GDN2_F32 if dtype == torch.float32 else GDN2_BF16
+    return int(raw().gdn2_workspace_size(which, dt, B, T, H, Dk, Dv))
+
+
+def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_state=True,
+                   workspace=None, stream=None):
+    """Chunkwise forward.  Returns (o, S_T); S_T is None when want_state is False."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    if o is None:
+        o = torch.empty(B, T, H, Dv, dtype=q.dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)
+    ws = workspace
+    st = raw().gdn2_chunk_fwd(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                              _p(S0), _p(o), _p(S_T), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                              _stream(stream))
+    _check("gdn2_chunk_fwd", st)
+    return o, S_T
+
+
+def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
+    """One decode step; S [N,H,Dk,Dv] fp32 is updated in place.  Returns o [N,H,Dv]."""
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S", S, torch.float32)
+    if o is None:
+        o = torch.empty(N, H, Dv, dtype=q.dtype, device=q.device)
+    st = raw().gdn2_decode_step(dt, N, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                _p(S), _p(o), _stream(stream))
+    _check("gdn2_decode_step", st)
+    return o
+
+
+def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace=None, out=None, stream=None):
+    """Gate-aware backward.  Returns dict(dq, dk, dv, dlog_alpha, db, dw, dS0)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("d_o", d_o)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    _cuda_contig("dS_T", dS_T, torch.float32)
+    if out is None:
+        out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+               "dlog_alpha": torch.empty_like(log_alpha), "db": torch.empty_like(b),
+               "dw": torch.empty_like(w),
+               "dS0": torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)}
+    if workspace is None:
+        nbytes = gdn2_workspace_size(1, q.dtype, B, T, H, Dk, Dv)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    st = raw().gdn2_chunk_bwd(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                              _p(S0), _p(d_o), _p(dS_T), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                              _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]), _p(out["dS0"]),
+                              _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn2_chunk_bwd", st)
+    return out
+
+
+def gdn2_sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the kernel status word."""
+    return int(raw().gdn2_sync_status(_stream(stream)))
+
+
+def gdn2_strerror(status: int) -> str:
+    return raw().gdn2_strerror(status).decode()

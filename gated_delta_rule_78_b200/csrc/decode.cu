@@ -1,0 +1,130 @@
+// Single-token GDN-2 decode step: S <- (I - k (b.k)^T) Diag(alpha) S + k (w.v)^T in place,
+// o = S^T q, for N sequences x H heads.
+//
+// The state (D x D fp32 per sequence-head, 64 KiB at D = 128) is the whole
+// cost: it is read once and written once, so the kernel streams it.  One CTA
+// owns one (sequence, head); its 8 warps each hold D/8 state rows in
+// registers, each lane a 16-byte (D = 128) or 8-byte (D = 64) column slice,
+// so every warp-wide access is one contiguous row segment.
+//   S'  = Diag(alpha) S                     in registers
+//   r   = S'^T (b.k),  p = S'^T q           per-warp partial sums, then a shared-memory tree
+//   u   = w.v - r,     o = p + (k.q) u      since S_new^T q = S'^T q + k^T q u
+//   S   = S' + k u^T                        written back with streaming stores
+// Recurrent decode with constant memory per token is the property the aixai.ru
+// post's opening section and its "Почему это важно" section point to.
+#include "gdn2_internal.cuh"
+
+namespace gdn2 {
+namespace {
+
+constexpr int kWarps = 8;
+
+template <int D> struct Vec;
+template <> struct Vec<128> { using T = float4; };
+template <> struct Vec<64> { using T = float2; };
+
+__device__ __forceinline__ void scale_fma(float4 &s, float a) { s.x *= a; s.y *= a; s.z *= a; s.w *= a; }
+__device__ __forceinline__ void scale_fma(float2 &s, float a) { s.x *= a; s.y *= a; }
+
+template <int D, typename Tin>
+__global__ void __launch_bounds__(kWarps * 32)
+decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+              const float *__restrict__ g, const Tin *__restrict__ b, const Tin *__restrict__ w,
+              float *__restrict__ S, Tin *__restrict__ o)
+{
+    constexpr int CPT = D / 32;      // columns per lane
+    constexpr int RPW = D / kWarps;  // rows per warp
+    using V = typename Vec<D>::T;
+    __shared__ float s_q[D], s_k[D], s_e[D], s_a[D], s_u[D];
+    __shared__ float s_r[kWarps][D], s_p[kWarps][D];
+    __shared__ float s_kq;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t nh = blockIdx.x;
+    const size_t vec = nh * D;
+    float *Sp = S + nh * D * D;
+
+    // issue the state loads first: they are the long pole
+    V sv[RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        const int row = warp * RPW + r;
+        sv[r] = __ldcs(reinterpret_cast<const V *>(Sp + (size_t)row * D) + lane);
+    }
+    if (tid < D) {
+        const float kv = to_f(k[vec + tid]), qv = to_f(q[vec + tid]);
+        s_q[tid] = qv;
+        s_k[tid] = kv;
+        s_e[tid] = to_f(b[vec + tid]) * kv;
+        s_a[tid] = expf(g[vec + tid]);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float kq = 0.f;
+        for (int i = lane; i < D; i += 32) kq += s_k[i] * s_q[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        if (lane == 0) s_kq = kq;
+    }
+    float pr[CPT], pp[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) { pr[c] = 0.f; pp[c] = 0.f; }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        const int row = warp * RPW + r;
+        const float a = s_a[row], e = s_e[row], qq = s_q[row];
+        scale_fma(sv[r], a);
+        const float *x = reinterpret_cast<const float *>(&sv[r]);
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) { pr[c] += x[c] * e; pp[c] += x[c] * qq; }
+    }
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) { s_r[warp][lane * CPT + c] = pr[c]; s_p[warp][lane * CPT + c] = pp[c]; }
+    __syncthreads();
+    if (tid < D) {
+        float r = 0.f, pq = 0.f;
+#pragma unroll
+        for (int wi = 0; wi < kWarps; ++wi) { r += s_r[wi][tid]; pq += s_p[wi][tid]; }
+        const float u = to_f(w[vec + tid]) * to_f(v[vec + tid]) - r;
+        s_u[tid] = u;
+        o[vec + tid] = from_f<Tin>(pq + s_kq * u);
+    }
+    __syncthreads();
+    float uu[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) uu[c] = s_u[lane * CPT + c];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        const int row = warp * RPW + r;
+        const float kk = s_k[row];
+        float *x = reinterpret_cast<float *>(&sv[r]);
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) x[c] += kk * uu[c];
+        __stcs(reinterpret_cast<V *>(Sp + (size_t)row * D) + lane, sv[r]);
+    }
+}
+
+template <int D, typename Tin>
+cudaError_t launch_t(int N, int H, const void *q, const void *k, const void *v, const float *g,
+                     const void *b, const void *w, float *S, void *o, cudaStream_t s)
+{
+    decode_kernel<D, Tin><<<N * H, kWarps * 32, 0, s>>>(H, (const Tin *)q, (const Tin *)k,
+                                                        (const Tin *)v, g, (const Tin *)b,
+                                                        (const Tin *)w, S, (Tin *)o);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
+                          const void *v, const float *g, const void *b, const void *w, float *S,
+                          void *o, cudaStream_t s)
+{
+    if (dt == GDN2_F32)
+        return D == 64 ? launch_t<64, float>(N, H, q, k, v, g, b, w, S, o, s)
+                       : launch_t<128, float>(N, H, q, k, v, g, b, w, S, o, s);
+    return D == 64 ? launch_t<64, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, s)
+                   : launch_t<128, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, s);
+}
+
+}  // namespace gdn2

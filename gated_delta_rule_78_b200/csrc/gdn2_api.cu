@@ -1,0 +1,164 @@
+// C ABI of libgdn2.so: argument validation, workspace sizing, kernel dispatch.
+// Declarations and the contract of every entry point are in include/gdn2.h.
+#include <stdint.h>
+
+#include "gdn2_internal.cuh"
+
+// Per-device kernel status word (0 = fine).  Kernels that give up a bounded
+// wait store a non-zero code here; gdn2_sync_status() reads and clears it.
+__device__ int g_gdn2_status = 0;
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+gdn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
+
+// Common checks for the chunked entry points.  Returns GDN2_OK when the sizes
+// are inside the v1 contract.
+gdn2_status check_sizes(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
+{
+    if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (B <= 0 || H <= 0 || T < 0 || Dk <= 0 || Dv <= 0) return GDN2_ERR_SHAPE;
+    if (Dk != Dv || (Dk != 64 && Dk != 128)) return GDN2_ERR_UNSUPPORTED;
+    // element counts must fit comfortably in the kernels' 64-bit index math and
+    // the grid's x dimension
+    if ((long long)B * H > (1LL << 30)) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)B * T * H * Dk > (1LL << 40)) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+gdn2_status check_ptrs(std::initializer_list<const void *> required,
+                       std::initializer_list<const void *> optional)
+{
+    for (const void *p : required)
+        if (!p) return GDN2_ERR_NULL;
+    for (const void *p : required)
+        if (!aligned16(p)) return GDN2_ERR_ALIGN;
+    for (const void *p : optional)
+        if (p && !aligned16(p)) return GDN2_ERR_ALIGN;
+    return GDN2_OK;
+}
+
+gdn2::Problem make_problem(int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                           const float *g, const void *b, const void *w, const float *S0)
+{
+    gdn2::Problem p;
+    p.B = B; p.T = T; p.H = H; p.D = D;
+    p.q = q; p.k = k; p.v = v; p.b = b; p.w = w; p.g = g; p.S0 = S0;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn2_strerror(gdn2_status s)
+{
+    switch (s) {
+    case GDN2_OK: return "success";
+    case GDN2_ERR_NULL: return "a required pointer is NULL";
+    case GDN2_ERR_SHAPE: return "invalid size (negative, or zero where positive is required)";
+    case GDN2_ERR_DTYPE: return "unknown dtype";
+    case GDN2_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case GDN2_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDN2_ERR_CUDA: return "a CUDA runtime call failed";
+    case GDN2_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case GDN2_ERR_UNSUPPORTED: return "outside the supported shapes (Dk == Dv in {64, 128})";
+    }
+    return "unknown status";
+}
+
+size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
+{
+    if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK) return 0;
+    if (which == 0) return 0;
+    if (which == 1) return T == 0 ? 0 : gdn2::bwd_workspace_bytes(B, T, H, Dk);
+    return 0;
+}
+
+gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                           const void *k, const void *v, const float *log_alpha, const void *b,
+                           const void *w, const float *S0, void *o, float *S_T, void *workspace,
+                           size_t ws_bytes, void *stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (T > 0) st = check_ptrs({q, k, v, log_alpha, b, w, o}, {S0, S_T});
+    else st = check_ptrs({}, {S0, S_T});
+    if (st != GDN2_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+    if (T == 0) {
+        if (!S_T) return GDN2_OK;
+        if (S0) return S0 == S_T ? GDN2_OK : from_cuda(cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(S_T, 0, state_bytes, s));
+    }
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    if (dt == GDN2_BF16) {
+        int *status = nullptr;
+        if (cudaGetSymbolAddress((void **)&status, g_gdn2_status) != cudaSuccess) return GDN2_ERR_CUDA;
+        cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, status, s);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();  // clear the sticky "not supported" code; fall through to FMA path
+    }
+    return from_cuda(gdn2::launch_fwd_simt(dt, p, o, S_T, nullptr, s));
+}
+
+gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int Dv, const void *q,
+                             const void *k, const void *v, const float *log_alpha, const void *b,
+                             const void *w, float *S, void *o, void *stream)
+{
+    gdn2_status st = check_sizes(dt, N, 1, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    st = check_ptrs({q, k, v, log_alpha, b, w, S, o}, {});
+    if (st != GDN2_OK) return st;
+    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, q, k, v, log_alpha, b, w, S, o,
+                                         (cudaStream_t)stream));
+}
+
+gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                           const void *k, const void *v, const float *log_alpha, const void *b,
+                           const void *w, const float *S0, const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (T > 0)
+        st = check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0},
+                        {S0, dS_T});
+    else
+        st = check_ptrs({dS0}, {S0, dS_T});
+    if (st != GDN2_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+    if (T == 0) {
+        if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
+    }
+    const size_t need = gdn2::bwd_workspace_bytes(B, T, H, Dk);
+    if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
+    return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s));
+}
+
+gdn2_status gdn2_sync_status(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gdn2_status, sizeof(int)) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_gdn2_status, &zero, sizeof(int)) != cudaSuccess) return GDN2_ERR_CUDA;
+        return GDN2_ERR_TIMEOUT;
+    }
+    return GDN2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Internal declarations shared by the kernels and the C ABI layer of libgdn2.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn2.h"
+
+namespace gdn2 {
+
+constexpr int kChunk = 64;  // tokens per chunk
+
+// Device status word values (written by kernels, read by gdn2_sync_status).
+constexpr int kStatusTimeout = 1;
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Problem description handed from the C ABI layer to the launchers.  All
+// pointers are device pointers; layouts as in gdn2.h.
+struct Problem {
+    int B, T, H, D;  // Dk == Dv == D
+    const void *q, *k, *v, *b, *w;
+    const float *g;   // log alpha
+    const float *S0;  // may be null
+};
+
+// forward (SIMT fp32 FMA path).  `states`, when non-null, receives the state at
+// the start of every chunk: [B*H][nchunks][D][D] fp32.  `o` may be null (states only).
+cudaError_t launch_fwd_simt(gdn2_dtype dt, const Problem &p, void *o, float *S_T, float *states,
+                            cudaStream_t s);
+
+// forward on the tensor cores (bf16 operands); returns cudaErrorNotSupported when
+// the shape is outside what the kernel handles.
+cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, int *status, cudaStream_t s);
+
+cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
+                          const void *v, const float *g, const void *b, const void *w, float *S,
+                          void *o, cudaStream_t s);
+
+struct BwdOut {
+    void *dq, *dk, *dv, *db, *dw;
+    float *dg, *dS0;
+};
+size_t bwd_workspace_bytes(int B, int T, int H, int D);
+cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
+                       const BwdOut &out, void *ws, cudaStream_t s);
+
+}  // namespace gdn2

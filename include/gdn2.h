@@ -1,0 +1,131 @@
+/*
+ * gdn2.h -- C ABI of libgdn2.so: the Gated DeltaNet-2 chunkwise gated
+ * delta-rule recurrence on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch b and head h, tokens t = 1..T, S_0 given or zero):
+ *
+ *     alpha_t = exp(log_alpha_t)            channel-wise decay, d_k entries
+ *     S'      = Diag(alpha_t) S_{t-1}       decay first
+ *     u_t     = w_t (.) v_t - S'^T (b_t (.) k_t)
+ *     S_t     = S' + k_t u_t^T  =  (I - k_t (b_t (.) k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t (.) v_t)^T
+ *     o_t     = S_t^T q_t
+ *
+ * b_t (key side, d_k entries) is the erase gate, w_t (value side, d_v
+ * entries) the write gate.  Sources: aixai.ru "Gated DeltaNet-2" post, section
+ * "Один скаляр не может решать два разных вопроса" (the update in prose) and
+ * "Как это реализуется на практике" (chunkwise computation, gate-weighted
+ * keys/values, A and T, gate-aware backward, log-decay in fp32); aiexpert.news
+ * article, gate paragraph (b_t in [0,1]^{d_k}, w_t in [0,1]^{d_v}, exact
+ * reduction to KDA when b_t = w_t = beta_t 1) and implementation paragraph
+ * (chunkwise WY algorithm with the decay absorbed into asymmetric erase
+ * factors).  No 1/sqrt(d) scale is applied: fold any scale into q.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are caller-owned DEVICE pointers to contiguous
+ *    row-major memory, 16-byte aligned (GDN2_ERR_ALIGN otherwise).  The
+ *    library allocates no device memory and keeps no pointer after a call.
+ *  - q, k, b: [B, T, H, Dk]; v, w, o (and their gradients): [B, T, H, Dv];
+ *    element type given by `dt` (fp32 or bf16).  log_alpha and its gradient
+ *    are [B, T, H, Dk] fp32 always.  States S0, S_T, dS_T, dS0 are
+ *    [B, H, Dk, Dv] fp32 always (d_v contiguous).
+ *  - v1 shape contract: Dk == Dv in {64, 128}; B, H >= 1; T >= 0 (any T;
+ *    T = 0 copies S0 to S_T).  Other shapes give GDN2_ERR_UNSUPPORTED.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    are asynchronous on it: a GDN2_OK return means the arguments were valid
+ *    and the kernels were enqueued.  An error raised inside a kernel (a
+ *    bounded wait that gave up) is recorded in a per-device status word that
+ *    gdn2_sync_status() reports.
+ *  - Every call validates all arguments before it launches anything; on an
+ *    error nothing is launched and no output is written.  No C++ exception
+ *    crosses this boundary.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_NULL = -1,        /* a required pointer is NULL */
+    GDN2_ERR_SHAPE = -2,       /* a size is negative or zero where it must be positive */
+    GDN2_ERR_DTYPE = -3,       /* dt is not a gdn2_dtype value */
+    GDN2_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned */
+    GDN2_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than gdn2_workspace_size() */
+    GDN2_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch error, no device, ...) */
+    GDN2_ERR_TIMEOUT = -7,     /* a kernel's bounded wait gave up (reported by gdn2_sync_status) */
+    GDN2_ERR_UNSUPPORTED = -8  /* valid but outside the v1 shape contract */
+} gdn2_status;
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+/*
+ * Chunkwise forward (chunk length 64): o and the final state S_T.
+ *   S0:  initial state, or NULL for zeros.
+ *   o:   output [B,T,H,Dv] of type dt.
+ *   S_T: final state, or NULL when not wanted.  May alias S0 (in-place
+ *        state update), but no other argument.
+ *   workspace / ws_bytes: scratch of at least gdn2_workspace_size(0, ...)
+ *        bytes (currently 0; NULL is then accepted).
+ * bf16 inputs run on the tensor cores (bf16 operands, fp32 accumulation,
+ * fp32 state); fp32 inputs run in fp32 FMA arithmetic throughout.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * One recurrent decode step for N independent sequences (one token each).
+ *   q, k, b: [N,H,Dk]; v, w, o: [N,H,Dv] of type dt; log_alpha [N,H,Dk] fp32.
+ *   S: [N,H,Dk,Dv] fp32, read and overwritten in place with S_t.
+ * Same update as above with T = 1; the state is read once and written once.
+ */
+GDN2_API gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int Dv,
+                             const void *q, const void *k, const void *v, const float *log_alpha,
+                             const void *b, const void *w, float *S, void *o, void *stream);
+
+/*
+ * Gate-aware backward of L = <o, d_o> + <S_T, dS_T> for the forward above.
+ *   d_o: [B,T,H,Dv] of type dt.  dS_T: fp32 state gradient, or NULL for zero.
+ *   Outputs: dq, dk, db [B,T,H,Dk] and dv, dw [B,T,H,Dv] of type dt;
+ *            dlog_alpha [B,T,H,Dk] fp32; dS0 [B,H,Dk,Dv] fp32.
+ *   S0 may be NULL (zeros).  All outputs must be distinct from the inputs.
+ *   workspace: at least gdn2_workspace_size(1, ...) bytes (chunk-start
+ *   states and per-tile partial gradients, fp32).
+ * The gates enter inside the chunk products (gate-weighted keys and values),
+ * as the aixai.ru post's implementation section requires.
+ */
+GDN2_API gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream);
+
+/* Workspace bytes for which = 0 (gdn2_chunk_fwd) or 1 (gdn2_chunk_bwd);
+ * 0 for invalid or unsupported arguments. */
+GDN2_API size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv);
+
+/* Static, NUL-terminated description of a status code. */
+GDN2_API const char *gdn2_strerror(gdn2_status status);
+
+/* Synchronises `stream`, then returns and clears the current device's kernel
+ * status word: GDN2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last check, GDN2_ERR_CUDA if the stream reported an error, else GDN2_OK. */
+GDN2_API gdn2_status gdn2_sync_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

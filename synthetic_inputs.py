@@ -34,24 +34,26 @@ def _l2norm(x: torch.Tensor) -> torch.Tensor:
 
 def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16",
                 seed: int = 0, s0: str = "normal", with_do: bool = False,
-                b_scale: float = 1.0, x_mean: float = -3.0) -> dict:
+                b_scale: float = 1.0, x_mean: float = -3.0, device: str = "cpu") -> dict:
     """Draw one forward (or forward+backward) problem.
 
     Layouts: q, k, b, log_alpha are [B, T, H, Dk]; v, w, do are [B, T, H, Dv];
     S0 is [B, H, Dk, Dv] fp32.  ``b_scale`` stretches the erase gate range
     (2.0 gives b in [0, 2]); ``x_mean`` moves the decay logits (a larger
-    value gives stronger decay).
+    value gives stronger decay).  ``device="cuda"`` draws the same
+    distributions with a seeded CUDA generator (a different stream of numbers,
+    used for timing only, never for parity).
     """
     dt = DTYPES[dtype]
-    gen = torch.Generator().manual_seed(seed)
-    f32 = torch.float32
-    q = _l2norm(torch.randn(B, T, H, Dk, generator=gen, dtype=f32))
-    k = _l2norm(torch.randn(B, T, H, Dk, generator=gen, dtype=f32))
-    v = torch.randn(B, T, H, Dv, generator=gen, dtype=f32)
-    x = torch.randn(B, T, H, Dk, generator=gen, dtype=f32) + x_mean
-    bl = torch.randn(B, T, H, Dk, generator=gen, dtype=f32)
-    wl = torch.randn(B, T, H, Dv, generator=gen, dtype=f32)
-    S0 = torch.randn(B, H, Dk, Dv, generator=gen, dtype=f32) * 0.02
+    gen = torch.Generator(device=device).manual_seed(seed)
+    kw = dict(generator=gen, dtype=torch.float32, device=device)
+    q = _l2norm(torch.randn(B, T, H, Dk, **kw))
+    k = _l2norm(torch.randn(B, T, H, Dk, **kw))
+    v = torch.randn(B, T, H, Dv, **kw)
+    x = torch.randn(B, T, H, Dk, **kw) + x_mean
+    bl = torch.randn(B, T, H, Dk, **kw)
+    wl = torch.randn(B, T, H, Dv, **kw)
+    S0 = torch.randn(B, H, Dk, Dv, **kw) * 0.02
     if s0 == "zeros":
         S0 = torch.zeros_like(S0)
     out = {
@@ -62,28 +64,30 @@ def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16"
         "S0": S0,
     }
     if with_do:
-        out["do"] = torch.randn(B, T, H, Dv, generator=gen, dtype=f32).to(dt)
+        out["do"] = torch.randn(B, T, H, Dv, **kw).to(dt)
     return out
 
 
 class DecodeStream:
     """Per-step single-token inputs for ``N`` sequences, drawn in order."""
 
-    def __init__(self, N: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16", seed: int = 0):
+    def __init__(self, N: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16", seed: int = 0,
+                 device: str = "cpu"):
         self.N, self.H, self.Dk, self.Dv = N, H, Dk, Dv
         self.dt = DTYPES[dtype]
-        self.gen = torch.Generator().manual_seed(seed)
+        self.gen = torch.Generator(device=device).manual_seed(seed)
+        self.kw = dict(generator=self.gen, dtype=torch.float32, device=device)
         # initial state first, so that erase acts from step one
-        self.S0 = torch.randn(N, H, Dk, Dv, generator=self.gen, dtype=torch.float32) * 0.02
+        self.S0 = torch.randn(N, H, Dk, Dv, **self.kw) * 0.02
 
     def step(self) -> dict:
-        N, H, Dk, Dv, gen, f32 = self.N, self.H, self.Dk, self.Dv, self.gen, torch.float32
-        q = _l2norm(torch.randn(N, H, Dk, generator=gen, dtype=f32))
-        k = _l2norm(torch.randn(N, H, Dk, generator=gen, dtype=f32))
-        v = torch.randn(N, H, Dv, generator=gen, dtype=f32)
-        x = torch.randn(N, H, Dk, generator=gen, dtype=f32) - 3.0
-        bl = torch.randn(N, H, Dk, generator=gen, dtype=f32)
-        wl = torch.randn(N, H, Dv, generator=gen, dtype=f32)
+        N, H, Dk, Dv, kw = self.N, self.H, self.Dk, self.Dv, self.kw
+        q = _l2norm(torch.randn(N, H, Dk, **kw))
+        k = _l2norm(torch.randn(N, H, Dk, **kw))
+        v = torch.randn(N, H, Dv, **kw)
+        x = torch.randn(N, H, Dk, **kw) - 3.0
+        bl = torch.randn(N, H, Dk, **kw)
+        wl = torch.randn(N, H, Dv, **kw)
         return {
             "q": q.to(self.dt), "k": k.to(self.dt), "v": v.to(self.dt),
             "log_alpha": -torch.nn.functional.softplus(x),

@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects invalid
+arguments with the documented status codes before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_78_b200 as g
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+F32, BF16 = 0, 1
+P = ctypes.c_void_p(0x7F0000000000)         # aligned stand-in address, never dereferenced
+MIS = ctypes.c_void_p(0x7F0000000004)       # 4-byte aligned only
+NUL = ctypes.c_void_p(0)
+S = ctypes.c_void_p(0)                      # stream
+
+
+def declared_symbols():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        names += re.findall(r"GDN2_API\s+[\w\s\*]+?\b(gdn2_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return g.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert set(g.EXPORTS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror_covers_all_codes(lib):
+    for code in g.STATUS_NAMES:
+        assert len(lib.gdn2_strerror(code)) > 0
+    assert lib.gdn2_strerror(12345) == b"unknown status"
+
+
+def fwd(lib, dt=BF16, B=1, T=64, H=1, Dk=128, Dv=128, q=P, o=P, S0=NUL, ST=NUL):
+    return lib.gdn2_chunk_fwd(dt, B, T, H, Dk, Dv, q, P, P, P, P, P, S0, o, ST, NUL, 0, S)
+
+
+def bwd(lib, dt=BF16, B=1, T=64, H=1, Dk=128, Dv=128, ws=P, ws_bytes=1 << 40, dq=P):
+    return lib.gdn2_chunk_bwd(dt, B, T, H, Dk, Dv, P, P, P, P, P, P, NUL, P, NUL,
+                              dq, P, P, P, P, P, P, ws, ws_bytes, S)
+
+
+def dec(lib, dt=BF16, N=1, H=1, Dk=128, Dv=128, S_=P):
+    return lib.gdn2_decode_step(dt, N, H, Dk, Dv, P, P, P, P, P, P, S_, P, S)
+
+
+def test_invalid_arguments_return_status(lib):
+    assert fwd(lib, dt=7) == -3
+    assert fwd(lib, B=0) == -2
+    assert fwd(lib, H=-1) == -2
+    assert fwd(lib, T=-5) == -2
+    assert fwd(lib, Dk=96, Dv=96) == -8
+    assert fwd(lib, Dk=128, Dv=64) == -8
+    assert fwd(lib, q=NUL) == -1
+    assert fwd(lib, o=NUL) == -1
+    assert fwd(lib, q=MIS) == -4
+    assert fwd(lib, S0=MIS) == -4
+    assert fwd(lib, ST=MIS) == -4
+    assert dec(lib, N=0) == -2
+    assert dec(lib, S_=NUL) == -1
+    assert dec(lib, S_=MIS) == -4
+    assert dec(lib, Dk=32, Dv=32) == -8
+    assert bwd(lib, dq=NUL) == -1
+    assert bwd(lib, ws=NUL) == -5
+    assert bwd(lib, ws_bytes=16) == -5
+    assert bwd(lib, ws=MIS) == -4
+
+
+def test_workspace_size(lib):
+    assert lib.gdn2_workspace_size(0, BF16, 8, 4096, 16, 128, 128) == 0
+    need = lib.gdn2_workspace_size(1, BF16, 8, 4096, 16, 128, 128)
+    states = 8 * 16 * 64 * 128 * 128 * 4
+    assert need >= states
+    assert lib.gdn2_workspace_size(1, BF16, 8, 4096, 16, 96, 96) == 0
+    assert lib.gdn2_workspace_size(1, 9, 8, 4096, 16, 128, 128) == 0
+    assert lib.gdn2_workspace_size(5, BF16, 8, 4096, 16, 128, 128) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import importlib
+    mod = importlib.import_module("gated_delta_rule_78_b200._lib")
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(OSError):
+            mod.load(str(tmp_path / "nope.so"))
+    finally:
+        mod._lib = saved
