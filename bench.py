@@ -202,8 +202,9 @@ def cpu_baseline(w, target_s=12.0, seed=0):
     t0 = time.perf_counter()
     oracle.ref_fwd(one["q"], one["k"], one["v"], one["log_alpha"], one["b"], one["w"], one["S0"], nthreads=1)
     per_seq = time.perf_counter() - t0
-    nseq = max(cores, min(w["B"] * w["H"], int(target_s * cores / max(per_seq, 1e-3))))
-    nseq = (nseq // cores) * cores or cores
+    # as many full-length sequences of the workload's shape as fit about target_s seconds
+    nseq = max(cores, int(target_s * cores / max(per_seq, 1e-3)))
+    nseq = min((nseq // cores) * cores or cores, 64 * cores)
     x = make_inputs(1, T, nseq, D, D, dtype=w["dtype"], seed=seed + 1)
     t0 = time.perf_counter()
     oracle.ref_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], nthreads=cores)
