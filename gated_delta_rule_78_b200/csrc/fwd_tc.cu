@@ -6,23 +6,29 @@
 // aiexpert.news article's implementation paragraph describes, and the
 // auxiliary matrices of the aixai.ru post's "Как это реализуется на практике"):
 //   G  = inclusive cumulative sum of log alpha over the chunk (fp32)
-//   Q~ = q e^G,  E~ = (b.k) e^G,  K~ = k e^-G,  K^ = k e^(G_L - G),  gamma = e^G_L
+//   Q~ = q e^G,  E~ = (b.k) e^G,  K~ = k e^-G,  gamma = e^G_L,  X = w.v
 //   [A; P] = [E~; Q~] K~^T          A strictly lower, P lower incl. (one M=128 MMA)
-//   T  = (I + A)^-1                  blocked 16x16 substitution in shared memory
-//   W^T = E~^T T^T,  U^T = X^T T^T  (X = w.v)
-//   U~^T = U^T + S^T (-W^T)          S^T (bf16) is the TMEM A operand
-//   O^T  = S^T Q~^T + U~^T P^T
-//   S   <- Diag(gamma) S + (U~^T K^)^T   (update done in fp32 registers)
-// Everything is formulated transposed so that every product has M = 128
-// (d_k or d_v, or the stacked [E~; Q~]) and runs as a full-height tcgen05.mma.
+//   Y   = X - E~ S                  (the gated value minus what the erase-weighted
+//                                    keys read from the chunk-start state)
+//   T   = (I + A)^-1                 blocked: 16x16 diagonal blocks by substitution,
+//                                    the doubling levels on warp-level TF32 MMAs
+//   U~  = T Y                        (= (I+A)^-1 (w.V) - (I+A)^-1 E~ S)
+//   O   = Q~ S + P U~
+//   S  <- Diag(gamma) (S + K~^T U~)  (K~ e^G_L is the decay from token t to the
+//                                    chunk end, so gamma is applied once, in fp32)
+// Everything is formulated transposed (S^T, Y^T, U~^T, O^T with d_v as the row
+// index) so that every tcgen05.mma has M = 128; S^T, Y^T and U~^T are TMEM
+// operands, and S^T [E~; Q~]^T is one N = 128 product.
 //
-// Work decomposition: one CTA per (batch, head), 8 warps.  Warp w owns TMEM
-// lanes 32 (w & 3) .. +31 and column half (w >> 2) of every readback; its
-// threads hold their 64 columns of S^T (row j = d_v index) in fp32 registers.
-// The raw inputs of chunk c+1 are fetched by TMA (128-byte swizzle, the same
-// layout the MMA descriptors read) into each buffer as soon as chunk c no
-// longer needs it, so the loads overlap chunk c's compute; the elementwise pass
-// converts them in place into the factors.
+// Work decomposition: one CTA per (batch, head), two warp groups that run one
+// chunk apart.  The E group (warps 8-15) folds the decay of chunk c+1 into its
+// factors (shared-memory buffers for q/b, k and v are double-buffered, log
+// alpha is read from L2 where a TMA prefetch has put it) while the M group
+// (warps 0-7) runs chunk c's chain: MMA, readback, solve, MMA, readback, MMA,
+// state update and output.  Warp m of M owns TMEM lanes 32 (m & 3) .. +31 and
+// column half (m >> 2) of every readback and holds its 64 columns of S^T in
+// fp32 registers.  The output tile is staged in shared memory and written by a
+// TMA store.  Cross-group hand-offs use mbarriers, one per chunk parity.
 #include <cuda.h>
 
 #include "gdn2_internal.cuh"
@@ -35,444 +41,534 @@ using namespace tc;
 
 constexpr int D = 128;
 constexpr int C = 64;
-constexpr int kThreads = 256;
-constexpr int LDA = 68;  // fp32 row stride of the A / T scratch
+constexpr int kThreads = 512;
+constexpr int kGroup = 256;  // threads per warp group
+constexpr int LDA = 68;      // fp32 row stride of the A / T scratch
 
 // shared-memory map (bytes from a 1024-byte aligned base)
-constexpr uint32_t OFF_QE = 0;          // [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
-constexpr uint32_t OFF_K = 32768;       // K~ (raw k), 2 atoms
-constexpr uint32_t OFF_KH = 49152;      // K^, 2 atoms
-constexpr uint32_t OFF_G = 65536;       // log alpha fp32, 4 atoms of 32 channels
-constexpr uint32_t OFF_V = 98304;       // X = w.v (raw v), 2 atoms
-constexpr uint32_t OFF_W = 114688;      // raw w, 2 atoms
-constexpr uint32_t OFF_WT = 131072;     // -W^T: 128 rows (d_k) x 64 tokens
-constexpr uint32_t OFF_TT = 147456;     // T: 64 rows (i) x 64 (j)
-constexpr uint32_t OFF_PT = 155648;     // P: 64 rows (t) x 64 (i)
+constexpr uint32_t OFF_QE = 0;          // 2 x [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
+constexpr uint32_t OFF_K = 65536;       // 2 x K~ (raw k), 2 atoms
+constexpr uint32_t OFF_V = 98304;       // 2 x X = w.v (raw v), 2 atoms
+constexpr uint32_t OFF_W = 131072;      // raw w, 2 atoms
+constexpr uint32_t OFF_TT = 147456;     // T: 64 rows (i) x 64 (j), bf16      } output tile (64 x 128
+constexpr uint32_t OFF_PT = 155648;     // P: 64 rows (t) x 64 (i), bf16      }  bf16) after MMA 3
+constexpr uint32_t OFF_O = OFF_TT;
 constexpr uint32_t OFF_SA = 163840;     // A fp32 [64][LDA]
 constexpr uint32_t OFF_ST = OFF_SA + 64 * LDA * 4;   // T fp32 [64][LDA]
-constexpr uint32_t OFF_TOT = OFF_ST + 64 * LDA * 4;  // per-quarter decay totals [4][128] fp32
-constexpr uint32_t OFF_GAM = OFF_TOT + 4 * 128 * 4;  // gamma [128] fp32
-constexpr uint32_t SMEM_USED = OFF_GAM + 128 * 4;
+constexpr uint32_t OFF_TOT = OFF_ST + 64 * LDA * 4;  // per-group decay totals [4][128] fp32
+constexpr uint32_t OFF_GAM = OFF_TOT + 4 * 128 * 4;  // gamma [2][128] fp32
+constexpr uint32_t SMEM_USED = OFF_GAM + 2 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for the 1024-byte alignment
 
 // TMEM columns
 constexpr uint32_t TM_SBF = 0;     // S^T bf16 (A operand), 64 columns
-constexpr uint32_t TM_AP = 64;     // [A; P] fp32, 64 columns
-constexpr uint32_t TM_WT = 128;    // W^T fp32
-constexpr uint32_t TM_UT = 192;    // U^T, then U~^T, fp32
-constexpr uint32_t TM_OT = 256;    // O^T fp32
-constexpr uint32_t TM_UB = 320;    // U~^T bf16 (A operand), 32 columns
-constexpr uint32_t TM_DS = 384;    // (K^^T U~)^T fp32, 128 columns
+constexpr uint32_t TM_AP = 64;     // [A; P] fp32
+constexpr uint32_t TM_YO = 128;    // [S^T E~^T | O^T] fp32, 128 columns
+constexpr uint32_t TM_O = 192;     //   O^T half
+constexpr uint32_t TM_UT = 256;    // U~^T fp32
+constexpr uint32_t TM_YB = 320;    // Y^T bf16 (A operand), 32 columns
+constexpr uint32_t TM_UB = 352;    // U~^T bf16 (A operand), 32 columns
+constexpr uint32_t TM_DS = 384;    // (K~^T U~)^T fp32, 128 columns
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = idesc_bf16(128, 64, 0, 0);
-constexpr uint32_t IDESC_N64_AMN = idesc_bf16(128, 64, 1, 0);
-constexpr uint32_t IDESC_N64_BMN = idesc_bf16(128, 64, 0, 1);
+constexpr uint32_t IDESC_N128 = idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_N128_BMN = idesc_bf16(128, 128, 0, 1);
 
 struct TcParams {
     int B, T, H;
     const float *S0;
+    const float *g;   // log alpha [B,T,H,D] fp32
     __nv_bfloat16 *o;
     float *S_T;
     int *status;
 };
 
 struct TcMaps {
-    CUtensorMap q, k, v, b, w, g;
+    CUtensorMap q, k, v, b, w, g, o;
 };
+
+// barrier over `count` threads (id 0 is __syncthreads)
+__device__ __forceinline__ void named_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// One warp inverts the 16x16 unit lower-triangular diagonal block (I + A_pp) that
+// starts at row/column r0: closed-form 4x4 inverses, then two doubling steps
+// T21 = -T22 (A21 T11) inside the warp.  Only lower blocks of sT are written.
+__device__ __forceinline__ void invert_diag16(const float *sA, float *sT, int r0, int lane)
+{
+    if (lane < 4) {
+        const int b = r0 + 4 * lane;
+        const float *a = sA + b * LDA + b;
+        const float a10 = a[1 * LDA + 0], a20 = a[2 * LDA + 0], a21 = a[2 * LDA + 1];
+        const float a30 = a[3 * LDA + 0], a31 = a[3 * LDA + 1], a32 = a[3 * LDA + 2];
+        const float t10 = -a10, t21 = -a21, t32 = -a32;
+        const float t20 = -(a20 + a21 * t10);
+        const float t31 = -(a31 + a32 * t21);
+        const float t30 = -(a30 + a31 * t10 + a32 * t20);
+        float *t = sT + b * LDA + b;
+        t[0 * LDA + 0] = 1.f;
+        t[1 * LDA + 0] = t10; t[1 * LDA + 1] = 1.f;
+        t[2 * LDA + 0] = t20; t[2 * LDA + 1] = t21; t[2 * LDA + 2] = 1.f;
+        t[3 * LDA + 0] = t30; t[3 * LDA + 1] = t31; t[3 * LDA + 2] = t32; t[3 * LDA + 3] = 1.f;
+    }
+    __syncwarp();
+    {  // 4 -> 8: two 4x4 blocks, one output per lane
+        const int q = lane >> 4, r = (lane >> 2) & 3, c = lane & 3;
+        const int R = r0 + 8 * q + 4, Cc = r0 + 8 * q;
+        float y = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) y += sA[(R + r) * LDA + Cc + u] * sT[(Cc + u) * LDA + Cc + c];
+        __syncwarp();
+        sT[(R + r) * LDA + Cc + c] = y;
+        __syncwarp();
+        float x = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x += sT[(R + r) * LDA + R + u] * sT[(R + u) * LDA + Cc + c];
+        __syncwarp();
+        sT[(R + r) * LDA + Cc + c] = -x;
+        __syncwarp();
+    }
+    {  // 8 -> 16: one 8x8 block, two outputs per lane
+        const int r = lane >> 2, c = 2 * (lane & 3);
+        const int R = r0 + 8, Cc = r0;
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float a = sA[(R + r) * LDA + Cc + u];
+            y0 += a * sT[(Cc + u) * LDA + Cc + c];
+            y1 += a * sT[(Cc + u) * LDA + Cc + c + 1];
+        }
+        __syncwarp();
+        sT[(R + r) * LDA + Cc + c] = y0;
+        sT[(R + r) * LDA + Cc + c + 1] = y1;
+        __syncwarp();
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float t = sT[(R + r) * LDA + R + u];
+            x0 += t * sT[(R + u) * LDA + Cc + c];
+            x1 += t * sT[(R + u) * LDA + Cc + c + 1];
+        }
+        __syncwarp();
+        sT[(R + r) * LDA + Cc + c] = -x0;
+        sT[(R + r) * LDA + Cc + c + 1] = -x1;
+    }
+}
+
+// acc (16x8 tile) += X[0:16, 0:K] * Y[0:K, 0:8] for fp32 shared-memory operands with
+// row stride LDA (X and Y point at the tile origins), rounded to TF32 on load.
+template <int K>
+__device__ __forceinline__ void tile_mma_tf32(const float *X, const float *Y, float (&acc)[4], int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a[4] = {to_tf32(X[g * LDA + k0 + t]), to_tf32(X[(g + 8) * LDA + k0 + t]),
+                               to_tf32(X[g * LDA + k0 + t + 4]), to_tf32(X[(g + 8) * LDA + k0 + t + 4])};
+        const uint32_t b[2] = {to_tf32(Y[(k0 + t) * LDA + g]), to_tf32(Y[(k0 + t + 4) * LDA + g])};
+        mma_tf32_16x8x8(acc, a, b);
+    }
+}
+__device__ __forceinline__ void tile_store(float *Z, const float (&acc)[4], float sign, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    Z[g * LDA + 2 * t] = sign * acc[0];
+    Z[g * LDA + 2 * t + 1] = sign * acc[1];
+    Z[(g + 8) * LDA + 2 * t] = sign * acc[2];
+    Z[(g + 8) * LDA + 2 * t + 1] = sign * acc[3];
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar_g, bar_k, bar_bv, bar_q, bar_mma;
+    // bar_in: this chunk's k, b, q, v, w have landed (E waits)      bar_mma: M's tcgen05 batches
+    // bar_fact[2]: E -> M, the factors of a chunk are ready          bar_m1[2]: M -> E, q/b/v buffers free
+    // bar_kf[2]: M -> E, the k buffer is free
+    __shared__ __align__(8) uint64_t bar_in, bar_mma, bar_fact[2], bar_m1[2], bar_kf[2];
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
+    __shared__ int s_abort_m, s_abort_e;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3, hcol = warp >> 2;
+    const bool is_m = warp < 8;
     const int bh = blockIdx.x, bb = bh / p.H, hh = bh % p.H;
     const int T = p.T;
     const int nchunks = (T + C - 1) / C;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float *sA = reinterpret_cast<float *>(sm + OFF_SA);
     float *sT = reinterpret_cast<float *>(sm + OFF_ST);
     float *sTot = reinterpret_cast<float *>(sm + OFF_TOT);
     float *sGam = reinterpret_cast<float *>(sm + OFF_GAM);
 
-    auto issue_loads = [&](int ci, int which) {
-        // which: 0 = g + w, 1 = k, 2 = b + v, 3 = q
-        const int y = bb * T + ci * C;
-        if (which == 0) {
-            mbar_expect_tx(&bar_g, 4 * 8192 + 2 * 8192);
-            for (int a = 0; a < 4; ++a) tma_load_3d(sm + OFF_G + a * 8192, &maps.g, a * 32, hh, y, &bar_g);
-            for (int a = 0; a < 2; ++a) tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_g);
-        } else if (which == 1) {
-            mbar_expect_tx(&bar_k, 2 * 8192);
-            for (int a = 0; a < 2; ++a) tma_load_3d(sm + OFF_K + a * 8192, &maps.k, a * 64, hh, y, &bar_k);
-        } else if (which == 2) {
-            mbar_expect_tx(&bar_bv, 4 * 8192);
-            for (int a = 0; a < 2; ++a) tma_load_3d(sm + OFF_QE + a * 16384, &maps.b, a * 64, hh, y, &bar_bv);
-            for (int a = 0; a < 2; ++a) tma_load_3d(sm + OFF_V + a * 8192, &maps.v, a * 64, hh, y, &bar_bv);
-        } else {
-            mbar_expect_tx(&bar_q, 2 * 8192);
-            for (int a = 0; a < 2; ++a) tma_load_3d(sm + OFF_QE + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_q);
-        }
-    };
-    auto fail = [&]() {
-        s_abort = 1;
-        atomicExch(p.status, kStatusTimeout);
-    };
-
     if (tid == 0) {
-        s_abort = 0;
-        mbar_init(&bar_g, 1);
-        mbar_init(&bar_k, 1);
-        mbar_init(&bar_bv, 1);
-        mbar_init(&bar_q, 1);
+        s_abort_m = 0;
+        s_abort_e = 0;
+        mbar_init(&bar_in, 1);
         mbar_init(&bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_fact[i], 1);
+            mbar_init(&bar_m1[i], 1);
+            mbar_init(&bar_kf[i], 1);
+        }
         fence_mbar_init();
         prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.v);
-        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w); prefetch_tmap(&maps.g);
+        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w); prefetch_tmap(&maps.g); prefetch_tmap(&maps.o);
     }
     if (warp == 0) {
         tmem_alloc(&s_tmem, TM_COLS);
         tmem_relinquish();
     }
+    // T's strictly-upper blocks stay zero for the whole kernel
+    for (int idx = tid; idx < 64 * LDA; idx += kThreads) sT[idx] = 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    if (tid == 0 && nchunks > 0)
-        for (int wch = 0; wch < 4; ++wch) issue_loads(0, wch);
 
-    // fp32 state: this thread holds S^T[j][64 hcol + i], j = 32 quarter + lane
-    const int jrow = quarter * 32 + lane;
-    float Sf[64];
+    if (is_m) {
+        // =========================== M group: the per-chunk tensor-core chain ===========================
+        // Register split: the launch holds 512 x 128 registers; M takes 176 per thread and E
+        // gives back to 80 (256 x 176 + 256 x 80 = 65536, exactly the launch's total).
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+        const int mw = warp, quarter = mw & 3, half = mw >> 2;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const int jrow = quarter * 32 + lane;  // d_v index of this thread's S^T row
+        auto fail = [&]() {
+            s_abort_m = 1;
+            atomicExch(p.status, kStatusTimeout);
+        };
+        float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
-        Sf[i] = p.S0 ? p.S0[((size_t)bh * D + 64 * hcol + i) * D + jrow] : 0.f;
-    {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(Sf[2 * i], Sf[2 * i + 1]);
-        tmem_st32(tmem + TM_SBF + 32 * hcol + lane_off, pk);
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    uint32_t mma_phase = 0;
-    for (int ci = 0; ci < nchunks; ++ci) {
-        const uint32_t par = ci & 1;
-        const int L = min(C, T - ci * C);
-        const bool has_next = ci + 1 < nchunks;
-        // ---------------- wait for this chunk's inputs
-        if (!mbar_wait(&bar_g, par) || !mbar_wait(&bar_k, par) || !mbar_wait(&bar_bv, par) ||
-            !mbar_wait(&bar_q, par))
-            fail();
-        __syncthreads();
-        if (s_abort) break;
-        // ---------------- decay folding (elementwise, in place)
+        for (int i = 0; i < 64; ++i)
+            Sf[i] = p.S0 ? p.S0[((size_t)bh * D + 64 * half + i) * D + jrow] : 0.f;
         {
-            const int cb = warp & 1, tq = warp >> 1;  // channel block of 64, token quarter of 16
-            float Gl[16][2];
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(Sf[2 * i], Sf[2 * i + 1]);
+            tmem_st32(tmem + TM_SBF + 32 * half + lane_off, pk);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        named_sync(1, kGroup);
+        uint32_t mma_phase = 0;
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int buf = ci & 1;
+            const uint32_t fpar = (ci >> 1) & 1;
+            const int L = min(C, T - ci * C);
+            const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384, ov = OFF_V + buf * 16384;
+            // ---- factors of chunk ci are ready
+            if (!mbar_wait(&bar_fact[buf], fpar)) fail();
+            // ---- MMA 1: [A; P] = [E~; Q~] K~^T  and  [S^T E~^T | O^T] = S^T [E~; Q~]^T
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t qd = sdesc_sw128(sbase + oqe + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    mma_ss(tmem + TM_AP, qd, sdesc_sw128(sbase + ok + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                           IDESC_N64, ks > 0);
+                    mma_ts(tmem + TM_YO, tmem + TM_SBF + 8 * ks, qd, IDESC_N128, ks > 0);
+                }
+                mma_commit(&bar_mma);
+            }
+            if (!mbar_wait(&bar_mma, mma_phase)) fail();
+            mma_phase ^= 1;
+            tc_fence_after();
+            if (tid == 0) bulk_wait_read0();  // the previous output tile has left OFF_TT / OFF_PT
+            named_sync(1, kGroup);
+            if (s_abort_m) break;
+            {  // [A; P] readback: A -> fp32 scratch, P (masked) -> bf16 operand rows
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
+                tmem_wait_ld();
+                const int row = quarter * 32 + lane;
+                if (row < 64) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int j = 32 * half + u;
+                        sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
+                    }
+                } else {
+                    const int t = row - 64;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 32 * half + 8 * m + 2 * e;
+                            const float lo = (i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f;
+                            const float hi = (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f;
+                            w4[e] = pack_bf16x2(lo, hi);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + OFF_PT + sw128(t, 64 * half + 16 * m)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+            }
+            named_sync(1, kGroup);
+            // ---- warps 0-3: diagonal 16x16 blocks of T; warps 4-7: Y^T = X^T - S^T E~^T -> bf16 operand
+            if (mw < 4) {
+                invert_diag16(sA, sT, 16 * mw, lane);
+            } else {
+                const uint8_t *px = sm + ov;
+#pragma unroll
+                for (int hh2 = 0; hh2 < 2; ++hh2) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + TM_YO + 32 * hh2 + lane_off, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int t = 32 * hh2 + 2 * e;
+                        const uint32_t xo = (jrow >> 6) * 8192 + (jrow & 63) * 2;
+                        const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + (xo & ~127u) + sw128(t, xo & 127)));
+                        const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + (xo & ~127u) + sw128(t + 1, xo & 127)));
+                        pk[e] = pack_bf16x2(x0 - __uint_as_float(r[2 * e]), x1 - __uint_as_float(r[2 * e + 1]));
+                    }
+                    tmem_st16(tmem + TM_YB + 16 * hh2 + lane_off, pk);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            named_sync(1, kGroup);
+            if (tid == 0) mbar_arrive(&bar_m1[buf]);  // q/b/v buffers of this chunk are free
+            // ---- off-diagonal levels of T on warp-level TF32 MMAs (warps 0-3)
+            if (mw < 2) {  // 32x32 level: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
+                const int R = 32 * mw + 16, Cc = 32 * mw;
+                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc, y0, lane);
+                tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc + 8, y1, lane);
+                tile_store(sT + R * LDA + Cc, y0, 1.f, lane);
+                tile_store(sT + R * LDA + Cc + 8, y1, 1.f, lane);
+                __syncwarp();
+                float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc, x0, lane);
+                tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc + 8, x1, lane);
+                __syncwarp();
+                tile_store(sT + R * LDA + Cc, x0, -1.f, lane);
+                tile_store(sT + R * LDA + Cc + 8, x1, -1.f, lane);
+            }
+            if (mw < 4) {  // 64x64 level: T_BA = -T_BB (A_BA T_AA); warp: one 16-row tile, two 8-col tiles
+                named_sync(3, 128);
+                const int mt = mw & 1, n0 = 16 * (mw >> 1);
+                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0, y0, lane);
+                tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0 + 8, y1, lane);
+                tile_store(sT + (32 + 16 * mt) * LDA + n0, y0, 1.f, lane);
+                tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, y1, 1.f, lane);
+                named_sync(3, 128);
+                float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0, x0, lane);
+                tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0 + 8, x1, lane);
+                named_sync(3, 128);
+                tile_store(sT + (32 + 16 * mt) * LDA + n0, x0, -1.f, lane);
+                tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, x1, -1.f, lane);
+            }
+            named_sync(1, kGroup);
+            {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
+                const int i = tid >> 2, qq = tid & 3;
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j0 = 16 * qq + 8 * m + 2 * e;
+                        const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
+                        const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
+                        w4[e] = pack_bf16x2(lo, hi);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_TT + sw128(i, 32 * qq + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(1, kGroup);
+            // ---- MMA 2: U~^T = Y^T T^T
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(tmem + TM_UT, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + OFF_TT + ks * 32, 16, 1024),
+                           IDESC_N64, ks > 0);
+                mma_commit(&bar_mma);
+            }
+            if (!mbar_wait(&bar_mma, mma_phase)) fail();
+            mma_phase ^= 1;
+            tc_fence_after();
+            {  // U~^T -> bf16 TMEM operand
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_UT + 32 * half + lane_off, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                tmem_st16(tmem + TM_UB + 16 * half + lane_off, pk);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            named_sync(1, kGroup);
+            if (s_abort_m) break;
+            // ---- MMA 3: (K~^T U~)^T = U~^T K~ ;  O^T += U~^T P^T
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    mma_ts(tmem + TM_DS, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + ok + ks * 2048, 8192, 1024),
+                           IDESC_N128_BMN, ks > 0);
+                    mma_ts(tmem + TM_O, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + OFF_PT + ks * 32, 16, 1024),
+                           IDESC_N64, 1);
+                }
+                mma_commit(&bar_mma);
+            }
+            if (!mbar_wait(&bar_mma, mma_phase)) fail();
+            mma_phase ^= 1;
+            tc_fence_after();
+            {  // S = gamma (S + K~^T U~) in fp32 registers; bf16 copy back to TMEM
+                const float *gam = sGam + buf * 128 + 64 * half;
+#pragma unroll
+                for (int hh2 = 0; hh2 < 2; ++hh2) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + TM_DS + 64 * half + 32 * hh2 + lane_off, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        Sf[32 * hh2 + u] = gam[32 * hh2 + u] * (Sf[32 * hh2 + u] + __uint_as_float(r[u]));
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * hh2 + 2 * e], Sf[32 * hh2 + 2 * e + 1]);
+                    tmem_st16(tmem + TM_SBF + 32 * half + 16 * hh2 + lane_off, pk);
+                }
+            }
+            named_sync(1, kGroup);
+            if (tid == 0) mbar_arrive(&bar_kf[buf]);  // this chunk's k buffer and gamma are no longer read
+            {  // O^T -> bf16 output tile (row-major [t][channel]) in shared memory
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_O + 32 * half + lane_off, r);
+                tmem_wait_ld();
+                __nv_bfloat16 *so = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_O);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) so[(32 * half + u) * D + jrow] = __float2bfloat16_rn(__uint_as_float(r[u]));
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(1, kGroup);
+            if (L == C) {
+                if (tid == 0) {
+                    tma_store_3d(&maps.o, sm + OFF_O, 0, hh, bb * T + ci * C);
+                    bulk_commit();
+                }
+            } else {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
+                const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_O);
+                __nv_bfloat16 *dst = p.o + ((size_t)bb * T + (size_t)ci * C) * p.H * D + (size_t)hh * D;
+                for (int idx = tid; idx < L * D; idx += kGroup) dst[(size_t)(idx / D) * p.H * D + idx % D] = so[idx];
+                named_sync(1, kGroup);
+            }
+        }
+        if (!s_abort_m && p.S_T) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) p.S_T[((size_t)bh * D + 64 * half + i) * D + jrow] = Sf[i];
+        }
+        if (tid == 0) bulk_wait0();
+    } else {
+        // =========================== E group: decay folding, one chunk ahead ===========================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+        const int ew = warp - 8, etid = tid - kGroup;
+        const int cb = ew & 1, tg = ew >> 1;  // channel block of 64, token group of 16
+        const int ch = 64 * cb + 2 * lane;
+        auto fail = [&]() {
+            s_abort_e = 1;
+            atomicExch(p.status, kStatusTimeout);
+        };
+        auto issue = [&](int ci) {  // chunk ci's k, b, q, v, w into buffers ci & 1; log alpha into L2
+            const int y = bb * T + ci * C, bf = ci & 1;
+            mbar_expect_tx(&bar_in, 10 * 8192);
+            for (int a = 0; a < 2; ++a) {
+                tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in);
+                tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in);
+                tma_load_3d(sm + OFF_QE + bf * 32768 + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_in);
+                tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in);
+                tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in);
+            }
+            for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
+        };
+        if (etid == 0 && nchunks > 0) issue(0);
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int buf = ci & 1;
+            const int L = min(C, T - ci * C);
+            const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384, ov = OFF_V + buf * 16384;
+            // log alpha of this warp's 16 tokens x 2 channels, straight from L2
+            float2 gv[16];
+            const float *gsrc = p.g + ((size_t)bb * T + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
+                                          : make_float2(0.f, 0.f);
+            if (!mbar_wait(&bar_in, ci & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
-            const uint8_t *gatom = sm + OFF_G + (2 * cb + (lane >> 4)) * 8192;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int t = 16 * tq + i;
-                float2 gv = *reinterpret_cast<const float2 *>(gatom + sw128(t, 8 * (lane & 15)));
-                if (t >= L) gv = make_float2(0.f, 0.f);
-                run0 += gv.x;
-                run1 += gv.y;
-                Gl[i][0] = run0;
-                Gl[i][1] = run1;
+                run0 += gv[i].x;
+                run1 += gv[i].y;
+                gv[i] = make_float2(run0, run1);
             }
-            const int ch = 64 * cb + 2 * lane;
-            *reinterpret_cast<float2 *>(sTot + tq * 128 + ch) = make_float2(run0, run1);
-            __syncthreads();
+            *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
+            named_sync(2, kGroup);
+            if (s_abort_e) break;
             float c0 = 0.f, c1 = 0.f, gl0 = 0.f, gl1 = 0.f;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float2 tv = *reinterpret_cast<const float2 *>(sTot + u * 128 + ch);
-                if (u < tq) { c0 += tv.x; c1 += tv.y; }
+                if (u < tg) { c0 += tv.x; c1 += tv.y; }
                 gl0 += tv.x;
                 gl1 += tv.y;
             }
-            if (tq == 0) *reinterpret_cast<float2 *>(sGam + ch) = make_float2(__expf(gl0), __expf(gl1));
-            uint8_t *pe = sm + OFF_QE + cb * 16384;
+            if (tg == 0) *reinterpret_cast<float2 *>(sGam + buf * 128 + ch) = make_float2(__expf(gl0), __expf(gl1));
+            uint8_t *pe = sm + oqe + cb * 16384;
             uint8_t *pq = pe + 8192;
-            uint8_t *pk = sm + OFF_K + cb * 8192;
-            uint8_t *ph = sm + OFF_KH + cb * 8192;
-            uint8_t *pv = sm + OFF_V + cb * 8192;
+            uint8_t *pk = sm + ok + cb * 8192;
+            uint8_t *pv = sm + ov + cb * 8192;
             const uint8_t *pw = sm + OFF_W + cb * 8192;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int t = 16 * tq + i;
+                const int t = 16 * tg + i;
                 const uint32_t off = sw128(t, 4 * lane);
-                const float G0 = c0 + Gl[i][0], G1 = c1 + Gl[i][1];
+                const float G0 = c0 + gv[i].x, G1 = c1 + gv[i].y;
                 const float e0 = __expf(G0), e1 = __expf(G1);
                 const float m0 = __expf(-G0), m1 = __expf(-G1);
-                const float h0 = __expf(gl0 - G0), h1 = __expf(gl1 - G1);
                 uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
                 uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
                 uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
                 uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
-                uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
+                const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
                 if (t >= L) { qw = 0u; kw = 0u; bw = 0u; vw = 0u; }
                 const float k0 = bf_lo(kw), k1 = bf_hi(kw);
                 *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
                 *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
                 *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
-                *reinterpret_cast<uint32_t *>(ph + off) = pack_bf16x2(k0 * h0, k1 * h1);
                 *reinterpret_cast<uint32_t *>(pv + off) = pack_bf16x2(bf_lo(vw) * bf_lo(ww), bf_hi(vw) * bf_hi(ww));
             }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        // ---------------- MMA 1: [A; P] = [E~; Q~] K~^T ; prefetch g, w of the next chunk
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_QE + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(sbase + OFF_K + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                mma_ss(tmem + TM_AP, ad, bd, IDESC_N64, ks > 0);
-            }
-            mma_commit(&bar_mma);
-            if (has_next) issue_loads(ci + 1, 0);
-        }
-        if (!mbar_wait(&bar_mma, mma_phase)) fail();
-        mma_phase ^= 1;
-        tc_fence_after();
-        if (tid == 0 && has_next) issue_loads(ci + 1, 1);
-        {
-            uint32_t r[32];
-            tmem_ld32(tmem + TM_AP + 32 * hcol + lane_off, r);
-            tmem_wait_ld();
-            const int row = quarter * 32 + lane;
-            if (row < 64) {  // A, strictly lower
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int j = 32 * hcol + u;
-                    sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
-                }
-            } else {  // P, lower including the diagonal -> bf16 rows of SPT
-                const int t = row - 64;
-                uint8_t *dst = sm + OFF_PT;
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = 32 * hcol + 8 * m + 2 * e;
-                        const float lo = (i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f;
-                        const float hi = (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f;
-                        w4[e] = pack_bf16x2(lo, hi);
+            fence_proxy_async_smem();
+            named_sync(2, kGroup);
+            if (etid == 0) {
+                mbar_arrive(&bar_fact[buf]);
+                if (ci + 1 < nchunks) {
+                    // buffers (ci+1) & 1 were last used by chunk ci-1 in the M group
+                    if (ci >= 1) {
+                        const uint32_t ppar = ((ci - 1) >> 1) & 1;
+                        if (!mbar_wait(&bar_m1[buf ^ 1], ppar) || !mbar_wait(&bar_kf[buf ^ 1], ppar)) fail();
                     }
-                    *reinterpret_cast<uint4 *>(dst + sw128(t, 64 * hcol + 16 * m)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    fence_proxy_async_smem();
+                    issue(ci + 1);
                 }
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        if (s_abort) break;
-        // ---------------- T = (I + A)^-1, blocked by 16
-        if (tid < 64) {  // diagonal blocks: column j of block pblk
-            const int pblk = tid >> 4, j = tid & 15, r0 = 16 * pblk;
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float s = 0.f;
-#pragma unroll
-                for (int m = 0; m < i; ++m) s += sA[(r0 + i) * LDA + r0 + m] * x[m];
-                x[i] = (i > j) ? -s : (i == j ? 1.f : 0.f);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sT[(r0 + i) * LDA + r0 + j] = x[i];
-        }
-        __syncthreads();
-        {
-            const int rr = tid >> 4, ss = tid & 15;
-            for (int d = 1; d < 4; ++d) {
-                const int nb = 4 - d;
-                float y[3];
-#pragma unroll
-                for (int pb = 0; pb < 3; ++pb) {
-                    if (pb >= nb) break;
-                    const int R = 16 * (pb + d), Cc = 16 * pb;
-                    float s = 0.f;
-                    for (int m = pb; m < pb + d; ++m)
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) s += sA[(R + rr) * LDA + 16 * m + u] * sT[(16 * m + u) * LDA + Cc + ss];
-                    y[pb] = s;
-                }
-                // stash Y in the (still empty) T block, then T_block = -T_diag Y
-#pragma unroll
-                for (int pb = 0; pb < 3; ++pb)
-                    if (pb < nb) sT[(16 * (pb + d) + rr) * LDA + 16 * pb + ss] = y[pb];
-                __syncthreads();
-#pragma unroll
-                for (int pb = 0; pb < 3; ++pb) {
-                    if (pb >= nb) break;
-                    const int R = 16 * (pb + d), Cc = 16 * pb;
-                    float s = 0.f;
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) s += sT[(R + rr) * LDA + R + u] * sT[(R + u) * LDA + Cc + ss];
-                    y[pb] = -s;
-                }
-                __syncthreads();
-#pragma unroll
-                for (int pb = 0; pb < 3; ++pb)
-                    if (pb < nb) sT[(16 * (pb + d) + rr) * LDA + 16 * pb + ss] = y[pb];
-                __syncthreads();
-            }
-        }
-        {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
-            const int i = tid >> 2, qq = tid & 3;
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j0 = 16 * qq + 8 * m + 2 * e;
-                    const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
-                    const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
-                    w4[e] = pack_bf16x2(lo, hi);
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_TT + sw128(i, 32 * qq + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        // ---------------- MMA 2: W^T = E~^T T^T, U^T = X^T T^T
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t bd = sdesc_sw128(sbase + OFF_TT + ks * 32, 16, 1024);
-                mma_ss(tmem + TM_WT, sdesc_sw128(sbase + OFF_QE + ks * 2048, 16384, 1024), bd, IDESC_N64_AMN, ks > 0);
-                mma_ss(tmem + TM_UT, sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), bd, IDESC_N64_AMN, ks > 0);
-            }
-            mma_commit(&bar_mma);
-        }
-        if (!mbar_wait(&bar_mma, mma_phase)) fail();
-        mma_phase ^= 1;
-        tc_fence_after();
-        if (tid == 0 && has_next) {
-            fence_proxy_async_smem();
-            issue_loads(ci + 1, 2);
-        }
-        {  // -W^T -> bf16 rows (d_k) of SWT
-            uint32_t r[32];
-            tmem_ld32(tmem + TM_WT + 32 * hcol + lane_off, r);
-            tmem_wait_ld();
-            const int c = quarter * 32 + lane;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w4[e] = pack_bf16x2(-__uint_as_float(r[8 * m + 2 * e]), -__uint_as_float(r[8 * m + 2 * e + 1]));
-                *reinterpret_cast<uint4 *>(sm + OFF_WT + sw128(c, 64 * hcol + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_abort) break;
-        // ---------------- MMA 3: U~^T = U^T + S^T (-W^T);  O^T = S^T Q~^T
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ts(tmem + TM_UT, tmem + TM_SBF + 8 * ks, sdesc_sw128(sbase + OFF_WT + ks * 2048, 8192, 1024),
-                       IDESC_N64_BMN, 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ts(tmem + TM_OT, tmem + TM_SBF + 8 * ks,
-                       sdesc_sw128(sbase + OFF_QE + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), IDESC_N64,
-                       ks > 0);
-            mma_commit(&bar_mma);
-        }
-        if (!mbar_wait(&bar_mma, mma_phase)) fail();
-        mma_phase ^= 1;
-        tc_fence_after();
-        if (tid == 0 && has_next) {
-            fence_proxy_async_smem();
-            issue_loads(ci + 1, 3);
-        }
-        {  // U~^T -> bf16 TMEM operand
-            uint32_t r[32];
-            tmem_ld32(tmem + TM_UT + 32 * hcol + lane_off, r);
-            tmem_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-            tmem_st16(tmem + TM_UB + 16 * hcol + lane_off, pk);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (s_abort) break;
-        // ---------------- MMA 4: dS^T = U~^T K^ ;  O^T += U~^T P^T
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_ts(tmem + TM_DS, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + OFF_KH + ks * 2048, 8192, 1024),
-                       IDESC_N128_BMN, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_ts(tmem + TM_OT, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + OFF_PT + ks * 32, 16, 1024), IDESC_N64, 1);
-            mma_commit(&bar_mma);
-        }
-        if (!mbar_wait(&bar_mma, mma_phase)) fail();
-        mma_phase ^= 1;
-        tc_fence_after();
-        {  // state update in fp32 registers, bf16 copy back to TMEM
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32(tmem + TM_DS + 64 * hcol + 32 * half + lane_off, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int i = 32 * half + u;
-                    Sf[i] = sGam[64 * hcol + i] * Sf[i] + __uint_as_float(r[u]);
-                }
-            }
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(Sf[2 * i], Sf[2 * i + 1]);
-            tmem_st32(tmem + TM_SBF + 32 * hcol + lane_off, pk);
-        }
-        {  // O^T -> o (bf16)
-            uint32_t r[32];
-            tmem_ld32(tmem + TM_OT + 32 * hcol + lane_off, r);
-            tmem_wait_ld();
-            __nv_bfloat16 *orow = p.o + ((size_t)bb * T + (size_t)ci * C) * p.H * D + (size_t)hh * D + jrow;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int t = 32 * hcol + u;
-                if (t < L) orow[(size_t)t * p.H * D] = __float2bfloat16_rn(__uint_as_float(r[u]));
-            }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
-    }
-    if (!s_abort && p.S_T) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) p.S_T[((size_t)bh * D + 64 * hcol + i) * D + jrow] = Sf[i];
     }
     tc_fence_before();
     __syncthreads();
@@ -499,19 +595,22 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 3-D view (channel, head, token) of a [B,T,H,D] tensor; box = (inner, 1, 64 tokens), 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H)
+// 3-D view (channel, head, token) of a [B,T,H,D] tensor.  Loads: box = (one 128-byte
+// row of channels, 1 head, 64 tokens) with the 128-byte swizzle; the output store:
+// box = (all 128 channels, 1, 64 tokens), no swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, bool store = false)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t es = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
     cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es};
-    cuuint32_t box[3] = {fp32 ? 32u : 64u, 1u, (cuuint32_t)C};
+    cuuint32_t box[3] = {store ? (cuuint32_t)D : (fp32 ? 32u : 64u), 1u, (cuuint32_t)C};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
-               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -522,7 +621,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, int *status, c
     TcMaps maps;
     if (!make_map(&maps.q, pr.q, false, pr.B, pr.T, pr.H) || !make_map(&maps.k, pr.k, false, pr.B, pr.T, pr.H) ||
         !make_map(&maps.v, pr.v, false, pr.B, pr.T, pr.H) || !make_map(&maps.b, pr.b, false, pr.B, pr.T, pr.H) ||
-        !make_map(&maps.w, pr.w, false, pr.B, pr.T, pr.H) || !make_map(&maps.g, pr.g, true, pr.B, pr.T, pr.H))
+        !make_map(&maps.w, pr.w, false, pr.B, pr.T, pr.H) || !make_map(&maps.g, pr.g, true, pr.B, pr.T, pr.H) ||
+        !make_map(&maps.o, o, false, pr.B, pr.T, pr.H, true))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
@@ -530,7 +630,7 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, int *status, c
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    TcParams prm{pr.B, pr.T, pr.H, pr.S0, (__nv_bfloat16 *)o, S_T, status};
+    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, status};
     fwd_tc_kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
     return cudaGetLastError();
 }
