@@ -8,27 +8,30 @@
 //   G  = inclusive cumulative sum of log alpha over the chunk (fp32)
 //   Q~ = q e^G,  E~ = (b.k) e^G,  K~ = k e^-G,  gamma = e^G_L,  X = w.v
 //   [A; P] = [E~; Q~] K~^T          A strictly lower, P lower incl. (one M=128 MMA)
-//   Y   = X - E~ S                  (the gated value minus what the erase-weighted
-//                                    keys read from the chunk-start state)
 //   T   = (I + A)^-1                 blocked: 16x16 diagonal blocks by substitution,
 //                                    the doubling levels on warp-level TF32 MMAs
+//   Y   = X - E~ S                  (the gated value minus what the erase-weighted
+//                                    keys read from the chunk-start state)
 //   U~  = T Y                        (= (I+A)^-1 (w.V) - (I+A)^-1 E~ S)
 //   O   = Q~ S + P U~
 //   S  <- Diag(gamma) (S + K~^T U~)  (K~ e^G_L is the decay from token t to the
 //                                    chunk end, so gamma is applied once, in fp32)
-// Everything is formulated transposed (S^T, Y^T, U~^T, O^T with d_v as the row
-// index) so that every tcgen05.mma has M = 128; S^T, Y^T and U~^T are TMEM
-// operands, and S^T [E~; Q~]^T is one N = 128 product.
+// Everything S-dependent is formulated transposed (S^T, Y^T, U~^T, O^T with
+// d_v as the row index) so that every tcgen05.mma has M = 128; S^T, Y^T and
+// U~^T are TMEM operands, and S^T [E~; Q~]^T is one N = 128 product.
 //
 // Work decomposition: one CTA per (batch, head), two warp groups that run one
-// chunk apart.  The E group (warps 8-15) folds the decay of chunk c+1 into its
-// factors (shared-memory buffers for q/b, k and v are double-buffered, log
-// alpha is read from L2 where a TMA prefetch has put it) while the M group
-// (warps 0-7) runs chunk c's chain: MMA, readback, solve, MMA, readback, MMA,
-// state update and output.  Warp m of M owns TMEM lanes 32 (m & 3) .. +31 and
-// column half (m >> 2) of every readback and holds its 64 columns of S^T in
-// fp32 registers.  The output tile is staged in shared memory and written by a
-// TMA store.  Cross-group hand-offs use mbarriers, one per chunk parity.
+// chunk apart.  The E group (warps 8-15) does the key-side work that does not
+// depend on the state for chunk c+1: decay folding (log alpha is read from L2
+// where a TMA prefetch has put it), the [A; P] product, and T = (I+A)^-1.  The
+// M group (warps 0-7) runs chunk c's state chain: S^T [E~; Q~]^T, Y, U~, the
+// state update and the output; at the end of its chunk it folds the next
+// chunk's write gate into its values (X = w.v) and releases the chunk's
+// buffers, into which an otherwise idle E warp then loads the chunk after.  All buffers handed from E to M are double-buffered
+// by chunk parity; mbarriers, one per parity, carry the hand-offs.  Warp m of
+// M owns TMEM lanes 32 (m & 3) .. +31 and column half (m >> 2) of every
+// readback and holds its 64 columns of S^T in fp32 registers.  The output tile
+// is staged in shared memory and written by a TMA store.
 #include <cuda.h>
 
 #include "gdn2_internal.cuh"
@@ -45,15 +48,14 @@ constexpr int kThreads = 512;
 constexpr int kGroup = 256;  // threads per warp group
 constexpr int LDA = 68;      // fp32 row stride of the A / T scratch
 
-// shared-memory map (bytes from a 1024-byte aligned base)
-constexpr uint32_t OFF_QE = 0;          // 2 x [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
-constexpr uint32_t OFF_K = 65536;       // 2 x K~ (raw k), 2 atoms
-constexpr uint32_t OFF_V = 98304;       // 2 x X = w.v (raw v), 2 atoms
+// shared-memory map (bytes from a 1024-byte aligned base); [2] = by chunk parity
+constexpr uint32_t OFF_QE = 0;          // [2] x [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
+constexpr uint32_t OFF_K = 65536;       // [2] x K~ (raw k), 2 atoms
+constexpr uint32_t OFF_V = 98304;       // [2] x X = w.v (raw v), 2 atoms
 constexpr uint32_t OFF_W = 131072;      // raw w, 2 atoms
-constexpr uint32_t OFF_TT = 147456;     // T: 64 rows (i) x 64 (j), bf16      } output tile (64 x 128
-constexpr uint32_t OFF_PT = 155648;     // P: 64 rows (t) x 64 (i), bf16      }  bf16) after MMA 3
-constexpr uint32_t OFF_O = OFF_TT;
-constexpr uint32_t OFF_SA = 163840;     // A fp32 [64][LDA]
+constexpr uint32_t OFF_TP = 147456;     // [2] x [T bf16 (64 x 64) | P bf16 (64 x 64)]; the output
+                                        //  tile (64 x 128 bf16, row-major) after M is done with them
+constexpr uint32_t OFF_SA = 180224;     // A fp32 [64][LDA]
 constexpr uint32_t OFF_ST = OFF_SA + 64 * LDA * 4;   // T fp32 [64][LDA]
 constexpr uint32_t OFF_TOT = OFF_ST + 64 * LDA * 4;  // per-group decay totals [4][128] fp32
 constexpr uint32_t OFF_GAM = OFF_TOT + 4 * 128 * 4;  // gamma [2][128] fp32
@@ -61,19 +63,25 @@ constexpr uint32_t SMEM_USED = OFF_GAM + 2 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for the 1024-byte alignment
 
 // TMEM columns
-constexpr uint32_t TM_SBF = 0;     // S^T bf16 (A operand), 64 columns
-constexpr uint32_t TM_AP = 64;     // [A; P] fp32
-constexpr uint32_t TM_YO = 128;    // [S^T E~^T | O^T] fp32, 128 columns
+constexpr uint32_t TM_SBF = 0;     // S^T bf16 (A operand), 64 columns                 (M)
+constexpr uint32_t TM_AP = 64;     // [A; P] fp32                                      (E)
+constexpr uint32_t TM_YO = 128;    // [S^T E~^T | O^T] fp32, 128 columns               (M)
 constexpr uint32_t TM_O = 192;     //   O^T half
-constexpr uint32_t TM_UT = 256;    // U~^T fp32
-constexpr uint32_t TM_YB = 320;    // Y^T bf16 (A operand), 32 columns
-constexpr uint32_t TM_UB = 352;    // U~^T bf16 (A operand), 32 columns
-constexpr uint32_t TM_DS = 384;    // (K~^T U~)^T fp32, 128 columns
+constexpr uint32_t TM_UT = 256;    // U~^T fp32                                        (M)
+constexpr uint32_t TM_YB = 320;    // Y^T bf16 (A operand), 32 columns                 (M)
+constexpr uint32_t TM_UB = 352;    // U~^T bf16 (A operand), 32 columns                (M)
+constexpr uint32_t TM_DS = 384;    // (K~^T U~)^T fp32, 128 columns                    (M)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_N128 = idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_N128_BMN = idesc_bf16(128, 128, 0, 1);
+
+// Register split: the launch holds 512 x 128 registers; M takes 152 per thread and
+// E 104 (256 x 152 + 256 x 104 = 65536, exactly the launch's total).
+constexpr int kRegM = 152;
+constexpr int kRegE = 104;
+static_assert(kGroup * kRegM + kGroup * kRegE == kThreads * 128, "register split must match the launch");
 
 struct TcParams {
     int B, T, H;
@@ -188,11 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // bar_in: this chunk's k, b, q, v, w have landed (E waits)      bar_mma: M's tcgen05 batches
-    // bar_fact[2]: E -> M, the factors of a chunk are ready          bar_m1[2]: M -> E, q/b/v buffers free
-    // bar_kf[2]: M -> E, the k buffer is free
-    __shared__ __align__(8) uint64_t bar_in, bar_mma, bar_fact[2], bar_m1[2], bar_kf[2];
+    // Offset (not integer-cast) so that the compiler keeps the shared address space and
+    // emits shared-memory instructions for every access through `sm`.
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    // bar_in[2]: a chunk's k, b, q, v, w have landed     bar_emma / bar_mma: E's / M's tcgen05 batches
+    // bar_fact[2]: E -> M, factors, P and T of a chunk   bar_mdone[2]: M -> E, a chunk's buffers are free
+    __shared__ __align__(8) uint64_t bar_in[2], bar_emma, bar_mma, bar_fact[2], bar_mdone[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort_m, s_abort_e;
 
@@ -210,12 +219,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     if (tid == 0) {
         s_abort_m = 0;
         s_abort_e = 0;
-        mbar_init(&bar_in, 1);
+        mbar_init(&bar_emma, 1);
         mbar_init(&bar_mma, 1);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_in[i], 1);
             mbar_init(&bar_fact[i], 1);
-            mbar_init(&bar_m1[i], 1);
-            mbar_init(&bar_kf[i], 1);
+            mbar_init(&bar_mdone[i], 1);
         }
         fence_mbar_init();
         prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.v);
@@ -232,11 +241,25 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
+    // TMA loads of chunk ci's k, b, q, v, w into the buffers of parity ci & 1, log alpha into L2.
+    // The issuing thread may block while the TMA engine drains earlier boxes, so the loads are
+    // issued from an E warp that is idle during the solve.
+    auto issue = [&](int ci) {
+        const int y = bb * T + ci * C, bf = ci & 1;
+        mbar_expect_tx(&bar_in[bf], 10 * 8192);
+        for (int a = 0; a < 2; ++a) {
+            tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in[bf]);
+            tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in[bf]);
+            tma_load_3d(sm + OFF_QE + bf * 32768 + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_in[bf]);
+            tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in[bf]);
+            tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
+        }
+        for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
+    };
+
     if (is_m) {
-        // =========================== M group: the per-chunk tensor-core chain ===========================
-        // Register split: the launch holds 512 x 128 registers; M takes 176 per thread and E
-        // gives back to 80 (256 x 176 + 256 x 80 = 65536, exactly the launch's total).
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+        // =========================== M group: the state chain of chunk ci ===========================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegM) : "memory");
         const int mw = warp, quarter = mw & 3, half = mw >> 2;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const int jrow = quarter * 32 + lane;  // d_v index of this thread's S^T row
@@ -244,158 +267,91 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             s_abort_m = 1;
             atomicExch(p.status, kStatusTimeout);
         };
+        // X = w.v of chunk ci, in place of v (one token row of 64 channels per warp step)
+        auto fold_value = [&](int ci) {
+            const int Lc = min(C, T - ci * C);
+            uint8_t *pv = sm + OFF_V + (ci & 1) * 16384;
+            const uint8_t *pw = sm + OFF_W;
+#pragma unroll
+            for (int it = 0; it < 2 * C / 8; ++it) {  // (atom, token) rows, one per warp step
+                const int idx = mw + 8 * it;
+                const int a = idx >> 6, t = idx & 63;
+                const uint32_t off = a * 8192 + sw128(t, 4 * lane);
+                const uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
+                const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
+                *reinterpret_cast<uint32_t *>(pv + off) =
+                    (t < Lc) ? pack_bf16x2(bf_lo(vw) * bf_lo(ww), bf_hi(vw) * bf_hi(ww)) : 0u;
+            }
+        };
+        if (tid == 0 && nchunks > 0) issue(0);
+        if (nchunks > 0) {
+            if (!mbar_wait(&bar_in[0], 0)) fail();
+            fold_value(0);
+        }
+        fence_proxy_async_smem();
+        named_sync(1, kGroup);
+        if (tid == 0 && nchunks > 1) issue(1);  // w(1) may only land after w(0) was folded
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
             Sf[i] = p.S0 ? p.S0[((size_t)bh * D + 64 * half + i) * D + jrow] : 0.f;
-        {
-            uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(Sf[2 * i], Sf[2 * i + 1]);
-            tmem_st32(tmem + TM_SBF + 32 * half + lane_off, pk);
-            tmem_wait_st();
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * h2 + 2 * e], Sf[32 * h2 + 2 * e + 1]);
+            tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
         }
+        tmem_wait_st();
         tc_fence_before();
         named_sync(1, kGroup);
         uint32_t mma_phase = 0;
         for (int ci = 0; ci < nchunks; ++ci) {
             const int buf = ci & 1;
-            const uint32_t fpar = (ci >> 1) & 1;
             const int L = min(C, T - ci * C);
             const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384, ov = OFF_V + buf * 16384;
-            // ---- factors of chunk ci are ready
-            if (!mbar_wait(&bar_fact[buf], fpar)) fail();
-            // ---- MMA 1: [A; P] = [E~; Q~] K~^T  and  [S^T E~^T | O^T] = S^T [E~; Q~]^T
+            const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
+            // ---- factors, P and T of chunk ci are ready
+            if (!mbar_wait(&bar_fact[buf], (ci >> 1) & 1)) fail();
+            // ---- MMA 1: [S^T E~^T | O^T] = S^T [E~; Q~]^T
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t qd = sdesc_sw128(sbase + oqe + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    mma_ss(tmem + TM_AP, qd, sdesc_sw128(sbase + ok + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                           IDESC_N64, ks > 0);
-                    mma_ts(tmem + TM_YO, tmem + TM_SBF + 8 * ks, qd, IDESC_N128, ks > 0);
-                }
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ts(tmem + TM_YO, tmem + TM_SBF + 8 * ks,
+                           sdesc_sw128(sbase + oqe + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), IDESC_N128, ks > 0);
                 mma_commit(&bar_mma);
             }
             if (!mbar_wait(&bar_mma, mma_phase)) fail();
             mma_phase ^= 1;
             tc_fence_after();
-            if (tid == 0) bulk_wait_read0();  // the previous output tile has left OFF_TT / OFF_PT
-            named_sync(1, kGroup);
-            if (s_abort_m) break;
-            {  // [A; P] readback: A -> fp32 scratch, P (masked) -> bf16 operand rows
+            {  // Y^T = X^T - S^T E~^T -> bf16 TMEM operand (this warp: 32 tokens)
+                const uint8_t *px = sm + ov + (jrow >> 6) * 8192;
+                const uint32_t xb = (jrow & 63) * 2;
                 uint32_t r[32];
-                tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
+                tmem_ld32(tmem + TM_YO + 32 * half + lane_off, r);
                 tmem_wait_ld();
-                const int row = quarter * 32 + lane;
-                if (row < 64) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int j = 32 * half + u;
-                        sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
-                    }
-                } else {
-                    const int t = row - 64;
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = 32 * half + 8 * m + 2 * e;
-                            const float lo = (i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f;
-                            const float hi = (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f;
-                            w4[e] = pack_bf16x2(lo, hi);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OFF_PT + sw128(t, 64 * half + 16 * m)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
+                for (int e = 0; e < 16; ++e) {
+                    const int t = 32 * half + 2 * e;
+                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t, xb)));
+                    const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t + 1, xb)));
+                    pk[e] = pack_bf16x2(x0 - __uint_as_float(r[2 * e]), x1 - __uint_as_float(r[2 * e + 1]));
                 }
-            }
-            named_sync(1, kGroup);
-            // ---- warps 0-3: diagonal 16x16 blocks of T; warps 4-7: Y^T = X^T - S^T E~^T -> bf16 operand
-            if (mw < 4) {
-                invert_diag16(sA, sT, 16 * mw, lane);
-            } else {
-                const uint8_t *px = sm + ov;
-#pragma unroll
-                for (int hh2 = 0; hh2 < 2; ++hh2) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + TM_YO + 32 * hh2 + lane_off, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int t = 32 * hh2 + 2 * e;
-                        const uint32_t xo = (jrow >> 6) * 8192 + (jrow & 63) * 2;
-                        const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + (xo & ~127u) + sw128(t, xo & 127)));
-                        const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + (xo & ~127u) + sw128(t + 1, xo & 127)));
-                        pk[e] = pack_bf16x2(x0 - __uint_as_float(r[2 * e]), x1 - __uint_as_float(r[2 * e + 1]));
-                    }
-                    tmem_st16(tmem + TM_YB + 16 * hh2 + lane_off, pk);
-                }
+                tmem_st16(tmem + TM_YB + 16 * half + lane_off, pk);
                 tmem_wait_st();
             }
             tc_fence_before();
             named_sync(1, kGroup);
-            if (tid == 0) mbar_arrive(&bar_m1[buf]);  // q/b/v buffers of this chunk are free
-            // ---- off-diagonal levels of T on warp-level TF32 MMAs (warps 0-3)
-            if (mw < 2) {  // 32x32 level: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
-                const int R = 32 * mw + 16, Cc = 32 * mw;
-                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc, y0, lane);
-                tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc + 8, y1, lane);
-                tile_store(sT + R * LDA + Cc, y0, 1.f, lane);
-                tile_store(sT + R * LDA + Cc + 8, y1, 1.f, lane);
-                __syncwarp();
-                float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc, x0, lane);
-                tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc + 8, x1, lane);
-                __syncwarp();
-                tile_store(sT + R * LDA + Cc, x0, -1.f, lane);
-                tile_store(sT + R * LDA + Cc + 8, x1, -1.f, lane);
-            }
-            if (mw < 4) {  // 64x64 level: T_BA = -T_BB (A_BA T_AA); warp: one 16-row tile, two 8-col tiles
-                named_sync(3, 128);
-                const int mt = mw & 1, n0 = 16 * (mw >> 1);
-                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0, y0, lane);
-                tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0 + 8, y1, lane);
-                tile_store(sT + (32 + 16 * mt) * LDA + n0, y0, 1.f, lane);
-                tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, y1, 1.f, lane);
-                named_sync(3, 128);
-                float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-                tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0, x0, lane);
-                tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0 + 8, x1, lane);
-                named_sync(3, 128);
-                tile_store(sT + (32 + 16 * mt) * LDA + n0, x0, -1.f, lane);
-                tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, x1, -1.f, lane);
-            }
-            named_sync(1, kGroup);
-            {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
-                const int i = tid >> 2, qq = tid & 3;
-#pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j0 = 16 * qq + 8 * m + 2 * e;
-                        const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
-                        const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
-                        w4[e] = pack_bf16x2(lo, hi);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_TT + sw128(i, 32 * qq + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_sync(1, kGroup);
+            if (s_abort_m) break;
             // ---- MMA 2: U~^T = Y^T T^T
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ts(tmem + TM_UT, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + OFF_TT + ks * 32, 16, 1024),
-                           IDESC_N64, ks > 0);
+                    mma_ts(tmem + TM_UT, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + ott + ks * 32, 16, 1024), IDESC_N64,
+                           ks > 0);
                 mma_commit(&bar_mma);
             }
             if (!mbar_wait(&bar_mma, mma_phase)) fail();
@@ -421,8 +377,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 for (int ks = 0; ks < 4; ++ks) {
                     mma_ts(tmem + TM_DS, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + ok + ks * 2048, 8192, 1024),
                            IDESC_N128_BMN, ks > 0);
-                    mma_ts(tmem + TM_O, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + OFF_PT + ks * 32, 16, 1024),
-                           IDESC_N64, 1);
+                    mma_ts(tmem + TM_O, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64, 1);
                 }
                 mma_commit(&bar_mma);
             }
@@ -432,26 +387,24 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             {  // S = gamma (S + K~^T U~) in fp32 registers; bf16 copy back to TMEM
                 const float *gam = sGam + buf * 128 + 64 * half;
 #pragma unroll
-                for (int hh2 = 0; hh2 < 2; ++hh2) {
+                for (int h2 = 0; h2 < 2; ++h2) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + TM_DS + 64 * half + 32 * hh2 + lane_off, r);
+                    tmem_ld32(tmem + TM_DS + 64 * half + 32 * h2 + lane_off, r);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int u = 0; u < 32; ++u)
-                        Sf[32 * hh2 + u] = gam[32 * hh2 + u] * (Sf[32 * hh2 + u] + __uint_as_float(r[u]));
+                        Sf[32 * h2 + u] = gam[32 * h2 + u] * (Sf[32 * h2 + u] + __uint_as_float(r[u]));
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * hh2 + 2 * e], Sf[32 * hh2 + 2 * e + 1]);
-                    tmem_st16(tmem + TM_SBF + 32 * half + 16 * hh2 + lane_off, pk);
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * h2 + 2 * e], Sf[32 * h2 + 2 * e + 1]);
+                    tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
                 }
             }
-            named_sync(1, kGroup);
-            if (tid == 0) mbar_arrive(&bar_kf[buf]);  // this chunk's k buffer and gamma are no longer read
-            {  // O^T -> bf16 output tile (row-major [t][channel]) in shared memory
+            {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
                 uint32_t r[32];
                 tmem_ld32(tmem + TM_O + 32 * half + lane_off, r);
                 tmem_wait_ld();
-                __nv_bfloat16 *so = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_O);
+                __nv_bfloat16 *so = reinterpret_cast<__nv_bfloat16 *>(sm + ott);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) so[(32 * half + u) * D + jrow] = __float2bfloat16_rn(__uint_as_float(r[u]));
             }
@@ -461,15 +414,24 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             named_sync(1, kGroup);
             if (L == C) {
                 if (tid == 0) {
-                    tma_store_3d(&maps.o, sm + OFF_O, 0, hh, bb * T + ci * C);
+                    tma_store_3d(&maps.o, sm + ott, 0, hh, bb * T + ci * C);
                     bulk_commit();
+                    bulk_wait_read0();
                 }
             } else {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
-                const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_O);
+                const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
                 __nv_bfloat16 *dst = p.o + ((size_t)bb * T + (size_t)ci * C) * p.H * D + (size_t)hh * D;
                 for (int idx = tid; idx < L * D; idx += kGroup) dst[(size_t)(idx / D) * p.H * D + idx % D] = so[idx];
                 named_sync(1, kGroup);
             }
+            // ---- next chunk's values (w is single-buffered), then chunk ci+2's loads into this parity
+            if (ci + 1 < nchunks) {
+                if (!mbar_wait(&bar_in[buf ^ 1], ((ci + 1) >> 1) & 1)) fail();
+                fold_value(ci + 1);
+            }
+            fence_proxy_async_smem();
+            named_sync(1, kGroup);
+            if (tid == 0) mbar_arrive(&bar_mdone[buf]);  // this parity's buffers and w are free
         }
         if (!s_abort_m && p.S_T) {
 #pragma unroll
@@ -477,32 +439,22 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         }
         if (tid == 0) bulk_wait0();
     } else {
-        // =========================== E group: decay folding, one chunk ahead ===========================
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+        // =========== E group: decay folding, [A; P] and T = (I+A)^-1, one chunk ahead of M ===========
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegE) : "memory");
         const int ew = warp - 8, etid = tid - kGroup;
-        const int cb = ew & 1, tg = ew >> 1;  // channel block of 64, token group of 16
+        const int quarter = ew & 3, half = ew >> 2;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const int cb = ew & 1, tg = ew >> 1;  // elementwise: channel block of 64, token group of 16
         const int ch = 64 * cb + 2 * lane;
         auto fail = [&]() {
             s_abort_e = 1;
             atomicExch(p.status, kStatusTimeout);
         };
-        auto issue = [&](int ci) {  // chunk ci's k, b, q, v, w into buffers ci & 1; log alpha into L2
-            const int y = bb * T + ci * C, bf = ci & 1;
-            mbar_expect_tx(&bar_in, 10 * 8192);
-            for (int a = 0; a < 2; ++a) {
-                tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in);
-                tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in);
-                tma_load_3d(sm + OFF_QE + bf * 32768 + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_in);
-                tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in);
-                tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in);
-            }
-            for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
-        };
-        if (etid == 0 && nchunks > 0) issue(0);
         for (int ci = 0; ci < nchunks; ++ci) {
             const int buf = ci & 1;
             const int L = min(C, T - ci * C);
-            const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384, ov = OFF_V + buf * 16384;
+            const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384;
+            const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
             // log alpha of this warp's 16 tokens x 2 channels, straight from L2
             float2 gv[16];
             const float *gsrc = p.g + ((size_t)bb * T + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
@@ -510,7 +462,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             for (int i = 0; i < 16; ++i)
                 gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
                                           : make_float2(0.f, 0.f);
-            if (!mbar_wait(&bar_in, ci & 1)) fail();
+            if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -521,53 +473,142 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
             named_sync(2, kGroup);
             if (s_abort_e) break;
-            float c0 = 0.f, c1 = 0.f, gl0 = 0.f, gl1 = 0.f;
+            {  // decay folding, in place
+                float c0 = 0.f, c1 = 0.f, gl0 = 0.f, gl1 = 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float2 tv = *reinterpret_cast<const float2 *>(sTot + u * 128 + ch);
-                if (u < tg) { c0 += tv.x; c1 += tv.y; }
-                gl0 += tv.x;
-                gl1 += tv.y;
-            }
-            if (tg == 0) *reinterpret_cast<float2 *>(sGam + buf * 128 + ch) = make_float2(__expf(gl0), __expf(gl1));
-            uint8_t *pe = sm + oqe + cb * 16384;
-            uint8_t *pq = pe + 8192;
-            uint8_t *pk = sm + ok + cb * 8192;
-            uint8_t *pv = sm + ov + cb * 8192;
-            const uint8_t *pw = sm + OFF_W + cb * 8192;
+                for (int u = 0; u < 4; ++u) {
+                    const float2 tv = *reinterpret_cast<const float2 *>(sTot + u * 128 + ch);
+                    if (u < tg) { c0 += tv.x; c1 += tv.y; }
+                    gl0 += tv.x;
+                    gl1 += tv.y;
+                }
+                if (tg == 0) *reinterpret_cast<float2 *>(sGam + buf * 128 + ch) = make_float2(__expf(gl0), __expf(gl1));
+                uint8_t *pe = sm + oqe + cb * 16384;
+                uint8_t *pq = pe + 8192;
+                uint8_t *pk = sm + ok + cb * 8192;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = 16 * tg + i;
-                const uint32_t off = sw128(t, 4 * lane);
-                const float G0 = c0 + gv[i].x, G1 = c1 + gv[i].y;
-                const float e0 = __expf(G0), e1 = __expf(G1);
-                const float m0 = __expf(-G0), m1 = __expf(-G1);
-                uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
-                uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
-                uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
-                uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
-                const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
-                if (t >= L) { qw = 0u; kw = 0u; bw = 0u; vw = 0u; }
-                const float k0 = bf_lo(kw), k1 = bf_hi(kw);
-                *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
-                *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
-                *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
-                *reinterpret_cast<uint32_t *>(pv + off) = pack_bf16x2(bf_lo(vw) * bf_lo(ww), bf_hi(vw) * bf_hi(ww));
+                for (int i = 0; i < 16; ++i) {
+                    const int t = 16 * tg + i;
+                    const uint32_t off = sw128(t, 4 * lane);
+                    const float G0 = c0 + gv[i].x, G1 = c1 + gv[i].y;
+                    const float e0 = __expf(G0), e1 = __expf(G1);
+                    const float m0 = __expf(-G0), m1 = __expf(-G1);
+                    uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
+                    uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
+                    uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
+                    if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
+                    const float k0 = bf_lo(kw), k1 = bf_hi(kw);
+                    *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
+                    *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
+                    *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
+                }
             }
             fence_proxy_async_smem();
             named_sync(2, kGroup);
+            // ---- [A; P] = [E~; Q~] K~^T on the tensor core
             if (etid == 0) {
-                mbar_arrive(&bar_fact[buf]);
-                if (ci + 1 < nchunks) {
-                    // buffers (ci+1) & 1 were last used by chunk ci-1 in the M group
-                    if (ci >= 1) {
-                        const uint32_t ppar = ((ci - 1) >> 1) & 1;
-                        if (!mbar_wait(&bar_m1[buf ^ 1], ppar) || !mbar_wait(&bar_kf[buf ^ 1], ppar)) fail();
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ss(tmem + TM_AP, sdesc_sw128(sbase + oqe + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                           sdesc_sw128(sbase + ok + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_N64, ks > 0);
+                mma_commit(&bar_emma);
+            }
+            if (!mbar_wait(&bar_emma, ci & 1)) fail();
+            tc_fence_after();
+            {  // A -> fp32 scratch (strictly lower), P -> bf16 operand rows (lower incl.)
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
+                tmem_wait_ld();
+                const int row = quarter * 32 + lane;
+                if (row < 64) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int j = 32 * half + u;
+                        sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
                     }
-                    fence_proxy_async_smem();
-                    issue(ci + 1);
+                } else {
+                    const int t = row - 64;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 32 * half + 8 * m + 2 * e;
+                            const float lo = (i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f;
+                            const float hi = (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f;
+                            w4[e] = pack_bf16x2(lo, hi);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + opt + sw128(t, 64 * half + 16 * m)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
                 }
             }
+            tc_fence_before();
+            named_sync(2, kGroup);
+            if (s_abort_e) break;
+            // ---- T = (I + A)^-1 on warps 8-11: diagonal 16x16 blocks, then the doubling levels on
+            //      warp-level TF32 MMAs; meanwhile warp 12 issues the next chunk's loads
+            if (ew < 4) {
+                invert_diag16(sA, sT, 16 * ew, lane);
+                named_sync(3, 128);
+                if (ew < 2) {  // 32x32 level: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
+                    const int R = 32 * ew + 16, Cc = 32 * ew;
+                    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc, y0, lane);
+                    tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc + 8, y1, lane);
+                    tile_store(sT + R * LDA + Cc, y0, 1.f, lane);
+                    tile_store(sT + R * LDA + Cc + 8, y1, 1.f, lane);
+                    __syncwarp();
+                    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc, x0, lane);
+                    tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc + 8, x1, lane);
+                    __syncwarp();
+                    tile_store(sT + R * LDA + Cc, x0, -1.f, lane);
+                    tile_store(sT + R * LDA + Cc + 8, x1, -1.f, lane);
+                }
+                named_sync(3, 128);
+                {  // 64x64 level: T_BA = -T_BB (A_BA T_AA); warp: one 16-row tile, two 8-col tiles
+                    const int mt = ew & 1, n0 = 16 * (ew >> 1);
+                    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0, y0, lane);
+                    tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0 + 8, y1, lane);
+                    tile_store(sT + (32 + 16 * mt) * LDA + n0, y0, 1.f, lane);
+                    tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, y1, 1.f, lane);
+                    named_sync(3, 128);
+                    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0, x0, lane);
+                    tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0 + 8, x1, lane);
+                    named_sync(3, 128);
+                    tile_store(sT + (32 + 16 * mt) * LDA + n0, x0, -1.f, lane);
+                    tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, x1, -1.f, lane);
+                }
+                named_sync(3, 128);
+                {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
+                    const int i = etid >> 1, hf = etid & 1;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j0 = 32 * hf + 8 * m + 2 * e;
+                            const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
+                            const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
+                            w4[e] = pack_bf16x2(lo, hi);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + ott + sw128(i, 64 * hf + 16 * m)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+            } else if (ew == 4 && lane == 0 && ci >= 1 && ci + 1 < nchunks) {
+                // chunk ci+1's loads go to the buffers chunk ci-1 used; M frees them with bar_mdone
+                if (!mbar_wait(&bar_mdone[buf ^ 1], ((ci - 1) >> 1) & 1)) fail();
+                fence_proxy_async_smem();
+                issue(ci + 1);
+            }
+            named_sync(2, kGroup);
+            if (etid == 0) mbar_arrive(&bar_fact[buf]);
         }
     }
     tc_fence_before();
