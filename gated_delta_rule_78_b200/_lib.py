@@ -18,10 +18,13 @@ LIB_PATH = os.path.join(_HERE, "libgdn2.so")
 GDN2_OK = 0
 STATUS_NAMES = {0: "GDN2_OK", -1: "GDN2_ERR_NULL", -2: "GDN2_ERR_SHAPE", -3: "GDN2_ERR_DTYPE",
                 -4: "GDN2_ERR_ALIGN", -5: "GDN2_ERR_WORKSPACE", -6: "GDN2_ERR_CUDA",
-                -7: "GDN2_ERR_TIMEOUT", -8: "GDN2_ERR_UNSUPPORTED"}
+                -7: "GDN2_ERR_TIMEOUT", -8: "GDN2_ERR_UNSUPPORTED", -9: "GDN2_ERR_TOO_LARGE"}
 GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
-           "gdn2_strerror", "gdn2_sync_status")
+           "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc")
+# Size of the library's static scratch array used by gdn2_chunk_bwd_noalloc
+# (GDN2_NOALLOC_MAX_SCRATCH_BYTES in include/gdn2.h).
+NOALLOC_MAX_SCRATCH_BYTES = 32 << 20
 
 _lib = None
 
@@ -49,6 +52,8 @@ def load(path: str | None = None):
     lib.gdn2_decode_step.restype = i
     lib.gdn2_chunk_bwd.argtypes = [i] * 6 + [vp] * 17 + [sz, vp]
     lib.gdn2_chunk_bwd.restype = i
+    lib.gdn2_chunk_bwd_noalloc.argtypes = [i] * 6 + [vp] * 16 + [vp]
+    lib.gdn2_chunk_bwd_noalloc.restype = i
     lib.gdn2_workspace_size.argtypes = [i] * 7
     lib.gdn2_workspace_size.restype = sz
     lib.gdn2_strerror.argtypes = [i]
@@ -165,6 +170,34 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace=No
                               _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]), _p(out["dS0"]),
                               _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdn2_chunk_bwd", st)
+    return out
+
+
+def gdn2_chunk_bwd_noalloc(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, out, stream=None):
+    """The backward with the library's static scratch array instead of a workspace.
+
+    ``out`` holds caller-allocated gradient tensors (keys as returned by
+    gdn2_chunk_bwd); nothing is allocated here or in the library.  Problems
+    whose workspace would exceed NOALLOC_MAX_SCRATCH_BYTES raise
+    GDN2_ERR_TOO_LARGE.  Calls that overlap on the GPU share the array and race.
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("d_o", d_o)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    _cuda_contig("dS_T", dS_T, torch.float32)
+    for n in ("dq", "dk", "dv", "db", "dw"):
+        _cuda_contig(n, out[n], q.dtype)
+    _cuda_contig("dlog_alpha", out["dlog_alpha"], torch.float32)
+    _cuda_contig("dS0", out["dS0"], torch.float32)
+    st = raw().gdn2_chunk_bwd_noalloc(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b),
+                                      _p(w), _p(S0), _p(d_o), _p(dS_T), _p(out["dq"]), _p(out["dk"]),
+                                      _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["db"]),
+                                      _p(out["dw"]), _p(out["dS0"]), _stream(stream))
+    _check("gdn2_chunk_bwd_noalloc", st)
     return out
 
 

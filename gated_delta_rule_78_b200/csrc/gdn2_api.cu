@@ -65,6 +65,7 @@ const char *gdn2_strerror(gdn2_status s)
     case GDN2_ERR_CUDA: return "a CUDA runtime call failed";
     case GDN2_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
     case GDN2_ERR_UNSUPPORTED: return "outside the supported shapes (Dk == Dv in {64, 128})";
+    case GDN2_ERR_TOO_LARGE: return "problem needs more scratch than the library's static array holds";
     }
     return "unknown status";
 }

@@ -63,7 +63,9 @@ typedef enum {
     GDN2_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than gdn2_workspace_size() */
     GDN2_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch error, no device, ...) */
     GDN2_ERR_TIMEOUT = -7,     /* a kernel's bounded wait gave up (reported by gdn2_sync_status) */
-    GDN2_ERR_UNSUPPORTED = -8  /* valid but outside the v1 shape contract */
+    GDN2_ERR_UNSUPPORTED = -8, /* valid but outside the v1 shape contract */
+    GDN2_ERR_TOO_LARGE = -9    /* needs more scratch than GDN2_NOALLOC_MAX_SCRATCH_BYTES
+                                  (gdn2_chunk_bwd_noalloc only) */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
@@ -111,6 +113,42 @@ GDN2_API gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, 
                            const void *d_o, const float *dS_T,
                            void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
                            float *dS0, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * gdn2_chunk_bwd without a workspace argument, for callers that cannot
+ * allocate device memory when they run the backward: code running inside a
+ * custom allocator or memory pool (allocating there would recurse), runtimes
+ * that fix their device-memory budget at start-up and forbid cudaMalloc
+ * afterwards, and plain C hosts that have no tensor library to hand them a
+ * buffer.  The operation has no counterpart in the paper: it is the same
+ * backward as gdn2_chunk_bwd, with the same arguments minus the workspace and
+ * the same gradients.
+ *   Scratch: a file-scope device array of GDN2_NOALLOC_MAX_SCRATCH_BYTES
+ *   bytes inside the library.  Every GPU that loads the library reserves it
+ *   and holds it until the process exits.  A problem is accepted when
+ *   gdn2_workspace_size(1, ...) <= GDN2_NOALLOC_MAX_SCRATCH_BYTES (for
+ *   example B*H = 2, T = 1024, d = 128 needs 20.5 MiB); larger ones return
+ *   GDN2_ERR_TOO_LARGE before anything is launched.
+ *   Allocation: none.  No cudaMalloc, cudaFree or allocating library call.
+ *   First call per device: looks up the array's device address with
+ *   cudaGetSymbolAddress for the device current at the call (which must be
+ *   the device that holds the arguments and the stream); later calls on that
+ *   device reuse it.  Make that first call before any stream capture.
+ *   Sharing: all calls on one device use the same array, and it keeps what
+ *   the last call left there.  Calls whose kernels overlap on the GPU (on
+ *   different streams, or from different threads) race on it and give wrong
+ *   gradients: order them on one stream or with events.  Nothing in the
+ *   array needs to start at zero: each call writes every scratch byte it
+ *   reads before reading it.
+ */
+#define GDN2_NOALLOC_MAX_SCRATCH_BYTES ((size_t)32 << 20)
+
+GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *stream);
 
 /* Workspace bytes for which = 0 (gdn2_chunk_fwd) or 1 (gdn2_chunk_bwd);
  * 0 for invalid or unsupported arguments. */
