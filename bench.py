@@ -276,15 +276,19 @@ def run_ours(args):
     def fwd():
         g.gdn2_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], o=o, S_T=ST)
 
+    parts = {"fwd", "bwd", "decode"} if not args.only else {args.only}
+    if args.fwd_only:
+        parts = {"fwd"}
     clocks.start()
-    ms_fwd = time_region(fwd, args.steps, args.warmup, stream) / args.steps
-    assert g.gdn2_sync_status() == 0, "a kernel reported a timeout"
     fb = fwd_bytes(B, T, H, D)
-    value = world * tokens / (ms_fwd * 1e-3)
+    ms_fwd = None
+    if "fwd" in parts:
+        ms_fwd = time_region(fwd, args.steps, args.warmup, stream) / args.steps
+        assert g.gdn2_sync_status() == 0, "a kernel reported a timeout"
 
     # ---- forward + backward on the same batch
     extras = {}
-    if not args.fwd_only:
+    if "bwd" in parts:
         nws = g.gdn2_workspace_size(1, x["q"].dtype, B, T, H, D, D)
         ws = torch.empty(nws, dtype=torch.uint8, device=dev)
         grads = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
@@ -299,14 +303,16 @@ def run_ours(args):
         ms_bwd = time_region(bwd, ksteps, max(3, args.warmup // 2), stream) / ksteps
         assert g.gdn2_sync_status() == 0
         bb = bwd_bytes(B, T, H, D)
-        ms_fb = ms_fwd + ms_bwd
-        extras["fwd_bwd"] = {
-            "value": round(world * tokens / (ms_fb * 1e-3), 1), "unit": "tokens/s",
-            "ms_per_step": round(ms_fb, 4), "bwd_ms": round(ms_bwd, 4), "steps": ksteps,
-            "roofline": roofline(fb + bb, ms_fb, pk), "bwd_roofline": roofline(bb, ms_bwd, pk),
-            "launches_per_step": 1 + 3}
+        extras["fwd_bwd"] = {"bwd_ms": round(ms_bwd, 4), "steps": ksteps,
+                             "bwd_roofline": roofline(bb, ms_bwd, pk), "launches_per_step": 1 + 3}
+        if ms_fwd is not None:
+            ms_fb = ms_fwd + ms_bwd
+            extras["fwd_bwd"].update({
+                "value": round(world * tokens / (ms_fb * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(ms_fb, 4), "roofline": roofline(fb + bb, ms_fb, pk)})
         del ws, grads
 
+    if "decode" in parts:
         # ---- decode: 256 sequences, 1024 steps, per-step inputs resident
         dw = DECODE_WORKLOAD
         N, Hd, Dd, nsteps = dw["N"], dw["H"], dw["Dk"], dw["steps"]
@@ -332,6 +338,16 @@ def run_ours(args):
             "launches_per_step": 1}
         del steps_in
     clocks.stop()
+    if ms_fwd is None:
+        # a single non-forward part was asked for (profiling runs): report it alone
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "only": args.only, "steps": args.steps,
+                              "warmup": args.warmup, "config": {"workload": args.workload},
+                              **extras}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    value = world * tokens / (ms_fwd * 1e-3)
 
     # ---- end to end through the binding with host buffers
     hx = {n: t.to("cpu").pin_memory() for n, t in x.items() if n != "do"}
@@ -389,6 +405,8 @@ def main():
     ap.add_argument("--workload", default="layer_4k", choices=sorted(WORKLOADS))
     ap.add_argument("--fwd-only", action="store_true", help="skip the fwd+bwd and decode figures")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--only", choices=["fwd", "bwd", "decode"], default=None,
+                    help="time one part only (for profiling runs)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
