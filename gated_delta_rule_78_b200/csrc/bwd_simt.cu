@@ -423,11 +423,20 @@ cudaError_t launch_t(const Problem &p, const void *d_o, const float *dS_T, const
 
 }  // namespace
 
-size_t bwd_workspace_bytes(int B, int T, int H, int D) { return ws_layout(B, T, H, D).total; }
+size_t bwd_workspace_bytes(gdn2_dtype dt, int B, int T, int H, int D)
+{
+    if (dt == GDN2_BF16 && D == 128) return bwd_tc_workspace_bytes(B, T, H);
+    return ws_layout(B, T, H, D).total;
+}
 
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
                        const BwdOut &out, void *ws, cudaStream_t s)
 {
+    if (dt == GDN2_BF16 && p.D == 128) {
+        int *status = status_word();
+        if (!status) return cudaErrorInvalidSymbol;
+        return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
+    }
     if (dt == GDN2_F32)
         return p.D == 64 ? launch_t<64, float>(p, d_o, dS_T, out, ws, s)
                          : launch_t<128, float>(p, d_o, dS_T, out, ws, s);

@@ -1,0 +1,749 @@
+// Gate-aware backward of the chunkwise GDN-2 recurrence on the tensor cores
+// (bf16 operands, fp32 accumulation), d_k = d_v = 128, chunk C = 64.
+//
+// Forward per chunk (S the fp32 state at the chunk start; the chunkwise WY form
+// with the decay folded into asymmetric factors, as in the aiexpert.news
+// article's implementation paragraph and the aixai.ru post's section "Как это
+// реализуется на практике"):
+//   G = cumsum(log alpha), Q~ = q e^G, E~ = (b.k) e^G, K~ = k e^-G, gamma = e^G_C,
+//   A = strictly_lower(E~ K~^T), P = lower_incl(Q~ K~^T), T = (I + A)^-1, X = w.v,
+//   Y = X - E~ S, U~ = T Y, O = Q~ S + P U~, S' = Diag(gamma) (S + K~^T U~).
+// Reverse mode (dS_n = dL/dS', dO = dL/dO), the gates staying inside the
+// gate-weighted products E~ and X as the aixai.ru post requires:
+//   dU~ = P^T dO + K~ Diag(gamma) dS_n        dY = T^T dU~ (= dX)
+//   dP  = lower_incl(dO U~^T)                 dA = -strictly_lower(dY U~^T)
+//   dQ~ = dO S^T + dP K~                      dE~ = -dY S^T + dA K~
+//   dK~ = dA^T E~ + dP^T Q~ + U~ (Diag(gamma) dS_n)^T
+//   gamma dgamma = rowsum(dS_n . S')          dS = gamma dS_n + Q~^T dO - E~^T dY
+// and through the factors: dq = dQ~ e^G, db = dE~ e^G k, dk = dE~ e^G b + dK~ e^-G,
+// dw = dY v, dv = dY w, dG = dQ~ Q~ + dE~ E~ - dK~ K~ (+ gamma dgamma on the last
+// row), dlog alpha = reverse cumulative sum of dG inside the chunk.
+//
+// The only serial dependence is the dS chain.  With W = T E~ and K^ = K~ Diag(gamma):
+//   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO),
+// so the work splits into four launches:
+//   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary;
+//   2. bwd_prep_kernel, one CTA per chunk: factors, [A; P], T, W, R (no state needed);
+//   3. bwd_chain_kernel, one CTA per (batch, head, half of d_v): the reverse dS chain,
+//      two warp MMAs per chunk with dS^T kept in registers; stores dS_n per chunk;
+//   4. bwd_grad_kernel, one CTA per chunk: recomputes U~ from the stored state and
+//      produces every gradient of the chunk.
+// All products are bf16 warp MMAs (m16n8k16) on ldmatrix-fed swizzled tiles.
+#include <cuda.h>
+
+#include "gdn2_internal.cuh"
+#include "tc_util.cuh"
+#include "warp_mma.cuh"
+
+namespace gdn2 {
+namespace {
+
+using namespace tc;
+using namespace wm;
+
+constexpr int D = 128;
+constexpr int C = 64;
+constexpr int LDA = 68;  // fp32 row stride of the A / T scratch of the solve
+
+// ------------------------------------------------------------------ workspace
+struct BwdTcLayout {
+    size_t states, W, Kh, gam, Rt, Tm, Pm, dSn, total;
+};
+
+// Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W and K^ bf16
+// [C][D], gamma fp32 [D], R^T fp32 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
+BwdTcLayout tc_layout(int B, int T, int H)
+{
+    const size_t bh = (size_t)B * H, nc = (size_t)(T + C - 1) / C;
+    BwdTcLayout l;
+    size_t off = 0;
+    l.states = off; off += bh * (nc + 1) * D * D * 2;
+    l.W = off;      off += bh * nc * C * D * 2;
+    l.Kh = off;     off += bh * nc * C * D * 2;
+    l.gam = off;    off += bh * nc * D * 4;
+    l.Rt = off;     off += bh * nc * D * D * 4;
+    l.Tm = off;     off += bh * nc * C * C * 2;
+    l.Pm = off;     off += bh * nc * C * C * 2;
+    l.dSn = off;    off += bh * nc * D * D * 2;
+    l.total = off;
+    return l;
+}
+
+struct BwdTcArgs {
+    int B, T, H, nchunks;
+    const __nv_bfloat16 *q, *k, *v, *b, *w, *dO;
+    const float *g;
+    const float *dS_T;  // may be null
+    __nv_bfloat16 *states, *W, *Kh, *Tm, *Pm, *dSn;
+    float *gam, *Rt;
+    __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
+    float *dg, *dS0;
+};
+
+// ------------------------------------------------------------------ small helpers
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Row t of chunk `ci` of head hh, batch bb in a [B, T, H, D] tensor.
+__device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bb, int hh, int ci, int t)
+{
+    return (((size_t)bb * a.T + (size_t)ci * C + t) * a.H + hh) * D;
+}
+
+// Copy the chunk's [C][D] bf16 token rows into a swizzled tile (256-byte rows), zero
+// rows past the sequence end.  All threads of the block take part.
+__device__ __forceinline__ void load_tok_tile(uint8_t *dst, const __nv_bfloat16 *src, const BwdTcArgs &a, int bb,
+                                              int hh, int ci, int L, int tid, int nthreads)
+{
+    for (int idx = tid; idx < C * 16; idx += nthreads) {
+        const int t = idx >> 4, ch = idx & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (t < L) v = *reinterpret_cast<const uint4 *>(src + tok_off(a, bb, hh, ci, t) + 8 * ch);
+        *reinterpret_cast<uint4 *>(dst + swz(t, 8 * ch, 256)) = v;
+    }
+}
+
+// Copy a dense row-major bf16 matrix (rows x cols, cols 64 or 128) into a swizzled tile.
+__device__ __forceinline__ void load_dense_tile(uint8_t *dst, const __nv_bfloat16 *src, int rows, int cols, int tid,
+                                                int nthreads)
+{
+    const int cpr = cols / 8, rb = cols * 2;
+    for (int idx = tid; idx < rows * cpr; idx += nthreads) {
+        const int r = idx / cpr, ch = idx % cpr;
+        *reinterpret_cast<uint4 *>(dst + swz(r, 8 * ch, rb)) =
+            *reinterpret_cast<const uint4 *>(src + (size_t)r * cols + 8 * ch);
+    }
+}
+
+// store a bf16 pair at (row, col) of a swizzled tile
+__device__ __forceinline__ void st_pair(uint8_t *tile, int rb, int row, int col, float lo, float hi)
+{
+    *reinterpret_cast<uint32_t *>(tile + swz(row, col, rb)) = pack_bf16x2(lo, hi);
+}
+__device__ __forceinline__ uint32_t ld_pair(const uint8_t *tile, int rb, int row, int col)
+{
+    return *reinterpret_cast<const uint32_t *>(tile + swz(row, col, rb));
+}
+
+// Per-thread cumulative log decay: thread (channel c, quarter q4) owns tokens
+// 16 q4 .. 16 q4 + 15; on return G[i] is the inclusive cumsum at token 16 q4 + i and
+// `total` the chunk total G_C.  sTot is a [4][D] fp32 scratch.  Needs 512 threads.
+__device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const BwdTcArgs &a, int bb, int hh,
+                                             int ci, int L, int c, int q4, float *sTot)
+{
+    float run = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = 16 * q4 + i;
+        const float gv = (t < L) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
+        run += gv;
+        G[i] = run;
+    }
+    sTot[q4 * D + c] = run;
+    __syncthreads();
+    float off = 0.f, tot = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const float v = sTot[u * D + c];
+        if (u < q4) off += v;
+        tot += v;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) G[i] += off;
+    total = tot;
+}
+
+// ================================================================== 2. prep
+// smem map (bytes): six [C][D] bf16 tiles, T and P bf16 [C][C], A and T fp32 [C][LDA],
+// the cumsum scratch.
+constexpr uint32_t P_Q = 0, P_E = 16384, P_K = 32768, P_DO = 49152, P_W = 65536, P_Z = 81920;
+constexpr uint32_t P_TB = 98304, P_PB = 106496, P_SA = 114688, P_ST = P_SA + C * LDA * 4;
+constexpr uint32_t P_TOT = P_ST + C * LDA * 4;
+constexpr uint32_t P_SMEM = P_TOT + 4 * D * 4;
+constexpr int kPrepThreads = 512;
+
+__global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ci = blockIdx.x % a.nchunks, bh = blockIdx.x / a.nchunks;
+    const int bb = bh / a.H, hh = bh % a.H;
+    const int L = min(C, a.T - ci * C);
+    const size_t cidx = (size_t)bh * a.nchunks + ci;
+    const uint32_t sb = smem_u32(sm);
+    float *sA = reinterpret_cast<float *>(sm + P_SA);
+    float *sT = reinterpret_cast<float *>(sm + P_ST);
+
+    // ---- raw q, k, b, dO tiles; T scratch zeroed (its upper blocks stay zero)
+    load_tok_tile(sm + P_Q, a.q, a, bb, hh, ci, L, tid, kPrepThreads);
+    load_tok_tile(sm + P_K, a.k, a, bb, hh, ci, L, tid, kPrepThreads);
+    load_tok_tile(sm + P_E, a.b, a, bb, hh, ci, L, tid, kPrepThreads);
+    load_tok_tile(sm + P_DO, a.dO, a, bb, hh, ci, L, tid, kPrepThreads);
+    for (int idx = tid; idx < C * LDA; idx += kPrepThreads) sT[idx] = 0.f;
+    // ---- decay folding (thread: channel c, 16 tokens); K^ and gamma go straight out
+    {
+        const int c = tid & (D - 1), q4 = tid >> 7;
+        float G[16], GC;
+        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
+        if (q4 == 0) a.gam[cidx * D + c] = __expf(GC);
+        __nv_bfloat16 *kh = a.Kh + cidx * C * D;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * q4 + i;
+            const uint32_t off = swz(t, c, 256);
+            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + P_Q + off);
+            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + P_K + off);
+            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + P_E + off);
+            const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk), bv = __bfloat162float(*pe);
+            const float eG = __expf(G[i]), emG = __expf(-G[i]);
+            *pq = __float2bfloat16_rn(qv * eG);
+            *pe = __float2bfloat16_rn(bv * kv * eG);
+            *pk = __float2bfloat16_rn(kv * emG);
+            kh[t * D + c] = __float2bfloat16_rn(kv * __expf(GC - G[i]));
+        }
+    }
+    __syncthreads();
+    // ---- [A; P] = [E~; Q~] K~^T (128 x 64, K = 128): warp = 16 stacked rows x 32 columns
+    {
+        const int mt = warp & 7, nh = warp >> 3;
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, false, false>(acc, sb + (mt < 4 ? P_E : P_Q), 256, 16 * (mt & 3), sb + P_K, 256, 32 * nh, D,
+                                      lane);
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = 16 * (mt & 3) + g + 8 * hr, col = 32 * nh + 8 * nt + 2 * t4;
+                const float v0 = acc[0][nt][2 * hr], v1 = acc[0][nt][2 * hr + 1];
+                if (mt < 4) {
+                    sA[row * LDA + col] = (col < row) ? v0 : 0.f;
+                    sA[row * LDA + col + 1] = (col + 1 < row) ? v1 : 0.f;
+                } else {
+                    st_pair(sm + P_PB, 128, row, col, (col <= row) ? v0 : 0.f, (col + 1 <= row) ? v1 : 0.f);
+                }
+            }
+    }
+    __syncthreads();
+    // ---- T = (I + A)^-1 on warps 0-3; meanwhile warps 8-15 form -Z = -(P^T dO)
+    if (warp < 4) {
+        solve_unit_lower64<LDA>(sA, sT, warp, lane, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
+    } else if (warp >= 8) {
+        const int mt = warp & 3, nh = (warp >> 2) & 1;
+        float acc[1][8][4];
+        zero_acc(acc);
+        warp_gemm<1, 8, true, true>(acc, sb + P_PB, 128, 16 * mt, sb + P_DO, 256, 64 * nh, C, lane);
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+                st_pair(sm + P_Z, 256, 16 * mt + g + 8 * hr, 64 * nh + 8 * nt + 2 * t4, -acc[0][nt][2 * hr],
+                        -acc[0][nt][2 * hr + 1]);
+    }
+    __syncthreads();
+    // ---- T -> bf16 tile and global; P -> global (one 16-byte chunk per thread)
+    {
+        const int i = tid >> 3, jc = tid & 7;
+        float tv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tv[e] = (8 * jc + e <= i) ? sT[i * LDA + 8 * jc + e] : 0.f;
+        const uint4 pk = make_uint4(pack_bf16x2(tv[0], tv[1]), pack_bf16x2(tv[2], tv[3]), pack_bf16x2(tv[4], tv[5]),
+                                    pack_bf16x2(tv[6], tv[7]));
+        *reinterpret_cast<uint4 *>(sm + P_TB + swz(i, 8 * jc, 128)) = pk;
+        *reinterpret_cast<uint4 *>(a.Tm + cidx * C * C + i * C + 8 * jc) = pk;
+        *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 8 * jc) =
+            *reinterpret_cast<const uint4 *>(sm + P_PB + swz(i, 8 * jc, 128));
+    }
+    __syncthreads();
+    // ---- W = T E~ (64 x 128, K = 64): warp = 16 rows x 32 columns
+    {
+        const int mt = warp & 3, nq = warp >> 2;
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, false, true>(acc, sb + P_TB, 128, 16 * mt, sb + P_E, 256, 32 * nq, C, lane);
+        const int g = lane >> 2, t4 = lane & 3;
+        __nv_bfloat16 *wg = a.W + cidx * C * D;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = 16 * mt + g + 8 * hr, col = 32 * nq + 8 * nt + 2 * t4;
+                const uint32_t pk = pack_bf16x2(acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
+                *reinterpret_cast<uint32_t *>(sm + P_W + swz(row, col, 256)) = pk;
+                *reinterpret_cast<uint32_t *>(wg + row * D + col) = pk;
+            }
+    }
+    __syncthreads();
+    // ---- R^T = dO^T Q~ + (-Z)^T W (128 x 128, K = 64 + 64): warp = 32 x 32
+    {
+        const int mb = warp & 3, nb = warp >> 2;
+        float acc[2][4][4];
+        zero_acc(acc);
+        warp_gemm<2, 4, true, true>(acc, sb + P_DO, 256, 32 * mb, sb + P_Q, 256, 32 * nb, C, lane);
+        warp_gemm<2, 4, true, true>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, C, lane);
+        const int g = lane >> 2, t4 = lane & 3;
+        float *rt = a.Rt + cidx * D * D;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int row = 32 * mb + 16 * mt + g + 8 * hr, col = 32 * nb + 8 * nt + 2 * t4;
+                    *reinterpret_cast<float2 *>(rt + row * D + col) =
+                        make_float2(acc[mt][nt][2 * hr], acc[mt][nt][2 * hr + 1]);
+                }
+    }
+}
+
+// ================================================================== 3. chain
+// One CTA per (batch, head, half of d_v); warp w owns 16 rows j of dS^T (d_v x d_k)
+// and keeps them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
+//   store dS_n^T (bf16) for the gradient kernel;
+//   Z^T = dS_n^T K^^T          (16 x 64 per warp, K = 128; A operand from registers)
+//   dS^T = dS_n^T Diag(gamma) + R^T - Z^T W   (K = 64; A operand = -Z^T from registers)
+// W, K^ and gamma of the next chunk are copied in (cp.async) during the current one.
+constexpr int kChainThreads = 128;
+constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_BUF = 33280;  // per buffer
+constexpr uint32_t CH_SMEM = 2 * CH_BUF;
+
+__global__ void __launch_bounds__(kChainThreads) bwd_chain_kernel(const BwdTcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, vh = blockIdx.y;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int j0 = 64 * vh + 16 * warp;  // this warp's first row of dS^T
+    const int nc = a.nchunks;
+    const uint32_t sb = smem_u32(sm);
+
+    auto prefetch = [&](int ci, int buf) {
+        const size_t cidx = (size_t)bh * nc + ci;
+        const uint32_t base = sb + buf * CH_BUF;
+        const __nv_bfloat16 *wsrc = a.W + cidx * C * D, *ksrc = a.Kh + cidx * C * D;
+        for (int idx = tid; idx < C * 16; idx += kChainThreads) {
+            const int t = idx >> 4, ch = idx & 15;
+            cp_async16(base + CH_W + swz(t, 8 * ch, 256), wsrc + t * D + 8 * ch);
+            cp_async16(base + CH_K + swz(t, 8 * ch, 256), ksrc + t * D + 8 * ch);
+        }
+        if (tid < 32) cp_async16(base + CH_G + 16 * tid, a.gam + cidx * D + 4 * tid);
+        cp_async_commit();
+    };
+
+    // dS^T rows j0 + g (+8), columns 8 nt + 2 t4 (+1)
+    float dS[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
+            dS[nt][e] = a.dS_T ? a.dS_T[((size_t)bh * D + c) * D + j] : 0.f;
+        }
+    if (nc > 0) prefetch(nc - 1, 0);
+    for (int ci = nc - 1; ci >= 0; --ci) {
+        const int buf = (nc - 1 - ci) & 1;
+        const size_t cidx = (size_t)bh * nc + ci;
+        if (ci > 0) {
+            prefetch(ci - 1, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const uint32_t wb = sb + buf * CH_BUF + CH_W, kb = sb + buf * CH_BUF + CH_K;
+        const float *gam = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_G);
+        // R^T of this chunk (issued early, used after the first product)
+        float2 R[16][2];
+        const float *rsrc = a.Rt + cidx * D * D;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+                R[nt][hr] = __ldcs(reinterpret_cast<const float2 *>(rsrc + (size_t)(j0 + g + 8 * hr) * D + 8 * nt + 2 * t4));
+        // dS_n^T for the gradient kernel, and as bf16 A fragments
+        uint32_t aS[8][4];
+        __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+            acc_to_a(aS[kc], dS[2 * kc], dS[2 * kc + 1], 1.f);
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const size_t row = (size_t)(j0 + g + 8 * hr) * D;
+                *reinterpret_cast<uint32_t *>(dsn + row + 16 * kc + 2 * t4) = aS[kc][hr];
+                *reinterpret_cast<uint32_t *>(dsn + row + 16 * kc + 8 + 2 * t4) = aS[kc][2 + hr];
+            }
+        }
+        // Z^T = dS_n^T K^^T: B operand K^ stored [t][c] = [n][k]
+        float Z[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) Z[nt][e] = 0.f;
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc)
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bfr[4];
+                load_b2<false>(bfr, kb, 256, 16 * kc, 16 * np, lane);
+                mma_bf16(Z[2 * np], aS[kc], bfr[0], bfr[1]);
+                mma_bf16(Z[2 * np + 1], aS[kc], bfr[2], bfr[3]);
+            }
+        // dS^T <- dS_n^T Diag(gamma) + R^T - Z^T W: B operand W stored [t][c] = [k][n]
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const float2 gm = *reinterpret_cast<const float2 *>(gam + 8 * nt + 2 * t4);
+            dS[nt][0] = dS[nt][0] * gm.x + R[nt][0].x;
+            dS[nt][1] = dS[nt][1] * gm.y + R[nt][0].y;
+            dS[nt][2] = dS[nt][2] * gm.x + R[nt][1].x;
+            dS[nt][3] = dS[nt][3] * gm.y + R[nt][1].y;
+        }
+#pragma unroll
+        for (int kt = 0; kt < 4; ++kt) {
+            uint32_t aZ[4];
+            acc_to_a(aZ, Z[2 * kt], Z[2 * kt + 1], -1.f);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bfr[4];
+                load_b2<true>(bfr, wb, 256, 16 * kt, 16 * np, lane);
+                mma_bf16(dS[2 * np], aZ, bfr[0], bfr[1]);
+                mma_bf16(dS[2 * np + 1], aZ, bfr[2], bfr[3]);
+            }
+        }
+        __syncthreads();  // every warp is done with this buffer before it is refilled
+    }
+    // dS0 = dS (stored [c][j])
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
+            a.dS0[((size_t)bh * D + c) * D + j] = dS[nt][e];
+        }
+}
+
+// ================================================================== 4. gradients
+// smem map (bytes): [C][D] bf16 tiles Q~, E~, K~; S^T and (Diag(gamma) dS_n)^T [D][D] bf16;
+// X -> U~, w -> Y -> dU~ -> [dP | dA], dO, -dY; T, P [C][C] bf16; scratch.  After the
+// products, dQ~, dE~, dK~ (fp32 [C][LDF]) reuse the first 104 KB.
+constexpr uint32_t G_Q = 0, G_E = 16384, G_K = 32768, G_S = 49152, G_DS = 81920, G_X = 114688, G_Y = 131072;
+constexpr uint32_t G_DO = 147456, G_DY = 163840, G_TB = 180224, G_PB = 188416, G_TOT = 196608;
+constexpr uint32_t G_GAM = G_TOT + 4 * D * 4, G_DGP = G_GAM + D * 4, G_DGF = G_DGP + 16 * D * 4;
+constexpr uint32_t G_SMEM = G_DGF + D * 4;
+constexpr int LDF = 136;  // fp32 row stride of the dQ~ / dE~ / dK~ tiles
+constexpr uint32_t G_FQ = 0, G_FE = C * LDF * 4, G_FK = 2 * C * LDF * 4;
+static_assert(G_FK + C * LDF * 4 <= G_X, "fp32 gradient tiles must fit in the dead operand tiles");
+constexpr int kGradThreads = 512;
+
+__global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int ci = blockIdx.x % a.nchunks, bh = blockIdx.x / a.nchunks;
+    const int bb = bh / a.H, hh = bh % a.H;
+    const int L = min(C, a.T - ci * C);
+    const size_t cidx = (size_t)bh * a.nchunks + ci;
+    const uint32_t sb = smem_u32(sm);
+    float *sTot = reinterpret_cast<float *>(sm + G_TOT);
+    float *sGam = reinterpret_cast<float *>(sm + G_GAM);
+    float *sDgp = reinterpret_cast<float *>(sm + G_DGP);
+    float *sDgf = reinterpret_cast<float *>(sm + G_DGF);
+    const int c = tid & (D - 1), q4 = tid >> 7;  // elementwise mapping: channel, quarter of the tokens
+
+    // ---- P0: operands
+    load_tok_tile(sm + G_Q, a.q, a, bb, hh, ci, L, tid, kGradThreads);
+    load_tok_tile(sm + G_K, a.k, a, bb, hh, ci, L, tid, kGradThreads);
+    load_tok_tile(sm + G_E, a.b, a, bb, hh, ci, L, tid, kGradThreads);
+    load_tok_tile(sm + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
+    load_tok_tile(sm + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
+    load_tok_tile(sm + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
+    const __nv_bfloat16 *st_c = a.states + ((size_t)bh * (a.nchunks + 1) + ci) * D * D;
+    load_dense_tile(sm + G_S, st_c, D, D, tid, kGradThreads);
+    load_dense_tile(sm + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
+    load_dense_tile(sm + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
+    {
+        float G[16], GC;
+        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // its barrier also covers the tile loads
+        if (q4 == 0) sGam[c] = __expf(GC);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * q4 + i;
+            const uint32_t off = swz(t, c, 256);
+            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + G_Q + off);
+            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + G_K + off);
+            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + G_E + off);
+            __nv_bfloat16 *px = reinterpret_cast<__nv_bfloat16 *>(sm + G_X + off);
+            const __nv_bfloat16 *pw = reinterpret_cast<const __nv_bfloat16 *>(sm + G_Y + off);
+            const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk), bv = __bfloat162float(*pe);
+            const float eG = __expf(G[i]), emG = __expf(-G[i]);
+            *pq = __float2bfloat16_rn(qv * eG);
+            *pe = __float2bfloat16_rn(bv * kv * eG);
+            *pk = __float2bfloat16_rn(kv * emG);
+            *px = __float2bfloat16_rn(__bfloat162float(*px) * __bfloat162float(*pw));  // X = w.v (column c = j)
+        }
+    }
+    __syncthreads();
+    {  // (Diag(gamma) dS_n)^T tile, and gamma dgamma = rowsum(dS_n . S') partials
+        const __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
+        const __nv_bfloat16 *st_n = st_c + (size_t)D * D;
+        const int ch = tid & 15;
+        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float gm[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[e] = sGam[8 * ch + e];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = (tid >> 4) + 32 * u;
+            const uint4 dv4 = *reinterpret_cast<const uint4 *>(dsn + (size_t)j * D + 8 * ch);
+            const uint4 sv4 = *reinterpret_cast<const uint4 *>(st_n + (size_t)j * D + 8 * ch);
+            const uint32_t dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w}, sw[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float d0 = bf_lo(dw[e]), d1 = bf_hi(dw[e]);
+                part[2 * e] += d0 * bf_lo(sw[e]);
+                part[2 * e + 1] += d1 * bf_hi(sw[e]);
+                o[e] = pack_bf16x2(d0 * gm[2 * e], d1 * gm[2 * e + 1]);
+            }
+            *reinterpret_cast<uint4 *>(sm + G_DS + swz(j, 8 * ch, 256)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[e] += __shfl_xor_sync(0xffffffffu, part[e], 16);
+        if (lane < 16) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sDgp[warp * D + 8 * ch + e] = part[e];
+        }
+    }
+    __syncthreads();
+    if (tid < D) {
+        float s = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
+        sDgf[tid] = s;
+    }
+    // warp tiling of the [C][D] products: 16 rows x 32 columns
+    const int mt = warp & 3, nq = warp >> 2;
+    const int r0 = 16 * mt + g, c0 = 32 * nq + 2 * t4;  // + 8 hr rows, + 8 nt columns
+    // ---- P1: Y = X - E~ S  -> bf16 over the raw w tile
+    {
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, false, false>(acc, sb + G_E, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
+                const uint32_t x = ld_pair(sm + G_X, 256, row, col);
+                st_pair(sm + G_Y, 256, row, col, bf_lo(x) - acc[0][nt][2 * hr], bf_hi(x) - acc[0][nt][2 * hr + 1]);
+            }
+    }
+    __syncthreads();
+    // ---- P2: U~ = T Y  -> bf16 over X
+    {
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, false, true>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, C, lane);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+                st_pair(sm + G_X, 256, r0 + 8 * hr, c0 + 8 * nt, acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
+    }
+    __syncthreads();
+    // ---- P3: dU~ = P^T dO + K~ (Diag(gamma) dS_n)  -> bf16 over Y
+    {
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, true, true>(acc, sb + G_PB, 128, 16 * mt, sb + G_DO, 256, 32 * nq, C, lane);
+        warp_gemm<1, 4, false, false>(acc, sb + G_K, 256, 16 * mt, sb + G_DS, 256, 32 * nq, D, lane);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+                st_pair(sm + G_Y, 256, r0 + 8 * hr, c0 + 8 * nt, acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
+    }
+    __syncthreads();
+    // ---- P4: dY = T^T dU~ -> dv = dY w, dw = dY v (global), -dY (bf16)
+    {
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, true, true>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, C, lane);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
+                const float d0 = acc[0][nt][2 * hr], d1 = acc[0][nt][2 * hr + 1];
+                st_pair(sm + G_DY, 256, row, col, -d0, -d1);
+                if (row < L) {
+                    const size_t off = tok_off(a, bb, hh, ci, row) + col;
+                    const uint32_t vv = *reinterpret_cast<const uint32_t *>(a.v + off);
+                    const uint32_t ww = *reinterpret_cast<const uint32_t *>(a.w + off);
+                    *reinterpret_cast<uint32_t *>(a.dv + off) = pack_bf16x2(d0 * bf_lo(ww), d1 * bf_hi(ww));
+                    *reinterpret_cast<uint32_t *>(a.dw + off) = pack_bf16x2(d0 * bf_lo(vv), d1 * bf_hi(vv));
+                }
+            }
+    }
+    __syncthreads();
+    // ---- P5: [dP; dA] = [dO; -dY] U~^T (128 x 64, K = 128) -> bf16 [C][C] tiles over dU~
+    {
+        const int ms = warp & 7, nh = warp >> 3;
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, false, false>(acc, sb + (ms < 4 ? G_DO : G_DY), 256, 16 * (ms & 3), sb + G_X, 256, 32 * nh, D,
+                                      lane);
+        uint8_t *dst = sm + G_Y + (ms < 4 ? 0 : 8192);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = 16 * (ms & 3) + g + 8 * hr, col = 32 * nh + 8 * nt + 2 * t4;
+                const float v0 = acc[0][nt][2 * hr], v1 = acc[0][nt][2 * hr + 1];
+                if (ms < 4)
+                    st_pair(dst, 128, row, col, (col <= row) ? v0 : 0.f, (col + 1 <= row) ? v1 : 0.f);
+                else
+                    st_pair(dst, 128, row, col, (col < row) ? v0 : 0.f, (col + 1 < row) ? v1 : 0.f);
+            }
+    }
+    __syncthreads();
+    const uint32_t dPb = sb + G_Y, dAb = sb + G_Y + 8192;
+    // ---- P6-P8: dQ~, dE~, dK~ in registers
+    float aq[1][4][4], ae[1][4][4], ak[1][4][4];
+    zero_acc(aq);
+    zero_acc(ae);
+    zero_acc(ak);
+    warp_gemm<1, 4, false, true>(aq, sb + G_DO, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
+    warp_gemm<1, 4, false, true>(aq, dPb, 128, 16 * mt, sb + G_K, 256, 32 * nq, C, lane);
+    warp_gemm<1, 4, false, true>(ae, sb + G_DY, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
+    warp_gemm<1, 4, false, true>(ae, dAb, 128, 16 * mt, sb + G_K, 256, 32 * nq, C, lane);
+    warp_gemm<1, 4, true, true>(ak, dAb, 128, 16 * mt, sb + G_E, 256, 32 * nq, C, lane);
+    warp_gemm<1, 4, true, true>(ak, dPb, 128, 16 * mt, sb + G_Q, 256, 32 * nq, C, lane);
+    warp_gemm<1, 4, false, true>(ak, sb + G_X, 256, 16 * mt, sb + G_DS, 256, 32 * nq, D, lane);
+    __syncthreads();  // all operand tiles are dead from here on
+    {
+        float *fq = reinterpret_cast<float *>(sm + G_FQ), *fe = reinterpret_cast<float *>(sm + G_FE);
+        float *fk = reinterpret_cast<float *>(sm + G_FK);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int o = (r0 + 8 * hr) * LDF + c0 + 8 * nt;
+                *reinterpret_cast<float2 *>(fq + o) = make_float2(aq[0][nt][2 * hr], aq[0][nt][2 * hr + 1]);
+                *reinterpret_cast<float2 *>(fe + o) = make_float2(ae[0][nt][2 * hr], ae[0][nt][2 * hr + 1]);
+                *reinterpret_cast<float2 *>(fk + o) = make_float2(ak[0][nt][2 * hr], ak[0][nt][2 * hr + 1]);
+            }
+    }
+    __syncthreads();
+    // ---- P10: through the factors (thread: channel c, tokens 16 q4 .. +15), fp32
+    {
+        const float *fq = reinterpret_cast<const float *>(sm + G_FQ), *fe = reinterpret_cast<const float *>(sm + G_FE);
+        const float *fk = reinterpret_cast<const float *>(sm + G_FK);
+        float G[16], GC;
+        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, sTot + 0);  // sTot is free again (P0 finished)
+        float dG[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * q4 + i;
+            const float dQ = fq[t * LDF + c], dE = fe[t * LDF + c], dK = fk[t * LDF + c];
+            float qv = 0.f, kv = 0.f, bv = 0.f;
+            size_t off = 0;
+            if (t < L) {
+                off = tok_off(a, bb, hh, ci, t) + c;
+                qv = __bfloat162float(a.q[off]);
+                kv = __bfloat162float(a.k[off]);
+                bv = __bfloat162float(a.b[off]);
+            }
+            const float eG = __expf(G[i]), emG = __expf(-G[i]);
+            const float de = dE * eG;
+            dG[i] = dQ * qv * eG + de * bv * kv - dK * kv * emG;
+            if (t < L) {
+                a.dq[off] = __float2bfloat16_rn(dQ * eG);
+                a.db[off] = __float2bfloat16_rn(de * kv);
+                a.dk[off] = __float2bfloat16_rn(de * bv + dK * emG);
+            }
+        }
+        if (q4 == 3) dG[15] += sDgf[c];  // gamma dgamma enters at the last row of the chunk
+        // reverse cumulative sum inside the chunk
+        float run = 0.f;
+#pragma unroll
+        for (int i = 15; i >= 0; --i) {
+            run += dG[i];
+            dG[i] = run;
+        }
+        __syncthreads();  // everyone has read sTot (forward cumsum) before it is reused
+        sTot[q4 * D + c] = run;
+        __syncthreads();
+        float after = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u > q4) after += sTot[u * D + c];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * q4 + i;
+            if (t < L) a.dg[tok_off(a, bb, hh, ci, t) + c] = dG[i] + after;
+        }
+    }
+}
+
+}  // namespace
+
+size_t bwd_tc_workspace_bytes(int B, int T, int H) { return tc_layout(B, T, H).total; }
+
+cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
+                          int *status, cudaStream_t s)
+{
+    if (p.D != D) return cudaErrorNotSupported;
+    const BwdTcLayout l = tc_layout(p.B, p.T, p.H);
+    char *base = static_cast<char *>(ws);
+    BwdTcArgs a;
+    a.B = p.B; a.T = p.T; a.H = p.H; a.nchunks = (p.T + C - 1) / C;
+    a.q = static_cast<const __nv_bfloat16 *>(p.q);
+    a.k = static_cast<const __nv_bfloat16 *>(p.k);
+    a.v = static_cast<const __nv_bfloat16 *>(p.v);
+    a.b = static_cast<const __nv_bfloat16 *>(p.b);
+    a.w = static_cast<const __nv_bfloat16 *>(p.w);
+    a.dO = static_cast<const __nv_bfloat16 *>(d_o);
+    a.g = p.g;
+    a.dS_T = dS_T;
+    a.states = reinterpret_cast<__nv_bfloat16 *>(base + l.states);
+    a.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
+    a.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
+    a.gam = reinterpret_cast<float *>(base + l.gam);
+    a.Rt = reinterpret_cast<float *>(base + l.Rt);
+    a.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
+    a.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
+    a.dSn = reinterpret_cast<__nv_bfloat16 *>(base + l.dSn);
+    a.dq = static_cast<__nv_bfloat16 *>(out.dq);
+    a.dk = static_cast<__nv_bfloat16 *>(out.dk);
+    a.dv = static_cast<__nv_bfloat16 *>(out.dv);
+    a.db = static_cast<__nv_bfloat16 *>(out.db);
+    a.dw = static_cast<__nv_bfloat16 *>(out.dw);
+    a.dg = out.dg;
+    a.dS0 = out.dS0;
+
+    cudaError_t e = launch_fwd_tc(p, nullptr, nullptr, a.states, status, s);
+    if (e != cudaSuccess) return e;
+    const unsigned nblk = (unsigned)((size_t)p.B * p.H * a.nchunks);
+    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_kernel), (int)P_SMEM)) != cudaSuccess) return e;
+    bwd_prep_kernel<<<nblk, kPrepThreads, P_SMEM, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
+    bwd_chain_kernel<<<dim3(p.B * p.H, 2), kChainThreads, CH_SMEM, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)G_SMEM)) != cudaSuccess) return e;
+    bwd_grad_kernel<<<nblk, kGradThreads, G_SMEM, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn2

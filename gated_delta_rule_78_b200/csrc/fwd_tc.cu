@@ -33,9 +33,11 @@
 // readback and holds its 64 columns of S^T in fp32 registers.  The output tile
 // is staged in shared memory and written by a TMA store.
 #include <cuda.h>
+#include <string.h>
 
 #include "gdn2_internal.cuh"
 #include "tc_util.cuh"
+#include "warp_mma.cuh"
 
 namespace gdn2 {
 namespace {
@@ -87,8 +89,10 @@ struct TcParams {
     int B, T, H;
     const float *S0;
     const float *g;   // log alpha [B,T,H,D] fp32
-    __nv_bfloat16 *o;
+    __nv_bfloat16 *o;        // may be null (states-only run)
     float *S_T;
+    __nv_bfloat16 *states;   // may be null; else [B*H][nchunks + 1][D (d_v)][D (d_k)]: S^T at every
+                             // chunk boundary, the final state last
     int *status;
 };
 
@@ -104,93 +108,6 @@ __device__ __forceinline__ void named_sync(int id, int count)
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-
-// One warp inverts the 16x16 unit lower-triangular diagonal block (I + A_pp) that
-// starts at row/column r0: closed-form 4x4 inverses, then two doubling steps
-// T21 = -T22 (A21 T11) inside the warp.  Only lower blocks of sT are written.
-__device__ __forceinline__ void invert_diag16(const float *sA, float *sT, int r0, int lane)
-{
-    if (lane < 4) {
-        const int b = r0 + 4 * lane;
-        const float *a = sA + b * LDA + b;
-        const float a10 = a[1 * LDA + 0], a20 = a[2 * LDA + 0], a21 = a[2 * LDA + 1];
-        const float a30 = a[3 * LDA + 0], a31 = a[3 * LDA + 1], a32 = a[3 * LDA + 2];
-        const float t10 = -a10, t21 = -a21, t32 = -a32;
-        const float t20 = -(a20 + a21 * t10);
-        const float t31 = -(a31 + a32 * t21);
-        const float t30 = -(a30 + a31 * t10 + a32 * t20);
-        float *t = sT + b * LDA + b;
-        t[0 * LDA + 0] = 1.f;
-        t[1 * LDA + 0] = t10; t[1 * LDA + 1] = 1.f;
-        t[2 * LDA + 0] = t20; t[2 * LDA + 1] = t21; t[2 * LDA + 2] = 1.f;
-        t[3 * LDA + 0] = t30; t[3 * LDA + 1] = t31; t[3 * LDA + 2] = t32; t[3 * LDA + 3] = 1.f;
-    }
-    __syncwarp();
-    {  // 4 -> 8: two 4x4 blocks, one output per lane
-        const int q = lane >> 4, r = (lane >> 2) & 3, c = lane & 3;
-        const int R = r0 + 8 * q + 4, Cc = r0 + 8 * q;
-        float y = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) y += sA[(R + r) * LDA + Cc + u] * sT[(Cc + u) * LDA + Cc + c];
-        __syncwarp();
-        sT[(R + r) * LDA + Cc + c] = y;
-        __syncwarp();
-        float x = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) x += sT[(R + r) * LDA + R + u] * sT[(R + u) * LDA + Cc + c];
-        __syncwarp();
-        sT[(R + r) * LDA + Cc + c] = -x;
-        __syncwarp();
-    }
-    {  // 8 -> 16: one 8x8 block, two outputs per lane
-        const int r = lane >> 2, c = 2 * (lane & 3);
-        const int R = r0 + 8, Cc = r0;
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const float a = sA[(R + r) * LDA + Cc + u];
-            y0 += a * sT[(Cc + u) * LDA + Cc + c];
-            y1 += a * sT[(Cc + u) * LDA + Cc + c + 1];
-        }
-        __syncwarp();
-        sT[(R + r) * LDA + Cc + c] = y0;
-        sT[(R + r) * LDA + Cc + c + 1] = y1;
-        __syncwarp();
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const float t = sT[(R + r) * LDA + R + u];
-            x0 += t * sT[(R + u) * LDA + Cc + c];
-            x1 += t * sT[(R + u) * LDA + Cc + c + 1];
-        }
-        __syncwarp();
-        sT[(R + r) * LDA + Cc + c] = -x0;
-        sT[(R + r) * LDA + Cc + c + 1] = -x1;
-    }
-}
-
-// acc (16x8 tile) += X[0:16, 0:K] * Y[0:K, 0:8] for fp32 shared-memory operands with
-// row stride LDA (X and Y point at the tile origins), rounded to TF32 on load.
-template <int K>
-__device__ __forceinline__ void tile_mma_tf32(const float *X, const float *Y, float (&acc)[4], int lane)
-{
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a[4] = {to_tf32(X[g * LDA + k0 + t]), to_tf32(X[(g + 8) * LDA + k0 + t]),
-                               to_tf32(X[g * LDA + k0 + t + 4]), to_tf32(X[(g + 8) * LDA + k0 + t + 4])};
-        const uint32_t b[2] = {to_tf32(Y[(k0 + t) * LDA + g]), to_tf32(Y[(k0 + t + 4) * LDA + g])};
-        mma_tf32_16x8x8(acc, a, b);
-    }
-}
-__device__ __forceinline__ void tile_store(float *Z, const float (&acc)[4], float sign, int lane)
-{
-    const int g = lane >> 2, t = lane & 3;
-    Z[g * LDA + 2 * t] = sign * acc[0];
-    Z[g * LDA + 2 * t + 1] = sign * acc[1];
-    Z[(g + 8) * LDA + 2 * t] = sign * acc[2];
-    Z[(g + 8) * LDA + 2 * t + 1] = sign * acc[3];
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
@@ -228,7 +145,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         }
         fence_mbar_init();
         prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.v);
-        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w); prefetch_tmap(&maps.g); prefetch_tmap(&maps.o);
+        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w); prefetch_tmap(&maps.g);
+        if (p.o) prefetch_tmap(&maps.o);
     }
     if (warp == 0) {
         tmem_alloc(&s_tmem, TM_COLS);
@@ -291,10 +209,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         fence_proxy_async_smem();
         named_sync(1, kGroup);
         if (tid == 0 && nchunks > 1) issue(1);  // w(1) may only land after w(0) was folded
+        // bf16 copy of this thread's 64 entries of S^T at chunk boundary `idx`
+        auto store_state = [&](const float *Sv, int idx) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.states + (((size_t)bh * (nchunks + 1) + idx) * D + jrow) * D +
+                                                   64 * half);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                dst[u] = make_uint4(pack_bf16x2(Sv[8 * u], Sv[8 * u + 1]), pack_bf16x2(Sv[8 * u + 2], Sv[8 * u + 3]),
+                                    pack_bf16x2(Sv[8 * u + 4], Sv[8 * u + 5]), pack_bf16x2(Sv[8 * u + 6], Sv[8 * u + 7]));
+        };
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
             Sf[i] = p.S0 ? p.S0[((size_t)bh * D + 64 * half + i) * D + jrow] : 0.f;
+        if (p.states) store_state(Sf, 0);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             uint32_t pk[16];
@@ -399,8 +327,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * h2 + 2 * e], Sf[32 * h2 + 2 * e + 1]);
                     tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
                 }
+                if (p.states) store_state(Sf, ci + 1);
             }
-            {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
+            if (p.o) {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
                 uint32_t r[32];
                 tmem_ld32(tmem + TM_O + 32 * half + lane_off, r);
                 tmem_wait_ld();
@@ -412,13 +341,13 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(1, kGroup);
-            if (L == C) {
+            if (p.o && L == C) {
                 if (tid == 0) {
                     tma_store_3d(&maps.o, sm + ott, 0, hh, bb * T + ci * C);
                     bulk_commit();
                     bulk_wait_read0();
                 }
-            } else {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
+            } else if (p.o) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
                 const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
                 __nv_bfloat16 *dst = p.o + ((size_t)bb * T + (size_t)ci * C) * p.H * D + (size_t)hh * D;
                 for (int idx = tid; idx < L * D; idx += kGroup) dst[(size_t)(idx / D) * p.H * D + idx % D] = so[idx];
@@ -550,40 +479,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             // ---- T = (I + A)^-1 on warps 8-11: diagonal 16x16 blocks, then the doubling levels on
             //      warp-level TF32 MMAs; meanwhile warp 12 issues the next chunk's loads
             if (ew < 4) {
-                invert_diag16(sA, sT, 16 * ew, lane);
-                named_sync(3, 128);
-                if (ew < 2) {  // 32x32 level: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
-                    const int R = 32 * ew + 16, Cc = 32 * ew;
-                    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc, y0, lane);
-                    tile_mma_tf32<16>(sA + R * LDA + Cc, sT + Cc * LDA + Cc + 8, y1, lane);
-                    tile_store(sT + R * LDA + Cc, y0, 1.f, lane);
-                    tile_store(sT + R * LDA + Cc + 8, y1, 1.f, lane);
-                    __syncwarp();
-                    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc, x0, lane);
-                    tile_mma_tf32<16>(sT + R * LDA + R, sT + R * LDA + Cc + 8, x1, lane);
-                    __syncwarp();
-                    tile_store(sT + R * LDA + Cc, x0, -1.f, lane);
-                    tile_store(sT + R * LDA + Cc + 8, x1, -1.f, lane);
-                }
-                named_sync(3, 128);
-                {  // 64x64 level: T_BA = -T_BB (A_BA T_AA); warp: one 16-row tile, two 8-col tiles
-                    const int mt = ew & 1, n0 = 16 * (ew >> 1);
-                    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0, y0, lane);
-                    tile_mma_tf32<32>(sA + (32 + 16 * mt) * LDA, sT + n0 + 8, y1, lane);
-                    tile_store(sT + (32 + 16 * mt) * LDA + n0, y0, 1.f, lane);
-                    tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, y1, 1.f, lane);
-                    named_sync(3, 128);
-                    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0, x0, lane);
-                    tile_mma_tf32<32>(sT + (32 + 16 * mt) * LDA + 32, sT + 32 * LDA + n0 + 8, x1, lane);
-                    named_sync(3, 128);
-                    tile_store(sT + (32 + 16 * mt) * LDA + n0, x0, -1.f, lane);
-                    tile_store(sT + (32 + 16 * mt) * LDA + n0 + 8, x1, -1.f, lane);
-                }
-                named_sync(3, 128);
+                wm::solve_unit_lower64<LDA>(sA, sT, ew, lane, [] { named_sync(3, 128); });
                 {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
                     const int i = etid >> 1, hf = etid & 1;
 #pragma unroll
@@ -656,22 +552,20 @@ bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, b
 
 }  // namespace
 
-cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, int *status, cudaStream_t s)
+cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
+                          cudaStream_t s)
 {
     if (pr.D != D) return cudaErrorNotSupported;
     TcMaps maps;
+    memset(&maps, 0, sizeof(maps));
     if (!make_map(&maps.q, pr.q, false, pr.B, pr.T, pr.H) || !make_map(&maps.k, pr.k, false, pr.B, pr.T, pr.H) ||
         !make_map(&maps.v, pr.v, false, pr.B, pr.T, pr.H) || !make_map(&maps.b, pr.b, false, pr.B, pr.T, pr.H) ||
         !make_map(&maps.w, pr.w, false, pr.B, pr.T, pr.H) || !make_map(&maps.g, pr.g, true, pr.B, pr.T, pr.H) ||
-        !make_map(&maps.o, o, false, pr.B, pr.T, pr.H, true))
+        (o && !make_map(&maps.o, o, false, pr.B, pr.T, pr.H, true)))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, status};
+    cudaError_t e = set_smem_attr(reinterpret_cast<const void *>(fwd_tc_kernel), (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status};
     fwd_tc_kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
     return cudaGetLastError();
 }

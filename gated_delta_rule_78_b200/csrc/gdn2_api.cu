@@ -2,11 +2,48 @@
 // Declarations and the contract of every entry point are in include/gdn2.h.
 #include <stdint.h>
 
+#include <mutex>
+
 #include "gdn2_internal.cuh"
+
+namespace gdn2 {
+
+cudaError_t set_smem_attr(const void *kernel, int bytes)
+{
+    // (kernel, device) pairs already raised; a small table is enough for the handful of kernels here
+    struct Entry { const void *fn; uint64_t devices; };
+    static Entry table[32];
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = -1;
+    for (int i = 0; i < 32; ++i) {
+        if (table[i].fn == kernel) { slot = i; break; }
+        if (!table[i].fn && slot < 0) slot = i;
+    }
+    if (slot >= 0 && table[slot].fn == kernel && (table[slot].devices >> dev & 1u)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && slot >= 0) {
+        table[slot].fn = kernel;
+        table[slot].devices |= 1ull << dev;
+    }
+    return e;
+}
+
+}  // namespace gdn2
 
 // Per-device kernel status word (0 = fine).  Kernels that give up a bounded
 // wait store a non-zero code here; gdn2_sync_status() reads and clears it.
 __device__ int g_gdn2_status = 0;
+
+int *gdn2::status_word()
+{
+    int *p = nullptr;
+    return cudaGetSymbolAddress((void **)&p, g_gdn2_status) == cudaSuccess ? p : nullptr;
+}
 
 namespace {
 
@@ -74,7 +111,7 @@ size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk
 {
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK) return 0;
     if (which == 0) return 0;
-    if (which == 1) return T == 0 ? 0 : gdn2::bwd_workspace_bytes(B, T, H, Dk);
+    if (which == 1) return T == 0 ? 0 : gdn2::bwd_workspace_bytes(dt, B, T, H, Dk);
     return 0;
 }
 
@@ -101,7 +138,7 @@ gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
     if (dt == GDN2_BF16) {
         int *status = nullptr;
         if (cudaGetSymbolAddress((void **)&status, g_gdn2_status) != cudaSuccess) return GDN2_ERR_CUDA;
-        cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, status, s);
+        cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();  // clear the sticky "not supported" code; fall through to FMA path
     }
@@ -140,7 +177,7 @@ gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
         if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
         return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
     }
-    const size_t need = gdn2::bwd_workspace_bytes(B, T, H, Dk);
+    const size_t need = gdn2::bwd_workspace_bytes(dt, B, T, H, Dk);
     if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);

@@ -37,9 +37,16 @@ struct Problem {
 cudaError_t launch_fwd_simt(gdn2_dtype dt, const Problem &p, void *o, float *S_T, float *states,
                             cudaStream_t s);
 
+// Raise a kernel's dynamic shared-memory limit on the current device (once per
+// kernel and device; thread-safe).
+cudaError_t set_smem_attr(const void *kernel, int bytes);
+
 // forward on the tensor cores (bf16 operands); returns cudaErrorNotSupported when
-// the shape is outside what the kernel handles.
-cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, int *status, cudaStream_t s);
+// the shape is outside what the kernel handles.  `o` may be null (no output);
+// `states`, when non-null, receives S^T in bf16 at every chunk boundary:
+// [B*H][nchunks + 1][D][D], entry c the state before chunk c, the last entry S_T.
+cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *states, int *status,
+                          cudaStream_t s);
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
@@ -49,8 +56,19 @@ struct BwdOut {
     void *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
 };
-size_t bwd_workspace_bytes(int B, int T, int H, int D);
+// Backward workspace bytes (depends on the path: bf16 with D = 128 runs on the
+// tensor cores, everything else on the fp32 FMA kernels).
+size_t bwd_workspace_bytes(gdn2_dtype dt, int B, int T, int H, int D);
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
                        const BwdOut &out, void *ws, cudaStream_t s);
+
+// tensor-core backward (bf16, D = 128): the forward in states mode, then the prep,
+// chain and gradient kernels
+size_t bwd_tc_workspace_bytes(int B, int T, int H);
+cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
+                          int *status, cudaStream_t s);
+
+// device address of the library's kernel status word on the current device
+int *status_word();
 
 }  // namespace gdn2

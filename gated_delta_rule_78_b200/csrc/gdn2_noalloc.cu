@@ -83,7 +83,7 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(
         if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
         return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
     }
-    if (gdn2::bwd_workspace_bytes(B, T, H, Dk) > kScratchBytes) return GDN2_ERR_TOO_LARGE;
+    if (gdn2::bwd_workspace_bytes(dt, B, T, H, Dk) > kScratchBytes) return GDN2_ERR_TOO_LARGE;
 
     void *scratch = nullptr;
     const gdn2_status st = scratch_address(&scratch);

@@ -102,8 +102,10 @@ GDN2_API gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int D
  *   Outputs: dq, dk, db [B,T,H,Dk] and dv, dw [B,T,H,Dv] of type dt;
  *            dlog_alpha [B,T,H,Dk] fp32; dS0 [B,H,Dk,Dv] fp32.
  *   S0 may be NULL (zeros).  All outputs must be distinct from the inputs.
- *   workspace: at least gdn2_workspace_size(1, ...) bytes (chunk-start
- *   states and per-tile partial gradients, fp32).
+ *   workspace: at least gdn2_workspace_size(1, ...) bytes.  bf16 with
+ *   d = 128: chunk-boundary states and per-chunk factors (bf16), the chain's
+ *   per-chunk inputs (fp32) and the state gradients at chunk ends (bf16);
+ *   otherwise fp32 chunk-start states and per-tile partial gradients.
  * The gates enter inside the chunk products (gate-weighted keys and values),
  * as the aixai.ru post's implementation section requires.
  */
@@ -127,8 +129,9 @@ GDN2_API gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, 
  *   bytes inside the library.  Every GPU that loads the library reserves it
  *   and holds it until the process exits.  A problem is accepted when
  *   gdn2_workspace_size(1, ...) <= GDN2_NOALLOC_MAX_SCRATCH_BYTES (for
- *   example B*H = 2, T = 1024, d = 128 needs 20.5 MiB); larger ones return
- *   GDN2_ERR_TOO_LARGE before anything is launched.
+ *   example B*H = 2, T = 1024, d = 128 needs 20.5 MiB with fp32 inputs and
+ *   5.5 MiB with bf16 inputs); larger ones return GDN2_ERR_TOO_LARGE before
+ *   anything is launched.
  *   Allocation: none.  No cudaMalloc, cudaFree or allocating library call.
  *   First call per device: looks up the array's device address with
  *   cudaGetSymbolAddress for the device current at the call (which must be

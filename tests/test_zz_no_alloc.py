@@ -28,9 +28,12 @@ def test_noalloc_rejects_before_any_cuda_call():
     """Size and argument errors come back before the library touches a device."""
     lib = g.load()
     assert g.NOALLOC_MAX_SCRATCH_BYTES == 32 << 20
-    # B*H = 1, T = 4096, d = 128 needs 37.25 MiB of scratch: over the limit
-    assert lib.gdn2_workspace_size(1, 1, 1, 4096, 1, 128, 128) > g.NOALLOC_MAX_SCRATCH_BYTES
-    assert noalloc_raw(lib, 1, 1, 4096, 1, 128) == -9
+    # fp32, B*H = 1, T = 4096, d = 128 needs 37.25 MiB of scratch: over the limit
+    assert lib.gdn2_workspace_size(1, 0, 1, 4096, 1, 128, 128) > g.NOALLOC_MAX_SCRATCH_BYTES
+    assert noalloc_raw(lib, 0, 1, 4096, 1, 128) == -9
+    # bf16, B*H = 4, T = 4096, d = 128 needs 44.25 MiB
+    assert lib.gdn2_workspace_size(1, 1, 1, 4096, 4, 128, 128) > g.NOALLOC_MAX_SCRATCH_BYTES
+    assert noalloc_raw(lib, 1, 1, 4096, 4, 128) == -9
     assert b"static" in lib.gdn2_strerror(-9)
     assert noalloc_raw(lib, 1, 1, 64, 1, 96) == -8
     assert noalloc_raw(lib, 7, 1, 64, 1, 128) == -3
@@ -56,7 +59,8 @@ CALLS = [("bf16", 1, 200, 2, 128, 11, False),
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_backward(cuda_lib):
     for dtype, B, T, H, D, seed, with_dst in CALLS:
-        assert g.gdn2_workspace_size(1, torch.float32, B, T, H, D, D) <= g.NOALLOC_MAX_SCRATCH_BYTES
+        tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+        assert g.gdn2_workspace_size(1, tdt, B, T, H, D, D) <= g.NOALLOC_MAX_SCRATCH_BYTES
         x = to_dev(make_inputs(B, T, H, D, D, dtype=dtype, seed=seed, with_do=True))
         dST = (torch.randn(B, H, D, D, generator=torch.Generator().manual_seed(seed)).cuda()
                if with_dst else None)
@@ -75,7 +79,7 @@ def test_noalloc_matches_workspace_backward(cuda_lib):
 
 @pytest.mark.gpu
 def test_noalloc_over_limit_writes_nothing(cuda_lib):
-    x = to_dev(make_inputs(1, 4096, 1, 128, 128, dtype="bf16", seed=5, with_do=True))
+    x = to_dev(make_inputs(1, 4096, 4, 128, 128, dtype="bf16", seed=5, with_do=True))
     out = _grads_like(x)
     for t in out.values():
         t.fill_(7.0)
