@@ -175,13 +175,30 @@ def time_region(fn, steps, warmup, stream):
     e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if torch.distributed.is_initialized():
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-        torch.distributed.barrier()
-    return ms
+    return max_over_ranks(e0.elapsed_time(e1))
+
+
+# ------------------------------------------------------------------ multi-rank plumbing
+def max_over_ranks(ms: float) -> float:
+    """The slowest rank's time: every rank joins the same all-reduce (MAX), then a barrier.
+    The tensor lives where the process group's backend wants it (cuda for nccl, cpu for gloo)."""
+    if not torch.distributed.is_initialized():
+        return ms
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.barrier()
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch of the workload (weak scaling, no data-path collective)."""
+    return 1234 + rank
+
+
+def job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
 
 
 def roofline(bytes_per_launch, ms_per_launch, pk, traffic=None, bound="hbm"):
@@ -269,7 +286,7 @@ def run_ours(args):
     clocks = ClockSampler(dev.index)
 
     # ---- forward (headline)
-    x = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=1234 + rank, device=str(dev), with_do=True)
+    x = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=rank_seed(rank), device=str(dev), with_do=True)
     o = torch.empty_like(x["v"])
     ST = torch.empty_like(x["S0"])
 
@@ -308,7 +325,7 @@ def run_ours(args):
         if ms_fwd is not None:
             ms_fb = ms_fwd + ms_bwd
             extras["fwd_bwd"].update({
-                "value": round(world * tokens / (ms_fb * 1e-3), 1), "unit": "tokens/s",
+                "value": round(job_rate(tokens, world, ms_fb), 1), "unit": "tokens/s",
                 "ms_per_step": round(ms_fb, 4), "roofline": roofline(fb + bb, ms_fb, pk)})
         del ws, grads
 
@@ -347,7 +364,7 @@ def run_ours(args):
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    value = world * tokens / (ms_fwd * 1e-3)
+    value = job_rate(tokens, world, ms_fwd)
 
     # ---- end to end through the binding with host buffers
     hx = {n: t.to("cpu").pin_memory() for n, t in x.items() if n != "do"}
@@ -380,7 +397,7 @@ def run_ours(args):
                    "inputs": "bf16 q,k,v,b,w; fp32 log alpha and state; S0 ~ N(0, 0.02)",
                    "l2": f"inputs exceed L2 ({fb / 1e9:.2f} GB per step vs 126 MB): no flush",
                    "parallelism": f"dp{world}: independent (batch, head) sequences per rank, no collective"},
-        "e2e": {"value": round(world * tokens / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_rate(tokens, world, ms_e2e), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3)},
         "gpu_launches": args.steps,
         "roofline": roofline(fb, ms_fwd, pk, kernel_traffic("fwd_tc.cu")),

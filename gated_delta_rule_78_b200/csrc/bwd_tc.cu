@@ -24,7 +24,7 @@
 // so the work splits into four launches:
 //   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary;
 //   2. bwd_prep_kernel, one CTA per chunk: factors, [A; P], T, W, R (no state needed);
-//   3. bwd_chain_kernel, one CTA per (batch, head, half of d_v): the reverse dS chain,
+//   3. bwd_chain_kernel, one CTA per (batch, head): the reverse dS chain,
 //      two warp MMAs per chunk with dS^T kept in registers; stores dS_n per chunk;
 //   4. bwd_grad_kernel, one CTA per chunk: recomputes U~ from the stored state and
 //      produces every gradient of the chunk.
@@ -98,28 +98,29 @@ __device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bb, int hh, in
     return (((size_t)bb * a.T + (size_t)ci * C + t) * a.H + hh) * D;
 }
 
-// Copy the chunk's [C][D] bf16 token rows into a swizzled tile (256-byte rows), zero
-// rows past the sequence end.  All threads of the block take part.
-__device__ __forceinline__ void load_tok_tile(uint8_t *dst, const __nv_bfloat16 *src, const BwdTcArgs &a, int bb,
-                                              int hh, int ci, int L, int tid, int nthreads)
+// cp.async versions: the copies stay in flight until cp_async_wait; rows past the
+// sequence end are zero-filled (source size 0).
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_tok_tile(uint32_t dst, const __nv_bfloat16 *src, const BwdTcArgs &a, int bb,
+                                            int hh, int ci, int L, int tid, int nthreads)
 {
     for (int idx = tid; idx < C * 16; idx += nthreads) {
         const int t = idx >> 4, ch = idx & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (t < L) v = *reinterpret_cast<const uint4 *>(src + tok_off(a, bb, hh, ci, t) + 8 * ch);
-        *reinterpret_cast<uint4 *>(dst + swz(t, 8 * ch, 256)) = v;
+        const bool ok = t < L;
+        cp_async16_zfill(dst + swz(t, 8 * ch, 256), src + (ok ? tok_off(a, bb, hh, ci, t) + 8 * ch : 0), ok);
     }
 }
-
-// Copy a dense row-major bf16 matrix (rows x cols, cols 64 or 128) into a swizzled tile.
-__device__ __forceinline__ void load_dense_tile(uint8_t *dst, const __nv_bfloat16 *src, int rows, int cols, int tid,
-                                                int nthreads)
+__device__ __forceinline__ void cp_dense_tile(uint32_t dst, const __nv_bfloat16 *src, int rows, int cols, int tid,
+                                              int nthreads)
 {
     const int cpr = cols / 8, rb = cols * 2;
     for (int idx = tid; idx < rows * cpr; idx += nthreads) {
         const int r = idx / cpr, ch = idx % cpr;
-        *reinterpret_cast<uint4 *>(dst + swz(r, 8 * ch, rb)) =
-            *reinterpret_cast<const uint4 *>(src + (size_t)r * cols + 8 * ch);
+        cp_async16(dst + swz(r, 8 * ch, rb), src + (size_t)r * cols + 8 * ch);
     }
 }
 
@@ -136,6 +137,7 @@ __device__ __forceinline__ uint32_t ld_pair(const uint8_t *tile, int rb, int row
 // Per-thread cumulative log decay: thread (channel c, quarter q4) owns tokens
 // 16 q4 .. 16 q4 + 15; on return G[i] is the inclusive cumsum at token 16 q4 + i and
 // `total` the chunk total G_C.  sTot is a [4][D] fp32 scratch.  Needs 512 threads.
+template <bool kWaitCopies = false>
 __device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const BwdTcArgs &a, int bb, int hh,
                                              int ci, int L, int c, int q4, float *sTot)
 {
@@ -148,6 +150,7 @@ __device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const
         G[i] = run;
     }
     sTot[q4 * D + c] = run;
+    if (kWaitCopies) cp_async_wait<0>();  // this thread's tile copies have landed
     __syncthreads();
     float off = 0.f, tot = 0.f;
 #pragma unroll
@@ -183,16 +186,17 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
     float *sT = reinterpret_cast<float *>(sm + P_ST);
 
     // ---- raw q, k, b, dO tiles; T scratch zeroed (its upper blocks stay zero)
-    load_tok_tile(sm + P_Q, a.q, a, bb, hh, ci, L, tid, kPrepThreads);
-    load_tok_tile(sm + P_K, a.k, a, bb, hh, ci, L, tid, kPrepThreads);
-    load_tok_tile(sm + P_E, a.b, a, bb, hh, ci, L, tid, kPrepThreads);
-    load_tok_tile(sm + P_DO, a.dO, a, bb, hh, ci, L, tid, kPrepThreads);
+    cp_tok_tile(sb + P_Q, a.q, a, bb, hh, ci, L, tid, kPrepThreads);
+    cp_tok_tile(sb + P_K, a.k, a, bb, hh, ci, L, tid, kPrepThreads);
+    cp_tok_tile(sb + P_E, a.b, a, bb, hh, ci, L, tid, kPrepThreads);
+    cp_tok_tile(sb + P_DO, a.dO, a, bb, hh, ci, L, tid, kPrepThreads);
+    cp_async_commit();
     for (int idx = tid; idx < C * LDA; idx += kPrepThreads) sT[idx] = 0.f;
     // ---- decay folding (thread: channel c, 16 tokens); K^ and gamma go straight out
     {
         const int c = tid & (D - 1), q4 = tid >> 7;
         float G[16], GC;
-        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
+        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
         if (q4 == 0) a.gam[cidx * D + c] = __expf(GC);
         __nv_bfloat16 *kh = a.Kh + cidx * C * D;
 #pragma unroll
@@ -216,8 +220,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 7, nh = warp >> 3;
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, false>(acc, sb + (mt < 4 ? P_E : P_Q), 256, 16 * (mt & 3), sb + P_K, 256, 32 * nh, D,
-                                      lane);
+        warp_gemm<1, 4, false, false, D>(acc, sb + (mt < 4 ? P_E : P_Q), 256, 16 * (mt & 3), sb + P_K, 256, 32 * nh,
+                                         lane);
         const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 3, nh = (warp >> 2) & 1;
         float acc[1][8][4];
         zero_acc(acc);
-        warp_gemm<1, 8, true, true>(acc, sb + P_PB, 128, 16 * mt, sb + P_DO, 256, 64 * nh, C, lane);
+        warp_gemm<1, 8, true, true, C>(acc, sb + P_PB, 128, 16 * mt, sb + P_DO, 256, 64 * nh, lane);
         const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 3, nq = warp >> 2;
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, true>(acc, sb + P_TB, 128, 16 * mt, sb + P_E, 256, 32 * nq, C, lane);
+        warp_gemm<1, 4, false, true, C>(acc, sb + P_TB, 128, 16 * mt, sb + P_E, 256, 32 * nq, lane);
         const int g = lane >> 2, t4 = lane & 3;
         __nv_bfloat16 *wg = a.W + cidx * C * D;
 #pragma unroll
@@ -289,8 +293,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mb = warp & 3, nb = warp >> 2;
         float acc[2][4][4];
         zero_acc(acc);
-        warp_gemm<2, 4, true, true>(acc, sb + P_DO, 256, 32 * mb, sb + P_Q, 256, 32 * nb, C, lane);
-        warp_gemm<2, 4, true, true>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, C, lane);
+        warp_gemm<2, 4, true, true, C>(acc, sb + P_DO, 256, 32 * mb, sb + P_Q, 256, 32 * nb, lane);
+        warp_gemm<2, 4, true, true, C>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, lane);
         const int g = lane >> 2, t4 = lane & 3;
         float *rt = a.Rt + cidx * D * D;
 #pragma unroll
@@ -307,23 +311,25 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
 }
 
 // ================================================================== 3. chain
-// One CTA per (batch, head, half of d_v); warp w owns 16 rows j of dS^T (d_v x d_k)
-// and keeps them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
+// One CTA per (batch, head); warp w owns rows 16 w .. 16 w + 15 of dS^T (d_v x d_k) and
+// keeps them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
 //   store dS_n^T (bf16) for the gradient kernel;
 //   Z^T = dS_n^T K^^T          (16 x 64 per warp, K = 128; A operand from registers)
 //   dS^T = dS_n^T Diag(gamma) + R^T - Z^T W   (K = 64; A operand = -Z^T from registers)
-// W, K^ and gamma of the next chunk are copied in (cp.async) during the current one.
-constexpr int kChainThreads = 128;
-constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_BUF = 33280;  // per buffer
+// W, K^, gamma and R^T of the next chunk are copied in (cp.async) during the current one.
+constexpr int kChainThreads = 256;
+constexpr int LDR = 136;  // fp32 row stride of the R^T tile (conflict-free fragment reads)
+constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_R = 33280;
+constexpr uint32_t CH_BUF = CH_R + D * LDR * 4;  // per buffer
 constexpr uint32_t CH_SMEM = 2 * CH_BUF;
 
-__global__ void __launch_bounds__(kChainThreads) bwd_chain_kernel(const BwdTcArgs a)
+__global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, vh = blockIdx.y;
+    const int bh = blockIdx.x;
     const int g = lane >> 2, t4 = lane & 3;
-    const int j0 = 64 * vh + 16 * warp;  // this warp's first row of dS^T
+    const int j0 = 16 * warp;  // this warp's first row of dS^T
     const int nc = a.nchunks;
     const uint32_t sb = smem_u32(sm);
 
@@ -335,6 +341,11 @@ __global__ void __launch_bounds__(kChainThreads) bwd_chain_kernel(const BwdTcArg
             const int t = idx >> 4, ch = idx & 15;
             cp_async16(base + CH_W + swz(t, 8 * ch, 256), wsrc + t * D + 8 * ch);
             cp_async16(base + CH_K + swz(t, 8 * ch, 256), ksrc + t * D + 8 * ch);
+        }
+        const float *rsrc = a.Rt + cidx * D * D;
+        for (int idx = tid; idx < D * 32; idx += kChainThreads) {
+            const int r = idx >> 5, ch = idx & 31;
+            cp_async16(base + CH_R + (r * LDR + 4 * ch) * 4, rsrc + r * D + 4 * ch);
         }
         if (tid < 32) cp_async16(base + CH_G + 16 * tid, a.gam + cidx * D + 4 * tid);
         cp_async_commit();
@@ -362,14 +373,7 @@ __global__ void __launch_bounds__(kChainThreads) bwd_chain_kernel(const BwdTcArg
         __syncthreads();
         const uint32_t wb = sb + buf * CH_BUF + CH_W, kb = sb + buf * CH_BUF + CH_K;
         const float *gam = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_G);
-        // R^T of this chunk (issued early, used after the first product)
-        float2 R[16][2];
-        const float *rsrc = a.Rt + cidx * D * D;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-                R[nt][hr] = __ldcs(reinterpret_cast<const float2 *>(rsrc + (size_t)(j0 + g + 8 * hr) * D + 8 * nt + 2 * t4));
+        const float *rt = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_R);
         // dS_n^T for the gradient kernel, and as bf16 A fragments
         uint32_t aS[8][4];
         __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
@@ -402,10 +406,12 @@ __global__ void __launch_bounds__(kChainThreads) bwd_chain_kernel(const BwdTcArg
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
             const float2 gm = *reinterpret_cast<const float2 *>(gam + 8 * nt + 2 * t4);
-            dS[nt][0] = dS[nt][0] * gm.x + R[nt][0].x;
-            dS[nt][1] = dS[nt][1] * gm.y + R[nt][0].y;
-            dS[nt][2] = dS[nt][2] * gm.x + R[nt][1].x;
-            dS[nt][3] = dS[nt][3] * gm.y + R[nt][1].y;
+            const float2 r0 = *reinterpret_cast<const float2 *>(rt + (j0 + g) * LDR + 8 * nt + 2 * t4);
+            const float2 r1 = *reinterpret_cast<const float2 *>(rt + (j0 + g + 8) * LDR + 8 * nt + 2 * t4);
+            dS[nt][0] = dS[nt][0] * gm.x + r0.x;
+            dS[nt][1] = dS[nt][1] * gm.y + r0.y;
+            dS[nt][2] = dS[nt][2] * gm.x + r1.x;
+            dS[nt][3] = dS[nt][3] * gm.y + r1.y;
         }
 #pragma unroll
         for (int kt = 0; kt < 4; ++kt) {
@@ -461,19 +467,20 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     const int c = tid & (D - 1), q4 = tid >> 7;  // elementwise mapping: channel, quarter of the tokens
 
     // ---- P0: operands
-    load_tok_tile(sm + G_Q, a.q, a, bb, hh, ci, L, tid, kGradThreads);
-    load_tok_tile(sm + G_K, a.k, a, bb, hh, ci, L, tid, kGradThreads);
-    load_tok_tile(sm + G_E, a.b, a, bb, hh, ci, L, tid, kGradThreads);
-    load_tok_tile(sm + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
-    load_tok_tile(sm + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
-    load_tok_tile(sm + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_Q, a.q, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_K, a.k, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_E, a.b, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
     const __nv_bfloat16 *st_c = a.states + ((size_t)bh * (a.nchunks + 1) + ci) * D * D;
-    load_dense_tile(sm + G_S, st_c, D, D, tid, kGradThreads);
-    load_dense_tile(sm + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
-    load_dense_tile(sm + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
+    cp_dense_tile(sb + G_S, st_c, D, D, tid, kGradThreads);
+    cp_dense_tile(sb + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
+    cp_dense_tile(sb + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
+    cp_async_commit();
     {
         float G[16], GC;
-        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // its barrier also covers the tile loads
+        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // its barrier also publishes the tiles
         if (q4 == 0) sGam[c] = __expf(GC);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     {
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, false>(acc, sb + G_E, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
+        warp_gemm<1, 4, false, false, D>(acc, sb + G_E, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -553,7 +560,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     {
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, true>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, C, lane);
+        warp_gemm<1, 4, false, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -565,8 +572,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     {
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, true, true>(acc, sb + G_PB, 128, 16 * mt, sb + G_DO, 256, 32 * nq, C, lane);
-        warp_gemm<1, 4, false, false>(acc, sb + G_K, 256, 16 * mt, sb + G_DS, 256, 32 * nq, D, lane);
+        warp_gemm<1, 4, true, true, C>(acc, sb + G_PB, 128, 16 * mt, sb + G_DO, 256, 32 * nq, lane);
+        warp_gemm<1, 4, false, false, D>(acc, sb + G_K, 256, 16 * mt, sb + G_DS, 256, 32 * nq, lane);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -578,7 +585,20 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     {
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, true, true>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, C, lane);
+        warp_gemm<1, 4, true, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
+        uint32_t vv[4][2], ww[4][2];  // all loads first, so that they are in flight together
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
+                vv[nt][hr] = ww[nt][hr] = 0u;
+                if (row < L) {
+                    const size_t off = tok_off(a, bb, hh, ci, row) + col;
+                    vv[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.v + off));
+                    ww[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.w + off));
+                }
+            }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -588,10 +608,9 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
                 st_pair(sm + G_DY, 256, row, col, -d0, -d1);
                 if (row < L) {
                     const size_t off = tok_off(a, bb, hh, ci, row) + col;
-                    const uint32_t vv = *reinterpret_cast<const uint32_t *>(a.v + off);
-                    const uint32_t ww = *reinterpret_cast<const uint32_t *>(a.w + off);
-                    *reinterpret_cast<uint32_t *>(a.dv + off) = pack_bf16x2(d0 * bf_lo(ww), d1 * bf_hi(ww));
-                    *reinterpret_cast<uint32_t *>(a.dw + off) = pack_bf16x2(d0 * bf_lo(vv), d1 * bf_hi(vv));
+                    const uint32_t v2 = vv[nt][hr], w2 = ww[nt][hr];
+                    *reinterpret_cast<uint32_t *>(a.dv + off) = pack_bf16x2(d0 * bf_lo(w2), d1 * bf_hi(w2));
+                    *reinterpret_cast<uint32_t *>(a.dw + off) = pack_bf16x2(d0 * bf_lo(v2), d1 * bf_hi(v2));
                 }
             }
     }
@@ -601,8 +620,8 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
         const int ms = warp & 7, nh = warp >> 3;
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, false>(acc, sb + (ms < 4 ? G_DO : G_DY), 256, 16 * (ms & 3), sb + G_X, 256, 32 * nh, D,
-                                      lane);
+        warp_gemm<1, 4, false, false, D>(acc, sb + (ms < 4 ? G_DO : G_DY), 256, 16 * (ms & 3), sb + G_X, 256, 32 * nh,
+                                         lane);
         uint8_t *dst = sm + G_Y + (ms < 4 ? 0 : 8192);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
@@ -623,14 +642,19 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     zero_acc(aq);
     zero_acc(ae);
     zero_acc(ak);
-    warp_gemm<1, 4, false, true>(aq, sb + G_DO, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
-    warp_gemm<1, 4, false, true>(aq, dPb, 128, 16 * mt, sb + G_K, 256, 32 * nq, C, lane);
-    warp_gemm<1, 4, false, true>(ae, sb + G_DY, 256, 16 * mt, sb + G_S, 256, 32 * nq, D, lane);
-    warp_gemm<1, 4, false, true>(ae, dAb, 128, 16 * mt, sb + G_K, 256, 32 * nq, C, lane);
-    warp_gemm<1, 4, true, true>(ak, dAb, 128, 16 * mt, sb + G_E, 256, 32 * nq, C, lane);
-    warp_gemm<1, 4, true, true>(ak, dPb, 128, 16 * mt, sb + G_Q, 256, 32 * nq, C, lane);
-    warp_gemm<1, 4, false, true>(ak, sb + G_X, 256, 16 * mt, sb + G_DS, 256, 32 * nq, D, lane);
+    warp_gemm<1, 4, false, true, D>(aq, sb + G_DO, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
+    warp_gemm<1, 4, false, true, C>(aq, dPb, 128, 16 * mt, sb + G_K, 256, 32 * nq, lane);
+    warp_gemm<1, 4, false, true, D>(ae, sb + G_DY, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
+    warp_gemm<1, 4, false, true, C>(ae, dAb, 128, 16 * mt, sb + G_K, 256, 32 * nq, lane);
+    warp_gemm<1, 4, true, true, C>(ak, dAb, 128, 16 * mt, sb + G_E, 256, 32 * nq, lane);
+    warp_gemm<1, 4, true, true, C>(ak, dPb, 128, 16 * mt, sb + G_Q, 256, 32 * nq, lane);
+    warp_gemm<1, 4, false, true, D>(ak, sb + G_X, 256, 16 * mt, sb + G_DS, 256, 32 * nq, lane);
     __syncthreads();  // all operand tiles are dead from here on
+    // raw q, k, b for the factor chain, into tiles that the fp32 gradients do not cover
+    cp_tok_tile(sb + G_X, a.q, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_Y, a.k, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_tok_tile(sb + G_DO, a.b, a, bb, hh, ci, L, tid, kGradThreads);
+    cp_async_commit();
     {
         float *fq = reinterpret_cast<float *>(sm + G_FQ), *fe = reinterpret_cast<float *>(sm + G_FE);
         float *fk = reinterpret_cast<float *>(sm + G_FK);
@@ -650,20 +674,17 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
         const float *fq = reinterpret_cast<const float *>(sm + G_FQ), *fe = reinterpret_cast<const float *>(sm + G_FE);
         const float *fk = reinterpret_cast<const float *>(sm + G_FK);
         float G[16], GC;
-        chunk_cumsum(G, GC, a, bb, hh, ci, L, c, q4, sTot + 0);  // sTot is free again (P0 finished)
+        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // sTot is free again (P0 finished)
         float dG[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * q4 + i;
             const float dQ = fq[t * LDF + c], dE = fe[t * LDF + c], dK = fk[t * LDF + c];
-            float qv = 0.f, kv = 0.f, bv = 0.f;
-            size_t off = 0;
-            if (t < L) {
-                off = tok_off(a, bb, hh, ci, t) + c;
-                qv = __bfloat162float(a.q[off]);
-                kv = __bfloat162float(a.k[off]);
-                bv = __bfloat162float(a.b[off]);
-            }
+            const uint32_t off_s = swz(t, c, 256);
+            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_X + off_s));
+            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_Y + off_s));
+            const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_DO + off_s));
+            const size_t off = (t < L) ? tok_off(a, bb, hh, ci, t) + c : 0;
             const float eG = __expf(G[i]), emG = __expf(-G[i]);
             const float de = dE * eG;
             dG[i] = dQ * qv * eG + de * bv * kv - dK * kv * emG;
@@ -739,7 +760,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     bwd_prep_kernel<<<nblk, kPrepThreads, P_SMEM, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
-    bwd_chain_kernel<<<dim3(p.B * p.H, 2), kChainThreads, CH_SMEM, s>>>(a);
+    bwd_chain_kernel<<<p.B * p.H, kChainThreads, CH_SMEM, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)G_SMEM)) != cudaSuccess) return e;
     bwd_grad_kernel<<<nblk, kGradThreads, G_SMEM, s>>>(a);

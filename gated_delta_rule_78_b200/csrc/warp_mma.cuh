@@ -216,11 +216,13 @@ __device__ __forceinline__ void load_b2(uint32_t (&b)[4], uint32_t base, int row
 }
 
 // acc[MT][NT] (a (16 MT) x (8 NT) tile at (m0, n0)) += op(A)[m0.., 0:K] op(B)[0:K, n0..]
-template <int MT, int NT, bool A_KM, bool B_KN>
+// (K fixed at compile time so that the fragment loads of later k-steps are issued early)
+template <int MT, int NT, bool A_KM, bool B_KN, int K>
 __device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], uint32_t a_base, int a_rb, int m0,
-                                          uint32_t b_base, int b_rb, int n0, int K, int lane)
+                                          uint32_t b_base, int b_rb, int n0, int lane)
 {
     static_assert(NT % 2 == 0, "B fragments come in pairs of 8-column tiles");
+#pragma unroll
     for (int k0 = 0; k0 < K; k0 += 16) {
         uint32_t a[MT][4];
 #pragma unroll
