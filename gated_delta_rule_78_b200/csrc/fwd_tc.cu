@@ -345,7 +345,6 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 if (tid == 0) {
                     tma_store_3d(&maps.o, sm + ott, 0, hh, bb * T + ci * C);
                     bulk_commit();
-                    bulk_wait_read0();
                 }
             } else if (p.o) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
                 const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
@@ -360,7 +359,10 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             }
             fence_proxy_async_smem();
             named_sync(1, kGroup);
-            if (tid == 0) mbar_arrive(&bar_mdone[buf]);  // this parity's buffers and w are free
+            if (tid == 0) {
+                bulk_wait_read0();                 // the output store has read its tile
+                mbar_arrive(&bar_mdone[buf]);      // this parity's buffers and w are free
+            }
         }
         if (!s_abort_m && p.S_T) {
 #pragma unroll
