@@ -13,7 +13,9 @@ steps) and the roofline fraction of each, plus:
 * `e2e`: the same forward through the public binding with host buffers:
   pinned-host inputs copied in and o/S_T copied out inside the timed region;
 * `cpu_baseline`: the fp64 oracle timed on a bounded sample on the host cores;
-* `clocks`: SM clock and throttle reasons sampled during the timed regions.
+* `clocks`: SM clock and throttle reasons sampled during the timed regions;
+* `sweep`: forward throughput at 65,536 tokens per call for T = 2K ... 32K (B = 32 ... 2),
+  with the number of (batch, head) CTAs each shape gives the 148 SMs.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 independent (batch, head) sequences; there is no collective on the data path
@@ -354,6 +356,28 @@ def run_ours(args):
             "roofline": roofline(decode_bytes(N, Hd, Dd), ms_dec, pk, kernel_traffic("decode.cu")),
             "launches_per_step": 1}
         del steps_in
+    if "fwd" in parts and not args.no_sweep:
+        # ---- sequence-length sweep at a fixed 65,536 tokens per call (one forward per step)
+        sweep = {}
+        for name in ("sweep_2k", "sweep_4k", "sweep_8k", "sweep_16k", "sweep_32k"):
+            sw = WORKLOADS[name]
+            xs = make_inputs(sw["B"], sw["T"], sw["H"], sw["Dk"], sw["Dv"], dtype=sw["dtype"], seed=rank_seed(rank),
+                             device=str(dev))
+            os_ = torch.empty_like(xs["v"])
+            Ss = torch.empty_like(xs["S0"])
+
+            def fwd_s():
+                g.gdn2_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["b"], xs["w"], xs["S0"], o=os_, S_T=Ss)
+
+            ks = 10
+            ms_s = time_region(fwd_s, ks, 3, stream) / ks
+            assert g.gdn2_sync_status() == 0
+            bs = fwd_bytes(sw["B"], sw["T"], sw["H"], sw["Dk"])
+            sweep[name] = {"T": sw["T"], "B": sw["B"], "ctas": sw["B"] * sw["H"], "ms": round(ms_s, 4),
+                           "tokens_per_s": round(job_rate(sw["B"] * sw["T"], world, ms_s), 1),
+                           "hbm_frac": round(bs / (ms_s * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+            del xs, os_, Ss
+        extras["sweep"] = sweep
     clocks.stop()
     if ms_fwd is None:
         # a single non-forward part was asked for (profiling runs): report it alone
@@ -422,6 +446,7 @@ def main():
     ap.add_argument("--workload", default="layer_4k", choices=sorted(WORKLOADS))
     ap.add_argument("--fwd-only", action="store_true", help="skip the fwd+bwd and decode figures")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the sequence-length sweep")
     ap.add_argument("--only", choices=["fwd", "bwd", "decode"], default=None,
                     help="time one part only (for profiling runs)")
     args = ap.parse_args()
