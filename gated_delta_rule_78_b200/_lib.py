@@ -18,10 +18,12 @@ LIB_PATH = os.path.join(_HERE, "libgdn2.so")
 GDN2_OK = 0
 STATUS_NAMES = {0: "GDN2_OK", -1: "GDN2_ERR_NULL", -2: "GDN2_ERR_SHAPE", -3: "GDN2_ERR_DTYPE",
                 -4: "GDN2_ERR_ALIGN", -5: "GDN2_ERR_WORKSPACE", -6: "GDN2_ERR_CUDA",
-                -7: "GDN2_ERR_TIMEOUT", -8: "GDN2_ERR_UNSUPPORTED", -9: "GDN2_ERR_TOO_LARGE"}
+                -7: "GDN2_ERR_TIMEOUT", -8: "GDN2_ERR_UNSUPPORTED", -9: "GDN2_ERR_TOO_LARGE",
+                -10: "GDN2_ERR_SEQLENS"}
 GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
-           "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc")
+           "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
+           "gdn2_chunk_bwd_varlen")
 # Size of the library's static scratch array used by gdn2_chunk_bwd_noalloc
 # (GDN2_NOALLOC_MAX_SCRATCH_BYTES in include/gdn2.h).
 NOALLOC_MAX_SCRATCH_BYTES = 32 << 20
@@ -54,6 +56,10 @@ def load(path: str | None = None):
     lib.gdn2_chunk_bwd.restype = i
     lib.gdn2_chunk_bwd_noalloc.argtypes = [i] * 6 + [vp] * 16 + [vp]
     lib.gdn2_chunk_bwd_noalloc.restype = i
+    lib.gdn2_chunk_fwd_varlen.argtypes = [i] * 6 + [vp] * 11 + [sz, vp]
+    lib.gdn2_chunk_fwd_varlen.restype = i
+    lib.gdn2_chunk_bwd_varlen.argtypes = [i] * 6 + [vp] * 18 + [sz, vp]
+    lib.gdn2_chunk_bwd_varlen.restype = i
     lib.gdn2_workspace_size.argtypes = [i] * 7
     lib.gdn2_workspace_size.restype = sz
     lib.gdn2_strerror.argtypes = [i]
@@ -198,6 +204,71 @@ def gdn2_chunk_bwd_noalloc(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, out,
                                       _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["db"]),
                                       _p(out["dw"]), _p(out["dS0"]), _stream(stream))
     _check("gdn2_chunk_bwd_noalloc", st)
+    return out
+
+
+def _packed(t):
+    """[total_T, H, D] view of a packed token tensor given as [total_T, H, D] or [1, total_T, H, D]."""
+    if t.dim() == 4:
+        if t.shape[0] != 1:
+            raise ValueError("packed tensors are [total_T, H, D] (or [1, total_T, H, D])")
+        return t[0]
+    return t
+
+
+def gdn2_chunk_fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0=None, *, o=None, S_T=None, want_state=True,
+                          workspace=None, stream=None):
+    """Forward over N packed sequences (cu_seqlens int32 [N+1] on the device).
+    Returns (o [total_T, H, Dv], S_T [N, H, Dk, Dv] or None)."""
+    q3, k3, v3, g3, b3, w3 = (_packed(t) for t in (q, k, v, log_alpha, b, w))
+    total_T, H, Dk = q3.shape
+    Dv = v3.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt = _dt(q3)
+    for n, t in (("q", q3), ("k", k3), ("v", v3), ("b", b3), ("w", w3)):
+        _cuda_contig(n, t, q3.dtype)
+    _cuda_contig("log_alpha", g3, torch.float32)
+    _cuda_contig("cu_seqlens", cu_seqlens, torch.int32)
+    _cuda_contig("S0", S0, torch.float32)
+    if o is None:
+        o = torch.empty(total_T, H, Dv, dtype=q3.dtype, device=q3.device)
+    if S_T is None and want_state:
+        S_T = torch.empty(N, H, Dk, Dv, dtype=torch.float32, device=q3.device)
+    ws = workspace
+    st = raw().gdn2_chunk_fwd_varlen(dt, N, total_T, H, Dk, Dv, _p(cu_seqlens), _p(q3), _p(k3), _p(v3), _p(g3),
+                                     _p(b3), _p(w3), _p(S0), _p(o), _p(S_T), _p(ws),
+                                     0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("gdn2_chunk_fwd_varlen", st)
+    return o, S_T
+
+
+def gdn2_chunk_bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0, d_o, dS_T=None, *, workspace=None, out=None,
+                          stream=None):
+    """Backward over N packed sequences.  Returns dict(dq, dk, dv, dlog_alpha, db, dw, dS0)."""
+    q3, k3, v3, g3, b3, w3, do3 = (_packed(t) for t in (q, k, v, log_alpha, b, w, d_o))
+    total_T, H, Dk = q3.shape
+    Dv = v3.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt = _dt(q3)
+    for n, t in (("q", q3), ("k", k3), ("v", v3), ("b", b3), ("w", w3), ("d_o", do3)):
+        _cuda_contig(n, t, q3.dtype)
+    _cuda_contig("log_alpha", g3, torch.float32)
+    _cuda_contig("cu_seqlens", cu_seqlens, torch.int32)
+    _cuda_contig("S0", S0, torch.float32)
+    _cuda_contig("dS_T", dS_T, torch.float32)
+    if out is None:
+        out = {"dq": torch.empty_like(q3), "dk": torch.empty_like(k3), "dv": torch.empty_like(v3),
+               "dlog_alpha": torch.empty_like(g3), "db": torch.empty_like(b3), "dw": torch.empty_like(w3),
+               "dS0": torch.empty(N, H, Dk, Dv, dtype=torch.float32, device=q3.device)}
+    if workspace is None:
+        nbytes = gdn2_workspace_size(3, q3.dtype, N, total_T, H, Dk, Dv)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q3.device)
+    st = raw().gdn2_chunk_bwd_varlen(dt, N, total_T, H, Dk, Dv, _p(cu_seqlens), _p(q3), _p(k3), _p(v3), _p(g3),
+                                     _p(b3), _p(w3), _p(S0), _p(do3), _p(dS_T), _p(out["dq"]), _p(out["dk"]),
+                                     _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]),
+                                     _p(out["dS0"]), _p(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    _check("gdn2_chunk_bwd_varlen", st)
     return out
 
 

@@ -84,10 +84,12 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdArgs a)
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, bb = bh / p.H, hh = bh % p.H;
     const int tile = blockIdx.y, j0 = tile * kDVT;
-    const int T = p.T;
+    const SeqSpan sp = seq_span(p, bb);
+    if (sp.len < 0) return;  // invalid cu_seqlens (reported by the offsets pass)
+    const int T = sp.len;
     const size_t tok = (size_t)p.H * D;
-    const size_t base = ((size_t)bb * T * p.H + hh) * D;
-    const size_t total = (size_t)p.B * T * p.H * D;
+    const size_t base = tok_row(p, sp, hh, 0);
+    const size_t total = token_rows(p) * p.H * D;
     const int nchunks = (T + C - 1) / C;
     const Tin *q = (const Tin *)p.q, *k = (const Tin *)p.k, *v = (const Tin *)p.v;
     const Tin *bg = (const Tin *)p.b, *wg = (const Tin *)p.w, *dog = (const Tin *)a.d_o;
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdArgs a)
             }
         }
         {
-            const float *src = a.states + (((size_t)bh * nchunks + ci) * D) * D;
+            const float *src = a.states + chunk_slot(p, bb, hh, nchunks, ci) * D * D;
             for (int idx = tid; idx < D * kDVT; idx += kThreads) {
                 const int c = idx / kDVT, j = idx % kDVT;
                 Sc[idx] = src[(size_t)c * D + j0 + j];
@@ -379,32 +381,40 @@ __global__ void reduce_parts_kernel(const float *__restrict__ part, int nt, size
 }
 
 struct WsLayout {
-    size_t states, scratch, part, total;
+    size_t coff, states, scratch, part, total;
 };
 
-WsLayout ws_layout(int B, int T, int H, int D)
+// [chunk_off (variable length only)] [chunk-start states] [per-CTA scratch] [partials]
+WsLayout ws_layout(const Problem &p, int D)
 {
-    const size_t nc = (size_t)(T + kChunk - 1) / kChunk;
     const size_t nt = D / kDVT;
     WsLayout l;
-    l.states = (size_t)B * H * nc * D * D * sizeof(float);
-    l.scratch = (size_t)B * H * nt * kScratchMats * kChunk * D * sizeof(float);
-    l.part = 4 * nt * (size_t)B * T * H * D * sizeof(float);
-    l.total = l.states + l.scratch + l.part;
+    l.coff = p.cu_seqlens ? varlen_offsets_bytes(p.B) : 0;
+    l.states = (size_t)p.H * chunk_bound(p) * D * D * sizeof(float);
+    l.scratch = (size_t)p.B * p.H * nt * kScratchMats * kChunk * D * sizeof(float);
+    l.part = 4 * nt * token_rows(p) * p.H * D * sizeof(float);
+    l.total = l.coff + l.states + l.scratch + l.part;
     return l;
 }
 
 template <int D, typename Tin>
-cudaError_t launch_t(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out,
-                     void *ws, cudaStream_t s)
+cudaError_t launch_t(const Problem &p0, const void *d_o, const float *dS_T, const BwdOut &out,
+                     void *ws, int *status, cudaStream_t s)
 {
-    const WsLayout l = ws_layout(p.B, p.T, p.H, D);
+    const WsLayout l = ws_layout(p0, D);
     char *base = (char *)ws;
+    Problem p = p0;
+    cudaError_t e;
+    if (p.cu_seqlens) {
+        int *coff = reinterpret_cast<int *>(base);
+        if ((e = launch_chunk_offsets(p.cu_seqlens, p.B, p.T, coff, status, s)) != cudaSuccess) return e;
+        p.chunk_off = coff;
+    }
+    base += l.coff;
     float *states = (float *)base;
     float *scratch = (float *)(base + l.states);
     float *part = (float *)(base + l.states + l.scratch);
-    cudaError_t e = launch_fwd_simt(sizeof(Tin) == 4 ? GDN2_F32 : GDN2_BF16, p, nullptr, nullptr,
-                                    states, s);
+    e = launch_fwd_simt(sizeof(Tin) == 4 ? GDN2_F32 : GDN2_BF16, p, nullptr, nullptr, states, s);
     if (e != cudaSuccess) return e;
     const size_t smem = BwdSmem<D>::bytes;
     e = cudaFuncSetAttribute(bwd_chunk_kernel<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -414,7 +424,7 @@ cudaError_t launch_t(const Problem &p, const void *d_o, const float *dS_T, const
     bwd_chunk_kernel<D, Tin><<<dim3(p.B * p.H, D / kDVT), kThreads, smem, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t total = (size_t)p.B * p.T * p.H * D;
+    const size_t total = token_rows(p) * p.H * D;
     const int blocks = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
     reduce_parts_kernel<Tin><<<blocks, 256, 0, s>>>(part, D / kDVT, total, (Tin *)out.dq,
                                                     (Tin *)out.dk, (Tin *)out.db, out.dg);
@@ -423,25 +433,23 @@ cudaError_t launch_t(const Problem &p, const void *d_o, const float *dS_T, const
 
 }  // namespace
 
-size_t bwd_workspace_bytes(gdn2_dtype dt, int B, int T, int H, int D)
+size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p)
 {
-    if (dt == GDN2_BF16 && D == 128) return bwd_tc_workspace_bytes(B, T, H);
-    return ws_layout(B, T, H, D).total;
+    if (dt == GDN2_BF16 && p.D == 128) return bwd_tc_workspace_bytes(p);
+    return ws_layout(p, p.D).total;
 }
 
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
                        const BwdOut &out, void *ws, cudaStream_t s)
 {
-    if (dt == GDN2_BF16 && p.D == 128) {
-        int *status = status_word();
-        if (!status) return cudaErrorInvalidSymbol;
-        return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
-    }
+    int *status = status_word();
+    if (!status) return cudaErrorInvalidSymbol;
+    if (dt == GDN2_BF16 && p.D == 128) return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
     if (dt == GDN2_F32)
-        return p.D == 64 ? launch_t<64, float>(p, d_o, dS_T, out, ws, s)
-                         : launch_t<128, float>(p, d_o, dS_T, out, ws, s);
-    return p.D == 64 ? launch_t<64, __nv_bfloat16>(p, d_o, dS_T, out, ws, s)
-                     : launch_t<128, __nv_bfloat16>(p, d_o, dS_T, out, ws, s);
+        return p.D == 64 ? launch_t<64, float>(p, d_o, dS_T, out, ws, status, s)
+                         : launch_t<128, float>(p, d_o, dS_T, out, ws, status, s);
+    return p.D == 64 ? launch_t<64, __nv_bfloat16>(p, d_o, dS_T, out, ws, status, s)
+                     : launch_t<128, __nv_bfloat16>(p, d_o, dS_T, out, ws, status, s);
 }
 
 }  // namespace gdn2

@@ -47,30 +47,33 @@ constexpr int LDA = 68;  // fp32 row stride of the A / T scratch of the solve
 
 // ------------------------------------------------------------------ workspace
 struct BwdTcLayout {
-    size_t states, W, Kh, gam, Rt, Tm, Pm, dSn, total;
+    size_t coff, states, W, Kh, gam, Rt, Tm, Pm, dSn, total;
 };
 
 // Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W and K^ bf16
 // [C][D], gamma fp32 [D], R^T fp32 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
-BwdTcLayout tc_layout(int B, int T, int H)
+// Variable length puts chunk_off first; chunk lists are sized by the chunk bound.
+BwdTcLayout tc_layout(const Problem &p)
 {
-    const size_t bh = (size_t)B * H, nc = (size_t)(T + C - 1) / C;
+    const size_t H = p.H, nchunk = chunk_bound(p), nbound = nchunk + p.B;
     BwdTcLayout l;
-    size_t off = 0;
-    l.states = off; off += bh * (nc + 1) * D * D * 2;
-    l.W = off;      off += bh * nc * C * D * 2;
-    l.Kh = off;     off += bh * nc * C * D * 2;
-    l.gam = off;    off += bh * nc * D * 4;
-    l.Rt = off;     off += bh * nc * D * D * 4;
-    l.Tm = off;     off += bh * nc * C * C * 2;
-    l.Pm = off;     off += bh * nc * C * C * 2;
-    l.dSn = off;    off += bh * nc * D * D * 2;
+    size_t off = p.cu_seqlens ? varlen_offsets_bytes(p.B) : 0;
+    l.coff = 0;
+    l.states = off; off += H * nbound * D * D * 2;
+    l.W = off;      off += H * nchunk * C * D * 2;
+    l.Kh = off;     off += H * nchunk * C * D * 2;
+    l.gam = off;    off += H * nchunk * D * 4;
+    l.Rt = off;     off += H * nchunk * D * D * 4;
+    l.Tm = off;     off += H * nchunk * C * C * 2;
+    l.Pm = off;     off += H * nchunk * C * C * 2;
+    l.dSn = off;    off += H * nchunk * D * D * 2;
     l.total = off;
     return l;
 }
 
 struct BwdTcArgs {
-    int B, T, H, nchunks;
+    Problem pr;          // sizes, cu_seqlens and chunk_off (the data pointers are below)
+    int H;
     const __nv_bfloat16 *q, *k, *v, *b, *w, *dO;
     const float *g;
     const float *dS_T;  // may be null
@@ -92,10 +95,46 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Row t of chunk `ci` of head hh, batch bb in a [B, T, H, D] tensor.
-__device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bb, int hh, int ci, int t)
+// Row t of chunk `ci` of head hh of the sequence whose first token row is `bos`.
+__device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bos, int hh, int ci, int t)
 {
-    return (((size_t)bb * a.T + (size_t)ci * C + t) * a.H + hh) * D;
+    return (((size_t)bos + (size_t)ci * C + t) * a.H + hh) * D;
+}
+
+// The chunk a block of the chunk-parallel kernels works on: blockIdx.y is the head,
+// blockIdx.x the chunk over all sequences (fixed length: sequence-major; variable
+// length: found in chunk_off; blocks past the last chunk have nothing to do).
+struct ChunkRef {
+    int n, h, ci, nch;
+    SeqSpan sp;
+    size_t cidx;  // per-chunk workspace slot
+};
+__device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
+{
+    const Problem &p = a.pr;
+    const int gc = blockIdx.x;
+    r.h = blockIdx.y;
+    if (!p.cu_seqlens) {
+        const int nc = seq_chunks(p.T);
+        r.n = gc / nc;
+        r.ci = gc % nc;
+    } else {
+        if (gc >= p.chunk_off[p.B]) return false;
+        int lo = 0, hi = p.B;  // last n with chunk_off[n] <= gc
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.chunk_off[mid] <= gc) lo = mid;
+            else hi = mid;
+        }
+        r.n = lo;
+        r.ci = gc - p.chunk_off[lo];
+    }
+    r.sp = seq_span(p, r.n);
+    if (r.sp.len < 0) return false;
+    r.nch = seq_chunks(r.sp.len);
+    if (r.ci >= r.nch) return false;
+    r.cidx = chunk_slot(p, r.n, r.h, r.nch, r.ci);
+    return true;
 }
 
 // cp.async versions: the copies stay in flight until cp_async_wait; rows past the
@@ -177,10 +216,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ci = blockIdx.x % a.nchunks, bh = blockIdx.x / a.nchunks;
-    const int bb = bh / a.H, hh = bh % a.H;
-    const int L = min(C, a.T - ci * C);
-    const size_t cidx = (size_t)bh * a.nchunks + ci;
+    ChunkRef cr;
+    if (!chunk_ref(a, cr)) return;
+    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
+    const int L = min(C, cr.sp.len - ci * C);
+    const size_t cidx = cr.cidx;
     const uint32_t sb = smem_u32(sm);
     float *sA = reinterpret_cast<float *>(sm + P_SA);
     float *sT = reinterpret_cast<float *>(sm + P_ST);
@@ -327,14 +367,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x, n = bh / a.H, hh = bh % a.H;
     const int g = lane >> 2, t4 = lane & 3;
     const int j0 = 16 * warp;  // this warp's first row of dS^T
-    const int nc = a.nchunks;
+    const SeqSpan sp = seq_span(a.pr, n);
+    if (sp.len < 0) return;  // invalid cu_seqlens (reported by the offsets pass)
+    const int nc = seq_chunks(sp.len);
     const uint32_t sb = smem_u32(sm);
 
     auto prefetch = [&](int ci, int buf) {
-        const size_t cidx = (size_t)bh * nc + ci;
+        const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         const uint32_t base = sb + buf * CH_BUF;
         const __nv_bfloat16 *wsrc = a.W + cidx * C * D, *ksrc = a.Kh + cidx * C * D;
         for (int idx = tid; idx < C * 16; idx += kChainThreads) {
@@ -363,7 +405,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
     if (nc > 0) prefetch(nc - 1, 0);
     for (int ci = nc - 1; ci >= 0; --ci) {
         const int buf = (nc - 1 - ci) & 1;
-        const size_t cidx = (size_t)bh * nc + ci;
+        const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         if (ci > 0) {
             prefetch(ci - 1, buf ^ 1);
             cp_async_wait<1>();
@@ -455,10 +497,11 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
-    const int ci = blockIdx.x % a.nchunks, bh = blockIdx.x / a.nchunks;
-    const int bb = bh / a.H, hh = bh % a.H;
-    const int L = min(C, a.T - ci * C);
-    const size_t cidx = (size_t)bh * a.nchunks + ci;
+    ChunkRef cr;
+    if (!chunk_ref(a, cr)) return;
+    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
+    const int L = min(C, cr.sp.len - ci * C);
+    const size_t cidx = cr.cidx;
     const uint32_t sb = smem_u32(sm);
     float *sTot = reinterpret_cast<float *>(sm + G_TOT);
     float *sGam = reinterpret_cast<float *>(sm + G_GAM);
@@ -473,7 +516,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     cp_tok_tile(sb + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
     cp_tok_tile(sb + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
     cp_tok_tile(sb + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
-    const __nv_bfloat16 *st_c = a.states + ((size_t)bh * (a.nchunks + 1) + ci) * D * D;
+    const __nv_bfloat16 *st_c = a.states + bound_slot(a.pr, cr.n, hh, cr.nch, ci) * D * D;
     cp_dense_tile(sb + G_S, st_c, D, D, tid, kGradThreads);
     cp_dense_tile(sb + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
     cp_dense_tile(sb + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
@@ -719,16 +762,23 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
 
 }  // namespace
 
-size_t bwd_tc_workspace_bytes(int B, int T, int H) { return tc_layout(B, T, H).total; }
+size_t bwd_tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
 
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
                           int *status, cudaStream_t s)
 {
     if (p.D != D) return cudaErrorNotSupported;
-    const BwdTcLayout l = tc_layout(p.B, p.T, p.H);
+    const BwdTcLayout l = tc_layout(p);
     char *base = static_cast<char *>(ws);
     BwdTcArgs a;
-    a.B = p.B; a.T = p.T; a.H = p.H; a.nchunks = (p.T + C - 1) / C;
+    a.pr = p;
+    a.H = p.H;
+    if (p.cu_seqlens) {
+        int *coff = reinterpret_cast<int *>(base);
+        cudaError_t e0 = launch_chunk_offsets(p.cu_seqlens, p.B, p.T, coff, status, s);
+        if (e0 != cudaSuccess) return e0;
+        a.pr.chunk_off = coff;
+    }
     a.q = static_cast<const __nv_bfloat16 *>(p.q);
     a.k = static_cast<const __nv_bfloat16 *>(p.k);
     a.v = static_cast<const __nv_bfloat16 *>(p.v);
@@ -753,9 +803,9 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.dg = out.dg;
     a.dS0 = out.dS0;
 
-    cudaError_t e = launch_fwd_tc(p, nullptr, nullptr, a.states, status, s);
+    cudaError_t e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s);
     if (e != cudaSuccess) return e;
-    const unsigned nblk = (unsigned)((size_t)p.B * p.H * a.nchunks);
+    const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_kernel), (int)P_SMEM)) != cudaSuccess) return e;
     bwd_prep_kernel<<<nblk, kPrepThreads, P_SMEM, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -53,9 +53,11 @@ fwd_simt_kernel(Problem p, Tin *__restrict__ o, float *__restrict__ S_T, float *
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, bb = bh / p.H, hh = bh % p.H;
     const int j0 = blockIdx.y * kDVT;
-    const int T = p.T;
+    const SeqSpan sp = seq_span(p, bb);
+    if (sp.len < 0) return;  // invalid cu_seqlens (reported by the offsets pass)
+    const int T = sp.len;
     const size_t tok = (size_t)p.H * D;                      // token stride (elements)
-    const size_t base = ((size_t)bb * T * p.H + hh) * D;      // (b, t=0, h, 0)
+    const size_t base = tok_row(p, sp, hh, 0);               // (sequence bb, t = 0, h, 0)
     const Tin *q = (const Tin *)p.q, *k = (const Tin *)p.k, *v = (const Tin *)p.v;
     const Tin *bg = (const Tin *)p.b, *wg = (const Tin *)p.w;
     const int nchunks = (T + C - 1) / C;
@@ -70,7 +72,7 @@ fwd_simt_kernel(Problem p, Tin *__restrict__ o, float *__restrict__ S_T, float *
         const int L = min(C, T - c0);
         __syncthreads();  // S ready; previous chunk done with every buffer
         if (states) {
-            float *dst = states + (((size_t)bh * nchunks + ci) * D) * D;
+            float *dst = states + chunk_slot(p, bb, hh, nchunks, ci) * D * D;
             for (int idx = tid; idx < D * kDVT; idx += kThreads) {
                 const int c = idx / kDVT, j = idx % kDVT;
                 dst[(size_t)c * D + j0 + j] = S[idx];

@@ -91,9 +91,11 @@ struct TcParams {
     const float *g;   // log alpha [B,T,H,D] fp32
     __nv_bfloat16 *o;        // may be null (states-only run)
     float *S_T;
-    __nv_bfloat16 *states;   // may be null; else [B*H][nchunks + 1][D (d_v)][D (d_k)]: S^T at every
-                             // chunk boundary, the final state last
+    __nv_bfloat16 *states;   // may be null; else S^T (d_v x d_k) at every chunk boundary, the final
+                             // state last, per (sequence, head) at the boundary slots of gdn2_internal.cuh
     int *status;
+    const int *cu_seqlens;   // null: B sequences of T tokens; else B packed sequences in T rows
+    const int *chunk_off;    // variable length with states only: first chunk of each sequence
 };
 
 struct TcMaps {
@@ -125,7 +127,16 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool is_m = warp < 8;
     const int bh = blockIdx.x, bb = bh / p.H, hh = bh % p.H;
-    const int T = p.T;
+    int bos = bb * p.T, T = p.T;  // this sequence's first token row and its length
+    if (p.cu_seqlens) {
+        const int b0 = p.cu_seqlens[bb], b1 = p.cu_seqlens[bb + 1];
+        if (b0 < 0 || b1 < b0 || b1 > p.T) {  // nothing launched yet: leave before any barrier
+            if (tid == 0) atomicExch(p.status, kStatusBadSeqlens);
+            return;
+        }
+        bos = b0;
+        T = b1 - b0;
+    }
     const int nchunks = (T + C - 1) / C;
     const uint32_t sbase = smem_u32(sm);
     float *sA = reinterpret_cast<float *>(sm + OFF_SA);
@@ -163,7 +174,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     // The issuing thread may block while the TMA engine drains earlier boxes, so the loads are
     // issued from an E warp that is idle during the solve.
     auto issue = [&](int ci) {
-        const int y = bb * T + ci * C, bf = ci & 1;
+        const int y = bos + ci * C, bf = ci & 1;
         mbar_expect_tx(&bar_in[bf], 10 * 8192);
         for (int a = 0; a < 2; ++a) {
             tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in[bf]);
@@ -211,8 +222,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         if (tid == 0 && nchunks > 1) issue(1);  // w(1) may only land after w(0) was folded
         // bf16 copy of this thread's 64 entries of S^T at chunk boundary `idx`
         auto store_state = [&](const float *Sv, int idx) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.states + (((size_t)bh * (nchunks + 1) + idx) * D + jrow) * D +
-                                                   64 * half);
+            const size_t first = p.chunk_off ? (size_t)p.chunk_off[bb] : (size_t)bb * nchunks;
+            const size_t slot = (first + bb) * p.H + (size_t)hh * (nchunks + 1) + idx;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.states + (slot * D + jrow) * D + 64 * half);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 dst[u] = make_uint4(pack_bf16x2(Sv[8 * u], Sv[8 * u + 1]), pack_bf16x2(Sv[8 * u + 2], Sv[8 * u + 3]),
@@ -343,12 +355,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             named_sync(1, kGroup);
             if (p.o && L == C) {
                 if (tid == 0) {
-                    tma_store_3d(&maps.o, sm + ott, 0, hh, bb * T + ci * C);
+                    tma_store_3d(&maps.o, sm + ott, 0, hh, bos + ci * C);
                     bulk_commit();
                 }
             } else if (p.o) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
                 const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
-                __nv_bfloat16 *dst = p.o + ((size_t)bb * T + (size_t)ci * C) * p.H * D + (size_t)hh * D;
+                __nv_bfloat16 *dst = p.o + ((size_t)bos + (size_t)ci * C) * p.H * D + (size_t)hh * D;
                 for (int idx = tid; idx < L * D; idx += kGroup) dst[(size_t)(idx / D) * p.H * D + idx % D] = so[idx];
                 named_sync(1, kGroup);
             }
@@ -388,7 +400,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
             // log alpha of this warp's 16 tokens x 2 channels, straight from L2
             float2 gv[16];
-            const float *gsrc = p.g + ((size_t)bb * T + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
+            const float *gsrc = p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
@@ -560,14 +572,15 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     if (pr.D != D) return cudaErrorNotSupported;
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
-    if (!make_map(&maps.q, pr.q, false, pr.B, pr.T, pr.H) || !make_map(&maps.k, pr.k, false, pr.B, pr.T, pr.H) ||
-        !make_map(&maps.v, pr.v, false, pr.B, pr.T, pr.H) || !make_map(&maps.b, pr.b, false, pr.B, pr.T, pr.H) ||
-        !make_map(&maps.w, pr.w, false, pr.B, pr.T, pr.H) || !make_map(&maps.g, pr.g, true, pr.B, pr.T, pr.H) ||
-        (o && !make_map(&maps.o, o, false, pr.B, pr.T, pr.H, true)))
+    const int rows = (int)token_rows(pr);  // the maps view every tensor as [rows, H, D]
+    if (!make_map(&maps.q, pr.q, false, 1, rows, pr.H) || !make_map(&maps.k, pr.k, false, 1, rows, pr.H) ||
+        !make_map(&maps.v, pr.v, false, 1, rows, pr.H) || !make_map(&maps.b, pr.b, false, 1, rows, pr.H) ||
+        !make_map(&maps.w, pr.w, false, 1, rows, pr.H) || !make_map(&maps.g, pr.g, true, 1, rows, pr.H) ||
+        (o && !make_map(&maps.o, o, false, 1, rows, pr.H, true)))
         return cudaErrorInvalidValue;
     cudaError_t e = set_smem_attr(reinterpret_cast<const void *>(fwd_tc_kernel), (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status};
+    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off};
     fwd_tc_kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
     return cudaGetLastError();
 }

@@ -60,7 +60,7 @@ gdn2_status check_sizes(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
     if (Dk != Dv || (Dk != 64 && Dk != 128)) return GDN2_ERR_UNSUPPORTED;
     // element counts must fit comfortably in the kernels' 64-bit index math and
     // the grid's x dimension
-    if ((long long)B * H > (1LL << 30)) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1LL << 30) || H > 65535) return GDN2_ERR_UNSUPPORTED;
     if ((long long)B * T * H * Dk > (1LL << 40)) return GDN2_ERR_UNSUPPORTED;
     return GDN2_OK;
 }
@@ -86,6 +86,24 @@ gdn2::Problem make_problem(int B, int T, int H, int D, const void *q, const void
     return p;
 }
 
+// Launch the forward of a validated problem (T > 0): bf16 with D = 128 on the tensor
+// cores, everything else on the FMA kernel.  Variable length first checks cu_seqlens.
+gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s)
+{
+    int *status = gdn2::status_word();
+    if (!status) return GDN2_ERR_CUDA;
+    if (p.cu_seqlens) {
+        cudaError_t e = gdn2::launch_chunk_offsets(p.cu_seqlens, p.B, p.T, nullptr, status, s);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    }
+    if (dt == GDN2_BF16) {
+        cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();  // clear the sticky "not supported" code; fall through to FMA path
+    }
+    return from_cuda(gdn2::launch_fwd_simt(dt, p, o, S_T, nullptr, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,6 +121,7 @@ const char *gdn2_strerror(gdn2_status s)
     case GDN2_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
     case GDN2_ERR_UNSUPPORTED: return "outside the supported shapes (Dk == Dv in {64, 128})";
     case GDN2_ERR_TOO_LARGE: return "problem needs more scratch than the library's static array holds";
+    case GDN2_ERR_SEQLENS: return "cu_seqlens is not 0 = c_0 <= c_1 <= ... <= c_N = total_T";
     }
     return "unknown status";
 }
@@ -110,9 +129,12 @@ const char *gdn2_strerror(gdn2_status s)
 size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
 {
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK) return 0;
-    if (which == 0) return 0;
-    if (which == 1) return T == 0 ? 0 : gdn2::bwd_workspace_bytes(dt, B, T, H, Dk);
-    return 0;
+    if (T == 0 || which == 0 || which == 2) return 0;
+    if (which != 1 && which != 3) return 0;
+    gdn2::Problem p = make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+    static const int marker = 0;
+    if (which == 3) p.cu_seqlens = &marker;  // sizes only: the pointer is not read
+    return gdn2::bwd_workspace_bytes(dt, p);
 }
 
 gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
@@ -135,14 +157,7 @@ gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
         return from_cuda(cudaMemsetAsync(S_T, 0, state_bytes, s));
     }
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
-    if (dt == GDN2_BF16) {
-        int *status = nullptr;
-        if (cudaGetSymbolAddress((void **)&status, g_gdn2_status) != cudaSuccess) return GDN2_ERR_CUDA;
-        cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s);
-        if (e != cudaErrorNotSupported) return from_cuda(e);
-        cudaGetLastError();  // clear the sticky "not supported" code; fall through to FMA path
-    }
-    return from_cuda(gdn2::launch_fwd_simt(dt, p, o, S_T, nullptr, s));
+    return run_fwd(dt, p, o, S_T, s);
 }
 
 gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int Dv, const void *q,
@@ -177,10 +192,68 @@ gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
         if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
         return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
     }
-    const size_t need = gdn2::bwd_workspace_bytes(dt, B, T, H, Dk);
+    const size_t need = gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr,
+                                                                    nullptr, nullptr, nullptr));
     if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
+    return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s));
+}
+
+gdn2_status gdn2_chunk_fwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int Dk, int Dv,
+                                  const int *cu_seqlens, const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const void *b, const void *w, const float *S0, void *o,
+                                  float *S_T, void *workspace, size_t ws_bytes, void *stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    gdn2_status st = check_sizes(dt, N, total_T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (!cu_seqlens) return GDN2_ERR_NULL;
+    if (((uintptr_t)cu_seqlens & 3u) != 0) return GDN2_ERR_ALIGN;
+    if (total_T > 0) st = check_ptrs({q, k, v, log_alpha, b, w, o}, {S0, S_T});
+    else st = check_ptrs({}, {S0, S_T});
+    if (st != GDN2_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)N * H * Dk * Dv * sizeof(float);
+    if (total_T == 0) {  // every sequence is empty: S_T = S0
+        if (!S_T) return GDN2_OK;
+        if (S0) return S0 == S_T ? GDN2_OK : from_cuda(cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(S_T, 0, state_bytes, s));
+    }
+    gdn2::Problem p = make_problem(N, total_T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    p.cu_seqlens = cu_seqlens;
+    return run_fwd(dt, p, o, S_T, s);
+}
+
+gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int Dk, int Dv,
+                                  const int *cu_seqlens, const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const void *b, const void *w, const float *S0,
+                                  const void *d_o, const float *dS_T, void *dq, void *dk, void *dv,
+                                  float *dlog_alpha, void *db, void *dw, float *dS0, void *workspace,
+                                  size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_sizes(dt, N, total_T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (!cu_seqlens) return GDN2_ERR_NULL;
+    if (((uintptr_t)cu_seqlens & 3u) != 0) return GDN2_ERR_ALIGN;
+    if (total_T > 0)
+        st = check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0}, {S0, dS_T});
+    else
+        st = check_ptrs({dS0}, {S0, dS_T});
+    if (st != GDN2_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)N * H * Dk * Dv * sizeof(float);
+    if (total_T == 0) {
+        if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
+    }
+    gdn2::Problem p = make_problem(N, total_T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    p.cu_seqlens = cu_seqlens;
+    const size_t need = gdn2::bwd_workspace_bytes(dt, p);
+    if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
     return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s));
 }
@@ -194,7 +267,7 @@ gdn2_status gdn2_sync_status(void *stream)
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_gdn2_status, &zero, sizeof(int)) != cudaSuccess) return GDN2_ERR_CUDA;
-        return GDN2_ERR_TIMEOUT;
+        return v == gdn2::kStatusBadSeqlens ? GDN2_ERR_SEQLENS : GDN2_ERR_TIMEOUT;
     }
     return GDN2_OK;
 }

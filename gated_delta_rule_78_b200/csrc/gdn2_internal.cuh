@@ -14,6 +14,7 @@ constexpr int kChunk = 64;  // tokens per chunk
 
 // Device status word values (written by kernels, read by gdn2_sync_status).
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadSeqlens = 2;  // cu_seqlens not non-decreasing inside [0, total_T]
 
 template <typename T> __device__ __forceinline__ float to_f(T x);
 template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
@@ -25,12 +26,71 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 
 // Problem description handed from the C ABI layer to the launchers.  All
 // pointers are device pointers; layouts as in gdn2.h.
+//
+// Fixed length (cu_seqlens == null): B sequences of T tokens, tensors [B, T, H, D].
+// Variable length: B sequences packed into T rows, tensors [T, H, D]; sequence n is rows
+// cu_seqlens[n] .. cu_seqlens[n+1].  chunk_off (device, B + 1 entries, variable length
+// only, filled by launch_chunk_offsets) is the exclusive prefix sum of the sequences'
+// chunk counts; per-chunk workspace lists of (sequence n, head h) start at
+// chunk_off[n] * H + h * nchunks(n), which for fixed length is (n * H + h) * nchunks.
 struct Problem {
     int B, T, H, D;  // Dk == Dv == D
     const void *q, *k, *v, *b, *w;
     const float *g;   // log alpha
     const float *S0;  // may be null
+    const int *cu_seqlens = nullptr;
+    const int *chunk_off = nullptr;
 };
+
+// rows of the token tensors
+__host__ __device__ inline size_t token_rows(const Problem &p)
+{
+    return p.cu_seqlens ? (size_t)p.T : (size_t)p.B * p.T;
+}
+// upper bound of the total number of chunks over all sequences (per head)
+__host__ __device__ inline size_t chunk_bound(const Problem &p)
+{
+    return p.cu_seqlens ? (size_t)(p.T + kChunk - 1) / kChunk + p.B : (size_t)p.B * ((p.T + kChunk - 1) / kChunk);
+}
+
+struct SeqSpan {
+    int bos, len;  // first row and token count of the sequence
+};
+// Span of sequence n; len = -1 marks invalid cu_seqlens (the caller reports it).
+__device__ __forceinline__ SeqSpan seq_span(const Problem &p, int n)
+{
+    if (!p.cu_seqlens) return {n * p.T, p.T};
+    const int b0 = p.cu_seqlens[n], b1 = p.cu_seqlens[n + 1];
+    if (b0 < 0 || b1 < b0 || b1 > p.T) return {0, -1};
+    return {b0, b1 - b0};
+}
+__device__ __forceinline__ int seq_chunks(int len) { return (len + kChunk - 1) / kChunk; }
+// first chunk (over all sequences) of sequence n
+__device__ __forceinline__ size_t chunk_first(const Problem &p, int n)
+{
+    return p.chunk_off ? (size_t)p.chunk_off[n] : (size_t)n * seq_chunks(p.T);
+}
+// index of chunk ci of (sequence n, head h) in a per-chunk workspace list
+__device__ __forceinline__ size_t chunk_slot(const Problem &p, int n, int h, int nch, int ci)
+{
+    return chunk_first(p, n) * p.H + (size_t)h * nch + ci;
+}
+// index of boundary state ci (0 .. nch) of (sequence n, head h) in a per-boundary list
+__device__ __forceinline__ size_t bound_slot(const Problem &p, int n, int h, int nch, int ci)
+{
+    return (chunk_first(p, n) + n) * p.H + (size_t)h * (nch + 1) + ci;
+}
+// offset of token row t of sequence span sp, head h, in a [rows, H, D] tensor
+__device__ __forceinline__ size_t tok_row(const Problem &p, const SeqSpan &sp, int h, int t)
+{
+    return ((size_t)(sp.bos + t) * p.H + h) * p.D;
+}
+
+// Variable length: checks cu_seqlens (sets the status word to kStatusBadSeqlens if it is
+// not non-decreasing inside [0, total_rows]) and writes chunk_off (n_seqs + 1 ints) when
+// chunk_off is non-null.  One small launch.
+cudaError_t launch_chunk_offsets(const int *cu_seqlens, int n_seqs, int total_rows, int *chunk_off, int *status,
+                                 cudaStream_t s);
 
 // forward (SIMT fp32 FMA path).  `states`, when non-null, receives the state at
 // the start of every chunk: [B*H][nchunks][D][D] fp32.  `o` may be null (states only).
@@ -56,15 +116,19 @@ struct BwdOut {
     void *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
 };
+// bytes reserved at the front of a variable-length workspace for chunk_off (256-aligned)
+inline size_t varlen_offsets_bytes(int n_seqs) { return ((size_t)(n_seqs + 1) * sizeof(int) + 255) / 256 * 256; }
+
 // Backward workspace bytes (depends on the path: bf16 with D = 128 runs on the
-// tensor cores, everything else on the fp32 FMA kernels).
-size_t bwd_workspace_bytes(gdn2_dtype dt, int B, int T, int H, int D);
+// tensor cores, everything else on the fp32 FMA kernels).  Only the sizes and
+// whether cu_seqlens is set are read from p.
+size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p);
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
                        const BwdOut &out, void *ws, cudaStream_t s);
 
 // tensor-core backward (bf16, D = 128): the forward in states mode, then the prep,
 // chain and gradient kernels
-size_t bwd_tc_workspace_bytes(int B, int T, int H);
+size_t bwd_tc_workspace_bytes(const Problem &p);
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
                           int *status, cudaStream_t s);
 

@@ -83,7 +83,10 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(
         if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
         return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
     }
-    if (gdn2::bwd_workspace_bytes(dt, B, T, H, Dk) > kScratchBytes) return GDN2_ERR_TOO_LARGE;
+    gdn2::Problem p;
+    p.B = B; p.T = T; p.H = H; p.D = Dk;
+    p.q = q; p.k = k; p.v = v; p.b = b; p.w = w; p.g = log_alpha; p.S0 = S0;
+    if (gdn2::bwd_workspace_bytes(dt, p) > kScratchBytes) return GDN2_ERR_TOO_LARGE;
 
     void *scratch = nullptr;
     const gdn2_status st = scratch_address(&scratch);
@@ -91,9 +94,6 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(
     // Every scratch byte the kernels read is written earlier in the same call
     // (chunk-start states, per-chunk matrices, per-slice partial gradients), so
     // nothing left by an earlier call needs clearing.
-    gdn2::Problem p;
-    p.B = B; p.T = T; p.H = H; p.D = Dk;
-    p.q = q; p.k = k; p.v = v; p.b = b; p.w = w; p.g = log_alpha; p.S0 = S0;
     gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
     return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, scratch, s));
 }

@@ -28,8 +28,8 @@
  *    element type given by `dt` (fp32 or bf16).  log_alpha and its gradient
  *    are [B, T, H, Dk] fp32 always.  States S0, S_T, dS_T, dS0 are
  *    [B, H, Dk, Dv] fp32 always (d_v contiguous).
- *  - v1 shape contract: Dk == Dv in {64, 128}; B, H >= 1; T >= 0 (any T;
- *    T = 0 copies S0 to S_T).  Other shapes give GDN2_ERR_UNSUPPORTED.
+ *  - v1 shape contract: Dk == Dv in {64, 128}; B >= 1; 1 <= H <= 65535; T >= 0
+ *    (any T; T = 0 copies S0 to S_T).  Other shapes give GDN2_ERR_UNSUPPORTED.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *    are asynchronous on it: a GDN2_OK return means the arguments were valid
  *    and the kernels were enqueued.  An error raised inside a kernel (a
@@ -64,8 +64,9 @@ typedef enum {
     GDN2_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch error, no device, ...) */
     GDN2_ERR_TIMEOUT = -7,     /* a kernel's bounded wait gave up (reported by gdn2_sync_status) */
     GDN2_ERR_UNSUPPORTED = -8, /* valid but outside the v1 shape contract */
-    GDN2_ERR_TOO_LARGE = -9    /* needs more scratch than GDN2_NOALLOC_MAX_SCRATCH_BYTES
+    GDN2_ERR_TOO_LARGE = -9,   /* needs more scratch than GDN2_NOALLOC_MAX_SCRATCH_BYTES
                                   (gdn2_chunk_bwd_noalloc only) */
+    GDN2_ERR_SEQLENS = -10     /* a kernel found cu_seqlens invalid (reported by gdn2_sync_status) */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
@@ -153,7 +154,33 @@ GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(gdn2_dtype dt, int B, int T, int H, 
                            void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
                            float *dS0, void *stream);
 
-/* Workspace bytes for which = 0 (gdn2_chunk_fwd) or 1 (gdn2_chunk_bwd);
+/*
+ * Variable-length batches: N sequences packed along the token axis.
+ *   cu_seqlens: DEVICE int32 [N + 1] with 0 = c_0 <= c_1 <= ... <= c_N = total_T;
+ *               sequence n is token rows c_n .. c_{n+1} (empty sequences allowed).
+ *   q, k, b, log_alpha: [total_T, H, Dk]; v, w, o (and gradients): [total_T, H, Dv];
+ *   S0, S_T, dS_T, dS0: [N, H, Dk, Dv] fp32, one state per sequence and head.
+ * Every sequence runs the recurrence of gdn2_chunk_fwd / gdn2_chunk_bwd on its own,
+ * from its own S0.  cu_seqlens lives on the device, so the library cannot check it
+ * before launching: a kernel that finds it invalid skips the affected sequences and
+ * records GDN2_ERR_SEQLENS for gdn2_sync_status.  When total_T == 0 it is not read.
+ * Workspace: gdn2_workspace_size(2, ...) (forward, 0) and gdn2_workspace_size(3, ...)
+ * (backward), with B = N and T = total_T.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int Dk, int Dv,
+                           const int *cu_seqlens, const void *q, const void *k, const void *v,
+                           const float *log_alpha, const void *b, const void *w, const float *S0,
+                           void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream);
+
+GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int Dk, int Dv,
+                           const int *cu_seqlens, const void *q, const void *k, const void *v,
+                           const float *log_alpha, const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream);
+
+/* Workspace bytes for which = 0 (gdn2_chunk_fwd), 1 (gdn2_chunk_bwd),
+ * 2 (gdn2_chunk_fwd_varlen) or 3 (gdn2_chunk_bwd_varlen, B = N, T = total_T);
  * 0 for invalid or unsupported arguments. */
 GDN2_API size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv);
 
@@ -162,7 +189,8 @@ GDN2_API const char *gdn2_strerror(gdn2_status status);
 
 /* Synchronises `stream`, then returns and clears the current device's kernel
  * status word: GDN2_ERR_TIMEOUT if a kernel gave up a bounded wait since the
- * last check, GDN2_ERR_CUDA if the stream reported an error, else GDN2_OK. */
+ * last check, GDN2_ERR_SEQLENS if a kernel found cu_seqlens invalid,
+ * GDN2_ERR_CUDA if the stream reported an error, else GDN2_OK. */
 GDN2_API gdn2_status gdn2_sync_status(void *stream);
 
 #ifdef __cplusplus

@@ -79,6 +79,37 @@ def test_invalid_arguments_return_status(lib):
     assert bwd(lib, ws=MIS) == -4
 
 
+def fwd_v(lib, dt=BF16, N=2, T=64, H=1, Dk=128, cu=P, q=P):
+    return lib.gdn2_chunk_fwd_varlen(dt, N, T, H, Dk, Dk, cu, q, P, P, P, P, P, NUL, P, NUL, NUL, 0, S)
+
+
+def bwd_v(lib, dt=BF16, N=2, T=64, H=1, Dk=128, cu=P, ws=P, ws_bytes=1 << 40):
+    return lib.gdn2_chunk_bwd_varlen(dt, N, T, H, Dk, Dk, cu, P, P, P, P, P, P, NUL, P, NUL,
+                                     P, P, P, P, P, P, P, ws, ws_bytes, S)
+
+
+def test_varlen_invalid_arguments_return_status(lib):
+    assert fwd_v(lib, cu=NUL) == -1
+    assert fwd_v(lib, cu=ctypes.c_void_p(0x7F0000000002)) == -4
+    assert fwd_v(lib, q=NUL) == -1
+    assert fwd_v(lib, N=0) == -2
+    assert fwd_v(lib, Dk=96) == -8
+    assert fwd_v(lib, H=70000) == -8
+    assert bwd_v(lib, cu=NUL) == -1
+    assert bwd_v(lib, ws=NUL) == -5
+    assert bwd_v(lib, ws_bytes=16) == -5
+
+
+def test_varlen_workspace_size(lib):
+    assert lib.gdn2_workspace_size(2, BF16, 4, 1000, 16, 128, 128) == 0
+    fixed = lib.gdn2_workspace_size(1, BF16, 4, 1024, 16, 128, 128)
+    packed = lib.gdn2_workspace_size(3, BF16, 4, 4096, 16, 128, 128)
+    # four sequences in 4096 packed rows: room for 64 + 4 chunks per head instead of 4 x 16
+    assert fixed < packed < fixed * 1.1
+    assert lib.gdn2_workspace_size(3, F32, 4, 4096, 16, 64, 64) > 0
+    assert lib.gdn2_workspace_size(3, BF16, 4, 0, 16, 128, 128) == 0
+
+
 def test_workspace_size(lib):
     assert lib.gdn2_workspace_size(0, BF16, 8, 4096, 16, 128, 128) == 0
     need = lib.gdn2_workspace_size(1, BF16, 8, 4096, 16, 128, 128)
