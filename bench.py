@@ -15,7 +15,9 @@ steps) and the roofline fraction of each, plus:
 * `cpu_baseline`: the fp64 oracle timed on a bounded sample on the host cores;
 * `clocks`: SM clock and throttle reasons sampled during the timed regions;
 * `sweep`: forward throughput at 65,536 tokens per call for T = 2K ... 32K (B = 32 ... 2),
-  with the number of (batch, head) CTAs each shape gives the 148 SMs.
+  with the number of (batch, head) CTAs each shape gives the 148 SMs;
+* `varlen`: the headline's 32,768 tokens as 16 packed sequences of log-uniform length
+  (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 independent (batch, head) sequences; there is no collective on the data path
@@ -35,6 +37,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -357,6 +360,37 @@ def run_ours(args):
             "launches_per_step": 1}
         del steps_in
     if "fwd" in parts and not args.no_sweep:
+        # ---- variable length: the same 32,768 tokens as the headline, as 16 packed sequences whose
+        #      lengths are log-uniform in [256, 8192] (seeded), forward and backward
+        rng = np.random.default_rng(7)
+        lens = np.exp(rng.uniform(np.log(256), np.log(8192), 16))
+        lens = np.maximum(1, np.round(lens / lens.sum() * tokens)).astype(np.int64)
+        lens[-1] += tokens - lens.sum()
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+        xv = make_inputs(1, tokens, H, D, D, dtype=w["dtype"], seed=rank_seed(rank) + 17, device=str(dev), with_do=True)
+        S0v = torch.zeros(len(lens), H, D, D, device=dev)
+        ov = torch.empty_like(xv["v"][0])
+        Sv = torch.empty_like(S0v)
+
+        def fwd_v():
+            g.gdn2_chunk_fwd_varlen(xv["q"], xv["k"], xv["v"], xv["log_alpha"], xv["b"], xv["w"], cu, S0v, o=ov, S_T=Sv)
+
+        ms_v = time_region(fwd_v, 10, 3, stream) / 10
+        wsv = torch.empty(g.gdn2_workspace_size(3, xv["q"].dtype, len(lens), tokens, H, D, D), dtype=torch.uint8,
+                          device=dev)
+
+        def bwd_v():
+            g.gdn2_chunk_bwd_varlen(xv["q"], xv["k"], xv["v"], xv["log_alpha"], xv["b"], xv["w"], cu, S0v, xv["do"],
+                                    workspace=wsv)
+
+        ms_vb = time_region(bwd_v, 5, 3, stream) / 5
+        assert g.gdn2_sync_status() == 0
+        extras["varlen"] = {"sequences": len(lens), "lengths": [int(v) for v in lens], "tokens": tokens,
+                            "fwd_ms": round(ms_v, 4), "fwd_tokens_per_s": round(job_rate(tokens, world, ms_v), 1),
+                            "fwd_hbm_frac": round(fwd_bytes(1, tokens, H, D) / (ms_v * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                            "bwd_ms": round(ms_vb, 4)}
+        del xv, ov, Sv, wsv
+
         # ---- sequence-length sweep at a fixed 65,536 tokens per call (one forward per step)
         sweep = {}
         for name in ("sweep_2k", "sweep_4k", "sweep_8k", "sweep_16k", "sweep_32k"):
