@@ -23,7 +23,10 @@ STATUS_NAMES = {0: "GDN2_OK", -1: "GDN2_ERR_NULL", -2: "GDN2_ERR_SHAPE", -3: "GD
 GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
            "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
-           "gdn2_chunk_bwd_varlen")
+           "gdn2_chunk_bwd_varlen", "gdn2_chunk_fwd_gated", "gdn2_chunk_bwd_gated", "gdn2_decode_step_gated",
+           "gdn2_workspace_size_gated")
+# gate layout flags (gdn2_gate_flags in include/gdn2.h)
+DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE = 1, 2, 4, 8, 16, 32
 # Size of the library's static scratch array used by gdn2_chunk_bwd_noalloc
 # (GDN2_NOALLOC_MAX_SCRATCH_BYTES in include/gdn2.h).
 NOALLOC_MAX_SCRATCH_BYTES = 32 << 20
@@ -60,6 +63,14 @@ def load(path: str | None = None):
     lib.gdn2_chunk_fwd_varlen.restype = i
     lib.gdn2_chunk_bwd_varlen.argtypes = [i] * 6 + [vp] * 18 + [sz, vp]
     lib.gdn2_chunk_bwd_varlen.restype = i
+    lib.gdn2_chunk_fwd_gated.argtypes = [i] * 7 + [vp] * 10 + [sz, vp]
+    lib.gdn2_chunk_fwd_gated.restype = i
+    lib.gdn2_chunk_bwd_gated.argtypes = [i] * 7 + [vp] * 17 + [sz, vp]
+    lib.gdn2_chunk_bwd_gated.restype = i
+    lib.gdn2_decode_step_gated.argtypes = [i] * 6 + [vp] * 9 + [sz, vp]
+    lib.gdn2_decode_step_gated.restype = i
+    lib.gdn2_workspace_size_gated.argtypes = [i] * 8
+    lib.gdn2_workspace_size_gated.restype = sz
     lib.gdn2_workspace_size.argtypes = [i] * 7
     lib.gdn2_workspace_size.restype = sz
     lib.gdn2_strerror.argtypes = [i]
@@ -270,6 +281,85 @@ def gdn2_chunk_bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, S0, d_o, dS_T=No
                                      _stream(stream))
     _check("gdn2_chunk_bwd_varlen", st)
     return out
+
+
+def gdn2_workspace_size_gated(which: int, flags: int, dtype: torch.dtype, B: int, T: int, H: int, Dk: int,
+                              Dv: int) -> int:
+    dt = GDN2_F32 if dtype == torch.float32 else GDN2_BF16
+    return int(raw().gdn2_workspace_size_gated(which, flags, dt, B, T, H, Dk, Dv))
+
+
+def _ws(workspace, nbytes, device):
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, (0 if workspace is None else workspace.numel() * workspace.element_size())
+
+
+def gdn2_chunk_fwd_gated(q, k, v, log_alpha, b, w, S0=None, *, flags, o=None, S_T=None, want_state=True,
+                         workspace=None, stream=None):
+    """Forward with gate layouts given by `flags` (scalar gates are [B, T, H]; absent ones may be None)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_contig(n, t, q.dtype)
+    for n, t in (("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    if o is None:
+        o = torch.empty(B, T, H, Dv, dtype=q.dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)
+    ws, nb = _ws(workspace, gdn2_workspace_size_gated(0, flags, q.dtype, B, T, H, Dk, Dv), q.device)
+    st = raw().gdn2_chunk_fwd_gated(flags, dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                    _p(S0), _p(o), _p(S_T), _p(ws), nb, _stream(stream))
+    _check("gdn2_chunk_fwd_gated", st)
+    return o, S_T
+
+
+def gdn2_chunk_bwd_gated(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, flags, workspace=None, out=None,
+                         stream=None):
+    """Backward with gate layouts given by `flags`; gate gradients come back in the gates' layouts
+    (None for absent gates)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("d_o", d_o), ("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    _cuda_contig("dS_T", dS_T, torch.float32)
+    if out is None:
+        out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+               "dlog_alpha": None if log_alpha is None else torch.empty_like(log_alpha),
+               "db": None if b is None else torch.empty_like(b), "dw": None if w is None else torch.empty_like(w),
+               "dS0": torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)}
+    ws, nb = _ws(workspace, gdn2_workspace_size_gated(1, flags, q.dtype, B, T, H, Dk, Dv), q.device)
+    st = raw().gdn2_chunk_bwd_gated(flags, dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                    _p(S0), _p(d_o), _p(dS_T), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                                    _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]), _p(out["dS0"]), _p(ws), nb,
+                                    _stream(stream))
+    _check("gdn2_chunk_bwd_gated", st)
+    return out
+
+
+def gdn2_decode_step_gated(q, k, v, log_alpha, b, w, S, *, flags, o=None, workspace=None, stream=None):
+    """Decode step with gate layouts given by `flags` (scalar gates are [N, H])."""
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S", S, torch.float32)
+    if o is None:
+        o = torch.empty(N, H, Dv, dtype=q.dtype, device=q.device)
+    ws, nb = _ws(workspace, gdn2_workspace_size_gated(2, flags, q.dtype, N, 1, H, Dk, Dv), q.device)
+    st = raw().gdn2_decode_step_gated(flags, dt, N, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                      _p(S), _p(o), _p(ws), nb, _stream(stream))
+    _check("gdn2_decode_step_gated", st)
+    return o
 
 
 def gdn2_sync_status(stream=None) -> int:

@@ -104,6 +104,73 @@ gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, 
     return from_cuda(gdn2::launch_fwd_simt(dt, p, o, S_T, nullptr, s));
 }
 
+
+// ---- gate layouts (the gdn2_*_gated entry points)
+// gate i: 0 = log decay, 1 = erase gate b, 2 = write gate w
+bool gate_scalar(int flags, int i) { return (flags >> i) & 1; }
+bool gate_none(int flags, int i) { return (flags >> (3 + i)) & 1; }
+bool gate_full(int flags, int i) { return !gate_scalar(flags, i) && !gate_none(flags, i); }
+
+gdn2_status check_gate_flags(int flags)
+{
+    if (flags & ~0x3F) return GDN2_ERR_UNSUPPORTED;
+    for (int i = 0; i < 3; ++i)
+        if (gate_scalar(flags, i) && gate_none(flags, i)) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// [expanded g | b | w] [full-size gradients of dg | db | dw (backward)] [core workspace]
+struct GatedWs {
+    size_t off[3], grad[3], core, total;
+};
+GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes)
+{
+    GatedWs l;
+    const size_t n = rows * H * D;
+    const size_t es[3] = {4, dt == GDN2_F32 ? 4u : 2u, dt == GDN2_F32 ? 4u : 2u};
+    size_t off = 0;
+    for (int i = 0; i < 3; ++i) {
+        l.off[i] = off;
+        if (!gate_full(flags, i)) off += round256(n * es[i]);
+    }
+    for (int i = 0; i < 3; ++i) {
+        l.grad[i] = off;
+        if (bwd && !gate_full(flags, i)) off += round256(n * es[i]);
+    }
+    l.core = off;
+    l.total = off + core_bytes;
+    return l;
+}
+
+// Broadcast the non-per-channel gates into the workspace; gp[i] is replaced by the full
+// tensor's address.  Absent gates are 0 (log decay) or 1 (b, w).
+gdn2_status expand_gates(int flags, gdn2_dtype dt, const GatedWs &l, char *ws, size_t rows, int H, int D,
+                         const void *gp[3], cudaStream_t s)
+{
+    for (int i = 0; i < 3; ++i) {
+        if (gate_full(flags, i)) continue;
+        void *dst = ws + l.off[i];
+        const bool fp32 = (i == 0) || dt == GDN2_F32;
+        cudaError_t e = gdn2::launch_expand_gate(fp32, gate_none(flags, i) ? nullptr : gp[i], dst, rows * H, D,
+                                                 i == 0 ? 0.f : 1.f, s);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        gp[i] = dst;
+    }
+    return GDN2_OK;
+}
+
+gdn2_status check_gate_ptrs(int flags, const void *g, const void *b, const void *w)
+{
+    const void *gp[3] = {g, b, w};
+    for (int i = 0; i < 3; ++i) {
+        if (gate_none(flags, i)) continue;
+        if (!gp[i]) return GDN2_ERR_NULL;
+        if (!aligned16(gp[i])) return GDN2_ERR_ALIGN;
+    }
+    return GDN2_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -256,6 +323,102 @@ gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int 
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
     return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s));
+}
+
+size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
+{
+    if (check_gate_flags(flags) != GDN2_OK) return 0;
+    if (which == 2) {  // decode: B sequences of one token
+        if (check_sizes(dt, B, 1, H, Dk, Dv) != GDN2_OK) return 0;
+        return gated_ws(false, flags, dt, (size_t)B, H, Dk, 0).total;
+    }
+    if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK || T == 0 || (which != 0 && which != 1)) return 0;
+    const size_t core = which == 1 ? gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr,
+                                                                                nullptr, nullptr, nullptr, nullptr))
+                                   : 0;
+    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core).total;
+}
+
+gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                                 const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                                 const float *S0, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_gate_flags(flags);
+    if (st != GDN2_OK) return st;
+    if ((st = check_sizes(dt, B, T, H, Dk, Dv)) != GDN2_OK) return st;
+    if (T == 0) return gdn2_chunk_fwd(dt, B, 0, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, o, S_T, nullptr, 0, stream);
+    if ((st = check_ptrs({q, k, v, o}, {S0, S_T})) != GDN2_OK) return st;
+    if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0);
+    if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
+    if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    const void *gp[3] = {log_alpha, b, w};
+    if ((st = expand_gates(flags, dt, l, static_cast<char *>(workspace), (size_t)B * T, H, Dk, gp, s)) != GDN2_OK)
+        return st;
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S0);
+    return run_fwd(dt, p, o, S_T, s);
+}
+
+gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                                 const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                                 const float *S0, const void *d_o, const float *dS_T, void *dq, void *dk, void *dv,
+                                 float *dlog_alpha, void *db, void *dw, float *dS0, void *workspace, size_t ws_bytes,
+                                 void *stream)
+{
+    gdn2_status st = check_gate_flags(flags);
+    if (st != GDN2_OK) return st;
+    if ((st = check_sizes(dt, B, T, H, Dk, Dv)) != GDN2_OK) return st;
+    if (T == 0)
+        return gdn2_chunk_bwd(dt, B, 0, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, d_o, dS_T, dq, dk, dv, dlog_alpha, db,
+                              dw, dS0, nullptr, 0, stream);
+    if ((st = check_ptrs({q, k, v, d_o, dq, dk, dv, dS0}, {S0, dS_T})) != GDN2_OK) return st;
+    if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
+    if ((st = check_gate_ptrs(flags, dlog_alpha, db, dw)) != GDN2_OK) return st;
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p));
+    if (!workspace || ws_bytes < l.total) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *ws = static_cast<char *>(workspace);
+    const void *gp[3] = {log_alpha, b, w};
+    if ((st = expand_gates(flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s)) != GDN2_OK) return st;
+    p.g = static_cast<const float *>(gp[0]);
+    p.b = gp[1];
+    p.w = gp[2];
+    void *grads[3] = {dlog_alpha, db, dw};
+    for (int i = 0; i < 3; ++i)
+        if (!gate_full(flags, i)) grads[i] = ws + l.grad[i];  // full-size gradient, reduced below
+    gdn2::BwdOut out{dq, dk, dv, grads[1], grads[2], static_cast<float *>(grads[0]), dS0};
+    if (gdn2::launch_bwd(dt, p, d_o, dS_T, out, ws + l.core, s) != cudaSuccess) return GDN2_ERR_CUDA;
+    void *user[3] = {dlog_alpha, db, dw};
+    for (int i = 0; i < 3; ++i) {
+        if (!gate_scalar(flags, i)) continue;
+        const bool fp32 = (i == 0) || dt == GDN2_F32;
+        if (gdn2::launch_channel_sum(fp32, grads[i], user[i], (size_t)B * T * H, Dk, s) != cudaSuccess)
+            return GDN2_ERR_CUDA;
+    }
+    return GDN2_OK;
+}
+
+gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int H, int Dk, int Dv, const void *q,
+                                   const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                                   float *S, void *o, void *workspace, size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_gate_flags(flags);
+    if (st != GDN2_OK) return st;
+    if ((st = check_sizes(dt, N, 1, H, Dk, Dv)) != GDN2_OK) return st;
+    if ((st = check_ptrs({q, k, v, S, o}, {})) != GDN2_OK) return st;
+    if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)N, H, Dk, 0);
+    if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
+    if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    const void *gp[3] = {log_alpha, b, w};
+    if ((st = expand_gates(flags, dt, l, static_cast<char *>(workspace), (size_t)N, H, Dk, gp, s)) != GDN2_OK)
+        return st;
+    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, q, k, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S, o,
+                                         s));
 }
 
 gdn2_status gdn2_sync_status(void *stream)

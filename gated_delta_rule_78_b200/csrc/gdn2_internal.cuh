@@ -132,6 +132,12 @@ size_t bwd_tc_workspace_bytes(const Problem &p);
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
                           int *status, cudaStream_t s);
 
+// Gate layouts (gates.cu): fill dst ([n_rows, D]) with src[row] (a per-row scalar) or,
+// when src is null, with `fill`; and sum src ([n_rows, D]) over D into dst ([n_rows]).
+// fp32 selects float, otherwise bf16.
+cudaError_t launch_expand_gate(bool fp32, const void *src, void *dst, size_t n_rows, int D, float fill, cudaStream_t s);
+cudaError_t launch_channel_sum(bool fp32, const void *src, void *dst, size_t n_rows, int D, cudaStream_t s);
+
 // device address of the library's kernel status word on the current device
 int *status_word();
 

@@ -179,6 +179,54 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
                            void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
                            float *dS0, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * Gate layouts.  The calls above take every gate with one value per channel.  The
+ * *_gated calls take a flags word that gives each gate one of three layouts:
+ *   per channel (no flag): as above, [B, T, H, D];
+ *   scalar (GDN2_*_SCALAR): one value per token and head, [B, T, H] (decode:
+ *     [N, H]), used for every channel;
+ *   absent (GDN2_*_NONE): the pointer is ignored; b and w are 1 and log_alpha is 0.
+ * With b = w = beta scalar the recurrence is KDA; with a scalar decay as well it
+ * is Gated DeltaNet; with no decay and scalar b = w it is DeltaNet (the
+ * needhelp.icu write-up's generalisation hierarchy).  Absent b or w gives the
+ * write-only and erase-only ablations of the aixai.ru post ("Абляции").
+ * The results are identical to the plain calls made with the gates broadcast to
+ * per-channel tensors: the library broadcasts them into the workspace and runs the
+ * same kernels.  In the backward the gradient of a scalar gate is the sum of the
+ * per-channel gradients over the channels.  An absent gate's gradient pointer is
+ * ignored (NULL allowed).  Flags outside the six below, or scalar and absent set
+ * for one gate, give GDN2_ERR_UNSUPPORTED.
+ * Workspace: gdn2_workspace_size_gated(which, flags, ...) with which = 0 (forward),
+ * 1 (backward), 2 (decode; B = N, T ignored).  Fixed-length batches only.
+ */
+typedef enum {
+    GDN2_DECAY_SCALAR = 1,
+    GDN2_ERASE_SCALAR = 2,
+    GDN2_WRITE_SCALAR = 4,
+    GDN2_DECAY_NONE = 8,
+    GDN2_ERASE_NONE = 16,
+    GDN2_WRITE_NONE = 32
+} gdn2_gate_flags;
+
+GDN2_API gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream);
+
+GDN2_API gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream);
+
+GDN2_API gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, float *S, void *o,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+GDN2_API size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv);
+
 /* Workspace bytes for which = 0 (gdn2_chunk_fwd), 1 (gdn2_chunk_bwd),
  * 2 (gdn2_chunk_fwd_varlen) or 3 (gdn2_chunk_bwd_varlen, B = N, T = total_T);
  * 0 for invalid or unsupported arguments. */

@@ -110,6 +110,26 @@ def test_varlen_workspace_size(lib):
     assert lib.gdn2_workspace_size(3, BF16, 4, 0, 16, 128, 128) == 0
 
 
+def fwd_g(lib, flags, g=P, b=P, w=P, ws=P, ws_bytes=1 << 40):
+    return lib.gdn2_chunk_fwd_gated(flags, BF16, 1, 64, 1, 128, 128, P, P, P, g, b, w, NUL, P, NUL, ws, ws_bytes, S)
+
+
+def test_gated_flags_and_workspace(lib):
+    assert fwd_g(lib, 64) == -8                       # unknown flag bit
+    assert fwd_g(lib, g.ERASE_SCALAR | g.ERASE_NONE) == -8  # scalar and absent for one gate
+    assert fwd_g(lib, g.ERASE_SCALAR, b=NUL) == -1     # a scalar gate needs its tensor
+    assert fwd_g(lib, g.ERASE_SCALAR, ws=NUL) == -5    # and a workspace to broadcast it into
+    # per-channel gates need no workspace in the forward
+    assert lib.gdn2_workspace_size_gated(0, 0, BF16, 2, 128, 4, 128, 128) == 0
+    one = 2 * 128 * 4 * 128 * 2                        # one broadcast bf16 gate
+    assert lib.gdn2_workspace_size_gated(0, g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == one
+    assert lib.gdn2_workspace_size_gated(0, g.DECAY_NONE, BF16, 2, 128, 4, 128, 128) == 2 * one
+    plain = lib.gdn2_workspace_size(1, BF16, 2, 128, 4, 128, 128)
+    assert lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR | g.WRITE_SCALAR, BF16, 2, 128, 4, 128, 128) == plain + 4 * one
+    assert lib.gdn2_workspace_size_gated(2, g.ERASE_SCALAR, BF16, 8, 0, 4, 128, 128) == 8 * 4 * 128 * 2
+    assert lib.gdn2_workspace_size_gated(0, 64, BF16, 2, 128, 4, 128, 128) == 0
+
+
 def test_workspace_size(lib):
     assert lib.gdn2_workspace_size(0, BF16, 8, 4096, 16, 128, 128) == 0
     need = lib.gdn2_workspace_size(1, BF16, 8, 4096, 16, 128, 128)

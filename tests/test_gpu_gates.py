@@ -1,0 +1,121 @@
+"""Gate layouts other than one value per channel (per-(token, head) scalars, absent gates).
+
+The gated calls must give exactly what the plain calls give on the same gates broadcast to
+per-channel tensors; scalar-gate gradients are the per-channel gradients summed over the
+channels.  One KDA-shaped and one Gated-DeltaNet-shaped case are also checked against the
+separately written KDA / Gated DeltaNet recurrences of the oracle's checks module."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_78_b200 as g
+from oracle import checks
+from parity import assert_close
+from synthetic_inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+KDA = g.ERASE_SCALAR | g.WRITE_SCALAR
+GDN = KDA | g.DECAY_SCALAR
+DELTANET = g.DECAY_NONE | g.ERASE_SCALAR | g.WRITE_SCALAR
+ERASE_ONLY = g.WRITE_NONE            # per-channel b, w = 1
+WRITE_ONLY = g.ERASE_NONE            # per-channel w, b = 1
+MIXED = g.DECAY_SCALAR | g.ERASE_NONE | g.WRITE_SCALAR
+CASES = [("kda", KDA), ("gdn", GDN), ("deltanet", DELTANET), ("erase_only", ERASE_ONLY),
+         ("write_only", WRITE_ONLY), ("mixed", MIXED)]
+
+
+def gated_inputs(B, T, H, D, dtype, flags, seed):
+    """Per-channel inputs plus the gates in the layouts `flags` asks for, and their broadcasts."""
+    x = make_inputs(B, T, H, D, D, dtype=dtype, seed=seed, with_do=True)
+    gen = torch.Generator().manual_seed(seed + 100)
+    tdt = x["q"].dtype
+    gates, full = {}, {}
+    for i, name in enumerate(("log_alpha", "b", "w")):
+        if flags & (1 << i):  # scalar per (token, head)
+            if name == "log_alpha":
+                sc = -torch.nn.functional.softplus(torch.randn(B, T, H, generator=gen) - 3.0)
+            else:
+                sc = torch.sigmoid(torch.randn(B, T, H, generator=gen)).to(tdt)
+            gates[name] = sc
+            full[name] = sc[..., None].expand(B, T, H, D).contiguous()
+        elif flags & (8 << i):  # absent
+            gates[name] = None
+            full[name] = (torch.zeros(B, T, H, D) if name == "log_alpha" else torch.ones(B, T, H, D, dtype=tdt))
+        else:
+            gates[name] = x[name]
+            full[name] = x[name]
+    return x, gates, full
+
+
+def dev(t):
+    return None if t is None else t.cuda()
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("name,flags", CASES)
+def test_gated_forward_equals_broadcast_plain_forward(cuda_lib, dtype, D, name, flags):
+    x, gates, full = gated_inputs(2, 130, 2, D, dtype, flags, seed=11)
+    o_g, S_g = g.gdn2_chunk_fwd_gated(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(gates["log_alpha"]),
+                                      dev(gates["b"]), dev(gates["w"]), dev(x["S0"]), flags=flags)
+    o_p, S_p = g.gdn2_chunk_fwd(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(full["log_alpha"]), dev(full["b"]),
+                                dev(full["w"]), dev(x["S0"]))
+    assert g.gdn2_sync_status() == 0
+    assert torch.equal(o_g, o_p), name
+    assert torch.equal(S_g, S_p), name
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("name,flags", CASES)
+def test_gated_backward_equals_broadcast_plain_backward(cuda_lib, dtype, D, name, flags):
+    x, gates, full = gated_inputs(2, 130, 2, D, dtype, flags, seed=13)
+    common = (dev(x["q"]), dev(x["k"]), dev(x["v"]))
+    gr = g.gdn2_chunk_bwd_gated(*common, dev(gates["log_alpha"]), dev(gates["b"]), dev(gates["w"]), dev(x["S0"]),
+                                dev(x["do"]), flags=flags)
+    pr = g.gdn2_chunk_bwd(*common, dev(full["log_alpha"]), dev(full["b"]), dev(full["w"]), dev(x["S0"]), dev(x["do"]))
+    assert g.gdn2_sync_status() == 0
+    for k in ("dq", "dk", "dv", "dS0"):
+        assert torch.equal(gr[k], pr[k]), (name, k)
+    for i, (gk, src) in enumerate((("dlog_alpha", "log_alpha"), ("db", "b"), ("dw", "w"))):
+        if flags & (8 << i):
+            continue
+        if flags & (1 << i):
+            ref = pr[gk].float().sum(-1)
+            assert_close(gr[gk].float(), ref, "f32" if gk == "dlog_alpha" or dtype == "f32" else "bf16",
+                         f"{name} {gk}")
+        else:
+            assert torch.equal(gr[gk], pr[gk]), (name, gk)
+
+
+@pytest.mark.parametrize("name,flags", CASES)
+def test_gated_decode_equals_broadcast_plain_decode(cuda_lib, name, flags):
+    N, H, D = 8, 2, 128
+    x, gates, full = gated_inputs(N, 1, H, D, "bf16", flags, seed=17)
+    sq = lambda t: None if t is None else t[:, 0].contiguous().cuda()
+    S1 = x["S0"].clone().cuda()
+    S2 = x["S0"].clone().cuda()
+    o_g = g.gdn2_decode_step_gated(sq(x["q"]), sq(x["k"]), sq(x["v"]), sq(gates["log_alpha"]), sq(gates["b"]),
+                                   sq(gates["w"]), S1, flags=flags)
+    o_p = g.gdn2_decode_step(sq(x["q"]), sq(x["k"]), sq(x["v"]), sq(full["log_alpha"]), sq(full["b"]),
+                             sq(full["w"]), S2)
+    assert g.gdn2_sync_status() == 0
+    assert torch.equal(o_g, o_p) and torch.equal(S1, S2), name
+
+
+def test_kda_and_gated_deltanet_match_their_own_recurrences(cuda_lib):
+    """Scalar gates against the separately written KDA and Gated DeltaNet recurrences (fp32, d = 64)."""
+    B, T, H, D = 1, 100, 2, 64
+    x, gates, _ = gated_inputs(B, T, H, D, "f32", KDA, seed=19)
+    beta = gates["b"]  # use the erase gate's scalar as beta for both gates
+    o, ST = g.gdn2_chunk_fwd_gated(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["log_alpha"]), dev(beta), dev(beta),
+                                   dev(x["S0"]), flags=KDA)
+    ro, rS = checks.kda_recurrence(x["q"], x["k"], x["v"], x["log_alpha"], beta, x["S0"])
+    assert_close(o, ro, "f32", "kda o")
+    assert_close(ST, rS, "f32", "kda S_T")
+    gs = -torch.nn.functional.softplus(torch.randn(B, T, H, generator=torch.Generator().manual_seed(23)) - 3.0)
+    o, ST = g.gdn2_chunk_fwd_gated(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(gs), dev(beta), dev(beta),
+                                   dev(x["S0"]), flags=GDN)
+    ro, rS = checks.gated_deltanet_recurrence(x["q"], x["k"], x["v"], gs, beta, x["S0"])
+    assert g.gdn2_sync_status() == 0
+    assert_close(o, ro, "f32", "gdn o")
+    assert_close(ST, rS, "f32", "gdn S_T")
