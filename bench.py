@@ -17,7 +17,9 @@ steps) and the roofline fraction of each, plus:
 * `sweep`: forward throughput at 65,536 tokens per call for T = 2K ... 32K (B = 32 ... 2),
   with the number of (batch, head) CTAs each shape gives the 148 SMs;
 * `varlen`: the headline's 32,768 tokens as 16 packed sequences of log-uniform length
-  (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen.
+  (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen;
+* `scalar_decay`: the headline batch with one log decay per (token, head) through
+  gdn2_chunk_fwd_gated (the tensor-core forward's scalar-decay path).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 independent (batch, head) sequences; there is no collective on the data path
@@ -385,6 +387,25 @@ def run_ours(args):
 
         ms_vb = time_region(bwd_v, 5, 3, stream) / 5
         assert g.gdn2_sync_status() == 0
+        # ---- scalar decay (one log alpha per token and head, Gated DeltaNet style), per-channel b, w:
+        #      the tensor-core forward computes one exponential pair per token instead of per channel
+        gsc = -torch.nn.functional.softplus(
+            torch.randn(B, T, H, generator=torch.Generator(device=str(dev)).manual_seed(5), device=dev) - 3.0)
+        wsg = torch.empty(max(16, g.gdn2_workspace_size_gated(0, g.DECAY_SCALAR, x["q"].dtype, B, T, H, D, D)),
+                          dtype=torch.uint8, device=dev)
+
+        def fwd_sd():
+            g.gdn2_chunk_fwd_gated(x["q"], x["k"], x["v"], gsc, x["b"], x["w"], x["S0"], flags=g.DECAY_SCALAR, o=o,
+                                   S_T=ST, workspace=wsg)
+
+        ms_sd = time_region(fwd_sd, 20, 3, stream) / 20
+        assert g.gdn2_sync_status() == 0
+        sd_bytes = fwd_bytes(B, T, H, D) - B * T * H * (4 * D - 4)
+        extras["scalar_decay"] = {"workload": f"B={B}, T={T}, H={H}, d={D}; log alpha [B,T,H], b and w per channel",
+                                  "ms": round(ms_sd, 4), "tokens_per_s": round(job_rate(tokens, world, ms_sd), 1),
+                                  "algorithmic_bytes": sd_bytes,
+                                  "hbm_frac": round(sd_bytes / (ms_sd * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del wsg
         extras["varlen"] = {"sequences": len(lens), "lengths": [int(v) for v in lens], "tokens": tokens,
                             "fwd_ms": round(ms_v, 4), "fwd_tokens_per_s": round(job_rate(tokens, world, ms_v), 1),
                             "fwd_hbm_frac": round(fwd_bytes(1, tokens, H, D) / (ms_v * 1e-3) / 1e9 / pk["hbm_gbs"], 4),

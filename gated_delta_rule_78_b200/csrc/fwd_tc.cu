@@ -96,6 +96,7 @@ struct TcParams {
     int *status;
     const int *cu_seqlens;   // null: B sequences of T tokens; else B packed sequences in T rows
     const int *chunk_off;    // variable length with states only: first chunk of each sequence
+    int g_scalar;            // log alpha is one value per (token, head), [rows, H]: a scalar decay
 };
 
 struct TcMaps {
@@ -111,6 +112,8 @@ __device__ __forceinline__ void named_sync(int id, int count)
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// kGScalar: log alpha is one value per (token, head) (TcParams::g_scalar)
+template <bool kGScalar>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -156,7 +159,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         }
         fence_mbar_init();
         prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.v);
-        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w); prefetch_tmap(&maps.g);
+        prefetch_tmap(&maps.b); prefetch_tmap(&maps.w);
+        if (!kGScalar) prefetch_tmap(&maps.g);  // a scalar decay has no tensor map
         if (p.o) prefetch_tmap(&maps.o);
     }
     if (warp == 0) {
@@ -183,7 +187,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in[bf]);
             tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
         }
-        for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
+        if (!kGScalar)
+            for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
     };
 
     if (is_m) {
@@ -400,11 +405,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
             // log alpha of this warp's 16 tokens x 2 channels, straight from L2
             float2 gv[16];
-            const float *gsrc = p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
+            if (kGScalar) {  // one decay per (token, head), the same for both channels
+                const float *gsrc = p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H + hh;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
-                                          : make_float2(0.f, 0.f);
+                for (int i = 0; i < 16; ++i) {
+                    const float gs = (16 * tg + i < L) ? __ldg(gsrc + (size_t)i * p.H) : 0.f;
+                    gv[i] = make_float2(gs, gs);
+                }
+            } else {
+                const float *gsrc = p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
+                                              : make_float2(0.f, 0.f);
+            }
             if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
 #pragma unroll
@@ -434,8 +448,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     const int t = 16 * tg + i;
                     const uint32_t off = sw128(t, 4 * lane);
                     const float G0 = c0 + gv[i].x, G1 = c1 + gv[i].y;
-                    const float e0 = __expf(G0), e1 = __expf(G1);
-                    const float m0 = __expf(-G0), m1 = __expf(-G1);
+                    const float e0 = __expf(G0), m0 = __expf(-G0);
+                    const float e1 = kGScalar ? e0 : __expf(G1), m1 = kGScalar ? m0 : __expf(-G1);
                     uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
                     uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
                     uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
@@ -575,13 +589,17 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     const int rows = (int)token_rows(pr);  // the maps view every tensor as [rows, H, D]
     if (!make_map(&maps.q, pr.q, false, 1, rows, pr.H) || !make_map(&maps.k, pr.k, false, 1, rows, pr.H) ||
         !make_map(&maps.v, pr.v, false, 1, rows, pr.H) || !make_map(&maps.b, pr.b, false, 1, rows, pr.H) ||
-        !make_map(&maps.w, pr.w, false, 1, rows, pr.H) || !make_map(&maps.g, pr.g, true, 1, rows, pr.H) ||
+        !make_map(&maps.w, pr.w, false, 1, rows, pr.H) || (!pr.g_scalar && !make_map(&maps.g, pr.g, true, 1, rows, pr.H)) ||
         (o && !make_map(&maps.o, o, false, 1, rows, pr.H, true)))
         return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_attr(reinterpret_cast<const void *>(fwd_tc_kernel), (int)SMEM_BYTES);
+    const void *kfn = pr.g_scalar ? reinterpret_cast<const void *>(fwd_tc_kernel<true>)
+                                  : reinterpret_cast<const void *>(fwd_tc_kernel<false>);
+    cudaError_t e = set_smem_attr(kfn, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off};
-    fwd_tc_kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
+    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
+                 pr.g_scalar ? 1 : 0};
+    if (pr.g_scalar) fwd_tc_kernel<true><<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
+    else fwd_tc_kernel<false><<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
     return cudaGetLastError();
 }
 

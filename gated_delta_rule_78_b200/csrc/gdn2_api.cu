@@ -353,10 +353,19 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
+    // a scalar decay goes to the tensor-core forward as it is (one exponential pair per token)
+    const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16 && Dk == 128;
+    const int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
     const void *gp[3] = {log_alpha, b, w};
-    if ((st = expand_gates(flags, dt, l, static_cast<char *>(workspace), (size_t)B * T, H, Dk, gp, s)) != GDN2_OK)
+    if ((st = expand_gates(expand_flags, dt, l, static_cast<char *>(workspace), (size_t)B * T, H, Dk, gp, s)) != GDN2_OK)
         return st;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S0);
+    if (native_decay) {
+        p.g_scalar = true;
+        int *status = gdn2::status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        return from_cuda(gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s));
+    }
     return run_fwd(dt, p, o, S_T, s);
 }
 

@@ -40,6 +40,7 @@ struct Problem {
     const float *S0;  // may be null
     const int *cu_seqlens = nullptr;
     const int *chunk_off = nullptr;
+    bool g_scalar = false;  // tensor-core forward only: log alpha is [rows, H] (one decay per head)
 };
 
 // rows of the token tensors
