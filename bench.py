@@ -19,7 +19,8 @@ steps) and the roofline fraction of each, plus:
 * `varlen`: the headline's 32,768 tokens as 16 packed sequences of log-uniform length
   (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen;
 * `scalar_decay`: the headline batch with one log decay per (token, head) through
-  gdn2_chunk_fwd_gated (the tensor-core forward's scalar-decay path).
+  gdn2_chunk_fwd_gated (the tensor-core forward's scalar-decay path);
+* `d64`: the same model width with head size 64 (H = 32).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 independent (batch, head) sequences; there is no collective on the data path
@@ -406,6 +407,22 @@ def run_ours(args):
                                   "algorithmic_bytes": sd_bytes,
                                   "hbm_frac": round(sd_bytes / (ms_sd * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
         del wsg
+        # ---- head size 64 (same model width: H = 32), bf16, on the tensor-core forward
+        x64 = make_inputs(B, T, 2 * H, D // 2, D // 2, dtype=w["dtype"], seed=rank_seed(rank) + 29, device=str(dev))
+        o64 = torch.empty_like(x64["v"])
+        S64 = torch.empty_like(x64["S0"])
+
+        def fwd_64():
+            g.gdn2_chunk_fwd(x64["q"], x64["k"], x64["v"], x64["log_alpha"], x64["b"], x64["w"], x64["S0"], o=o64,
+                             S_T=S64)
+
+        ms_64 = time_region(fwd_64, 10, 3, stream) / 10
+        assert g.gdn2_sync_status() == 0
+        b64 = fwd_bytes(B, T, 2 * H, D // 2)
+        extras["d64"] = {"workload": f"B={B}, T={T}, H={2 * H}, d={D // 2}, bf16", "ms": round(ms_64, 4),
+                         "tokens_per_s": round(job_rate(tokens, world, ms_64), 1), "algorithmic_bytes": b64,
+                         "hbm_frac": round(b64 / (ms_64 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del x64, o64, S64
         extras["varlen"] = {"sequences": len(lens), "lengths": [int(v) for v in lens], "tokens": tokens,
                             "fwd_ms": round(ms_v, 4), "fwd_tokens_per_s": round(job_rate(tokens, world, ms_v), 1),
                             "fwd_hbm_frac": round(fwd_bytes(1, tokens, H, D) / (ms_v * 1e-3) / 1e9 / pk["hbm_gbs"], 4),

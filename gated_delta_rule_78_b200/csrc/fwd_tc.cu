@@ -112,8 +112,12 @@ __device__ __forceinline__ void named_sync(int id, int count)
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-// kGScalar: log alpha is one value per (token, head) (TcParams::g_scalar)
-template <bool kGScalar>
+// kGScalar: log alpha is one value per (token, head) (TcParams::g_scalar).
+// DIN: the head size of the tensors, 128 or 64.  A d = 64 head runs as a d = 128 head
+// whose channels 64..127 are zero: the TMA boxes past the tensors' channel extent are
+// zero-filled, so k, q, b, v and w vanish there, the state's extra rows and columns stay
+// zero, and only the first 64 channels of o, S_T are stored.
+template <bool kGScalar, int DIN>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -188,7 +192,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
         }
         if (!kGScalar)
-            for (int a = 0; a < 4; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
+            for (int a = 0; a < DIN / 32; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
     };
 
     if (is_m) {
@@ -238,7 +242,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-            Sf[i] = p.S0 ? p.S0[((size_t)bh * D + 64 * half + i) * D + jrow] : 0.f;
+            Sf[i] = (p.S0 && 64 * half + i < DIN && jrow < DIN) ? p.S0[((size_t)bh * DIN + 64 * half + i) * DIN + jrow]
+                                                                 : 0.f;
         if (p.states) store_state(Sf, 0);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -351,8 +356,11 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 tmem_ld32(tmem + TM_O + 32 * half + lane_off, r);
                 tmem_wait_ld();
                 __nv_bfloat16 *so = reinterpret_cast<__nv_bfloat16 *>(sm + ott);
+                if (jrow < DIN) {  // row-major [t][channel] with the tensors' head size as row length
 #pragma unroll
-                for (int u = 0; u < 32; ++u) so[(32 * half + u) * D + jrow] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                    for (int u = 0; u < 32; ++u)
+                        so[(32 * half + u) * DIN + jrow] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                }
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -365,8 +373,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 }
             } else if (p.o) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
                 const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
-                __nv_bfloat16 *dst = p.o + ((size_t)bos + (size_t)ci * C) * p.H * D + (size_t)hh * D;
-                for (int idx = tid; idx < L * D; idx += kGroup) dst[(size_t)(idx / D) * p.H * D + idx % D] = so[idx];
+                __nv_bfloat16 *dst = p.o + ((size_t)bos + (size_t)ci * C) * p.H * DIN + (size_t)hh * DIN;
+                for (int idx = tid; idx < L * DIN; idx += kGroup)
+                    dst[(size_t)(idx / DIN) * p.H * DIN + idx % DIN] = so[idx];
                 named_sync(1, kGroup);
             }
             // ---- next chunk's values (w is single-buffered), then chunk ci+2's loads into this parity
@@ -383,7 +392,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         }
         if (!s_abort_m && p.S_T) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) p.S_T[((size_t)bh * D + 64 * half + i) * D + jrow] = Sf[i];
+            for (int i = 0; i < 64; ++i)
+                if (64 * half + i < DIN && jrow < DIN) p.S_T[((size_t)bh * DIN + 64 * half + i) * DIN + jrow] = Sf[i];
         }
         if (tid == 0) bulk_wait0();
     } else {
@@ -413,11 +423,13 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     gv[i] = make_float2(gs, gs);
                 }
             } else {
-                const float *gsrc = p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H * D + (size_t)hh * D + ch;
+                const float *gsrc =
+                    p.g + ((size_t)bos + (size_t)ci * C + 16 * tg) * p.H * DIN + (size_t)hh * DIN + ch;
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    gv[i] = (16 * tg + i < L) ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * D))
-                                              : make_float2(0.f, 0.f);
+                    gv[i] = (16 * tg + i < L && ch < DIN)
+                                ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * DIN))
+                                : make_float2(0.f, 0.f);
             }
             if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
@@ -560,17 +572,17 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 3-D view (channel, head, token) of a [B,T,H,D] tensor.  Loads: box = (one 128-byte
-// row of channels, 1 head, 64 tokens) with the 128-byte swizzle; the output store:
-// box = (all 128 channels, 1, 64 tokens), no swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, bool store = false)
+// 3-D view (channel, head, token) of a [B,T,H,din] tensor.  Loads: box = (one 128-byte
+// row of channels, 1 head, 64 tokens) with the 128-byte swizzle (a box past the channel
+// extent reads zeros); the output store: box = (all din channels, 1, 64 tokens), no swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, int din, bool store = false)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t es = fp32 ? 4 : 2;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
-    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es};
-    cuuint32_t box[3] = {store ? (cuuint32_t)D : (fp32 ? 32u : 64u), 1u, (cuuint32_t)C};
+    cuuint64_t dims[3] = {(cuuint64_t)din, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)din * es, (cuuint64_t)H * din * es};
+    cuuint32_t box[3] = {store ? (cuuint32_t)din : (fp32 ? 32u : 64u), 1u, (cuuint32_t)C};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -583,24 +595,28 @@ bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, b
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s)
 {
-    if (pr.D != D) return cudaErrorNotSupported;
+    // d = 64 runs zero-padded to 128 (see the kernel); chunk-boundary states only for d = 128
+    if ((pr.D != 128 && pr.D != 64) || (pr.D == 64 && states)) return cudaErrorNotSupported;
+    const int din = pr.D;
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
-    const int rows = (int)token_rows(pr);  // the maps view every tensor as [rows, H, D]
-    if (!make_map(&maps.q, pr.q, false, 1, rows, pr.H) || !make_map(&maps.k, pr.k, false, 1, rows, pr.H) ||
-        !make_map(&maps.v, pr.v, false, 1, rows, pr.H) || !make_map(&maps.b, pr.b, false, 1, rows, pr.H) ||
-        !make_map(&maps.w, pr.w, false, 1, rows, pr.H) || (!pr.g_scalar && !make_map(&maps.g, pr.g, true, 1, rows, pr.H)) ||
-        (o && !make_map(&maps.o, o, false, 1, rows, pr.H, true)))
+    const int rows = (int)token_rows(pr);  // the maps view every tensor as [rows, H, din]
+    if (!make_map(&maps.q, pr.q, false, 1, rows, pr.H, din) || !make_map(&maps.k, pr.k, false, 1, rows, pr.H, din) ||
+        !make_map(&maps.v, pr.v, false, 1, rows, pr.H, din) || !make_map(&maps.b, pr.b, false, 1, rows, pr.H, din) ||
+        !make_map(&maps.w, pr.w, false, 1, rows, pr.H, din) ||
+        (!pr.g_scalar && !make_map(&maps.g, pr.g, true, 1, rows, pr.H, din)) ||
+        (o && !make_map(&maps.o, o, false, 1, rows, pr.H, din, true)))
         return cudaErrorInvalidValue;
-    const void *kfn = pr.g_scalar ? reinterpret_cast<const void *>(fwd_tc_kernel<true>)
-                                  : reinterpret_cast<const void *>(fwd_tc_kernel<false>);
-    cudaError_t e = set_smem_attr(kfn, (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
                  pr.g_scalar ? 1 : 0};
-    if (pr.g_scalar) fwd_tc_kernel<true><<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
-    else fwd_tc_kernel<false><<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
-    return cudaGetLastError();
+    auto run = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = set_smem_attr(reinterpret_cast<const void *>(kernel), (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
+        return cudaGetLastError();
+    };
+    if (din == 128) return pr.g_scalar ? run(fwd_tc_kernel<true, 128>) : run(fwd_tc_kernel<false, 128>);
+    return pr.g_scalar ? run(fwd_tc_kernel<true, 64>) : run(fwd_tc_kernel<false, 64>);
 }
 
 }  // namespace gdn2

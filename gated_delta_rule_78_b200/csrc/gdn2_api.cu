@@ -354,7 +354,7 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
     // a scalar decay goes to the tensor-core forward as it is (one exponential pair per token)
-    const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16 && Dk == 128;
+    const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16;
     const int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
     const void *gp[3] = {log_alpha, b, w};
     if ((st = expand_gates(expand_flags, dt, l, static_cast<char *>(workspace), (size_t)B * T, H, Dk, gp, s)) != GDN2_OK)
