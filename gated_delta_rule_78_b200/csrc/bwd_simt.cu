@@ -435,7 +435,7 @@ cudaError_t launch_t(const Problem &p0, const void *d_o, const float *dS_T, cons
 
 size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p)
 {
-    if (dt == GDN2_BF16 && p.D == 128) return bwd_tc_workspace_bytes(p);
+    if (dt == GDN2_BF16) return bwd_tc_workspace_bytes(p);  // d = 128, and d = 64 zero-padded
     return ws_layout(p, p.D).total;
 }
 
@@ -444,7 +444,7 @@ cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const f
 {
     int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
-    if (dt == GDN2_BF16 && p.D == 128) return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
+    if (dt == GDN2_BF16) return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
     if (dt == GDN2_F32)
         return p.D == 64 ? launch_t<64, float>(p, d_o, dS_T, out, ws, status, s)
                          : launch_t<128, float>(p, d_o, dS_T, out, ws, status, s);

@@ -74,6 +74,7 @@ BwdTcLayout tc_layout(const Problem &p)
 struct BwdTcArgs {
     Problem pr;          // sizes, cu_seqlens and chunk_off (the data pointers are below)
     int H;
+    int din;             // head size of the tensors: 128, or 64 run zero-padded to 128
     const __nv_bfloat16 *q, *k, *v, *b, *w, *dO;
     const float *g;
     const float *dS_T;  // may be null
@@ -98,7 +99,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Row t of chunk `ci` of head hh of the sequence whose first token row is `bos`.
 __device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bos, int hh, int ci, int t)
 {
-    return (((size_t)bos + (size_t)ci * C + t) * a.H + hh) * D;
+    return (((size_t)bos + (size_t)ci * C + t) * a.H + hh) * a.din;
 }
 
 // The chunk a block of the chunk-parallel kernels works on: blockIdx.y is the head,
@@ -149,7 +150,7 @@ __device__ __forceinline__ void cp_tok_tile(uint32_t dst, const __nv_bfloat16 *s
 {
     for (int idx = tid; idx < C * 16; idx += nthreads) {
         const int t = idx >> 4, ch = idx & 15;
-        const bool ok = t < L;
+        const bool ok = t < L && 8 * ch < a.din;  // channels past the head size read zeros
         cp_async16_zfill(dst + swz(t, 8 * ch, 256), src + (ok ? tok_off(a, bb, hh, ci, t) + 8 * ch : 0), ok);
     }
 }
@@ -184,7 +185,7 @@ __device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int t = 16 * q4 + i;
-        const float gv = (t < L) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
+        const float gv = (t < L && c < a.din) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
         run += gv;
         G[i] = run;
     }
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
-            dS[nt][e] = a.dS_T ? a.dS_T[((size_t)bh * D + c) * D + j] : 0.f;
+            dS[nt][e] = (a.dS_T && c < a.din && j < a.din) ? a.dS_T[((size_t)bh * a.din + c) * a.din + j] : 0.f;
         }
     if (nc > 0) prefetch(nc - 1, 0);
     for (int ci = nc - 1; ci >= 0; --ci) {
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
-            a.dS0[((size_t)bh * D + c) * D + j] = dS[nt][e];
+            if (c < a.din && j < a.din) a.dS0[((size_t)bh * a.din + c) * a.din + j] = dS[nt][e];
         }
 }
 
@@ -636,7 +637,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
             for (int hr = 0; hr < 2; ++hr) {
                 const int row = r0 + 8 * hr, col = c0 + 8 * nt;
                 vv[nt][hr] = ww[nt][hr] = 0u;
-                if (row < L) {
+                if (row < L && col < a.din) {
                     const size_t off = tok_off(a, bb, hh, ci, row) + col;
                     vv[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.v + off));
                     ww[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.w + off));
@@ -649,7 +650,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
                 const int row = r0 + 8 * hr, col = c0 + 8 * nt;
                 const float d0 = acc[0][nt][2 * hr], d1 = acc[0][nt][2 * hr + 1];
                 st_pair(sm + G_DY, 256, row, col, -d0, -d1);
-                if (row < L) {
+                if (row < L && col < a.din) {
                     const size_t off = tok_off(a, bb, hh, ci, row) + col;
                     const uint32_t v2 = vv[nt][hr], w2 = ww[nt][hr];
                     *reinterpret_cast<uint32_t *>(a.dv + off) = pack_bf16x2(d0 * bf_lo(w2), d1 * bf_hi(w2));
@@ -727,11 +728,12 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
             const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_X + off_s));
             const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_Y + off_s));
             const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_DO + off_s));
-            const size_t off = (t < L) ? tok_off(a, bb, hh, ci, t) + c : 0;
+            const bool out_ok = t < L && c < a.din;
+            const size_t off = out_ok ? tok_off(a, bb, hh, ci, t) + c : 0;
             const float eG = __expf(G[i]), emG = __expf(-G[i]);
             const float de = dE * eG;
             dG[i] = dQ * qv * eG + de * bv * kv - dK * kv * emG;
-            if (t < L) {
+            if (out_ok) {
                 a.dq[off] = __float2bfloat16_rn(dQ * eG);
                 a.db[off] = __float2bfloat16_rn(de * kv);
                 a.dk[off] = __float2bfloat16_rn(de * bv + dK * emG);
@@ -755,7 +757,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * q4 + i;
-            if (t < L) a.dg[tok_off(a, bb, hh, ci, t) + c] = dG[i] + after;
+            if (t < L && c < a.din) a.dg[tok_off(a, bb, hh, ci, t) + c] = dG[i] + after;
         }
     }
 }
@@ -767,12 +769,13 @@ size_t bwd_tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
                           int *status, cudaStream_t s)
 {
-    if (p.D != D) return cudaErrorNotSupported;
+    if (p.D != 128 && p.D != 64) return cudaErrorNotSupported;
     const BwdTcLayout l = tc_layout(p);
     char *base = static_cast<char *>(ws);
     BwdTcArgs a;
     a.pr = p;
     a.H = p.H;
+    a.din = p.D;
     if (p.cu_seqlens) {
         int *coff = reinterpret_cast<int *>(base);
         cudaError_t e0 = launch_chunk_offsets(p.cu_seqlens, p.B, p.T, coff, status, s);

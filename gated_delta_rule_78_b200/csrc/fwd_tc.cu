@@ -595,8 +595,9 @@ bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, i
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s)
 {
-    // d = 64 runs zero-padded to 128 (see the kernel); chunk-boundary states only for d = 128
-    if ((pr.D != 128 && pr.D != 64) || (pr.D == 64 && states)) return cudaErrorNotSupported;
+    // d = 64 runs zero-padded to 128 (see the kernel); chunk-boundary states keep the padded
+    // 128 x 128 layout (they are the backward's internal workspace)
+    if (pr.D != 128 && pr.D != 64) return cudaErrorNotSupported;
     const int din = pr.D;
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));

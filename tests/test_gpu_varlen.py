@@ -51,7 +51,7 @@ def test_varlen_forward_matches_each_sequence(cuda_lib, dtype, D):
         assert_close(ST[n], rS[0], dtype, f"S_T seq {n} (T={L})")
 
 
-@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64), ("bf16", 64)])
 def test_varlen_backward_matches_each_sequence(cuda_lib, dtype, D):
     g = cuda_lib
     x, S0, cu = packed_inputs(LENS, 2, D, dtype, seed=37)
