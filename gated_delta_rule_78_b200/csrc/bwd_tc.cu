@@ -110,11 +110,10 @@ struct ChunkRef {
     SeqSpan sp;
     size_t cidx;  // per-chunk workspace slot
 };
-__device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
+__device__ __forceinline__ bool chunk_ref_at(const BwdTcArgs &a, int gc, int h, ChunkRef &r)
 {
     const Problem &p = a.pr;
-    const int gc = blockIdx.x;
-    r.h = blockIdx.y;
+    r.h = h;
     if (!p.cu_seqlens) {
         const int nc = seq_chunks(p.T);
         r.n = gc / nc;
@@ -136,6 +135,10 @@ __device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
     if (r.ci >= r.nch) return false;
     r.cidx = chunk_slot(p, r.n, r.h, r.nch, r.ci);
     return true;
+}
+__device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
+{
+    return chunk_ref_at(a, blockIdx.x, blockIdx.y, r);
 }
 
 // cp.async versions: the copies stay in flight until cp_async_wait; rows past the
@@ -177,20 +180,32 @@ __device__ __forceinline__ uint32_t ld_pair(const uint8_t *tile, int rb, int row
 // Per-thread cumulative log decay: thread (channel c, quarter q4) owns tokens
 // 16 q4 .. 16 q4 + 15; on return G[i] is the inclusive cumsum at token 16 q4 + i and
 // `total` the chunk total G_C.  sTot is a [4][D] fp32 scratch.  Needs 512 threads.
-template <bool kWaitCopies = false>
-__device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const BwdTcArgs &a, int bb, int hh,
-                                             int ci, int L, int c, int q4, float *sTot)
+// log alpha of this thread's 16 tokens (channel c, quarter q4), zero past the sequence end
+__device__ __forceinline__ void load_g16(float (&G)[16], const BwdTcArgs &a, int bb, int hh, int ci, int L, int c,
+                                         int q4)
 {
-    float run = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int t = 16 * q4 + i;
-        const float gv = (t < L && c < a.din) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
-        run += gv;
+        G[i] = (t < L && c < a.din) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
+    }
+}
+
+// kWaitCopies: wait for this thread's cp.async groups except the newest kKeep ones before the barrier.
+// kLoaded: G already holds the log alpha values (load_g16).
+template <bool kWaitCopies = false, int kKeep = 0, bool kLoaded = false>
+__device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const BwdTcArgs &a, int bb, int hh,
+                                             int ci, int L, int c, int q4, float *sTot)
+{
+    if (!kLoaded) load_g16(G, a, bb, hh, ci, L, c, q4);
+    float run = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        run += G[i];
         G[i] = run;
     }
     sTot[q4 * D + c] = run;
-    if (kWaitCopies) cp_async_wait<0>();  // this thread's tile copies have landed
+    if (kWaitCopies) cp_async_wait<kKeep>();  // this thread's tile copies have landed
     __syncthreads();
     float off = 0.f, tot = 0.f;
 #pragma unroll
@@ -210,43 +225,74 @@ __device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const
 constexpr uint32_t P_Q = 0, P_E = 16384, P_K = 32768, P_DO = 49152, P_W = 65536, P_Z = 81920;
 constexpr uint32_t P_TB = 98304, P_PB = 106496, P_SA = 114688, P_ST = P_SA + C * LDA * 4;
 constexpr uint32_t P_TOT = P_ST + C * LDA * 4;
-constexpr uint32_t P_SMEM = P_TOT + 4 * D * 4;
+constexpr uint32_t P_SET1 = P_TOT + 4 * D * 4;     // second set of the raw q, b, k, dO tiles
+constexpr uint32_t P_SMEM = P_SET1 + 4 * 16384;
 constexpr int kPrepThreads = 512;
 
-__global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcArgs a)
+// Persistent: block x takes the (chunk, head) tasks x, x + gridDim.x, ...  The raw tiles of
+// the next task are copied (cp.async) into the other tile set, and its log alpha loaded,
+// while the current task computes.
+__global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcArgs a, int nbound)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    ChunkRef cr;
-    if (!chunk_ref(a, cr)) return;
-    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
-    const int L = min(C, cr.sp.len - ci * C);
-    const size_t cidx = cr.cidx;
+    const int c = tid & (D - 1), q4 = tid >> 7;  // decay-folding mapping
     const uint32_t sb = smem_u32(sm);
     float *sA = reinterpret_cast<float *>(sm + P_SA);
     float *sT = reinterpret_cast<float *>(sm + P_ST);
-
-    // ---- raw q, k, b, dO tiles; T scratch zeroed (its upper blocks stay zero)
-    cp_tok_tile(sb + P_Q, a.q, a, bb, hh, ci, L, tid, kPrepThreads);
-    cp_tok_tile(sb + P_K, a.k, a, bb, hh, ci, L, tid, kPrepThreads);
-    cp_tok_tile(sb + P_E, a.b, a, bb, hh, ci, L, tid, kPrepThreads);
-    cp_tok_tile(sb + P_DO, a.dO, a, bb, hh, ci, L, tid, kPrepThreads);
+    const int ntasks = nbound * a.H;
+    // tile set offsets (the raw tiles become the factors in place)
+    auto tile = [](int buf, int which) -> uint32_t {  // which: 0 q, 1 b, 2 k, 3 dO
+        const uint32_t base0[4] = {P_Q, P_E, P_K, P_DO};
+        return buf ? P_SET1 + which * 16384u : base0[which];
+    };
+    auto issue = [&](int task, int buf, float (&Gn)[16]) {
+        ChunkRef r;
+        if (task >= ntasks || !chunk_ref_at(a, task % nbound, task / nbound, r)) return;
+        const int Lr = min(C, r.sp.len - r.ci * C);
+        cp_tok_tile(sb + tile(buf, 0), a.q, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
+        cp_tok_tile(sb + tile(buf, 2), a.k, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
+        cp_tok_tile(sb + tile(buf, 1), a.b, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
+        cp_tok_tile(sb + tile(buf, 3), a.dO, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
+        load_g16(Gn, a, r.sp.bos, r.h, r.ci, Lr, c, q4);
+    };
+    float Gnext[16];
+    issue(blockIdx.x, 0, Gnext);
     cp_async_commit();
+    int it = 0;
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x, ++it) {
+    const int buf = it & 1;
+    float G[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) G[i] = Gnext[i];
+    issue(task + gridDim.x, buf ^ 1, Gnext);  // the next task's copies, into the other set
+    cp_async_commit();
+    ChunkRef cr;
+    if (!chunk_ref_at(a, task % nbound, task / nbound, cr)) {
+        cp_async_wait<1>();
+        __syncthreads();
+        continue;
+    }
+    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
+    const int L = min(C, cr.sp.len - ci * C);
+    const size_t cidx = cr.cidx;
+    const uint32_t P_Qb = tile(buf, 0), P_Eb = tile(buf, 1), P_Kb = tile(buf, 2), P_DOb = tile(buf, 3);
+
+    // ---- T scratch zeroed (its upper blocks stay zero)
     for (int idx = tid; idx < C * LDA; idx += kPrepThreads) sT[idx] = 0.f;
     // ---- decay folding (thread: channel c, 16 tokens); K^ and gamma go straight out
     {
-        const int c = tid & (D - 1), q4 = tid >> 7;
-        float G[16], GC;
-        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
+        float GC;
+        chunk_cumsum<true, 1, true>(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
         if (q4 == 0) a.gam[cidx * D + c] = __expf(GC);
         __nv_bfloat16 *kh = a.Kh + cidx * C * D;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * q4 + i;
             const uint32_t off = swz(t, c, 256);
-            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + P_Q + off);
-            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + P_K + off);
-            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + P_E + off);
+            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + P_Qb + off);
+            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + P_Kb + off);
+            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + P_Eb + off);
             const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk), bv = __bfloat162float(*pe);
             const float eG = __expf(G[i]), emG = __expf(-G[i]);
             *pq = __float2bfloat16_rn(qv * eG);
@@ -261,7 +307,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 7, nh = warp >> 3;
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, false, D>(acc, sb + (mt < 4 ? P_E : P_Q), 256, 16 * (mt & 3), sb + P_K, 256, 32 * nh,
+        warp_gemm<1, 4, false, false, D>(acc, sb + (mt < 4 ? P_Eb : P_Qb), 256, 16 * (mt & 3), sb + P_Kb, 256, 32 * nh,
                                          lane);
         const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
@@ -286,7 +332,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 3, nh = (warp >> 2) & 1;
         float acc[1][8][4];
         zero_acc(acc);
-        warp_gemm<1, 8, true, true, C>(acc, sb + P_PB, 128, 16 * mt, sb + P_DO, 256, 64 * nh, lane);
+        warp_gemm<1, 8, true, true, C>(acc, sb + P_PB, 128, 16 * mt, sb + P_DOb, 256, 64 * nh, lane);
         const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
@@ -315,7 +361,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mt = warp & 3, nq = warp >> 2;
         float acc[1][4][4];
         zero_acc(acc);
-        warp_gemm<1, 4, false, true, C>(acc, sb + P_TB, 128, 16 * mt, sb + P_E, 256, 32 * nq, lane);
+        warp_gemm<1, 4, false, true, C>(acc, sb + P_TB, 128, 16 * mt, sb + P_Eb, 256, 32 * nq, lane);
         const int g = lane >> 2, t4 = lane & 3;
         __nv_bfloat16 *wg = a.W + cidx * C * D;
 #pragma unroll
@@ -334,7 +380,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const int mb = warp & 3, nb = warp >> 2;
         float acc[2][4][4];
         zero_acc(acc);
-        warp_gemm<2, 4, true, true, C>(acc, sb + P_DO, 256, 32 * mb, sb + P_Q, 256, 32 * nb, lane);
+        warp_gemm<2, 4, true, true, C>(acc, sb + P_DOb, 256, 32 * mb, sb + P_Qb, 256, 32 * nb, lane);
         warp_gemm<2, 4, true, true, C>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, lane);
         const int g = lane >> 2, t4 = lane & 3;
         float *rt = a.Rt + cidx * D * D;
@@ -349,6 +395,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
                         make_float2(acc[mt][nt][2 * hr], acc[mt][nt][2 * hr + 1]);
                 }
     }
+    __syncthreads();  // every warp is done with this task's tiles before they are refilled
+    }
+    cp_async_wait<0>();
 }
 
 // ================================================================== 3. chain
@@ -810,7 +859,14 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     if (e != cudaSuccess) return e;
     const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_kernel), (int)P_SMEM)) != cudaSuccess) return e;
-    bwd_prep_kernel<<<nblk, kPrepThreads, P_SMEM, s>>>(a);
+    {  // persistent: one block per SM, each streaming (chunk, head) tasks
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int nbound = (int)chunk_bound(p);
+        const long long ntasks = (long long)nbound * p.H;
+        const int grid = (int)(ntasks < sms ? ntasks : sms);
+        bwd_prep_kernel<<<grid, kPrepThreads, P_SMEM, s>>>(a, nbound);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
     bwd_chain_kernel<<<p.B * p.H, kChainThreads, CH_SMEM, s>>>(a);
