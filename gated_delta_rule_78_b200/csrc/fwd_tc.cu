@@ -7,6 +7,12 @@
 // auxiliary matrices of the aixai.ru post's "Как это реализуется на практике"):
 //   G  = inclusive cumulative sum of log alpha over the chunk (fp32)
 //   Q~ = q e^G,  E~ = (b.k) e^G,  K~ = k e^-G,  gamma = e^G_L,  X = w.v
+//                                    (one exponential per element, alpha = e^g: e^G is a
+//                                    running product of alpha forwards from the token
+//                                    group's start, e^-G one backwards from its end.  The
+//                                    factors are bf16x2 products of the bf16 inputs and
+//                                    e^+-G rounded to bf16; X is one, exact before its
+//                                    single rounding)
 //   [A; P] = [E~; Q~] K~^T          A strictly lower, P lower incl. (one M=128 MMA)
 //   T   = (I + A)^-1                 blocked: 16x16 diagonal blocks by substitution,
 //                                    the doubling levels on warp-level TF32 MMAs
@@ -109,8 +115,13 @@ __device__ __forceinline__ void named_sync(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+// bf16x2 product, rounded to nearest even
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
 
 // kGScalar: log alpha is one value per (token, head) (TcParams::g_scalar).
 // DIN: the head size of the tensors, 128 or 64.  A d = 64 head runs as a d = 128 head
@@ -217,8 +228,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 const uint32_t off = a * 8192 + sw128(t, 4 * lane);
                 const uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
                 const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
-                *reinterpret_cast<uint32_t *>(pv + off) =
-                    (t < Lc) ? pack_bf16x2(bf_lo(vw) * bf_lo(ww), bf_hi(vw) * bf_hi(ww)) : 0u;
+                *reinterpret_cast<uint32_t *>(pv + off) = (t < Lc) ? bmul2(vw, ww) : 0u;
             }
         };
         if (tid == 0 && nchunks > 0) issue(0);
@@ -437,7 +447,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             for (int i = 0; i < 16; ++i) {
                 run0 += gv[i].x;
                 run1 += gv[i].y;
-                gv[i] = make_float2(run0, run1);
+                const float a0 = __expf(gv[i].x);
+                gv[i] = make_float2(a0, kGScalar ? a0 : __expf(gv[i].y));  // alpha
             }
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
             named_sync(2, kGroup);
@@ -455,21 +466,32 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 uint8_t *pe = sm + oqe + cb * 16384;
                 uint8_t *pq = pe + 8192;
                 uint8_t *pk = sm + ok + cb * 8192;
+                float2 mv[16];  // e^-G of each token: backwards from the group's last token
+                {
+                    float r0 = __expf(-(c0 + run0)), r1 = kGScalar ? r0 : __expf(-(c1 + run1));
+#pragma unroll
+                    for (int i = 15; i >= 0; --i) {
+                        mv[i] = make_float2(r0, r1);
+                        r0 *= gv[i].x;
+                        r1 *= gv[i].y;
+                    }
+                }
+                float e0 = __expf(c0), e1 = kGScalar ? e0 : __expf(c1);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int t = 16 * tg + i;
                     const uint32_t off = sw128(t, 4 * lane);
-                    const float G0 = c0 + gv[i].x, G1 = c1 + gv[i].y;
-                    const float e0 = __expf(G0), m0 = __expf(-G0);
-                    const float e1 = kGScalar ? e0 : __expf(G1), m1 = kGScalar ? m0 : __expf(-G1);
+                    e0 *= gv[i].x;
+                    e1 *= gv[i].y;
+                    const float m0 = mv[i].x, m1 = mv[i].y;
                     uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
                     uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
                     uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
                     if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
-                    const float k0 = bf_lo(kw), k1 = bf_hi(kw);
-                    *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
-                    *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
-                    *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
+                    const uint32_t e01 = pack_bf16x2(e0, e1), m01 = pack_bf16x2(m0, m1);
+                    *reinterpret_cast<uint32_t *>(pq + off) = bmul2(qw, e01);
+                    *reinterpret_cast<uint32_t *>(pe + off) = bmul2(bmul2(bw, kw), e01);
+                    *reinterpret_cast<uint32_t *>(pk + off) = bmul2(kw, m01);
                 }
             }
             fence_proxy_async_smem();
