@@ -82,6 +82,7 @@ struct BwdTcArgs {
     float *gam, *Rt;
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
+    int n_sm;            // multiprocessors of the device (L2 prefetch distance of the gradient kernel)
 };
 
 // ------------------------------------------------------------------ small helpers
@@ -177,46 +178,72 @@ __device__ __forceinline__ uint32_t ld_pair(const uint8_t *tile, int rb, int row
     return *reinterpret_cast<const uint32_t *>(tile + swz(row, col, rb));
 }
 
-// Per-thread cumulative log decay: thread (channel c, quarter q4) owns tokens
-// 16 q4 .. 16 q4 + 15; on return G[i] is the inclusive cumsum at token 16 q4 + i and
-// `total` the chunk total G_C.  sTot is a [4][D] fp32 scratch.  Needs 512 threads.
-// log alpha of this thread's 16 tokens (channel c, quarter q4), zero past the sequence end
-__device__ __forceinline__ void load_g16(float (&G)[16], const BwdTcArgs &a, int bb, int hh, int ci, int L, int c,
-                                         int q4)
+// Two-channel layout of the prep and gradient kernels' elementwise work: thread (channel pair cp,
+// token group g8) owns channels 2 cp, 2 cp + 1 and tokens 8 g8 .. 8 g8 + 7 (64 x 8 = 512
+// threads).  log alpha of those 16 values, zero past the sequence end and the head size.
+__device__ __forceinline__ void load_g8(float2 (&g)[8], const BwdTcArgs &a, int bb, int hh, int ci, int L, int cp,
+                                        int g8)
 {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int t = 16 * q4 + i;
-        G[i] = (t < L && c < a.din) ? __ldg(a.g + tok_off(a, bb, hh, ci, t) + c) : 0.f;
+    for (int i = 0; i < 8; ++i) {
+        const int t = 8 * g8 + i;
+        g[i] = (t < L && 2 * cp < a.din)
+                   ? __ldg(reinterpret_cast<const float2 *>(a.g + tok_off(a, bb, hh, ci, t) + 2 * cp))
+                   : make_float2(0.f, 0.f);
     }
 }
 
-// kWaitCopies: wait for this thread's cp.async groups except the newest kKeep ones before the barrier.
-// kLoaded: G already holds the log alpha values (load_g16).
-template <bool kWaitCopies = false, int kKeep = 0, bool kLoaded = false>
-__device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const BwdTcArgs &a, int bb, int hh,
-                                             int ci, int L, int c, int q4, float *sTot)
+// e^G and e^-G of this thread's 16 values (G the inclusive cumulative sum of log alpha over
+// the chunk) with one exponential per value: alpha = e^g, then e^G as a running product
+// forwards from the token group's start and e^-G as one backwards from its end.  The group
+// totals go through sTot ([8][D] fp32); `total` is G at the chunk end.  Contains a
+// __syncthreads; kWait: this thread's cp.async copies, except the newest kKeep groups,
+// are waited for before it.
+template <bool kWait, int kKeep = 0>
+__device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8], float2 (&emG)[8], float2 &total,
+                                            int cp, int g8, float *sTot)
 {
-    if (!kLoaded) load_g16(G, a, bb, hh, ci, L, c, q4);
-    float run = 0.f;
+    float run0 = 0.f, run1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        run += G[i];
-        G[i] = run;
+    for (int i = 0; i < 8; ++i) {
+        run0 += g[i].x;
+        run1 += g[i].y;
+        eG[i] = make_float2(__expf(g[i].x), __expf(g[i].y));  // alpha for now
     }
-    sTot[q4 * D + c] = run;
-    if (kWaitCopies) cp_async_wait<kKeep>();  // this thread's tile copies have landed
+    *reinterpret_cast<float2 *>(sTot + g8 * D + 2 * cp) = make_float2(run0, run1);
+    if (kWait) cp_async_wait<kKeep>();
     __syncthreads();
-    float off = 0.f, tot = 0.f;
+    float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const float v = sTot[u * D + c];
-        if (u < q4) off += v;
-        tot += v;
+    for (int u = 0; u < 8; ++u) {
+        const float2 v = *reinterpret_cast<const float2 *>(sTot + u * D + 2 * cp);
+        if (u < g8) { off0 += v.x; off1 += v.y; }
+        tot0 += v.x;
+        tot1 += v.y;
     }
+    float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) G[i] += off;
-    total = tot;
+    for (int i = 7; i >= 0; --i) {
+        emG[i] = make_float2(r0, r1);
+        r0 *= eG[i].x;
+        r1 *= eG[i].y;
+    }
+    float e0 = __expf(off0), e1 = __expf(off1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        e0 *= eG[i].x;
+        e1 *= eG[i].y;
+        eG[i] = make_float2(e0, e1);
+    }
+    total = make_float2(tot0, tot1);
+}
+
+// bf16x2 product, rounded to nearest even (exact before the rounding for bf16 inputs)
+__device__ __forceinline__ uint32_t bmul2(uint32_t x, uint32_t y)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
+    return r;
 }
 
 // ================================================================== 2. prep
@@ -225,9 +252,15 @@ __device__ __forceinline__ void chunk_cumsum(float (&G)[16], float &total, const
 constexpr uint32_t P_Q = 0, P_E = 16384, P_K = 32768, P_DO = 49152, P_W = 65536, P_Z = 81920;
 constexpr uint32_t P_TB = 98304, P_PB = 106496, P_SA = 114688, P_ST = P_SA + C * LDA * 4;
 constexpr uint32_t P_TOT = P_ST + C * LDA * 4;
-constexpr uint32_t P_SET1 = P_TOT + 4 * D * 4;     // second set of the raw q, b, k, dO tiles
+constexpr uint32_t P_SET1 = P_TOT + 8 * D * 4;     // second set of the raw q, b, k, dO tiles
 constexpr uint32_t P_SMEM = P_SET1 + 4 * 16384;
 constexpr int kPrepThreads = 512;
+
+// L2 prefetch (bulk, no shared-memory destination)
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // Persistent: block x takes the (chunk, head) tasks x, x + gridDim.x, ...  The raw tiles of
 // the next task are copied (cp.async) into the other tile set, and its log alpha loaded,
@@ -236,7 +269,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = tid & (D - 1), q4 = tid >> 7;  // decay-folding mapping
+    const int cp = tid & 63, g8 = tid >> 6;  // decay-folding mapping: channel pair, group of 8 tokens
     const uint32_t sb = smem_u32(sm);
     float *sA = reinterpret_cast<float *>(sm + P_SA);
     float *sT = reinterpret_cast<float *>(sm + P_ST);
@@ -246,7 +279,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         const uint32_t base0[4] = {P_Q, P_E, P_K, P_DO};
         return buf ? P_SET1 + which * 16384u : base0[which];
     };
-    auto issue = [&](int task, int buf, float (&Gn)[16]) {
+    auto issue = [&](int task, int buf, float2 (&Gn)[8]) {
         ChunkRef r;
         if (task >= ntasks || !chunk_ref_at(a, task % nbound, task / nbound, r)) return;
         const int Lr = min(C, r.sp.len - r.ci * C);
@@ -254,17 +287,17 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         cp_tok_tile(sb + tile(buf, 2), a.k, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
         cp_tok_tile(sb + tile(buf, 1), a.b, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
         cp_tok_tile(sb + tile(buf, 3), a.dO, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
-        load_g16(Gn, a, r.sp.bos, r.h, r.ci, Lr, c, q4);
+        load_g8(Gn, a, r.sp.bos, r.h, r.ci, Lr, cp, g8);
     };
-    float Gnext[16];
+    float2 Gnext[8];
     issue(blockIdx.x, 0, Gnext);
     cp_async_commit();
     int it = 0;
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x, ++it) {
     const int buf = it & 1;
-    float G[16];
+    float2 G[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) G[i] = Gnext[i];
+    for (int i = 0; i < 8; ++i) G[i] = Gnext[i];
     issue(task + gridDim.x, buf ^ 1, Gnext);  // the next task's copies, into the other set
     cp_async_commit();
     ChunkRef cr;
@@ -273,32 +306,33 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         __syncthreads();
         continue;
     }
-    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
-    const int L = min(C, cr.sp.len - ci * C);
+    const int L = min(C, cr.sp.len - cr.ci * C);
     const size_t cidx = cr.cidx;
     const uint32_t P_Qb = tile(buf, 0), P_Eb = tile(buf, 1), P_Kb = tile(buf, 2), P_DOb = tile(buf, 3);
 
     // ---- T scratch zeroed (its upper blocks stay zero)
     for (int idx = tid; idx < C * LDA; idx += kPrepThreads) sT[idx] = 0.f;
-    // ---- decay folding (thread: channel c, 16 tokens); K^ and gamma go straight out
+    // ---- decay folding (thread: channels 2 cp, 2 cp + 1, 8 tokens); K^ and gamma go straight out
     {
-        float GC;
-        chunk_cumsum<true, 1, true>(G, GC, a, bb, hh, ci, L, c, q4, reinterpret_cast<float *>(sm + P_TOT));
-        if (q4 == 0) a.gam[cidx * D + c] = __expf(GC);
+        float2 eG[8], emG[8], tot;
+        decay_pair8<true, 1>(G, eG, emG, tot, cp, g8, reinterpret_cast<float *>(sm + P_TOT));
+        const float gam0 = __expf(tot.x), gam1 = __expf(tot.y);  // K^ = k e^(G_C - G) = gamma K~
+        if (g8 == 0) *reinterpret_cast<float2 *>(a.gam + cidx * D + 2 * cp) = make_float2(gam0, gam1);
         __nv_bfloat16 *kh = a.Kh + cidx * C * D;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * q4 + i;
-            const uint32_t off = swz(t, c, 256);
-            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + P_Qb + off);
-            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + P_Kb + off);
-            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + P_Eb + off);
-            const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk), bv = __bfloat162float(*pe);
-            const float eG = __expf(G[i]), emG = __expf(-G[i]);
-            *pq = __float2bfloat16_rn(qv * eG);
-            *pe = __float2bfloat16_rn(bv * kv * eG);
-            *pk = __float2bfloat16_rn(kv * emG);
-            kh[t * D + c] = __float2bfloat16_rn(kv * __expf(GC - G[i]));
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            const uint32_t off = swz(t, 2 * cp, 256);
+            uint32_t *pq = reinterpret_cast<uint32_t *>(sm + P_Qb + off);
+            uint32_t *pk = reinterpret_cast<uint32_t *>(sm + P_Kb + off);
+            uint32_t *pe = reinterpret_cast<uint32_t *>(sm + P_Eb + off);
+            const uint32_t q2 = *pq, k2 = *pk, b2 = *pe;
+            const float k0 = bf_lo(k2), k1 = bf_hi(k2);
+            *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
+            *pe = pack_bf16x2(bf_lo(b2) * k0 * eG[i].x, bf_hi(b2) * k1 * eG[i].y);
+            *pk = pack_bf16x2(k0 * emG[i].x, k1 * emG[i].y);
+            *reinterpret_cast<uint32_t *>(kh + t * D + 2 * cp) =
+                pack_bf16x2(k0 * emG[i].x * gam0, k1 * emG[i].y * gam1);
         }
     }
     __syncthreads();
@@ -535,7 +569,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 // products, dQ~, dE~, dK~ (fp32 [C][LDF]) reuse the first 104 KB.
 constexpr uint32_t G_Q = 0, G_E = 16384, G_K = 32768, G_S = 49152, G_DS = 81920, G_X = 114688, G_Y = 131072;
 constexpr uint32_t G_DO = 147456, G_DY = 163840, G_TB = 180224, G_PB = 188416, G_TOT = 196608;
-constexpr uint32_t G_GAM = G_TOT + 4 * D * 4, G_DGP = G_GAM + D * 4, G_DGF = G_DGP + 16 * D * 4;
+constexpr uint32_t G_GAM = G_TOT + 8 * D * 4, G_DGP = G_GAM + D * 4, G_DGF = G_DGP + 16 * D * 4;
 constexpr uint32_t G_SMEM = G_DGF + D * 4;
 constexpr int LDF = 136;  // fp32 row stride of the dQ~ / dE~ / dK~ tiles
 constexpr uint32_t G_FQ = 0, G_FE = C * LDF * 4, G_FK = 2 * C * LDF * 4;
@@ -557,7 +591,22 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     float *sGam = reinterpret_cast<float *>(sm + G_GAM);
     float *sDgp = reinterpret_cast<float *>(sm + G_DGP);
     float *sDgf = reinterpret_cast<float *>(sm + G_DGF);
-    const int c = tid & (D - 1), q4 = tid >> 7;  // elementwise mapping: channel, quarter of the tokens
+    const int cp = tid & 63, g8 = tid >> 6;  // elementwise mapping: channel pair, group of 8 tokens
+    const __nv_bfloat16 *st_c = a.states + bound_slot(a.pr, cr.n, hh, cr.nch, ci) * D * D;
+    // dS_n and the chunk-end state, for (Diag(gamma) dS_n)^T and gamma dgamma: loaded first, so
+    // that their latency hides behind the operand copies and the decay folding
+    const int dch = tid & 15;
+    uint4 dsv[4], ssv[4];
+    {
+        const __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
+        const __nv_bfloat16 *st_n = st_c + (size_t)D * D;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = (tid >> 4) + 32 * u;
+            dsv[u] = __ldg(reinterpret_cast<const uint4 *>(dsn + (size_t)j * D + 8 * dch));
+            ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)j * D + 8 * dch));
+        }
+    }
 
     // ---- P0: operands
     cp_tok_tile(sb + G_Q, a.q, a, bb, hh, ci, L, tid, kGradThreads);
@@ -566,37 +615,34 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     cp_tok_tile(sb + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
     cp_tok_tile(sb + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
     cp_tok_tile(sb + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
-    const __nv_bfloat16 *st_c = a.states + bound_slot(a.pr, cr.n, hh, cr.nch, ci) * D * D;
     cp_dense_tile(sb + G_S, st_c, D, D, tid, kGradThreads);
     cp_dense_tile(sb + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
     cp_dense_tile(sb + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
     cp_async_commit();
     {
-        float G[16], GC;
-        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // its barrier also publishes the tiles
-        if (q4 == 0) sGam[c] = __expf(GC);
+        float2 gl[8], eG[8], emG[8], tot;
+        load_g8(gl, a, bb, hh, ci, L, cp, g8);
+        decay_pair8<true>(gl, eG, emG, tot, cp, g8, sTot);  // its barrier also publishes the tiles
+        if (g8 == 0) *reinterpret_cast<float2 *>(sGam + 2 * cp) = make_float2(__expf(tot.x), __expf(tot.y));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * q4 + i;
-            const uint32_t off = swz(t, c, 256);
-            __nv_bfloat16 *pq = reinterpret_cast<__nv_bfloat16 *>(sm + G_Q + off);
-            __nv_bfloat16 *pk = reinterpret_cast<__nv_bfloat16 *>(sm + G_K + off);
-            __nv_bfloat16 *pe = reinterpret_cast<__nv_bfloat16 *>(sm + G_E + off);
-            __nv_bfloat16 *px = reinterpret_cast<__nv_bfloat16 *>(sm + G_X + off);
-            const __nv_bfloat16 *pw = reinterpret_cast<const __nv_bfloat16 *>(sm + G_Y + off);
-            const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk), bv = __bfloat162float(*pe);
-            const float eG = __expf(G[i]), emG = __expf(-G[i]);
-            *pq = __float2bfloat16_rn(qv * eG);
-            *pe = __float2bfloat16_rn(bv * kv * eG);
-            *pk = __float2bfloat16_rn(kv * emG);
-            *px = __float2bfloat16_rn(__bfloat162float(*px) * __bfloat162float(*pw));  // X = w.v (column c = j)
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            const uint32_t off = swz(t, 2 * cp, 256);
+            uint32_t *pq = reinterpret_cast<uint32_t *>(sm + G_Q + off);
+            uint32_t *pk = reinterpret_cast<uint32_t *>(sm + G_K + off);
+            uint32_t *pe = reinterpret_cast<uint32_t *>(sm + G_E + off);
+            uint32_t *px = reinterpret_cast<uint32_t *>(sm + G_X + off);
+            const uint32_t q2 = *pq, k2 = *pk, b2 = *pe, x2 = *px, w2 = *reinterpret_cast<const uint32_t *>(sm + G_Y + off);
+            const float k0 = bf_lo(k2), k1 = bf_hi(k2);
+            *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
+            *pe = pack_bf16x2(bf_lo(b2) * k0 * eG[i].x, bf_hi(b2) * k1 * eG[i].y);
+            *pk = pack_bf16x2(k0 * emG[i].x, k1 * emG[i].y);
+            *px = bmul2(x2, w2);  // X = w.v (columns = j)
         }
     }
     __syncthreads();
     {  // (Diag(gamma) dS_n)^T tile, and gamma dgamma = rowsum(dS_n . S') partials
-        const __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
-        const __nv_bfloat16 *st_n = st_c + (size_t)D * D;
-        const int ch = tid & 15;
+        const int ch = dch;
         float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         float gm[8];
 #pragma unroll
@@ -604,8 +650,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int j = (tid >> 4) + 32 * u;
-            const uint4 dv4 = *reinterpret_cast<const uint4 *>(dsn + (size_t)j * D + 8 * ch);
-            const uint4 sv4 = *reinterpret_cast<const uint4 *>(st_n + (size_t)j * D + 8 * ch);
+            const uint4 dv4 = dsv[u], sv4 = ssv[u];
             const uint32_t dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w}, sw[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
             uint32_t o[4];
 #pragma unroll
@@ -630,6 +675,32 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
 #pragma unroll
         for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
         sDgf[tid] = s;
+    }
+    {  // everything the block one wave later reads, into L2 (one bulk prefetch per thread)
+        const int nblk = gridDim.x * gridDim.y, nxt = blockIdx.y * gridDim.x + blockIdx.x + a.n_sm;
+        ChunkRef r;
+        if (nxt < nblk && chunk_ref_at(a, nxt % gridDim.x, nxt / gridDim.x, r)) {
+            const int Ln = min(C, r.sp.len - r.ci * C);
+            const uint32_t rowb = (uint32_t)a.din * 2;
+            if (tid < 7 * C) {
+                const int which = tid / C, t = tid % C;
+                if (t < Ln) {
+                    const size_t off = tok_off(a, r.sp.bos, r.h, r.ci, t);
+                    const __nv_bfloat16 *src = which == 0 ? a.q : which == 1 ? a.k : which == 2 ? a.b
+                                             : which == 3 ? a.v : which == 4 ? a.w : a.dO;
+                    if (which < 6) bulk_prefetch_l2(src + off, rowb);
+                    else bulk_prefetch_l2(a.g + off, 2 * rowb);
+                }
+            } else if (tid == 7 * C) {
+                bulk_prefetch_l2(a.states + bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D * D, 2 * D * D * 2);
+            } else if (tid == 7 * C + 1) {
+                bulk_prefetch_l2(a.Tm + r.cidx * C * C, C * C * 2);
+            } else if (tid == 7 * C + 2) {
+                bulk_prefetch_l2(a.Pm + r.cidx * C * C, C * C * 2);
+            } else if (tid == 7 * C + 3) {
+                bulk_prefetch_l2(a.dSn + r.cidx * D * D, D * D * 2);
+            }
+        }
     }
     // warp tiling of the [C][D] products: 16 rows x 32 columns
     const int mt = warp & 3, nq = warp >> 2;
@@ -676,10 +747,7 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
     __syncthreads();
     // ---- P4: dY = T^T dU~ -> dv = dY w, dw = dY v (global), -dY (bf16)
     {
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, true, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
-        uint32_t vv[4][2], ww[4][2];  // all loads first, so that they are in flight together
+        uint32_t vv[4][2], ww[4][2];  // all loads first, in flight during the product
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -692,6 +760,9 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
                     ww[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.w + off));
                 }
             }
+        float acc[1][4][4];
+        zero_acc(acc);
+        warp_gemm<1, 4, true, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -762,51 +833,66 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
             }
     }
     __syncthreads();
-    // ---- P10: through the factors (thread: channel c, tokens 16 q4 .. +15), fp32
+    // ---- P10: through the factors (thread: channels 2 cp, 2 cp + 1, tokens 8 g8 .. +7), fp32
     {
         const float *fq = reinterpret_cast<const float *>(sm + G_FQ), *fe = reinterpret_cast<const float *>(sm + G_FE);
         const float *fk = reinterpret_cast<const float *>(sm + G_FK);
-        float G[16], GC;
-        chunk_cumsum<true>(G, GC, a, bb, hh, ci, L, c, q4, sTot);  // sTot is free again (P0 finished)
-        float dG[16];
+        float2 gl[8], eG[8], emG[8], tot;
+        load_g8(gl, a, bb, hh, ci, L, cp, g8);
+        decay_pair8<true>(gl, eG, emG, tot, cp, g8, sTot);  // sTot is free again (P0 finished)
+        const bool ch_ok = 2 * cp < a.din;
+        const size_t base = tok_off(a, bb, hh, ci, 8 * g8) + 2 * cp, stride = (size_t)a.H * a.din;
+        float2 dG[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * q4 + i;
-            const float dQ = fq[t * LDF + c], dE = fe[t * LDF + c], dK = fk[t * LDF + c];
-            const uint32_t off_s = swz(t, c, 256);
-            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_X + off_s));
-            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_Y + off_s));
-            const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + G_DO + off_s));
-            const bool out_ok = t < L && c < a.din;
-            const size_t off = out_ok ? tok_off(a, bb, hh, ci, t) + c : 0;
-            const float eG = __expf(G[i]), emG = __expf(-G[i]);
-            const float de = dE * eG;
-            dG[i] = dQ * qv * eG + de * bv * kv - dK * kv * emG;
-            if (out_ok) {
-                a.dq[off] = __float2bfloat16_rn(dQ * eG);
-                a.db[off] = __float2bfloat16_rn(de * kv);
-                a.dk[off] = __float2bfloat16_rn(de * bv + dK * emG);
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            const float2 dQ = *reinterpret_cast<const float2 *>(fq + t * LDF + 2 * cp);
+            const float2 dE = *reinterpret_cast<const float2 *>(fe + t * LDF + 2 * cp);
+            const float2 dK = *reinterpret_cast<const float2 *>(fk + t * LDF + 2 * cp);
+            const uint32_t off_s = swz(t, 2 * cp, 256);
+            const uint32_t q2 = *reinterpret_cast<const uint32_t *>(sm + G_X + off_s);
+            const uint32_t k2 = *reinterpret_cast<const uint32_t *>(sm + G_Y + off_s);
+            const uint32_t b2 = *reinterpret_cast<const uint32_t *>(sm + G_DO + off_s);
+            const float q0 = bf_lo(q2), q1 = bf_hi(q2), k0 = bf_lo(k2), k1 = bf_hi(k2), b0 = bf_lo(b2), b1 = bf_hi(b2);
+            const float de0 = dE.x * eG[i].x, de1 = dE.y * eG[i].y;
+            dG[i].x = dQ.x * q0 * eG[i].x + de0 * b0 * k0 - dK.x * k0 * emG[i].x;
+            dG[i].y = dQ.y * q1 * eG[i].y + de1 * b1 * k1 - dK.y * k1 * emG[i].y;
+            if (t < L && ch_ok) {
+                const size_t off = base + (size_t)i * stride;
+                *reinterpret_cast<uint32_t *>(a.dq + off) = pack_bf16x2(dQ.x * eG[i].x, dQ.y * eG[i].y);
+                *reinterpret_cast<uint32_t *>(a.db + off) = pack_bf16x2(de0 * k0, de1 * k1);
+                *reinterpret_cast<uint32_t *>(a.dk + off) =
+                    pack_bf16x2(de0 * b0 + dK.x * emG[i].x, de1 * b1 + dK.y * emG[i].y);
             }
         }
-        if (q4 == 3) dG[15] += sDgf[c];  // gamma dgamma enters at the last row of the chunk
+        if (g8 == 7) {  // gamma dgamma enters at the last row of the chunk
+            dG[7].x += sDgf[2 * cp];
+            dG[7].y += sDgf[2 * cp + 1];
+        }
         // reverse cumulative sum inside the chunk
-        float run = 0.f;
+        float run0 = 0.f, run1 = 0.f;
 #pragma unroll
-        for (int i = 15; i >= 0; --i) {
-            run += dG[i];
-            dG[i] = run;
+        for (int i = 7; i >= 0; --i) {
+            run0 += dG[i].x;
+            run1 += dG[i].y;
+            dG[i] = make_float2(run0, run1);
         }
         __syncthreads();  // everyone has read sTot (forward cumsum) before it is reused
-        sTot[q4 * D + c] = run;
+        *reinterpret_cast<float2 *>(sTot + g8 * D + 2 * cp) = make_float2(run0, run1);
         __syncthreads();
-        float after = 0.f;
+        float after0 = 0.f, after1 = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (u > q4) after += sTot[u * D + c];
+        for (int u = 0; u < 8; ++u)
+            if (u > g8) {
+                after0 += sTot[u * D + 2 * cp];
+                after1 += sTot[u * D + 2 * cp + 1];
+            }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * q4 + i;
-            if (t < L && c < a.din) a.dg[tok_off(a, bb, hh, ci, t) + c] = dG[i] + after;
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            if (t < L && ch_ok)
+                *reinterpret_cast<float2 *>(a.dg + base + (size_t)i * stride) =
+                    make_float2(dG[i].x + after0, dG[i].y + after1);
         }
     }
 }
@@ -854,6 +940,11 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.dw = static_cast<__nv_bfloat16 *>(out.dw);
     a.dg = out.dg;
     a.dS0 = out.dS0;
+    {
+        int dev = 0;
+        a.n_sm = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&a.n_sm, cudaDevAttrMultiProcessorCount, dev);
+    }
 
     cudaError_t e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s);
     if (e != cudaSuccess) return e;
