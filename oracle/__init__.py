@@ -106,3 +106,49 @@ def ref_decode(q, k, v, g, b, w, S, nthreads=None):
     if rc != 0:
         raise RuntimeError(f"gdn2_ref_decode failed ({rc})")
     return o, S
+
+
+# ---------------------------------------------------------------- input prologue
+# The aixai.ru post's architecture paragraph ("Как это реализуется на практике"): queries and
+# keys are L2-normalised before the recurrent update, the erase and write gates come from
+# their own projections (logits through the logistic sigmoid, gates in [0, 1]), and log alpha
+# is computed outside the kernel (so it is an input of every function below).
+NORM_EPS = 1e-6
+
+
+def ref_prologue(q, k, b, w, norm=True, sigmoid=True):
+    """q, k -> x / sqrt(sum_c x^2 + NORM_EPS) per (token, head) over the last axis;
+    b, w -> 1 / (1 + exp(-x)) elementwise (any layout; None passes through).  fp64."""
+    q, k = _f64(q), _f64(k)
+    if norm:
+        q = q / np.sqrt((q * q).sum(-1, keepdims=True) + NORM_EPS)
+        k = k / np.sqrt((k * k).sum(-1, keepdims=True) + NORM_EPS)
+    if sigmoid:
+        b = None if b is None else 1.0 / (1.0 + np.exp(-_f64(b)))
+        w = None if w is None else 1.0 / (1.0 + np.exp(-_f64(w)))
+    return q, k, (None if b is None else _f64(b)), (None if w is None else _f64(w))
+
+
+def ref_fwd_prologue(q, k, v, g, b, w, S0=None, norm=True, sigmoid=True, nthreads=None):
+    """The forward on raw q, k and gate logits: ref_fwd after ref_prologue."""
+    qn, kn, bs, ws = ref_prologue(q, k, b, w, norm, sigmoid)
+    return ref_fwd(qn, kn, v, g, bs, ws, S0, nthreads)
+
+
+def ref_bwd_prologue(q, k, v, g, b, w, S0, do, dST=None, norm=True, sigmoid=True, nthreads=None):
+    """Gradients with respect to the raw q, k and the gate logits: ref_bwd at the normalised /
+    activated inputs, then the two derivatives of the prologue.  For x_n = x r with
+    r = (|x|^2 + eps)^-1/2, d x_n / d x = r (I - x_n x_n^T), so dx = r (dx_n - x_n (x_n . dx_n));
+    the sigmoid's derivative is s (1 - s)."""
+    qn, kn, bs, ws = ref_prologue(q, k, b, w, norm, sigmoid)
+    out = ref_bwd(qn, kn, v, g, bs, ws, S0, do, dST, nthreads)
+    if norm:
+        for x, key in ((_f64(q), "dq"), (_f64(k), "dk")):
+            r = 1.0 / np.sqrt((x * x).sum(-1, keepdims=True) + NORM_EPS)
+            xn = x * r
+            dxn = out[key]
+            out[key] = r * (dxn - xn * (xn * dxn).sum(-1, keepdims=True))
+    if sigmoid:
+        out["db"] = out["db"] * bs * (1.0 - bs)
+        out["dw"] = out["dw"] * ws * (1.0 - ws)
+    return out

@@ -34,7 +34,7 @@ def _l2norm(x: torch.Tensor) -> torch.Tensor:
 
 def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16",
                 seed: int = 0, s0: str = "normal", with_do: bool = False,
-                b_scale: float = 1.0, x_mean: float = -3.0, device: str = "cpu") -> dict:
+                b_scale: float = 1.0, x_mean: float = -3.0, device: str = "cpu", raw: bool = False) -> dict:
     """Draw one forward (or forward+backward) problem.
 
     Layouts: q, k, b, log_alpha are [B, T, H, Dk]; v, w, do are [B, T, H, Dv];
@@ -42,13 +42,17 @@ def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16"
     (2.0 gives b in [0, 2]); ``x_mean`` moves the decay logits (a larger
     value gives stronger decay).  ``device="cuda"`` draws the same
     distributions with a seeded CUDA generator (a different stream of numbers,
-    used for timing only, never for parity).
+    used for timing only, never for parity).  ``raw=True`` returns the same draws
+    before the input prologue: q, k unnormalised (N(0, 1) per channel) and b, w as
+    their N(0, 1) logits.
     """
     dt = DTYPES[dtype]
     gen = torch.Generator(device=device).manual_seed(seed)
     kw = dict(generator=gen, dtype=torch.float32, device=device)
-    q = _l2norm(torch.randn(B, T, H, Dk, **kw))
-    k = _l2norm(torch.randn(B, T, H, Dk, **kw))
+    q = torch.randn(B, T, H, Dk, **kw)
+    k = torch.randn(B, T, H, Dk, **kw)
+    if not raw:
+        q, k = _l2norm(q), _l2norm(k)
     v = torch.randn(B, T, H, Dv, **kw)
     x = torch.randn(B, T, H, Dk, **kw) + x_mean
     bl = torch.randn(B, T, H, Dk, **kw)
@@ -59,8 +63,8 @@ def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype: str = "bf16"
     out = {
         "q": q.to(dt), "k": k.to(dt), "v": v.to(dt),
         "log_alpha": -torch.nn.functional.softplus(x),
-        "b": (torch.sigmoid(bl) * b_scale).to(dt),
-        "w": torch.sigmoid(wl).to(dt),
+        "b": (bl if raw else torch.sigmoid(bl) * b_scale).to(dt),
+        "w": (wl if raw else torch.sigmoid(wl)).to(dt),
         "S0": S0,
     }
     if with_do:
@@ -80,10 +84,13 @@ class DecodeStream:
         # initial state first, so that erase acts from step one
         self.S0 = torch.randn(N, H, Dk, Dv, **self.kw) * 0.02
 
-    def step(self) -> dict:
+    def step(self, raw: bool = False) -> dict:
+        """One step's inputs; ``raw=True``: q, k unnormalised and b, w as logits."""
         N, H, Dk, Dv, kw = self.N, self.H, self.Dk, self.Dv, self.kw
-        q = _l2norm(torch.randn(N, H, Dk, **kw))
-        k = _l2norm(torch.randn(N, H, Dk, **kw))
+        q = torch.randn(N, H, Dk, **kw)
+        k = torch.randn(N, H, Dk, **kw)
+        if not raw:
+            q, k = _l2norm(q), _l2norm(k)
         v = torch.randn(N, H, Dv, **kw)
         x = torch.randn(N, H, Dk, **kw) - 3.0
         bl = torch.randn(N, H, Dk, **kw)
@@ -91,7 +98,7 @@ class DecodeStream:
         return {
             "q": q.to(self.dt), "k": k.to(self.dt), "v": v.to(self.dt),
             "log_alpha": -torch.nn.functional.softplus(x),
-            "b": torch.sigmoid(bl).to(self.dt), "w": torch.sigmoid(wl).to(self.dt),
+            "b": (bl if raw else torch.sigmoid(bl)).to(self.dt), "w": (wl if raw else torch.sigmoid(wl)).to(self.dt),
         }
 
 
