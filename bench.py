@@ -20,7 +20,10 @@ steps) and the roofline fraction of each, plus:
   (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen;
 * `scalar_decay`: the headline batch with one log decay per (token, head) through
   gdn2_chunk_fwd_gated (the tensor-core forward's scalar-decay path);
-* `d64`: the same model width with head size 64 (H = 32).
+* `d64`: the same model width with head size 64 (H = 32);
+* `prologue`: raw q, k and gate logits, with the input prologue (L2-normalised q, k;
+  sigmoid b, w) fused into the tensor-core forward, against the same prologue run as a
+  separate pass (gdn2_prologue) before the plain forward.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 independent (batch, head) sequences; there is no collective on the data path
@@ -407,6 +410,31 @@ def run_ours(args):
                                   "algorithmic_bytes": sd_bytes,
                                   "hbm_frac": round(sd_bytes / (ms_sd * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
         del wsg
+        # ---- input prologue fused in the chunk kernel, against a separate pass + the plain forward
+        xr = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=rank_seed(rank) + 31, device=str(dev), raw=True)
+        pro_flags = g.QK_L2NORM | g.BW_LOGITS
+        pro_out = {n: torch.empty_like(xr[n]) for n in ("q", "k", "b", "w")}
+
+        def fwd_pro():
+            g.gdn2_chunk_fwd_gated(xr["q"], xr["k"], xr["v"], xr["log_alpha"], xr["b"], xr["w"], xr["S0"],
+                                   flags=pro_flags, o=o, S_T=ST)
+
+        def fwd_unfused():
+            g.gdn2_prologue(xr["q"], xr["k"], xr["b"], xr["w"], flags=pro_flags, out=pro_out)
+            g.gdn2_chunk_fwd(pro_out["q"], pro_out["k"], xr["v"], xr["log_alpha"], pro_out["b"], pro_out["w"], xr["S0"],
+                             o=o, S_T=ST)
+
+        ms_pro = time_region(fwd_pro, 20, 3, stream) / 20
+        ms_unf = time_region(fwd_unfused, 20, 3, stream) / 20
+        assert g.gdn2_sync_status() == 0
+        fb_pro = fwd_bytes(B, T, H, D)
+        extras["prologue"] = {"workload": f"B={B}, T={T}, H={H}, d={D}; raw q, k and b, w logits",
+                              "fused_ms": round(ms_pro, 4), "unfused_ms": round(ms_unf, 4),
+                              "fused_tokens_per_s": round(job_rate(tokens, world, ms_pro), 1),
+                              "algorithmic_bytes": fb_pro,
+                              "fused_hbm_frac": round(fb_pro / (ms_pro * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                              "unfused_extra_bytes": 8 * B * T * H * D * xr["q"].element_size()}
+        del xr, pro_out
         # ---- head size 64 (same model width: H = 32), bf16, on the tensor-core forward
         x64 = make_inputs(B, T, 2 * H, D // 2, D // 2, dtype=w["dtype"], seed=rank_seed(rank) + 29, device=str(dev))
         o64 = torch.empty_like(x64["v"])

@@ -12,7 +12,9 @@ package is its thin Python binding.  Functions carry the C names:
   packed along the token axis (``cu_seqlens`` int32 [N+1] on the device)
 * ``gdn2_chunk_fwd_gated`` / ``gdn2_chunk_bwd_gated`` / ``gdn2_decode_step_gated``: gates given
   per channel, as per-(token, head) scalars, or absent (``flags``: DECAY_SCALAR, ERASE_SCALAR,
-  WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE)
+  WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE), and the input prologue (QK_L2NORM: raw q, k
+  normalised in the call; BW_LOGITS: b, w given as logits)
+* ``gdn2_prologue``: the input prologue alone (normalised q, k; sigmoid gates)
 * ``gdn2_workspace_size``, ``gdn2_sync_status``, ``gdn2_strerror``
 
 The library is loaded lazily by ``load()``; a missing library raises.
@@ -21,5 +23,5 @@ from ._lib import (EXPORTS, GDN2_BF16, GDN2_F32, GDN2_OK, LIB_PATH, NOALLOC_MAX_
                    STATUS_NAMES, Gdn2Error, gdn2_chunk_bwd, gdn2_chunk_bwd_noalloc, gdn2_chunk_bwd_varlen,
                    gdn2_chunk_fwd, gdn2_chunk_fwd_varlen, gdn2_chunk_fwd_gated, gdn2_chunk_bwd_gated,
                    gdn2_decode_step_gated, gdn2_workspace_size_gated, DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR,
-                   DECAY_NONE, ERASE_NONE, WRITE_NONE, gdn2_decode_step, gdn2_strerror, gdn2_sync_status,
+                   DECAY_NONE, ERASE_NONE, WRITE_NONE, QK_L2NORM, BW_LOGITS, gdn2_decode_step, gdn2_prologue, gdn2_strerror, gdn2_sync_status,
                    gdn2_workspace_size, load, raw)

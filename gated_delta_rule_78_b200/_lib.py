@@ -24,9 +24,11 @@ GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
            "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
            "gdn2_chunk_bwd_varlen", "gdn2_chunk_fwd_gated", "gdn2_chunk_bwd_gated", "gdn2_decode_step_gated",
-           "gdn2_workspace_size_gated")
+           "gdn2_workspace_size_gated", "gdn2_prologue")
 # gate layout flags (gdn2_gate_flags in include/gdn2.h)
 DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE = 1, 2, 4, 8, 16, 32
+# input prologue: q, k L2-normalised in the call; b, w given as logits (sigmoid in the call)
+QK_L2NORM, BW_LOGITS = 64, 128
 # Size of the library's static scratch array used by gdn2_chunk_bwd_noalloc
 # (GDN2_NOALLOC_MAX_SCRATCH_BYTES in include/gdn2.h).
 NOALLOC_MAX_SCRATCH_BYTES = 32 << 20
@@ -69,6 +71,8 @@ def load(path: str | None = None):
     lib.gdn2_chunk_bwd_gated.restype = i
     lib.gdn2_decode_step_gated.argtypes = [i] * 6 + [vp] * 9 + [sz, vp]
     lib.gdn2_decode_step_gated.restype = i
+    lib.gdn2_prologue.argtypes = [i] * 5 + [vp] * 8 + [vp]
+    lib.gdn2_prologue.restype = i
     lib.gdn2_workspace_size_gated.argtypes = [i] * 8
     lib.gdn2_workspace_size_gated.restype = sz
     lib.gdn2_workspace_size.argtypes = [i] * 7
@@ -360,6 +364,29 @@ def gdn2_decode_step_gated(q, k, v, log_alpha, b, w, S, *, flags, o=None, worksp
                                       _p(S), _p(o), _p(ws), nb, _stream(stream))
     _check("gdn2_decode_step_gated", st)
     return o
+
+
+def gdn2_prologue(q, k, b, w, *, flags, out=None, stream=None):
+    """The input prologue alone: returns dict(q, k, b, w) with q, k normalised (QK_L2NORM) and
+    b, w through the sigmoid (BW_LOGITS); parts the flags do not ask for come back as None.
+    q, k: [..., H, D]; b, w: [..., H, D] or, with ERASE_SCALAR / WRITE_SCALAR, [..., H]."""
+    H, D = q.shape[-2], q.shape[-1]
+    N = q.numel() // (H * D)
+    dt = _dt(q)
+    norm = bool(flags & QK_L2NORM)
+    sig_b = bool(flags & BW_LOGITS) and not flags & ERASE_NONE
+    sig_w = bool(flags & BW_LOGITS) and not flags & WRITE_NONE
+    for n, t, used in (("q", q, norm), ("k", k, norm), ("b", b, sig_b), ("w", w, sig_w)):
+        if used:
+            _cuda_contig(n, t, q.dtype)
+    if out is None:
+        out = {"q": torch.empty_like(q) if norm else None, "k": torch.empty_like(k) if norm else None,
+               "b": torch.empty_like(b) if sig_b else None, "w": torch.empty_like(w) if sig_w else None}
+    st = raw().gdn2_prologue(flags, dt, N, H, D, _p(q if norm else None), _p(k if norm else None),
+                             _p(b if sig_b else None), _p(w if sig_w else None), _p(out["q"]), _p(out["k"]),
+                             _p(out["b"]), _p(out["w"]), _stream(stream))
+    _check("gdn2_prologue", st)
+    return out
 
 
 def gdn2_sync_status(stream=None) -> int:

@@ -41,6 +41,8 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "gdn2_internal.cuh"
 #include "tc_util.cuh"
 #include "warp_mma.cuh"
@@ -67,7 +69,9 @@ constexpr uint32_t OFF_SA = 180224;     // A fp32 [64][LDA]
 constexpr uint32_t OFF_ST = OFF_SA + 64 * LDA * 4;   // T fp32 [64][LDA]
 constexpr uint32_t OFF_TOT = OFF_ST + 64 * LDA * 4;  // per-group decay totals [4][128] fp32
 constexpr uint32_t OFF_GAM = OFF_TOT + 4 * 128 * 4;  // gamma [2][128] fp32
-constexpr uint32_t SMEM_USED = OFF_GAM + 2 * 128 * 4;
+constexpr uint32_t OFF_NRM = OFF_GAM + 2 * 128 * 4;  // prologue: sum of squares [q|k][channel half][64] fp32
+constexpr uint32_t OFF_RN = OFF_NRM + 2 * 2 * 64 * 4;  // prologue: 1/|q|, 1/|k| [2][q|k][64] fp32
+constexpr uint32_t SMEM_USED = OFF_RN + 2 * 2 * 64 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for the 1024-byte alignment
 
 // TMEM columns
@@ -123,12 +127,50 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b)
     return r;
 }
 
+// logistic sigmoid through the tanh unit: 1 / (1 + e^-x) = (1 + tanh(x / 2)) / 2,
+// on a bf16x2 pair: the tanh unit's bf16x2 form, then 1/2 + t/2 as one bf16x2 fma (x/2 is exact)
+__device__ __forceinline__ uint32_t sigmoid_bf16x2(uint32_t x)
+{
+    const uint32_t half2 = 0x3f003f00u;  // (0.5, 0.5) in bf16
+    uint32_t h, t, r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(h) : "r"(x), "r"(half2));
+    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
+    asm("fma.rn.bf16x2 %0, %1, %2, %2;" : "=r"(r) : "r"(t), "r"(half2));
+    return r;
+}
+
+// Sum over the 32 lanes of each of 16 per-lane values v[0..15], by halving exchanges (16
+// shuffles instead of 80): on return lanes 2i and 2i + 1 hold the total of value i in v[0].
+__device__ __forceinline__ void lane_sum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int m = 16, n = 8; m >= 2; m >>= 1, n >>= 1) {
+        const bool up = lane & m;
+#pragma unroll
+        for (int j = 0; j < n; ++j) {
+            const float send = up ? v[j] : v[j + n];
+            const float keep = up ? v[j + n] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 // kGScalar: log alpha is one value per (token, head) (TcParams::g_scalar).
 // DIN: the head size of the tensors, 128 or 64.  A d = 64 head runs as a d = 128 head
 // whose channels 64..127 are zero: the TMA boxes past the tensors' channel extent are
 // zero-filled, so k, q, b, v and w vanish there, the state's extra rows and columns stay
 // zero, and only the first 64 channels of o, S_T are stored.
-template <bool kGScalar, int DIN>
+// kPro: the fused input prologue (kProNorm | kProSigmoid of gdn2_internal.cuh).  With
+// normalised q_n = R_q q, k_n = R_k k (R = Diag of the per-token reciprocal norms) the chunk
+// step keeps the raw-key factors and moves the scales.  The normalised A is R_k A R_k, and
+// (I + R_k A R_k)^-1 = R_k^-1 (I + R_k^2 A)^-1 R_k, so with T'' = (I + R_k^2 A)^-1 (A's rows
+// scaled at the readback) the product the state update K~^T U' and P U' both take is
+// U' = R_k U~_n = T'' (R_k X - R_k^2 E~ S); the output is O = R_q (Q~ S + P U').  The
+// squares come from the decay folding's loads; the reduction over the lanes runs while the
+// [A; P] product is in flight.  The sigmoid of b is applied in the decay folding, that of w
+// in the X = w.v fold.
+template <bool kGScalar, int DIN, int kPro>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -161,6 +203,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     float *sT = reinterpret_cast<float *>(sm + OFF_ST);
     float *sTot = reinterpret_cast<float *>(sm + OFF_TOT);
     float *sGam = reinterpret_cast<float *>(sm + OFF_GAM);
+    float *sNrm = reinterpret_cast<float *>(sm + OFF_NRM);  // [q|k][channel half][64]
+    float *sRn = reinterpret_cast<float *>(sm + OFF_RN);    // [parity][q|k][64]
 
     if (tid == 0) {
         s_abort_m = 0;
@@ -228,7 +272,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 const uint32_t off = a * 8192 + sw128(t, 4 * lane);
                 const uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
                 const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
-                *reinterpret_cast<uint32_t *>(pv + off) = (t < Lc) ? bmul2(vw, ww) : 0u;
+                const uint32_t wg = (kPro & kProSigmoid) ? sigmoid_bf16x2(ww) : ww;
+                *reinterpret_cast<uint32_t *>(pv + off) = (t < Lc) ? bmul2(vw, wg) : 0u;
             }
         };
         if (tid == 0 && nchunks > 0) issue(0);
@@ -288,6 +333,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             {  // Y^T = X^T - S^T E~^T -> bf16 TMEM operand (this warp: 32 tokens)
                 const uint8_t *px = sm + ov + (jrow >> 6) * 8192;
                 const uint32_t xb = (jrow & 63) * 2;
+                const float *rk = sRn + (buf * 2 + 1) * 64;
                 uint32_t r[32];
                 tmem_ld32(tmem + TM_YO + 32 * half + lane_off, r);
                 tmem_wait_ld();
@@ -297,7 +343,13 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     const int t = 32 * half + 2 * e;
                     const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t, xb)));
                     const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t + 1, xb)));
-                    pk[e] = pack_bf16x2(x0 - __uint_as_float(r[2 * e]), x1 - __uint_as_float(r[2 * e + 1]));
+                    const float a0 = __uint_as_float(r[2 * e]), a1 = __uint_as_float(r[2 * e + 1]);
+                    if (kPro & kProNorm) {  // R_k X - R_k^2 E~ S
+                        const float r0 = rk[t], r1 = rk[t + 1];
+                        pk[e] = pack_bf16x2(r0 * (x0 - r0 * a0), r1 * (x1 - r1 * a1));
+                    } else {
+                        pk[e] = pack_bf16x2(x0 - a0, x1 - a1);
+                    }
                 }
                 tmem_st16(tmem + TM_YB + 16 * half + lane_off, pk);
                 tmem_wait_st();
@@ -317,7 +369,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             if (!mbar_wait(&bar_mma, mma_phase)) fail();
             mma_phase ^= 1;
             tc_fence_after();
-            {  // U~^T -> bf16 TMEM operand
+            {  // U~^T (U' with the prologue) -> bf16 TMEM operand
                 uint32_t r[32];
                 tmem_ld32(tmem + TM_UT + 32 * half + lane_off, r);
                 tmem_wait_ld();
@@ -367,9 +419,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 tmem_wait_ld();
                 __nv_bfloat16 *so = reinterpret_cast<__nv_bfloat16 *>(sm + ott);
                 if (jrow < DIN) {  // row-major [t][channel] with the tensors' head size as row length
+                    const float *rq = sRn + (buf * 2) * 64 + 32 * half;
 #pragma unroll
-                    for (int u = 0; u < 32; ++u)
-                        so[(32 * half + u) * DIN + jrow] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                    for (int u = 0; u < 32; ++u) {
+                        const float ov_ = (kPro & kProNorm) ? __uint_as_float(r[u]) * rq[u] : __uint_as_float(r[u]);
+                        so[(32 * half + u) * DIN + jrow] = __float2bfloat16_rn(ov_);
+                    }
                 }
             }
             tmem_wait_st();
@@ -453,6 +508,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
             named_sync(2, kGroup);
             if (s_abort_e) break;
+            float sqq[16], sqk[16];  // prologue: this thread's share of |q|^2, |k|^2 per token
             {  // decay folding, in place
                 float c0 = 0.f, c1 = 0.f, gl0 = 0.f, gl1 = 0.f;
 #pragma unroll
@@ -488,7 +544,14 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
                     uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
                     if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
+                    if (kPro & kProNorm) {
+                        const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
+                        const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xffff0000u);
+                        sqq[i] = fmaf(q0, q0, q1 * q1);
+                        sqk[i] = fmaf(k0, k0, k1 * k1);
+                    }
                     const uint32_t e01 = pack_bf16x2(e0, e1), m01 = pack_bf16x2(m0, m1);
+                    if (kPro & kProSigmoid) bw = sigmoid_bf16x2(bw);  // kw is 0 past the sequence end
                     *reinterpret_cast<uint32_t *>(pq + off) = bmul2(qw, e01);
                     *reinterpret_cast<uint32_t *>(pe + off) = bmul2(bmul2(bw, kw), e01);
                     *reinterpret_cast<uint32_t *>(pk + off) = bmul2(kw, m01);
@@ -505,6 +568,15 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                            sdesc_sw128(sbase + ok + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_N64, ks > 0);
                 mma_commit(&bar_emma);
             }
+            if (kPro & kProNorm) {  // while the product runs: |q|^2, |k|^2 of this chunk's tokens
+                lane_sum16(sqq, lane);
+                lane_sum16(sqk, lane);
+                if (!(lane & 1)) {
+                    sNrm[cb * 64 + 16 * tg + (lane >> 1)] = sqq[0];
+                    sNrm[(2 + cb) * 64 + 16 * tg + (lane >> 1)] = sqk[0];
+                }
+                named_sync(2, kGroup);
+            }
             if (!mbar_wait(&bar_emma, ci & 1)) fail();
             tc_fence_after();
             {  // A -> fp32 scratch (strictly lower), P -> bf16 operand rows (lower incl.)
@@ -512,11 +584,19 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
                 tmem_wait_ld();
                 const int row = quarter * 32 + lane;
+                float rr2 = 1.f;  // prologue: 1/|k_row|^2 (A rows)
+                if (kPro & kProNorm) {
+                    const int which = row < 64 ? 1 : 0, t = row & 63;
+                    const float n2 = sNrm[(which * 2) * 64 + t] + sNrm[(which * 2 + 1) * 64 + t] + kNormEps;
+                    rr2 = __frcp_rn(n2);
+                    if (half == 0) sRn[(buf * 2 + which) * 64 + t] = rsqrtf(n2);  // for M: 1/|k|, 1/|q|
+                }
                 if (row < 64) {
 #pragma unroll
                     for (int u = 0; u < 32; ++u) {
                         const int j = 32 * half + u;
-                        sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
+                        const float av = (kPro & kProNorm) ? __uint_as_float(r[u]) * rr2 : __uint_as_float(r[u]);
+                        sA[row * LDA + j] = (j < row) ? av : 0.f;
                     }
                 } else {
                     const int t = row - 64;
@@ -638,8 +718,23 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
         return cudaGetLastError();
     };
-    if (din == 128) return pr.g_scalar ? run(fwd_tc_kernel<true, 128>) : run(fwd_tc_kernel<false, 128>);
-    return pr.g_scalar ? run(fwd_tc_kernel<true, 64>) : run(fwd_tc_kernel<false, 64>);
+    if (pr.prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
+    auto by_pro = [&](auto gs, auto dn) -> cudaError_t {
+        constexpr bool kGS = decltype(gs)::value;
+        constexpr int kDin = decltype(dn)::value;
+        switch (pr.prologue) {
+        case kProNorm: return run(fwd_tc_kernel<kGS, kDin, kProNorm>);
+        case kProSigmoid: return run(fwd_tc_kernel<kGS, kDin, kProSigmoid>);
+        case kProNorm | kProSigmoid: return run(fwd_tc_kernel<kGS, kDin, kProNorm | kProSigmoid>);
+        default: return run(fwd_tc_kernel<kGS, kDin, 0>);
+        }
+    };
+    using T1 = std::true_type;
+    using F1 = std::false_type;
+    using D128 = std::integral_constant<int, 128>;
+    using D64 = std::integral_constant<int, 64>;
+    if (din == 128) return pr.g_scalar ? by_pro(T1{}, D128{}) : by_pro(F1{}, D128{});
+    return pr.g_scalar ? by_pro(T1{}, D64{}) : by_pro(F1{}, D64{});
 }
 
 }  // namespace gdn2

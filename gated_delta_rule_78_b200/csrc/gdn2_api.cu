@@ -1,5 +1,6 @@
 // C ABI of libgdn2.so: argument validation, workspace sizing, kernel dispatch.
 // Declarations and the contract of every entry point are in include/gdn2.h.
+#include <vector>
 #include <stdint.h>
 
 #include <mutex>
@@ -113,7 +114,7 @@ bool gate_full(int flags, int i) { return !gate_scalar(flags, i) && !gate_none(f
 
 gdn2_status check_gate_flags(int flags)
 {
-    if (flags & ~0x3F) return GDN2_ERR_UNSUPPORTED;
+    if (flags & ~0xFF) return GDN2_ERR_UNSUPPORTED;
     for (int i = 0; i < 3; ++i)
         if (gate_scalar(flags, i) && gate_none(flags, i)) return GDN2_ERR_UNSUPPORTED;
     return GDN2_OK;
@@ -121,16 +122,38 @@ gdn2_status check_gate_flags(int flags)
 
 size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 
-// [expanded g | b | w] [full-size gradients of dg | db | dw (backward)] [core workspace]
+// The input prologue: GDN2_QK_L2NORM normalises q and k, GDN2_BW_LOGITS takes b and w (where
+// present) as logits.  The bf16 forward with per-channel b and w applies it inside the
+// tensor-core kernel; every other call runs it as a pass into the workspace first.
+bool pro_any(int flags) { return flags & (GDN2_QK_L2NORM | GDN2_BW_LOGITS); }
+bool pro_fused(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_full(flags, 1) && gate_full(flags, 2); }
+// prologue mode of gate i (1 = b, 2 = w): 0 none, 1 per channel, 2 per token
+int pro_gate_mode(int flags, int i)
+{
+    if (!(flags & GDN2_BW_LOGITS) || gate_none(flags, i)) return 0;
+    return gate_scalar(flags, i) ? 2 : 1;
+}
+
+// [prologue outputs q_n | k_n | b_s | w_s] [expanded g | b | w]
+// [full-size gradients of dg | db | dw (backward)] [core workspace]
 struct GatedWs {
-    size_t off[3], grad[3], core, total;
+    size_t pro[4], off[3], grad[3], core, total;
 };
-GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes)
+GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes, bool pro_pass)
 {
     GatedWs l;
     const size_t n = rows * H * D;
     const size_t es[3] = {4, dt == GDN2_F32 ? 4u : 2u, dt == GDN2_F32 ? 4u : 2u};
     size_t off = 0;
+    for (int i = 0; i < 4; ++i) {
+        l.pro[i] = off;
+        if (!pro_pass) continue;
+        if (i < 2 && (flags & GDN2_QK_L2NORM)) off += round256(n * es[1]);
+        if (i >= 2) {
+            const int m = pro_gate_mode(flags, i - 1);
+            if (m) off += round256((m == 1 ? n : rows * H) * es[1]);
+        }
+    }
     for (int i = 0; i < 3; ++i) {
         l.off[i] = off;
         if (!gate_full(flags, i)) off += round256(n * es[i]);
@@ -158,6 +181,26 @@ gdn2_status expand_gates(int flags, gdn2_dtype dt, const GatedWs &l, char *ws, s
         if (e != cudaSuccess) return GDN2_ERR_CUDA;
         gp[i] = dst;
     }
+    return GDN2_OK;
+}
+
+// The prologue as a pass: q, k, b, w are replaced by the normalised / activated copies.
+gdn2_status prologue_pass(int flags, gdn2_dtype dt, const GatedWs &l, char *ws, size_t rows, int H, int D,
+                          const void *&q, const void *&k, const void *&b, const void *&w, cudaStream_t s)
+{
+    const bool norm = flags & GDN2_QK_L2NORM;
+    const int bm = pro_gate_mode(flags, 1), wm = pro_gate_mode(flags, 2);
+    void *qn = norm ? ws + l.pro[0] : nullptr, *kn = norm ? ws + l.pro[1] : nullptr;
+    void *bs = bm ? ws + l.pro[2] : nullptr, *wsg = wm ? ws + l.pro[3] : nullptr;
+    if (gdn2::launch_prologue_fwd(dt == GDN2_F32, rows * H, D, norm, q, k, qn, kn, bm, b, bs, wm, w, wsg, s) !=
+        cudaSuccess)
+        return GDN2_ERR_CUDA;
+    if (norm) {
+        q = qn;
+        k = kn;
+    }
+    if (bm) b = bs;
+    if (wm) w = wsg;
     return GDN2_OK;
 }
 
@@ -330,13 +373,14 @@ size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int
     if (check_gate_flags(flags) != GDN2_OK) return 0;
     if (which == 2) {  // decode: B sequences of one token
         if (check_sizes(dt, B, 1, H, Dk, Dv) != GDN2_OK) return 0;
-        return gated_ws(false, flags, dt, (size_t)B, H, Dk, 0).total;
+        return gated_ws(false, flags, dt, (size_t)B, H, Dk, 0, pro_any(flags)).total;
     }
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK || T == 0 || (which != 0 && which != 1)) return 0;
     const size_t core = which == 1 ? gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr,
                                                                                 nullptr, nullptr, nullptr, nullptr))
                                    : 0;
-    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core).total;
+    const bool pro_pass = pro_any(flags) && (which == 1 || !pro_fused(flags, dt));
+    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass).total;
 }
 
 gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
@@ -349,19 +393,26 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if (T == 0) return gdn2_chunk_fwd(dt, B, 0, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, o, S_T, nullptr, 0, stream);
     if ((st = check_ptrs({q, k, v, o}, {S0, S_T})) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
-    const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0);
+    const bool fused = pro_any(flags) && pro_fused(flags, dt);
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0, pro_any(flags) && !fused);
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
-    // a scalar decay goes to the tensor-core forward as it is (one exponential pair per token)
+    char *ws = static_cast<char *>(workspace);
+    const void *qq = q, *kk = k, *bq = b, *wq = w;
+    if (pro_any(flags) && !fused &&
+        (st = prologue_pass(flags, dt, l, ws, (size_t)B * T, H, Dk, qq, kk, bq, wq, s)) != GDN2_OK)
+        return st;
+    // a scalar decay goes to the tensor-core forward as it is (one exponential per token)
     const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16;
     const int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
-    const void *gp[3] = {log_alpha, b, w};
-    if ((st = expand_gates(expand_flags, dt, l, static_cast<char *>(workspace), (size_t)B * T, H, Dk, gp, s)) != GDN2_OK)
-        return st;
-    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S0);
-    if (native_decay) {
-        p.g_scalar = true;
+    const void *gp[3] = {log_alpha, bq, wq};
+    if ((st = expand_gates(expand_flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s)) != GDN2_OK) return st;
+    gdn2::Problem p = make_problem(B, T, H, Dk, qq, kk, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S0);
+    if (native_decay || fused) {
+        p.g_scalar = native_decay;
+        if (fused)
+            p.prologue = ((flags & GDN2_QK_L2NORM) ? gdn2::kProNorm : 0) | ((flags & GDN2_BW_LOGITS) ? gdn2::kProSigmoid : 0);
         int *status = gdn2::status_word();
         if (!status) return GDN2_ERR_CUDA;
         return from_cuda(gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s));
@@ -385,12 +436,17 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, dlog_alpha, db, dw)) != GDN2_OK) return st;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
-    const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p));
+    const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p), pro_any(flags));
     if (!workspace || ws_bytes < l.total) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
     char *ws = static_cast<char *>(workspace);
-    const void *gp[3] = {log_alpha, b, w};
+    const void *qq = q, *kk = k, *bq = b, *wq = w;
+    if (pro_any(flags) && (st = prologue_pass(flags, dt, l, ws, (size_t)B * T, H, Dk, qq, kk, bq, wq, s)) != GDN2_OK)
+        return st;
+    p.q = qq;
+    p.k = kk;
+    const void *gp[3] = {log_alpha, bq, wq};
     if ((st = expand_gates(flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s)) != GDN2_OK) return st;
     p.g = static_cast<const float *>(gp[0]);
     p.b = gp[1];
@@ -407,6 +463,10 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
         if (gdn2::launch_channel_sum(fp32, grads[i], user[i], (size_t)B * T * H, Dk, s) != cudaSuccess)
             return GDN2_ERR_CUDA;
     }
+    if (pro_any(flags) &&  // back through the prologue, in place, against the raw inputs
+        gdn2::launch_prologue_bwd(dt == GDN2_F32, (size_t)B * T * H, Dk, flags & GDN2_QK_L2NORM, q, k, dq, dk,
+                                  pro_gate_mode(flags, 1), b, db, pro_gate_mode(flags, 2), w, dw, s) != cudaSuccess)
+        return GDN2_ERR_CUDA;
     return GDN2_OK;
 }
 
@@ -419,15 +479,41 @@ gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int H, int D
     if ((st = check_sizes(dt, N, 1, H, Dk, Dv)) != GDN2_OK) return st;
     if ((st = check_ptrs({q, k, v, S, o}, {})) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
-    const GatedWs l = gated_ws(false, flags, dt, (size_t)N, H, Dk, 0);
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)N, H, Dk, 0, pro_any(flags));
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
-    const void *gp[3] = {log_alpha, b, w};
-    if ((st = expand_gates(flags, dt, l, static_cast<char *>(workspace), (size_t)N, H, Dk, gp, s)) != GDN2_OK)
+    char *ws = static_cast<char *>(workspace);
+    const void *qq = q, *kk = k, *bq = b, *wq = w;
+    if (pro_any(flags) && (st = prologue_pass(flags, dt, l, ws, (size_t)N, H, Dk, qq, kk, bq, wq, s)) != GDN2_OK)
         return st;
-    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, q, k, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S, o,
+    const void *gp[3] = {log_alpha, bq, wq};
+    if ((st = expand_gates(flags, dt, l, ws, (size_t)N, H, Dk, gp, s)) != GDN2_OK) return st;
+    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, qq, kk, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S, o,
                                          s));
+}
+
+gdn2_status gdn2_prologue(int flags, gdn2_dtype dt, int N, int H, int D, const void *q, const void *k, const void *b,
+                          const void *w, void *q_n, void *k_n, void *b_s, void *w_s, void *stream)
+{
+    gdn2_status st = check_gate_flags(flags);
+    if (st != GDN2_OK) return st;
+    if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
+    if (N < 0 || H < 1) return GDN2_ERR_SHAPE;
+    if (D != 64 && D != 128) return GDN2_ERR_UNSUPPORTED;
+    const bool norm = flags & GDN2_QK_L2NORM;
+    const int bm = pro_gate_mode(flags, 1), wm = pro_gate_mode(flags, 2);
+    std::vector<const void *> need;
+    if (norm) need.insert(need.end(), {q, k, q_n, k_n});
+    if (bm) need.insert(need.end(), {b, b_s});
+    if (wm) need.insert(need.end(), {w, w_s});
+    for (const void *ptr : need) {
+        if (!ptr) return GDN2_ERR_NULL;
+        if (!aligned16(ptr)) return GDN2_ERR_ALIGN;
+    }
+    if (N == 0) return GDN2_OK;
+    return from_cuda(gdn2::launch_prologue_fwd(dt == GDN2_F32, (size_t)N * H, D, norm, q, k, q_n, k_n, bm, b, b_s, wm,
+                                               w, w_s, (cudaStream_t)stream));
 }
 
 gdn2_status gdn2_sync_status(void *stream)

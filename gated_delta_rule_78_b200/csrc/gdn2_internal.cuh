@@ -41,7 +41,14 @@ struct Problem {
     const int *cu_seqlens = nullptr;
     const int *chunk_off = nullptr;
     bool g_scalar = false;  // tensor-core forward only: log alpha is [rows, H] (one decay per head)
+    int prologue = 0;       // tensor-core forward only: kProNorm | kProSigmoid, applied inside the kernel
 };
+
+// Fused input prologue (tensor-core forward): q and k are L2-normalised per token and head,
+// x / sqrt(sum x^2 + kNormEps); b and w are logits and pass through the logistic sigmoid.
+constexpr int kProNorm = 1;
+constexpr int kProSigmoid = 2;
+constexpr float kNormEps = 1e-6f;
 
 // rows of the token tensors
 __host__ __device__ inline size_t token_rows(const Problem &p)
@@ -106,6 +113,14 @@ cudaError_t set_smem_attr(const void *kernel, int bytes);
 // the shape is outside what the kernel handles.  `o` may be null (no output);
 // `states`, when non-null, receives S^T in bf16 at every chunk boundary:
 // [B*H][nchunks + 1][D][D], entry c the state before chunk c, the last entry S_T.
+// The input prologue as separate passes (prologue.cu).  rows = token rows x heads; gate modes:
+// 0 untouched, 1 per channel ([rows, D]), 2 per token ([rows]).
+cudaError_t launch_prologue_fwd(bool fp32, size_t rows, int D, bool norm, const void *q, const void *k, void *qn,
+                                void *kn, int b_mode, const void *b, void *bs, int w_mode, const void *w, void *ws,
+                                cudaStream_t s);
+cudaError_t launch_prologue_bwd(bool fp32, size_t rows, int D, bool norm, const void *q, const void *k, void *dq,
+                                void *dk, int b_mode, const void *b, void *db, int w_mode, const void *w, void *dw,
+                                cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s);
 

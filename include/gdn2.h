@@ -194,10 +194,23 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
  * per-channel tensors: the library broadcasts them into the workspace and runs the
  * same kernels.  In the backward the gradient of a scalar gate is the sum of the
  * per-channel gradients over the channels.  An absent gate's gradient pointer is
- * ignored (NULL allowed).  Flags outside the six below, or scalar and absent set
+ * ignored (NULL allowed).  Flags outside the eight below, or scalar and absent set
  * for one gate, give GDN2_ERR_UNSUPPORTED.
  * Workspace: gdn2_workspace_size_gated(which, flags, ...) with which = 0 (forward),
  * 1 (backward), 2 (decode; B = N, T ignored).  Fixed-length batches only.
+ *
+ * Input prologue (two more flags, combinable with the layouts above).  The aixai.ru
+ * post's architecture paragraph normalises queries and keys before the recurrent update
+ * and takes the erase and write gates from their own projections; log alpha is computed
+ * outside the kernel, so it stays an input here.
+ *   GDN2_QK_L2NORM: q and k are raw; each token's q and k (per head, over the head
+ *     dimension) is replaced by x / sqrt(sum x^2 + 1e-6) in fp32.
+ *   GDN2_BW_LOGITS: b and w, where present, are logits (either layout) and pass through
+ *     the logistic sigmoid 1 / (1 + e^-x).
+ * The bf16 forward with per-channel b and w applies both inside the tensor-core chunk
+ * kernel (the sigmoid there goes through the hardware tanh, 1/2 + tanh(x/2)/2); every
+ * other call writes the normalised / activated inputs into its workspace first.  The
+ * backward returns dq, dk for the raw q, k and db, dw for the logits.
  */
 typedef enum {
     GDN2_DECAY_SCALAR = 1,
@@ -205,7 +218,9 @@ typedef enum {
     GDN2_WRITE_SCALAR = 4,
     GDN2_DECAY_NONE = 8,
     GDN2_ERASE_NONE = 16,
-    GDN2_WRITE_NONE = 32
+    GDN2_WRITE_NONE = 32,
+    GDN2_QK_L2NORM = 64,
+    GDN2_BW_LOGITS = 128
 } gdn2_gate_flags;
 
 GDN2_API gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
@@ -226,6 +241,21 @@ GDN2_API gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int
                            void *workspace, size_t ws_bytes, void *stream);
 
 GDN2_API size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv);
+
+/* The input prologue on its own (the pass the gated calls run before the recurrence where
+ * it is not fused): for N token rows of H heads and head size D, writes
+ *   q_n, k_n = x / sqrt(sum x^2 + 1e-6) per (row, head)      (flags & GDN2_QK_L2NORM)
+ *   b_s, w_s = 1 / (1 + e^-x)                               (flags & GDN2_BW_LOGITS)
+ * with b and w per channel [N, H, D] or per token [N, H] as GDN2_ERASE_SCALAR /
+ * GDN2_WRITE_SCALAR say, or skipped with GDN2_ERASE_NONE / GDN2_WRITE_NONE.  Inputs and
+ * outputs have dtype dt (bf16 results are rounded once from fp32); outputs that the flags
+ * do not ask for may be NULL.  Decay flags are ignored.  Asynchronous on `stream`.
+ * Errors: GDN2_ERR_SHAPE for N < 0 or H < 1, GDN2_ERR_UNSUPPORTED for D not 64 or 128 or
+ * unknown flags, GDN2_ERR_NULL / GDN2_ERR_ALIGN for a missing or unaligned tensor that the
+ * flags need. */
+GDN2_API gdn2_status gdn2_prologue(int flags, gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
+                                   const void *b, const void *w, void *q_n, void *k_n, void *b_s, void *w_s,
+                                   void *stream);
 
 /* Workspace bytes for which = 0 (gdn2_chunk_fwd), 1 (gdn2_chunk_bwd),
  * 2 (gdn2_chunk_fwd_varlen) or 3 (gdn2_chunk_bwd_varlen, B = N, T = total_T);

@@ -115,7 +115,7 @@ def fwd_g(lib, flags, g=P, b=P, w=P, ws=P, ws_bytes=1 << 40):
 
 
 def test_gated_flags_and_workspace(lib):
-    assert fwd_g(lib, 64) == -8                       # unknown flag bit
+    assert fwd_g(lib, 256) == -8                      # unknown flag bit
     assert fwd_g(lib, g.ERASE_SCALAR | g.ERASE_NONE) == -8  # scalar and absent for one gate
     assert fwd_g(lib, g.ERASE_SCALAR, b=NUL) == -1     # a scalar gate needs its tensor
     assert fwd_g(lib, g.ERASE_SCALAR, ws=NUL) == -5    # and a workspace to broadcast it into
@@ -127,7 +127,16 @@ def test_gated_flags_and_workspace(lib):
     plain = lib.gdn2_workspace_size(1, BF16, 2, 128, 4, 128, 128)
     assert lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR | g.WRITE_SCALAR, BF16, 2, 128, 4, 128, 128) == plain + 4 * one
     assert lib.gdn2_workspace_size_gated(2, g.ERASE_SCALAR, BF16, 8, 0, 4, 128, 128) == 8 * 4 * 128 * 2
-    assert lib.gdn2_workspace_size_gated(0, 64, BF16, 2, 128, 4, 128, 128) == 0
+    # input prologue: fused in the bf16 forward with per-channel gates (no workspace); a pass
+    # into the workspace (q_n, k_n, b_s, w_s) everywhere else
+    pro = g.QK_L2NORM | g.BW_LOGITS
+    assert lib.gdn2_workspace_size_gated(0, pro, BF16, 2, 128, 4, 128, 128) == 0
+    assert lib.gdn2_workspace_size_gated(0, g.QK_L2NORM, BF16, 2, 128, 4, 128, 128) == 0
+    assert lib.gdn2_workspace_size_gated(0, pro, F32, 2, 128, 4, 64, 64) == 4 * (2 * 128 * 4 * 64 * 4)
+    assert lib.gdn2_workspace_size_gated(1, pro, BF16, 2, 128, 4, 128, 128) == plain + 4 * one
+    # scalar b logits: q_n, k_n, per-token b_s, w_s, then the broadcast b
+    assert lib.gdn2_workspace_size_gated(0, pro | g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == 4 * one + 2 * 128 * 4 * 2
+    assert lib.gdn2_workspace_size_gated(2, g.QK_L2NORM, BF16, 8, 0, 4, 128, 128) == 2 * 8 * 4 * 128 * 2
 
 
 def test_workspace_size(lib):
@@ -150,3 +159,21 @@ def test_missing_library_fails_loudly(tmp_path):
             mod.load(str(tmp_path / "nope.so"))
     finally:
         mod._lib = saved
+
+
+def pro(lib, flags=g.QK_L2NORM | g.BW_LOGITS, dt=BF16, N=4, H=2, D=128, q=P, b=P, qn=P):
+    return lib.gdn2_prologue(flags, dt, N, H, D, q, P, b, P, qn, P, P, P, S)
+
+
+def test_prologue_arguments(lib):
+    assert pro(lib, flags=256) == -8                  # unknown flag bit
+    assert pro(lib, dt=9) == -3
+    assert pro(lib, N=-1) == -2
+    assert pro(lib, H=0) == -2
+    assert pro(lib, D=96) == -8
+    assert pro(lib, q=NUL) == -1                      # normalisation needs q
+    assert pro(lib, qn=MIS) == -4
+    assert pro(lib, b=NUL) == -1                      # logits need b
+    assert pro(lib, flags=g.BW_LOGITS | g.ERASE_NONE, b=NUL, q=NUL, qn=NUL, N=0) == 0  # only w is needed
+    assert pro(lib, N=0) == 0                         # nothing to do, no launch
+    assert pro(lib, flags=g.QK_L2NORM, b=NUL, N=0) == 0  # b unused without BW_LOGITS
