@@ -15,7 +15,8 @@ steps) and the roofline fraction of each, plus:
 * `cpu_baseline`: the fp64 oracle timed on a bounded sample on the host cores;
 * `clocks`: SM clock and throttle reasons sampled during the timed regions;
 * `sweep`: forward throughput at 65,536 tokens per call for T = 2K ... 32K (B = 32 ... 2),
-  with the number of (batch, head) CTAs each shape gives the 148 SMs;
+  with the number of (batch, head) chains each shape gives the 148 SMs (`scan`: the shape
+  takes the chunk-parallel scan, for at most 48 chains);
 * `varlen`: the headline's 32,768 tokens as 16 packed sequences of log-uniform length
   (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen;
 * `scalar_decay`: the headline batch with one log decay per (token, head) through
@@ -465,18 +466,22 @@ def run_ours(args):
                              device=str(dev))
             os_ = torch.empty_like(xs["v"])
             Ss = torch.empty_like(xs["S0"])
+            # few long chains take the chunk-parallel scan, which needs a workspace
+            nws = g.gdn2_workspace_size(0, xs["q"].dtype, sw["B"], sw["T"], sw["H"], sw["Dk"], sw["Dv"])
+            wss = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
 
             def fwd_s():
-                g.gdn2_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["b"], xs["w"], xs["S0"], o=os_, S_T=Ss)
+                g.gdn2_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["b"], xs["w"], xs["S0"], o=os_, S_T=Ss,
+                                 workspace=wss)
 
             ks = 10
             ms_s = time_region(fwd_s, ks, 3, stream) / ks
             assert g.gdn2_sync_status() == 0
             bs = fwd_bytes(sw["B"], sw["T"], sw["H"], sw["Dk"])
-            sweep[name] = {"T": sw["T"], "B": sw["B"], "ctas": sw["B"] * sw["H"], "ms": round(ms_s, 4),
+            sweep[name] = {"T": sw["T"], "B": sw["B"], "ctas": sw["B"] * sw["H"], "scan": nws > 0, "ms": round(ms_s, 4),
                            "tokens_per_s": round(job_rate(sw["B"] * sw["T"], world, ms_s), 1),
                            "hbm_frac": round(bs / (ms_s * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-            del xs, os_, Ss
+            del xs, os_, Ss, wss
         extras["sweep"] = sweep
     clocks.stop()
     if ms_fwd is None:

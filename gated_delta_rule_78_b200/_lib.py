@@ -144,6 +144,9 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, want_
     if S_T is None and want_state:
         S_T = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)
     ws = workspace
+    if ws is None:  # few long chains run as a chunk-parallel scan, which needs a workspace
+        nb = gdn2_workspace_size(0, q.dtype, B, T, H, Dk, Dv)
+        ws = torch.empty(nb, dtype=torch.uint8, device=q.device) if nb > 0 else None
     st = raw().gdn2_chunk_fwd(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
                               _p(S0), _p(o), _p(S_T), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                               _stream(stream))

@@ -107,6 +107,7 @@ struct TcParams {
     const int *cu_seqlens;   // null: B sequences of T tokens; else B packed sequences in T rows
     const int *chunk_off;    // variable length with states only: first chunk of each sequence
     int g_scalar;            // log alpha is one value per (token, head), [rows, H]: a scalar decay
+    ScanArgs scan;           // chunk-parallel scan instances only (gdn2_internal.cuh)
 };
 
 struct TcMaps {
@@ -170,7 +171,10 @@ __device__ __forceinline__ void lane_sum16(float (&v)[16], int lane)
 // squares come from the decay folding's loads; the reduction over the lanes runs while the
 // [A; P] product is in flight.  The sigmoid of b is applied in the decay folding, that of w
 // in the X = w.v fold.
-template <bool kGScalar, int DIN, int kPro>
+// kScan: a pass of the chunk-parallel scan (ScanArgs): every CTA decodes its segment, its state
+// source and destination, whether it writes o, and whether it runs the transition (the
+// chain's linear part on the identity: X = 0, S = I at the segment start).
+template <bool kGScalar, int DIN, int kPro, bool kScan = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -183,11 +187,40 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     __shared__ __align__(8) uint64_t bar_in[2], bar_emma, bar_mma, bar_fact[2], bar_mdone[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort_m, s_abort_e;
+    __shared__ float *s_stp;  // this CTA's end-state destination (read once, at the end)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool is_m = warp < 8;
     const int bh = blockIdx.x, bb = bh / p.H, hh = bh % p.H;
     int bos = bb * p.T, T = p.T;  // this sequence's first token row and its length
+    const float *S0p = p.S0 ? p.S0 + (size_t)bh * DIN * DIN : nullptr;  // this CTA's start state
+    float *STp = p.S_T ? p.S_T + (size_t)bh * DIN * DIN : nullptr;     // and its end state
+    bool o_on = p.o != nullptr, trans = false;
+    if (kScan) {
+        const ScanArgs &sc = p.scan;
+        const int u = bh / p.H, mid = sc.nseg - 2;
+        int b, sg;
+        if (sc.pass == 0 && u < p.B) {  // segment 0, from S0, with its output
+            b = u;
+            sg = 0;
+            STp = sc.send0 + ((size_t)b * p.H + hh) * DIN * DIN;
+        } else if (sc.pass == 0) {  // a middle segment: local end state (even) or transition (odd)
+            const int v = u - p.B, pair = v >> 1;
+            b = pair / mid;
+            sg = 1 + pair % mid;
+            trans = v & 1;
+            S0p = nullptr;
+            STp = (trans ? sc.phi : sc.shat) + (((size_t)b * mid + sg - 1) * p.H + hh) * DIN * DIN;
+            o_on = false;
+        } else {  // segments 1 .. nseg-1 from their start states; the last one gives S_T
+            b = u / (sc.nseg - 1);
+            sg = 1 + u % (sc.nseg - 1);
+            S0p = sc.sstart + (((size_t)b * (sc.nseg - 1) + sg - 1) * p.H + hh) * DIN * DIN;
+            STp = (sg == sc.nseg - 1 && p.S_T) ? p.S_T + ((size_t)b * p.H + hh) * DIN * DIN : nullptr;
+        }
+        bos = b * p.T + sg * sc.seg_len;
+        T = max(0, min(sc.seg_len, p.T - sg * sc.seg_len));
+    }
     if (p.cu_seqlens) {
         const int b0 = p.cu_seqlens[bb], b1 = p.cu_seqlens[bb + 1];
         if (b0 < 0 || b1 < b0 || b1 > p.T) {  // nothing launched yet: leave before any barrier
@@ -209,6 +242,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     if (tid == 0) {
         s_abort_m = 0;
         s_abort_e = 0;
+        s_stp = STp;
         mbar_init(&bar_emma, 1);
         mbar_init(&bar_mma, 1);
         for (int i = 0; i < 2; ++i) {
@@ -262,6 +296,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         };
         // X = w.v of chunk ci, in place of v (one token row of 64 channels per warp step)
         auto fold_value = [&](int ci) {
+            if (kScan && trans) return;  // X = 0
             const int Lc = min(C, T - ci * C);
             uint8_t *pv = sm + OFF_V + (ci & 1) * 16384;
             const uint8_t *pw = sm + OFF_W;
@@ -297,8 +332,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-            Sf[i] = (p.S0 && 64 * half + i < DIN && jrow < DIN) ? p.S0[((size_t)bh * DIN + 64 * half + i) * DIN + jrow]
-                                                                 : 0.f;
+            Sf[i] = (kScan && trans) ? ((64 * half + i == jrow && jrow < DIN) ? 1.f : 0.f)
+                    : (S0p && 64 * half + i < DIN && jrow < DIN) ? S0p[(64 * half + i) * DIN + jrow] : 0.f;
         if (p.states) store_state(Sf, 0);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -341,8 +376,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int t = 32 * half + 2 * e;
-                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t, xb)));
-                    const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t + 1, xb)));
+                    float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t, xb)));
+                    float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(px + sw128(t + 1, xb)));
+                    if (kScan && trans) x0 = x1 = 0.f;
                     const float a0 = __uint_as_float(r[2 * e]), a1 = __uint_as_float(r[2 * e + 1]);
                     if (kPro & kProNorm) {  // R_k X - R_k^2 E~ S
                         const float r0 = rk[t], r1 = rk[t + 1];
@@ -413,7 +449,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 }
                 if (p.states) store_state(Sf, ci + 1);
             }
-            if (p.o) {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
+            if (o_on) {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
                 uint32_t r[32];
                 tmem_ld32(tmem + TM_O + 32 * half + lane_off, r);
                 tmem_wait_ld();
@@ -431,12 +467,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(1, kGroup);
-            if (p.o && L == C) {
+            if (o_on && L == C) {
                 if (tid == 0) {
                     tma_store_3d(&maps.o, sm + ott, 0, hh, bos + ci * C);
                     bulk_commit();
                 }
-            } else if (p.o) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
+            } else if (o_on) {  // ragged last chunk: only the valid rows (the tile would spill into the next sequence)
                 const __nv_bfloat16 *so = reinterpret_cast<const __nv_bfloat16 *>(sm + ott);
                 __nv_bfloat16 *dst = p.o + ((size_t)bos + (size_t)ci * C) * p.H * DIN + (size_t)hh * DIN;
                 for (int idx = tid; idx < L * DIN; idx += kGroup)
@@ -455,10 +491,11 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 mbar_arrive(&bar_mdone[buf]);      // this parity's buffers and w are free
             }
         }
-        if (!s_abort_m && p.S_T) {
+        float *const st_dst = s_stp;
+        if (!s_abort_m && st_dst) {
 #pragma unroll
             for (int i = 0; i < 64; ++i)
-                if (64 * half + i < DIN && jrow < DIN) p.S_T[((size_t)bh * DIN + 64 * half + i) * DIN + jrow] = Sf[i];
+                if (64 * half + i < DIN && jrow < DIN) st_dst[(64 * half + i) * DIN + jrow] = Sf[i];
         }
         if (tid == 0) bulk_wait0();
     } else {
@@ -695,7 +732,7 @@ bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, i
 }  // namespace
 
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
-                          cudaStream_t s)
+                          cudaStream_t s, const ScanArgs *scan)
 {
     // d = 64 runs zero-padded to 128 (see the kernel); chunk-boundary states keep the padded
     // 128 x 128 layout (they are the backward's internal workspace)
@@ -711,13 +748,21 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         (o && !make_map(&maps.o, o, false, 1, rows, pr.H, din, true)))
         return cudaErrorInvalidValue;
     TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
-                 pr.g_scalar ? 1 : 0};
+                 pr.g_scalar ? 1 : 0, ScanArgs{}};
+    int grid = pr.B * pr.H;
+    if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)
+        if (pr.g_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C)
+            return cudaErrorInvalidValue;
+        prm.scan = *scan;
+        grid = (scan->pass == 0 ? pr.B * (1 + 2 * (scan->nseg - 2)) : pr.B * (scan->nseg - 1)) * pr.H;
+    }
     auto run = [&](auto kernel) -> cudaError_t {
         cudaError_t e = set_smem_attr(reinterpret_cast<const void *>(kernel), (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        kernel<<<pr.B * pr.H, kThreads, SMEM_BYTES, s>>>(maps, prm);
+        kernel<<<grid, kThreads, SMEM_BYTES, s>>>(maps, prm);
         return cudaGetLastError();
     };
+    if (scan) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, true>) : run(fwd_tc_kernel<false, 64, 0, true>);
     if (pr.prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
     auto by_pro = [&](auto gs, auto dn) -> cudaError_t {
         constexpr bool kGS = decltype(gs)::value;

@@ -239,9 +239,10 @@ const char *gdn2_strerror(gdn2_status s)
 size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv)
 {
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK) return 0;
-    if (T == 0 || which == 0 || which == 2) return 0;
-    if (which != 1 && which != 3) return 0;
+    if (T == 0 || which == 2) return 0;
+    if (which != 0 && which != 1 && which != 3) return 0;
     gdn2::Problem p = make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+    if (which == 0) return dt == GDN2_BF16 ? gdn2::fwd_scan_workspace_bytes(p) : 0;  // the chunk-parallel scan
     static const int marker = 0;
     if (which == 3) p.cu_seqlens = &marker;  // sizes only: the pointer is not read
     return gdn2::bwd_workspace_bytes(dt, p);
@@ -252,8 +253,6 @@ gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
                            const void *w, const float *S0, void *o, float *S_T, void *workspace,
                            size_t ws_bytes, void *stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
     if (st != GDN2_OK) return st;
     if (T > 0) st = check_ptrs({q, k, v, log_alpha, b, w, o}, {S0, S_T});
@@ -267,6 +266,12 @@ gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
         return from_cuda(cudaMemsetAsync(S_T, 0, state_bytes, s));
     }
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    const size_t scan_need = dt == GDN2_BF16 ? gdn2::fwd_scan_workspace_bytes(p) : 0;
+    if (scan_need && workspace && ws_bytes >= scan_need && aligned16(workspace)) {  // few long chains
+        int *status = gdn2::status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        return from_cuda(gdn2::launch_fwd_scan(p, o, S_T, workspace, ws_bytes, status, s));
+    }
     return run_fwd(dt, p, o, S_T, s);
 }
 

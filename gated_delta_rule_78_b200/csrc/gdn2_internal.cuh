@@ -113,6 +113,25 @@ cudaError_t set_smem_attr(const void *kernel, int bytes);
 // the shape is outside what the kernel handles.  `o` may be null (no output);
 // `states`, when non-null, receives S^T in bf16 at every chunk boundary:
 // [B*H][nchunks + 1][D][D], entry c the state before chunk c, the last entry S_T.
+// Chunk-parallel scan of the forward (scan.cu): each sequence is cut into nseg segments of
+// seg_len tokens (a multiple of the chunk).  Pass 0 runs, in one launch, segment 0 from S0 with
+// its output (end state -> send0), and for every middle segment s = 1 .. nseg-2 its local end
+// state from zero (-> shat) and its transition, the state map's linear part applied to the
+// identity (-> phi).  The combine gives every later segment its start state (sstart); pass 1
+// runs segments 1 .. nseg-1 from those with their output, the last one writing S_T.
+// Layouts, fp32 [.., H, D, D]: send0 [B], shat and phi [B][nseg-2], sstart [B][nseg-1].
+struct ScanArgs {
+    int nseg, seg_len, pass;
+    float *send0, *shat, *phi;
+    const float *sstart;
+};
+
+// Workspace of the chunk-parallel scan for this problem; 0 when the scan is not used for it
+// (variable length, scalar decay, prologue, more than 48 chains, or short sequences).
+size_t fwd_scan_workspace_bytes(const Problem &p);
+cudaError_t launch_fwd_scan(const Problem &p, void *o, float *S_T, void *ws, size_t ws_bytes, int *status,
+                            cudaStream_t s);
+
 // The input prologue as separate passes (prologue.cu).  rows = token rows x heads; gate modes:
 // 0 untouched, 1 per channel ([rows, D]), 2 per token ([rows]).
 cudaError_t launch_prologue_fwd(bool fp32, size_t rows, int D, bool norm, const void *q, const void *k, void *qn,
@@ -122,7 +141,8 @@ cudaError_t launch_prologue_bwd(bool fp32, size_t rows, int D, bool norm, const 
                                 void *dk, int b_mode, const void *b, void *db, int w_mode, const void *w, void *dw,
                                 cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *states, int *status,
-                          cudaStream_t s);
+                          cudaStream_t s,
+                          const ScanArgs *scan = nullptr);
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,

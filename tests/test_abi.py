@@ -177,3 +177,15 @@ def test_prologue_arguments(lib):
     assert pro(lib, flags=g.BW_LOGITS | g.ERASE_NONE, b=NUL, q=NUL, qn=NUL, N=0) == 0  # only w is needed
     assert pro(lib, N=0) == 0                         # nothing to do, no launch
     assert pro(lib, flags=g.QK_L2NORM, b=NUL, N=0) == 0  # b unused without BW_LOGITS
+
+
+def test_forward_workspace_for_the_scan(lib):
+    # few long chains (at most 48 (batch, head) pairs, at least 48 chunks): the chunk-parallel scan
+    st = 128 * 128 * 4
+    assert lib.gdn2_workspace_size(0, BF16, 2, 32768, 16, 128, 128) == 32 * st * 5
+    assert lib.gdn2_workspace_size(0, BF16, 1, 3072, 2, 64, 64) == 2 * 64 * 64 * 4 * 5
+    assert lib.gdn2_workspace_size(0, BF16, 1, 3008, 2, 128, 128) == 0   # 47 chunks: serial
+    assert lib.gdn2_workspace_size(0, BF16, 4, 16384, 16, 128, 128) == 0  # 64 chains: serial
+    assert lib.gdn2_workspace_size(0, F32, 2, 32768, 16, 128, 128) == 0   # fp32 path: serial
+    # fewer chains get more segments: 16 chains fill 148 slots with 6 segments (9 CTAs each)
+    assert lib.gdn2_workspace_size(0, BF16, 1, 32768, 16, 128, 128) == 16 * st * (3 * 6 - 4)
