@@ -7,7 +7,9 @@ model (B=8, H=16, T=4096, d_k=d_v=128, bf16 inputs, fp32 log-decay and state;
 a token covers all 16 heads).  A step is one gdn2_chunk_fwd call over the
 batch, inputs resident in HBM (1.09 GB per step, larger than the 126 MB L2, so
 no flush is needed).  The same line carries the forward+backward figure on the
-same batch (`fwd_bwd`), the decode figure (`decode`, 256 sequences, 1024
+same batch (`fwd_bwd`: a training step, gdn2_chunk_fwd_save + gdn2_chunk_bwd_saved, the
+forward recording the chunk-boundary states the backward needs; `bwd_ms` is the standalone
+backward, which recomputes them), the decode figure (`decode`, 256 sequences, 1024
 steps) and the roofline fraction of each, plus:
 
 * `e2e`: the same forward through the public binding with host buffers:
@@ -333,12 +335,27 @@ def run_ours(args):
         assert g.gdn2_sync_status() == 0
         bb = bwd_bytes(B, T, H, D)
         extras["fwd_bwd"] = {"bwd_ms": round(ms_bwd, 4), "steps": ksteps,
-                             "bwd_roofline": roofline(bb, ms_bwd, pk), "launches_per_step": 1 + 3}
+                             "bwd_roofline": roofline(bb, ms_bwd, pk), "bwd_launches": 1 + 3}
         if ms_fwd is not None:
-            ms_fb = ms_fwd + ms_bwd
+            # a training step: the forward records the chunk-boundary states into the backward's
+            # workspace, and the backward skips its own states pass
+            o_tr = torch.empty_like(x["v"])
+            S_tr = torch.empty_like(x["S0"])
+
+            def train_step():
+                g.gdn2_chunk_fwd_save(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], workspace=ws,
+                                      o=o_tr, S_T=S_tr)
+                g.gdn2_chunk_bwd_saved(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], x["do"],
+                                       None, workspace=ws, out=grads)
+
+            ms_fb = time_region(train_step, ksteps, max(3, args.warmup // 2), stream) / ksteps
+            assert g.gdn2_sync_status() == 0
             extras["fwd_bwd"].update({
+                "step": "gdn2_chunk_fwd_save + gdn2_chunk_bwd_saved", "launches_per_step": 1 + 3,
                 "value": round(job_rate(tokens, world, ms_fb), 1), "unit": "tokens/s",
-                "ms_per_step": round(ms_fb, 4), "roofline": roofline(fb + bb, ms_fb, pk)})
+                "ms_per_step": round(ms_fb, 4), "roofline": roofline(fb + bb, ms_fb, pk),
+                "fwd_plus_standalone_bwd_ms": round(ms_fwd + ms_bwd, 4)})
+            del o_tr, S_tr
         del ws, grads
 
     if "decode" in parts:

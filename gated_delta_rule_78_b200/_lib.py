@@ -24,7 +24,7 @@ GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
            "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
            "gdn2_chunk_bwd_varlen", "gdn2_chunk_fwd_gated", "gdn2_chunk_bwd_gated", "gdn2_decode_step_gated",
-           "gdn2_workspace_size_gated", "gdn2_prologue")
+           "gdn2_workspace_size_gated", "gdn2_prologue", "gdn2_chunk_fwd_save", "gdn2_chunk_bwd_saved")
 # gate layout flags (gdn2_gate_flags in include/gdn2.h)
 DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE = 1, 2, 4, 8, 16, 32
 # input prologue: q, k L2-normalised in the call; b, w given as logits (sigmoid in the call)
@@ -71,6 +71,10 @@ def load(path: str | None = None):
     lib.gdn2_chunk_bwd_gated.restype = i
     lib.gdn2_decode_step_gated.argtypes = [i] * 6 + [vp] * 9 + [sz, vp]
     lib.gdn2_decode_step_gated.restype = i
+    lib.gdn2_chunk_fwd_save.argtypes = [i] * 6 + [vp] * 10 + [sz, vp]
+    lib.gdn2_chunk_fwd_save.restype = i
+    lib.gdn2_chunk_bwd_saved.argtypes = [i] * 6 + [vp] * 17 + [sz, vp]
+    lib.gdn2_chunk_bwd_saved.restype = i
     lib.gdn2_prologue.argtypes = [i] * 5 + [vp] * 8 + [vp]
     lib.gdn2_prologue.restype = i
     lib.gdn2_workspace_size_gated.argtypes = [i] * 8
@@ -171,7 +175,38 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
     return o
 
 
-def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace=None, out=None, stream=None):
+def gdn2_chunk_fwd_save(q, k, v, log_alpha, b, w, S0=None, *, workspace=None, o=None, S_T=None, stream=None):
+    """The forward that also records the chunk-boundary states into the backward's workspace.
+    Returns (o, S_T, workspace); pass the workspace to gdn2_chunk_bwd_saved."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w)):
+        _cuda_contig(n, t, q.dtype)
+    _cuda_contig("log_alpha", log_alpha, torch.float32)
+    _cuda_contig("S0", S0, torch.float32)
+    if o is None:
+        o = torch.empty(B, T, H, Dv, dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = gdn2_workspace_size(1, q.dtype, B, T, H, Dk, Dv)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    st = raw().gdn2_chunk_fwd_save(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                   _p(S0), _p(o), _p(S_T), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn2_chunk_fwd_save", st)
+    return o, S_T, workspace
+
+
+def gdn2_chunk_bwd_saved(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace, out=None, stream=None):
+    """gdn2_chunk_bwd on the states gdn2_chunk_fwd_save recorded into ``workspace``."""
+    return gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T, workspace=workspace, out=out, stream=stream,
+                          _saved=True)
+
+
+def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace=None, out=None, stream=None,
+                   _saved=False):
     """Gate-aware backward.  Returns dict(dq, dk, dv, dlog_alpha, db, dw, dS0)."""
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -189,11 +224,12 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T=None, *, workspace=No
     if workspace is None:
         nbytes = gdn2_workspace_size(1, q.dtype, B, T, H, Dk, Dv)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-    st = raw().gdn2_chunk_bwd(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
-                              _p(S0), _p(d_o), _p(dS_T), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
-                              _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]), _p(out["dS0"]),
-                              _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdn2_chunk_bwd", st)
+    fn = raw().gdn2_chunk_bwd_saved if _saved else raw().gdn2_chunk_bwd
+    st = fn(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+            _p(S0), _p(d_o), _p(dS_T), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+            _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]), _p(out["dS0"]),
+            _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn2_chunk_bwd_saved" if _saved else "gdn2_chunk_bwd", st)
     return out
 
 

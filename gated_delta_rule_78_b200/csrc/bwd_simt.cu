@@ -440,11 +440,11 @@ size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p)
 }
 
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
-                       const BwdOut &out, void *ws, cudaStream_t s)
+                       const BwdOut &out, void *ws, cudaStream_t s, bool states_saved)
 {
     int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
-    if (dt == GDN2_BF16) return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s);
+    if (dt == GDN2_BF16) return launch_bwd_tc(p, d_o, dS_T, out, ws, status, s, states_saved);
     if (dt == GDN2_F32)
         return p.D == 64 ? launch_t<64, float>(p, d_o, dS_T, out, ws, status, s)
                          : launch_t<128, float>(p, d_o, dS_T, out, ws, status, s);

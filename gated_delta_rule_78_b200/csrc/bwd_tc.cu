@@ -901,8 +901,15 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
 
 size_t bwd_tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
 
+cudaError_t launch_fwd_save(const Problem &p, void *o, float *S_T, void *ws, int *status, cudaStream_t s)
+{
+    if (p.cu_seqlens || (p.D != 128 && p.D != 64)) return cudaErrorNotSupported;
+    const BwdTcLayout l = tc_layout(p);
+    return launch_fwd_tc(p, o, S_T, reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + l.states), status, s);
+}
+
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
-                          int *status, cudaStream_t s)
+                          int *status, cudaStream_t s, bool states_saved)
 {
     if (p.D != 128 && p.D != 64) return cudaErrorNotSupported;
     const BwdTcLayout l = tc_layout(p);
@@ -946,8 +953,11 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&a.n_sm, cudaDevAttrMultiProcessorCount, dev);
     }
 
-    cudaError_t e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!states_saved || p.cu_seqlens) {  // chunk-boundary states, unless the forward recorded them
+        e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s);
+        if (e != cudaSuccess) return e;
+    }
     const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_kernel), (int)P_SMEM)) != cudaSuccess) return e;
     {  // persistent: one block per SM, each streaming (chunk, head) tasks

@@ -216,6 +216,38 @@ gdn2_status check_gate_ptrs(int flags, const void *g, const void *b, const void 
 }
 }  // namespace
 
+namespace {
+gdn2_status chunk_bwd_impl(bool saved, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                           const void *k, const void *v, const float *log_alpha, const void *b,
+                           const void *w, const float *S0, const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (T > 0)
+        st = check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0},
+                        {S0, dS_T});
+    else
+        st = check_ptrs({dS0}, {S0, dS_T});
+    if (st != GDN2_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+    if (T == 0) {
+        if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
+        return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
+    }
+    const size_t need = gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr,
+                                                                    nullptr, nullptr, nullptr));
+    if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
+    return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s, saved));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *gdn2_strerror(gdn2_status s)
@@ -293,27 +325,34 @@ gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, c
                            void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
                            float *dS0, void *workspace, size_t ws_bytes, void *stream)
 {
+    return chunk_bwd_impl(false, dt, B, T, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, d_o, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0, workspace, ws_bytes, stream);
+}
+
+gdn2_status gdn2_chunk_bwd_saved(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
+                           const void *k, const void *v, const float *log_alpha, const void *b,
+                           const void *w, const float *S0, const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream)
+{
+    return chunk_bwd_impl(true, dt, B, T, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, d_o, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0, workspace, ws_bytes, stream);
+}
+
+gdn2_status gdn2_chunk_fwd_save(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q, const void *k,
+                                const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                                void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream)
+{
     gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
     if (st != GDN2_OK) return st;
-    if (T > 0)
-        st = check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0},
-                        {S0, dS_T});
-    else
-        st = check_ptrs({dS0}, {S0, dS_T});
-    if (st != GDN2_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
-    if (T == 0) {
-        if (dS_T) return from_cuda(cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s));
-        return from_cuda(cudaMemsetAsync(dS0, 0, state_bytes, s));
-    }
-    const size_t need = gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr,
-                                                                    nullptr, nullptr, nullptr));
+    if (T == 0 || dt != GDN2_BF16)  // nothing to record (fp32: the backward recomputes its states)
+        return gdn2_chunk_fwd(dt, B, T, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, o, S_T, nullptr, 0, stream);
+    if ((st = check_ptrs({q, k, v, log_alpha, b, w, o}, {S0, S_T})) != GDN2_OK) return st;
+    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
+    const size_t need = gdn2::bwd_workspace_bytes(dt, p);
     if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
-    gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
-    gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
-    return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, workspace, s));
+    int *status = gdn2::status_word();
+    if (!status) return GDN2_ERR_CUDA;
+    return from_cuda(gdn2::launch_fwd_save(p, o, S_T, workspace, status, (cudaStream_t)stream));
 }
 
 gdn2_status gdn2_chunk_fwd_varlen(gdn2_dtype dt, int N, int total_T, int H, int Dk, int Dv,

@@ -159,14 +159,19 @@ inline size_t varlen_offsets_bytes(int n_seqs) { return ((size_t)(n_seqs + 1) * 
 // tensor cores, everything else on the fp32 FMA kernels).  Only the sizes and
 // whether cu_seqlens is set are read from p.
 size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p);
+// states_saved: the bf16 backward's chunk-boundary states are already in ws (launch_fwd_save
+// wrote them with the same inputs), so its states pass is skipped; ignored for fp32.
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
-                       const BwdOut &out, void *ws, cudaStream_t s);
+                       const BwdOut &out, void *ws, cudaStream_t s, bool states_saved = false);
 
 // tensor-core backward (bf16, D = 128): the forward in states mode, then the prep,
 // chain and gradient kernels
 size_t bwd_tc_workspace_bytes(const Problem &p);
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
-                          int *status, cudaStream_t s);
+                          int *status, cudaStream_t s, bool states_saved = false);
+// the bf16 forward (o, S_T) that also records the chunk-boundary states into the backward's
+// workspace ws, for launch_bwd_tc(..., states_saved = true); fixed-length batches
+cudaError_t launch_fwd_save(const Problem &p, void *o, float *S_T, void *ws, int *status, cudaStream_t s);
 
 // Gate layouts (gates.cu): fill dst ([n_rows, D]) with src[row] (a per-row scalar) or,
 // when src is null, with `fill`; and sum src ([n_rows, D]) over D into dst ([n_rows]).

@@ -77,8 +77,10 @@ typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
  *   o:   output [B,T,H,Dv] of type dt.
  *   S_T: final state, or NULL when not wanted.  May alias S0 (in-place
  *        state update), but no other argument.
- *   workspace / ws_bytes: scratch of at least gdn2_workspace_size(0, ...)
- *        bytes (currently 0; NULL is then accepted).
+ *   workspace / ws_bytes: scratch of gdn2_workspace_size(0, ...) bytes.  That is 0
+ *        (NULL accepted) except for bf16 batches of at most 48 (batch, head) chains of
+ *        at least 48 chunks, which run as a chunk-parallel scan over segments of each
+ *        sequence when given it (the serial chain runs when it is missing or short).
  * bf16 inputs run on the tensor cores (bf16 operands, fp32 accumulation,
  * fp32 state); fp32 inputs run in fp32 FMA arithmetic throughout.
  */
@@ -111,6 +113,27 @@ GDN2_API gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int D
  * as the aixai.ru post's implementation section requires.
  */
 GDN2_API gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                           float *dS0, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Training pair.  gdn2_chunk_fwd_save is gdn2_chunk_fwd (same o and S_T, bit for bit)
+ * that also records the chunk-boundary states into `workspace`, the backward's
+ * workspace of gdn2_workspace_size(1, ...) bytes; gdn2_chunk_bwd_saved is
+ * gdn2_chunk_bwd taking those recorded states instead of running its own forward
+ * pass over the batch.  Call the backward with the same inputs, S0 and workspace,
+ * with nothing written to the workspace in between; the gradients equal
+ * gdn2_chunk_bwd's bit for bit.  fp32 batches record nothing (the backward recomputes).
+ * gdn2_chunk_fwd_save returns GDN2_ERR_WORKSPACE for a missing or short workspace.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_save(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream);
+GDN2_API gdn2_status gdn2_chunk_bwd_saved(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
                            const void *q, const void *k, const void *v, const float *log_alpha,
                            const void *b, const void *w, const float *S0,
                            const void *d_o, const float *dS_T,

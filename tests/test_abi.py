@@ -189,3 +189,15 @@ def test_forward_workspace_for_the_scan(lib):
     assert lib.gdn2_workspace_size(0, F32, 2, 32768, 16, 128, 128) == 0   # fp32 path: serial
     # fewer chains get more segments: 16 chains fill 148 slots with 6 segments (9 CTAs each)
     assert lib.gdn2_workspace_size(0, BF16, 1, 32768, 16, 128, 128) == 16 * st * (3 * 6 - 4)
+
+
+def test_training_pair_arguments(lib):
+    def fsave(ws=P, ws_bytes=1 << 40, T=64, dt=BF16):
+        return lib.gdn2_chunk_fwd_save(dt, 1, T, 1, 128, 128, P, P, P, P, P, P, NUL, P, NUL, ws, ws_bytes, S)
+    assert fsave(ws=NUL) == -5                        # the states go into the backward's workspace
+    assert fsave(ws_bytes=16) == -5
+    assert fsave(ws=MIS) == -4
+    assert fsave(T=-1) == -2
+    assert fsave(dt=7) == -3
+    assert lib.gdn2_chunk_bwd_saved(BF16, 1, 64, 1, 128, 128, P, P, P, P, P, P, NUL, P, NUL,
+                                    P, P, P, P, P, P, P, NUL, 0, S) == -5

@@ -71,3 +71,23 @@ def test_bwd_full_size_layer_4k(cuda_lib):
         else:
             gs = torch.stack([out[gk][b, :, h] for b, h in pairs])
             assert_close(gs, r[rk][:, :, 0], "bf16", gk)
+
+
+@pytest.mark.parametrize("dtype,D,T", [("bf16", 128, 200), ("bf16", 64, 130), ("f32", 64, 100)])
+def test_training_pair_equals_plain_calls(cuda_lib, dtype, D, T):
+    """gdn2_chunk_fwd_save / gdn2_chunk_bwd_saved give the plain calls' results bit for bit."""
+    g = cuda_lib
+    x = make_inputs(2, T, 2, D, D, dtype=dtype, seed=61, with_do=True)
+    d = to_dev(x)
+    args = (d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"])
+    o1, S1, ws = g.gdn2_chunk_fwd_save(*args)
+    gr1 = g.gdn2_chunk_bwd_saved(*args, d["do"], workspace=ws)
+    o2, S2 = g.gdn2_chunk_fwd(*args)
+    gr2 = g.gdn2_chunk_bwd(*args, d["do"])
+    assert g.gdn2_sync_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    for k in gr1:
+        assert torch.equal(gr1[k], gr2[k]), k
+    ref = ref_bwd(x)
+    for gk, rk in GRADS:
+        assert_close(gr1[gk], ref[rk], dtype, gk)
