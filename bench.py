@@ -12,8 +12,9 @@ forward recording the chunk-boundary states the backward needs; `bwd_ms` is the 
 backward, which recomputes them), the decode figure (`decode`, 256 sequences, 1024
 steps) and the roofline fraction of each, plus:
 
-* `e2e`: the same forward through the public binding with host buffers:
-  pinned-host inputs copied in and o/S_T copied out inside the timed region;
+* `e2e`: the same forward through the C-ABI call with host buffers (gdn2_chunk_fwd_host):
+  pinned-host inputs copied in and o/S_T copied out inside the timed region, pipelined with
+  the kernels by batch rows;
 * `cpu_baseline`: the fp64 oracle timed on a bounded sample on the host cores;
 * `clocks`: SM clock and throttle reasons sampled during the timed regions;
 * `sweep`: forward throughput at 65,536 tokens per call for T = 2K ... 32K (B = 32 ... 2),
@@ -512,18 +513,16 @@ def run_ours(args):
         return
     value = job_rate(tokens, world, ms_fwd)
 
-    # ---- end to end through the binding with host buffers
+    # ---- end to end through the C-ABI call with host buffers (gdn2_chunk_fwd_host: the copies in,
+    #      the kernels and the copies out pipelined by batch rows inside the call)
     hx = {n: t.to("cpu").pin_memory() for n, t in x.items() if n != "do"}
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     hS = torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True)
-    dx = {n: torch.empty_like(t) for n, t in x.items() if n != "do"}
+    wsh = torch.empty(max(16, g.gdn2_workspace_size(4, x["q"].dtype, B, T, H, D, D)), dtype=torch.uint8, device=dev)
 
     def e2e():
-        for n in dx:
-            dx[n].copy_(hx[n], non_blocking=True)
-        g.gdn2_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["log_alpha"], dx["b"], dx["w"], dx["S0"], o=o, S_T=ST)
-        ho.copy_(o, non_blocking=True)
-        hS.copy_(ST, non_blocking=True)
+        g.gdn2_chunk_fwd_host(hx["q"], hx["k"], hx["v"], hx["log_alpha"], hx["b"], hx["w"], hx["S0"], o=ho, S_T=hS,
+                              workspace=wsh)
 
     ke = max(3, args.steps // 4)
     ms_e2e = time_region(e2e, ke, 2, stream) / ke

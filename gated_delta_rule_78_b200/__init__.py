@@ -6,6 +6,7 @@ package is its thin Python binding.  Functions carry the C names:
 * ``gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0) -> (o, S_T)``
 * ``gdn2_decode_step(q, k, v, log_alpha, b, w, S) -> o``   (S updated in place)
 * ``gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, d_o, dS_T) -> grads``
+* ``gdn2_chunk_fwd_host``: the forward on host tensors, copies pipelined with the kernels
 * ``gdn2_chunk_fwd_save`` / ``gdn2_chunk_bwd_saved``: the training pair, whose forward records the
   chunk-boundary states into the backward's workspace
 * ``gdn2_chunk_bwd_noalloc(..., out=grads)``: the backward with the library's
@@ -25,5 +26,5 @@ from ._lib import (EXPORTS, GDN2_BF16, GDN2_F32, GDN2_OK, LIB_PATH, NOALLOC_MAX_
                    STATUS_NAMES, Gdn2Error, gdn2_chunk_bwd, gdn2_chunk_bwd_noalloc, gdn2_chunk_bwd_varlen,
                    gdn2_chunk_fwd, gdn2_chunk_fwd_varlen, gdn2_chunk_fwd_gated, gdn2_chunk_bwd_gated,
                    gdn2_decode_step_gated, gdn2_workspace_size_gated, DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR,
-                   DECAY_NONE, ERASE_NONE, WRITE_NONE, QK_L2NORM, BW_LOGITS, gdn2_decode_step, gdn2_prologue, gdn2_chunk_fwd_save, gdn2_chunk_bwd_saved, gdn2_strerror, gdn2_sync_status,
+                   DECAY_NONE, ERASE_NONE, WRITE_NONE, QK_L2NORM, BW_LOGITS, gdn2_decode_step, gdn2_prologue, gdn2_chunk_fwd_save, gdn2_chunk_bwd_saved, gdn2_chunk_fwd_host, gdn2_strerror, gdn2_sync_status,
                    gdn2_workspace_size, load, raw)

@@ -24,7 +24,8 @@ GDN2_F32, GDN2_BF16 = 0, 1
 EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspace_size",
            "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
            "gdn2_chunk_bwd_varlen", "gdn2_chunk_fwd_gated", "gdn2_chunk_bwd_gated", "gdn2_decode_step_gated",
-           "gdn2_workspace_size_gated", "gdn2_prologue", "gdn2_chunk_fwd_save", "gdn2_chunk_bwd_saved")
+           "gdn2_workspace_size_gated", "gdn2_prologue", "gdn2_chunk_fwd_save", "gdn2_chunk_bwd_saved",
+           "gdn2_chunk_fwd_host")
 # gate layout flags (gdn2_gate_flags in include/gdn2.h)
 DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE = 1, 2, 4, 8, 16, 32
 # input prologue: q, k L2-normalised in the call; b, w given as logits (sigmoid in the call)
@@ -71,6 +72,8 @@ def load(path: str | None = None):
     lib.gdn2_chunk_bwd_gated.restype = i
     lib.gdn2_decode_step_gated.argtypes = [i] * 6 + [vp] * 9 + [sz, vp]
     lib.gdn2_decode_step_gated.restype = i
+    lib.gdn2_chunk_fwd_host.argtypes = [i] * 6 + [vp] * 10 + [sz, vp]
+    lib.gdn2_chunk_fwd_host.restype = i
     lib.gdn2_chunk_fwd_save.argtypes = [i] * 6 + [vp] * 10 + [sz, vp]
     lib.gdn2_chunk_fwd_save.restype = i
     lib.gdn2_chunk_bwd_saved.argtypes = [i] * 6 + [vp] * 17 + [sz, vp]
@@ -173,6 +176,32 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
                                 _p(S), _p(o), _stream(stream))
     _check("gdn2_decode_step", st)
     return o
+
+
+def gdn2_chunk_fwd_host(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, workspace=None, stream=None,
+                        device=None):
+    """The forward on host (CPU) tensors: inputs copied in and o, S_T copied out inside the call,
+    pipelined by batch rows.  Pinned host tensors let the copies overlap.  Returns (o, S_T) as
+    host tensors; ``workspace`` is device staging of gdn2_workspace_size(4, ...) bytes."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dt(q)
+    for n, t in (("q", q), ("k", k), ("v", v), ("b", b), ("w", w), ("log_alpha", log_alpha)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous host tensor")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if o is None:
+        o = torch.empty(B, T, H, Dv, dtype=q.dtype, pin_memory=True)
+    if S_T is None:
+        S_T = torch.empty(B, H, Dk, Dv, dtype=torch.float32, pin_memory=True)
+    if workspace is None:
+        nbytes = gdn2_workspace_size(4, q.dtype, B, T, H, Dk, Dv)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    st = raw().gdn2_chunk_fwd_host(dt, B, T, H, Dk, Dv, _p(q), _p(k), _p(v), _p(log_alpha), _p(b), _p(w),
+                                   _p(S0), _p(o), _p(S_T), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn2_chunk_fwd_host", st)
+    return o, S_T
 
 
 def gdn2_chunk_fwd_save(q, k, v, log_alpha, b, w, S0=None, *, workspace=None, o=None, S_T=None, stream=None):

@@ -1,6 +1,7 @@
 // C ABI of libgdn2.so: argument validation, workspace sizing, kernel dispatch.
 // Declarations and the contract of every entry point are in include/gdn2.h.
 #include <vector>
+#include <string.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -89,6 +90,13 @@ gdn2::Problem make_problem(int B, int T, int H, int D, const void *q, const void
 
 // Launch the forward of a validated problem (T > 0): bf16 with D = 128 on the tensor
 // cores, everything else on the FMA kernel.  Variable length first checks cu_seqlens.
+gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s);
+// the device forward of one host-pipeline slice
+cudaError_t run_fwd_slice(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s)
+{
+    return run_fwd(dt, p, o, S_T, s) == GDN2_OK ? cudaSuccess : cudaErrorLaunchFailure;
+}
+
 gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s)
 {
     int *status = gdn2::status_word();
@@ -272,6 +280,7 @@ size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk
 {
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK) return 0;
     if (T == 0 || which == 2) return 0;
+    if (which == 4) return gdn2::host_fwd_workspace_bytes(dt == GDN2_F32 ? 4 : 2, B, T, H, Dk);
     if (which != 0 && which != 1 && which != 3) return 0;
     gdn2::Problem p = make_problem(B, T, H, Dk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
     if (which == 0) return dt == GDN2_BF16 ? gdn2::fwd_scan_workspace_bytes(p) : 0;  // the chunk-parallel scan
@@ -558,6 +567,29 @@ gdn2_status gdn2_prologue(int flags, gdn2_dtype dt, int N, int H, int D, const v
     if (N == 0) return GDN2_OK;
     return from_cuda(gdn2::launch_prologue_fwd(dt == GDN2_F32, (size_t)N * H, D, norm, q, k, q_n, k_n, bm, b, b_s, wm,
                                                w, w_s, (cudaStream_t)stream));
+}
+
+gdn2_status gdn2_chunk_fwd_host(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q, const void *k,
+                                const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                                void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream)
+{
+    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (T == 0) {  // S_T = S0 (or zeros), host to host
+        if (!S_T) return GDN2_OK;
+        const size_t n = (size_t)B * H * Dk * Dv * sizeof(float);
+        cudaStream_t s = (cudaStream_t)stream;
+        if (S0) return S0 == S_T ? GDN2_OK : from_cuda(cudaMemcpyAsync(S_T, S0, n, cudaMemcpyHostToHost, s));
+        memset(S_T, 0, n);
+        return GDN2_OK;
+    }
+    for (const void *ptr : {q, k, v, static_cast<const void *>(log_alpha), b, w, static_cast<const void *>(o)})
+        if (!ptr) return GDN2_ERR_NULL;
+    const size_t need = gdn2::host_fwd_workspace_bytes(dt == GDN2_F32 ? 4 : 2, B, T, H, Dk);
+    if (!workspace || ws_bytes < need) return GDN2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
+    return from_cuda(gdn2::launch_fwd_host(dt, B, T, H, Dk, q, k, v, log_alpha, b, w, S0, o, S_T, workspace,
+                                           (cudaStream_t)stream, run_fwd_slice));
 }
 
 gdn2_status gdn2_sync_status(void *stream)

@@ -132,6 +132,14 @@ size_t fwd_scan_workspace_bytes(const Problem &p);
 cudaError_t launch_fwd_scan(const Problem &p, void *o, float *S_T, void *ws, size_t ws_bytes, int *status,
                             cudaStream_t s);
 
+// The forward on host buffers (host_fwd.cu): device staging bytes, and the pipelined run;
+// `run` is the device forward on one slice.
+size_t host_fwd_workspace_bytes(size_t elem_bytes, int B, int T, int H, int D);
+cudaError_t launch_fwd_host(gdn2_dtype dt, int B, int T, int H, int D, const void *q, const void *k, const void *v,
+                            const float *g, const void *b, const void *w, const float *S0, void *o, float *S_T,
+                            void *ws, cudaStream_t s,
+                            cudaError_t (*run)(gdn2_dtype, const Problem &, void *, float *, cudaStream_t));
+
 // The input prologue as separate passes (prologue.cu).  rows = token rows x heads; gate modes:
 // 0 untouched, 1 per channel ([rows, D]), 2 per token ([rows]).
 cudaError_t launch_prologue_fwd(bool fp32, size_t rows, int D, bool norm, const void *q, const void *k, void *qn,

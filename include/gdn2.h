@@ -120,6 +120,23 @@ GDN2_API gdn2_status gdn2_chunk_bwd(gdn2_dtype dt, int B, int T, int H, int Dk, 
                            float *dS0, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * The forward on HOST buffers: q, k, v, log_alpha, b, w, S0 (S0 may be NULL) are read from
+ * host memory and o, S_T (S_T may be NULL) written to host memory, with the layouts of
+ * gdn2_chunk_fwd.  The call pipelines slices of batch rows: the copies in, the chunk
+ * kernels (on `stream`) and the copies out overlap, through three rotating staging slots
+ * in the device `workspace` (gdn2_workspace_size(4, ...) bytes) and two library-owned
+ * streams.  Asynchronous on `stream`: the outputs are in host memory once `stream` has
+ * completed; the host buffers must stay valid until then.  Page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister) lets the copies overlap; pageable memory works but
+ * serialises them.  The results equal gdn2_chunk_fwd's on the same values bit for bit.
+ * Errors as gdn2_chunk_fwd, plus GDN2_ERR_WORKSPACE for a missing or short workspace.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_host(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
+                           const void *q, const void *k, const void *v, const float *log_alpha,
+                           const void *b, const void *w, const float *S0,
+                           void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Training pair.  gdn2_chunk_fwd_save is gdn2_chunk_fwd (same o and S_T, bit for bit)
  * that also records the chunk-boundary states into `workspace`, the backward's
  * workspace of gdn2_workspace_size(1, ...) bytes; gdn2_chunk_bwd_saved is
@@ -281,8 +298,8 @@ GDN2_API gdn2_status gdn2_prologue(int flags, gdn2_dtype dt, int N, int H, int D
                                    void *stream);
 
 /* Workspace bytes for which = 0 (gdn2_chunk_fwd), 1 (gdn2_chunk_bwd),
- * 2 (gdn2_chunk_fwd_varlen) or 3 (gdn2_chunk_bwd_varlen, B = N, T = total_T);
- * 0 for invalid or unsupported arguments. */
+ * 2 (gdn2_chunk_fwd_varlen), 3 (gdn2_chunk_bwd_varlen, B = N, T = total_T) or
+ * 4 (gdn2_chunk_fwd_host's device staging); 0 for invalid or unsupported arguments. */
 GDN2_API size_t gdn2_workspace_size(int which, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv);
 
 /* Static, NUL-terminated description of a status code. */

@@ -201,3 +201,18 @@ def test_training_pair_arguments(lib):
     assert fsave(dt=7) == -3
     assert lib.gdn2_chunk_bwd_saved(BF16, 1, 64, 1, 128, 128, P, P, P, P, P, P, NUL, P, NUL,
                                     P, P, P, P, P, P, P, NUL, 0, S) == -5
+
+
+def test_host_forward_arguments(lib):
+    def fh(ws=P, ws_bytes=1 << 40, q=P):
+        return lib.gdn2_chunk_fwd_host(BF16, 2, 64, 1, 128, 128, q, P, P, P, P, P, NUL, P, NUL, ws, ws_bytes, S)
+    assert fh(ws=NUL) == -5
+    assert fh(ws_bytes=16) == -5
+    assert fh(q=NUL) == -1
+    assert fh(ws=MIS) == -4
+    # three staging slots of one batch row each (B >= 6): q, k, v, b, w, o bf16, log alpha fp32, S0, S_T
+    B, T, H, D = 8, 4096, 16, 128
+    tok = T * H * D
+    slot = 6 * tok * 2 + tok * 4 + 2 * H * D * D * 4
+    assert lib.gdn2_workspace_size(4, BF16, B, T, H, D, D) == 3 * slot
+    assert lib.gdn2_workspace_size(4, BF16, B, 0, H, D, D) == 0
