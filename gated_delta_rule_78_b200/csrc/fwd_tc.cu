@@ -218,8 +218,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             S0p = sc.sstart + (((size_t)b * (sc.nseg - 1) + sg - 1) * p.H + hh) * DIN * DIN;
             STp = (sg == sc.nseg - 1 && p.S_T) ? p.S_T + ((size_t)b * p.H + hh) * DIN * DIN : nullptr;
         }
-        bos = b * p.T + sg * sc.seg_len;
-        T = max(0, min(sc.seg_len, p.T - sg * sc.seg_len));
+        const int start = sg == 0 ? 0 : sc.seg0_len + (sg - 1) * sc.seg_len;
+        bos = b * p.T + start;
+        T = max(0, min(sg == 0 ? sc.seg0_len : sc.seg_len, p.T - start));
     }
     if (p.cu_seqlens) {
         const int b0 = p.cu_seqlens[bb], b1 = p.cu_seqlens[bb + 1];
@@ -751,7 +752,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
                  pr.g_scalar ? 1 : 0, ScanArgs{}};
     int grid = pr.B * pr.H;
     if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)
-        if (pr.g_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C)
+        if (pr.g_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C ||
+            scan->seg0_len % C)
             return cudaErrorInvalidValue;
         prm.scan = *scan;
         grid = (scan->pass == 0 ? pr.B * (1 + 2 * (scan->nseg - 2)) : pr.B * (scan->nseg - 1)) * pr.H;

@@ -113,15 +113,16 @@ cudaError_t set_smem_attr(const void *kernel, int bytes);
 // the shape is outside what the kernel handles.  `o` may be null (no output);
 // `states`, when non-null, receives S^T in bf16 at every chunk boundary:
 // [B*H][nchunks + 1][D][D], entry c the state before chunk c, the last entry S_T.
-// Chunk-parallel scan of the forward (scan.cu): each sequence is cut into nseg segments of
-// seg_len tokens (a multiple of the chunk).  Pass 0 runs, in one launch, segment 0 from S0 with
+// Chunk-parallel scan of the forward (scan.cu): each sequence is cut into nseg segments, the
+// first of seg0_len tokens and the others of seg_len (multiples of the chunk; the last may be
+// shorter).  Pass 0 runs, in one launch, segment 0 from S0 with
 // its output (end state -> send0), and for every middle segment s = 1 .. nseg-2 its local end
 // state from zero (-> shat) and its transition, the state map's linear part applied to the
 // identity (-> phi).  The combine gives every later segment its start state (sstart); pass 1
 // runs segments 1 .. nseg-1 from those with their output, the last one writing S_T.
 // Layouts, fp32 [.., H, D, D]: send0 [B], shat and phi [B][nseg-2], sstart [B][nseg-1].
 struct ScanArgs {
-    int nseg, seg_len, pass;
+    int nseg, seg_len, pass, seg0_len;
     float *send0, *shat, *phi;
     const float *sstart;
 };

@@ -10,10 +10,13 @@
 //   combine:             S_start(1) = S_end(0), S_start(s+1) = Phi_s S_start(s) + S^_s;
 //   pass 1 (one launch): segments 1 .. nseg-1 from their start states with their output.
 // Each combine step costs a d_k x d_k x d_v product, and pass 0 runs two chains per middle
-// segment, so the scan pays only where the serial chain leaves SMs idle: used for at most
-// kScanMaxChains (batch, head) chains and segments of at least kScanMinChunks chunks.  The
-// number of segments n is the largest (up to kScanMaxSegments) whose pass 0, (2n - 3) CTAs
-// per chain, still fits one wave of kScanSlots CTAs (the B200's 148 SMs, one CTA each).
+// segment, so the scan pays only where the serial chain leaves SMs idle (kScanSlots: the
+// B200's 148 SMs, one CTA each), for segments of at least kScanMinChunks chunks:
+// * up to 48 chains: n equal segments, n the largest (up to kScanMaxSegments) whose pass 0,
+//   (2n - 3) CTAs per chain, fits one wave; pass 0 and pass 1 each take one segment's time;
+// * 49 to 74 chains: segment 0 twice as long as the two after it.  Pass 0 has 3 CTAs per
+//   chain; the first wave holds every segment-0 CTA and half of the middle ones, and the
+//   other half runs when those finish, within segment 0's time.  T = 4 L gives 2 L + L.
 #include "gdn2_internal.cuh"
 
 namespace gdn2 {
@@ -21,7 +24,8 @@ namespace {
 
 constexpr int kScanSlots = 148;
 constexpr int kScanMaxSegments = 8;
-constexpr int kScanMaxChains = kScanSlots / 3;  // 3 segments: 3 CTAs per chain in pass 0
+constexpr int kScanMaxChains = kScanSlots / 3;  // equal segments: 3 CTAs per chain in pass 0
+constexpr int kScanMaxChainsLong0 = kScanSlots / 2;  // long segment 0: 2 chains' worth per wave
 constexpr int kScanMinChunks = 16;              // per segment
 
 // S_start(s) for s = 1 .. nseg-1 of one (b, h), 16 state columns per block.
@@ -68,7 +72,7 @@ __global__ void __launch_bounds__(256) scan_combine_kernel(int H, int nseg, cons
 }
 
 struct ScanLayout {
-    int nseg, seg_len;
+    int nseg, seg_len, seg0_len;
     size_t send0, shat, phi, sstart, total;
 };
 
@@ -77,11 +81,22 @@ ScanLayout scan_layout(const Problem &p)
     ScanLayout l{};
     const int nch = (p.T + kChunk - 1) / kChunk;
     const long long chains = (long long)p.B * p.H;
-    if (p.cu_seqlens || p.g_scalar || p.prologue || chains > kScanMaxChains || nch < 3 * kScanMinChunks) return l;
-    int n = 3;
-    while (n < kScanMaxSegments && chains * (2 * (n + 1) - 3) <= kScanSlots && nch >= (n + 1) * kScanMinChunks) ++n;
-    l.nseg = n;
-    l.seg_len = (nch + l.nseg - 1) / l.nseg * kChunk;
+    if (p.cu_seqlens || p.g_scalar || p.prologue || nch < 3 * kScanMinChunks) return l;
+    if (chains <= kScanMaxChains) {
+        int n = 3;
+        while (n < kScanMaxSegments && chains * (2 * (n + 1) - 3) <= kScanSlots && nch >= (n + 1) * kScanMinChunks)
+            ++n;
+        l.nseg = n;
+        l.seg_len = (nch + l.nseg - 1) / l.nseg * kChunk;
+        l.seg0_len = l.seg_len;
+    } else if (chains <= kScanMaxChainsLong0 && nch >= 4 * kScanMinChunks) {
+        l.nseg = 3;
+        const int b = (nch + 3) / 4;  // chunks of segments 1 and 2; segment 0 takes the rest
+        l.seg_len = b * kChunk;
+        l.seg0_len = (nch - 2 * b) * kChunk;
+    } else {
+        return l;
+    }
     const size_t st = (size_t)p.B * p.H * p.D * p.D * sizeof(float);
     l.send0 = 0;
     l.shat = l.send0 + st;
@@ -103,7 +118,7 @@ cudaError_t launch_fwd_scan(const Problem &p, void *o, float *S_T, void *ws, siz
     char *base = static_cast<char *>(ws);
     float *send0 = reinterpret_cast<float *>(base + l.send0), *shat = reinterpret_cast<float *>(base + l.shat);
     float *phi = reinterpret_cast<float *>(base + l.phi), *sstart = reinterpret_cast<float *>(base + l.sstart);
-    ScanArgs a{l.nseg, l.seg_len, 0, send0, shat, phi, nullptr};
+    ScanArgs a{l.nseg, l.seg_len, 0, l.seg0_len, send0, shat, phi, nullptr};
     cudaError_t e = launch_fwd_tc(p, o, S_T, nullptr, status, s, &a);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(p.B * p.H), (unsigned)(p.D / 16));

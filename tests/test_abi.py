@@ -185,7 +185,10 @@ def test_forward_workspace_for_the_scan(lib):
     assert lib.gdn2_workspace_size(0, BF16, 2, 32768, 16, 128, 128) == 32 * st * 5
     assert lib.gdn2_workspace_size(0, BF16, 1, 3072, 2, 64, 64) == 2 * 64 * 64 * 4 * 5
     assert lib.gdn2_workspace_size(0, BF16, 1, 3008, 2, 128, 128) == 0   # 47 chunks: serial
-    assert lib.gdn2_workspace_size(0, BF16, 4, 16384, 16, 128, 128) == 0  # 64 chains: serial
+    # 49 to 74 chains: 3 segments, the first twice as long
+    assert lib.gdn2_workspace_size(0, BF16, 4, 16384, 16, 128, 128) == 64 * st * 5
+    assert lib.gdn2_workspace_size(0, BF16, 4, 4032, 16, 128, 128) == 0  # 63 chunks: too short for that plan
+    assert lib.gdn2_workspace_size(0, BF16, 5, 16384, 15, 128, 128) == 0  # 75 chains: serial
     assert lib.gdn2_workspace_size(0, F32, 2, 32768, 16, 128, 128) == 0   # fp32 path: serial
     # fewer chains get more segments: 16 chains fill 148 slots with 6 segments (9 CTAs each)
     assert lib.gdn2_workspace_size(0, BF16, 1, 32768, 16, 128, 128) == 16 * st * (3 * 6 - 4)

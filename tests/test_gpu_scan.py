@@ -63,3 +63,22 @@ def test_scan_sweep_32k_sampled(cuda_lib):
     for i, (b, h) in enumerate(pairs):
         assert_close(oc[b, :, h], ro[i, :, 0], "bf16", f"o[{b},{h}]")
         assert_close(Sc[b, h], rS[i, 0], "bf16", f"S_T[{b},{h}]")
+
+
+def test_scan_long_first_segment(cuda_lib):
+    """64 chains (49 to 74): segment 0 twice as long as the two after it."""
+    B, T, H, D = 4, 4200, 16, 128  # 66 chunks: 32, 17, 17
+    assert g.gdn2_workspace_size(0, torch.bfloat16, B, T, H, D, D) == B * H * D * D * 4 * 5
+    x = make_inputs(B, T, H, D, D, dtype="bf16", seed=57)
+    args = [dev(x[n]) for n in ("q", "k", "v", "log_alpha", "b", "w", "S0")]
+    o1, S1 = g.gdn2_chunk_fwd(*args)                                             # scan
+    o2, S2 = g.gdn2_chunk_fwd(*args, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))  # serial
+    assert g.gdn2_sync_status() == 0
+    assert l2_rel(o1, o2) < 1e-2 and l2_rel(S1, S2) < 1e-2
+    pairs = sample_pairs(B, H, 1, seed=7)
+    xs = bh_slice({n: x[n] for n in ("q", "k", "v", "log_alpha", "b", "w", "S0")}, pairs)
+    ro, rS = oracle.ref_fwd(*(xs[n] for n in ("q", "k", "v", "log_alpha", "b", "w", "S0")))
+    oc, Sc = o1.cpu(), S1.cpu()
+    for i, (b, h) in enumerate(pairs):
+        assert_close(oc[b, :, h], ro[i, :, 0], "bf16", f"o[{b},{h}]")
+        assert_close(Sc[b, h], rS[i, 0], "bf16", f"S_T[{b},{h}]")
