@@ -86,14 +86,27 @@ cudaError_t launch_fwd_host(gdn2_dtype dt, int B, int T, int H, int D, const voi
     if (e != cudaSuccess) return e;
     const int nslice = (B + rps - 1) / rps;
     const size_t tok_row = (size_t)T * H * D, st_row = (size_t)H * D * D;
-    // events: the caller's prior work; per slice copy-in done and forward done; per slot free
-    cudaEvent_t ev_start, ev_in[kSlots], ev_comp[kSlots], ev_free[kSlots];
+    // events: the caller's prior work; per slot copy-in done, forward done, slot free.  A
+    // destroyed event whose recorded work is still pending is released when that work ends.
+    struct Events {
+        cudaEvent_t start = nullptr, in[kSlots] = {}, comp[kSlots] = {}, free_[kSlots] = {};
+        ~Events()
+        {
+            if (start) cudaEventDestroy(start);
+            for (int j = 0; j < kSlots; ++j) {
+                if (in[j]) cudaEventDestroy(in[j]);
+                if (comp[j]) cudaEventDestroy(comp[j]);
+                if (free_[j]) cudaEventDestroy(free_[j]);
+            }
+        }
+    } evs;
     auto mk = [](cudaEvent_t *ev) { return cudaEventCreateWithFlags(ev, cudaEventDisableTiming); };
-    if ((e = mk(&ev_start)) != cudaSuccess) return e;
+    if ((e = mk(&evs.start)) != cudaSuccess) return e;
     for (int j = 0; j < kSlots; ++j)
-        if ((e = mk(&ev_in[j])) != cudaSuccess || (e = mk(&ev_comp[j])) != cudaSuccess ||
-            (e = mk(&ev_free[j])) != cudaSuccess)
+        if ((e = mk(&evs.in[j])) != cudaSuccess || (e = mk(&evs.comp[j])) != cudaSuccess ||
+            (e = mk(&evs.free_[j])) != cudaSuccess)
             return e;
+    cudaEvent_t &ev_start = evs.start, *ev_in = evs.in, *ev_comp = evs.comp, *ev_free = evs.free_;
     char *base = static_cast<char *>(ws);
     auto H2D = [&](void *dst, const void *src, size_t n) {
         return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, hs.in);
@@ -142,12 +155,6 @@ cudaError_t launch_fwd_host(gdn2_dtype dt, int B, int T, int H, int D, const voi
     // the caller's stream completes when the last copy-out has
     if (e == cudaSuccess) e = cudaEventRecord(ev_start, hs.out);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_start, 0);
-    cudaEventDestroy(ev_start);  // released once recorded work completes
-    for (int j = 0; j < kSlots; ++j) {
-        cudaEventDestroy(ev_in[j]);
-        cudaEventDestroy(ev_comp[j]);
-        cudaEventDestroy(ev_free[j]);
-    }
     return e;
 }
 
