@@ -28,3 +28,15 @@ def test_host_forward_equals_device_forward(cuda_lib, dtype, B, T, D, pinned, wi
     o_d, S_d = g.gdn2_chunk_fwd(*(d[n] for n in NAMES[:6]), d["S0"] if with_s0 else None)
     assert g.gdn2_sync_status() == 0
     assert torch.equal(o_h, o_d.cpu()) and torch.equal(S_h, S_d.cpu())
+
+
+def test_host_forward_zero_length(cuda_lib):
+    B, H, D = 3, 2, 64
+    x = make_inputs(B, 1, H, D, D, dtype="bf16", seed=73)
+    empty = {n: t[:, :0].contiguous() if n != "S0" else t for n, t in x.items()}
+    o, S_T = g.gdn2_chunk_fwd_host(*(empty[n] for n in NAMES[:6]), x["S0"])
+    torch.cuda.synchronize()
+    assert o.shape[1] == 0 and torch.equal(S_T, x["S0"])
+    o, S_T = g.gdn2_chunk_fwd_host(*(empty[n] for n in NAMES[:6]), None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S_T) == 0
