@@ -300,6 +300,10 @@ def run_ours(args):
     tokens = B * T  # per rank
     clocks = ClockSampler(dev.index)
 
+    if args.only in ("prologue", "scan"):
+        run_part(args, g, w, dev, stream, rank, world, pk)
+        return
+
     # ---- forward (headline)
     x = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=rank_seed(rank), device=str(dev), with_do=True)
     o = torch.empty_like(x["v"])
@@ -558,6 +562,54 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_part(args, g, w, dev, stream, rank, world, pk):
+    """One extra measured alone, for profiling runs: `prologue` (layer_4k with raw q, k and gate
+    logits: the fused forward, then the separate pass + plain forward) or `scan` (B=2, T=32768,
+    H=16: the chunk-parallel scan, then the serial chain)."""
+    out = {"metric": METRIC, "only": args.only, "steps": args.steps, "warmup": args.warmup}
+    if args.only == "prologue":
+        B, T, H, D = w["B"], w["T"], w["H"], w["Dk"]
+        xr = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=rank_seed(rank) + 31, device=str(dev), raw=True)
+        o = torch.empty_like(xr["v"])
+        ST = torch.empty_like(xr["S0"])
+        flags = g.QK_L2NORM | g.BW_LOGITS
+        pro = {n: torch.empty_like(xr[n]) for n in ("q", "k", "b", "w")}
+
+        def fused():
+            g.gdn2_chunk_fwd_gated(xr["q"], xr["k"], xr["v"], xr["log_alpha"], xr["b"], xr["w"], xr["S0"],
+                                   flags=flags, o=o, S_T=ST)
+
+        def unfused():
+            g.gdn2_prologue(xr["q"], xr["k"], xr["b"], xr["w"], flags=flags, out=pro)
+            g.gdn2_chunk_fwd(pro["q"], pro["k"], xr["v"], xr["log_alpha"], pro["b"], pro["w"], xr["S0"], o=o, S_T=ST)
+
+        out["fused_ms"] = round(time_region(fused, args.steps, args.warmup, stream) / args.steps, 4)
+        out["unfused_ms"] = round(time_region(unfused, args.steps, args.warmup, stream) / args.steps, 4)
+        out["config"] = {"workload": f"{args.workload}, raw q, k and b, w logits"}
+    else:
+        sw = WORKLOADS["sweep_32k"]
+        B, T, H, D = sw["B"], sw["T"], sw["H"], sw["Dk"]
+        xs = make_inputs(B, T, H, D, D, dtype=sw["dtype"], seed=rank_seed(rank), device=str(dev))
+        o = torch.empty_like(xs["v"])
+        ST = torch.empty_like(xs["S0"])
+        nws = g.gdn2_workspace_size(0, xs["q"].dtype, B, T, H, D, D)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        none = torch.empty(16, dtype=torch.uint8, device=dev)
+
+        def run(wsp):
+            return lambda: g.gdn2_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["b"], xs["w"], xs["S0"],
+                                            o=o, S_T=ST, workspace=wsp)
+
+        out["scan_ms"] = round(time_region(run(ws), args.steps, args.warmup, stream) / args.steps, 4)
+        out["serial_ms"] = round(time_region(run(none), args.steps, args.warmup, stream) / args.steps, 4)
+        out["config"] = {"workload": "sweep_32k", "B": B, "T": T, "H": H, "chains": B * H, "workspace": nws}
+    assert g.gdn2_sync_status() == 0
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -568,8 +620,10 @@ def main():
     ap.add_argument("--fwd-only", action="store_true", help="skip the fwd+bwd and decode figures")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-sweep", action="store_true", help="skip the sequence-length sweep")
-    ap.add_argument("--only", choices=["fwd", "bwd", "decode"], default=None,
-                    help="time one part only (for profiling runs)")
+    ap.add_argument("--only", choices=["fwd", "bwd", "decode", "prologue", "scan"], default=None,
+                    help="time one part only (for profiling runs): the headline forward, the backward, "
+                         "decode, the fused input prologue against a separate pass, or the chunk-parallel "
+                         "scan against the serial chain at B=2, T=32K")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
