@@ -51,7 +51,7 @@ struct BwdTcLayout {
 };
 
 // Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W and K^ bf16
-// [C][D], gamma fp32 [D], R^T fp32 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
+// [C][D], gamma fp32 [D], R^T bf16 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
 // Variable length puts chunk_off first; chunk lists are sized by the chunk bound.
 BwdTcLayout tc_layout(const Problem &p)
 {
@@ -63,7 +63,7 @@ BwdTcLayout tc_layout(const Problem &p)
     l.W = off;      off += H * nchunk * C * D * 2;
     l.Kh = off;     off += H * nchunk * C * D * 2;
     l.gam = off;    off += H * nchunk * D * 4;
-    l.Rt = off;     off += H * nchunk * D * D * 4;
+    l.Rt = off;     off += H * nchunk * D * D * 2;
     l.Tm = off;     off += H * nchunk * C * C * 2;
     l.Pm = off;     off += H * nchunk * C * C * 2;
     l.dSn = off;    off += H * nchunk * D * D * 2;
@@ -79,7 +79,8 @@ struct BwdTcArgs {
     const float *g;
     const float *dS_T;  // may be null
     __nv_bfloat16 *states, *W, *Kh, *Tm, *Pm, *dSn;
-    float *gam, *Rt;
+    float *gam;
+    __nv_bfloat16 *Rt;  // R^T per chunk, bf16
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
     int n_sm;            // multiprocessors of the device (L2 prefetch distance of the gradient kernel)
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
         warp_gemm<2, 4, true, true, C>(acc, sb + P_DOb, 256, 32 * mb, sb + P_Qb, 256, 32 * nb, lane);
         warp_gemm<2, 4, true, true, C>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, lane);
         const int g = lane >> 2, t4 = lane & 3;
-        float *rt = a.Rt + cidx * D * D;
+        __nv_bfloat16 *rt = a.Rt + cidx * D * D;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -425,8 +426,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int row = 32 * mb + 16 * mt + g + 8 * hr, col = 32 * nb + 8 * nt + 2 * t4;
-                    *reinterpret_cast<float2 *>(rt + row * D + col) =
-                        make_float2(acc[mt][nt][2 * hr], acc[mt][nt][2 * hr + 1]);
+                    *reinterpret_cast<uint32_t *>(rt + row * D + col) =
+                        pack_bf16x2(acc[mt][nt][2 * hr], acc[mt][nt][2 * hr + 1]);
                 }
     }
     __syncthreads();  // every warp is done with this task's tiles before they are refilled
@@ -442,9 +443,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcAr
 //   dS^T = dS_n^T Diag(gamma) + R^T - Z^T W   (K = 64; A operand = -Z^T from registers)
 // W, K^, gamma and R^T of the next chunk are copied in (cp.async) during the current one.
 constexpr int kChainThreads = 256;
-constexpr int LDR = 136;  // fp32 row stride of the R^T tile (conflict-free fragment reads)
+constexpr int LDR = 136;  // bf16 row stride of the R^T tile (conflict-free fragment reads)
 constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_R = 33280;
-constexpr uint32_t CH_BUF = CH_R + D * LDR * 4;  // per buffer
+constexpr uint32_t CH_BUF = CH_R + D * LDR * 2;  // per buffer
 constexpr uint32_t CH_SMEM = 2 * CH_BUF;
 
 __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTcArgs a)
@@ -468,10 +469,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
             cp_async16(base + CH_W + swz(t, 8 * ch, 256), wsrc + t * D + 8 * ch);
             cp_async16(base + CH_K + swz(t, 8 * ch, 256), ksrc + t * D + 8 * ch);
         }
-        const float *rsrc = a.Rt + cidx * D * D;
-        for (int idx = tid; idx < D * 32; idx += kChainThreads) {
-            const int r = idx >> 5, ch = idx & 31;
-            cp_async16(base + CH_R + (r * LDR + 4 * ch) * 4, rsrc + r * D + 4 * ch);
+        const __nv_bfloat16 *rsrc = a.Rt + cidx * D * D;
+        for (int idx = tid; idx < D * 16; idx += kChainThreads) {  // 16 x 16 bytes per bf16 row
+            const int r = idx >> 4, ch = idx & 15;
+            cp_async16(base + CH_R + (r * LDR + 8 * ch) * 2, rsrc + r * D + 8 * ch);
         }
         if (tid < 32) cp_async16(base + CH_G + 16 * tid, a.gam + cidx * D + 4 * tid);
         cp_async_commit();
@@ -499,7 +500,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
         __syncthreads();
         const uint32_t wb = sb + buf * CH_BUF + CH_W, kb = sb + buf * CH_BUF + CH_K;
         const float *gam = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_G);
-        const float *rt = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_R);
+        const __nv_bfloat16 *rt = reinterpret_cast<const __nv_bfloat16 *>(sm + buf * CH_BUF + CH_R);
         // dS_n^T for the gradient kernel, and as bf16 A fragments
         uint32_t aS[8][4];
         __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
@@ -532,8 +533,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
             const float2 gm = *reinterpret_cast<const float2 *>(gam + 8 * nt + 2 * t4);
-            const float2 r0 = *reinterpret_cast<const float2 *>(rt + (j0 + g) * LDR + 8 * nt + 2 * t4);
-            const float2 r1 = *reinterpret_cast<const float2 *>(rt + (j0 + g + 8) * LDR + 8 * nt + 2 * t4);
+            const uint32_t r0w = *reinterpret_cast<const uint32_t *>(rt + (j0 + g) * LDR + 8 * nt + 2 * t4);
+            const uint32_t r1w = *reinterpret_cast<const uint32_t *>(rt + (j0 + g + 8) * LDR + 8 * nt + 2 * t4);
+            const float2 r0 = make_float2(bf_lo(r0w), bf_hi(r0w)), r1 = make_float2(bf_lo(r1w), bf_hi(r1w));
             dS[nt][0] = dS[nt][0] * gm.x + r0.x;
             dS[nt][1] = dS[nt][1] * gm.y + r0.y;
             dS[nt][2] = dS[nt][2] * gm.x + r1.x;
@@ -936,7 +938,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
     a.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
     a.gam = reinterpret_cast<float *>(base + l.gam);
-    a.Rt = reinterpret_cast<float *>(base + l.Rt);
+    a.Rt = reinterpret_cast<__nv_bfloat16 *>(base + l.Rt);
     a.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
     a.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
     a.dSn = reinterpret_cast<__nv_bfloat16 *>(base + l.dSn);

@@ -171,7 +171,7 @@ GDN2_API gdn2_status gdn2_chunk_bwd_saved(gdn2_dtype dt, int B, int T, int H, in
  *   and holds it until the process exits.  A problem is accepted when
  *   gdn2_workspace_size(1, ...) <= GDN2_NOALLOC_MAX_SCRATCH_BYTES (for
  *   example B*H = 2, T = 1024, d = 128 needs 20.5 MiB with fp32 inputs and
- *   5.5 MiB with bf16 inputs); larger ones return GDN2_ERR_TOO_LARGE before
+ *   4.6 MiB with bf16 inputs); larger ones return GDN2_ERR_TOO_LARGE before
  *   anything is launched.
  *   Allocation: none.  No cudaMalloc, cudaFree or allocating library call.
  *   First call per device: looks up the array's device address with

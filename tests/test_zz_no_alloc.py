@@ -31,7 +31,7 @@ def test_noalloc_rejects_before_any_cuda_call():
     # fp32, B*H = 1, T = 4096, d = 128 needs 37.25 MiB of scratch: over the limit
     assert lib.gdn2_workspace_size(1, 0, 1, 4096, 1, 128, 128) > g.NOALLOC_MAX_SCRATCH_BYTES
     assert noalloc_raw(lib, 0, 1, 4096, 1, 128) == -9
-    # bf16, B*H = 4, T = 4096, d = 128 needs 44.25 MiB
+    # bf16, B*H = 4, T = 4096, d = 128 needs 36.25 MiB
     assert lib.gdn2_workspace_size(1, 1, 1, 4096, 4, 128, 128) > g.NOALLOC_MAX_SCRATCH_BYTES
     assert noalloc_raw(lib, 1, 1, 4096, 4, 128) == -9
     assert b"static" in lib.gdn2_strerror(-9)
