@@ -26,7 +26,11 @@ template <> struct Vec<64> { using T = float2; };
 __device__ __forceinline__ void scale_fma(float4 &s, float a) { s.x *= a; s.y *= a; s.z *= a; s.w *= a; }
 __device__ __forceinline__ void scale_fma(float2 &s, float a) { s.x *= a; s.y *= a; }
 
-template <int D, typename Tin>
+__device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
+
+// kPro: the fused input prologue (kProNorm | kProSigmoid of gdn2_internal.cuh): q and k are
+// L2-normalised in the block before use, b and w pass through the sigmoid.
+template <int D, typename Tin, int kPro>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const Tin *__restrict__ b, const Tin *__restrict__ w,
@@ -38,6 +42,7 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
     __shared__ float s_q[D], s_k[D], s_e[D], s_a[D], s_u[D];
     __shared__ float s_r[kWarps][D], s_p[kWarps][D];
     __shared__ float s_kq;
+    __shared__ float s_nrm[D / 32][2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t nh = blockIdx.x;
@@ -52,11 +57,37 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
         sv[r] = __ldcs(reinterpret_cast<const V *>(Sp + (size_t)row * D) + lane);
     }
     if (tid < D) {
-        const float kv = to_f(k[vec + tid]), qv = to_f(q[vec + tid]);
+        float kv = to_f(k[vec + tid]), qv = to_f(q[vec + tid]);
+        if (kPro & kProNorm) {  // |q|^2, |k|^2: warp sums, combined below
+            float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            }
+            if (lane == 0) {
+                s_nrm[warp][0] = sq;
+                s_nrm[warp][1] = sk;
+            }
+        }
+        s_a[tid] = expf(g[vec + tid]);
         s_q[tid] = qv;
         s_k[tid] = kv;
-        s_e[tid] = to_f(b[vec + tid]) * kv;
-        s_a[tid] = expf(g[vec + tid]);
+    }
+    if (kPro & kProNorm) __syncthreads();
+    if (tid < D) {
+        float qv = s_q[tid], kv = s_k[tid];
+        if (kPro & kProNorm) {
+            float nq = 0.f, nk = 0.f;
+#pragma unroll
+            for (int wi = 0; wi < D / 32; ++wi) { nq += s_nrm[wi][0]; nk += s_nrm[wi][1]; }
+            qv *= rsqrtf(nq + kNormEps);
+            kv *= rsqrtf(nk + kNormEps);
+            s_q[tid] = qv;
+            s_k[tid] = kv;
+        }
+        const float bv = to_f(b[vec + tid]);
+        s_e[tid] = ((kPro & kProSigmoid) ? sigmoid(bv) : bv) * kv;
     }
     __syncthreads();
     if (warp == 0) {
@@ -85,7 +116,8 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
         float r = 0.f, pq = 0.f;
 #pragma unroll
         for (int wi = 0; wi < kWarps; ++wi) { r += s_r[wi][tid]; pq += s_p[wi][tid]; }
-        const float u = to_f(w[vec + tid]) * to_f(v[vec + tid]) - r;
+        const float wv = to_f(w[vec + tid]);
+        const float u = ((kPro & kProSigmoid) ? sigmoid(wv) : wv) * to_f(v[vec + tid]) - r;
         s_u[tid] = u;
         o[vec + tid] = from_f<Tin>(pq + s_kq * u);
     }
@@ -106,25 +138,33 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
 
 template <int D, typename Tin>
 cudaError_t launch_t(int N, int H, const void *q, const void *k, const void *v, const float *g,
-                     const void *b, const void *w, float *S, void *o, cudaStream_t s)
+                     const void *b, const void *w, float *S, void *o, int pro, cudaStream_t s)
 {
-    decode_kernel<D, Tin><<<N * H, kWarps * 32, 0, s>>>(H, (const Tin *)q, (const Tin *)k,
-                                                        (const Tin *)v, g, (const Tin *)b,
-                                                        (const Tin *)w, S, (Tin *)o);
-    return cudaGetLastError();
+    auto go = [&](auto kernel) {
+        kernel<<<N * H, kWarps * 32, 0, s>>>(H, (const Tin *)q, (const Tin *)k, (const Tin *)v, g, (const Tin *)b,
+                                             (const Tin *)w, S, (Tin *)o);
+        return cudaGetLastError();
+    };
+    switch (pro) {
+    case kProNorm: return go(decode_kernel<D, Tin, kProNorm>);
+    case kProSigmoid: return go(decode_kernel<D, Tin, kProSigmoid>);
+    case kProNorm | kProSigmoid: return go(decode_kernel<D, Tin, kProNorm | kProSigmoid>);
+    default: return go(decode_kernel<D, Tin, 0>);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
-                          void *o, cudaStream_t s)
+                          void *o, cudaStream_t s, int prologue)
 {
+    if (prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
     if (dt == GDN2_F32)
-        return D == 64 ? launch_t<64, float>(N, H, q, k, v, g, b, w, S, o, s)
-                       : launch_t<128, float>(N, H, q, k, v, g, b, w, S, o, s);
-    return D == 64 ? launch_t<64, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, s)
-                   : launch_t<128, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, s);
+        return D == 64 ? launch_t<64, float>(N, H, q, k, v, g, b, w, S, o, prologue, s)
+                       : launch_t<128, float>(N, H, q, k, v, g, b, w, S, o, prologue, s);
+    return D == 64 ? launch_t<64, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, s)
+                   : launch_t<128, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, s);
 }
 
 }  // namespace gdn2

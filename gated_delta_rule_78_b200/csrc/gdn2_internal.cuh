@@ -155,7 +155,7 @@ cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
-                          void *o, cudaStream_t s);
+                          void *o, cudaStream_t s, int prologue = 0);
 
 struct BwdOut {
     void *dq, *dk, *dv, *db, *dw;

@@ -248,8 +248,9 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
  *   GDN2_BW_LOGITS: b and w, where present, are logits (either layout) and pass through
  *     the logistic sigmoid 1 / (1 + e^-x).
  * The bf16 forward with per-channel b and w applies both inside the tensor-core chunk
- * kernel (the sigmoid there goes through the hardware tanh, 1/2 + tanh(x/2)/2); every
- * other call writes the normalised / activated inputs into its workspace first.  The
+ * kernel (the sigmoid there goes through the hardware tanh, 1/2 + tanh(x/2)/2), and the
+ * decode step with per-channel b and w inside its kernel; every other call writes the
+ * normalised / activated inputs into its workspace first.  The
  * backward returns dq, dk for the raw q, k and db, dw for the logits.
  */
 typedef enum {

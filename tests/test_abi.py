@@ -136,7 +136,11 @@ def test_gated_flags_and_workspace(lib):
     assert lib.gdn2_workspace_size_gated(1, pro, BF16, 2, 128, 4, 128, 128) == plain + 4 * one
     # scalar b logits: q_n, k_n, per-token b_s, w_s, then the broadcast b
     assert lib.gdn2_workspace_size_gated(0, pro | g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == 4 * one + 2 * 128 * 4 * 2
-    assert lib.gdn2_workspace_size_gated(2, g.QK_L2NORM, BF16, 8, 0, 4, 128, 128) == 2 * 8 * 4 * 128 * 2
+    # decode: fused for per-channel b and w; a scalar b logit goes through the pass
+    # (q_n, k_n, w_s per channel, b_s per token, then the broadcast b)
+    assert lib.gdn2_workspace_size_gated(2, g.QK_L2NORM, BF16, 8, 0, 4, 128, 128) == 0
+    assert lib.gdn2_workspace_size_gated(2, pro | g.ERASE_SCALAR, BF16, 8, 0, 4, 128, 128) == \
+        3 * 8 * 4 * 128 * 2 + 256 + 8 * 4 * 128 * 2
 
 
 def test_workspace_size(lib):

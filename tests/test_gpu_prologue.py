@@ -168,3 +168,36 @@ def test_standalone_prologue_matches_oracle(cuda_lib, dtype, D):
     assert out["w"] is None
     assert_close(out["b"], oracle.ref_prologue(x["q"], x["k"], bl, None)[2], dtype, "b (per token)")
     assert g.gdn2_sync_status() == 0
+
+
+@pytest.mark.parametrize("dtype,flags", [("f32", PRO), ("bf16", g.QK_L2NORM), ("bf16", g.BW_LOGITS),
+                                         ("bf16", PRO | g.ERASE_SCALAR)])
+def test_decode_prologue_variants(cuda_lib, dtype, flags):
+    """Fused into the decode kernel for per-channel b and w (every flag combination, both dtypes);
+    a per-token erase-gate logit goes through the prologue pass."""
+    N, H, D, steps = 4, 2, 64 if dtype == "f32" else 128, 6
+    ds = DecodeStream(N, H, D, D, dtype=dtype, seed=47)
+    S = ds.S0.clone().cuda()
+    Sr = ds.S0.double().numpy().copy()
+    gen = torch.Generator().manual_seed(3)
+    for _ in range(steps):
+        s = ds.step(raw=True)
+        if not flags & g.BW_LOGITS:
+            s["b"] = torch.sigmoid(s["b"].float()).to(s["q"].dtype)
+            s["w"] = torch.sigmoid(s["w"].float()).to(s["q"].dtype)
+        if not flags & g.QK_L2NORM:
+            for n in ("q", "k"):
+                t = s[n].float()
+                s[n] = (t / t.norm(dim=-1, keepdim=True)).to(s["q"].dtype)
+        b_in, b_ref = s["b"], s["b"]
+        if flags & g.ERASE_SCALAR:
+            b_in = torch.randn(N, H, generator=gen).to(s["q"].dtype)
+            b_ref = b_in[..., None].expand(N, H, D)
+        o = g.gdn2_decode_step_gated(dev(s["q"]), dev(s["k"]), dev(s["v"]), dev(s["log_alpha"]), dev(b_in),
+                                     dev(s["w"]), S, flags=flags)
+        qn, kn, bs, ws = oracle.ref_prologue(s["q"], s["k"], b_ref, s["w"], norm=bool(flags & g.QK_L2NORM),
+                                             sigmoid=bool(flags & g.BW_LOGITS))
+        ro, Sr = oracle.ref_decode(qn, kn, s["v"], s["log_alpha"], bs, ws, Sr)
+        assert_close(o, ro, dtype, "o")
+    assert g.gdn2_sync_status() == 0
+    assert_close(S, Sr, dtype, "S")
