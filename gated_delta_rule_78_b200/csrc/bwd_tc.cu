@@ -23,13 +23,16 @@
 //   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO),
 // so the work splits into four launches:
 //   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary;
-//   2. bwd_prep_kernel, one CTA per chunk: factors, [A; P], T, W, R (no state needed);
+//   2. bwd_prep_tc_kernel, one CTA per chunk: factors, [A; P], T, W^T, R^T (no state
+//      needed), the products as tcgen05 MMAs with TMEM accumulators;
 //   3. bwd_chain_kernel, one CTA per (batch, head): the reverse dS chain,
 //      two warp MMAs per chunk with dS^T kept in registers; stores dS_n per chunk;
 //   4. bwd_grad_kernel, one CTA per chunk: recomputes U~ from the stored state and
 //      produces every gradient of the chunk.
-// All products are bf16 warp MMAs (m16n8k16) on ldmatrix-fed swizzled tiles.
+// The chain and gradient products are bf16 warp MMAs (m16n8k16) on ldmatrix-fed
+// swizzled tiles.
 #include <cuda.h>
+#include <string.h>
 
 #include "gdn2_internal.cuh"
 #include "tc_util.cuh"
@@ -50,8 +53,8 @@ struct BwdTcLayout {
     size_t coff, states, W, Kh, gam, Rt, Tm, Pm, dSn, total;
 };
 
-// Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W and K^ bf16
-// [C][D], gamma fp32 [D], R^T bf16 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
+// Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W^T bf16 [D][C],
+// K^ bf16 [C][D], gamma fp32 [D], R^T bf16 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
 // Variable length puts chunk_off first; chunk lists are sized by the chunk bound.
 BwdTcLayout tc_layout(const Problem &p)
 {
@@ -84,6 +87,7 @@ struct BwdTcArgs {
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
     int n_sm;            // multiprocessors of the device (L2 prefetch distance of the gradient kernel)
+    int *status;         // kernel status word (bounded waits that gave up)
 };
 
 // ------------------------------------------------------------------ small helpers
@@ -247,192 +251,332 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t x, uint32_t y)
     return r;
 }
 
-// ================================================================== 2. prep
-// smem map (bytes): six [C][D] bf16 tiles, T and P bf16 [C][C], A and T fp32 [C][LDA],
-// the cumsum scratch.
-constexpr uint32_t P_Q = 0, P_E = 16384, P_K = 32768, P_DO = 49152, P_W = 65536, P_Z = 81920;
-constexpr uint32_t P_TB = 98304, P_PB = 106496, P_SA = 114688, P_ST = P_SA + C * LDA * 4;
-constexpr uint32_t P_TOT = P_ST + C * LDA * 4;
-constexpr uint32_t P_SET1 = P_TOT + 8 * D * 4;     // second set of the raw q, b, k, dO tiles
-constexpr uint32_t P_SMEM = P_SET1 + 4 * 16384;
-constexpr int kPrepThreads = 512;
-
 // L2 prefetch (bulk, no shared-memory destination)
 __device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
 {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Persistent: block x takes the (chunk, head) tasks x, x + gridDim.x, ...  The raw tiles of
-// the next task are copied (cp.async) into the other tile set, and its log alpha loaded,
-// while the current task computes.
-__global__ void __launch_bounds__(kPrepThreads, 1) bwd_prep_kernel(const BwdTcArgs a, int nbound)
-{
-    extern __shared__ __align__(1024) uint8_t sm[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cp = tid & 63, g8 = tid >> 6;  // decay-folding mapping: channel pair, group of 8 tokens
-    const uint32_t sb = smem_u32(sm);
-    float *sA = reinterpret_cast<float *>(sm + P_SA);
-    float *sT = reinterpret_cast<float *>(sm + P_ST);
-    const int ntasks = nbound * a.H;
-    // tile set offsets (the raw tiles become the factors in place)
-    auto tile = [](int buf, int which) -> uint32_t {  // which: 0 q, 1 b, 2 k, 3 dO
-        const uint32_t base0[4] = {P_Q, P_E, P_K, P_DO};
-        return buf ? P_SET1 + which * 16384u : base0[which];
-    };
-    auto issue = [&](int task, int buf, float2 (&Gn)[8]) {
-        ChunkRef r;
-        if (task >= ntasks || !chunk_ref_at(a, task % nbound, task / nbound, r)) return;
-        const int Lr = min(C, r.sp.len - r.ci * C);
-        cp_tok_tile(sb + tile(buf, 0), a.q, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
-        cp_tok_tile(sb + tile(buf, 2), a.k, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
-        cp_tok_tile(sb + tile(buf, 1), a.b, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
-        cp_tok_tile(sb + tile(buf, 3), a.dO, a, r.sp.bos, r.h, r.ci, Lr, tid, kPrepThreads);
-        load_g8(Gn, a, r.sp.bos, r.h, r.ci, Lr, cp, g8);
-    };
-    float2 Gnext[8];
-    issue(blockIdx.x, 0, Gnext);
-    cp_async_commit();
-    int it = 0;
-    for (int task = blockIdx.x; task < ntasks; task += gridDim.x, ++it) {
-    const int buf = it & 1;
-    float2 G[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) G[i] = Gnext[i];
-    issue(task + gridDim.x, buf ^ 1, Gnext);  // the next task's copies, into the other set
-    cp_async_commit();
-    ChunkRef cr;
-    if (!chunk_ref_at(a, task % nbound, task / nbound, cr)) {
-        cp_async_wait<1>();
-        __syncthreads();
-        continue;
-    }
-    const int L = min(C, cr.sp.len - cr.ci * C);
-    const size_t cidx = cr.cidx;
-    const uint32_t P_Qb = tile(buf, 0), P_Eb = tile(buf, 1), P_Kb = tile(buf, 2), P_DOb = tile(buf, 3);
+// ================================================================== 2. prep on the tensor cores
+// One 512-thread CTA per (chunk, head): the raw q, b, k, dO tiles arrive by TMA (SW128 atoms),
+// the decay folds into them in place, and the four products run as tcgen05 MMAs with TMEM
+// accumulators:
+//   [A; P] = [E~; Q~] K~^T             M = 128 (stacked tokens), N = 64, K = 128
+//   Z^T    = dO^T P                    M = 128 (d_v), N = 64, K = 64   (dO, P MN-major)
+//   W^T    = E~^T T^T                  M = 128 (d_k), N = 64, K = 64   (E~ MN-major)
+//   R^T    = dO^T Q~ + (-Z^T) W        M = 128 (d_v), N = 128, K = 64 + 64 (-Z^T from TMEM)
+// T = (I + A)^-1 is the blocked solve on four warps, as in the forward.  Written out: K^, gamma,
+// T, P, W^T (rows d_k, for the chain) and R^T (bf16).
+namespace prep_tc {
+constexpr uint32_t QE = 0;          // [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
+constexpr uint32_t KT = 32768;      // K~ [a0 | a1]
+constexpr uint32_t DO = 49152;      // dO [a0 | a1]
+constexpr uint32_t TT = 65536;      // T bf16 [64][64]
+constexpr uint32_t PP = 73728;      // P bf16 [64][64]
+constexpr uint32_t WT = 81920;      // W^T bf16 [128 rows d_k][64 tokens]
+constexpr uint32_t SA = 98304;      // A fp32 [64][LDA]
+constexpr uint32_t ST = SA + 64 * LDA * 4;   // T fp32 [64][LDA]
+constexpr uint32_t TOT = ST + 64 * LDA * 4;  // decay totals [8][D] fp32
+constexpr uint32_t USED = TOT + 8 * D * 4;
+constexpr uint32_t SMEM = USED + 1024;       // slack for the 1024-byte alignment
+constexpr uint32_t TM_AP = 0, TM_WT = 64, TM_ZT = 128, TM_ZB = 192, TM_RT = 256, TM_COLS = 512;
+constexpr uint32_t IDESC_AP = tc::idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 1, 1);
+constexpr uint32_t IDESC_W = tc::idesc_bf16(128, 64, 1, 0);
+constexpr uint32_t IDESC_R1 = tc::idesc_bf16(128, 128, 1, 1);
+constexpr uint32_t IDESC_R2 = tc::idesc_bf16(128, 128, 0, 0);
+constexpr int kThreads = 512;
+}  // namespace prep_tc
 
-    // ---- T scratch zeroed (its upper blocks stay zero)
-    for (int idx = tid; idx < C * LDA; idx += kPrepThreads) sT[idx] = 0.f;
-    // ---- decay folding (thread: channels 2 cp, 2 cp + 1, 8 tokens); K^ and gamma go straight out
+struct PrepMaps {
+    CUtensorMap q, k, b, dO, g;
+};
+
+__device__ __forceinline__ void named_bar(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__global__ void __launch_bounds__(prep_tc::kThreads, 1)
+bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
+{
+    using namespace prep_tc;
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_in, bar_ap, bar_z, bar_w, bar_r;
+    __shared__ uint32_t s_tmem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    ChunkRef cr;
+    if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
+    const int ci = cr.ci, hh = cr.h, bos = cr.sp.bos;
+    const int L = min(C, cr.sp.len - ci * C);
+    const size_t cidx = cr.cidx;
+    const uint32_t sb = smem_u32(sm);
+    float *sA = reinterpret_cast<float *>(sm + SA);
+    float *sT = reinterpret_cast<float *>(sm + ST);
+    float *sTot = reinterpret_cast<float *>(sm + TOT);
+
+    if (tid == 0) {
+        mbar_init(&bar_in, 1);
+        mbar_init(&bar_ap, 1);
+        mbar_init(&bar_z, 1);
+        mbar_init(&bar_w, 1);
+        mbar_init(&bar_r, 1);
+        fence_mbar_init();
+        prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b); prefetch_tmap(&maps.dO);
+        prefetch_tmap(&maps.g);
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, TM_COLS);
+        tmem_relinquish();
+    }
+    for (int idx = tid; idx < 64 * LDA; idx += kThreads) sT[idx] = 0.f;  // upper blocks stay zero
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const int y = bos + ci * C;
+    if (tid == 0) {
+        mbar_expect_tx(&bar_in, 8 * 8192);
+        for (int at = 0; at < 2; ++at) {
+            tma_load_3d(sm + KT + at * 8192, &maps.k, at * 64, hh, y, &bar_in);
+            tma_load_3d(sm + QE + at * 16384, &maps.b, at * 64, hh, y, &bar_in);
+            tma_load_3d(sm + QE + 8192 + at * 16384, &maps.q, at * 64, hh, y, &bar_in);
+            tma_load_3d(sm + DO + at * 8192, &maps.dO, at * 64, hh, y, &bar_in);
+        }
+        for (int at = 0; at < a.din / 32; ++at) tma_prefetch_3d(&maps.g, at * 32, hh, y);
+    }
+
+    // ---- decay folding: thread (channel block cb, token group tg of 8, lane): channels
+    //      64 cb + 2 lane (+1), tokens 8 tg .. 8 tg + 7
+    const int cb = warp & 1, tg = warp >> 1, ch = 64 * cb + 2 * lane;
     {
-        float2 eG[8], emG[8], tot;
-        decay_pair8<true, 1>(G, eG, emG, tot, cp, g8, reinterpret_cast<float *>(sm + P_TOT));
-        const float gam0 = __expf(tot.x), gam1 = __expf(tot.y);  // K^ = k e^(G_C - G) = gamma K~
-        if (g8 == 0) *reinterpret_cast<float2 *>(a.gam + cidx * D + 2 * cp) = make_float2(gam0, gam1);
+        float2 gv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * tg + i;
+            gv[i] = (t < L && ch < a.din)
+                        ? __ldg(reinterpret_cast<const float2 *>(a.g + tok_off(a, bos, hh, ci, t) + ch))
+                        : make_float2(0.f, 0.f);
+        }
+        float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            run0 += gv[i].x;
+            run1 += gv[i].y;
+            gv[i] = make_float2(__expf(gv[i].x), __expf(gv[i].y));  // alpha
+        }
+        *reinterpret_cast<float2 *>(sTot + tg * D + ch) = make_float2(run0, run1);
+        if (!mbar_wait(&bar_in, 0)) atomicExch(a.status, kStatusTimeout);
+        __syncthreads();
+        float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float2 v = *reinterpret_cast<const float2 *>(sTot + u * D + ch);
+            if (u < tg) { off0 += v.x; off1 += v.y; }
+            tot0 += v.x;
+            tot1 += v.y;
+        }
+        const float gam0 = __expf(tot0), gam1 = __expf(tot1);
+        if (tg == 0) *reinterpret_cast<float2 *>(a.gam + cidx * D + ch) = make_float2(gam0, gam1);
+        float2 mv[8];  // e^-G, backwards from the group's last token
+        {
+            float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
+#pragma unroll
+            for (int i = 7; i >= 0; --i) {
+                mv[i] = make_float2(r0, r1);
+                r0 *= gv[i].x;
+                r1 *= gv[i].y;
+            }
+        }
+        float e0 = __expf(off0), e1 = __expf(off1);
+        uint8_t *pe = sm + QE + cb * 16384, *pq = pe + 8192, *pk = sm + KT + cb * 8192;
         __nv_bfloat16 *kh = a.Kh + cidx * C * D;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int t = 8 * g8 + i;
-            const uint32_t off = swz(t, 2 * cp, 256);
-            uint32_t *pq = reinterpret_cast<uint32_t *>(sm + P_Qb + off);
-            uint32_t *pk = reinterpret_cast<uint32_t *>(sm + P_Kb + off);
-            uint32_t *pe = reinterpret_cast<uint32_t *>(sm + P_Eb + off);
-            const uint32_t q2 = *pq, k2 = *pk, b2 = *pe;
-            const float k0 = bf_lo(k2), k1 = bf_hi(k2);
-            *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
-            *pe = pack_bf16x2(bf_lo(b2) * k0 * eG[i].x, bf_hi(b2) * k1 * eG[i].y);
-            *pk = pack_bf16x2(k0 * emG[i].x, k1 * emG[i].y);
-            *reinterpret_cast<uint32_t *>(kh + t * D + 2 * cp) =
-                pack_bf16x2(k0 * emG[i].x * gam0, k1 * emG[i].y * gam1);
+            const int t = 8 * tg + i;
+            e0 *= gv[i].x;
+            e1 *= gv[i].y;
+            const uint32_t off = sw128(t, 4 * lane);
+            uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
+            uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
+            uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
+            if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
+            const float k0 = bf_lo(kw), k1 = bf_hi(kw), m0 = mv[i].x, m1 = mv[i].y;
+            *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
+            *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
+            *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
+            *reinterpret_cast<uint32_t *>(kh + t * D + ch) = pack_bf16x2(k0 * m0 * gam0, k1 * m1 * gam1);
         }
     }
+    fence_proxy_async_smem();
     __syncthreads();
-    // ---- [A; P] = [E~; Q~] K~^T (128 x 64, K = 128): warp = 16 stacked rows x 32 columns
-    {
-        const int mt = warp & 7, nh = warp >> 3;
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, false, false, D>(acc, sb + (mt < 4 ? P_Eb : P_Qb), 256, 16 * (mt & 3), sb + P_Kb, 256, 32 * nh,
-                                         lane);
-        const int g = lane >> 2, t4 = lane & 3;
+    // ---- [A; P] = [E~; Q~] K~^T
+    if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = 16 * (mt & 3) + g + 8 * hr, col = 32 * nh + 8 * nt + 2 * t4;
-                const float v0 = acc[0][nt][2 * hr], v1 = acc[0][nt][2 * hr + 1];
-                if (mt < 4) {
-                    sA[row * LDA + col] = (col < row) ? v0 : 0.f;
-                    sA[row * LDA + col + 1] = (col + 1 < row) ? v1 : 0.f;
-                } else {
-                    st_pair(sm + P_PB, 128, row, col, (col <= row) ? v0 : 0.f, (col + 1 <= row) ? v1 : 0.f);
-                }
-            }
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_AP, sdesc_sw128(sb + QE + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sb + KT + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_AP, ks > 0);
+        mma_commit(&bar_ap);
     }
+    if (!mbar_wait(&bar_ap, 0)) atomicExch(a.status, kStatusTimeout);
+    tc_fence_after();
+    if (warp < 8) {  // A -> fp32 scratch (strictly lower), P -> bf16 tile (lower incl.)
+        const int quarter = warp & 3, half = warp >> 2;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint32_t r[32];
+        tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
+        tmem_wait_ld();
+        const int row = quarter * 32 + lane;
+        if (row < 64) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int j = 32 * half + u;
+                sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
+            }
+        } else {
+            const int t = row - 64;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i0 = 32 * half + 8 * m + 2 * e;
+                    w4[e] = pack_bf16x2((i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f,
+                                        (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(sm + PP + sw128(t, 64 * half + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // ---- T = (I + A)^-1 on warps 0-3; meanwhile warps 8-15 form -Z = -(P^T dO)
+    // ---- T = (I + A)^-1 on warps 0-3; Z^T = dO^T P issued meanwhile
     if (warp < 4) {
-        solve_unit_lower64<LDA>(sA, sT, warp, lane, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
-    } else if (warp >= 8) {
-        const int mt = warp & 3, nh = (warp >> 2) & 1;
-        float acc[1][8][4];
-        zero_acc(acc);
-        warp_gemm<1, 8, true, true, C>(acc, sb + P_PB, 128, 16 * mt, sb + P_DOb, 256, 64 * nh, lane);
-        const int g = lane >> 2, t4 = lane & 3;
+        wm::solve_unit_lower64<LDA>(sA, sT, warp, lane, [] { named_bar(1, 128); });
+    } else if (tid == 128) {
+        tc_fence_after();
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-                st_pair(sm + P_Z, 256, 16 * mt + g + 8 * hr, 64 * nh + 8 * nt + 2 * t4, -acc[0][nt][2 * hr],
-                        -acc[0][nt][2 * hr + 1]);
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_ZT, sdesc_sw128(sb + DO + ks * 2048, 8192, 1024), sdesc_sw128(sb + PP + ks * 2048, 8192, 1024),
+                   IDESC_Z, ks > 0);
+        mma_commit(&bar_z);
     }
     __syncthreads();
-    // ---- T -> bf16 tile and global; P -> global (one 16-byte chunk per thread)
+    // ---- T -> bf16 tile and global (threads 0-255), P -> global (threads 256-511): 16 columns each
     {
-        const int i = tid >> 3, jc = tid & 7;
-        float tv[8];
+        const int u = tid & 255, i = u >> 2, jq = u & 3;
+        if (tid < 256) {
+            uint32_t w8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) tv[e] = (8 * jc + e <= i) ? sT[i * LDA + 8 * jc + e] : 0.f;
-        const uint4 pk = make_uint4(pack_bf16x2(tv[0], tv[1]), pack_bf16x2(tv[2], tv[3]), pack_bf16x2(tv[4], tv[5]),
-                                    pack_bf16x2(tv[6], tv[7]));
-        *reinterpret_cast<uint4 *>(sm + P_TB + swz(i, 8 * jc, 128)) = pk;
-        *reinterpret_cast<uint4 *>(a.Tm + cidx * C * C + i * C + 8 * jc) = pk;
-        *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 8 * jc) =
-            *reinterpret_cast<const uint4 *>(sm + P_PB + swz(i, 8 * jc, 128));
-    }
-    __syncthreads();
-    // ---- W = T E~ (64 x 128, K = 64): warp = 16 rows x 32 columns
-    {
-        const int mt = warp & 3, nq = warp >> 2;
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, false, true, C>(acc, sb + P_TB, 128, 16 * mt, sb + P_Eb, 256, 32 * nq, lane);
-        const int g = lane >> 2, t4 = lane & 3;
-        __nv_bfloat16 *wg = a.W + cidx * C * D;
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = 16 * mt + g + 8 * hr, col = 32 * nq + 8 * nt + 2 * t4;
-                const uint32_t pk = pack_bf16x2(acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
-                *reinterpret_cast<uint32_t *>(sm + P_W + swz(row, col, 256)) = pk;
-                *reinterpret_cast<uint32_t *>(wg + row * D + col) = pk;
+            for (int e = 0; e < 8; ++e) {
+                const int j0 = 16 * jq + 2 * e;
+                w8[e] = pack_bf16x2((j0 <= i) ? sT[i * LDA + j0] : 0.f, (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f);
             }
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const uint4 v = make_uint4(w8[4 * h2], w8[4 * h2 + 1], w8[4 * h2 + 2], w8[4 * h2 + 3]);
+                *reinterpret_cast<uint4 *>(sm + TT + sw128(i, 32 * jq + 16 * h2)) = v;
+                *reinterpret_cast<uint4 *>(a.Tm + cidx * C * C + i * C + 16 * jq + 8 * h2) = v;
+            }
+        } else {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2)
+                *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 16 * jq + 8 * h2) =
+                    *reinterpret_cast<const uint4 *>(sm + PP + sw128(i, 32 * jq + 16 * h2));
+        }
     }
+    fence_proxy_async_smem();
     __syncthreads();
-    // ---- R^T = dO^T Q~ + (-Z)^T W (128 x 128, K = 64 + 64): warp = 32 x 32
-    {
-        const int mb = warp & 3, nb = warp >> 2;
-        float acc[2][4][4];
-        zero_acc(acc);
-        warp_gemm<2, 4, true, true, C>(acc, sb + P_DOb, 256, 32 * mb, sb + P_Qb, 256, 32 * nb, lane);
-        warp_gemm<2, 4, true, true, C>(acc, sb + P_Z, 256, 32 * mb, sb + P_W, 256, 32 * nb, lane);
-        const int g = lane >> 2, t4 = lane & 3;
-        __nv_bfloat16 *rt = a.Rt + cidx * D * D;
+    // ---- W^T = E~^T T^T
+    if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int row = 32 * mb + 16 * mt + g + 8 * hr, col = 32 * nb + 8 * nt + 2 * t4;
-                    *reinterpret_cast<uint32_t *>(rt + row * D + col) =
-                        pack_bf16x2(acc[mt][nt][2 * hr], acc[mt][nt][2 * hr + 1]);
-                }
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_WT, sdesc_sw128(sb + QE + ks * 2048, 16384, 1024), sdesc_sw128(sb + TT + ks * 32, 16, 1024),
+                   IDESC_W, ks > 0);
+        mma_commit(&bar_w);
     }
-    __syncthreads();  // every warp is done with this task's tiles before they are refilled
+    // -Z^T -> bf16 A operand (warps 0-3: lanes d_v, 64 columns)
+    if (!mbar_wait(&bar_z, 0)) atomicExch(a.status, kStatusTimeout);
+    tc_fence_after();
+    if (warp < 4) {
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t r[32], pk[16];
+            tmem_ld32(tmem + TM_ZT + 32 * h2 + lane_off, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(-__uint_as_float(r[2 * e]), -__uint_as_float(r[2 * e + 1]));
+            tmem_st16(tmem + TM_ZB + 16 * h2 + lane_off, pk);
+        }
+        tmem_wait_st();
     }
-    cp_async_wait<0>();
+    // W^T -> bf16 tile (rows d_k, the B operand of R^T) and global (warps 4-7)
+    if (!mbar_wait(&bar_w, 0)) atomicExch(a.status, kStatusTimeout);
+    tc_fence_after();
+    if (warp >= 4 && warp < 8) {
+        const int quarter = warp & 3, c = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        __nv_bfloat16 *wg = a.W + cidx * C * D + (size_t)c * C;  // W^T [d_k][C]
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t r[32];
+            tmem_ld32(tmem + TM_WT + 32 * h2 + lane_off, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[8 * m]), __uint_as_float(r[8 * m + 1])),
+                                           pack_bf16x2(__uint_as_float(r[8 * m + 2]), __uint_as_float(r[8 * m + 3])),
+                                           pack_bf16x2(__uint_as_float(r[8 * m + 4]), __uint_as_float(r[8 * m + 5])),
+                                           pack_bf16x2(__uint_as_float(r[8 * m + 6]), __uint_as_float(r[8 * m + 7])));
+                *reinterpret_cast<uint4 *>(sm + WT + sw128(c, 64 * h2 + 16 * m)) = v;
+                *reinterpret_cast<uint4 *>(wg + 32 * h2 + 8 * m) = v;
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- R^T = dO^T Q~ + (-Z^T) W
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_RT, sdesc_sw128(sb + DO + ks * 2048, 8192, 1024),
+                   sdesc_sw128(sb + QE + 8192 + ks * 2048, 16384, 1024), IDESC_R1, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tmem + TM_RT, tmem + TM_ZB + 8 * ks, sdesc_sw128(sb + WT + ks * 32, 16, 1024), IDESC_R2, 1);
+        mma_commit(&bar_r);
+    }
+    if (!mbar_wait(&bar_r, 0)) atomicExch(a.status, kStatusTimeout);
+    tc_fence_after();
+    {  // R^T -> bf16, global [d_v][d_k]: warp = lane quarter x 32-column block
+        const int quarter = warp & 3, cq = warp >> 2, j = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        uint32_t r[32];
+        tmem_ld32(tmem + TM_RT + 32 * cq + lane_off, r);
+        tmem_wait_ld();
+        __nv_bfloat16 *rt = a.Rt + cidx * D * D + (size_t)j * D + 32 * cq;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<uint4 *>(rt + 8 * m) =
+                make_uint4(pack_bf16x2(__uint_as_float(r[8 * m]), __uint_as_float(r[8 * m + 1])),
+                           pack_bf16x2(__uint_as_float(r[8 * m + 2]), __uint_as_float(r[8 * m + 3])),
+                           pack_bf16x2(__uint_as_float(r[8 * m + 4]), __uint_as_float(r[8 * m + 5])),
+                           pack_bf16x2(__uint_as_float(r[8 * m + 6]), __uint_as_float(r[8 * m + 7])));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
 }
 
 // ================================================================== 3. chain
@@ -466,8 +610,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
         const __nv_bfloat16 *wsrc = a.W + cidx * C * D, *ksrc = a.Kh + cidx * C * D;
         for (int idx = tid; idx < C * 16; idx += kChainThreads) {
             const int t = idx >> 4, ch = idx & 15;
-            cp_async16(base + CH_W + swz(t, 8 * ch, 256), wsrc + t * D + 8 * ch);
             cp_async16(base + CH_K + swz(t, 8 * ch, 256), ksrc + t * D + 8 * ch);
+        }
+        for (int idx = tid; idx < D * 8; idx += kChainThreads) {  // W^T: 128 rows of 64 tokens
+            const int c = idx >> 3, ch = idx & 7;
+            cp_async16(base + CH_W + swz(c, 8 * ch, 128), wsrc + c * C + 8 * ch);
         }
         const __nv_bfloat16 *rsrc = a.Rt + cidx * D * D;
         for (int idx = tid; idx < D * 16; idx += kChainThreads) {  // 16 x 16 bytes per bf16 row
@@ -548,7 +695,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 #pragma unroll
             for (int np = 0; np < 8; ++np) {
                 uint32_t bfr[4];
-                load_b2<true>(bfr, wb, 256, 16 * kt, 16 * np, lane);
+                load_b2<false>(bfr, wb, 128, 16 * kt, 16 * np, lane);  // W^T stored [c][t] = [n][k]
                 mma_bf16(dS[2 * np], aZ, bfr[0], bfr[1]);
                 mma_bf16(dS[2 * np + 1], aZ, bfr[2], bfr[3]);
             }
@@ -949,6 +1096,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.dw = static_cast<__nv_bfloat16 *>(out.dw);
     a.dg = out.dg;
     a.dS0 = out.dS0;
+    a.status = status;
     {
         int dev = 0;
         a.n_sm = 148;
@@ -961,14 +1109,17 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         if (e != cudaSuccess) return e;
     }
     const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
-    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_kernel), (int)P_SMEM)) != cudaSuccess) return e;
-    {  // persistent: one block per SM, each streaming (chunk, head) tasks
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int nbound = (int)chunk_bound(p);
-        const long long ntasks = (long long)nbound * p.H;
-        const int grid = (int)(ntasks < sms ? ntasks : sms);
-        bwd_prep_kernel<<<grid, kPrepThreads, P_SMEM, s>>>(a, nbound);
+    {  // prep on the tensor cores: one block per (chunk, head)
+        PrepMaps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int rows = (int)token_rows(p);
+        if (!make_map(&maps.q, p.q, false, 1, rows, p.H, p.D) || !make_map(&maps.k, p.k, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D))
+            return cudaErrorInvalidValue;
+        if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_tc_kernel), (int)prep_tc::SMEM)) != cudaSuccess)
+            return e;
+        bwd_prep_tc_kernel<<<nblk, prep_tc::kThreads, prep_tc::SMEM, s>>>(maps, a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;

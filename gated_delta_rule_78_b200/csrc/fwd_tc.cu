@@ -695,11 +695,13 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     }
 }
 
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn()
+static EncodeTiledFn encode_fn()
 {
     static EncodeTiledFn fn = [] {
         void *f = nullptr;
@@ -715,22 +717,20 @@ EncodeTiledFn encode_fn()
 // 3-D view (channel, head, token) of a [B,T,H,din] tensor.  Loads: box = (one 128-byte
 // row of channels, 1 head, 64 tokens) with the 128-byte swizzle (a box past the channel
 // extent reads zeros); the output store: box = (all din channels, 1, 64 tokens), no swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, int din, bool store = false)
+bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, int din, bool store)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t es = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)din, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
     cuuint64_t strides[2] = {(cuuint64_t)din * es, (cuuint64_t)H * din * es};
-    cuuint32_t box[3] = {store ? (cuuint32_t)din : (fp32 ? 32u : 64u), 1u, (cuuint32_t)C};
+    cuuint32_t box[3] = {store ? (cuuint32_t)din : (fp32 ? 32u : 64u), 1u, (cuuint32_t)kChunk};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s, const ScanArgs *scan)

@@ -14,6 +14,13 @@
 #include <stdint.h>
 
 namespace gdn2 {
+
+// TMA tensor map of a [B, T, H, din] token tensor as a 3-D (channel, head, token) view.  Loads:
+// box = (one 128-byte row of channels, 1 head, 64 tokens) with the 128-byte swizzle (a box past
+// the channel extent reads zeros); store = true: box = (all din channels, 1, 64 tokens), no
+// swizzle.  Host function (fwd_tc.cu); false if the driver entry point or the encoding fails.
+bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, int din, bool store = false);
+
 namespace tc {
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
