@@ -268,24 +268,27 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
 // T = (I + A)^-1 is the blocked solve on four warps, as in the forward.  Written out: K^, gamma,
 // T, P, W^T (rows d_k, for the chain) and R^T (bf16).
 namespace prep_tc {
+// Two blocks per SM: regions are reused once their first use is over.
 constexpr uint32_t QE = 0;          // [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
-constexpr uint32_t KT = 32768;      // K~ [a0 | a1]
+constexpr uint32_t KT = 32768;      // K~ [a0 | a1]; after [A; P]: W^T bf16 [128 rows d_k][64 tokens]
+constexpr uint32_t WT = KT;
 constexpr uint32_t DO = 49152;      // dO [a0 | a1]
-constexpr uint32_t TT = 65536;      // T bf16 [64][64]
-constexpr uint32_t PP = 73728;      // P bf16 [64][64]
-constexpr uint32_t WT = 81920;      // W^T bf16 [128 rows d_k][64 tokens]
-constexpr uint32_t SA = 98304;      // A fp32 [64][LDA]
+constexpr uint32_t PP = 65536;      // P bf16 [64][64]; during the folding: decay totals [4][D] fp32
+constexpr uint32_t TOT = PP;
+constexpr uint32_t SA = 73728;      // A fp32 [64][LDA]; after the solve: T bf16 [64][64]
+constexpr uint32_t TT = SA;
 constexpr uint32_t ST = SA + 64 * LDA * 4;   // T fp32 [64][LDA]
-constexpr uint32_t TOT = ST + 64 * LDA * 4;  // decay totals [8][D] fp32
-constexpr uint32_t USED = TOT + 8 * D * 4;
+constexpr uint32_t USED = ST + 64 * LDA * 4;
 constexpr uint32_t SMEM = USED + 1024;       // slack for the 1024-byte alignment
-constexpr uint32_t TM_AP = 0, TM_WT = 64, TM_ZT = 128, TM_ZB = 192, TM_RT = 256, TM_COLS = 512;
+// TMEM: [A; P] then Z^T in 0..63, W^T in 64..127, -Z^T bf16 in 128..159; R^T (issued once
+// Z^T and W^T are read back) in 0..127
+constexpr uint32_t TM_AP = 0, TM_ZT = 0, TM_WT = 64, TM_ZB = 128, TM_RT = 0, TM_COLS = 256;
 constexpr uint32_t IDESC_AP = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 1, 1);
 constexpr uint32_t IDESC_W = tc::idesc_bf16(128, 64, 1, 0);
 constexpr uint32_t IDESC_R1 = tc::idesc_bf16(128, 128, 1, 1);
 constexpr uint32_t IDESC_R2 = tc::idesc_bf16(128, 128, 0, 0);
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 }  // namespace prep_tc
 
 struct PrepMaps {
@@ -297,7 +300,7 @@ __device__ __forceinline__ void named_bar(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__global__ void __launch_bounds__(prep_tc::kThreads, 1)
+__global__ void __launch_bounds__(prep_tc::kThreads, 2)
 bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
 {
     using namespace prep_tc;
@@ -348,21 +351,21 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         for (int at = 0; at < a.din / 32; ++at) tma_prefetch_3d(&maps.g, at * 32, hh, y);
     }
 
-    // ---- decay folding: thread (channel block cb, token group tg of 8, lane): channels
-    //      64 cb + 2 lane (+1), tokens 8 tg .. 8 tg + 7
+    // ---- decay folding: thread (channel block cb, token group tg of 16, lane): channels
+    //      64 cb + 2 lane (+1), tokens 16 tg .. 16 tg + 15
     const int cb = warp & 1, tg = warp >> 1, ch = 64 * cb + 2 * lane;
     {
-        float2 gv[8];
+        float2 gv[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * tg + i;
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * tg + i;
             gv[i] = (t < L && ch < a.din)
                         ? __ldg(reinterpret_cast<const float2 *>(a.g + tok_off(a, bos, hh, ci, t) + ch))
                         : make_float2(0.f, 0.f);
         }
         float run0 = 0.f, run1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
             run0 += gv[i].x;
             run1 += gv[i].y;
             gv[i] = make_float2(__expf(gv[i].x), __expf(gv[i].y));  // alpha
@@ -372,7 +375,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         __syncthreads();
         float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 4; ++u) {
             const float2 v = *reinterpret_cast<const float2 *>(sTot + u * D + ch);
             if (u < tg) { off0 += v.x; off1 += v.y; }
             tot0 += v.x;
@@ -380,11 +383,11 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         }
         const float gam0 = __expf(tot0), gam1 = __expf(tot1);
         if (tg == 0) *reinterpret_cast<float2 *>(a.gam + cidx * D + ch) = make_float2(gam0, gam1);
-        float2 mv[8];  // e^-G, backwards from the group's last token
+        float2 mv[16];  // e^-G, backwards from the group's last token
         {
             float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
 #pragma unroll
-            for (int i = 7; i >= 0; --i) {
+            for (int i = 15; i >= 0; --i) {
                 mv[i] = make_float2(r0, r1);
                 r0 *= gv[i].x;
                 r1 *= gv[i].y;
@@ -394,8 +397,8 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         uint8_t *pe = sm + QE + cb * 16384, *pq = pe + 8192, *pk = sm + KT + cb * 8192;
         __nv_bfloat16 *kh = a.Kh + cidx * C * D;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * tg + i;
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * tg + i;
             e0 *= gv[i].x;
             e1 *= gv[i].y;
             const uint32_t off = sw128(t, 4 * lane);
@@ -468,8 +471,8 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     __syncthreads();
     // ---- T -> bf16 tile and global (threads 0-255), P -> global (threads 256-511): 16 columns each
     {
-        const int u = tid & 255, i = u >> 2, jq = u & 3;
-        if (tid < 256) {
+        const int i = tid >> 2, jq = tid & 3;
+        {
             uint32_t w8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -482,12 +485,11 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
                 *reinterpret_cast<uint4 *>(sm + TT + sw128(i, 32 * jq + 16 * h2)) = v;
                 *reinterpret_cast<uint4 *>(a.Tm + cidx * C * C + i * C + 16 * jq + 8 * h2) = v;
             }
-        } else {
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2)
-                *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 16 * jq + 8 * h2) =
-                    *reinterpret_cast<const uint4 *>(sm + PP + sw128(i, 32 * jq + 16 * h2));
         }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+            *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 16 * jq + 8 * h2) =
+                *reinterpret_cast<const uint4 *>(sm + PP + sw128(i, 32 * jq + 16 * h2));
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -556,8 +558,9 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     }
     if (!mbar_wait(&bar_r, 0)) atomicExch(a.status, kStatusTimeout);
     tc_fence_after();
-    {  // R^T -> bf16, global [d_v][d_k]: warp = lane quarter x 32-column block
-        const int quarter = warp & 3, cq = warp >> 2, j = quarter * 32 + lane;
+#pragma unroll
+    for (int cq2 = 0; cq2 < 2; ++cq2) {  // R^T -> bf16, global [d_v][d_k]: warp = lane quarter x 2 column blocks
+        const int quarter = warp & 3, cq = 2 * (warp >> 2) + cq2, j = quarter * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t r[32];
         tmem_ld32(tmem + TM_RT + 32 * cq + lane_off, r);
