@@ -147,64 +147,12 @@ __device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
     return chunk_ref_at(a, blockIdx.x, blockIdx.y, r);
 }
 
-// cp.async versions: the copies stay in flight until cp_async_wait; rows past the
-// sequence end are zero-filled (source size 0).
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, bool valid)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_tok_tile(uint32_t dst, const __nv_bfloat16 *src, const BwdTcArgs &a, int bb,
-                                            int hh, int ci, int L, int tid, int nthreads)
-{
-    for (int idx = tid; idx < C * 16; idx += nthreads) {
-        const int t = idx >> 4, ch = idx & 15;
-        const bool ok = t < L && 8 * ch < a.din;  // channels past the head size read zeros
-        cp_async16_zfill(dst + swz(t, 8 * ch, 256), src + (ok ? tok_off(a, bb, hh, ci, t) + 8 * ch : 0), ok);
-    }
-}
-__device__ __forceinline__ void cp_dense_tile(uint32_t dst, const __nv_bfloat16 *src, int rows, int cols, int tid,
-                                              int nthreads)
-{
-    const int cpr = cols / 8, rb = cols * 2;
-    for (int idx = tid; idx < rows * cpr; idx += nthreads) {
-        const int r = idx / cpr, ch = idx % cpr;
-        cp_async16(dst + swz(r, 8 * ch, rb), src + (size_t)r * cols + 8 * ch);
-    }
-}
-
-// store a bf16 pair at (row, col) of a swizzled tile
-__device__ __forceinline__ void st_pair(uint8_t *tile, int rb, int row, int col, float lo, float hi)
-{
-    *reinterpret_cast<uint32_t *>(tile + swz(row, col, rb)) = pack_bf16x2(lo, hi);
-}
-__device__ __forceinline__ uint32_t ld_pair(const uint8_t *tile, int rb, int row, int col)
-{
-    return *reinterpret_cast<const uint32_t *>(tile + swz(row, col, rb));
-}
-
-// Two-channel layout of the prep and gradient kernels' elementwise work: thread (channel pair cp,
-// token group g8) owns channels 2 cp, 2 cp + 1 and tokens 8 g8 .. 8 g8 + 7 (64 x 8 = 512
-// threads).  log alpha of those 16 values, zero past the sequence end and the head size.
-__device__ __forceinline__ void load_g8(float2 (&g)[8], const BwdTcArgs &a, int bb, int hh, int ci, int L, int cp,
-                                        int g8)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = 8 * g8 + i;
-        g[i] = (t < L && 2 * cp < a.din)
-                   ? __ldg(reinterpret_cast<const float2 *>(a.g + tok_off(a, bb, hh, ci, t) + 2 * cp))
-                   : make_float2(0.f, 0.f);
-    }
-}
-
-// e^G and e^-G of this thread's 16 values (G the inclusive cumulative sum of log alpha over
-// the chunk) with one exponential per value: alpha = e^g, then e^G as a running product
-// forwards from the token group's start and e^-G as one backwards from its end.  The group
-// totals go through sTot ([8][D] fp32); `total` is G at the chunk end.  Contains a
-// __syncthreads; kWait: this thread's cp.async copies, except the newest kKeep groups,
-// are waited for before it.
-template <bool kWait, int kKeep = 0>
+// Decay folding of the gradient kernel: thread (channel pair cp, token group g8) owns channels
+// 2 cp, 2 cp + 1 and tokens 8 g8 .. 8 g8 + 7 (64 x 8 = 512 threads).  e^G and e^-G of its 16
+// values (G the inclusive cumulative sum of log alpha over the chunk) with one exponential per
+// value: alpha = e^g, then e^G as a running product forwards from the token group's start and
+// e^-G as one backwards from its end.  The group totals go through sTot ([8][D] fp32); `total`
+// is G at the chunk end.  Contains a __syncthreads.
 __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8], float2 (&emG)[8], float2 &total,
                                             int cp, int g8, float *sTot)
 {
@@ -216,7 +164,6 @@ __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8
         eG[i] = make_float2(__expf(g[i].x), __expf(g[i].y));  // alpha for now
     }
     *reinterpret_cast<float2 *>(sTot + g8 * D + 2 * cp) = make_float2(run0, run1);
-    if (kWait) cp_async_wait<kKeep>();
     __syncthreads();
     float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
@@ -241,14 +188,6 @@ __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8
         eG[i] = make_float2(e0, e1);
     }
     total = make_float2(tot0, tot1);
-}
-
-// bf16x2 product, rounded to nearest even (exact before the rounding for bf16 inputs)
-__device__ __forceinline__ uint32_t bmul2(uint32_t x, uint32_t y)
-{
-    uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
-    return r;
 }
 
 // L2 prefetch (bulk, no shared-memory destination)
@@ -715,118 +654,141 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
         }
 }
 
-// ================================================================== 4. gradients
-// smem map (bytes): [C][D] bf16 tiles Q~, E~, K~; S^T and (Diag(gamma) dS_n)^T [D][D] bf16;
-// X -> U~, w -> Y -> dU~ -> [dP | dA], dO, -dY; T, P [C][C] bf16; scratch.  After the
-// products, dQ~, dE~, dK~ (fp32 [C][LDF]) reuse the first 104 KB.
-constexpr uint32_t G_Q = 0, G_E = 16384, G_K = 32768, G_S = 49152, G_DS = 81920, G_X = 114688, G_Y = 131072;
-constexpr uint32_t G_DO = 147456, G_DY = 163840, G_TB = 180224, G_PB = 188416, G_TOT = 196608;
-constexpr uint32_t G_GAM = G_TOT + 8 * D * 4, G_DGP = G_GAM + D * 4, G_DGF = G_DGP + 16 * D * 4;
-constexpr uint32_t G_SMEM = G_DGF + D * 4;
-constexpr int LDF = 136;  // fp32 row stride of the dQ~ / dE~ / dK~ tiles
-constexpr uint32_t G_FQ = 0, G_FE = C * LDF * 4, G_FK = 2 * C * LDF * 4;
-static_assert(G_FK + C * LDF * 4 <= G_X, "fp32 gradient tiles must fit in the dead operand tiles");
-constexpr int kGradThreads = 512;
+// ================================================================== 4. gradients on the tensor cores
+// One 512-thread CTA per (chunk, head).  Every product runs transposed, so that its M side is a
+// 128-wide feature dimension (d_v or d_k, or the two stacked 64-token tiles of [dP; dA]) and its
+// TMEM accumulator holds one feature row per lane (Gm = Diag(gamma)):
+//   Y^T  = X^T - S^T E~^T              M d_v, N 64, K d_k           -> bf16 A operand in TMEM
+//   dU~^T = dO^T P + (Gm dS_n)^T K~^T  M d_v, N 64, K 64 + d_k      -> bf16 A operand in TMEM
+//   U~^T = Y^T T^T                     A from TMEM, K 64            -> U~ tile [s][d_v]
+//   dY^T = dU~^T T                     A from TMEM, K 64            -> dv, dw, -dY tile
+//   [dP; dA] = [dO; -dY] U~^T          M 2 x 64 tokens, N 64, K d_v -> masked bf16 tile
+//   [dQ~^T | dE~^T] = S [dO; -dY]^T + K~^T [dP; dA]^T     M d_k, N 128, K d_v + 64
+//   dK~^T = (Gm dS_n) U~^T + Q~^T dP + E~^T dA            M d_k, N 64, K d_v + 128
+// The tiles arrive by TMA in 128-byte swizzled atoms; a [rows][128] tile is two column atoms
+// of [rows][64].  The factor chain reads dQ~^T, dE~^T, dK~^T straight from TMEM: a thread
+// owns one channel of d_k (its TMEM lane) and 16 tokens (its column block).
+namespace grad_tc {
+constexpr uint32_t RQ = 0;        // q -> Q~ [64][128]
+constexpr uint32_t RK = 16384;    // k -> K~
+constexpr uint32_t RB = 32768;    // b -> E~
+constexpr uint32_t GG = 49152;    // log alpha fp32 [64][128]: four 8 KiB boxes of 32 channels
+constexpr uint32_t SS = 81920;    // S^T [128][128] (atoms 16 KiB apart); after the S products: raw q, k
+constexpr uint32_t DS = 114688;   // dS_n^T -> (Gm dS_n)^T; after its products: raw b
+constexpr uint32_t DY = 147456;   // [dO; -dY] [128][128]: atom a = dO rows 0-63 then -dY rows 64-127
+constexpr uint32_t TT = 180224;   // T [64][64]; after dY: U~ [64][128] over T and P
+constexpr uint32_t PP = 188416;   // P [64][64]
+constexpr uint32_t UU = TT;
+constexpr uint32_t VV = 196608;   // v; after dv and dw: [dP; dA] [128][64]
+constexpr uint32_t PA = VV;
+constexpr uint32_t WW = 212992;   // w
+constexpr uint32_t DGF = 229376;  // gamma dgamma [D] fp32
+constexpr uint32_t USED = DGF + D * 4;
+constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
+// scratch inside the -dY rows (free until dY is read back), and inside DY once every product
+// is done (the factor chain)
+constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
+constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
+constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
+constexpr uint32_t SC_FIN = DY;                  // factor chain: group sums [4][D], twice
+// TMEM columns
+constexpr uint32_t TM_Y = 0, TM_DU = 64, TM_YB = 128, TM_DUB = 160, TM_U = 192, TM_DY = 256, TM_PA = 320;
+constexpr uint32_t TM_DQE = 384, TM_DK = 0, TM_COLS = 512;
+constexpr uint32_t IDESC_KK = tc::idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t IDESC_MM = tc::idesc_bf16(128, 64, 1, 1);
+constexpr uint32_t IDESC_KM = tc::idesc_bf16(128, 64, 0, 1);
+constexpr uint32_t IDESC_MK = tc::idesc_bf16(128, 64, 1, 0);
+constexpr uint32_t IDESC_MK2 = tc::idesc_bf16(128, 128, 1, 0);
+constexpr int kThreads = 512;
+}  // namespace grad_tc
 
-__global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcArgs a)
+struct GradMaps {
+    CUtensorMap q, k, b, v, w, dO, g, st, dsn, tm, pm;
+};
+
+__device__ __forceinline__ void wait_or_flag(uint64_t *bar, uint32_t parity, int *status)
 {
-    extern __shared__ __align__(1024) uint8_t sm[];
+    if (!tc::mbar_wait(bar, parity)) atomicExch(status, kStatusTimeout);
+}
+
+// bf16 element (t, c) of a [rows][128] tile whose two column atoms are `astride` bytes apart
+__device__ __forceinline__ uint32_t tile_off(int t, int c, uint32_t astride)
+{
+    return (uint32_t)(c >> 6) * astride + tc::sw128(t, (c & 63) * 2);
+}
+__device__ __forceinline__ float ld_bf(const uint8_t *p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p)); }
+__device__ __forceinline__ void st_bf(uint8_t *p, float x) { *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x); }
+
+__global__ void __launch_bounds__(grad_tc::kThreads, 1)
+bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
+{
+    using namespace grad_tc;
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_in0, bar_in1, bar_in2, bar_a, bar_b, bar_c, bar_d;
+    __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t4 = lane & 3;
     ChunkRef cr;
-    if (!chunk_ref(a, cr)) return;
+    if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
     const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
     const int L = min(C, cr.sp.len - ci * C);
     const size_t cidx = cr.cidx;
     const uint32_t sb = smem_u32(sm);
-    float *sTot = reinterpret_cast<float *>(sm + G_TOT);
-    float *sGam = reinterpret_cast<float *>(sm + G_GAM);
-    float *sDgp = reinterpret_cast<float *>(sm + G_DGP);
-    float *sDgf = reinterpret_cast<float *>(sm + G_DGF);
-    const int cp = tid & 63, g8 = tid >> 6;  // elementwise mapping: channel pair, group of 8 tokens
-    const __nv_bfloat16 *st_c = a.states + bound_slot(a.pr, cr.n, hh, cr.nch, ci) * D * D;
-    // dS_n and the chunk-end state, for (Diag(gamma) dS_n)^T and gamma dgamma: loaded first, so
-    // that their latency hides behind the operand copies and the decay folding
-    const int dch = tid & 15;
-    uint4 dsv[4], ssv[4];
-    {
-        const __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
-        const __nv_bfloat16 *st_n = st_c + (size_t)D * D;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = (tid >> 4) + 32 * u;
-            dsv[u] = __ldg(reinterpret_cast<const uint4 *>(dsn + (size_t)j * D + 8 * dch));
-            ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)j * D + 8 * dch));
-        }
-    }
+    const size_t slot = bound_slot(a.pr, cr.n, hh, cr.nch, ci);
+    // TMEM access: warp w reads lanes 32 (w & 3) .. + 31; column block w >> 2 (16 columns)
+    const int quarter = warp & 3, cg = warp >> 2, row = 32 * quarter + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
 
-    // ---- P0: operands
-    cp_tok_tile(sb + G_Q, a.q, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_K, a.k, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_E, a.b, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_X, a.v, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_Y, a.w, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_DO, a.dO, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_dense_tile(sb + G_S, st_c, D, D, tid, kGradThreads);
-    cp_dense_tile(sb + G_TB, a.Tm + cidx * C * C, C, C, tid, kGradThreads);
-    cp_dense_tile(sb + G_PB, a.Pm + cidx * C * C, C, C, tid, kGradThreads);
-    cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&bar_in0, 1);
+        mbar_init(&bar_in1, 1);
+        mbar_init(&bar_in2, 1);
+        mbar_init(&bar_a, 1);
+        mbar_init(&bar_b, 1);
+        mbar_init(&bar_c, 1);
+        mbar_init(&bar_d, 1);
+        fence_mbar_init();
+        const CUtensorMap *all[11] = {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w, &maps.dO,
+                                      &maps.g, &maps.st, &maps.dsn, &maps.tm, &maps.pm};
+        for (int i = 0; i < 11; ++i) prefetch_tmap(all[i]);
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const int y = bb + ci * C;
+    if (tid == 0) {
+        mbar_expect_tx(&bar_in0, 10 * 8192);
+        for (int at = 0; at < 2; ++at) {
+            tma_load_3d(sm + RQ + at * 8192, &maps.q, at * 64, hh, y, &bar_in0);
+            tma_load_3d(sm + RK + at * 8192, &maps.k, at * 64, hh, y, &bar_in0);
+            tma_load_3d(sm + RB + at * 8192, &maps.b, at * 64, hh, y, &bar_in0);
+        }
+        for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + GG + bx * 8192, &maps.g, bx * 32, hh, y, &bar_in0);
+        mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
+        for (int at = 0; at < 2; ++at) {
+            tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, (int)(slot * D), &bar_in1);
+            tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(cidx * D), &bar_in1);
+            tma_load_3d(sm + DY + at * 16384, &maps.dO, at * 64, hh, y, &bar_in1);
+            tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, hh, y, &bar_in1);
+            tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, hh, y, &bar_in1);
+        }
+        tma_load_2d(sm + TT, &maps.tm, 0, (int)(cidx * C), &bar_in1);
+        tma_load_2d(sm + PP, &maps.pm, 0, (int)(cidx * C), &bar_in1);
+    }
+    // the chunk-end state (for gamma dgamma), in flight during the folding
+    const int dch = tid & 15;
+    uint4 ssv[4];
     {
-        float2 gl[8], eG[8], emG[8], tot;
-        load_g8(gl, a, bb, hh, ci, L, cp, g8);
-        decay_pair8<true>(gl, eG, emG, tot, cp, g8, sTot);  // its barrier also publishes the tiles
-        if (g8 == 0) *reinterpret_cast<float2 *>(sGam + 2 * cp) = make_float2(__expf(tot.x), __expf(tot.y));
+        const __nv_bfloat16 *st_n = a.states + (slot + 1) * D * D;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * g8 + i;
-            const uint32_t off = swz(t, 2 * cp, 256);
-            uint32_t *pq = reinterpret_cast<uint32_t *>(sm + G_Q + off);
-            uint32_t *pk = reinterpret_cast<uint32_t *>(sm + G_K + off);
-            uint32_t *pe = reinterpret_cast<uint32_t *>(sm + G_E + off);
-            uint32_t *px = reinterpret_cast<uint32_t *>(sm + G_X + off);
-            const uint32_t q2 = *pq, k2 = *pk, b2 = *pe, x2 = *px, w2 = *reinterpret_cast<const uint32_t *>(sm + G_Y + off);
-            const float k0 = bf_lo(k2), k1 = bf_hi(k2);
-            *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
-            *pe = pack_bf16x2(bf_lo(b2) * k0 * eG[i].x, bf_hi(b2) * k1 * eG[i].y);
-            *pk = pack_bf16x2(k0 * emG[i].x, k1 * emG[i].y);
-            *px = bmul2(x2, w2);  // X = w.v (columns = j)
-        }
-    }
-    __syncthreads();
-    {  // (Diag(gamma) dS_n)^T tile, and gamma dgamma = rowsum(dS_n . S') partials
-        const int ch = dch;
-        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float gm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gm[e] = sGam[8 * ch + e];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = (tid >> 4) + 32 * u;
-            const uint4 dv4 = dsv[u], sv4 = ssv[u];
-            const uint32_t dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w}, sw[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float d0 = bf_lo(dw[e]), d1 = bf_hi(dw[e]);
-                part[2 * e] += d0 * bf_lo(sw[e]);
-                part[2 * e + 1] += d1 * bf_hi(sw[e]);
-                o[e] = pack_bf16x2(d0 * gm[2 * e], d1 * gm[2 * e + 1]);
-            }
-            *reinterpret_cast<uint4 *>(sm + G_DS + swz(j, 8 * ch, 256)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) part[e] += __shfl_xor_sync(0xffffffffu, part[e], 16);
-        if (lane < 16) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sDgp[warp * D + 8 * ch + e] = part[e];
-        }
-    }
-    __syncthreads();
-    if (tid < D) {
-        float s = 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
-        sDgf[tid] = s;
+        for (int u = 0; u < 4; ++u)
+            ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
     }
     {  // everything the block one wave later reads, into L2 (one bulk prefetch per thread)
         const int nblk = gridDim.x * gridDim.y, nxt = blockIdx.y * gridDim.x + blockIdx.x + a.n_sm;
@@ -854,198 +816,323 @@ __global__ void __launch_bounds__(kGradThreads, 1) bwd_grad_kernel(const BwdTcAr
             }
         }
     }
-    // warp tiling of the [C][D] products: 16 rows x 32 columns
-    const int mt = warp & 3, nq = warp >> 2;
-    const int r0 = 16 * mt + g, c0 = 32 * nq + 2 * t4;  // + 8 hr rows, + 8 nt columns
-    // ---- P1: Y = X - E~ S  -> bf16 over the raw w tile
+
+    // ---- decay folding in place: thread (channel pair cp, token group g8 of 8)
+    const int cp = tid & 63, g8 = tid >> 6;
+    float *sTot = reinterpret_cast<float *>(sm + SC_TOT);
+    float *sGam = reinterpret_cast<float *>(sm + SC_GAM);
+    wait_or_flag(&bar_in0, 0, a.status);
     {
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, false, false, D>(acc, sb + G_E, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
-                const uint32_t x = ld_pair(sm + G_X, 256, row, col);
-                st_pair(sm + G_Y, 256, row, col, bf_lo(x) - acc[0][nt][2 * hr], bf_hi(x) - acc[0][nt][2 * hr + 1]);
-            }
-    }
-    __syncthreads();
-    // ---- P2: U~ = T Y  -> bf16 over X
-    {
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, false, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-                st_pair(sm + G_X, 256, r0 + 8 * hr, c0 + 8 * nt, acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
-    }
-    __syncthreads();
-    // ---- P3: dU~ = P^T dO + K~ (Diag(gamma) dS_n)  -> bf16 over Y
-    {
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, true, true, C>(acc, sb + G_PB, 128, 16 * mt, sb + G_DO, 256, 32 * nq, lane);
-        warp_gemm<1, 4, false, false, D>(acc, sb + G_K, 256, 16 * mt, sb + G_DS, 256, 32 * nq, lane);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-                st_pair(sm + G_Y, 256, r0 + 8 * hr, c0 + 8 * nt, acc[0][nt][2 * hr], acc[0][nt][2 * hr + 1]);
-    }
-    __syncthreads();
-    // ---- P4: dY = T^T dU~ -> dv = dY w, dw = dY v (global), -dY (bf16)
-    {
-        uint32_t vv[4][2], ww[4][2];  // all loads first, in flight during the product
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
-                vv[nt][hr] = ww[nt][hr] = 0u;
-                if (row < L && col < a.din) {
-                    const size_t off = tok_off(a, bb, hh, ci, row) + col;
-                    vv[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.v + off));
-                    ww[nt][hr] = __ldg(reinterpret_cast<const unsigned int *>(a.w + off));
-                }
-            }
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, true, true, C>(acc, sb + G_TB, 128, 16 * mt, sb + G_Y, 256, 32 * nq, lane);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = r0 + 8 * hr, col = c0 + 8 * nt;
-                const float d0 = acc[0][nt][2 * hr], d1 = acc[0][nt][2 * hr + 1];
-                st_pair(sm + G_DY, 256, row, col, -d0, -d1);
-                if (row < L && col < a.din) {
-                    const size_t off = tok_off(a, bb, hh, ci, row) + col;
-                    const uint32_t v2 = vv[nt][hr], w2 = ww[nt][hr];
-                    *reinterpret_cast<uint32_t *>(a.dv + off) = pack_bf16x2(d0 * bf_lo(w2), d1 * bf_hi(w2));
-                    *reinterpret_cast<uint32_t *>(a.dw + off) = pack_bf16x2(d0 * bf_lo(v2), d1 * bf_hi(v2));
-                }
-            }
-    }
-    __syncthreads();
-    // ---- P5: [dP; dA] = [dO; -dY] U~^T (128 x 64, K = 128) -> bf16 [C][C] tiles over dU~
-    {
-        const int ms = warp & 7, nh = warp >> 3;
-        float acc[1][4][4];
-        zero_acc(acc);
-        warp_gemm<1, 4, false, false, D>(acc, sb + (ms < 4 ? G_DO : G_DY), 256, 16 * (ms & 3), sb + G_X, 256, 32 * nh,
-                                         lane);
-        uint8_t *dst = sm + G_Y + (ms < 4 ? 0 : 8192);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int row = 16 * (ms & 3) + g + 8 * hr, col = 32 * nh + 8 * nt + 2 * t4;
-                const float v0 = acc[0][nt][2 * hr], v1 = acc[0][nt][2 * hr + 1];
-                if (ms < 4)
-                    st_pair(dst, 128, row, col, (col <= row) ? v0 : 0.f, (col + 1 <= row) ? v1 : 0.f);
-                else
-                    st_pair(dst, 128, row, col, (col < row) ? v0 : 0.f, (col + 1 < row) ? v1 : 0.f);
-            }
-    }
-    __syncthreads();
-    const uint32_t dPb = sb + G_Y, dAb = sb + G_Y + 8192;
-    // ---- P6-P8: dQ~, dE~, dK~ in registers
-    float aq[1][4][4], ae[1][4][4], ak[1][4][4];
-    zero_acc(aq);
-    zero_acc(ae);
-    zero_acc(ak);
-    warp_gemm<1, 4, false, true, D>(aq, sb + G_DO, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
-    warp_gemm<1, 4, false, true, C>(aq, dPb, 128, 16 * mt, sb + G_K, 256, 32 * nq, lane);
-    warp_gemm<1, 4, false, true, D>(ae, sb + G_DY, 256, 16 * mt, sb + G_S, 256, 32 * nq, lane);
-    warp_gemm<1, 4, false, true, C>(ae, dAb, 128, 16 * mt, sb + G_K, 256, 32 * nq, lane);
-    warp_gemm<1, 4, true, true, C>(ak, dAb, 128, 16 * mt, sb + G_E, 256, 32 * nq, lane);
-    warp_gemm<1, 4, true, true, C>(ak, dPb, 128, 16 * mt, sb + G_Q, 256, 32 * nq, lane);
-    warp_gemm<1, 4, false, true, D>(ak, sb + G_X, 256, 16 * mt, sb + G_DS, 256, 32 * nq, lane);
-    __syncthreads();  // all operand tiles are dead from here on
-    // raw q, k, b for the factor chain, into tiles that the fp32 gradients do not cover
-    cp_tok_tile(sb + G_X, a.q, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_Y, a.k, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_tok_tile(sb + G_DO, a.b, a, bb, hh, ci, L, tid, kGradThreads);
-    cp_async_commit();
-    {
-        float *fq = reinterpret_cast<float *>(sm + G_FQ), *fe = reinterpret_cast<float *>(sm + G_FE);
-        float *fk = reinterpret_cast<float *>(sm + G_FK);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int o = (r0 + 8 * hr) * LDF + c0 + 8 * nt;
-                *reinterpret_cast<float2 *>(fq + o) = make_float2(aq[0][nt][2 * hr], aq[0][nt][2 * hr + 1]);
-                *reinterpret_cast<float2 *>(fe + o) = make_float2(ae[0][nt][2 * hr], ae[0][nt][2 * hr + 1]);
-                *reinterpret_cast<float2 *>(fk + o) = make_float2(ak[0][nt][2 * hr], ak[0][nt][2 * hr + 1]);
-            }
-    }
-    __syncthreads();
-    // ---- P10: through the factors (thread: channels 2 cp, 2 cp + 1, tokens 8 g8 .. +7), fp32
-    {
-        const float *fq = reinterpret_cast<const float *>(sm + G_FQ), *fe = reinterpret_cast<const float *>(sm + G_FE);
-        const float *fk = reinterpret_cast<const float *>(sm + G_FK);
-        float2 gl[8], eG[8], emG[8], tot;
-        load_g8(gl, a, bb, hh, ci, L, cp, g8);
-        decay_pair8<true>(gl, eG, emG, tot, cp, g8, sTot);  // sTot is free again (P0 finished)
         const bool ch_ok = 2 * cp < a.din;
-        const size_t base = tok_off(a, bb, hh, ci, 8 * g8) + 2 * cp, stride = (size_t)a.H * a.din;
-        float2 dG[8];
+        float2 gl[8], eG[8], emG[8], tot;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int t = 8 * g8 + i;
-            const float2 dQ = *reinterpret_cast<const float2 *>(fq + t * LDF + 2 * cp);
-            const float2 dE = *reinterpret_cast<const float2 *>(fe + t * LDF + 2 * cp);
-            const float2 dK = *reinterpret_cast<const float2 *>(fk + t * LDF + 2 * cp);
-            const uint32_t off_s = swz(t, 2 * cp, 256);
-            const uint32_t q2 = *reinterpret_cast<const uint32_t *>(sm + G_X + off_s);
-            const uint32_t k2 = *reinterpret_cast<const uint32_t *>(sm + G_Y + off_s);
-            const uint32_t b2 = *reinterpret_cast<const uint32_t *>(sm + G_DO + off_s);
-            const float q0 = bf_lo(q2), q1 = bf_hi(q2), k0 = bf_lo(k2), k1 = bf_hi(k2), b0 = bf_lo(b2), b1 = bf_hi(b2);
-            const float de0 = dE.x * eG[i].x, de1 = dE.y * eG[i].y;
-            dG[i].x = dQ.x * q0 * eG[i].x + de0 * b0 * k0 - dK.x * k0 * emG[i].x;
-            dG[i].y = dQ.y * q1 * eG[i].y + de1 * b1 * k1 - dK.y * k1 * emG[i].y;
+            gl[i] = (t < L && ch_ok)
+                        ? *reinterpret_cast<const float2 *>(sm + GG + (cp >> 4) * 8192 + sw128(t, (cp & 15) * 8))
+                        : make_float2(0.f, 0.f);
+        }
+        decay_pair8(gl, eG, emG, tot, cp, g8, sTot);
+        if (g8 == 0) *reinterpret_cast<float2 *>(sGam + 2 * cp) = make_float2(__expf(tot.x), __expf(tot.y));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * g8 + i;
+            const uint32_t off = (cp >> 5) * 8192 + sw128(t, (cp & 31) * 4);
+            uint32_t *pq = reinterpret_cast<uint32_t *>(sm + RQ + off);
+            uint32_t *pk = reinterpret_cast<uint32_t *>(sm + RK + off);
+            uint32_t *pe = reinterpret_cast<uint32_t *>(sm + RB + off);
+            uint32_t q2 = *pq, k2 = *pk, b2 = *pe;
+            if (t >= L) { q2 = 0u; k2 = 0u; b2 = 0u; }
+            const float k0 = bf_lo(k2), k1 = bf_hi(k2);
+            *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
+            *pe = pack_bf16x2(bf_lo(b2) * k0 * eG[i].x, bf_hi(b2) * k1 * eG[i].y);
+            *pk = pack_bf16x2(k0 * emG[i].x, k1 * emG[i].y);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    // ---- Y^T = S^T E~^T (into TM_Y; X is added at the read-back)
+    wait_or_flag(&bar_in1, 0, a.status);
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_Y, sdesc_sw128(sb + SS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sb + RB + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_KK, ks > 0);
+    }
+    // ---- dS_n^T -> (Gm dS_n)^T in place, gamma dgamma = column sums of dS_n^T . S_end^T
+    {
+        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float gm[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[e] = sGam[8 * dch + e];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = (tid >> 4) + 32 * u;
+            uint4 *p = reinterpret_cast<uint4 *>(sm + DS + (dch >> 3) * 16384 + sw128(j, (dch & 7) * 16));
+            const uint4 dv4 = *p, sv4 = ssv[u];
+            const uint32_t dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w}, sw[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float d0 = bf_lo(dw[e]), d1 = bf_hi(dw[e]);
+                part[2 * e] += d0 * bf_lo(sw[e]);
+                part[2 * e + 1] += d1 * bf_hi(sw[e]);
+                o[e] = pack_bf16x2(d0 * gm[2 * e], d1 * gm[2 * e + 1]);
+            }
+            *p = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[e] += __shfl_xor_sync(0xffffffffu, part[e], 16);
+        float *sDgp = reinterpret_cast<float *>(sm + SC_DGP);
+        if (lane < 16) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sDgp[warp * D + 8 * dch + e] = part[e];
+        }
+        if (L < C) {  // dO rows past the sequence end belong to the next one: zero them
+            for (int idx = tid; idx < (C - L) * 16; idx += kThreads) {
+                const int t = L + (idx >> 4), c = idx & 15;
+                *reinterpret_cast<uint4 *>(sm + DY + (c >> 3) * 16384 + sw128(t, (c & 7) * 16)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < D) {
+        const float *sDgp = reinterpret_cast<const float *>(sm + SC_DGP);
+        float s = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
+        reinterpret_cast<float *>(sm + DGF)[tid] = s;
+    }
+    // ---- dU~^T = dO^T P + (Gm dS_n)^T K~^T
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_DU, sdesc_sw128(sb + DY + ks * 2048, 16384, 1024), sdesc_sw128(sb + PP + ks * 2048, 8192, 1024),
+                   IDESC_MM, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_DU, sdesc_sw128(sb + DS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sb + RK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_KK, 1);
+        mma_commit(&bar_a);
+    }
+    // ---- read back: Y^T = X^T - acc and dU~^T, as bf16 A operands (lane = d_v, 16 tokens per warp)
+    wait_or_flag(&bar_a, 0, a.status);
+    tc_fence_after();
+    {
+        uint32_t r[16], pk[8];
+        tmem_ld16(tmem + TM_Y + 16 * cg + lane_off, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float y2[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int t = 16 * cg + 2 * e + h;
+                const uint32_t so = tile_off(t, row, 8192);
+                const float x = (t < L) ? ld_bf(sm + VV + so) * ld_bf(sm + WW + so) : 0.f;
+                y2[h] = x - __uint_as_float(r[2 * e + h]);
+            }
+            pk[e] = pack_bf16x2(y2[0], y2[1]);
+        }
+        tmem_st8(tmem + TM_YB + 8 * cg + lane_off, pk);
+        tmem_ld16(tmem + TM_DU + 16 * cg + lane_off, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+        tmem_st8(tmem + TM_DUB + 8 * cg + lane_off, pk);
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- U~^T = Y^T T^T, dY^T = dU~^T T
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tmem + TM_U, tmem + TM_YB + 8 * ks, sdesc_sw128(sb + TT + ks * 32, 16, 1024), IDESC_KK, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tmem + TM_DY, tmem + TM_DUB + 8 * ks, sdesc_sw128(sb + TT + ks * 2048, 8192, 1024), IDESC_KM, ks > 0);
+        mma_commit(&bar_b);
+    }
+    wait_or_flag(&bar_b, 0, a.status);
+    tc_fence_after();
+    // ---- read back: U~ tile [s][d_v] (over T and P, both consumed); dv = dY w, dw = dY v;
+    //      -dY into rows 64-127 of [dO; -dY]
+    {
+        uint32_t r[16];
+        tmem_ld16(tmem + TM_U + 16 * cg + lane_off, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_bf(sm + UU + tile_off(16 * cg + i, row, 8192), __uint_as_float(r[i]));
+        tmem_ld16(tmem + TM_DY + 16 * cg + lane_off, r);
+        tmem_wait_ld();
+        const bool ch_ok = row < a.din;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * cg + i;
+            const float d = __uint_as_float(r[i]);
+            st_bf(sm + DY + tile_off(64 + t, row, 16384), -d);
             if (t < L && ch_ok) {
-                const size_t off = base + (size_t)i * stride;
-                *reinterpret_cast<uint32_t *>(a.dq + off) = pack_bf16x2(dQ.x * eG[i].x, dQ.y * eG[i].y);
-                *reinterpret_cast<uint32_t *>(a.db + off) = pack_bf16x2(de0 * k0, de1 * k1);
-                *reinterpret_cast<uint32_t *>(a.dk + off) =
-                    pack_bf16x2(de0 * b0 + dK.x * emG[i].x, de1 * b1 + dK.y * emG[i].y);
+                const uint32_t so = tile_off(t, row, 8192);
+                const size_t go = tok_off(a, bb, hh, ci, t) + row;
+                a.dv[go] = __float2bfloat16_rn(d * ld_bf(sm + WW + so));
+                a.dw[go] = __float2bfloat16_rn(d * ld_bf(sm + VV + so));
             }
         }
-        if (g8 == 7) {  // gamma dgamma enters at the last row of the chunk
-            dG[7].x += sDgf[2 * cp];
-            dG[7].y += sDgf[2 * cp + 1];
-        }
-        // reverse cumulative sum inside the chunk
-        float run0 = 0.f, run1 = 0.f;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- [dP; dA] = [dO; -dY] U~^T;  [dQ~^T | dE~^T] = S [dO; -dY]^T;  dK~^T = (Gm dS_n) U~^T
+    if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
-        for (int i = 7; i >= 0; --i) {
-            run0 += dG[i].x;
-            run1 += dG[i].y;
-            dG[i] = make_float2(run0, run1);
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_PA, sdesc_sw128(sb + DY + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sb + UU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_KK, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_DQE, sdesc_sw128(sb + SS + ks * 2048, 16384, 1024),
+                   sdesc_sw128(sb + DY + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), IDESC_MK2, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_ss(tmem + TM_DK, sdesc_sw128(sb + DS + ks * 2048, 16384, 1024),
+                   sdesc_sw128(sb + UU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_MK, ks > 0);
+        mma_commit(&bar_c);
+    }
+    wait_or_flag(&bar_c, 0, a.status);
+    tc_fence_after();
+    if (tid == 0) {  // S^T and (Gm dS_n)^T are consumed: the raw q, k, b for the factor chain
+        mbar_expect_tx(&bar_in2, 6 * 8192);
+        for (int at = 0; at < 2; ++at) {
+            tma_load_3d(sm + SS + at * 8192, &maps.q, at * 64, hh, y, &bar_in2);
+            tma_load_3d(sm + SS + 16384 + at * 8192, &maps.k, at * 64, hh, y, &bar_in2);
+            tma_load_3d(sm + DS + at * 8192, &maps.b, at * 64, hh, y, &bar_in2);
         }
-        __syncthreads();  // everyone has read sTot (forward cumsum) before it is reused
-        *reinterpret_cast<float2 *>(sTot + g8 * D + 2 * cp) = make_float2(run0, run1);
+    }
+    {  // [dP; dA] -> bf16 tile [128][64] (over v): dP lower incl., dA strictly lower
+        uint32_t r[16], w8[8];
+        tmem_ld16(tmem + TM_PA + 16 * cg + lane_off, r);
+        tmem_wait_ld();
+        const int t = row & 63, strict = row >> 6;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int s0 = 16 * cg + 2 * e;
+            w8[e] = pack_bf16x2((s0 + strict <= t) ? __uint_as_float(r[2 * e]) : 0.f,
+                                (s0 + 1 + strict <= t) ? __uint_as_float(r[2 * e + 1]) : 0.f);
+        }
+        *reinterpret_cast<uint4 *>(sm + PA + sw128(row, 32 * cg)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        *reinterpret_cast<uint4 *>(sm + PA + sw128(row, 32 * cg + 16)) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- [dQ~^T | dE~^T] += K~^T [dP; dA]^T;  dK~^T += Q~^T dP + E~^T dA
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_DQE, sdesc_sw128(sb + RK + ks * 2048, 8192, 1024), sdesc_sw128(sb + PA + ks * 32, 16, 1024),
+                   IDESC_MK2, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_DK, sdesc_sw128(sb + RQ + ks * 2048, 8192, 1024), sdesc_sw128(sb + PA + ks * 2048, 8192, 1024),
+                   IDESC_MM, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_DK, sdesc_sw128(sb + RB + ks * 2048, 8192, 1024),
+                   sdesc_sw128(sb + PA + 8192 + ks * 2048, 8192, 1024), IDESC_MM, 1);
+        mma_commit(&bar_d);
+    }
+    // ---- through the factors: thread = channel `row` of d_k, tokens 16 cg .. 16 cg + 15
+    {
+        float *sFin = reinterpret_cast<float *>(sm + SC_FIN);  // DY is free once bar_d completes
+        const bool ch_ok = row < a.din;
+        float al[16];
+        float run = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * cg + i;
+            const float gv = (t < L && ch_ok) ? *reinterpret_cast<const float *>(sm + GG + (row >> 5) * 8192 +
+                                                                                  sw128(t, (row & 31) * 4))
+                                              : 0.f;
+            run += gv;
+            al[i] = __expf(gv);
+        }
+        wait_or_flag(&bar_d, 0, a.status);
+        tc_fence_after();
+        sFin[cg * D + row] = run;
         __syncthreads();
-        float after0 = 0.f, after1 = 0.f;
+        float off = 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (u > g8) {
-                after0 += sTot[u * D + 2 * cp];
-                after1 += sTot[u * D + 2 * cp + 1];
+        for (int u = 0; u < 4; ++u)
+            if (u < cg) off += sFin[u * D + row];
+        float emG[16];
+        {
+            float rr = __expf(-(off + run));
+#pragma unroll
+            for (int i = 15; i >= 0; --i) {
+                emG[i] = rr;
+                rr *= al[i];
             }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * g8 + i;
-            if (t < L && ch_ok)
-                *reinterpret_cast<float2 *>(a.dg + base + (size_t)i * stride) =
-                    make_float2(dG[i].x + after0, dG[i].y + after1);
         }
+        uint32_t rq[16], re[16], rk[16];
+        tmem_ld16(tmem + TM_DQE + 16 * cg + lane_off, rq);
+        tmem_ld16(tmem + TM_DQE + 64 + 16 * cg + lane_off, re);
+        tmem_ld16(tmem + TM_DK + 16 * cg + lane_off, rk);
+        tmem_wait_ld();
+        wait_or_flag(&bar_in2, 0, a.status);
+        float e = __expf(off);
+        float dG[16];
+        const size_t base = tok_off(a, bb, hh, ci, 16 * cg) + row, stride = (size_t)a.H * a.din;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * cg + i;
+            e *= al[i];
+            const uint32_t so = tile_off(t, row, 8192);
+            const bool ok = t < L;
+            const float q0 = ok ? ld_bf(sm + SS + so) : 0.f, k0 = ok ? ld_bf(sm + SS + 16384 + so) : 0.f;
+            const float b0 = ok ? ld_bf(sm + DS + so) : 0.f;
+            const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dK = __uint_as_float(rk[i]);
+            const float de = dE * e;
+            dG[i] = dQ * q0 * e + de * b0 * k0 - dK * k0 * emG[i];
+            if (ok && ch_ok) {
+                const size_t go = base + (size_t)i * stride;
+                a.dq[go] = __float2bfloat16_rn(dQ * e);
+                a.db[go] = __float2bfloat16_rn(de * k0);
+                a.dk[go] = __float2bfloat16_rn(de * b0 + dK * emG[i]);
+            }
+        }
+        if (cg == 3) dG[15] += reinterpret_cast<const float *>(sm + DGF)[row];  // gamma dgamma, last row
+        float rs = 0.f;
+#pragma unroll
+        for (int i = 15; i >= 0; --i) {
+            rs += dG[i];
+            dG[i] = rs;
+        }
+        sFin[4 * D + cg * D + row] = rs;
+        __syncthreads();
+        float after = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u > cg) after += sFin[4 * D + u * D + row];
+        if (ch_ok) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = 16 * cg + i;
+                if (t < L) a.dg[base + (size_t)i * stride] = dG[i] + after;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
     }
 }
 
@@ -1128,8 +1215,23 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
     bwd_chain_kernel<<<p.B * p.H, kChainThreads, CH_SMEM, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)G_SMEM)) != cudaSuccess) return e;
-    bwd_grad_kernel<<<nblk, kGradThreads, G_SMEM, s>>>(a);
+    {  // gradients on the tensor cores: one block per (chunk, head)
+        GradMaps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int rows = (int)token_rows(p);
+        const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p), nbound = (uint64_t)p.H * (chunk_bound(p) + p.B);
+        if (!make_map(&maps.q, p.q, false, 1, rows, p.H, p.D) || !make_map(&maps.k, p.k, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D) || !make_map(&maps.v, p.v, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.w, p.w, false, 1, rows, p.H, p.D) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D) ||
+            !make_map_2d(&maps.st, a.states, D, nbound * D, 64, D) ||
+            !make_map_2d(&maps.dsn, a.dSn, D, nchunk * D, 64, D) ||
+            !make_map_2d(&maps.tm, a.Tm, C, nchunk * C, 64, C) || !make_map_2d(&maps.pm, a.Pm, C, nchunk * C, 64, C))
+            return cudaErrorInvalidValue;
+        if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)grad_tc::SMEM)) != cudaSuccess)
+            return e;
+        bwd_grad_kernel<<<nblk, grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+    }
     return cudaGetLastError();
 }
 

@@ -732,6 +732,21 @@ bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D view of a row-major bf16 matrix [rows][cols]: box = (box_cols, box_rows) with the 128-byte
+// swizzle (box_cols * 2 must be 128).
+bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || box_cols * 2 != 128 || box_rows == 0 || box_rows > 256) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s, const ScanArgs *scan)
 {

@@ -20,6 +20,9 @@ namespace gdn2 {
 // the channel extent reads zeros); store = true: box = (all din channels, 1, 64 tokens), no
 // swizzle.  Host function (fwd_tc.cu); false if the driver entry point or the encoding fails.
 bool make_map(CUtensorMap *m, const void *ptr, bool fp32, int B, int T, int H, int din, bool store = false);
+// TMA tensor map of a row-major bf16 matrix [rows][cols] as a 2-D view, box = (box_cols, box_rows)
+// with the 128-byte swizzle; box_cols * 2 must be 128.  Host function (fwd_tc.cu).
+bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows);
 
 namespace tc {
 
@@ -89,6 +92,13 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
 // Bulk tensor store from shared memory (tracked by the issuing thread's bulk group).
