@@ -190,12 +190,6 @@ __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8
     total = make_float2(tot0, tot1);
 }
 
-// L2 prefetch (bulk, no shared-memory destination)
-__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // ================================================================== 2. prep on the tensor cores
 // One 512-thread CTA per (chunk, head): the raw q, b, k, dO tiles arrive by TMA (SW128 atoms),
 // the decay folds into them in place, and the four products run as tcgen05 MMAs with TMEM
@@ -676,12 +670,12 @@ constexpr uint32_t GG = 49152;    // log alpha fp32 [64][128]: four 8 KiB boxes 
 constexpr uint32_t SS = 81920;    // S^T [128][128] (atoms 16 KiB apart); after the S products: raw q, k
 constexpr uint32_t DS = 114688;   // dS_n^T -> (Gm dS_n)^T; after its products: raw b
 constexpr uint32_t DY = 147456;   // [dO; -dY] [128][128]: atom a = dO rows 0-63 then -dY rows 64-127
-constexpr uint32_t TT = 180224;   // T [64][64]; after dY: U~ [64][128] over T and P
-constexpr uint32_t PP = 188416;   // P [64][64]
+constexpr uint32_t TT = 180224;   // T [64][64]; after dY: U~ [64][128] over T and P; after U~'s
+constexpr uint32_t PP = 188416;   //   products: [dP; dA] [128][64]
 constexpr uint32_t UU = TT;
-constexpr uint32_t VV = 196608;   // v; after dv and dw: [dP; dA] [128][64]
-constexpr uint32_t PA = VV;
-constexpr uint32_t WW = 212992;   // w
+constexpr uint32_t PA = TT;
+constexpr uint32_t VV = 196608;   // v, then dw (full chunks: stored from here by TMA)
+constexpr uint32_t WW = 212992;   // w, then dv
 constexpr uint32_t DGF = 229376;  // gamma dgamma [D] fp32
 constexpr uint32_t USED = DGF + D * 4;
 constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
@@ -690,7 +684,8 @@ constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
 constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
 constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
-constexpr uint32_t SC_FIN = DY;                  // factor chain: group sums [4][D], twice
+constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [4][D], twice
+// full chunks stage dq, dk, db over Q~, K~, E~ and dg over [dO; -dY] for the TMA stores
 // TMEM columns
 constexpr uint32_t TM_Y = 0, TM_DU = 64, TM_YB = 128, TM_DUB = 160, TM_U = 192, TM_DY = 256, TM_PA = 320;
 constexpr uint32_t TM_DQE = 384, TM_DK = 0, TM_COLS = 512;
@@ -703,7 +698,8 @@ constexpr int kThreads = 512;
 }  // namespace grad_tc
 
 struct GradMaps {
-    CUtensorMap q, k, b, v, w, dO, g, st, dsn, tm, pm;
+    CUtensorMap q, k, b, v, w, dO, g, st, dsn, tm, pm;  // loads
+    CUtensorMap dq, dk, db, dv, dw, dg;                 // stores of full chunks
 };
 
 __device__ __forceinline__ void wait_or_flag(uint64_t *bar, uint32_t parity, int *status)
@@ -740,46 +736,65 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     const int quarter = warp & 3, cg = warp >> 2, row = 32 * quarter + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
 
-    if (tid == 0) {
-        mbar_init(&bar_in0, 1);
-        mbar_init(&bar_in1, 1);
-        mbar_init(&bar_in2, 1);
-        mbar_init(&bar_a, 1);
-        mbar_init(&bar_b, 1);
-        mbar_init(&bar_c, 1);
-        mbar_init(&bar_d, 1);
-        fence_mbar_init();
-        const CUtensorMap *all[11] = {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w, &maps.dO,
-                                      &maps.g, &maps.st, &maps.dsn, &maps.tm, &maps.pm};
-        for (int i = 0; i < 11; ++i) prefetch_tmap(all[i]);
-    }
-    if (warp == 0) {
+    const int y = bb + ci * C;
+    const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
+    if (warp == 0) {  // barriers, then one tile load per lane
+        if (lane == 0) {
+            mbar_init(&bar_in0, 1);
+            mbar_init(&bar_in1, 1);
+            mbar_init(&bar_in2, 1);
+            mbar_init(&bar_a, 1);
+            mbar_init(&bar_b, 1);
+            mbar_init(&bar_c, 1);
+            mbar_init(&bar_d, 1);
+            fence_mbar_init();
+            mbar_expect_tx(&bar_in0, 10 * 8192);
+            mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
+        }
+        __syncwarp();
+        if (lane < 6) {  // q, k, b -> RQ, RK, RB
+            const int at = lane & 1, which = lane >> 1;
+            const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : &maps.b;
+            tma_load_3d(sm + RQ + which * 16384 + at * 8192, mp, at * 64, hh, y, &bar_in0);
+        } else if (lane < 10) {
+            tma_load_3d(sm + GG + (lane - 6) * 8192, &maps.g, (lane - 6) * 32, hh, y, &bar_in0);
+        } else if (lane < 14) {
+            const int at = lane & 1;
+            if (lane < 12) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, (int)(slot * D), &bar_in1);
+            else tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(cidx * D), &bar_in1);
+        } else if (lane < 20) {
+            const int at = lane & 1, which = (lane - 14) >> 1;
+            if (which == 0) tma_load_3d(sm + DY + at * 16384, &maps.dO, at * 64, hh, y, &bar_in1);
+            else tma_load_3d(sm + (which == 1 ? VV : WW) + at * 8192, which == 1 ? &maps.v : &maps.w, at * 64, hh, y,
+                             &bar_in1);
+        } else if (lane < 22) {
+            tma_load_2d(sm + (lane == 20 ? TT : PP), lane == 20 ? &maps.tm : &maps.pm, 0, (int)(cidx * C), &bar_in1);
+        }
+    } else if (warp == 1) {
         tmem_alloc(&s_tmem, TM_COLS);
         tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    const int y = bb + ci * C;
-    if (tid == 0) {
-        mbar_expect_tx(&bar_in0, 10 * 8192);
-        for (int at = 0; at < 2; ++at) {
-            tma_load_3d(sm + RQ + at * 8192, &maps.q, at * 64, hh, y, &bar_in0);
-            tma_load_3d(sm + RK + at * 8192, &maps.k, at * 64, hh, y, &bar_in0);
-            tma_load_3d(sm + RB + at * 8192, &maps.b, at * 64, hh, y, &bar_in0);
+    } else if (warp == 2) {  // the tiles of the block one wave later (block id + SM count), into L2
+        const int nblk = gridDim.x * gridDim.y, nxt = blockIdx.y * gridDim.x + blockIdx.x + a.n_sm;
+        ChunkRef r;
+        if (nxt < nblk && chunk_ref_at(a, nxt % gridDim.x, nxt / gridDim.x, r)) {
+            const int yn = r.sp.bos + r.ci * C;
+            const int sn = (int)(bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D);
+            const int at = lane & 1;
+            if (lane < 12) {
+                const int which = lane >> 1;
+                const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : which == 2 ? &maps.b
+                                      : which == 3 ? &maps.v : which == 4 ? &maps.w : &maps.dO;
+                tma_prefetch_3d(mp, at * 64, r.h, yn);
+            } else if (lane < 16) {
+                tma_prefetch_3d(&maps.g, (lane - 12) * 32, r.h, yn);
+            } else if (lane < 20) {  // the chunk's start and end states
+                tma_prefetch_2d(&maps.st, at * 64, sn + (lane < 18 ? 0 : D));
+            } else if (lane < 22) {
+                tma_prefetch_2d(&maps.dsn, at * 64, (int)(r.cidx * D));
+            } else if (lane < 24) {
+                tma_prefetch_2d(lane == 22 ? &maps.tm : &maps.pm, 0, (int)(r.cidx * C));
+            }
         }
-        for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + GG + bx * 8192, &maps.g, bx * 32, hh, y, &bar_in0);
-        mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
-        for (int at = 0; at < 2; ++at) {
-            tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, (int)(slot * D), &bar_in1);
-            tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(cidx * D), &bar_in1);
-            tma_load_3d(sm + DY + at * 16384, &maps.dO, at * 64, hh, y, &bar_in1);
-            tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, hh, y, &bar_in1);
-            tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, hh, y, &bar_in1);
-        }
-        tma_load_2d(sm + TT, &maps.tm, 0, (int)(cidx * C), &bar_in1);
-        tma_load_2d(sm + PP, &maps.pm, 0, (int)(cidx * C), &bar_in1);
     }
     // the chunk-end state (for gamma dgamma), in flight during the folding
     const int dch = tid & 15;
@@ -790,32 +805,10 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         for (int u = 0; u < 4; ++u)
             ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
     }
-    {  // everything the block one wave later reads, into L2 (one bulk prefetch per thread)
-        const int nblk = gridDim.x * gridDim.y, nxt = blockIdx.y * gridDim.x + blockIdx.x + a.n_sm;
-        ChunkRef r;
-        if (nxt < nblk && chunk_ref_at(a, nxt % gridDim.x, nxt / gridDim.x, r)) {
-            const int Ln = min(C, r.sp.len - r.ci * C);
-            const uint32_t rowb = (uint32_t)a.din * 2;
-            if (tid < 7 * C) {
-                const int which = tid / C, t = tid % C;
-                if (t < Ln) {
-                    const size_t off = tok_off(a, r.sp.bos, r.h, r.ci, t);
-                    const __nv_bfloat16 *src = which == 0 ? a.q : which == 1 ? a.k : which == 2 ? a.b
-                                             : which == 3 ? a.v : which == 4 ? a.w : a.dO;
-                    if (which < 6) bulk_prefetch_l2(src + off, rowb);
-                    else bulk_prefetch_l2(a.g + off, 2 * rowb);
-                }
-            } else if (tid == 7 * C) {
-                bulk_prefetch_l2(a.states + bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D * D, 2 * D * D * 2);
-            } else if (tid == 7 * C + 1) {
-                bulk_prefetch_l2(a.Tm + r.cidx * C * C, C * C * 2);
-            } else if (tid == 7 * C + 2) {
-                bulk_prefetch_l2(a.Pm + r.cidx * C * C, C * C * 2);
-            } else if (tid == 7 * C + 3) {
-                bulk_prefetch_l2(a.dSn + r.cidx * D * D, D * D * 2);
-            }
-        }
-    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
 
     // ---- decay folding in place: thread (channel pair cp, token group g8 of 8)
     const int cp = tid & 63, g8 = tid >> 6;
@@ -960,8 +953,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     }
     wait_or_flag(&bar_b, 0, a.status);
     tc_fence_after();
-    // ---- read back: U~ tile [s][d_v] (over T and P, both consumed); dv = dY w, dw = dY v;
-    //      -dY into rows 64-127 of [dO; -dY]
+    // ---- read back: U~ tile [s][d_v] (over T and P, both consumed); dv = dY w, dw = dY v (full
+    //      chunks: over w and v); -dY into rows 64-127 of [dO; -dY]
     {
         uint32_t r[16];
         tmem_ld16(tmem + TM_U + 16 * cg + lane_off, r);
@@ -976,11 +969,15 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             const int t = 16 * cg + i;
             const float d = __uint_as_float(r[i]);
             st_bf(sm + DY + tile_off(64 + t, row, 16384), -d);
-            if (t < L && ch_ok) {
-                const uint32_t so = tile_off(t, row, 8192);
+            const uint32_t so = tile_off(t, row, 8192);
+            const float wv = ld_bf(sm + WW + so), vv = ld_bf(sm + VV + so);
+            if (full) {
+                st_bf(sm + WW + so, d * wv);
+                st_bf(sm + VV + so, d * vv);
+            } else if (t < L && ch_ok) {
                 const size_t go = tok_off(a, bb, hh, ci, t) + row;
-                a.dv[go] = __float2bfloat16_rn(d * ld_bf(sm + WW + so));
-                a.dw[go] = __float2bfloat16_rn(d * ld_bf(sm + VV + so));
+                a.dv[go] = __float2bfloat16_rn(d * wv);
+                a.dw[go] = __float2bfloat16_rn(d * vv);
             }
         }
     }
@@ -1004,6 +1001,13 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                    sdesc_sw128(sb + UU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_MK, ks > 0);
         mma_commit(&bar_c);
     }
+    if (tid == 32 && full) {  // dv, dw by TMA (thread 32 owns every bulk store of the block)
+        for (int at = 0; at < a.din / 64; ++at) {
+            tma_store_3d(&maps.dv, sm + WW + at * 8192, at * 64, hh, y);
+            tma_store_3d(&maps.dw, sm + VV + at * 8192, at * 64, hh, y);
+        }
+        bulk_commit();
+    }
     wait_or_flag(&bar_c, 0, a.status);
     tc_fence_after();
     if (tid == 0) {  // S^T and (Gm dS_n)^T are consumed: the raw q, k, b for the factor chain
@@ -1014,7 +1018,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             tma_load_3d(sm + DS + at * 8192, &maps.b, at * 64, hh, y, &bar_in2);
         }
     }
-    {  // [dP; dA] -> bf16 tile [128][64] (over v): dP lower incl., dA strictly lower
+    {  // [dP; dA] -> bf16 tile [128][64] (over U~): dP lower incl., dA strictly lower
         uint32_t r[16], w8[8];
         tmem_ld16(tmem + TM_PA + 16 * cg + lane_off, r);
         tmem_wait_ld();
@@ -1050,7 +1054,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     }
     // ---- through the factors: thread = channel `row` of d_k, tokens 16 cg .. 16 cg + 15
     {
-        float *sFin = reinterpret_cast<float *>(sm + SC_FIN);  // DY is free once bar_d completes
+        float *sFin = reinterpret_cast<float *>(sm + SC_FIN);
         const bool ch_ok = row < a.din;
         float al[16];
         float run = 0.f;
@@ -1100,7 +1104,11 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dK = __uint_as_float(rk[i]);
             const float de = dE * e;
             dG[i] = dQ * q0 * e + de * b0 * k0 - dK * k0 * emG[i];
-            if (ok && ch_ok) {
+            if (full) {  // Q~, K~, E~ are consumed (bar_d)
+                st_bf(sm + RQ + so, dQ * e);
+                st_bf(sm + RB + so, de * k0);
+                st_bf(sm + RK + so, de * b0 + dK * emG[i]);
+            } else if (ok && ch_ok) {
                 const size_t go = base + (size_t)i * stride;
                 a.dq[go] = __float2bfloat16_rn(dQ * e);
                 a.db[go] = __float2bfloat16_rn(de * k0);
@@ -1120,7 +1128,12 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             if (u > cg) after += sFin[4 * D + u * D + row];
-        if (ch_ok) {
+        if (full) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<float *>(sm + DY + (row >> 5) * 8192 + sw128(16 * cg + i, (row & 31) * 4)) =
+                    dG[i] + after;
+        } else if (ch_ok) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int t = 16 * cg + i;
@@ -1128,8 +1141,21 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             }
         }
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 32) {
+        if (full) {
+            for (int at = 0; at < a.din / 64; ++at) {
+                tma_store_3d(&maps.dq, sm + RQ + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.dk, sm + RK + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.db, sm + RB + at * 8192, at * 64, hh, y);
+            }
+            for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + DY + bx * 8192, bx * 32, hh, y);
+            bulk_commit();
+        }
+        bulk_wait_read0();  // the shared-memory sources are read before the block exits
+    }
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
@@ -1226,7 +1252,10 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
             !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D) ||
             !make_map_2d(&maps.st, a.states, D, nbound * D, 64, D) ||
             !make_map_2d(&maps.dsn, a.dSn, D, nchunk * D, 64, D) ||
-            !make_map_2d(&maps.tm, a.Tm, C, nchunk * C, 64, C) || !make_map_2d(&maps.pm, a.Pm, C, nchunk * C, 64, C))
+            !make_map_2d(&maps.tm, a.Tm, C, nchunk * C, 64, C) || !make_map_2d(&maps.pm, a.Pm, C, nchunk * C, 64, C) ||
+            !make_map(&maps.dq, out.dq, false, 1, rows, p.H, p.D) || !make_map(&maps.dk, out.dk, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.db, out.db, false, 1, rows, p.H, p.D) || !make_map(&maps.dv, out.dv, false, 1, rows, p.H, p.D) ||
+            !make_map(&maps.dw, out.dw, false, 1, rows, p.H, p.D) || !make_map(&maps.dg, out.dg, true, 1, rows, p.H, p.D))
             return cudaErrorInvalidValue;
         if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)grad_tc::SMEM)) != cudaSuccess)
             return e;
