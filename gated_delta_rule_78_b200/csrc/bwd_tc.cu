@@ -86,7 +86,6 @@ struct BwdTcArgs {
     __nv_bfloat16 *Rt;  // R^T per chunk, bf16
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
-    int n_sm;            // multiprocessors of the device (L2 prefetch distance of the gradient kernel)
     int *status;         // kernel status word (bounded waits that gave up)
 };
 
@@ -516,25 +515,29 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
 }
 
 // ================================================================== 3. chain
-// One CTA per (batch, head); warp w owns rows 16 w .. 16 w + 15 of dS^T (d_v x d_k) and
-// keeps them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
+// The rows of dS^T (d_v x d_k) evolve independently, so each (batch, head) is split over
+// kChainSplit CTAs of 64 rows; warp w owns rows 16 w .. 16 w + 15 of its CTA's block and keeps
+// them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
 //   store dS_n^T (bf16) for the gradient kernel;
 //   Z^T = dS_n^T K^^T          (16 x 64 per warp, K = 128; A operand from registers)
 //   dS^T = dS_n^T Diag(gamma) + R^T - Z^T W   (K = 64; A operand = -Z^T from registers)
 // W, K^, gamma and R^T of the next chunk are copied in (cp.async) during the current one.
-constexpr int kChainThreads = 256;
+constexpr int kChainSplit = 2;                  // CTAs per (batch, head), two per SM
+constexpr int kChainRows = D / kChainSplit;     // rows of dS^T per CTA
+constexpr int kChainThreads = 2 * kChainRows;   // a warp per 16 rows
 constexpr int LDR = 136;  // bf16 row stride of the R^T tile (conflict-free fragment reads)
 constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_R = 33280;
-constexpr uint32_t CH_BUF = CH_R + D * LDR * 2;  // per buffer
+constexpr uint32_t CH_BUF = CH_R + kChainRows * LDR * 2;  // per buffer
 constexpr uint32_t CH_SMEM = 2 * CH_BUF;
 
-__global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTcArgs a)
+__global__ void __launch_bounds__(kChainThreads, 2) bwd_chain_kernel(const BwdTcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, n = bh / a.H, hh = bh % a.H;
+    const int bh = blockIdx.x / kChainSplit, part = blockIdx.x % kChainSplit, n = bh / a.H, hh = bh % a.H;
     const int g = lane >> 2, t4 = lane & 3;
-    const int j0 = 16 * warp;  // this warp's first row of dS^T
+    const int jl0 = 16 * warp;                   // this warp's first row within the CTA's block
+    const int j0 = part * kChainRows + jl0;      // ... and of dS^T
     const SeqSpan sp = seq_span(a.pr, n);
     if (sp.len < 0) return;  // invalid cu_seqlens (reported by the offsets pass)
     const int nc = seq_chunks(sp.len);
@@ -552,8 +555,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
             const int c = idx >> 3, ch = idx & 7;
             cp_async16(base + CH_W + swz(c, 8 * ch, 128), wsrc + c * C + 8 * ch);
         }
-        const __nv_bfloat16 *rsrc = a.Rt + cidx * D * D;
-        for (int idx = tid; idx < D * 16; idx += kChainThreads) {  // 16 x 16 bytes per bf16 row
+        const __nv_bfloat16 *rsrc = a.Rt + cidx * D * D + (size_t)part * kChainRows * D;
+        for (int idx = tid; idx < kChainRows * 16; idx += kChainThreads) {  // 16 x 16 bytes per bf16 row
             const int r = idx >> 4, ch = idx & 15;
             cp_async16(base + CH_R + (r * LDR + 8 * ch) * 2, rsrc + r * D + 8 * ch);
         }
@@ -616,8 +619,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(const BwdTc
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
             const float2 gm = *reinterpret_cast<const float2 *>(gam + 8 * nt + 2 * t4);
-            const uint32_t r0w = *reinterpret_cast<const uint32_t *>(rt + (j0 + g) * LDR + 8 * nt + 2 * t4);
-            const uint32_t r1w = *reinterpret_cast<const uint32_t *>(rt + (j0 + g + 8) * LDR + 8 * nt + 2 * t4);
+            const uint32_t r0w = *reinterpret_cast<const uint32_t *>(rt + (jl0 + g) * LDR + 8 * nt + 2 * t4);
+            const uint32_t r1w = *reinterpret_cast<const uint32_t *>(rt + (jl0 + g + 8) * LDR + 8 * nt + 2 * t4);
             const float2 r0 = make_float2(bf_lo(r0w), bf_hi(r0w)), r1 = make_float2(bf_lo(r1w), bf_hi(r1w));
             dS[nt][0] = dS[nt][0] * gm.x + r0.x;
             dS[nt][1] = dS[nt][1] * gm.y + r0.y;
@@ -738,20 +741,20 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 
     const int y = bb + ci * C;
     const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
-    if (warp == 0) {  // barriers, then one tile load per lane
-        if (lane == 0) {
-            mbar_init(&bar_in0, 1);
-            mbar_init(&bar_in1, 1);
-            mbar_init(&bar_in2, 1);
-            mbar_init(&bar_a, 1);
-            mbar_init(&bar_b, 1);
-            mbar_init(&bar_c, 1);
-            mbar_init(&bar_d, 1);
-            fence_mbar_init();
-            mbar_expect_tx(&bar_in0, 10 * 8192);
-            mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
-        }
-        __syncwarp();
+    if (tid == 0) {
+        mbar_init(&bar_in0, 1);
+        mbar_init(&bar_in1, 1);
+        mbar_init(&bar_in2, 1);
+        mbar_init(&bar_a, 1);
+        mbar_init(&bar_b, 1);
+        mbar_init(&bar_c, 1);
+        mbar_init(&bar_d, 1);
+        fence_mbar_init();
+        mbar_expect_tx(&bar_in0, 10 * 8192);
+        mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
+    }
+    __syncthreads();  // the barriers are ready; the TMEM address is published by the folding's barrier
+    if (warp == 0) {  // one tile load per lane
         if (lane < 6) {  // q, k, b -> RQ, RK, RB
             const int at = lane & 1, which = lane >> 1;
             const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : &maps.b;
@@ -773,28 +776,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     } else if (warp == 1) {
         tmem_alloc(&s_tmem, TM_COLS);
         tmem_relinquish();
-    } else if (warp == 2) {  // the tiles of the block one wave later (block id + SM count), into L2
-        const int nblk = gridDim.x * gridDim.y, nxt = blockIdx.y * gridDim.x + blockIdx.x + a.n_sm;
-        ChunkRef r;
-        if (nxt < nblk && chunk_ref_at(a, nxt % gridDim.x, nxt / gridDim.x, r)) {
-            const int yn = r.sp.bos + r.ci * C;
-            const int sn = (int)(bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D);
-            const int at = lane & 1;
-            if (lane < 12) {
-                const int which = lane >> 1;
-                const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : which == 2 ? &maps.b
-                                      : which == 3 ? &maps.v : which == 4 ? &maps.w : &maps.dO;
-                tma_prefetch_3d(mp, at * 64, r.h, yn);
-            } else if (lane < 16) {
-                tma_prefetch_3d(&maps.g, (lane - 12) * 32, r.h, yn);
-            } else if (lane < 20) {  // the chunk's start and end states
-                tma_prefetch_2d(&maps.st, at * 64, sn + (lane < 18 ? 0 : D));
-            } else if (lane < 22) {
-                tma_prefetch_2d(&maps.dsn, at * 64, (int)(r.cidx * D));
-            } else if (lane < 24) {
-                tma_prefetch_2d(lane == 22 ? &maps.tm : &maps.pm, 0, (int)(r.cidx * C));
-            }
-        }
+        tc_fence_before();
     }
     // the chunk-end state (for gamma dgamma), in flight during the folding
     const int dch = tid & 15;
@@ -805,10 +787,6 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         for (int u = 0; u < 4; ++u)
             ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
 
     // ---- decay folding in place: thread (channel pair cp, token group g8 of 8)
     const int cp = tid & 63, g8 = tid >> 6;
@@ -844,6 +822,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     }
     fence_proxy_async_smem();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;  // written by warp 1 before the folding's first barrier
     // ---- Y^T = S^T E~^T (into TM_Y; X is added at the read-back)
     wait_or_flag(&bar_in1, 0, a.status);
     if (tid == 0) {
@@ -1213,11 +1193,6 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.dg = out.dg;
     a.dS0 = out.dS0;
     a.status = status;
-    {
-        int dev = 0;
-        a.n_sm = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&a.n_sm, cudaDevAttrMultiProcessorCount, dev);
-    }
 
     cudaError_t e = cudaSuccess;
     if (!states_saved || p.cu_seqlens) {  // chunk-boundary states, unless the forward recorded them
@@ -1239,7 +1214,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
-    bwd_chain_kernel<<<p.B * p.H, kChainThreads, CH_SMEM, s>>>(a);
+    bwd_chain_kernel<<<p.B * p.H * kChainSplit, kChainThreads, CH_SMEM, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {  // gradients on the tensor cores: one block per (chunk, head)
         GradMaps maps;
