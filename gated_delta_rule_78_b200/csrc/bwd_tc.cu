@@ -688,7 +688,7 @@ constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp
 constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
 constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [4][D], twice
-// full chunks stage dq, dk, db over Q~, K~, E~ and dg over [dO; -dY] for the TMA stores
+// full chunks stage dq, dk, db over the reloaded raw q, k, b and dg over v, w for the TMA stores
 // TMEM columns
 constexpr uint32_t TM_Y = 0, TM_DU = 64, TM_YB = 128, TM_DUB = 160, TM_U = 192, TM_DY = 256, TM_PA = 320;
 constexpr uint32_t TM_DQE = 384, TM_DK = 0, TM_COLS = 512;
@@ -728,19 +728,18 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     __shared__ __align__(8) uint64_t bar_in0, bar_in1, bar_in2, bar_a, bar_b, bar_c, bar_d;
     __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    ChunkRef cr;
-    if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
-    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
-    const int L = min(C, cr.sp.len - ci * C);
-    const size_t cidx = cr.cidx;
     const uint32_t sb = smem_u32(sm);
-    const size_t slot = bound_slot(a.pr, cr.n, hh, cr.nch, ci);
     // TMEM access: warp w reads lanes 32 (w & 3) .. + 31; column block w >> 2 (16 columns)
     const int quarter = warp & 3, cg = warp >> 2, row = 32 * quarter + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
-
-    const int y = bb + ci * C;
-    const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
+    // the block's tasks: blockIdx.x, + gridDim.x, ... over (chunk, head); chunks past a
+    // sequence's end are skipped
+    const int nchb = (int)chunk_bound(a.pr), ntask = nchb * a.H;
+    auto find_task = [&](int from, ChunkRef &r) -> int {
+        for (int t = from; t < ntask; t += gridDim.x)
+            if (chunk_ref_at(a, t % nchb, t / nchb, r)) return t;
+        return -1;
+    };
     if (tid == 0) {
         mbar_init(&bar_in0, 1);
         mbar_init(&bar_in1, 1);
@@ -750,34 +749,62 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         mbar_init(&bar_c, 1);
         mbar_init(&bar_d, 1);
         fence_mbar_init();
-        mbar_expect_tx(&bar_in0, 10 * 8192);
-        mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
     }
-    __syncthreads();  // the barriers are ready; the TMEM address is published by the folding's barrier
-    if (warp == 0) {  // one tile load per lane
-        if (lane < 6) {  // q, k, b -> RQ, RK, RB
-            const int at = lane & 1, which = lane >> 1;
-            const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : &maps.b;
-            tma_load_3d(sm + RQ + which * 16384 + at * 8192, mp, at * 64, hh, y, &bar_in0);
-        } else if (lane < 10) {
-            tma_load_3d(sm + GG + (lane - 6) * 8192, &maps.g, (lane - 6) * 32, hh, y, &bar_in0);
-        } else if (lane < 14) {
-            const int at = lane & 1;
-            if (lane < 12) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, (int)(slot * D), &bar_in1);
-            else tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(cidx * D), &bar_in1);
-        } else if (lane < 20) {
-            const int at = lane & 1, which = (lane - 14) >> 1;
-            if (which == 0) tma_load_3d(sm + DY + at * 16384, &maps.dO, at * 64, hh, y, &bar_in1);
-            else tma_load_3d(sm + (which == 1 ? VV : WW) + at * 8192, which == 1 ? &maps.v : &maps.w, at * 64, hh, y,
-                             &bar_in1);
-        } else if (lane < 22) {
-            tma_load_2d(sm + (lane == 20 ? TT : PP), lane == 20 ? &maps.tm : &maps.pm, 0, (int)(cidx * C), &bar_in1);
-        }
-    } else if (warp == 1) {
+    if (warp == 1) {
         tmem_alloc(&s_tmem, TM_COLS);
         tmem_relinquish();
-        tc_fence_before();
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    // A task's tile loads, issued by warp 0 in three parts as their regions free up during the
+    // task before: part 0 q, k, b, dO, T, P (and both input barriers' byte counts); part 1 log
+    // alpha; part 2 S^T, dS_n^T, v, w.
+    auto issue = [&](int part, const ChunkRef &r) {
+        const int yy = r.sp.bos + r.ci * C, h = r.h, at = lane & 1;
+        if (part == 0) {
+            if (lane == 0) {
+                mbar_expect_tx(&bar_in0, 10 * 8192);
+                mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
+            }
+            __syncwarp();
+            if (lane < 6) {
+                const int which = lane >> 1;
+                const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : &maps.b;
+                tma_load_3d(sm + RQ + which * 16384 + at * 8192, mp, at * 64, h, yy, &bar_in0);
+            } else if (lane < 8) {
+                tma_load_3d(sm + DY + at * 16384, &maps.dO, at * 64, h, yy, &bar_in1);
+            } else if (lane < 10) {
+                tma_load_2d(sm + (lane == 8 ? TT : PP), lane == 8 ? &maps.tm : &maps.pm, 0, (int)(r.cidx * C), &bar_in1);
+            }
+        } else if (part == 1) {
+            if (lane < 4) tma_load_3d(sm + GG + lane * 8192, &maps.g, lane * 32, h, yy, &bar_in0);
+        } else {
+            const int sl = (int)(bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D);
+            if (lane < 2) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, sl, &bar_in1);
+            else if (lane < 4) tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(r.cidx * D), &bar_in1);
+            else if (lane < 6) tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, h, yy, &bar_in1);
+            else if (lane < 8) tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, h, yy, &bar_in1);
+        }
+    };
+    ChunkRef cr;
+    int task = find_task(blockIdx.x, cr);
+    if (warp == 0 && task >= 0) {
+        issue(0, cr);
+        issue(1, cr);
+        issue(2, cr);
+    }
+    uint32_t ph = 0;  // parity of this task's barrier phases
+    while (task >= 0) {
+    ChunkRef nx;
+    const int next = find_task(task + gridDim.x, nx);
+    const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
+    const int L = min(C, cr.sp.len - ci * C);
+    const size_t cidx = cr.cidx;
+    const size_t slot = bound_slot(a.pr, cr.n, hh, cr.nch, ci);
+    const int y = bb + ci * C;
+    const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
     // the chunk-end state (for gamma dgamma), in flight during the folding
     const int dch = tid & 15;
     uint4 ssv[4];
@@ -792,7 +819,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     const int cp = tid & 63, g8 = tid >> 6;
     float *sTot = reinterpret_cast<float *>(sm + SC_TOT);
     float *sGam = reinterpret_cast<float *>(sm + SC_GAM);
-    wait_or_flag(&bar_in0, 0, a.status);
+    wait_or_flag(&bar_in0, ph, a.status);
     {
         const bool ch_ok = 2 * cp < a.din;
         float2 gl[8], eG[8], emG[8], tot;
@@ -823,9 +850,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = s_tmem;  // written by warp 1 before the folding's first barrier
     // ---- Y^T = S^T E~^T (into TM_Y; X is added at the read-back)
-    wait_or_flag(&bar_in1, 0, a.status);
+    wait_or_flag(&bar_in1, ph, a.status);
     if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -892,7 +918,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         mma_commit(&bar_a);
     }
     // ---- read back: Y^T = X^T - acc and dU~^T, as bf16 A operands (lane = d_v, 16 tokens per warp)
-    wait_or_flag(&bar_a, 0, a.status);
+    wait_or_flag(&bar_a, ph, a.status);
     tc_fence_after();
     {
         uint32_t r[16], pk[8];
@@ -931,7 +957,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             mma_ts(tmem + TM_DY, tmem + TM_DUB + 8 * ks, sdesc_sw128(sb + TT + ks * 2048, 8192, 1024), IDESC_KM, ks > 0);
         mma_commit(&bar_b);
     }
-    wait_or_flag(&bar_b, 0, a.status);
+    wait_or_flag(&bar_b, ph, a.status);
     tc_fence_after();
     // ---- read back: U~ tile [s][d_v] (over T and P, both consumed); dv = dY w, dw = dY v (full
     //      chunks: over w and v); -dY into rows 64-127 of [dO; -dY]
@@ -988,7 +1014,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         }
         bulk_commit();
     }
-    wait_or_flag(&bar_c, 0, a.status);
+    wait_or_flag(&bar_c, ph, a.status);
     tc_fence_after();
     if (tid == 0) {  // S^T and (Gm dS_n)^T are consumed: the raw q, k, b for the factor chain
         mbar_expect_tx(&bar_in2, 6 * 8192);
@@ -1047,10 +1073,12 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             run += gv;
             al[i] = __expf(gv);
         }
-        wait_or_flag(&bar_d, 0, a.status);
+        wait_or_flag(&bar_d, ph, a.status);
         tc_fence_after();
+        if (warp == 0 && next >= 0) issue(0, nx);  // Q~, K~, E~, [dO; -dY], T, P are consumed
         sFin[cg * D + row] = run;
         __syncthreads();
+        if (warp == 0 && next >= 0) issue(1, nx);  // log alpha is read
         float off = 0.f;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -1069,7 +1097,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         tmem_ld16(tmem + TM_DQE + 64 + 16 * cg + lane_off, re);
         tmem_ld16(tmem + TM_DK + 16 * cg + lane_off, rk);
         tmem_wait_ld();
-        wait_or_flag(&bar_in2, 0, a.status);
+        wait_or_flag(&bar_in2, ph, a.status);
         float e = __expf(off);
         float dG[16];
         const size_t base = tok_off(a, bb, hh, ci, 16 * cg) + row, stride = (size_t)a.H * a.din;
@@ -1084,10 +1112,10 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dK = __uint_as_float(rk[i]);
             const float de = dE * e;
             dG[i] = dQ * q0 * e + de * b0 * k0 - dK * k0 * emG[i];
-            if (full) {  // Q~, K~, E~ are consumed (bar_d)
-                st_bf(sm + RQ + so, dQ * e);
-                st_bf(sm + RB + so, de * k0);
-                st_bf(sm + RK + so, de * b0 + dK * emG[i]);
+            if (full) {  // over the raw q, k, b just read
+                st_bf(sm + SS + so, dQ * e);
+                st_bf(sm + DS + so, de * k0);
+                st_bf(sm + SS + 16384 + so, de * b0 + dK * emG[i]);
             } else if (ok && ch_ok) {
                 const size_t go = base + (size_t)i * stride;
                 a.dq[go] = __float2bfloat16_rn(dQ * e);
@@ -1103,6 +1131,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             dG[i] = rs;
         }
         sFin[4 * D + cg * D + row] = rs;
+        if (tid == 32) bulk_wait_read0();  // dv and dw have left v and w, which now take dg
         __syncthreads();
         float after = 0.f;
 #pragma unroll
@@ -1111,7 +1140,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         if (full) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                *reinterpret_cast<float *>(sm + DY + (row >> 5) * 8192 + sw128(16 * cg + i, (row & 31) * 4)) =
+                *reinterpret_cast<float *>(sm + VV + (row >> 5) * 8192 + sw128(16 * cg + i, (row & 31) * 4)) =
                     dG[i] + after;
         } else if (ch_ok) {
 #pragma unroll
@@ -1127,16 +1156,24 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     if (tid == 32) {
         if (full) {
             for (int at = 0; at < a.din / 64; ++at) {
-                tma_store_3d(&maps.dq, sm + RQ + at * 8192, at * 64, hh, y);
-                tma_store_3d(&maps.dk, sm + RK + at * 8192, at * 64, hh, y);
-                tma_store_3d(&maps.db, sm + RB + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.dq, sm + SS + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
             }
-            for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + DY + bx * 8192, bx * 32, hh, y);
+            for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + VV + bx * 8192, bx * 32, hh, y);
             bulk_commit();
         }
-        bulk_wait_read0();  // the shared-memory sources are read before the block exits
+        bulk_wait_read0();  // the staged gradients are read before their tiles are refilled
     }
-    if (warp == 0) {
+    __syncthreads();
+    if (warp == 0 && next >= 0) issue(2, nx);
+    task = next;
+    cr = nx;
+    ph ^= 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }
@@ -1234,7 +1271,10 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
             return cudaErrorInvalidValue;
         if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)grad_tc::SMEM)) != cudaSuccess)
             return e;
-        bwd_grad_kernel<<<nblk, grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+        int dev = 0, n_sm = 148;  // persistent: one block per multiprocessor
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        const int ntask = (int)chunk_bound(p) * p.H;
+        bwd_grad_kernel<<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
     }
     return cudaGetLastError();
 }
