@@ -1077,6 +1077,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         tc_fence_after();
         if (warp == 0 && next >= 0) issue(0, nx);  // Q~, K~, E~, [dO; -dY], T, P are consumed
         sFin[cg * D + row] = run;
+        if (tid == 32) bulk_wait_read0();  // dv and dw have left v and w, which take dg below
         __syncthreads();
         if (warp == 0 && next >= 0) issue(1, nx);  // log alpha is read
         float off = 0.f;
@@ -1131,8 +1132,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             dG[i] = rs;
         }
         sFin[4 * D + cg * D + row] = rs;
-        if (tid == 32) bulk_wait_read0();  // dv and dw have left v and w, which now take dg
-        __syncthreads();
+        named_bar(1 + quarter, 4 * 32);  // the four warps of this TMEM lane quarter
         float after = 0.f;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -1153,8 +1153,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 32) {
-        if (full) {
+    if (warp == 1) {  // lane 0 owns every bulk store of the block
+        if (lane == 0 && full) {
             for (int at = 0; at < a.din / 64; ++at) {
                 tma_store_3d(&maps.dq, sm + SS + at * 8192, at * 64, hh, y);
                 tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
@@ -1163,10 +1163,10 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + VV + bx * 8192, bx * 32, hh, y);
             bulk_commit();
         }
-        bulk_wait_read0();  // the staged gradients are read before their tiles are refilled
+        if (lane == 0) bulk_wait_read0();  // the staged gradients are read before their tiles are refilled
+        __syncwarp();
+        if (next >= 0) issue(2, nx);  // S^T, dS_n^T, v, w into the freed tiles
     }
-    __syncthreads();
-    if (warp == 0 && next >= 0) issue(2, nx);
     task = next;
     cr = nx;
     ph ^= 1;

@@ -106,6 +106,8 @@ class DecodeStream:
 WORKLOADS = {
     "tiny_f32": dict(B=1, T=256, H=2, Dk=64, Dv=64, dtype="f32", s0="zeros"),
     "layer_4k": dict(B=8, T=4096, H=16, Dk=128, Dv=128, dtype="bf16", s0="normal"),
+    # the layer shape at batch 2: profiler captures of one launch (still larger than L2)
+    "layer_4k_b2": dict(B=2, T=4096, H=16, Dk=128, Dv=128, dtype="bf16", s0="normal"),
     "sweep_2k": dict(B=32, T=2048, H=16, Dk=128, Dv=128, dtype="bf16", s0="normal"),
     "sweep_4k": dict(B=16, T=4096, H=16, Dk=128, Dv=128, dtype="bf16", s0="normal"),
     "sweep_8k": dict(B=8, T=8192, H=16, Dk=128, Dv=128, dtype="bf16", s0="normal"),
