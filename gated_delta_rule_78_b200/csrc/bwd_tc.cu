@@ -24,13 +24,13 @@
 // so the work splits into four launches:
 //   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary;
 //   2. bwd_prep_tc_kernel, one CTA per chunk: factors, [A; P], T, W^T, R^T (no state
-//      needed), the products as tcgen05 MMAs with TMEM accumulators;
-//   3. bwd_chain_kernel, one CTA per (batch, head): the reverse dS chain,
-//      two warp MMAs per chunk with dS^T kept in registers; stores dS_n per chunk;
-//   4. bwd_grad_kernel, one CTA per chunk: recomputes U~ from the stored state and
-//      produces every gradient of the chunk.
-// The chain and gradient products are bf16 warp MMAs (m16n8k16) on ldmatrix-fed
-// swizzled tiles.
+//      needed);
+//   3. bwd_chain_tc_kernel, one CTA per (batch, head): the reverse dS chain with dS^T
+//      kept in TMEM; stores dS_n per chunk;
+//   4. bwd_grad_kernel, persistent over the chunks: recomputes U~ from the stored state
+//      and produces every gradient of the chunk.
+// Every product is a bf16 tcgen05 MMA with an fp32 TMEM accumulator, its operands
+// in 128-byte swizzled shared-memory tiles (most of them loaded by TMA) or in TMEM.
 #include <cuda.h>
 #include <string.h>
 
@@ -92,14 +92,6 @@ struct BwdTcArgs {
 // ------------------------------------------------------------------ small helpers
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Row t of chunk `ci` of head hh of the sequence whose first token row is `bos`.
 __device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bos, int hh, int ci, int t)
@@ -514,141 +506,195 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     }
 }
 
-// ================================================================== 3. chain
-// The rows of dS^T (d_v x d_k) evolve independently, so each (batch, head) is split over
-// kChainSplit CTAs of 64 rows; warp w owns rows 16 w .. 16 w + 15 of its CTA's block and keeps
-// them in fp32 registers in MMA accumulator layout.  Per chunk, newest first:
-//   store dS_n^T (bf16) for the gradient kernel;
-//   Z^T = dS_n^T K^^T          (16 x 64 per warp, K = 128; A operand from registers)
-//   dS^T = dS_n^T Diag(gamma) + R^T - Z^T W   (K = 64; A operand = -Z^T from registers)
-// W, K^, gamma and R^T of the next chunk are copied in (cp.async) during the current one.
-constexpr int kChainSplit = 2;                  // CTAs per (batch, head), two per SM
-constexpr int kChainRows = D / kChainSplit;     // rows of dS^T per CTA
-constexpr int kChainThreads = 2 * kChainRows;   // a warp per 16 rows
-constexpr int LDR = 136;  // bf16 row stride of the R^T tile (conflict-free fragment reads)
-constexpr uint32_t CH_W = 0, CH_K = 16384, CH_G = 32768, CH_R = 33280;
-constexpr uint32_t CH_BUF = CH_R + kChainRows * LDR * 2;  // per buffer
-constexpr uint32_t CH_SMEM = 2 * CH_BUF;
+// ================================================================== 3. chain on the tensor cores
+// One CTA per (batch, head).  dS^T (d_v x d_k, fp32) lives in TMEM as an MMA accumulator, one
+// row per lane.  Per chunk, newest first:
+//   read dS_n^T: bf16 copy to global (the gradient kernel's dS_n) and to TMEM (A operand);
+//     dS_n^T Diag(gamma) + R^T back into the accumulator;
+//   Z^T = dS_n^T K^^T                    M d_v, N 64, K d_k   (A from TMEM)
+//   dS^T += (-Z^T) W                     M d_v, N d_k, K 64   (A = -Z^T bf16 from TMEM)
+// K^, W^T, R^T and gamma arrive by TMA in a three-stage ring, two chunks ahead.
+namespace chain_tc {
+constexpr uint32_t ST_K = 0;          // K^ [64][128] (two 8 KiB atoms)
+constexpr uint32_t ST_W = 16384;      // W^T [128 d_k][64 tokens] (one 16 KiB atom)
+constexpr uint32_t ST_R = 32768;      // R^T [128][128] (two 16 KiB atoms)
+constexpr uint32_t ST_G = 65536;      // gamma [128] fp32
+constexpr uint32_t STAGE = 66560;     // 65 KiB, 1024-aligned
+constexpr int kStages = 3;
+constexpr uint32_t SMEM = kStages * STAGE + 1024;
+constexpr uint32_t STAGE_BYTES = 16384 + 16384 + 32768 + 512;
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_ZB = 256, TM_COLS = 512;
+constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);
+constexpr int kThreads = 256;
+}  // namespace chain_tc
 
-__global__ void __launch_bounds__(kChainThreads, 2) bwd_chain_kernel(const BwdTcArgs a)
+struct ChainMaps {
+    CUtensorMap kh, wt, rt;
+};
+
+__global__ void __launch_bounds__(chain_tc::kThreads, 1)
+bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
 {
-    extern __shared__ __align__(1024) uint8_t sm[];
+    using namespace chain_tc;
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_full[kStages], bar_z, bar_s;
+    __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x / kChainSplit, part = blockIdx.x % kChainSplit, n = bh / a.H, hh = bh % a.H;
-    const int g = lane >> 2, t4 = lane & 3;
-    const int jl0 = 16 * warp;                   // this warp's first row within the CTA's block
-    const int j0 = part * kChainRows + jl0;      // ... and of dS^T
+    const int bh = blockIdx.x, n = bh / a.H, hh = bh % a.H;
     const SeqSpan sp = seq_span(a.pr, n);
     if (sp.len < 0) return;  // invalid cu_seqlens (reported by the offsets pass)
     const int nc = seq_chunks(sp.len);
-    const uint32_t sb = smem_u32(sm);
+    // TMEM access: warp w reads lanes 32 (w & 3) .. + 31 (rows of dS^T) and column half w >> 2
+    const int quarter = warp & 3, half = warp >> 2, row = 32 * quarter + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
 
-    auto prefetch = [&](int ci, int buf) {
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bar_full[s], 1);
+        mbar_init(&bar_z, 1);
+        mbar_init(&bar_s, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&s_tmem, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    // chunk ci's K^, W^T, R^T, gamma into stage s
+    auto load = [&](int ci, int s) {
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
-        const uint32_t base = sb + buf * CH_BUF;
-        const __nv_bfloat16 *wsrc = a.W + cidx * C * D, *ksrc = a.Kh + cidx * C * D;
-        for (int idx = tid; idx < C * 16; idx += kChainThreads) {
-            const int t = idx >> 4, ch = idx & 15;
-            cp_async16(base + CH_K + swz(t, 8 * ch, 256), ksrc + t * D + 8 * ch);
+        uint8_t *st = sm + s * STAGE;
+        mbar_expect_tx(&bar_full[s], STAGE_BYTES);
+        for (int at = 0; at < 2; ++at) {
+            tma_load_2d(st + ST_K + at * 8192, &maps.kh, at * 64, (int)(cidx * C), &bar_full[s]);
+            tma_load_2d(st + ST_R + at * 16384, &maps.rt, at * 64, (int)(cidx * D), &bar_full[s]);
         }
-        for (int idx = tid; idx < D * 8; idx += kChainThreads) {  // W^T: 128 rows of 64 tokens
-            const int c = idx >> 3, ch = idx & 7;
-            cp_async16(base + CH_W + swz(c, 8 * ch, 128), wsrc + c * C + 8 * ch);
-        }
-        const __nv_bfloat16 *rsrc = a.Rt + cidx * D * D + (size_t)part * kChainRows * D;
-        for (int idx = tid; idx < kChainRows * 16; idx += kChainThreads) {  // 16 x 16 bytes per bf16 row
-            const int r = idx >> 4, ch = idx & 15;
-            cp_async16(base + CH_R + (r * LDR + 8 * ch) * 2, rsrc + r * D + 8 * ch);
-        }
-        if (tid < 32) cp_async16(base + CH_G + 16 * tid, a.gam + cidx * D + 4 * tid);
-        cp_async_commit();
+        tma_load_2d(st + ST_W, &maps.wt, 0, (int)(cidx * D), &bar_full[s]);
+        bulk_load(st + ST_G, a.gam + cidx * D, D * 4, &bar_full[s]);
     };
-
-    // dS^T rows j0 + g (+8), columns 8 nt + 2 t4 (+1)
-    float dS[16][4];
+    if (tid == 0) {
+        for (int u = 0; u < 2 && u < nc; ++u) load(nc - 1 - u, u);
+    }
+    // dS^T from dS_T (stored [c][j]: dS^T[j][c] = dS_T[c][j]); this thread: row j, 64 columns
+    {
+        uint32_t r[32];
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
-            dS[nt][e] = (a.dS_T && c < a.din && j < a.din) ? a.dS_T[((size_t)bh * a.din + c) * a.din + j] : 0.f;
+            for (int u = 0; u < 32; ++u) {
+                const int c = 64 * half + 32 * h2 + u;
+                r[u] = __float_as_uint((a.dS_T && c < a.din && row < a.din)
+                                           ? a.dS_T[((size_t)bh * a.din + c) * a.din + row] : 0.f);
+            }
+            tmem_st32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
         }
-    if (nc > 0) prefetch(nc - 1, 0);
-    for (int ci = nc - 1; ci >= 0; --ci) {
-        const int buf = (nc - 1 - ci) & 1;
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    for (int it = 0; it < nc; ++it) {
+        const int ci = nc - 1 - it, s = it % kStages;
+        const uint32_t par = (uint32_t)(it / kStages) & 1u, ph = (uint32_t)it & 1u;
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
-        if (ci > 0) {
-            prefetch(ci - 1, buf ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+        const uint8_t *st = sm + s * STAGE;
+        if (tid == 0 && ci - 2 >= 0) load(ci - 2, (it + 2) % kStages);  // stage freed by step it - 1
+        if (!mbar_wait(&bar_full[s], par)) atomicExch(a.status, kStatusTimeout);
+        // ---- dS_n^T: bf16 to global and to TMEM; dS_n^T Diag(gamma) + R^T back into the accumulator
+        {
+            const float *gam = reinterpret_cast<const float *>(st + ST_G) + 64 * half;
+            __nv_bfloat16 *dsn = a.dSn + cidx * D * D + (size_t)row * D + 64 * half;
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t r[32], pk[16];
+                tmem_ld32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                tmem_st16(tmem + TM_SB + 32 * half + 16 * h2 + lane_off, pk);
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(dsn + 32 * h2 + 8 * m) =
+                        make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {  // R^T row `row`, columns 64 half + 32 h2 + 8 m .. + 7
+                    const uint4 rv = *reinterpret_cast<const uint4 *>(st + ST_R + half * 16384 +
+                                                                      sw128(row, (32 * h2 + 8 * m) * 2));
+                    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int u = 8 * m + 2 * e;
+                        const float2 g2 = *reinterpret_cast<const float2 *>(gam + 32 * h2 + u);
+                        r[u] = __float_as_uint(__uint_as_float(r[u]) * g2.x + bf_lo(rw[e]));
+                        r[u + 1] = __float_as_uint(__uint_as_float(r[u + 1]) * g2.y + bf_hi(rw[e]));
+                    }
+                }
+                tmem_st32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
+            }
+            tmem_wait_st();
         }
+        tc_fence_before();
         __syncthreads();
-        const uint32_t wb = sb + buf * CH_BUF + CH_W, kb = sb + buf * CH_BUF + CH_K;
-        const float *gam = reinterpret_cast<const float *>(sm + buf * CH_BUF + CH_G);
-        const __nv_bfloat16 *rt = reinterpret_cast<const __nv_bfloat16 *>(sm + buf * CH_BUF + CH_R);
-        // dS_n^T for the gradient kernel, and as bf16 A fragments
-        uint32_t aS[8][4];
-        __nv_bfloat16 *dsn = a.dSn + cidx * D * D;
+        // ---- Z^T = dS_n^T K^^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t kb = smem_u32(st + ST_K);
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-            acc_to_a(aS[kc], dS[2 * kc], dS[2 * kc + 1], 1.f);
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const size_t row = (size_t)(j0 + g + 8 * hr) * D;
-                *reinterpret_cast<uint32_t *>(dsn + row + 16 * kc + 2 * t4) = aS[kc][hr];
-                *reinterpret_cast<uint32_t *>(dsn + row + 16 * kc + 8 + 2 * t4) = aS[kc][2 + hr];
-            }
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ts(tmem + TM_Z, tmem + TM_SB + 8 * ks, sdesc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                       IDESC_Z, ks > 0);
+            mma_commit(&bar_z);
         }
-        // Z^T = dS_n^T K^^T: B operand K^ stored [t][c] = [n][k]
-        float Z[8][4];
+        if (!mbar_wait(&bar_z, ph)) atomicExch(a.status, kStatusTimeout);
+        tc_fence_after();
+        {  // -Z^T -> bf16 A operand: warp = lane quarter x 32 columns
+            uint32_t r[32], pk[16];
+            tmem_ld32(tmem + TM_Z + 32 * half + lane_off, r);
+            tmem_wait_ld();
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) Z[nt][e] = 0.f;
-#pragma unroll
-        for (int kc = 0; kc < 8; ++kc)
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t bfr[4];
-                load_b2<false>(bfr, kb, 256, 16 * kc, 16 * np, lane);
-                mma_bf16(Z[2 * np], aS[kc], bfr[0], bfr[1]);
-                mma_bf16(Z[2 * np + 1], aS[kc], bfr[2], bfr[3]);
-            }
-        // dS^T <- dS_n^T Diag(gamma) + R^T - Z^T W: B operand W stored [t][c] = [k][n]
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const float2 gm = *reinterpret_cast<const float2 *>(gam + 8 * nt + 2 * t4);
-            const uint32_t r0w = *reinterpret_cast<const uint32_t *>(rt + (jl0 + g) * LDR + 8 * nt + 2 * t4);
-            const uint32_t r1w = *reinterpret_cast<const uint32_t *>(rt + (jl0 + g + 8) * LDR + 8 * nt + 2 * t4);
-            const float2 r0 = make_float2(bf_lo(r0w), bf_hi(r0w)), r1 = make_float2(bf_lo(r1w), bf_hi(r1w));
-            dS[nt][0] = dS[nt][0] * gm.x + r0.x;
-            dS[nt][1] = dS[nt][1] * gm.y + r0.y;
-            dS[nt][2] = dS[nt][2] * gm.x + r1.x;
-            dS[nt][3] = dS[nt][3] * gm.y + r1.y;
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(-__uint_as_float(r[2 * e]), -__uint_as_float(r[2 * e + 1]));
+            tmem_st16(tmem + TM_ZB + 16 * half + lane_off, pk);
+            tmem_wait_st();
         }
+        tc_fence_before();
+        __syncthreads();
+        // ---- dS^T += (-Z^T) W
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t wb = smem_u32(st + ST_W);
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            uint32_t aZ[4];
-            acc_to_a(aZ, Z[2 * kt], Z[2 * kt + 1], -1.f);
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t bfr[4];
-                load_b2<false>(bfr, wb, 128, 16 * kt, 16 * np, lane);  // W^T stored [c][t] = [n][k]
-                mma_bf16(dS[2 * np], aZ, bfr[0], bfr[1]);
-                mma_bf16(dS[2 * np + 1], aZ, bfr[2], bfr[3]);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ts(tmem + TM_S, tmem + TM_ZB + 8 * ks, sdesc_sw128(wb + ks * 32, 16, 1024), IDESC_S, 1);
+            mma_commit(&bar_s);
         }
-        __syncthreads();  // every warp is done with this buffer before it is refilled
+        if (!mbar_wait(&bar_s, ph)) atomicExch(a.status, kStatusTimeout);
+        tc_fence_after();
     }
     // dS0 = dS (stored [c][j])
+    {
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t r[32];
+            tmem_ld32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
+            tmem_wait_ld();
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = j0 + g + 8 * (e >> 1), c = 8 * nt + 2 * t4 + (e & 1);
-            if (c < a.din && j < a.din) a.dS0[((size_t)bh * a.din + c) * a.din + j] = dS[nt][e];
+            for (int u = 0; u < 32; ++u) {
+                const int c = 64 * half + 32 * h2 + u;
+                if (c < a.din && row < a.din) a.dS0[((size_t)bh * a.din + c) * a.din + row] = __uint_as_float(r[u]);
+            }
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
 }
 
 // ================================================================== 4. gradients on the tensor cores
@@ -801,7 +847,6 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     const int next = find_task(task + gridDim.x, nx);
     const int ci = cr.ci, hh = cr.h, bb = cr.sp.bos;  // bb: the sequence's first token row
     const int L = min(C, cr.sp.len - ci * C);
-    const size_t cidx = cr.cidx;
     const size_t slot = bound_slot(a.pr, cr.n, hh, cr.nch, ci);
     const int y = bb + ci * C;
     const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
@@ -1250,8 +1295,17 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         bwd_prep_tc_kernel<<<nblk, prep_tc::kThreads, prep_tc::SMEM, s>>>(maps, a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_kernel), (int)CH_SMEM)) != cudaSuccess) return e;
-    bwd_chain_kernel<<<p.B * p.H * kChainSplit, kChainThreads, CH_SMEM, s>>>(a);
+    {  // the dS chain on the tensor cores: one block per (batch, head)
+        ChainMaps cm;
+        memset(&cm, 0, sizeof(cm));
+        const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p);
+        if (!make_map_2d(&cm.kh, a.Kh, D, nchunk * C, 64, C) || !make_map_2d(&cm.wt, a.W, C, nchunk * D, 64, D) ||
+            !make_map_2d(&cm.rt, a.Rt, D, nchunk * D, 64, D))
+            return cudaErrorInvalidValue;
+        if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_tc_kernel), (int)chain_tc::SMEM)) != cudaSuccess)
+            return e;
+        bwd_chain_tc_kernel<<<p.B * p.H, chain_tc::kThreads, chain_tc::SMEM, s>>>(cm, a);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {  // gradients on the tensor cores: one block per (chunk, head)
         GradMaps maps;
