@@ -39,6 +39,19 @@ def test_bwd_small(cuda_lib, dtype, D, T):
         assert_close(out[gk], r[rk], dtype, gk)
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_bwd_several_chunks_per_block(cuda_lib, D):
+    """B=3, T=2000 (31 full chunks and a ragged one of 16 tokens), H=4: 384 chunk tasks, so
+    every block of the persistent gradient kernel runs two or three of them, full and ragged
+    ones mixed, and the chain runs 32 chunks through its three-stage ring; dS_T is nonzero."""
+    x = make_inputs(3, 2000, 4, D, D, dtype="bf16", seed=401 + D, with_do=True)
+    dST = torch.randn(3, 4, D, D, generator=torch.Generator().manual_seed(11))
+    out = run_bwd(cuda_lib, x, dST)
+    r = ref_bwd(x, dST)
+    for gk, rk in GRADS:
+        assert_close(out[gk], r[rk], "bf16", gk)
+
+
 def test_bwd_tiny_f32_workload_no_state_grad(cuda_lib):
     x = make_inputs(**WORKLOADS["tiny_f32"], seed=0, with_do=True)
     out = run_bwd(cuda_lib, x)
