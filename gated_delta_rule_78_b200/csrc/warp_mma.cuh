@@ -1,15 +1,7 @@
-// Warp-level tensor-core building blocks shared by the forward and backward
-// kernels:
-//  * the 64 x 64 unit lower-triangular inverse T = (I + A)^-1 that every chunk
-//    needs (closed-form 4x4 blocks, in-warp doubling to 16x16, then two
-//    doubling levels on TF32 warp MMAs);
-//  * bf16 m16n8k16 warp MMAs fed by ldmatrix from XOR-swizzled shared tiles.
-//
-// Swizzled bf16 tile convention ("swz"): a row-major tile whose rows are 128 or
-// 256 bytes long; the 16-byte chunk j of row r is stored at chunk position
-// j ^ (r & 7) of that row.  Eight consecutive rows read at the same logical
-// chunk therefore hit eight different 16-byte bank groups, which makes every
-// ldmatrix below conflict-free without padding.
+// Warp-level tensor-core building block shared by the forward and the backward prep
+// kernels: the 64 x 64 unit lower-triangular inverse T = (I + A)^-1 that every chunk
+// needs (closed-form 4x4 blocks, in-warp doubling to 16x16, then two doubling levels
+// on TF32 warp MMAs).
 #pragma once
 
 #include <stdint.h>
@@ -153,112 +145,6 @@ __device__ __forceinline__ void solve_unit_lower64(const float *sA, float *sT, i
         tile_store<LD>(sT + (32 + 16 * mt) * LD + n0 + 8, x1, -1.f, lane);
     }
     sync();
-}
-
-// ------------------------------------------------------------------ bf16 warp MMA from swizzled tiles
-// byte offset of bf16 element (row, col) in a swizzled tile with `rowbytes`-byte rows
-__host__ __device__ __forceinline__ uint32_t swz(int row, int col, int rowbytes)
-{
-    const uint32_t byte = static_cast<uint32_t>(col) * 2u;
-    return static_cast<uint32_t>(row) * rowbytes + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15u));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-// d (16x8 fp32) += a (16x16 bf16, row) * b (16x8 bf16, col).  Fragments (g = lane/4,
-// t = lane%4): a = {A[g][2t..], A[g+8][2t..], A[g][2t+8..], A[g+8][2t+8..]},
-// b = {B[2t..][g], B[2t+8..][g]}, d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// A fragment (16 x 16 at (m0, k0)) of op(A).  KM = false: A is stored [m][k];
-// KM = true: the storage holds A^T ([k][m]) and the load transposes.
-template <bool KM>
-__device__ __forceinline__ void load_a(uint32_t (&a)[4], uint32_t base, int rowbytes, int m0, int k0, int lane)
-{
-    const int mat = lane >> 3, r = lane & 7;
-    if (!KM) {
-        ldsm_x4(a, base + swz(m0 + r + 8 * (mat & 1), k0 + 8 * (mat >> 1), rowbytes));
-    } else {
-        ldsm_x4_t(a, base + swz(k0 + r + 8 * (mat >> 1), m0 + 8 * (mat & 1), rowbytes));
-    }
-}
-
-// B fragments of two adjacent 8-column tiles (16 x 16 at (k0, n0)) of op(B):
-// b[0], b[1] for columns n0..n0+7 and b[2], b[3] for n0+8..n0+15.  KN = false: B is
-// stored transposed ([n][k]); KN = true: stored [k][n] and the load transposes.
-template <bool KN>
-__device__ __forceinline__ void load_b2(uint32_t (&b)[4], uint32_t base, int rowbytes, int k0, int n0, int lane)
-{
-    const int mat = lane >> 3, r = lane & 7;
-    if (!KN) {
-        ldsm_x4(b, base + swz(n0 + r + 8 * (mat >> 1), k0 + 8 * (mat & 1), rowbytes));
-    } else {
-        ldsm_x4_t(b, base + swz(k0 + r + 8 * (mat & 1), n0 + 8 * (mat >> 1), rowbytes));
-    }
-}
-
-// acc[MT][NT] (a (16 MT) x (8 NT) tile at (m0, n0)) += op(A)[m0.., 0:K] op(B)[0:K, n0..]
-// (K fixed at compile time so that the fragment loads of later k-steps are issued early)
-template <int MT, int NT, bool A_KM, bool B_KN, int K>
-__device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], uint32_t a_base, int a_rb, int m0,
-                                          uint32_t b_base, int b_rb, int n0, int lane)
-{
-    static_assert(NT % 2 == 0, "B fragments come in pairs of 8-column tiles");
-#pragma unroll
-    for (int k0 = 0; k0 < K; k0 += 16) {
-        uint32_t a[MT][4];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) load_a<A_KM>(a[mt], a_base, a_rb, m0 + 16 * mt, k0, lane);
-#pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-            uint32_t b[4];
-            load_b2<B_KN>(b, b_base, b_rb, k0, n0 + 16 * np, lane);
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                mma_bf16(acc[mt][2 * np], a[mt], b[0], b[1]);
-                mma_bf16(acc[mt][2 * np + 1], a[mt], b[2], b[3]);
-            }
-        }
-    }
-}
-
-// The accumulator of two adjacent 8-column tiles, rounded to bf16, is the A fragment
-// of the 16-wide k slice they cover (row-major op(A)).
-__device__ __forceinline__ void acc_to_a(uint32_t (&a)[4], const float (&c0)[4], const float (&c1)[4], float s)
-{
-    a[0] = tc::pack_bf16x2(s * c0[0], s * c0[1]);
-    a[1] = tc::pack_bf16x2(s * c0[2], s * c0[3]);
-    a[2] = tc::pack_bf16x2(s * c1[0], s * c1[1]);
-    a[3] = tc::pack_bf16x2(s * c1[2], s * c1[3]);
-}
-
-template <int MT, int NT>
-__device__ __forceinline__ void zero_acc(float (&acc)[MT][NT][4])
-{
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 }
 
 }  // namespace wm
