@@ -698,9 +698,10 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
 }
 
 // ================================================================== 4. gradients on the tensor cores
-// One 512-thread CTA per (chunk, head).  Every product runs transposed, so that its M side is a
-// 128-wide feature dimension (d_v or d_k, or the two stacked 64-token tiles of [dP; dA]) and its
-// TMEM accumulator holds one feature row per lane (Gm = Diag(gamma)):
+// Persistent: one 512-thread CTA per multiprocessor loops over the (chunk, head) tasks, loading
+// the next task's tiles as this task's regions free up.  Every product runs transposed, so that
+// its M side is a 128-wide feature dimension (d_v or d_k, or the two stacked 64-token tiles of
+// [dP; dA]) and its TMEM accumulator holds one feature row per lane (Gm = Diag(gamma)):
 //   Y^T  = X^T - S^T E~^T              M d_v, N 64, K d_k           -> bf16 A operand in TMEM
 //   dU~^T = dO^T P + (Gm dS_n)^T K~^T  M d_v, N 64, K 64 + d_k      -> bf16 A operand in TMEM
 //   U~^T = Y^T T^T                     A from TMEM, K 64            -> U~ tile [s][d_v]
@@ -728,8 +729,8 @@ constexpr uint32_t WW = 212992;   // w, then dv
 constexpr uint32_t DGF = 229376;  // gamma dgamma [D] fp32
 constexpr uint32_t USED = DGF + D * 4;
 constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
-// scratch inside the -dY rows (free until dY is read back), and inside DY once every product
-// is done (the factor chain)
+// scratch inside the -dY rows (free until dY is read back), and in DS's second half (free once
+// (Gm dS_n)^T's products are done) for the factor chain
 constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
 constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
