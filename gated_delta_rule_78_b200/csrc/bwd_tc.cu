@@ -31,6 +31,7 @@
 //      and produces every gradient of the chunk.
 // Every product is a bf16 tcgen05 MMA with an fp32 TMEM accumulator, its operands
 // in 128-byte swizzled shared-memory tiles (most of them loaded by TMA) or in TMEM.
+#include <climits>
 #include <cuda.h>
 #include <string.h>
 
@@ -1240,6 +1241,11 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
                           int *status, cudaStream_t s, bool states_saved)
 {
     if (p.D != 128 && p.D != 64) return cudaErrorNotSupported;
+    {  // TMA row coordinates are 32-bit: the state rows (slot x 128) and the token rows
+        const uint64_t state_rows = (uint64_t)p.H * (chunk_bound(p) + p.B) * D;
+        if (state_rows > (uint64_t)INT_MAX || (uint64_t)token_rows(p) > (uint64_t)INT_MAX)
+            return cudaErrorInvalidValue;
+    }
     const BwdTcLayout l = tc_layout(p);
     char *base = static_cast<char *>(ws);
     BwdTcArgs a;
