@@ -98,19 +98,31 @@ def fwd_flops(B, T, H, D, C=CHUNK):
     return B * T * H * (10 * C * D + 6 * D * D)
 
 
+def device_code_sha(text: str, kernel_def: str):
+    """SHA-256 of a kernel source file's text up to the closing brace of the kernel's
+    definition: the device code the kernel is built from (constants, helpers and the kernel
+    itself), without the host code after it."""
+    i = text.index(kernel_def)
+    j = text.index("\n}\n", i) + 3
+    return hashlib.sha256(text[:j].encode()).hexdigest()
+
+
 def kernel_traffic(kernel_src: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current source of the kernel (same SHA-256), else None."""
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the kernel's
+    current device code (same SHA-256 of the file up to the kernel's end), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     src = os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", kernel_src)
-    if not os.path.exists(src):
-        return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
     e = d.get(kernel_src)
-    if not e or e.get("sha256") != h:
+    if not e or not os.path.exists(src):
+        return None
+    try:
+        h = device_code_sha(open(src).read(), e["kernel_def"])
+    except (KeyError, ValueError):
+        return None
+    if e.get("sha256_device") != h:
         return None
     return e.get("bytes_per_launch")
 
