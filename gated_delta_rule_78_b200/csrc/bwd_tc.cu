@@ -182,6 +182,19 @@ __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8
     total = make_float2(tot0, tot1);
 }
 
+// Bounded wait on an mbarrier phase.  A wait that gives up records the timeout in the status
+// word and in the block's abort flag; once that is set every later wait of the block returns at
+// once, so a block that lost a transfer ends (with garbage) after one wait limit instead of one
+// limit per remaining wait.
+__device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, int *status, volatile int *abort)
+{
+    if (*abort) return;
+    if (!tc::mbar_wait(bar, parity)) {
+        *abort = 1;
+        atomicExch(status, kStatusTimeout);
+    }
+}
+
 // ================================================================== 2. prep on the tensor cores
 // One 512-thread CTA per (chunk, head): the raw q, b, k, dO tiles arrive by TMA (SW128 atoms),
 // the decay folds into them in place, and the four products run as tcgen05 MMAs with TMEM
@@ -234,6 +247,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t bar_in, bar_ap, bar_z, bar_w, bar_r;
     __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     ChunkRef cr;
     if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
@@ -251,6 +265,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         mbar_init(&bar_z, 1);
         mbar_init(&bar_w, 1);
         mbar_init(&bar_r, 1);
+        s_abort = 0;
         fence_mbar_init();
         prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b); prefetch_tmap(&maps.dO);
         prefetch_tmap(&maps.g);
@@ -296,7 +311,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
             gv[i] = make_float2(__expf(gv[i].x), __expf(gv[i].y));  // alpha
         }
         *reinterpret_cast<float2 *>(sTot + tg * D + ch) = make_float2(run0, run1);
-        if (!mbar_wait(&bar_in, 0)) atomicExch(a.status, kStatusTimeout);
+        wait_or_abort(&bar_in, 0, a.status, &s_abort);
         __syncthreads();
         float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
@@ -349,7 +364,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
                    sdesc_sw128(sb + KT + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_AP, ks > 0);
         mma_commit(&bar_ap);
     }
-    if (!mbar_wait(&bar_ap, 0)) atomicExch(a.status, kStatusTimeout);
+    wait_or_abort(&bar_ap, 0, a.status, &s_abort);
     tc_fence_after();
     if (warp < 8) {  // A -> fp32 scratch (strictly lower), P -> bf16 tile (lower incl.)
         const int quarter = warp & 3, half = warp >> 2;
@@ -428,7 +443,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         mma_commit(&bar_w);
     }
     // -Z^T -> bf16 A operand (warps 0-3: lanes d_v, 64 columns)
-    if (!mbar_wait(&bar_z, 0)) atomicExch(a.status, kStatusTimeout);
+    wait_or_abort(&bar_z, 0, a.status, &s_abort);
     tc_fence_after();
     if (warp < 4) {
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
@@ -444,7 +459,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         tmem_wait_st();
     }
     // W^T -> bf16 tile (rows d_k, the B operand of R^T) and global (warps 4-7)
-    if (!mbar_wait(&bar_w, 0)) atomicExch(a.status, kStatusTimeout);
+    wait_or_abort(&bar_w, 0, a.status, &s_abort);
     tc_fence_after();
     if (warp >= 4 && warp < 8) {
         const int quarter = warp & 3, c = quarter * 32 + lane;
@@ -481,7 +496,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
             mma_ts(tmem + TM_RT, tmem + TM_ZB + 8 * ks, sdesc_sw128(sb + WT + ks * 32, 16, 1024), IDESC_R2, 1);
         mma_commit(&bar_r);
     }
-    if (!mbar_wait(&bar_r, 0)) atomicExch(a.status, kStatusTimeout);
+    wait_or_abort(&bar_r, 0, a.status, &s_abort);
     tc_fence_after();
 #pragma unroll
     for (int cq2 = 0; cq2 < 2; ++cq2) {  // R^T -> bf16, global [d_v][d_k]: warp = lane quarter x 2 column blocks
@@ -543,6 +558,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t bar_full[kStages], bar_z, bar_s;
     __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, n = bh / a.H, hh = bh % a.H;
     const SeqSpan sp = seq_span(a.pr, n);
@@ -556,6 +572,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
         for (int s = 0; s < kStages; ++s) mbar_init(&bar_full[s], 1);
         mbar_init(&bar_z, 1);
         mbar_init(&bar_s, 1);
+        s_abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -605,7 +622,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         const uint8_t *st = sm + s * STAGE;
         if (tid == 0 && ci - 2 >= 0) load(ci - 2, (it + 2) % kStages);  // stage freed by step it - 1
-        if (!mbar_wait(&bar_full[s], par)) atomicExch(a.status, kStatusTimeout);
+        wait_or_abort(&bar_full[s], par, a.status, &s_abort);
         // ---- dS_n^T: bf16 to global and to TMEM; dS_n^T Diag(gamma) + R^T back into the accumulator
         {
             const float *gam = reinterpret_cast<const float *>(st + ST_G) + 64 * half;
@@ -651,7 +668,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                        IDESC_Z, ks > 0);
             mma_commit(&bar_z);
         }
-        if (!mbar_wait(&bar_z, ph)) atomicExch(a.status, kStatusTimeout);
+        wait_or_abort(&bar_z, ph, a.status, &s_abort);
         tc_fence_after();
         {  // -Z^T -> bf16 A operand: warp = lane quarter x 32 columns
             uint32_t r[32], pk[16];
@@ -673,7 +690,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                 mma_ts(tmem + TM_S, tmem + TM_ZB + 8 * ks, sdesc_sw128(wb + ks * 32, 16, 1024), IDESC_S, 1);
             mma_commit(&bar_s);
         }
-        if (!mbar_wait(&bar_s, ph)) atomicExch(a.status, kStatusTimeout);
+        wait_or_abort(&bar_s, ph, a.status, &s_abort);
         tc_fence_after();
     }
     // dS0 = dS (stored [c][j])
@@ -753,10 +770,6 @@ struct GradMaps {
     CUtensorMap dq, dk, db, dv, dw, dg;                 // stores of full chunks
 };
 
-__device__ __forceinline__ void wait_or_flag(uint64_t *bar, uint32_t parity, int *status)
-{
-    if (!tc::mbar_wait(bar, parity)) atomicExch(status, kStatusTimeout);
-}
 
 // bf16 element (t, c) of a [rows][128] tile whose two column atoms are `astride` bytes apart
 __device__ __forceinline__ uint32_t tile_off(int t, int c, uint32_t astride)
@@ -775,6 +788,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(8) uint64_t bar_in0, bar_in1, bar_in2, bar_a, bar_b, bar_c, bar_d;
     __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = smem_u32(sm);
     // TMEM access: warp w reads lanes 32 (w & 3) .. + 31; column block w >> 2 (16 columns)
@@ -796,6 +810,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         mbar_init(&bar_b, 1);
         mbar_init(&bar_c, 1);
         mbar_init(&bar_d, 1);
+        s_abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -866,7 +881,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     const int cp = tid & 63, g8 = tid >> 6;
     float *sTot = reinterpret_cast<float *>(sm + SC_TOT);
     float *sGam = reinterpret_cast<float *>(sm + SC_GAM);
-    wait_or_flag(&bar_in0, ph, a.status);
+    wait_or_abort(&bar_in0, ph, a.status, &s_abort);
     {
         const bool ch_ok = 2 * cp < a.din;
         float2 gl[8], eG[8], emG[8], tot;
@@ -898,7 +913,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     __syncthreads();
     tc_fence_after();
     // ---- Y^T = S^T E~^T (into TM_Y; X is added at the read-back)
-    wait_or_flag(&bar_in1, ph, a.status);
+    wait_or_abort(&bar_in1, ph, a.status, &s_abort);
     if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -965,7 +980,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         mma_commit(&bar_a);
     }
     // ---- read back: Y^T = X^T - acc and dU~^T, as bf16 A operands (lane = d_v, 16 tokens per warp)
-    wait_or_flag(&bar_a, ph, a.status);
+    wait_or_abort(&bar_a, ph, a.status, &s_abort);
     tc_fence_after();
     {
         uint32_t r[16], pk[8];
@@ -1004,7 +1019,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             mma_ts(tmem + TM_DY, tmem + TM_DUB + 8 * ks, sdesc_sw128(sb + TT + ks * 2048, 8192, 1024), IDESC_KM, ks > 0);
         mma_commit(&bar_b);
     }
-    wait_or_flag(&bar_b, ph, a.status);
+    wait_or_abort(&bar_b, ph, a.status, &s_abort);
     tc_fence_after();
     // ---- read back: U~ tile [s][d_v] (over T and P, both consumed); dv = dY w, dw = dY v (full
     //      chunks: over w and v); -dY into rows 64-127 of [dO; -dY]
@@ -1061,7 +1076,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         }
         bulk_commit();
     }
-    wait_or_flag(&bar_c, ph, a.status);
+    wait_or_abort(&bar_c, ph, a.status, &s_abort);
     tc_fence_after();
     if (tid == 0) {  // S^T and (Gm dS_n)^T are consumed: the raw q, k, b for the factor chain
         mbar_expect_tx(&bar_in2, 6 * 8192);
@@ -1120,7 +1135,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             run += gv;
             al[i] = __expf(gv);
         }
-        wait_or_flag(&bar_d, ph, a.status);
+        wait_or_abort(&bar_d, ph, a.status, &s_abort);
         tc_fence_after();
         if (warp == 0 && next >= 0) issue(0, nx);  // Q~, K~, E~, [dO; -dY], T, P are consumed
         sFin[cg * D + row] = run;
@@ -1145,7 +1160,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         tmem_ld16(tmem + TM_DQE + 64 + 16 * cg + lane_off, re);
         tmem_ld16(tmem + TM_DK + 16 * cg + lane_off, rk);
         tmem_wait_ld();
-        wait_or_flag(&bar_in2, ph, a.status);
+        wait_or_abort(&bar_in2, ph, a.status, &s_abort);
         float e = __expf(off);
         float dG[16];
         const size_t base = tok_off(a, bb, hh, ci, 16 * cg) + row, stride = (size_t)a.H * a.din;
