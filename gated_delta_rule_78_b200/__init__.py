@@ -26,5 +26,5 @@ from ._lib import (EXPORTS, GDN2_BF16, GDN2_F32, GDN2_OK, LIB_PATH, NOALLOC_MAX_
                    STATUS_NAMES, Gdn2Error, gdn2_chunk_bwd, gdn2_chunk_bwd_noalloc, gdn2_chunk_bwd_varlen,
                    gdn2_chunk_fwd, gdn2_chunk_fwd_varlen, gdn2_chunk_fwd_gated, gdn2_chunk_bwd_gated,
                    gdn2_decode_step_gated, gdn2_workspace_size_gated, DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR,
-                   DECAY_NONE, ERASE_NONE, WRITE_NONE, QK_L2NORM, BW_LOGITS, gdn2_decode_step, gdn2_prologue, gdn2_chunk_fwd_save, gdn2_chunk_bwd_saved, gdn2_chunk_fwd_host, gdn2_strerror, gdn2_sync_status,
+                   DECAY_NONE, ERASE_NONE, WRITE_NONE, QK_L2NORM, BW_LOGITS, gdn2_decode_step, gdn2_prologue, gdn2_chunk_fwd_save, gdn2_chunk_bwd_saved, gdn2_chunk_fwd_host, gdn2_strerror, gdn2_sync_status, gdn2_selftest_timeout,
                    gdn2_workspace_size, load, raw)

@@ -25,7 +25,7 @@ EXPORTS = ("gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_bwd", "gdn2_workspa
            "gdn2_strerror", "gdn2_sync_status", "gdn2_chunk_bwd_noalloc", "gdn2_chunk_fwd_varlen",
            "gdn2_chunk_bwd_varlen", "gdn2_chunk_fwd_gated", "gdn2_chunk_bwd_gated", "gdn2_decode_step_gated",
            "gdn2_workspace_size_gated", "gdn2_prologue", "gdn2_chunk_fwd_save", "gdn2_chunk_bwd_saved",
-           "gdn2_chunk_fwd_host")
+           "gdn2_chunk_fwd_host", "gdn2_selftest_timeout")
 # gate layout flags (gdn2_gate_flags in include/gdn2.h)
 DECAY_SCALAR, ERASE_SCALAR, WRITE_SCALAR, DECAY_NONE, ERASE_NONE, WRITE_NONE = 1, 2, 4, 8, 16, 32
 # input prologue: q, k L2-normalised in the call; b, w given as logits (sigmoid in the call)
@@ -88,6 +88,8 @@ def load(path: str | None = None):
     lib.gdn2_strerror.restype = ctypes.c_char_p
     lib.gdn2_sync_status.argtypes = [vp]
     lib.gdn2_sync_status.restype = i
+    lib.gdn2_selftest_timeout.argtypes = [i, vp]
+    lib.gdn2_selftest_timeout.restype = i
     _lib = lib
     return lib
 
@@ -460,6 +462,12 @@ def gdn2_prologue(q, k, b, w, *, flags, out=None, stream=None):
 def gdn2_sync_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the kernel status word."""
     return int(raw().gdn2_sync_status(_stream(stream)))
+
+
+def gdn2_selftest_timeout(limit_us: int = 2000, stream=None):
+    """Failure-detection self-test: enqueue one bounded wait on a barrier phase nothing
+    completes; the next gdn2_sync_status() returns GDN2_ERR_TIMEOUT (-7)."""
+    _check("gdn2_selftest_timeout", raw().gdn2_selftest_timeout(int(limit_us), _stream(stream)))
 
 
 def gdn2_strerror(status: int) -> str:

@@ -598,6 +598,14 @@ gdn2_status gdn2_chunk_fwd_host(gdn2_dtype dt, int B, int T, int H, int Dk, int 
                                            (cudaStream_t)stream, run_fwd_slice));
 }
 
+gdn2_status gdn2_selftest_timeout(int limit_us, void *stream)
+{
+    if (limit_us < 1 || limit_us > 100000) return GDN2_ERR_SHAPE;
+    int *status = gdn2::status_word();
+    if (!status) return GDN2_ERR_CUDA;
+    return from_cuda(gdn2::launch_selftest_timeout(limit_us, status, (cudaStream_t)stream));
+}
+
 gdn2_status gdn2_sync_status(void *stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -190,5 +190,7 @@ cudaError_t launch_channel_sum(bool fp32, const void *src, void *dst, size_t n_r
 
 // device address of the library's kernel status word on the current device
 int *status_word();
+// Failure-detection self-test (selftest.cu): one bounded wait on a phase nothing completes.
+cudaError_t launch_selftest_timeout(int limit_us, int *status, cudaStream_t s);
 
 }  // namespace gdn2

@@ -312,6 +312,14 @@ GDN2_API const char *gdn2_strerror(gdn2_status status);
  * GDN2_ERR_CUDA if the stream reported an error, else GDN2_OK. */
 GDN2_API gdn2_status gdn2_sync_status(void *stream);
 
+/* Failure-detection self-test.  Enqueues one block whose thread waits on an mbarrier phase
+ * that nothing completes, bounded by `limit_us` microseconds: the same bounded wait every
+ * tensor-core kernel uses.  When the wait gives up, the kernel records a timeout in the status
+ * word, as a kernel that lost a transfer would, and returns.  The next gdn2_sync_status()
+ * reports GDN2_ERR_TIMEOUT (and clears it); the context stays usable.  Asynchronous on
+ * `stream`.  GDN2_ERR_SHAPE for limit_us outside 1 .. 100000 (nothing is launched). */
+GDN2_API gdn2_status gdn2_selftest_timeout(int limit_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

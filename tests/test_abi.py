@@ -223,3 +223,10 @@ def test_host_forward_arguments(lib):
     slot = 6 * tok * 2 + tok * 4 + 2 * H * D * D * 4
     assert lib.gdn2_workspace_size(4, BF16, B, T, H, D, D) == 3 * slot
     assert lib.gdn2_workspace_size(4, BF16, B, 0, H, D, D) == 0
+
+
+def test_selftest_timeout_arguments(lib):
+    """The failure-detection self-test validates its limit before it launches anything."""
+    assert lib.gdn2_selftest_timeout(0, S) == -2
+    assert lib.gdn2_selftest_timeout(-5, S) == -2
+    assert lib.gdn2_selftest_timeout(100001, S) == -2
