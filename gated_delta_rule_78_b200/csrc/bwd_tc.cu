@@ -31,12 +31,14 @@
 //      and produces every gradient of the chunk.
 // Every product is a bf16 tcgen05 MMA with an fp32 TMEM accumulator, its operands
 // in 128-byte swizzled shared-memory tiles (most of them loaded by TMA) or in TMEM.
+#include <algorithm>
 #include <climits>
 #include <cuda.h>
 #include <string.h>
 
 #include "gdn2_internal.cuh"
 #include "tc_util.cuh"
+#include "tok_util.cuh"
 #include "warp_mma.cuh"
 
 namespace gdn2 {
@@ -48,15 +50,22 @@ using namespace wm;
 constexpr int D = 128;
 constexpr int C = 64;
 constexpr int LDA = 68;  // fp32 row stride of the A / T scratch of the solve
+constexpr int GSTR = D + 4;  // per-chunk record of gamma: D floats, then the token-mode flag (int)
 
 // ------------------------------------------------------------------ workspace
 struct BwdTcLayout {
-    size_t coff, states, W, Kh, gam, Rt, Tm, Pm, dSn, total;
+    size_t coff, states, flist, W, Kh, gam, Rt, Tm, Pm, dSn, scratch, total;
+    int tok_blocks;  // blocks of the token-level gradient kernel
 };
 
+__host__ __device__ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
 // Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W^T bf16 [D][C],
-// K^ bf16 [C][D], gamma fp32 [D], R^T bf16 [D][D], T and P bf16 [C][C], dS_n^T bf16 [D][D].
-// Variable length puts chunk_off first; chunk lists are sized by the chunk bound.
+// K^ bf16 [C][D], gamma and the chunk's token-mode flag [GSTR] fp32, R^T bf16 [D][D], T and P
+// bf16 [C][C], dS_n^T bf16 [D][D].  flist: the count and the list of the chunk tasks that run
+// token by token.  Variable length puts chunk_off first; chunk lists are sized by the chunk
+// bound.  The token-level gradient kernel's scratch reuses W .. R^T, which only the chain reads
+// (one block's scratch at least; past the end of the workspace when that region is smaller).
 BwdTcLayout tc_layout(const Problem &p)
 {
     const size_t H = p.H, nchunk = chunk_bound(p), nbound = nchunk + p.B;
@@ -64,13 +73,24 @@ BwdTcLayout tc_layout(const Problem &p)
     size_t off = p.cu_seqlens ? varlen_offsets_bytes(p.B) : 0;
     l.coff = 0;
     l.states = off; off += H * nbound * D * D * 2;
+    l.flist = off;  off += round256((1 + H * nchunk) * 4);
     l.W = off;      off += H * nchunk * C * D * 2;
     l.Kh = off;     off += H * nchunk * C * D * 2;
-    l.gam = off;    off += H * nchunk * D * 4;
+    l.gam = off;    off += round256(H * nchunk * GSTR * 4);
     l.Rt = off;     off += H * nchunk * D * D * 2;
     l.Tm = off;     off += H * nchunk * C * C * 2;
     l.Pm = off;     off += H * nchunk * C * C * 2;
     l.dSn = off;    off += H * nchunk * D * D * 2;
+    const size_t blk = tok_grad_block_bytes(p.D), reuse = l.Tm - l.W;
+    const size_t fit = blk ? reuse / blk : 0;
+    if (fit >= 1) {
+        l.tok_blocks = (int)std::min<size_t>(fit, 148);
+        l.scratch = l.W;
+    } else {
+        l.tok_blocks = 1;
+        l.scratch = off;
+        off += blk;
+    }
     l.total = off;
     return l;
 }
@@ -83,7 +103,8 @@ struct BwdTcArgs {
     const float *g;
     const float *dS_T;  // may be null
     __nv_bfloat16 *states, *W, *Kh, *Tm, *Pm, *dSn;
-    float *gam;
+    float *gam;          // [chunk][GSTR]: gamma, then the chunk's token-mode flag
+    int *flist;          // flist[0]: count of the chunks that run token by token, then their tasks
     __nv_bfloat16 *Rt;  // R^T per chunk, bf16
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
@@ -101,38 +122,10 @@ __device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bos, int hh, i
 }
 
 // The chunk a block of the chunk-parallel kernels works on: blockIdx.y is the head,
-// blockIdx.x the chunk over all sequences (fixed length: sequence-major; variable
-// length: found in chunk_off; blocks past the last chunk have nothing to do).
-struct ChunkRef {
-    int n, h, ci, nch;
-    SeqSpan sp;
-    size_t cidx;  // per-chunk workspace slot
-};
+// blockIdx.x the chunk over all sequences (blocks past the last chunk have nothing to do).
 __device__ __forceinline__ bool chunk_ref_at(const BwdTcArgs &a, int gc, int h, ChunkRef &r)
 {
-    const Problem &p = a.pr;
-    r.h = h;
-    if (!p.cu_seqlens) {
-        const int nc = seq_chunks(p.T);
-        r.n = gc / nc;
-        r.ci = gc % nc;
-    } else {
-        if (gc >= p.chunk_off[p.B]) return false;
-        int lo = 0, hi = p.B;  // last n with chunk_off[n] <= gc
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (p.chunk_off[mid] <= gc) lo = mid;
-            else hi = mid;
-        }
-        r.n = lo;
-        r.ci = gc - p.chunk_off[lo];
-    }
-    r.sp = seq_span(p, r.n);
-    if (r.sp.len < 0) return false;
-    r.nch = seq_chunks(r.sp.len);
-    if (r.ci >= r.nch) return false;
-    r.cidx = chunk_slot(p, r.n, r.h, r.nch, r.ci);
-    return true;
+    return chunk_at(a.pr, gc, h, r);
 }
 __device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
 {
@@ -312,7 +305,14 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         }
         *reinterpret_cast<float2 *>(sTot + tg * D + ch) = make_float2(run0, run1);
         wait_or_abort(&bar_in, 0, a.status, &s_abort);
-        __syncthreads();
+        // a 16-token group whose log-decay falls below -kGroupDecayLimit on some channel takes
+        // e^{-G} out of range: the chain then steps this chunk token by token, and the
+        // token-level kernel rewrites its gradients
+        const int tokm = __syncthreads_or(run0 < -kGroupDecayLimit || run1 < -kGroupDecayLimit);
+        if (tid == 0) {
+            reinterpret_cast<int *>(a.gam + cidx * GSTR)[D] = tokm;
+            if (tokm) a.flist[1 + atomicAdd(a.flist, 1)] = (int)(blockIdx.x + gridDim.x * blockIdx.y);
+        }
         float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -322,7 +322,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
             tot1 += v.y;
         }
         const float gam0 = __expf(tot0), gam1 = __expf(tot1);
-        if (tg == 0) *reinterpret_cast<float2 *>(a.gam + cidx * D + ch) = make_float2(gam0, gam1);
+        if (tg == 0) *reinterpret_cast<float2 *>(a.gam + cidx * GSTR + ch) = make_float2(gam0, gam1);
         float2 mv[16];  // e^-G, backwards from the group's last token
         {
             float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
@@ -538,7 +538,7 @@ constexpr uint32_t ST_G = 65536;      // gamma [128] fp32
 constexpr uint32_t STAGE = 66560;     // 65 KiB, 1024-aligned
 constexpr int kStages = 3;
 constexpr uint32_t SMEM = kStages * STAGE + 1024;
-constexpr uint32_t STAGE_BYTES = 16384 + 16384 + 32768 + 512;
+constexpr uint32_t STAGE_BYTES = 16384 + 16384 + 32768 + GSTR * 4;
 constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_ZB = 256, TM_COLS = 512;
 constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);
@@ -593,7 +593,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
             tma_load_2d(st + ST_R + at * 16384, &maps.rt, at * 64, (int)(cidx * D), &bar_full[s]);
         }
         tma_load_2d(st + ST_W, &maps.wt, 0, (int)(cidx * D), &bar_full[s]);
-        bulk_load(st + ST_G, a.gam + cidx * D, D * 4, &bar_full[s]);
+        bulk_load(st + ST_G, a.gam + cidx * GSTR, GSTR * 4, &bar_full[s]);
     };
     if (tid == 0) {
         for (int u = 0; u < 2 && u < nc; ++u) load(nc - 1 - u, u);
@@ -616,13 +616,76 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    uint32_t ph = 0;  // phase of bar_z and bar_s (chunks stepped token by token issue no product)
     for (int it = 0; it < nc; ++it) {
         const int ci = nc - 1 - it, s = it % kStages;
-        const uint32_t par = (uint32_t)(it / kStages) & 1u, ph = (uint32_t)it & 1u;
+        const uint32_t par = (uint32_t)(it / kStages) & 1u;
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         const uint8_t *st = sm + s * STAGE;
         if (tid == 0 && ci - 2 >= 0) load(ci - 2, (it + 2) % kStages);  // stage freed by step it - 1
         wait_or_abort(&bar_full[s], par, a.status, &s_abort);
+        if (reinterpret_cast<const int *>(st + ST_G)[D]) {
+            // ---- a chunk whose decay is too strong for the factors: dS^T to registers (this
+            //      thread: row `row`, columns 64 half ..), its bf16 copy to global as dS_n, then the
+            //      reverse recurrence token by token; records and exchange buffers over this
+            //      stage's tiles, which are not needed
+            float dsr[64];
+            __nv_bfloat16 *dsn = a.dSn + cidx * D * D + (size_t)row * D + 64 * half;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t r[32];
+                tmem_ld32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) dsr[32 * h2 + u] = __uint_as_float(r[u]);
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(dsn + 32 * h2 + 8 * m) =
+                        make_uint4(pack_bf16x2(dsr[32 * h2 + 8 * m], dsr[32 * h2 + 8 * m + 1]),
+                                   pack_bf16x2(dsr[32 * h2 + 8 * m + 2], dsr[32 * h2 + 8 * m + 3]),
+                                   pack_bf16x2(dsr[32 * h2 + 8 * m + 4], dsr[32 * h2 + 8 * m + 5]),
+                                   pack_bf16x2(dsr[32 * h2 + 8 * m + 6], dsr[32 * h2 + 8 * m + 7]));
+            }
+            uint8_t *stw = sm + s * STAGE;
+            tok::Rec<D> *recs = reinterpret_cast<tok::Rec<D> *>(stw);
+            float *xch = reinterpret_cast<float *>(stw + 3 * sizeof(tok::Rec<D>));
+            const int L = min(C, sp.len - ci * C);
+            const size_t row0 = (size_t)sp.bos + (size_t)ci * C;
+            auto fill = [&](int t, tok::Rec<D> &rc) {
+                if (tid < D) {
+                    const int c = tid;
+                    float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f;
+                    if (c < a.din) {
+                        const size_t off = ((row0 + t) * a.H + hh) * a.din + c;
+                        qv = __bfloat162float(a.q[off]);
+                        kv = __bfloat162float(a.k[off]);
+                        bv = __bfloat162float(a.b[off]);
+                        gv = a.g[off];
+                    }
+                    rc.q[c] = qv;
+                    rc.k[c] = kv;
+                    rc.e[c] = bv * kv;
+                    rc.a[c] = expf(gv);
+                } else {
+                    const int jj = tid - D;
+                    rc.x[jj] = jj < a.din ? __bfloat162float(a.dO[((row0 + t) * a.H + hh) * a.din + jj]) : 0.f;
+                }
+            };
+            tok::chain_tokens<D>(dsr, L - 1, L, recs, xch, row, half, 1, fill);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t r[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(dsr[32 * h2 + u]);
+                tmem_st32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();  // the stage is refilled by TMA later
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            continue;
+        }
         // ---- dS_n^T: bf16 to global and to TMEM; dS_n^T Diag(gamma) + R^T back into the accumulator
         {
             const float *gam = reinterpret_cast<const float *>(st + ST_G) + 64 * half;
@@ -692,6 +755,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
         }
         wait_or_abort(&bar_s, ph, a.status, &s_abort);
         tc_fence_after();
+        ph ^= 1;
     }
     // dS0 = dS (stored [c][j])
     {
@@ -1285,6 +1349,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
     a.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
     a.gam = reinterpret_cast<float *>(base + l.gam);
+    a.flist = reinterpret_cast<int *>(base + l.flist);
     a.Rt = reinterpret_cast<__nv_bfloat16 *>(base + l.Rt);
     a.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
     a.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
@@ -1304,6 +1369,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         if (e != cudaSuccess) return e;
     }
     const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
+    if ((e = cudaMemsetAsync(a.flist, 0, sizeof(int), s)) != cudaSuccess) return e;  // no chunk flagged yet
     {  // prep on the tensor cores: one block per (chunk, head)
         PrepMaps maps;
         memset(&maps, 0, sizeof(maps));
@@ -1352,7 +1418,10 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         const int ntask = (int)chunk_bound(p) * p.H;
         bwd_grad_kernel<<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
     }
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the chunks that run token by token: their gradients, exact, over what the gradient kernel wrote
+    return launch_tok_grad_tc(a.pr, d_o, a.states, a.dSn, a.flist, reinterpret_cast<float *>(base + l.scratch),
+                              l.tok_blocks, out, s);
 }
 
 }  // namespace gdn2

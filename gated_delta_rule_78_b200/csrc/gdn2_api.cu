@@ -89,7 +89,7 @@ gdn2::Problem make_problem(int B, int T, int H, int D, const void *q, const void
 }
 
 // Launch the forward of a validated problem (T > 0): bf16 with D = 128 on the tensor
-// cores, everything else on the FMA kernel.  Variable length first checks cu_seqlens.
+// cores, everything else (fp32) on the token-level kernel.  Variable length first checks cu_seqlens.
 gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s);
 // the device forward of one host-pipeline slice
 cudaError_t run_fwd_slice(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, cudaStream_t s)
@@ -108,9 +108,9 @@ gdn2_status run_fwd(gdn2_dtype dt, const gdn2::Problem &p, void *o, float *S_T, 
     if (dt == GDN2_BF16) {
         cudaError_t e = gdn2::launch_fwd_tc(p, o, S_T, nullptr, status, s);
         if (e != cudaErrorNotSupported) return from_cuda(e);
-        cudaGetLastError();  // clear the sticky "not supported" code; fall through to FMA path
+        cudaGetLastError();  // clear the sticky "not supported" code; fall through to the token-level path
     }
-    return from_cuda(gdn2::launch_fwd_simt(dt, p, o, S_T, nullptr, s));
+    return from_cuda(gdn2::launch_fwd_tok(dt, p, o, S_T, nullptr, s));
 }
 
 

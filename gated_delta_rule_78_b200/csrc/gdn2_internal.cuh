@@ -88,6 +88,42 @@ __device__ __forceinline__ size_t bound_slot(const Problem &p, int n, int h, int
 {
     return (chunk_first(p, n) + n) * p.H + (size_t)h * (nch + 1) + ci;
 }
+// A chunk of the chunk-parallel kernels: (chunk gc over all sequences, head h) -> sequence n,
+// chunk ci of its nch, its span and its per-chunk workspace slot.  Fixed length: gc is
+// sequence-major; variable length: the sequence is found in chunk_off.  False for chunk indices
+// past the last chunk and for sequences with invalid cu_seqlens.
+struct ChunkRef {
+    int n, h, ci, nch;
+    SeqSpan sp;
+    size_t cidx;
+};
+__device__ __forceinline__ bool chunk_at(const Problem &p, int gc, int h, ChunkRef &r)
+{
+    r.h = h;
+    if (!p.cu_seqlens) {
+        const int nc = seq_chunks(p.T);
+        if (nc == 0) return false;
+        r.n = gc / nc;
+        r.ci = gc % nc;
+        if (r.n >= p.B) return false;
+    } else {
+        if (gc >= p.chunk_off[p.B]) return false;
+        int lo = 0, hi = p.B;  // last n with chunk_off[n] <= gc
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.chunk_off[mid] <= gc) lo = mid;
+            else hi = mid;
+        }
+        r.n = lo;
+        r.ci = gc - p.chunk_off[lo];
+    }
+    r.sp = seq_span(p, r.n);
+    if (r.sp.len < 0) return false;
+    r.nch = seq_chunks(r.sp.len);
+    if (r.ci >= r.nch) return false;
+    r.cidx = chunk_slot(p, r.n, r.h, r.nch, r.ci);
+    return true;
+}
 // offset of token row t of sequence span sp, head h, in a [rows, H, D] tensor
 __device__ __forceinline__ size_t tok_row(const Problem &p, const SeqSpan &sp, int h, int t)
 {
@@ -100,10 +136,17 @@ __device__ __forceinline__ size_t tok_row(const Problem &p, const SeqSpan &sp, i
 cudaError_t launch_chunk_offsets(const int *cu_seqlens, int n_seqs, int total_rows, int *chunk_off, int *status,
                                  cudaStream_t s);
 
-// forward (SIMT fp32 FMA path).  `states`, when non-null, receives the state at
-// the start of every chunk: [B*H][nchunks][D][D] fp32.  `o` may be null (states only).
-cudaError_t launch_fwd_simt(gdn2_dtype dt, const Problem &p, void *o, float *S_T, float *states,
-                            cudaStream_t s);
+// Chunks whose decay is too strong for the chunkwise factors.  The tensor-core kernels form
+// e^{-G} (G the cumulative log-decay inside a chunk) for the factor K~ = k e^{-G}; with every
+// 16-token group's log-decay above -kGroupDecayLimit on every channel, e^{-G} <= e^{80} and all
+// factors and products stay finite in fp32 and bf16.  Chunks past that limit run the
+// token-by-token form instead (tok_util.cuh), which is exact for any decay.
+constexpr float kGroupDecayLimit = 20.f;
+
+// The token-level forward (tok.cu): the fp32 path, any head size.  `states`, when non-null,
+// receives the fp32 state S ([c][j], d_k rows) at every chunk boundary, at the boundary slots
+// (bound_slot).  `o` may be null (states only).
+cudaError_t launch_fwd_tok(gdn2_dtype dt, const Problem &p, void *o, float *S_T, float *states, cudaStream_t s);
 
 // Raise a kernel's dynamic shared-memory limit on the current device (once per
 // kernel and device; thread-safe).
@@ -165,13 +208,23 @@ struct BwdOut {
 inline size_t varlen_offsets_bytes(int n_seqs) { return ((size_t)(n_seqs + 1) * sizeof(int) + 255) / 256 * 256; }
 
 // Backward workspace bytes (depends on the path: bf16 with D = 128 runs on the
-// tensor cores, everything else on the fp32 FMA kernels).  Only the sizes and
+// tensor cores, everything else on the token-level kernels).  Only the sizes and
 // whether cu_seqlens is set are read from p.
 size_t bwd_workspace_bytes(gdn2_dtype dt, const Problem &p);
 // states_saved: the bf16 backward's chunk-boundary states are already in ws (launch_fwd_save
 // wrote them with the same inputs), so its states pass is skipped; ignored for fp32.
 cudaError_t launch_bwd(gdn2_dtype dt, const Problem &p, const void *d_o, const float *dS_T,
                        const BwdOut &out, void *ws, cudaStream_t s, bool states_saved = false);
+
+// Token-level gradients of whole chunks (tok.cu), the exact path for chunks flagged by the
+// tensor-core backward: given each chunk's start state (the tensor-core workspace's bf16 S^T,
+// 128 x 128 per boundary slot) and its end-state gradient (bf16 dS^T, 128 x 128 per chunk slot),
+// writes dq, dk, dv, db, dw and dlog alpha of the chunk's tokens.  `list` (device): list[0]
+// chunk tasks follow, each gc + chunk_bound * h.  `scratch`: nblocks x tok_grad_block_bytes(D).
+size_t tok_grad_block_bytes(int D);
+cudaError_t launch_tok_grad_tc(const Problem &p, const void *d_o, const __nv_bfloat16 *states,
+                               const __nv_bfloat16 *dSn, const int *list, float *scratch, int nblocks,
+                               const BwdOut &out, cudaStream_t s);
 
 // tensor-core backward (bf16, D = 128): the forward in states mode, then the prep,
 // chain and gradient kernels
