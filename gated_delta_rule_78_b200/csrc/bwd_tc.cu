@@ -241,6 +241,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     __shared__ __align__(8) uint64_t bar_in, bar_ap, bar_z, bar_w, bar_r;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ int s_tok[2];  // per channel half: some channel's chunk log-decay is past kGradDecayLimit
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     ChunkRef cr;
     if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
@@ -305,14 +306,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
         }
         *reinterpret_cast<float2 *>(sTot + tg * D + ch) = make_float2(run0, run1);
         wait_or_abort(&bar_in, 0, a.status, &s_abort);
-        // a 16-token group whose log-decay falls below -kGroupDecayLimit on some channel takes
-        // e^{-G} out of range: the chain then steps this chunk token by token, and the
-        // token-level kernel rewrites its gradients
-        const int tokm = __syncthreads_or(run0 < -kGroupDecayLimit || run1 < -kGroupDecayLimit);
-        if (tid == 0) {
-            reinterpret_cast<int *>(a.gam + cidx * GSTR)[D] = tokm;
-            if (tokm) a.flist[1 + atomicAdd(a.flist, 1)] = (int)(blockIdx.x + gridDim.x * blockIdx.y);
-        }
+        __syncthreads();
         float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -322,7 +316,11 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
             tot1 += v.y;
         }
         const float gam0 = __expf(tot0), gam1 = __expf(tot1);
-        if (tg == 0) *reinterpret_cast<float2 *>(a.gam + cidx * GSTR + ch) = make_float2(gam0, gam1);
+        if (tg == 0) {  // warps 0 and 1: gamma, and whether the chunk's decay stays within kGradDecayLimit
+            *reinterpret_cast<float2 *>(a.gam + cidx * GSTR + ch) = make_float2(gam0, gam1);
+            const bool out_of_range = __any_sync(0xffffffffu, tot0 < -kGradDecayLimit || tot1 < -kGradDecayLimit);
+            if (lane == 0) s_tok[cb] = out_of_range;
+        }
         float2 mv[16];  // e^-G, backwards from the group's last token
         {
             float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
@@ -355,6 +353,12 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     }
     fence_proxy_async_smem();
     __syncthreads();
+    if (tid == 32) {  // a chunk past kGradDecayLimit: the chain steps it token by token, and the
+                      // token-level kernel rewrites its gradients
+        const int tokm = s_tok[0] | s_tok[1];
+        reinterpret_cast<int *>(a.gam + cidx * GSTR)[D] = tokm;
+        if (tokm) a.flist[1 + atomicAdd(a.flist, 1)] = (int)(blockIdx.x + gridDim.x * blockIdx.y);
+    }
     // ---- [A; P] = [E~; Q~] K~^T
     if (tid == 0) {
         tc_fence_after();

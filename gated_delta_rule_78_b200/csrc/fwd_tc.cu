@@ -98,6 +98,7 @@ static_assert(kGroup * kRegM + kGroup * kRegE == kThreads * 128, "register split
 
 struct TcParams {
     int B, T, H;
+    const __nv_bfloat16 *q, *k, *b;  // read directly by chunks that run token by token
     const float *S0;
     const float *g;   // log alpha [B,T,H,D] fp32
     __nv_bfloat16 *o;        // may be null (states-only run)
@@ -119,21 +120,6 @@ struct TcMaps {
 __device__ __forceinline__ void named_sync(int id, int count)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// barrier over `count` threads that also returns whether `pred` held on any of them
-__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
 }
 
 // bf16x2 product, rounded to nearest even
@@ -203,7 +189,9 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     __shared__ __align__(8) uint64_t bar_in[2], bar_emma, bar_mma, bar_fact[2], bar_mdone[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort_m, s_abort_e;
-    __shared__ int s_tok[2];  // E -> M with the factors: chunk of this parity runs token by token
+    // E -> M with a chunk's factors: [parity][channel half] some channel of the chunk decays past
+    // kChunkDecayLimit, so the chunk runs token by token
+    __shared__ int s_tok[2][2];
     __shared__ float *s_stp;  // this CTA's end-state destination (read once, at the end)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -371,30 +359,33 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
             // ---- factors, P and T of chunk ci are ready
             if (!mbar_wait(&bar_fact[buf], (ci >> 1) & 1)) fail();
-            if (s_tok[buf]) {
-                // ---- the chunk token by token (its decay is too strong for the factors): the raw
-                //      q, k, b tiles are untouched, X = w.v is folded; records and exchange
-                //      buffers over this parity's T / P tiles, which E left unwritten
+            if (s_tok[buf][0] | s_tok[buf][1]) {
+                // ---- the chunk token by token (its decay is too strong for the factors, whose
+                //      products E formed all the same): q, k, b from global memory (E folded the
+                //      tiles in place), X = w.v from its tile; records and exchange buffers over this
+                //      parity's T / P tiles, which M alone reads from here on
                 tok::Rec<128> *recs = reinterpret_cast<tok::Rec<128> *>(sm + ott);
                 float *xch = reinterpret_cast<float *>(sm + ott + 3 * sizeof(tok::Rec<128>));
-                const uint8_t *pqt = sm + oqe + 8192, *pbt = sm + oqe, *pkt = sm + ok, *pxt = sm + ov;
+                const uint8_t *pxt = sm + ov;
+                const __nv_bfloat16 *gq = p.q, *gk = p.k, *gb = p.b;
                 const float *rqn = sRn + (buf * 2) * 64, *rkn = sRn + (buf * 2 + 1) * 64;
                 const size_t row0 = (size_t)bos + (size_t)ci * C;
                 auto fill = [&](int t, tok::Rec<128> &r) {
                     if (tid < 128) {
                         const int c = tid;
-                        const uint32_t so = sw128(t, (c & 63) * 2);
-                        float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pqt + (c >> 6) * 16384 + so));
-                        float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pkt + (c >> 6) * 8192 + so));
-                        float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pbt + (c >> 6) * 16384 + so));
+                        float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f;
+                        if (c < DIN) {
+                            const size_t off = ((row0 + t) * p.H + hh) * DIN + c;
+                            qv = __bfloat162float(gq[off]);
+                            kv = __bfloat162float(gk[off]);
+                            bv = __bfloat162float(gb[off]);
+                            gv = kGScalar ? p.g[(row0 + t) * p.H + hh] : p.g[off];
+                        }
                         if (kPro & kProNorm) {
                             qv *= rqn[t];
                             kv *= rkn[t];
                         }
                         if (kPro & kProSigmoid) bv = 1.f / (1.f + __expf(-bv));
-                        float gv = 0.f;
-                        if (c < DIN)
-                            gv = kGScalar ? p.g[(row0 + t) * p.H + hh] : p.g[((row0 + t) * p.H + hh) * DIN + c];
                         r.q[c] = qv;
                         r.k[c] = kv;
                         r.e[c] = bv * kv;
@@ -580,7 +571,6 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             s_abort_e = 1;
             atomicExch(p.status, kStatusTimeout);
         };
-        uint32_t emma_ph = 0;  // phase of bar_emma (chunks run token by token issue no product)
         for (int ci = 0; ci < nchunks; ++ci) {
             const int buf = ci & 1;
             const int L = min(C, T - ci * C);
@@ -614,39 +604,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 gv[i] = make_float2(a0, kGScalar ? a0 : __expf(gv[i].y));  // alpha
             }
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
-            // a 16-token group whose log-decay falls below -kGroupDecayLimit on some channel would
-            // take e^{-G} out of range: the whole chunk then runs token by token in the M group
-            const bool tokm =
-                named_sync_or(2, kGroup, run0 < -kGroupDecayLimit || run1 < -kGroupDecayLimit);
+            named_sync(2, kGroup);
             if (s_abort_e) break;
-            if (tokm) {
-                if ((kPro & kProNorm) && etid < 128) {  // 1/|q|, 1/|k| of the chunk's tokens for M's records
-                    const int t = etid & 63, which = etid >> 6;  // which: 0 = q, 1 = k
-                    float n2 = 0.f;
-                    if (t < L) {
-                        for (int a = 0; a < 2; ++a) {
-                            const uint8_t *row = which ? sm + ok + a * 8192 : sm + oqe + a * 16384 + 8192;
-#pragma unroll 8
-                            for (int u = 0; u < 32; ++u) {
-                                const uint32_t w2 = *reinterpret_cast<const uint32_t *>(row + sw128(t, 4 * u));
-                                const float x0 = __uint_as_float(w2 << 16), x1 = __uint_as_float(w2 & 0xffff0000u);
-                                n2 = fmaf(x0, x0, fmaf(x1, x1, n2));
-                            }
-                        }
-                    }
-                    sRn[(buf * 2 + which) * 64 + t] = rsqrtf(n2 + kNormEps);
-                }
-                if (ew == 4 && lane == 0 && ci >= 1 && ci + 1 < nchunks) {
-                    if (!mbar_wait(&bar_mdone[buf ^ 1], ((ci - 1) >> 1) & 1)) fail();
-                    fence_proxy_async_smem();
-                    issue(ci + 1);
-                }
-                if (etid == 0) s_tok[buf] = 1;
-                named_sync(2, kGroup);
-                if (etid == 0) mbar_arrive(&bar_fact[buf]);
-                continue;
-            }
-            if (etid == 0) s_tok[buf] = 0;
             float sqq[16], sqk[16];  // prologue: this thread's share of |q|^2, |k|^2 per token
             {  // decay folding, in place
                 float c0 = 0.f, c1 = 0.f, gl0 = 0.f, gl1 = 0.f;
@@ -657,7 +616,11 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     gl0 += tv.x;
                     gl1 += tv.y;
                 }
-                if (tg == 0) *reinterpret_cast<float2 *>(sGam + buf * 128 + ch) = make_float2(__expf(gl0), __expf(gl1));
+                if (tg == 0) {  // warps 8 and 9: gamma, and whether e^{-G} stays in range on every channel
+                    *reinterpret_cast<float2 *>(sGam + buf * 128 + ch) = make_float2(__expf(gl0), __expf(gl1));
+                    const bool out_of_range = __any_sync(0xffffffffu, gl0 < -kChunkDecayLimit || gl1 < -kChunkDecayLimit);
+                    if (lane == 0) s_tok[buf][cb] = out_of_range;
+                }
                 uint8_t *pe = sm + oqe + cb * 16384;
                 uint8_t *pq = pe + 8192;
                 uint8_t *pk = sm + ok + cb * 8192;
@@ -716,8 +679,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 }
                 named_sync(2, kGroup);
             }
-            if (!mbar_wait(&bar_emma, emma_ph)) fail();
-            emma_ph ^= 1;
+            if (!mbar_wait(&bar_emma, ci & 1)) fail();
             tc_fence_after();
             {  // A -> fp32 scratch (strictly lower), P -> bf16 operand rows (lower incl.)
                 uint32_t r[32];
@@ -865,7 +827,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         (!pr.g_scalar && !make_map(&maps.g, pr.g, true, 1, rows, pr.H, din)) ||
         (o && !make_map(&maps.o, o, false, 1, rows, pr.H, din, true)))
         return cudaErrorInvalidValue;
-    TcParams prm{pr.B, pr.T, pr.H, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
+    TcParams prm{pr.B, pr.T, pr.H, (const __nv_bfloat16 *)pr.q, (const __nv_bfloat16 *)pr.k, (const __nv_bfloat16 *)pr.b,
+                 pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
                  pr.g_scalar ? 1 : 0, ScanArgs{}};
     int grid = pr.B * pr.H;
     if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)

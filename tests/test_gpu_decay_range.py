@@ -1,11 +1,13 @@
-"""Decay of any strength: the chunkwise tensor-core kernels form e^{-G} (G the cumulative
-log-decay inside a 64-token chunk), which leaves the fp32 range once G falls below about -88.
-The pages bound the decay only by alpha in (0, 1] (the aiexpert.news gate paragraph), so the
-library must stay exact past that point: chunks whose 16-token groups decay by more than
-kGroupDecayLimit (20) on some channel run the token-by-token form, and the fp32 path is
-token-level throughout.  Every case here is checked against the oracle's token recurrence,
-with the status word clear.
+"""Decay of any strength.  The chunkwise tensor-core kernels form e^{-G} (G the cumulative
+log-decay inside a 64-token chunk), which leaves the fp32 range once G falls below about -88,
+and the chunkwise backward's dlog alpha loses accuracy as the chunk's decay grows.  The pages
+bound the decay only by alpha in (0, 1] (the aiexpert.news gate paragraph), so the library must
+stay exact past those points: the forward runs chunks whose log-decay falls below -80 on some
+channel token by token, the backward does so below -16, and the fp32 path is token-level
+throughout.  Every case here is checked against the oracle's token recurrence, with the status
+word clear.
 
+* a sweep of uniform decay strengths, chunk log-decay 6 ... 96, on both sides of both limits;
 * x ~ N(+2, 1) (log alpha about -2.1 per token, about -135 per chunk): every chunk token by token;
 * one channel at log alpha = -10 per token (-640 per chunk), the others from the recipe;
 * strong decay in some chunks only, so that the two forms alternate along a sequence;
@@ -44,6 +46,16 @@ def fwd_bwd_check(x, dtype, dST=None):
     r = oracle.ref_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"], x["do"], dST)
     for gk, rk in GRADS:
         assert_close(gr[gk], r[rk], dtype, gk)
+
+
+@pytest.mark.parametrize("chunk_decay", [6, 12, 20, 40, 70, 96])
+def test_uniform_decay_sweep(cuda_lib, chunk_decay):
+    """log alpha = -(chunk_decay / 64) (0.5 + U(0, 1)) on every channel: below and above the
+    backward's limit (16) and the forward's (80)."""
+    x = make_inputs(1, 256, 2, 128, 128, dtype="bf16", seed=5, with_do=True)
+    u = torch.rand(x["log_alpha"].shape, generator=torch.Generator().manual_seed(2))
+    x["log_alpha"] = -(chunk_decay / 64.0) * (0.5 + u)
+    fwd_bwd_check(x, "bf16")
 
 
 @pytest.mark.parametrize("dtype,D", [("bf16", 128), ("bf16", 64), ("f32", 128), ("f32", 64)])
