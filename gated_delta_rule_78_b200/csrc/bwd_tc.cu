@@ -14,10 +14,14 @@
 //   dP  = lower_incl(dO U~^T)                 dA = -strictly_lower(dY U~^T)
 //   dQ~ = dO S^T + dP K~                      dE~ = -dY S^T + dA K~
 //   dK~ = dA^T E~ + dP^T Q~ + U~ (Diag(gamma) dS_n)^T
-//   gamma dgamma = rowsum(dS_n . S')          dS = gamma dS_n + Q~^T dO - E~^T dY
+//   gamma dgamma = rowsum(dS_n . S') = gamma rowsum(dS_n . S) + sum_t K~_t . (U~ (Diag(gamma) dS_n)^T)_t
+//                                              dS = gamma dS_n + Q~^T dO - E~^T dY
 // and through the factors: dq = dQ~ e^G, db = dE~ e^G k, dk = dE~ e^G b + dK~ e^-G,
 // dw = dY v, dv = dY w, dG = dQ~ Q~ + dE~ E~ - dK~ K~ (+ gamma dgamma on the last
-// row), dlog alpha = reverse cumulative sum of dG inside the chunk.
+// row), dlog alpha = reverse cumulative sum of dG inside the chunk.  The terms of that sum
+// cancel down to a result of the order of alpha, so dG is formed from the bf16 factors the
+// products used and gamma dgamma from the state-update part of dK~ (its own accumulator): the
+// cancelling pairs then cancel exactly, and dlog alpha keeps its accuracy at any decay.
 //
 // The only serial dependence is the dS chain.  With W = T E~ and K^ = K~ Diag(gamma):
 //   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO),
@@ -241,7 +245,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     __shared__ __align__(8) uint64_t bar_in, bar_ap, bar_z, bar_w, bar_r;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ int s_tok[2];  // per channel half: some channel's chunk log-decay is past kGradDecayLimit
+    __shared__ int s_tok[2];  // per channel half: some channel's chunk log-decay is past kChunkDecayLimit
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     ChunkRef cr;
     if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
@@ -316,9 +320,9 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
             tot1 += v.y;
         }
         const float gam0 = __expf(tot0), gam1 = __expf(tot1);
-        if (tg == 0) {  // warps 0 and 1: gamma, and whether the chunk's decay stays within kGradDecayLimit
+        if (tg == 0) {  // warps 0 and 1: gamma, and whether e^{-G} stays in range on every channel
             *reinterpret_cast<float2 *>(a.gam + cidx * GSTR + ch) = make_float2(gam0, gam1);
-            const bool out_of_range = __any_sync(0xffffffffu, tot0 < -kGradDecayLimit || tot1 < -kGradDecayLimit);
+            const bool out_of_range = __any_sync(0xffffffffu, tot0 < -kChunkDecayLimit || tot1 < -kChunkDecayLimit);
             if (lane == 0) s_tok[cb] = out_of_range;
         }
         float2 mv[16];  // e^-G, backwards from the group's last token
@@ -353,7 +357,7 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
     }
     fence_proxy_async_smem();
     __syncthreads();
-    if (tid == 32) {  // a chunk past kGradDecayLimit: the chain steps it token by token, and the
+    if (tid == 32) {  // a chunk past the factors' range: the chain steps it token by token, and the
                       // token-level kernel rewrites its gradients
         const int tokm = s_tok[0] | s_tok[1];
         reinterpret_cast<int *>(a.gam + cidx * GSTR)[D] = tokm;
@@ -794,7 +798,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
 //   dY^T = dU~^T T                     A from TMEM, K 64            -> dv, dw, -dY tile
 //   [dP; dA] = [dO; -dY] U~^T          M 2 x 64 tokens, N 64, K d_v -> masked bf16 tile
 //   [dQ~^T | dE~^T] = S [dO; -dY]^T + K~^T [dP; dA]^T     M d_k, N 128, K d_v + 64
-//   dK~^T = (Gm dS_n) U~^T + Q~^T dP + E~^T dA            M d_k, N 64, K d_v + 128
+//   dK~^T = [(Gm dS_n) U~^T] + [Q~^T dP + E~^T dA]        M d_k, N 64, K d_v | 128 (two accumulators)
 // The tiles arrive by TMA in 128-byte swizzled atoms; a [rows][128] tile is two column atoms
 // of [rows][64].  The factor chain reads dQ~^T, dE~^T, dK~^T straight from TMEM: a thread
 // owns one channel of d_k (its TMEM lane) and 16 tokens (its column block).
@@ -820,11 +824,11 @@ constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
 constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
 constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
-constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [4][D], twice
+constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [8][D], then [4][D] twice
 // full chunks stage dq, dk, db over the reloaded raw q, k, b and dg over v, w for the TMA stores
 // TMEM columns
 constexpr uint32_t TM_Y = 0, TM_DU = 64, TM_YB = 128, TM_DUB = 160, TM_U = 192, TM_DY = 256, TM_PA = 320;
-constexpr uint32_t TM_DQE = 384, TM_DK = 0, TM_COLS = 512;
+constexpr uint32_t TM_DQE = 384, TM_DK = 0, TM_DKU = 64, TM_COLS = 512;  // TM_DKU: dK~'s state-update part
 constexpr uint32_t IDESC_KK = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_MM = tc::idesc_bf16(128, 64, 1, 1);
 constexpr uint32_t IDESC_KM = tc::idesc_bf16(128, 64, 0, 1);
@@ -935,11 +939,11 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     const size_t slot = bound_slot(a.pr, cr.n, hh, cr.nch, ci);
     const int y = bb + ci * C;
     const bool full = L == C;  // full chunks store their gradients by TMA from shared memory
-    // the chunk-end state (for gamma dgamma), in flight during the folding
+    // the chunk-start state (for gamma dgamma's part gamma rowsum(dS_n . S)), in flight during the folding
     const int dch = tid & 15;
     uint4 ssv[4];
     {
-        const __nv_bfloat16 *st_n = a.states + (slot + 1) * D * D;
+        const __nv_bfloat16 *st_n = a.states + slot * D * D;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
@@ -989,7 +993,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             mma_ss(tmem + TM_Y, sdesc_sw128(sb + SS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                    sdesc_sw128(sb + RB + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_KK, ks > 0);
     }
-    // ---- dS_n^T -> (Gm dS_n)^T in place, gamma dgamma = column sums of dS_n^T . S_end^T
+    // ---- dS_n^T -> (Gm dS_n)^T in place; gamma dgamma's part gamma rowsum(dS_n . S) from the column
+    //      sums of dS_n^T . S^T
     {
         float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         float gm[8];
@@ -1032,7 +1037,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         float s = 0.f;
 #pragma unroll
         for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
-        reinterpret_cast<float *>(sm + DGF)[tid] = s;
+        reinterpret_cast<float *>(sm + DGF)[tid] = sGam[tid] * s;
     }
     // ---- dU~^T = dO^T P + (Gm dS_n)^T K~^T
     if (tid == 0) {
@@ -1133,7 +1138,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                    sdesc_sw128(sb + DY + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), IDESC_MK2, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + TM_DK, sdesc_sw128(sb + DS + ks * 2048, 16384, 1024),
+            mma_ss(tmem + TM_DKU, sdesc_sw128(sb + DS + ks * 2048, 16384, 1024),
                    sdesc_sw128(sb + UU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_MK, ks > 0);
         mma_commit(&bar_c);
     }
@@ -1181,68 +1186,81 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_ss(tmem + TM_DK, sdesc_sw128(sb + RQ + ks * 2048, 8192, 1024), sdesc_sw128(sb + PA + ks * 2048, 8192, 1024),
-                   IDESC_MM, 1);
+                   IDESC_MM, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_ss(tmem + TM_DK, sdesc_sw128(sb + RB + ks * 2048, 8192, 1024),
                    sdesc_sw128(sb + PA + 8192 + ks * 2048, 8192, 1024), IDESC_MM, 1);
         mma_commit(&bar_d);
     }
-    // ---- through the factors: thread = channel `row` of d_k, tokens 16 cg .. 16 cg + 15
+    // ---- through the factors: thread = channel `row` of d_k, tokens 16 cg .. 16 cg + 15.  The
+    //      terms of dG cancel down to a result of the order of alpha, so they are formed from the
+    //      bf16 factors the products used (the pair terms then cancel exactly): e^G and e^-G are
+    //      rebuilt here exactly as the folding built them, per 8-token group (decay_pair8), and
+    //      Q~, E~, K~ rounded to bf16 as there.
     {
         float *sFin = reinterpret_cast<float *>(sm + SC_FIN);
         const bool ch_ok = row < a.din;
         float al[16];
-        float run = 0.f;
+        float run2[2] = {0.f, 0.f};  // log-decay sums of this thread's two 8-token groups
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * cg + i;
             const float gv = (t < L && ch_ok) ? *reinterpret_cast<const float *>(sm + GG + (row >> 5) * 8192 +
                                                                                   sw128(t, (row & 31) * 4))
                                               : 0.f;
-            run += gv;
+            run2[i >> 3] += gv;
             al[i] = __expf(gv);
         }
         wait_or_abort(&bar_d, ph, a.status, &s_abort);
         tc_fence_after();
         if (warp == 0 && next >= 0) issue(0, nx);  // Q~, K~, E~, [dO; -dY], T, P are consumed
-        sFin[cg * D + row] = run;
+        sFin[(2 * cg) * D + row] = run2[0];
+        sFin[(2 * cg + 1) * D + row] = run2[1];
         if (tid == 32) bulk_wait_read0();  // dv and dw have left v and w, which take dg below
         __syncthreads();
         if (warp == 0 && next >= 0) issue(1, nx);  // log alpha is read
-        float off = 0.f;
+        float off2[2] = {0.f, 0.f};  // G before each group: the group sums in order, as the folding added them
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (u < cg) off += sFin[u * D + row];
+        for (int u = 0; u < 8; ++u)
+            if (u < 2 * cg) off2[0] += sFin[u * D + row];
+        off2[1] = off2[0] + run2[0];
         float emG[16];
-        {
-            float rr = __expf(-(off + run));
 #pragma unroll
-            for (int i = 15; i >= 0; --i) {
-                emG[i] = rr;
-                rr *= al[i];
+        for (int h8 = 0; h8 < 2; ++h8) {
+            float rr = __expf(-(off2[h8] + run2[h8]));
+#pragma unroll
+            for (int i = 7; i >= 0; --i) {
+                emG[8 * h8 + i] = rr;
+                rr *= al[8 * h8 + i];
             }
         }
-        uint32_t rq[16], re[16], rk[16];
+        uint32_t rq[16], re[16], rk[16], ru[16];
         tmem_ld16(tmem + TM_DQE + 16 * cg + lane_off, rq);
         tmem_ld16(tmem + TM_DQE + 64 + 16 * cg + lane_off, re);
         tmem_ld16(tmem + TM_DK + 16 * cg + lane_off, rk);
+        tmem_ld16(tmem + TM_DKU + 16 * cg + lane_off, ru);
         tmem_wait_ld();
         wait_or_abort(&bar_in2, ph, a.status, &s_abort);
-        float e = __expf(off);
+        float e = 0.f, kup = 0.f;  // kup: this thread's share of sum_s K~_s . dK~_s (state-update part)
         float dG[16];
         const size_t base = tok_off(a, bb, hh, ci, 16 * cg) + row, stride = (size_t)a.H * a.din;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * cg + i;
+            if ((i & 7) == 0) e = __expf(off2[i >> 3]);
             e *= al[i];
             const uint32_t so = tile_off(t, row, 8192);
             const bool ok = t < L;
             const float q0 = ok ? ld_bf(sm + SS + so) : 0.f, k0 = ok ? ld_bf(sm + SS + 16384 + so) : 0.f;
             const float b0 = ok ? ld_bf(sm + DS + so) : 0.f;
-            const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dK = __uint_as_float(rk[i]);
+            const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dKu = __uint_as_float(ru[i]);
+            const float dK = __uint_as_float(rk[i]) + dKu;
             const float de = dE * e;
-            dG[i] = dQ * q0 * e + de * b0 * k0 - dK * k0 * emG[i];
+            const uint32_t qe = pack_bf16x2(q0 * e, b0 * k0 * e);  // Q~, E~ as the folding rounded them
+            const float kt = __bfloat162float(__float2bfloat16_rn(k0 * emG[i]));  // K~, likewise
+            dG[i] = dQ * bf_lo(qe) + dE * bf_hi(qe) - dK * kt;
+            kup = fmaf(kt, dKu, kup);
             if (full) {  // over the raw q, k, b just read
                 st_bf(sm + SS + so, dQ * e);
                 st_bf(sm + DS + so, de * k0);
@@ -1261,12 +1279,17 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             rs += dG[i];
             dG[i] = rs;
         }
-        sFin[4 * D + cg * D + row] = rs;
+        sFin[8 * D + cg * D + row] = rs;
+        sFin[12 * D + cg * D + row] = kup;
         named_bar(1 + quarter, 4 * 32);  // the four warps of this TMEM lane quarter
+        // later groups, and the state-update part of gamma dgamma: sum over the chunk of K~ . dK~'s
+        // update part, formed from the very values dK~ and dG used, so that it cancels exactly
         float after = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (u > cg) after += sFin[4 * D + u * D + row];
+        for (int u = 0; u < 4; ++u) {
+            if (u > cg) after += sFin[8 * D + u * D + row];
+            after += sFin[12 * D + u * D + row];
+        }
         if (full) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)

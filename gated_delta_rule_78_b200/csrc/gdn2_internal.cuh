@@ -142,13 +142,6 @@ cudaError_t launch_chunk_offsets(const int *cu_seqlens, int n_seqs, int total_ro
 // and all factors and products stay finite in fp32 and bf16.  Chunks past that limit run the
 // token-by-token form instead (tok_util.cuh), which is exact for any decay.
 constexpr float kChunkDecayLimit = 80.f;
-// The chunkwise backward forms dlog alpha as a reverse cumulative sum of terms q.dq - k.dk ...
-// that cancel down to a result of the order of alpha: its bf16 operands leave a relative error
-// that grows with the chunk's decay (measured rel-L2 of dlog alpha against the oracle: 0.7e-2 at a
-// chunk log-decay of 3, 1.3e-2 at 19, 2.3e-2 at 48, 3.1e-2 at 64; every other output stays near
-// 0.4e-2).  The backward therefore takes the token-by-token form, whose dlog alpha is a direct
-// sum, for chunks whose total log-decay falls below -kGradDecayLimit on some channel.
-constexpr float kGradDecayLimit = 16.f;
 
 // The token-level forward (tok.cu): the fp32 path, any head size.  `states`, when non-null,
 // receives the fp32 state S ([c][j], d_k rows) at every chunk boundary, at the boundary slots

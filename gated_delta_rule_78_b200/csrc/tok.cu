@@ -4,7 +4,7 @@
 //   * the fp32 path: the forward, and the backward as three launches (the forward in states
 //     mode, the reverse dS chain, the per-chunk gradients);
 //   * the exact path for chunks of the bf16 tensor-core backward whose decay is too strong for
-//     the chunkwise form (kGradDecayLimit): their gradients are rewritten here.
+//     the chunkwise form (kChunkDecayLimit): their gradients are rewritten here.
 // The recurrence is the token form of the update (tok_util.cuh): no chunk factor e^{-G} is ever
 // formed, so the results are exact for any decay.
 //
