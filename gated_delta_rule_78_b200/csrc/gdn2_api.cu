@@ -224,6 +224,17 @@ gdn2_status check_gate_ptrs(int flags, const void *g, const void *b, const void 
 }
 }  // namespace
 
+gdn2_status gdn2::check_bwd_args(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q, const void *k,
+                                 const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                                 const void *d_o, const float *dS_T, const void *dq, const void *dk, const void *dv,
+                                 const float *dlog_alpha, const void *db, const void *dw, const float *dS0)
+{
+    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
+    if (st != GDN2_OK) return st;
+    if (T > 0) return check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0}, {S0, dS_T});
+    return check_ptrs({dS0}, {S0, dS_T});
+}
+
 namespace {
 gdn2_status chunk_bwd_impl(bool saved, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
                            const void *k, const void *v, const float *log_alpha, const void *b,
@@ -231,13 +242,8 @@ gdn2_status chunk_bwd_impl(bool saved, gdn2_dtype dt, int B, int T, int H, int D
                            void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
                            float *dS0, void *workspace, size_t ws_bytes, void *stream)
 {
-    gdn2_status st = check_sizes(dt, B, T, H, Dk, Dv);
-    if (st != GDN2_OK) return st;
-    if (T > 0)
-        st = check_ptrs({q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0},
-                        {S0, dS_T});
-    else
-        st = check_ptrs({dS0}, {S0, dS_T});
+    const gdn2_status st = gdn2::check_bwd_args(dt, B, T, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, d_o, dS_T, dq, dk,
+                                                dv, dlog_alpha, db, dw, dS0);
     if (st != GDN2_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);

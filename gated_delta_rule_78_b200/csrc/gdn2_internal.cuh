@@ -243,6 +243,13 @@ cudaError_t launch_channel_sum(bool fp32, const void *src, void *dst, size_t n_r
 
 // device address of the library's kernel status word on the current device
 int *status_word();
+// Argument checks of the backward entry points (sizes inside the contract, required pointers
+// non-null, every pointer 16-byte aligned), shared by gdn2_chunk_bwd and gdn2_chunk_bwd_noalloc
+// so that both reject exactly the same calls.
+gdn2_status check_bwd_args(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q, const void *k,
+                           const void *v, const float *log_alpha, const void *b, const void *w, const float *S0,
+                           const void *d_o, const float *dS_T, const void *dq, const void *dk, const void *dv,
+                           const float *dlog_alpha, const void *db, const void *dw, const float *dS0);
 // Failure-detection self-test (selftest.cu): one bounded wait on a phase nothing completes.
 cudaError_t launch_selftest_timeout(int limit_us, int *status, cudaStream_t s);
 

@@ -6,13 +6,19 @@
 // recurse into itself), runtimes that forbid device allocation after start-up
 // so that their memory budget stays fixed, and plain C hosts with no tensor
 // library around to hand them a buffer.  They pass inputs and outputs as usual;
-// the scratch comes from `g_bwd_scratch` below, which is reserved once on every
-// GPU that loads the library and stays reserved until the process exits.
+// the scratch comes from `g_bwd_scratch` below.
+//
+// When the array's memory is taken: CUDA loads a library's modules lazily by
+// default (CUDA_MODULE_LOADING=LAZY), so the 32 MiB are committed on a device at
+// the first call of this entry point with that device current, not when the
+// library is loaded.  From then on they stay reserved until the process exits.
+// A caller whose memory budget must not move, or that captures streams into CUDA
+// graphs, makes one call on every device at start-up, before the budget is fixed
+// and before any capture.
 //
 // This entry point allocates nothing: no cudaMalloc, no cudaFree, no library
 // routine that allocates.  It runs the same three kernels as gdn2_chunk_bwd,
 // with the same workspace layout, so both give the same gradients.
-#include <atomic>
 #include <stdint.h>
 
 #include "gdn2_internal.cuh"
@@ -20,32 +26,21 @@
 namespace {
 
 constexpr size_t kScratchBytes = GDN2_NOALLOC_MAX_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // The scratch.  In host code this name is only a handle for the runtime: its
-// device address comes from cudaGetSymbolAddress, once per device.
+// device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_bwd_scratch[kScratchBytes];
-
-// Device address of g_bwd_scratch per device ordinal (null until first use).
-std::atomic<void *> g_scratch_addr[kMaxDevices];
-
-bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 gdn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
 
-// The current device's address of g_bwd_scratch; looked up on the first call
-// made with that device current.  Two threads racing here both store the same
-// value, so the race is harmless.
+// The current device's address of g_bwd_scratch, looked up on every call (a
+// cheap lookup once the module is loaded), so that no address outlives the
+// context it came from: after cudaDeviceReset the module is loaded anew and its
+// address may change.
 gdn2_status scratch_address(void **out)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GDN2_ERR_UNSUPPORTED;
-    void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
-        g_scratch_addr[dev].store(p, std::memory_order_release);
-    }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
     *out = p;
     return GDN2_OK;
 }
@@ -58,24 +53,10 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(
     const float *dS_T, void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
     float *dS0, void *stream)
 {
-    // the same argument rules as gdn2_chunk_bwd
-    if (dt != GDN2_F32 && dt != GDN2_BF16) return GDN2_ERR_DTYPE;
-    if (B <= 0 || H <= 0 || T < 0 || Dk <= 0 || Dv <= 0) return GDN2_ERR_SHAPE;
-    if (Dk != Dv || (Dk != 64 && Dk != 128)) return GDN2_ERR_UNSUPPORTED;
-    if ((long long)B * H > (1LL << 30)) return GDN2_ERR_UNSUPPORTED;
-    if ((long long)B * T * H * Dk > (1LL << 40)) return GDN2_ERR_UNSUPPORTED;
-    if (T > 0) {
-        const void *req[] = {q, k, v, log_alpha, b, w, d_o, dq, dk, dv, dlog_alpha, db, dw, dS0};
-        for (const void *p : req)
-            if (!p) return GDN2_ERR_NULL;
-        for (const void *p : req)
-            if (!aligned16(p)) return GDN2_ERR_ALIGN;
-    } else if (!dS0) {
-        return GDN2_ERR_NULL;
-    } else if (!aligned16(dS0)) {
-        return GDN2_ERR_ALIGN;
-    }
-    if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T))) return GDN2_ERR_ALIGN;
+    // the argument rules of gdn2_chunk_bwd, from the same routine
+    const gdn2_status chk = gdn2::check_bwd_args(dt, B, T, H, Dk, Dv, q, k, v, log_alpha, b, w, S0, d_o, dS_T, dq,
+                                                 dk, dv, dlog_alpha, db, dw, dS0);
+    if (chk != GDN2_OK) return chk;
 
     cudaStream_t s = (cudaStream_t)stream;
     if (T == 0) {
@@ -92,8 +73,9 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_bwd_noalloc(
     const gdn2_status st = scratch_address(&scratch);
     if (st != GDN2_OK) return st;
     // Every scratch byte the kernels read is written earlier in the same call
-    // (chunk-start states, per-chunk matrices, per-slice partial gradients), so
-    // nothing left by an earlier call needs clearing.
+    // (chunk-start states, per-chunk matrices, the count of chunks that run token
+    // by token, which the call clears first), so nothing left by an earlier call
+    // is read.
     gdn2::BwdOut out{dq, dk, dv, db, dw, dlog_alpha, dS0};
     return from_cuda(gdn2::launch_bwd(dt, p, d_o, dS_T, out, scratch, s));
 }

@@ -152,10 +152,13 @@ cudaError_t launch_fwd_host(gdn2_dtype dt, int B, int T, int H, int D, const voi
             e = D2H(S_T + (size_t)r0 * st_row, slot + sl.st, (size_t)nr * st_row * 4);
         if (e == cudaSuccess) e = cudaEventRecord(ev_free[j], hs.out);
     }
-    // the caller's stream completes when the last copy-out has
-    if (e == cudaSuccess) e = cudaEventRecord(ev_start, hs.out);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_start, 0);
-    return e;
+    // the caller's stream completes when the last copy-out and the last copy-in have, also when an
+    // error cut the loop short: copies already enqueued still use the caller's host buffers
+    cudaError_t ej = cudaEventRecord(ev_start, hs.out);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, ev_start, 0);
+    if (ej == cudaSuccess) ej = cudaEventRecord(ev_in[0], hs.in);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, ev_in[0], 0);
+    return e != cudaSuccess ? e : ej;
 }
 
 }  // namespace gdn2

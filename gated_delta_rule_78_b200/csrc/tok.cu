@@ -369,7 +369,10 @@ TokWs tok_ws(const Problem &p)
     l.coff = 0;
     l.states = off;  off += H * nbound * D * D * 4;
     l.dSe = off;     off += H * nchunk * D * D * 4;
-    l.blocks = (int)std::max<size_t>(1, std::min<size_t>(H * nchunk, kGradBlocks));
+    // the gradient kernel's scratch grows with the problem: as many blocks as the boundary states'
+    // bytes pay for (one at least, one wave at most)
+    l.blocks = (int)std::max<size_t>(1, std::min<size_t>({H * nchunk, (size_t)kGradBlocks,
+                                                           (l.dSe - l.states) / tok_grad_block_bytes(p.D)}));
     l.scratch = off; off += (size_t)l.blocks * tok_grad_block_bytes(p.D);
     l.total = off;
     return l;

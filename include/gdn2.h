@@ -82,7 +82,10 @@ typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
  *        at least 48 chunks, which run as a chunk-parallel scan over segments of each
  *        sequence when given it (the serial chain runs when it is missing or short).
  * bf16 inputs run on the tensor cores (bf16 operands, fp32 accumulation,
- * fp32 state); fp32 inputs run in fp32 FMA arithmetic throughout.
+ * fp32 state); fp32 inputs run token by token in fp32 arithmetic throughout.
+ * Any decay alpha in [0, 1] is exact: a chunk whose log-decay falls below -80
+ * on some channel (where the chunkwise factor e^{-G} would leave the fp32
+ * range) runs token by token instead, slower but with the same results.
  */
 GDN2_API gdn2_status gdn2_chunk_fwd(gdn2_dtype dt, int B, int T, int H, int Dk, int Dv,
                            const void *q, const void *k, const void *v, const float *log_alpha,
@@ -105,10 +108,12 @@ GDN2_API gdn2_status gdn2_decode_step(gdn2_dtype dt, int N, int H, int Dk, int D
  *   Outputs: dq, dk, db [B,T,H,Dk] and dv, dw [B,T,H,Dv] of type dt;
  *            dlog_alpha [B,T,H,Dk] fp32; dS0 [B,H,Dk,Dv] fp32.
  *   S0 may be NULL (zeros).  All outputs must be distinct from the inputs.
- *   workspace: at least gdn2_workspace_size(1, ...) bytes.  bf16 with
- *   d = 128: chunk-boundary states and per-chunk factors (bf16), the chain's
- *   per-chunk inputs (fp32) and the state gradients at chunk ends (bf16);
- *   otherwise fp32 chunk-start states and per-tile partial gradients.
+ *   workspace: at least gdn2_workspace_size(1, ...) bytes.  bf16: chunk-boundary
+ *   states and per-chunk factors (bf16), the chain's per-chunk inputs and the
+ *   state gradients at chunk ends (bf16), and the scratch of the token-level
+ *   gradients of chunks whose decay is too strong for the chunkwise factors
+ *   (a chunk log-decay below -80 on some channel); fp32: fp32 chunk-boundary
+ *   states and chunk-end state gradients, and that scratch.
  * The gates enter inside the chunk products (gate-weighted keys and values),
  * as the aixai.ru post's implementation section requires.
  */
@@ -167,23 +172,28 @@ GDN2_API gdn2_status gdn2_chunk_bwd_saved(gdn2_dtype dt, int B, int T, int H, in
  * backward as gdn2_chunk_bwd, with the same arguments minus the workspace and
  * the same gradients.
  *   Scratch: a file-scope device array of GDN2_NOALLOC_MAX_SCRATCH_BYTES
- *   bytes inside the library.  Every GPU that loads the library reserves it
- *   and holds it until the process exits.  A problem is accepted when
+ *   bytes inside the library.  A problem is accepted when
  *   gdn2_workspace_size(1, ...) <= GDN2_NOALLOC_MAX_SCRATCH_BYTES (for
- *   example B*H = 2, T = 1024, d = 128 needs 20.5 MiB with fp32 inputs and
- *   4.6 MiB with bf16 inputs); larger ones return GDN2_ERR_TOO_LARGE before
- *   anything is launched.
+ *   example B*H = 2, T = 1024, d = 128 needs about 8 MiB with either dtype,
+ *   B*H = 4, T = 4096, d = 128 more than 32 MiB); larger ones return
+ *   GDN2_ERR_TOO_LARGE before anything is launched.  Arguments are checked by
+ *   the same rules as gdn2_chunk_bwd.
+ *   When the memory is taken: CUDA loads a library's code lazily by default
+ *   (CUDA_MODULE_LOADING=LAZY), so the array is committed on a device at the
+ *   first call of this entry point with that device current, and from then on
+ *   held until the process exits.  A caller whose budget must not move makes
+ *   one call on each device at start-up, before the budget is fixed and
+ *   before any stream capture.
  *   Allocation: none.  No cudaMalloc, cudaFree or allocating library call.
- *   First call per device: looks up the array's device address with
- *   cudaGetSymbolAddress for the device current at the call (which must be
- *   the device that holds the arguments and the stream); later calls on that
- *   device reuse it.  Make that first call before any stream capture.
+ *   Every call looks up the array's device address (cudaGetSymbolAddress) for
+ *   the device current at the call, which must be the device that holds the
+ *   arguments and the stream.
  *   Sharing: all calls on one device use the same array, and it keeps what
  *   the last call left there.  Calls whose kernels overlap on the GPU (on
  *   different streams, or from different threads) race on it and give wrong
  *   gradients: order them on one stream or with events.  Nothing in the
- *   array needs to start at zero: each call writes every scratch byte it
- *   reads before reading it.
+ *   array needs to start at zero: each call writes or clears every scratch
+ *   byte it reads before reading it.
  */
 #define GDN2_NOALLOC_MAX_SCRATCH_BYTES ((size_t)32 << 20)
 

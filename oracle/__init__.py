@@ -94,10 +94,15 @@ def ref_bwd(q, k, v, g, b, w, S0, do, dST=None, nthreads=None):
     return out
 
 
-def ref_decode(q, k, v, g, b, w, S, nthreads=None):
-    """One decode step: inputs [N,H,D], S [N,H,Dk,Dv].  Returns (o, S_new) in fp64."""
+def ref_decode(q, k, v, g, b, w, S, nthreads=None, inplace=False):
+    """One decode step: inputs [N,H,D], S [N,H,Dk,Dv].  Returns (o, S_new) in fp64.  With
+    inplace=True, S must be a C-contiguous fp64 array; it is updated in place and returned."""
     q, k, v, g, b, w = map(_f64, (q, k, v, g, b, w))
-    S = _f64(S).copy()
+    if inplace:
+        if not (isinstance(S, np.ndarray) and S.dtype == np.float64 and S.flags["C_CONTIGUOUS"]):
+            raise ValueError("inplace ref_decode needs a C-contiguous fp64 state")
+    else:
+        S = _f64(S).copy()
     N, H, Dk = q.shape
     Dv = v.shape[-1]
     o = np.empty((N, H, Dv))

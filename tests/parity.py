@@ -51,6 +51,18 @@ def bh_slice(x, pairs):
     return out
 
 
+def assert_chains_close(got, ref, dtype, name, head_axis=1):
+    """Every (batch, head) chain of one batch row: `got` (device or host tensor) and `ref` (fp64)
+    are [T, H, D] (head_axis=1) or [H, Dk, Dv] (head_axis=0); each head's chain must meet the
+    tolerance on its own.  Returns the worst error."""
+    g, r = f64(got), f64(ref)
+    worst = 0.0
+    for h in range(g.shape[head_axis]):
+        gh, rh = np.take(g, h, axis=head_axis), np.take(r, h, axis=head_axis)
+        worst = max(worst, assert_close(gh, rh, dtype, f"{name} head {h}"))
+    return worst
+
+
 def sample_pairs(B, H, n, seed=0):
     rng = np.random.default_rng(seed)
     idx = rng.choice(B * H, size=min(n, B * H), replace=False)

@@ -27,22 +27,28 @@ def test_decode_small(cuda_lib, dtype, D):
 
 
 def test_decode_1024_steps_full_size(cuda_lib):
-    """256 sequences, H=16, d=128, fp32 state in place, 1024 steps.  Every step's o
-    and the final S are compared on a sample of sequences (all heads)."""
+    """256 sequences, H=16, d=128, fp32 state in place, 1024 steps.  The oracle advances every
+    sequence; o of every sequence is compared at every 64th step and at the last, and the final
+    state of every sequence."""
     g = cuda_lib
     w = DECODE_WORKLOAD
     ds = DecodeStream(w["N"], w["H"], w["Dk"], w["Dv"], dtype=w["dtype"], seed=0)
-    seqs = [0, 97, 201, w["N"] - 1]
     S = ds.S0.cuda()
-    Sref = ds.S0[seqs].double().numpy()
-    worst = 0.0
+    Sref = np.ascontiguousarray(ds.S0.double().numpy())
+    checked = 0
     for step in range(w["steps"]):
         x = ds.step()
         d = to_dev(x)
         o = g.gdn2_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S)
-        xs = {n: t[seqs] for n, t in x.items()}
-        ro, Sref = oracle.ref_decode(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["b"], xs["w"], Sref)
-        worst = max(worst, assert_close(o[seqs], ro, "bf16", f"o step {step}"))
+        ro, Sref = oracle.ref_decode(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], Sref, inplace=True)
+        if step % 64 == 0 or step == w["steps"] - 1:
+            oc = o.cpu()
+            for n in range(w["N"]):
+                assert_close(oc[n], ro[n], "bf16", f"o step {step} seq {n}")
+            checked += 1
+    assert checked == w["steps"] // 64 + 1
     assert g.gdn2_sync_status() == 0
-    assert_close(S[seqs], Sref, "bf16", "final S")
-    assert torch.isfinite(S).all()
+    Sc = S.cpu()
+    assert torch.isfinite(Sc).all()
+    for n in range(w["N"]):
+        assert_close(Sc[n], Sref[n], "bf16", f"final S seq {n}")
