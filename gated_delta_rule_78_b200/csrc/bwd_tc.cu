@@ -24,15 +24,17 @@
 // cancelling pairs then cancel exactly, and dlog alpha keeps its accuracy at any decay.
 //
 // The only serial dependence is the dS chain.  With W = T E~ and K^ = K~ Diag(gamma):
-//   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO),
-// so the work splits into four launches:
-//   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary;
-//   2. bwd_prep_tc_kernel, one CTA per chunk: factors, [A; P], T, W^T, R^T (no state
-//      needed);
-//   3. bwd_chain_tc_kernel, one CTA per (batch, head): the reverse dS chain with dS^T
-//      kept in TMEM; stores dS_n per chunk;
-//   4. bwd_grad_kernel, persistent over the chunks: recomputes U~ from the stored state
+//   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO) = M^T dO,  M = Q~ - P W,
+// so the work splits into three launches:
+//   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary, and from
+//      its M group the state-independent factors W^T, K^, gamma, M^T, T and P of every chunk
+//      (BwdFactors), formed where the chunk's Q~, E~, K~, T and P already are;
+//   2. bwd_chain_tc_kernel, one CTA per (batch, head): the reverse dS chain with dS^T
+//      kept in TMEM, R^T = dO^T M formed on the tensor pipe beside it; stores dS_n per chunk;
+//   3. bwd_grad_kernel, persistent over the chunks: recomputes U~ from the stored state
 //      and produces every gradient of the chunk.
+// Chunks whose decay is past the factors' range (kChunkDecayLimit) are flagged by the forward;
+// the chain steps them token by token and tok.cu's kernel rewrites their gradients.
 // Every product is a bf16 tcgen05 MMA with an fp32 TMEM accumulator, its operands
 // in 128-byte swizzled shared-memory tiles (most of them loaded by TMA) or in TMEM.
 #include <algorithm>
@@ -43,32 +45,29 @@
 #include "gdn2_internal.cuh"
 #include "tc_util.cuh"
 #include "tok_util.cuh"
-#include "warp_mma.cuh"
 
 namespace gdn2 {
 namespace {
 
 using namespace tc;
-using namespace wm;
 
 constexpr int D = 128;
 constexpr int C = 64;
-constexpr int LDA = 68;  // fp32 row stride of the A / T scratch of the solve
-constexpr int GSTR = D + 4;  // per-chunk record of gamma: D floats, then the token-mode flag (int)
+constexpr int GSTR = kGamStride;  // per-chunk record of gamma: D floats, then the token-mode flag (int)
 
 // ------------------------------------------------------------------ workspace
 struct BwdTcLayout {
-    size_t coff, states, flist, W, Kh, gam, Rt, Tm, Pm, dSn, scratch, total;
+    size_t coff, states, flist, W, Kh, gam, Mc, Tm, Pm, dSn, scratch, total;
     int tok_blocks;  // blocks of the token-level gradient kernel
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W^T bf16 [D][C],
-// K^ bf16 [C][D], gamma and the chunk's token-mode flag [GSTR] fp32, R^T bf16 [D][D], T and P
+// K^ bf16 [C][D], gamma and the chunk's token-mode flag [GSTR] fp32, M^T bf16 [D][C], T and P
 // bf16 [C][C], dS_n^T bf16 [D][D].  flist: the count and the list of the chunk tasks that run
 // token by token.  Variable length puts chunk_off first; chunk lists are sized by the chunk
-// bound.  The token-level gradient kernel's scratch reuses W .. R^T, which only the chain reads
+// bound.  The token-level gradient kernel's scratch reuses W .. M^T, which only the chain reads
 // (one block's scratch at least; past the end of the workspace when that region is smaller).
 BwdTcLayout tc_layout(const Problem &p)
 {
@@ -81,7 +80,7 @@ BwdTcLayout tc_layout(const Problem &p)
     l.W = off;      off += H * nchunk * C * D * 2;
     l.Kh = off;     off += H * nchunk * C * D * 2;
     l.gam = off;    off += round256(H * nchunk * GSTR * 4);
-    l.Rt = off;     off += H * nchunk * D * D * 2;
+    l.Mc = off;     off += H * nchunk * D * C * 2;
     l.Tm = off;     off += H * nchunk * C * C * 2;
     l.Pm = off;     off += H * nchunk * C * C * 2;
     l.dSn = off;    off += H * nchunk * D * D * 2;
@@ -109,7 +108,7 @@ struct BwdTcArgs {
     __nv_bfloat16 *states, *W, *Kh, *Tm, *Pm, *dSn;
     float *gam;          // [chunk][GSTR]: gamma, then the chunk's token-mode flag
     int *flist;          // flist[0]: count of the chunks that run token by token, then their tasks
-    __nv_bfloat16 *Rt;  // R^T per chunk, bf16
+    __nv_bfloat16 *Mc;  // M^T per chunk, bf16 (R^T = dO^T M)
     __nv_bfloat16 *dq, *dk, *dv, *db, *dw;
     float *dg, *dS0;
     int *status;         // kernel status word (bounded waits that gave up)
@@ -130,10 +129,6 @@ __device__ __forceinline__ size_t tok_off(const BwdTcArgs &a, int bos, int hh, i
 __device__ __forceinline__ bool chunk_ref_at(const BwdTcArgs &a, int gc, int h, ChunkRef &r)
 {
     return chunk_at(a.pr, gc, h, r);
-}
-__device__ __forceinline__ bool chunk_ref(const BwdTcArgs &a, ChunkRef &r)
-{
-    return chunk_ref_at(a, blockIdx.x, blockIdx.y, r);
 }
 
 // Decay folding of the gradient kernel: thread (channel pair cp, token group g8) owns channels
@@ -179,6 +174,12 @@ __device__ __forceinline__ void decay_pair8(const float2 (&g)[8], float2 (&eG)[8
     total = make_float2(tot0, tot1);
 }
 
+// barrier over `count` threads (id 0 is __syncthreads)
+__device__ __forceinline__ void named_bar(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Bounded wait on an mbarrier phase.  A wait that gives up records the timeout in the status
 // word and in the block's abort flag; once that is set every later wait of the block returns at
 // once, so a block that lost a transfer ends (with garbage) after one wait limit instead of one
@@ -189,344 +190,6 @@ __device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, in
     if (!tc::mbar_wait(bar, parity)) {
         *abort = 1;
         atomicExch(status, kStatusTimeout);
-    }
-}
-
-// ================================================================== 2. prep on the tensor cores
-// One 512-thread CTA per (chunk, head): the raw q, b, k, dO tiles arrive by TMA (SW128 atoms),
-// the decay folds into them in place, and the four products run as tcgen05 MMAs with TMEM
-// accumulators:
-//   [A; P] = [E~; Q~] K~^T             M = 128 (stacked tokens), N = 64, K = 128
-//   Z^T    = dO^T P                    M = 128 (d_v), N = 64, K = 64   (dO, P MN-major)
-//   W^T    = E~^T T^T                  M = 128 (d_k), N = 64, K = 64   (E~ MN-major)
-//   R^T    = dO^T Q~ + (-Z^T) W        M = 128 (d_v), N = 128, K = 64 + 64 (-Z^T from TMEM)
-// T = (I + A)^-1 is the blocked solve on four warps, as in the forward.  Written out: K^, gamma,
-// T, P, W^T (rows d_k, for the chain) and R^T (bf16).
-namespace prep_tc {
-// Two blocks per SM: regions are reused once their first use is over.
-constexpr uint32_t QE = 0;          // [E~ a0 | Q~ a0 | E~ a1 | Q~ a1], 8 KiB each (raw b, q)
-constexpr uint32_t KT = 32768;      // K~ [a0 | a1]; after [A; P]: W^T bf16 [128 rows d_k][64 tokens]
-constexpr uint32_t WT = KT;
-constexpr uint32_t DO = 49152;      // dO [a0 | a1]
-constexpr uint32_t PP = 65536;      // P bf16 [64][64]; during the folding: decay totals [4][D] fp32
-constexpr uint32_t TOT = PP;
-constexpr uint32_t SA = 73728;      // A fp32 [64][LDA]; after the solve: T bf16 [64][64]
-constexpr uint32_t TT = SA;
-constexpr uint32_t ST = SA + 64 * LDA * 4;   // T fp32 [64][LDA]
-constexpr uint32_t USED = ST + 64 * LDA * 4;
-constexpr uint32_t SMEM = USED + 1024;       // slack for the 1024-byte alignment
-// TMEM: [A; P] then Z^T in 0..63, W^T in 64..127, -Z^T bf16 in 128..159; R^T (issued once
-// Z^T and W^T are read back) in 0..127
-constexpr uint32_t TM_AP = 0, TM_ZT = 0, TM_WT = 64, TM_ZB = 128, TM_RT = 0, TM_COLS = 256;
-constexpr uint32_t IDESC_AP = tc::idesc_bf16(128, 64, 0, 0);
-constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 1, 1);
-constexpr uint32_t IDESC_W = tc::idesc_bf16(128, 64, 1, 0);
-constexpr uint32_t IDESC_R1 = tc::idesc_bf16(128, 128, 1, 1);
-constexpr uint32_t IDESC_R2 = tc::idesc_bf16(128, 128, 0, 0);
-constexpr int kThreads = 256;
-}  // namespace prep_tc
-
-struct PrepMaps {
-    CUtensorMap q, k, b, dO, g;
-};
-
-__device__ __forceinline__ void named_bar(int id, int count)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-__global__ void __launch_bounds__(prep_tc::kThreads, 2)
-bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
-{
-    using namespace prep_tc;
-    using namespace tc;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_in, bar_ap, bar_z, bar_w, bar_r;
-    __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
-    __shared__ int s_tok[2];  // per channel half: some channel's chunk log-decay is past kChunkDecayLimit
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    ChunkRef cr;
-    if (!chunk_ref(a, cr)) return;  // uniform over the block, before any barrier
-    const int ci = cr.ci, hh = cr.h, bos = cr.sp.bos;
-    const int L = min(C, cr.sp.len - ci * C);
-    const size_t cidx = cr.cidx;
-    const uint32_t sb = smem_u32(sm);
-    float *sA = reinterpret_cast<float *>(sm + SA);
-    float *sT = reinterpret_cast<float *>(sm + ST);
-    float *sTot = reinterpret_cast<float *>(sm + TOT);
-
-    if (tid == 0) {
-        mbar_init(&bar_in, 1);
-        mbar_init(&bar_ap, 1);
-        mbar_init(&bar_z, 1);
-        mbar_init(&bar_w, 1);
-        mbar_init(&bar_r, 1);
-        s_abort = 0;
-        fence_mbar_init();
-        prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.b); prefetch_tmap(&maps.dO);
-        prefetch_tmap(&maps.g);
-    }
-    if (warp == 0) {
-        tmem_alloc(&s_tmem, TM_COLS);
-        tmem_relinquish();
-    }
-    for (int idx = tid; idx < 64 * LDA; idx += kThreads) sT[idx] = 0.f;  // upper blocks stay zero
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    const int y = bos + ci * C;
-    if (tid == 0) {
-        mbar_expect_tx(&bar_in, 8 * 8192);
-        for (int at = 0; at < 2; ++at) {
-            tma_load_3d(sm + KT + at * 8192, &maps.k, at * 64, hh, y, &bar_in);
-            tma_load_3d(sm + QE + at * 16384, &maps.b, at * 64, hh, y, &bar_in);
-            tma_load_3d(sm + QE + 8192 + at * 16384, &maps.q, at * 64, hh, y, &bar_in);
-            tma_load_3d(sm + DO + at * 8192, &maps.dO, at * 64, hh, y, &bar_in);
-        }
-        for (int at = 0; at < a.din / 32; ++at) tma_prefetch_3d(&maps.g, at * 32, hh, y);
-    }
-
-    // ---- decay folding: thread (channel block cb, token group tg of 16, lane): channels
-    //      64 cb + 2 lane (+1), tokens 16 tg .. 16 tg + 15
-    const int cb = warp & 1, tg = warp >> 1, ch = 64 * cb + 2 * lane;
-    {
-        float2 gv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * tg + i;
-            gv[i] = (t < L && ch < a.din)
-                        ? __ldg(reinterpret_cast<const float2 *>(a.g + tok_off(a, bos, hh, ci, t) + ch))
-                        : make_float2(0.f, 0.f);
-        }
-        float run0 = 0.f, run1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            run0 += gv[i].x;
-            run1 += gv[i].y;
-            gv[i] = make_float2(__expf(gv[i].x), __expf(gv[i].y));  // alpha
-        }
-        *reinterpret_cast<float2 *>(sTot + tg * D + ch) = make_float2(run0, run1);
-        wait_or_abort(&bar_in, 0, a.status, &s_abort);
-        __syncthreads();
-        float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float2 v = *reinterpret_cast<const float2 *>(sTot + u * D + ch);
-            if (u < tg) { off0 += v.x; off1 += v.y; }
-            tot0 += v.x;
-            tot1 += v.y;
-        }
-        const float gam0 = __expf(tot0), gam1 = __expf(tot1);
-        if (tg == 0) {  // warps 0 and 1: gamma, and whether e^{-G} stays in range on every channel
-            *reinterpret_cast<float2 *>(a.gam + cidx * GSTR + ch) = make_float2(gam0, gam1);
-            const bool out_of_range = __any_sync(0xffffffffu, tot0 < -kChunkDecayLimit || tot1 < -kChunkDecayLimit);
-            if (lane == 0) s_tok[cb] = out_of_range;
-        }
-        float2 mv[16];  // e^-G, backwards from the group's last token
-        {
-            float r0 = __expf(-(off0 + run0)), r1 = __expf(-(off1 + run1));
-#pragma unroll
-            for (int i = 15; i >= 0; --i) {
-                mv[i] = make_float2(r0, r1);
-                r0 *= gv[i].x;
-                r1 *= gv[i].y;
-            }
-        }
-        float e0 = __expf(off0), e1 = __expf(off1);
-        uint8_t *pe = sm + QE + cb * 16384, *pq = pe + 8192, *pk = sm + KT + cb * 8192;
-        __nv_bfloat16 *kh = a.Kh + cidx * C * D;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * tg + i;
-            e0 *= gv[i].x;
-            e1 *= gv[i].y;
-            const uint32_t off = sw128(t, 4 * lane);
-            uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
-            uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
-            uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
-            if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
-            const float k0 = bf_lo(kw), k1 = bf_hi(kw), m0 = mv[i].x, m1 = mv[i].y;
-            *reinterpret_cast<uint32_t *>(pq + off) = pack_bf16x2(bf_lo(qw) * e0, bf_hi(qw) * e1);
-            *reinterpret_cast<uint32_t *>(pe + off) = pack_bf16x2(bf_lo(bw) * k0 * e0, bf_hi(bw) * k1 * e1);
-            *reinterpret_cast<uint32_t *>(pk + off) = pack_bf16x2(k0 * m0, k1 * m1);
-            *reinterpret_cast<uint32_t *>(kh + t * D + ch) = pack_bf16x2(k0 * m0 * gam0, k1 * m1 * gam1);
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 32) {  // a chunk past the factors' range: the chain steps it token by token, and the
-                      // token-level kernel rewrites its gradients
-        const int tokm = s_tok[0] | s_tok[1];
-        reinterpret_cast<int *>(a.gam + cidx * GSTR)[D] = tokm;
-        if (tokm) a.flist[1 + atomicAdd(a.flist, 1)] = (int)(blockIdx.x + gridDim.x * blockIdx.y);
-    }
-    // ---- [A; P] = [E~; Q~] K~^T
-    if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + TM_AP, sdesc_sw128(sb + QE + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                   sdesc_sw128(sb + KT + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_AP, ks > 0);
-        mma_commit(&bar_ap);
-    }
-    wait_or_abort(&bar_ap, 0, a.status, &s_abort);
-    tc_fence_after();
-    if (warp < 8) {  // A -> fp32 scratch (strictly lower), P -> bf16 tile (lower incl.)
-        const int quarter = warp & 3, half = warp >> 2;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t r[32];
-        tmem_ld32(tmem + TM_AP + 32 * half + lane_off, r);
-        tmem_wait_ld();
-        const int row = quarter * 32 + lane;
-        if (row < 64) {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int j = 32 * half + u;
-                sA[row * LDA + j] = (j < row) ? __uint_as_float(r[u]) : 0.f;
-            }
-        } else {
-            const int t = row - 64;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i0 = 32 * half + 8 * m + 2 * e;
-                    w4[e] = pack_bf16x2((i0 <= t) ? __uint_as_float(r[8 * m + 2 * e]) : 0.f,
-                                        (i0 + 1 <= t) ? __uint_as_float(r[8 * m + 2 * e + 1]) : 0.f);
-                }
-                *reinterpret_cast<uint4 *>(sm + PP + sw128(t, 64 * half + 16 * m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- T = (I + A)^-1 on warps 0-3; Z^T = dO^T P issued meanwhile
-    if (warp < 4) {
-        wm::solve_unit_lower64<LDA>(sA, sT, warp, lane, [] { named_bar(1, 128); });
-    } else if (tid == 128) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + TM_ZT, sdesc_sw128(sb + DO + ks * 2048, 8192, 1024), sdesc_sw128(sb + PP + ks * 2048, 8192, 1024),
-                   IDESC_Z, ks > 0);
-        mma_commit(&bar_z);
-    }
-    __syncthreads();
-    // ---- T -> bf16 tile and global (threads 0-255), P -> global (threads 256-511): 16 columns each
-    {
-        const int i = tid >> 2, jq = tid & 3;
-        {
-            uint32_t w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int j0 = 16 * jq + 2 * e;
-                w8[e] = pack_bf16x2((j0 <= i) ? sT[i * LDA + j0] : 0.f, (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f);
-            }
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const uint4 v = make_uint4(w8[4 * h2], w8[4 * h2 + 1], w8[4 * h2 + 2], w8[4 * h2 + 3]);
-                *reinterpret_cast<uint4 *>(sm + TT + sw128(i, 32 * jq + 16 * h2)) = v;
-                *reinterpret_cast<uint4 *>(a.Tm + cidx * C * C + i * C + 16 * jq + 8 * h2) = v;
-            }
-        }
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2)
-            *reinterpret_cast<uint4 *>(a.Pm + cidx * C * C + i * C + 16 * jq + 8 * h2) =
-                *reinterpret_cast<const uint4 *>(sm + PP + sw128(i, 32 * jq + 16 * h2));
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    // ---- W^T = E~^T T^T
-    if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + TM_WT, sdesc_sw128(sb + QE + ks * 2048, 16384, 1024), sdesc_sw128(sb + TT + ks * 32, 16, 1024),
-                   IDESC_W, ks > 0);
-        mma_commit(&bar_w);
-    }
-    // -Z^T -> bf16 A operand (warps 0-3: lanes d_v, 64 columns)
-    wait_or_abort(&bar_z, 0, a.status, &s_abort);
-    tc_fence_after();
-    if (warp < 4) {
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t r[32], pk[16];
-            tmem_ld32(tmem + TM_ZT + 32 * h2 + lane_off, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(-__uint_as_float(r[2 * e]), -__uint_as_float(r[2 * e + 1]));
-            tmem_st16(tmem + TM_ZB + 16 * h2 + lane_off, pk);
-        }
-        tmem_wait_st();
-    }
-    // W^T -> bf16 tile (rows d_k, the B operand of R^T) and global (warps 4-7)
-    wait_or_abort(&bar_w, 0, a.status, &s_abort);
-    tc_fence_after();
-    if (warp >= 4 && warp < 8) {
-        const int quarter = warp & 3, c = quarter * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        __nv_bfloat16 *wg = a.W + cidx * C * D + (size_t)c * C;  // W^T [d_k][C]
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t r[32];
-            tmem_ld32(tmem + TM_WT + 32 * h2 + lane_off, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[8 * m]), __uint_as_float(r[8 * m + 1])),
-                                           pack_bf16x2(__uint_as_float(r[8 * m + 2]), __uint_as_float(r[8 * m + 3])),
-                                           pack_bf16x2(__uint_as_float(r[8 * m + 4]), __uint_as_float(r[8 * m + 5])),
-                                           pack_bf16x2(__uint_as_float(r[8 * m + 6]), __uint_as_float(r[8 * m + 7])));
-                *reinterpret_cast<uint4 *>(sm + WT + sw128(c, 64 * h2 + 16 * m)) = v;
-                *reinterpret_cast<uint4 *>(wg + 32 * h2 + 8 * m) = v;
-            }
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- R^T = dO^T Q~ + (-Z^T) W
-    if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + TM_RT, sdesc_sw128(sb + DO + ks * 2048, 8192, 1024),
-                   sdesc_sw128(sb + QE + 8192 + ks * 2048, 16384, 1024), IDESC_R1, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tmem + TM_RT, tmem + TM_ZB + 8 * ks, sdesc_sw128(sb + WT + ks * 32, 16, 1024), IDESC_R2, 1);
-        mma_commit(&bar_r);
-    }
-    wait_or_abort(&bar_r, 0, a.status, &s_abort);
-    tc_fence_after();
-#pragma unroll
-    for (int cq2 = 0; cq2 < 2; ++cq2) {  // R^T -> bf16, global [d_v][d_k]: warp = lane quarter x 2 column blocks
-        const int quarter = warp & 3, cq = 2 * (warp >> 2) + cq2, j = quarter * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t r[32];
-        tmem_ld32(tmem + TM_RT + 32 * cq + lane_off, r);
-        tmem_wait_ld();
-        __nv_bfloat16 *rt = a.Rt + cidx * D * D + (size_t)j * D + 32 * cq;
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<uint4 *>(rt + 8 * m) =
-                make_uint4(pack_bf16x2(__uint_as_float(r[8 * m]), __uint_as_float(r[8 * m + 1])),
-                           pack_bf16x2(__uint_as_float(r[8 * m + 2]), __uint_as_float(r[8 * m + 3])),
-                           pack_bf16x2(__uint_as_float(r[8 * m + 4]), __uint_as_float(r[8 * m + 5])),
-                           pack_bf16x2(__uint_as_float(r[8 * m + 6]), __uint_as_float(r[8 * m + 7])));
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, TM_COLS);
     }
 }
 
@@ -541,20 +204,22 @@ bwd_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const BwdTcArgs a)
 namespace chain_tc {
 constexpr uint32_t ST_K = 0;          // K^ [64][128] (two 8 KiB atoms)
 constexpr uint32_t ST_W = 16384;      // W^T [128 d_k][64 tokens] (one 16 KiB atom)
-constexpr uint32_t ST_R = 32768;      // R^T [128][128] (two 16 KiB atoms)
-constexpr uint32_t ST_G = 65536;      // gamma [128] fp32
+constexpr uint32_t ST_DO = 32768;     // dO [64 tokens][128 d_v] (two 8 KiB atoms)
+constexpr uint32_t ST_M = 49152;      // M^T [128 d_k][64 tokens] (one 16 KiB atom)
+constexpr uint32_t ST_G = 65536;      // gamma [128] fp32, then the token-mode flag
 constexpr uint32_t STAGE = 66560;     // 65 KiB, 1024-aligned
 constexpr int kStages = 3;
 constexpr uint32_t SMEM = kStages * STAGE + 1024;
-constexpr uint32_t STAGE_BYTES = 16384 + 16384 + 32768 + GSTR * 4;
-constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_ZB = 256, TM_COLS = 512;
+constexpr uint32_t STAGE_BYTES = 16384 + 16384 + 16384 + 16384 + GSTR * 4;
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_ZB = 256, TM_R = 288, TM_COLS = 512;
 constexpr uint32_t IDESC_Z = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, 0, 0);
+constexpr uint32_t IDESC_R = tc::idesc_bf16(128, 128, 1, 0);  // R^T = dO^T M: A (dO^T) MN-major
 constexpr int kThreads = 256;
 }  // namespace chain_tc
 
 struct ChainMaps {
-    CUtensorMap kh, wt, rt;
+    CUtensorMap kh, wt, mt, dO;
 };
 
 __global__ void __launch_bounds__(chain_tc::kThreads, 1)
@@ -564,7 +229,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_full[kStages], bar_z, bar_s;
+    __shared__ __align__(8) uint64_t bar_full[kStages], bar_z, bar_s, bar_r;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -580,6 +245,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
         for (int s = 0; s < kStages; ++s) mbar_init(&bar_full[s], 1);
         mbar_init(&bar_z, 1);
         mbar_init(&bar_s, 1);
+        mbar_init(&bar_r, 1);
         s_abort = 0;
         fence_mbar_init();
     }
@@ -591,20 +257,34 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    // chunk ci's K^, W^T, R^T, gamma into stage s
+    // chunk ci's K^, W^T, dO, M^T, gamma into stage s
     auto load = [&](int ci, int s) {
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         uint8_t *st = sm + s * STAGE;
         mbar_expect_tx(&bar_full[s], STAGE_BYTES);
         for (int at = 0; at < 2; ++at) {
             tma_load_2d(st + ST_K + at * 8192, &maps.kh, at * 64, (int)(cidx * C), &bar_full[s]);
-            tma_load_2d(st + ST_R + at * 16384, &maps.rt, at * 64, (int)(cidx * D), &bar_full[s]);
+            tma_load_3d(st + ST_DO + at * 8192, &maps.dO, at * 64, hh, sp.bos + ci * C, &bar_full[s]);
         }
         tma_load_2d(st + ST_W, &maps.wt, 0, (int)(cidx * D), &bar_full[s]);
+        tma_load_2d(st + ST_M, &maps.mt, 0, (int)(cidx * D), &bar_full[s]);
         bulk_load(st + ST_G, a.gam + cidx * GSTR, GSTR * 4, &bar_full[s]);
+    };
+    // R^T = dO^T M of the chunk in stage s (state-independent) into TM_R; thread 0, after the
+    // stage has landed and TM_R's last value was read
+    auto issue_r = [&](int s, uint32_t par) {
+        wait_or_abort(&bar_full[s], par, a.status, &s_abort);
+        tc_fence_after();
+        const uint32_t sb = smem_u32(sm + s * STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + TM_R, sdesc_sw128(sb + ST_DO + ks * 2048, 8192, 1024), sdesc_sw128(sb + ST_M + ks * 32, 16, 1024),
+                   IDESC_R, ks > 0);
+        mma_commit(&bar_r);
     };
     if (tid == 0) {
         for (int u = 0; u < 2 && u < nc; ++u) load(nc - 1 - u, u);
+        if (nc > 0) issue_r(0, 0);
     }
     // dS^T from dS_T (stored [c][j]: dS^T[j][c] = dS_T[c][j]); this thread: row j, 64 columns
     {
@@ -632,6 +312,12 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
         const uint8_t *st = sm + s * STAGE;
         if (tid == 0 && ci - 2 >= 0) load(ci - 2, (it + 2) % kStages);  // stage freed by step it - 1
         wait_or_abort(&bar_full[s], par, a.status, &s_abort);
+        wait_or_abort(&bar_r, (uint32_t)it & 1u, a.status, &s_abort);  // this chunk's R^T
+        tc_fence_after();
+        // the next chunk's R^T, issued right after this chunk's Z^T (products below) or its tokens
+        auto issue_next_r = [&]() {
+            if (tid == 0 && ci >= 1) issue_r((it + 1) % kStages, (uint32_t)((it + 1) / kStages) & 1u);
+        };
         if (reinterpret_cast<const int *>(st + ST_G)[D]) {
             // ---- a chunk whose decay is too strong for the factors: dS^T to registers (this
             //      thread: row `row`, columns 64 half ..), its bf16 copy to global as dS_n, then the
@@ -692,6 +378,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
+            issue_next_r();
             continue;
         }
         // ---- dS_n^T: bf16 to global and to TMEM; dS_n^T Diag(gamma) + R^T back into the accumulator
@@ -710,18 +397,14 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                 for (int m = 0; m < 4; ++m)
                     *reinterpret_cast<uint4 *>(dsn + 32 * h2 + 8 * m) =
                         make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                uint32_t rr[32];  // R^T row `row`, columns 64 half + 32 h2 ..
+                tmem_ld32(tmem + TM_R + 64 * half + 32 * h2 + lane_off, rr);
+                tmem_wait_ld();
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {  // R^T row `row`, columns 64 half + 32 h2 + 8 m .. + 7
-                    const uint4 rv = *reinterpret_cast<const uint4 *>(st + ST_R + half * 16384 +
-                                                                      sw128(row, (32 * h2 + 8 * m) * 2));
-                    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int u = 8 * m + 2 * e;
-                        const float2 g2 = *reinterpret_cast<const float2 *>(gam + 32 * h2 + u);
-                        r[u] = __float_as_uint(__uint_as_float(r[u]) * g2.x + bf_lo(rw[e]));
-                        r[u + 1] = __float_as_uint(__uint_as_float(r[u + 1]) * g2.y + bf_hi(rw[e]));
-                    }
+                for (int u = 0; u < 32; u += 2) {
+                    const float2 g2 = *reinterpret_cast<const float2 *>(gam + 32 * h2 + u);
+                    r[u] = __float_as_uint(fmaf(__uint_as_float(r[u]), g2.x, __uint_as_float(rr[u])));
+                    r[u + 1] = __float_as_uint(fmaf(__uint_as_float(r[u + 1]), g2.y, __uint_as_float(rr[u + 1])));
                 }
                 tmem_st32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
             }
@@ -739,6 +422,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                        IDESC_Z, ks > 0);
             mma_commit(&bar_z);
         }
+        issue_next_r();  // runs on the tensor pipe while Z^T is read back
         wait_or_abort(&bar_z, ph, a.status, &s_abort);
         tc_fence_after();
         {  // -Z^T -> bf16 A operand: warp = lane quarter x 32 columns
@@ -1336,11 +1020,30 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 
 size_t bwd_tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
 
+// The backward's per-chunk factors in workspace ws (layout l), written by the forward's states run.
+static BwdFactors bwd_factors(const Problem &p, const BwdTcLayout &l, char *base)
+{
+    BwdFactors f;
+    f.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
+    f.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
+    f.Mc = reinterpret_cast<__nv_bfloat16 *>(base + l.Mc);
+    f.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
+    f.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
+    f.gam = reinterpret_cast<float *>(base + l.gam);
+    f.flist = reinterpret_cast<int *>(base + l.flist);
+    f.nchb = (int)chunk_bound(p);
+    return f;
+}
+
 cudaError_t launch_fwd_save(const Problem &p, void *o, float *S_T, void *ws, int *status, cudaStream_t s)
 {
     if (p.cu_seqlens || (p.D != 128 && p.D != 64)) return cudaErrorNotSupported;
     const BwdTcLayout l = tc_layout(p);
-    return launch_fwd_tc(p, o, S_T, reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + l.states), status, s);
+    char *base = static_cast<char *>(ws);
+    const BwdFactors f = bwd_factors(p, l, base);
+    cudaError_t e = cudaMemsetAsync(f.flist, 0, sizeof(int), s);  // no chunk runs token by token yet
+    if (e != cudaSuccess) return e;
+    return launch_fwd_tc(p, o, S_T, reinterpret_cast<__nv_bfloat16 *>(base + l.states), status, s, nullptr, &f);
 }
 
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
@@ -1377,7 +1080,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
     a.gam = reinterpret_cast<float *>(base + l.gam);
     a.flist = reinterpret_cast<int *>(base + l.flist);
-    a.Rt = reinterpret_cast<__nv_bfloat16 *>(base + l.Rt);
+    a.Mc = reinterpret_cast<__nv_bfloat16 *>(base + l.Mc);
     a.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
     a.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
     a.dSn = reinterpret_cast<__nv_bfloat16 *>(base + l.dSn);
@@ -1391,31 +1094,21 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.status = status;
 
     cudaError_t e = cudaSuccess;
-    if (!states_saved || p.cu_seqlens) {  // chunk-boundary states, unless the forward recorded them
-        e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s);
+    if (!states_saved || p.cu_seqlens) {
+        // the forward in states mode: chunk-boundary states and the per-chunk factors of the chain
+        // and the gradient kernel, unless the forward recorded them (gdn2_chunk_fwd_save)
+        const BwdFactors f = bwd_factors(a.pr, l, base);
+        if ((e = cudaMemsetAsync(f.flist, 0, sizeof(int), s)) != cudaSuccess) return e;  // no chunk flagged yet
+        e = launch_fwd_tc(a.pr, nullptr, nullptr, a.states, status, s, nullptr, &f);
         if (e != cudaSuccess) return e;
     }
-    const dim3 nblk((unsigned)chunk_bound(p), (unsigned)p.H);
-    if ((e = cudaMemsetAsync(a.flist, 0, sizeof(int), s)) != cudaSuccess) return e;  // no chunk flagged yet
-    {  // prep on the tensor cores: one block per (chunk, head)
-        PrepMaps maps;
-        memset(&maps, 0, sizeof(maps));
-        const int rows = (int)token_rows(p);
-        if (!make_map(&maps.q, p.q, false, 1, rows, p.H, p.D) || !make_map(&maps.k, p.k, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D))
-            return cudaErrorInvalidValue;
-        if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_prep_tc_kernel), (int)prep_tc::SMEM)) != cudaSuccess)
-            return e;
-        bwd_prep_tc_kernel<<<nblk, prep_tc::kThreads, prep_tc::SMEM, s>>>(maps, a);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {  // the dS chain on the tensor cores: one block per (batch, head)
         ChainMaps cm;
         memset(&cm, 0, sizeof(cm));
         const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p);
         if (!make_map_2d(&cm.kh, a.Kh, D, nchunk * C, 64, C) || !make_map_2d(&cm.wt, a.W, C, nchunk * D, 64, D) ||
-            !make_map_2d(&cm.rt, a.Rt, D, nchunk * D, 64, D))
+            !make_map_2d(&cm.mt, a.Mc, C, nchunk * D, 64, D) ||
+            !make_map(&cm.dO, d_o, false, 1, (int)token_rows(p), p.H, p.D))
             return cudaErrorInvalidValue;
         if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_chain_tc_kernel), (int)chain_tc::SMEM)) != cudaSuccess)
             return e;

@@ -89,6 +89,7 @@ constexpr uint32_t TM_COLS = 512;
 constexpr uint32_t IDESC_N64 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_N128 = idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t IDESC_N128_BMN = idesc_bf16(128, 128, 0, 1);
+constexpr uint32_t IDESC_W = idesc_bf16(128, 64, 1, 0);  // W^T = E~^T T^T: A (E~^T) MN-major
 
 // Register split: the launch holds 512 x 128 registers; M takes 152 per thread and
 // E 104 (256 x 152 + 256 x 104 = 65536, exactly the launch's total).
@@ -110,6 +111,7 @@ struct TcParams {
     const int *chunk_off;    // variable length with states only: first chunk of each sequence
     int g_scalar;            // log alpha is one value per (token, head), [rows, H]: a scalar decay
     ScanArgs scan;           // chunk-parallel scan instances only (gdn2_internal.cuh)
+    BwdFactors bw;           // kBw instances: the backward's per-chunk factors
 };
 
 struct TcMaps {
@@ -173,10 +175,12 @@ __device__ __forceinline__ void lane_sum16(float (&v)[16], int lane)
 // squares come from the decay folding's loads; the reduction over the lanes runs while the
 // [A; P] product is in flight.  The sigmoid of b is applied in the decay folding, that of w
 // in the X = w.v fold.
+// kBw: the states run of the backward, which also writes the backward's per-chunk factors
+// (BwdFactors) from the M group, whose products leave it time while E prepares the next chunk.
 // kScan: a pass of the chunk-parallel scan (ScanArgs): every CTA decodes its segment, its state
 // source and destination, whether it writes o, and whether it runs the transition (the
 // chain's linear part on the identity: X = 0, S = I at the segment start).
-template <bool kGScalar, int DIN, int kPro, bool kScan = false>
+template <bool kGScalar, int DIN, int kPro, bool kScan = false, bool kBw = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -335,6 +339,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 dst[u] = make_uint4(pack_bf16x2(Sv[8 * u], Sv[8 * u + 1]), pack_bf16x2(Sv[8 * u + 2], Sv[8 * u + 3]),
                                     pack_bf16x2(Sv[8 * u + 4], Sv[8 * u + 5]), pack_bf16x2(Sv[8 * u + 6], Sv[8 * u + 7]));
         };
+        // first chunk of this sequence over all sequences (the backward's per-chunk slots)
+        const size_t bw_first = p.chunk_off ? (size_t)p.chunk_off[bb] : (size_t)bb * nchunks;
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
@@ -410,6 +416,11 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 }
                 tmem_wait_st();
                 if (p.states) store_state(Sf, ci + 1);
+                if (kBw && tid == 128) {  // the backward steps this chunk token by token too
+                    const size_t cidx = bw_first * p.H + (size_t)hh * nchunks + ci;
+                    reinterpret_cast<int *>(p.bw.gam + cidx * kGamStride)[D] = 1;
+                    p.bw.flist[1 + atomicAdd(p.bw.flist, 1)] = (int)(bw_first + ci + p.bw.nchb * hh);
+                }
                 tc_fence_before();
                 named_sync(1, kGroup);
             } else {
@@ -485,7 +496,15 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 for (int ks = 0; ks < 4; ++ks) {
                     mma_ts(tmem + TM_DS, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + ok + ks * 2048, 8192, 1024),
                            IDESC_N128_BMN, ks > 0);
-                    mma_ts(tmem + TM_O, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64, 1);
+                    if (o_on)
+                        mma_ts(tmem + TM_O, tmem + TM_UB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024),
+                               IDESC_N64, 1);
+                }
+                if (kBw) {  // the backward's W^T = E~^T T^T (d_k rows) into TM_UT, read back by now
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(tmem + TM_UT, sdesc_sw128(sbase + oqe + ks * 2048, 16384, 1024),
+                               sdesc_sw128(sbase + ott + ks * 32, 16, 1024), IDESC_W, ks > 0);
                 }
                 mma_commit(&bar_mma);
             }
@@ -508,6 +527,92 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
                 }
                 if (p.states) store_state(Sf, ci + 1);
+            }
+            if (kBw) {
+                // ---- the backward's per-chunk factors, state-independent: W^T, M^T = Q~^T - W^T P^T
+                //      (the chain forms R^T = dO^T M from them), K^ = K~ Diag(gamma), T, P, gamma and
+                //      the token-mode flag.  TMEM lanes are d_k channels here (jrow), columns tokens.
+                const BwdFactors &bw = p.bw;
+                const size_t cidx = bw_first * p.H + (size_t)hh * nchunks + ci;
+                {  // W^T -> bf16 to global, and -W^T as the A operand of M's product
+                    uint32_t r[32], pk[16], nk[16];
+                    tmem_ld32(tmem + TM_UT + 32 * half + lane_off, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float w0 = __uint_as_float(r[2 * e]), w1 = __uint_as_float(r[2 * e + 1]);
+                        pk[e] = pack_bf16x2(w0, w1);
+                        nk[e] = pack_bf16x2(-w0, -w1);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(bw.W + (cidx * D + jrow) * C + 32 * half);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) dst[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                    tmem_st16(tmem + TM_YB + 16 * half + lane_off, nk);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                named_sync(1, kGroup);
+                if (tid == 0) {  // (-W^T) P^T into TM_YO's first half (free since the Y read-back)
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ts(tmem + TM_YO, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64,
+                               ks > 0);
+                    mma_commit(&bar_mma);
+                }
+                {  // meanwhile K^ = K~ gamma ([t][d_k] row-major), T and P ([64][64]), gamma and the flag
+                    const int t = tid >> 2, cq = tid & 3;
+                    const float *gm = sGam + buf * 128 + 32 * cq;
+                    const uint8_t *kt = sm + ok + (cq >> 1) * 8192;
+                    uint4 *kd = reinterpret_cast<uint4 *>(bw.Kh + (cidx * C + t) * D + 32 * cq);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(kt + sw128(t, 64 * (cq & 1) + 16 * m));
+                        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t o4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float k0 = __uint_as_float(vw[e] << 16), k1 = __uint_as_float(vw[e] & 0xffff0000u);
+                            o4[e] = pack_bf16x2(k0 * gm[8 * m + 2 * e], k1 * gm[8 * m + 2 * e + 1]);
+                        }
+                        kd[m] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    }
+                    uint4 *td = reinterpret_cast<uint4 *>(bw.Tm + (cidx * C + t) * C + 16 * cq);
+                    uint4 *pd = reinterpret_cast<uint4 *>(bw.Pm + (cidx * C + t) * C + 16 * cq);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        td[h2] = *reinterpret_cast<const uint4 *>(sm + ott + sw128(t, 32 * cq + 16 * h2));
+                        pd[h2] = *reinterpret_cast<const uint4 *>(sm + opt + sw128(t, 32 * cq + 16 * h2));
+                    }
+                    if (tid < 128) bw.gam[cidx * kGamStride + tid] = sGam[buf * 128 + tid];
+                    if (tid == 128) {
+                        const int tokm = s_tok[buf][0] | s_tok[buf][1];
+                        reinterpret_cast<int *>(bw.gam + cidx * kGamStride)[D] = tokm;
+                        if (tokm) bw.flist[1 + atomicAdd(bw.flist, 1)] = (int)(bw_first + ci + bw.nchb * hh);
+                    }
+                }
+                if (!mbar_wait(&bar_mma, mma_phase)) fail();
+                mma_phase ^= 1;
+                tc_fence_after();
+                {  // M^T = Q~^T + (-W^T P^T) -> bf16 to global
+                    uint32_t r[32], pk[16];
+                    tmem_ld32(tmem + TM_YO + 32 * half + lane_off, r);
+                    tmem_wait_ld();
+                    const uint8_t *qt = sm + oqe + 8192 + (jrow >> 6) * 16384;
+                    const uint32_t cb2 = (jrow & 63) * 2;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int t0 = 32 * half + 2 * e;
+                        const float q0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qt + sw128(t0, cb2)));
+                        const float q1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qt + sw128(t0 + 1, cb2)));
+                        pk[e] = pack_bf16x2(q0 + __uint_as_float(r[2 * e]), q1 + __uint_as_float(r[2 * e + 1]));
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(bw.Mc + (cidx * D + jrow) * C + 32 * half);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) dst[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                }
+                tc_fence_before();
+                named_sync(1, kGroup);  // T and P are read before the output tile goes over them
             }
             if (o_on) {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
                 uint32_t r[32];
@@ -812,7 +917,7 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, 
 }
 
 cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 *states, int *status,
-                          cudaStream_t s, const ScanArgs *scan)
+                          cudaStream_t s, const ScanArgs *scan, const BwdFactors *bw)
 {
     // d = 64 runs zero-padded to 128 (see the kernel); chunk-boundary states keep the padded
     // 128 x 128 layout (they are the backward's internal workspace)
@@ -829,7 +934,11 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         return cudaErrorInvalidValue;
     TcParams prm{pr.B, pr.T, pr.H, (const __nv_bfloat16 *)pr.q, (const __nv_bfloat16 *)pr.k, (const __nv_bfloat16 *)pr.b,
                  pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
-                 pr.g_scalar ? 1 : 0, ScanArgs{}};
+                 pr.g_scalar ? 1 : 0, ScanArgs{}, BwdFactors{}};
+    if (bw) {  // the backward's factors: states runs with per-channel decay and no prologue only
+        if (!states || pr.g_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
+        prm.bw = *bw;
+    }
     int grid = pr.B * pr.H;
     if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)
         if (pr.g_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C ||
@@ -845,6 +954,7 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         return cudaGetLastError();
     };
     if (scan) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, true>) : run(fwd_tc_kernel<false, 64, 0, true>);
+    if (bw) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, false, true>) : run(fwd_tc_kernel<false, 64, 0, false, true>);
     if (pr.prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
     auto by_pro = [&](auto gs, auto dn) -> cudaError_t {
         constexpr bool kGS = decltype(gs)::value;

@@ -170,6 +170,20 @@ struct ScanArgs {
     const float *sstart;
 };
 
+// The backward's per-chunk factors, written by the tensor-core forward in states mode for the
+// dS chain and the gradient kernel (chunk slots of chunk_slot): W^T [D][C], K^ = K~ Diag(gamma)
+// [C][D], M^T [D][C] with M = Q~ - P W (so that R = Q~^T dO - W^T P^T dO = M^T dO), T = (I + A)^-1
+// and P [C][C], all bf16 with D = 128; gamma [kGamStride] fp32 with the chunk's token-mode flag
+// (an int) after the D values; flist[0] counts the chunks that run token by token and flist[1 ..]
+// lists them as tasks gc + nchb h (gc the chunk over all sequences).
+constexpr int kGamStride = 128 + 4;
+struct BwdFactors {
+    __nv_bfloat16 *W = nullptr, *Kh = nullptr, *Mc = nullptr, *Tm = nullptr, *Pm = nullptr;
+    float *gam = nullptr;
+    int *flist = nullptr;
+    int nchb = 0;
+};
+
 // Workspace of the chunk-parallel scan for this problem; 0 when the scan is not used for it
 // (variable length, scalar decay, prologue, more than 48 chains, or short sequences).
 size_t fwd_scan_workspace_bytes(const Problem &p);
@@ -194,7 +208,7 @@ cudaError_t launch_prologue_bwd(bool fp32, size_t rows, int D, bool norm, const 
                                 cudaStream_t s);
 cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *states, int *status,
                           cudaStream_t s,
-                          const ScanArgs *scan = nullptr);
+                          const ScanArgs *scan = nullptr, const BwdFactors *bw = nullptr);
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
