@@ -116,6 +116,7 @@ struct TcParams {
 
 struct TcMaps {
     CUtensorMap q, k, v, b, w, g, o;
+    CUtensorMap kh, wt, mt, tm, pm;  // kBw: stores of the backward's factors (2-D, 128-byte swizzle)
 };
 
 // barrier over `count` threads (id 0 is __syncthreads)
@@ -531,10 +532,14 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             if (kBw) {
                 // ---- the backward's per-chunk factors, state-independent: W^T, M^T = Q~^T - W^T P^T
                 //      (the chain forms R^T = dO^T M from them), K^ = K~ Diag(gamma), T, P, gamma and
-                //      the token-mode flag.  TMEM lanes are d_k channels here (jrow), columns tokens.
+                //      the token-mode flag.  W^T goes over the consumed E~ tile, K^ over K~ and M^T over
+                //      Q~ (128-byte swizzled, as TMA stores read them), and TMA stores take them and the
+                //      T, P tiles to global.  TMEM lanes are d_k channels here (jrow), columns tokens.
                 const BwdFactors &bw = p.bw;
                 const size_t cidx = bw_first * p.H + (size_t)hh * nchunks + ci;
-                {  // W^T -> bf16 to global, and -W^T as the A operand of M's product
+                uint8_t *const pe = sm + oqe, *const pq = sm + oqe + 8192, *const pkt = sm + ok;
+                const uint32_t arow = (jrow & 63), aoff = (jrow >> 6) * 16384;  // this row in a [128][64] E~ / Q~ tile
+                {  // W^T -> bf16 into the E~ tile, and -W^T as the A operand of M's product
                     uint32_t r[32], pk[16], nk[16];
                     tmem_ld32(tmem + TM_UT + 32 * half + lane_off, r);
                     tmem_wait_ld();
@@ -544,30 +549,21 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                         pk[e] = pack_bf16x2(w0, w1);
                         nk[e] = pack_bf16x2(-w0, -w1);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(bw.W + (cidx * D + jrow) * C + 32 * half);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) dst[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4 *>(pe + aoff + sw128(arow, 64 * half + 16 * m)) =
+                            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                     tmem_st16(tmem + TM_YB + 16 * half + lane_off, nk);
                     tmem_wait_st();
                 }
-                tc_fence_before();
-                named_sync(1, kGroup);
-                if (tid == 0) {  // (-W^T) P^T into TM_YO's first half (free since the Y read-back)
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ts(tmem + TM_YO, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64,
-                               ks > 0);
-                    mma_commit(&bar_mma);
-                }
-                {  // meanwhile K^ = K~ gamma ([t][d_k] row-major), T and P ([64][64]), gamma and the flag
+                {  // K^ = K~ gamma in place: thread (token t, 32 channels)
                     const int t = tid >> 2, cq = tid & 3;
                     const float *gm = sGam + buf * 128 + 32 * cq;
-                    const uint8_t *kt = sm + ok + (cq >> 1) * 8192;
-                    uint4 *kd = reinterpret_cast<uint4 *>(bw.Kh + (cidx * C + t) * D + 32 * cq);
+                    uint8_t *kt = pkt + (cq >> 1) * 8192;
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(kt + sw128(t, 64 * (cq & 1) + 16 * m));
+                        uint4 *pv = reinterpret_cast<uint4 *>(kt + sw128(t, 64 * (cq & 1) + 16 * m));
+                        const uint4 v = *pv;
                         const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
                         uint32_t o4[4];
 #pragma unroll
@@ -575,30 +571,42 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                             const float k0 = __uint_as_float(vw[e] << 16), k1 = __uint_as_float(vw[e] & 0xffff0000u);
                             o4[e] = pack_bf16x2(k0 * gm[8 * m + 2 * e], k1 * gm[8 * m + 2 * e + 1]);
                         }
-                        kd[m] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                        *pv = make_uint4(o4[0], o4[1], o4[2], o4[3]);
                     }
-                    uint4 *td = reinterpret_cast<uint4 *>(bw.Tm + (cidx * C + t) * C + 16 * cq);
-                    uint4 *pd = reinterpret_cast<uint4 *>(bw.Pm + (cidx * C + t) * C + 16 * cq);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_sync(1, kGroup);
+                if (tid == 0) {  // (-W^T) P^T into TM_YO's first half (free since the Y read-back); the stores
+                    tc_fence_after();
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        td[h2] = *reinterpret_cast<const uint4 *>(sm + ott + sw128(t, 32 * cq + 16 * h2));
-                        pd[h2] = *reinterpret_cast<const uint4 *>(sm + opt + sw128(t, 32 * cq + 16 * h2));
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ts(tmem + TM_YO, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64,
+                               ks > 0);
+                    mma_commit(&bar_mma);
+                    const int wrow = (int)(cidx * D), trow = (int)(cidx * C);
+                    for (int a = 0; a < 2; ++a) {
+                        tma_store_2d(&maps.wt, pe + a * 16384, 0, wrow + 64 * a);
+                        tma_store_2d(&maps.kh, pkt + a * 8192, 64 * a, trow);
                     }
-                    if (tid < 128) bw.gam[cidx * kGamStride + tid] = sGam[buf * 128 + tid];
-                    if (tid == 128) {
-                        const int tokm = s_tok[buf][0] | s_tok[buf][1];
-                        reinterpret_cast<int *>(bw.gam + cidx * kGamStride)[D] = tokm;
-                        if (tokm) bw.flist[1 + atomicAdd(bw.flist, 1)] = (int)(bw_first + ci + bw.nchb * hh);
-                    }
+                    tma_store_2d(&maps.tm, sm + ott, 0, trow);
+                    tma_store_2d(&maps.pm, sm + opt, 0, trow);
+                    bulk_commit();
+                }
+                if (tid < 128) bw.gam[cidx * kGamStride + tid] = sGam[buf * 128 + tid];
+                if (tid == 128) {
+                    const int tokm = s_tok[buf][0] | s_tok[buf][1];
+                    reinterpret_cast<int *>(bw.gam + cidx * kGamStride)[D] = tokm;
+                    if (tokm) bw.flist[1 + atomicAdd(bw.flist, 1)] = (int)(bw_first + ci + bw.nchb * hh);
                 }
                 if (!mbar_wait(&bar_mma, mma_phase)) fail();
                 mma_phase ^= 1;
                 tc_fence_after();
-                {  // M^T = Q~^T + (-W^T P^T) -> bf16 to global
+                {  // M^T = Q~^T + (-W^T P^T) -> bf16 over the Q~ tile, once every thread has read it
                     uint32_t r[32], pk[16];
                     tmem_ld32(tmem + TM_YO + 32 * half + lane_off, r);
                     tmem_wait_ld();
-                    const uint8_t *qt = sm + oqe + 8192 + (jrow >> 6) * 16384;
+                    const uint8_t *qt = pq + (jrow >> 6) * 16384;
                     const uint32_t cb2 = (jrow & 63) * 2;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -607,12 +615,21 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                         const float q1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qt + sw128(t0 + 1, cb2)));
                         pk[e] = pack_bf16x2(q0 + __uint_as_float(r[2 * e]), q1 + __uint_as_float(r[2 * e + 1]));
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(bw.Mc + (cidx * D + jrow) * C + 32 * half);
+                    named_sync(1, kGroup);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) dst[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4 *>(pq + aoff + sw128(arow, 64 * half + 16 * m)) =
+                            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                 }
+                fence_proxy_async_smem();
                 tc_fence_before();
-                named_sync(1, kGroup);  // T and P are read before the output tile goes over them
+                named_sync(1, kGroup);
+                if (tid == 0) {
+                    for (int a = 0; a < 2; ++a) tma_store_2d(&maps.mt, pq + a * 16384, 0, (int)(cidx * D) + 64 * a);
+                    bulk_commit();
+                    if (o_on) bulk_wait_read0();  // T and P are read before the output tile goes over them
+                }
+                if (o_on) named_sync(1, kGroup);
             }
             if (o_on) {  // O^T -> bf16 output tile (row-major [t][channel]) over this chunk's T/P tiles
                 uint32_t r[32];
@@ -938,6 +955,11 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     if (bw) {  // the backward's factors: states runs with per-channel decay and no prologue only
         if (!states || pr.g_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
         prm.bw = *bw;
+        const uint64_t nchunk = (uint64_t)pr.H * chunk_bound(pr);
+        if (!make_map_2d(&maps.kh, bw->Kh, D, nchunk * C, 64, C) || !make_map_2d(&maps.wt, bw->W, C, nchunk * D, 64, 64) ||
+            !make_map_2d(&maps.mt, bw->Mc, C, nchunk * D, 64, 64) || !make_map_2d(&maps.tm, bw->Tm, C, nchunk * C, 64, C) ||
+            !make_map_2d(&maps.pm, bw->Pm, C, nchunk * C, 64, C))
+            return cudaErrorInvalidValue;
     }
     int grid = pr.B * pr.H;
     if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)
