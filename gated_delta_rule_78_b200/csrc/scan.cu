@@ -11,12 +11,14 @@
 //   pass 1 (one launch): segments 1 .. nseg-1 from their start states with their output.
 // Each combine step costs a d_k x d_k x d_v product, and pass 0 runs two chains per middle
 // segment, so the scan pays only where the serial chain leaves SMs idle (kScanSlots: the
-// B200's 148 SMs, one CTA each), for segments of at least kScanMinChunks chunks:
-// * up to 48 chains: n equal segments, n the largest (up to kScanMaxSegments) whose pass 0,
-//   (2n - 3) CTAs per chain, fits one wave; pass 0 and pass 1 each take one segment's time;
-// * 49 to 74 chains: segment 0 twice as long as the two after it.  Pass 0 has 3 CTAs per
-//   chain; the first wave holds every segment-0 CTA and half of the middle ones, and the
-//   other half runs when those finish, within segment 0's time.  T = 4 L gives 2 L + L.
+// B200's 148 SMs, one CTA each).  The plan: segment 0 of k L chunks, then m middle segments and
+// a last one of L chunks each (at least kScanMinChunks), with k and m chosen to minimise the
+// modelled time over C chains.  Pass 0's segment-0 CTAs run first and hold C SMs for k L; the
+// 2 C m middle CTAs run on the other SMs in ceil(2 C m / (148 - C)) waves of L; pass 1 runs
+// C (m + 1) CTAs in ceil(C (m + 1) / 148) waves of L:
+//   time = max(k, waves_0) L + waves_1 L   against the serial chain's (k + m + 1) L.
+// For example 32 chains take k = 2, m = 3 (0.5 of the serial time; three equal segments give
+// 0.67), 64 chains k = 2, m = 1 (0.75), and 16 chains six equal segments (0.33).
 #include "gdn2_internal.cuh"
 
 namespace gdn2 {
@@ -24,8 +26,7 @@ namespace {
 
 constexpr int kScanSlots = 148;
 constexpr int kScanMaxSegments = 8;
-constexpr int kScanMaxChains = kScanSlots / 3;  // equal segments: 3 CTAs per chain in pass 0
-constexpr int kScanMaxChainsLong0 = kScanSlots / 2;  // long segment 0: 2 chains' worth per wave
+constexpr int kScanMaxK = 4;                    // segment 0 at most this many segment lengths
 constexpr int kScanMinChunks = 16;              // per segment
 
 // S_start(s) for s = 1 .. nseg-1 of one (b, h), 16 state columns per block.
@@ -81,22 +82,32 @@ ScanLayout scan_layout(const Problem &p)
     ScanLayout l{};
     const int nch = (p.T + kChunk - 1) / kChunk;
     const long long chains = (long long)p.B * p.H;
-    if (p.cu_seqlens || p.g_scalar || p.prologue || nch < 3 * kScanMinChunks) return l;
-    if (chains <= kScanMaxChains) {
-        int n = 3;
-        while (n < kScanMaxSegments && chains * (2 * (n + 1) - 3) <= kScanSlots && nch >= (n + 1) * kScanMinChunks)
-            ++n;
-        l.nseg = n;
-        l.seg_len = (nch + l.nseg - 1) / l.nseg * kChunk;
-        l.seg0_len = l.seg_len;
-    } else if (chains <= kScanMaxChainsLong0 && nch >= 4 * kScanMinChunks) {
-        l.nseg = 3;
-        const int b = (nch + 3) / 4;  // chunks of segments 1 and 2; segment 0 takes the rest
-        l.seg_len = b * kChunk;
-        l.seg0_len = (nch - 2 * b) * kChunk;
-    } else {
-        return l;
+    if (p.cu_seqlens || p.g_scalar || p.prologue || nch < 3 * kScanMinChunks || chains >= kScanSlots) return l;
+    // modelled time in chunk steps of every plan (k, m); the serial chain takes nch
+    long long best = nch;
+    for (int k = 1; k <= kScanMaxK; ++k) {
+        for (int m = 1; m + 2 <= kScanMaxSegments; ++m) {
+            const int tm = (nch + k + m) / (k + m + 1);  // middle segments' chunks
+            if (tm < kScanMinChunks) continue;
+            // the rounding remainder goes to the last segment (segment 0 of k tm chunks), or else
+            // to segment 0 (every later segment of tm chunks)
+            for (int v = 0; v < 2; ++v) {
+                const int t0 = v == 0 ? k * tm : nch - (m + 1) * tm;
+                const int last = nch - t0 - m * tm;
+                if (t0 < tm || last < 1 || last > tm) continue;
+                const long long w0 = (2 * chains * m + (kScanSlots - chains) - 1) / (kScanSlots - chains);
+                const long long w1 = (chains * (m + 1) + kScanSlots - 1) / kScanSlots;
+                const long long t = (t0 > w0 * tm ? t0 : w0 * tm) + w1 * tm;
+                if (t < best) {
+                    best = t;
+                    l.nseg = m + 2;
+                    l.seg_len = tm * kChunk;
+                    l.seg0_len = t0 * kChunk;
+                }
+            }
+        }
     }
+    if (!l.nseg) return l;
     const size_t st = (size_t)p.B * p.H * p.D * p.D * sizeof(float);
     l.send0 = 0;
     l.shat = l.send0 + st;
