@@ -445,6 +445,31 @@ def run_ours(args):
                                   "algorithmic_bytes": sd_bytes,
                                   "hbm_frac": round(sd_bytes / (ms_sd * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
         del wsg
+        # ---- KDA and Gated DeltaNet shapes: b = w = beta, one value per (token, head), with the
+        #      per-channel decay (KDA) or a scalar one (Gated DeltaNet); the tensor-core forward
+        #      reads the gates as they are
+        beta = torch.sigmoid(torch.randn(B, T, H, generator=torch.Generator(device=str(dev)).manual_seed(6),
+                                         device=dev)).to(x["q"].dtype)
+        gate_pts = {}
+        for name, fl, gdec in (("kda", g.ERASE_SCALAR | g.WRITE_SCALAR, x["log_alpha"]),
+                               ("gated_deltanet", g.ERASE_SCALAR | g.WRITE_SCALAR | g.DECAY_SCALAR, gsc)):
+            wsk = torch.empty(max(16, g.gdn2_workspace_size_gated(0, fl, x["q"].dtype, B, T, H, D, D)),
+                              dtype=torch.uint8, device=dev)
+
+            def fwd_k():
+                g.gdn2_chunk_fwd_gated(x["q"], x["k"], x["v"], gdec, beta, beta, x["S0"], flags=fl, o=o, S_T=ST,
+                                       workspace=wsk)
+
+            ms_k = time_region(fwd_k, 20, 3, stream) / 20
+            assert g.gdn2_sync_status() == 0
+            kb = fwd_bytes(B, T, H, D) - B * T * H * 2 * (2 * D - 2) - (B * T * H * (4 * D - 4) if gdec is gsc else 0)
+            gate_pts[name] = {"workload": f"B={B}, T={T}, H={H}, d={D}; b = w = beta [B,T,H]" +
+                              ("; log alpha [B,T,H]" if gdec is gsc else "; log alpha per channel"),
+                              "ms": round(ms_k, 4), "tokens_per_s": round(job_rate(tokens, world, ms_k), 1),
+                              "algorithmic_bytes": kb, "hbm_frac": round(kb / (ms_k * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                              "workspace_bytes": int(wsk.numel()) if wsk.numel() > 16 else 0}
+            del wsk
+        extras.update(gate_pts)
         # ---- input prologue fused in the chunk kernel, against a separate pass + the plain forward
         xr = make_inputs(B, T, H, D, D, dtype=w["dtype"], seed=rank_seed(rank) + 31, device=str(dev), raw=True)
         pro_flags = g.QK_L2NORM | g.BW_LOGITS

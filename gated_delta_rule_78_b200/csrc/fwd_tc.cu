@@ -99,7 +99,8 @@ static_assert(kGroup * kRegM + kGroup * kRegE == kThreads * 128, "register split
 
 struct TcParams {
     int B, T, H;
-    const __nv_bfloat16 *q, *k, *b;  // read directly by chunks that run token by token
+    const __nv_bfloat16 *q, *k, *b, *w;  // read directly by chunks that run token by token; with
+                                         // kGate, b and w are one value per (token, head) [rows, H]
     const float *S0;
     const float *g;   // log alpha [B,T,H,D] fp32
     __nv_bfloat16 *o;        // may be null (states-only run)
@@ -176,12 +177,14 @@ __device__ __forceinline__ void lane_sum16(float (&v)[16], int lane)
 // squares come from the decay folding's loads; the reduction over the lanes runs while the
 // [A; P] product is in flight.  The sigmoid of b is applied in the decay folding, that of w
 // in the X = w.v fold.
+// kGate: b and w are one value per (token, head) (the KDA and Gated DeltaNet shapes): no b, w
+// tiles; E folds E~ = (b_t k) e^G with b_t from a 64-entry table per chunk, M forms X = w_t v.
 // kBw: the states run of the backward, which also writes the backward's per-chunk factors
 // (BwdFactors) from the M group, whose products leave it time while E prepares the next chunk.
 // kScan: a pass of the chunk-parallel scan (ScanArgs): every CTA decodes its segment, its state
 // source and destination, whether it writes o, and whether it runs the transition (the
 // chain's linear part on the identity: X = 0, S = I at the segment start).
-template <bool kGScalar, int DIN, int kPro, bool kScan = false, bool kBw = false>
+template <bool kGScalar, int DIN, int kPro, bool kScan = false, bool kBw = false, bool kGate = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
 {
@@ -198,6 +201,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     // kChunkDecayLimit, so the chunk runs token by token
     __shared__ int s_tok[2][2];
     __shared__ float *s_stp;  // this CTA's end-state destination (read once, at the end)
+    __shared__ __nv_bfloat16 s_bsc[2][kGate ? 64 : 1];  // kGate: b_t of the chunk, by chunk parity
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool is_m = warp < 8;
@@ -283,16 +287,25 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     // issued from an E warp that is idle during the solve.
     auto issue = [&](int ci) {
         const int y = bos + ci * C, bf = ci & 1;
-        mbar_expect_tx(&bar_in[bf], 10 * 8192);
+        mbar_expect_tx(&bar_in[bf], (kGate ? 6 : 10) * 8192);
         for (int a = 0; a < 2; ++a) {
             tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in[bf]);
-            tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in[bf]);
+            if (!kGate) tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in[bf]);
             tma_load_3d(sm + OFF_QE + bf * 32768 + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_in[bf]);
             tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in[bf]);
-            tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
+            if (!kGate) tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
         }
         if (!kGScalar)
             for (int a = 0; a < DIN / 32; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
+        if (kGate) {  // the chunk's rows of b and w ([rows, H], contiguous) into L2
+            const int rows = min(C, T - ci * C);
+            const uint32_t bytes = (uint32_t)(rows * p.H * 2) & ~15u;
+            const size_t first = (size_t)y * p.H;
+            if (bytes && ((first * 2) & 15) == 0) {
+                bulk_prefetch_l2(p.b + first, bytes);
+                bulk_prefetch_l2(p.w + first, bytes);
+            }
+        }
     };
 
     if (is_m) {
@@ -304,6 +317,17 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         auto fail = [&]() {
             s_abort_m = 1;
             atomicExch(p.status, kStatusTimeout);
+        };
+        // kGate: w_t of this warp's eight token rows (mw + 8 j) of a chunk, loaded one chunk ahead
+        __nv_bfloat16 w_next[8];
+        auto load_w = [&](int ci) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int t = mw + 8 * j;
+                w_next[j] = (kGate && ci < nchunks && ci * C + t < T)
+                                ? p.w[((size_t)bos + (size_t)ci * C + t) * p.H + hh]
+                                : __float2bfloat16_rn(0.f);
+            }
         };
         // X = w.v of chunk ci, in place of v (one token row of 64 channels per warp step)
         auto fold_value = [&](int ci) {
@@ -317,11 +341,18 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 const int a = idx >> 6, t = idx & 63;
                 const uint32_t off = a * 8192 + sw128(t, 4 * lane);
                 const uint32_t vw = *reinterpret_cast<const uint32_t *>(pv + off);
-                const uint32_t ww = *reinterpret_cast<const uint32_t *>(pw + off);
+                uint32_t ww;
+                if (kGate) {  // one w per (token, head), the same for the whole row
+                    const uint32_t w16 = (uint32_t)__bfloat16_as_ushort(w_next[it & 7]);
+                    ww = w16 | (w16 << 16);
+                } else {
+                    ww = *reinterpret_cast<const uint32_t *>(pw + off);
+                }
                 const uint32_t wg = (kPro & kProSigmoid) ? sigmoid_bf16x2(ww) : ww;
                 *reinterpret_cast<uint32_t *>(pv + off) = (t < Lc) ? bmul2(vw, wg) : 0u;
             }
         };
+        if (kGate) load_w(0);
         if (tid == 0 && nchunks > 0) issue(0);
         if (nchunks > 0) {
             if (!mbar_wait(&bar_in[0], 0)) fail();
@@ -364,6 +395,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             const int L = min(C, T - ci * C);
             const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384, ov = OFF_V + buf * 16384;
             const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
+            if (kGate) load_w(ci + 1);  // in flight during the chunk
             // ---- factors, P and T of chunk ci are ready
             if (!mbar_wait(&bar_fact[buf], (ci >> 1) & 1)) fail();
             if (s_tok[buf][0] | s_tok[buf][1]) {
@@ -385,7 +417,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                             const size_t off = ((row0 + t) * p.H + hh) * DIN + c;
                             qv = __bfloat162float(gq[off]);
                             kv = __bfloat162float(gk[off]);
-                            bv = __bfloat162float(gb[off]);
+                            bv = __bfloat162float(kGate ? gb[(row0 + t) * p.H + hh] : gb[off]);
                             gv = kGScalar ? p.g[(row0 + t) * p.H + hh] : p.g[off];
                         }
                         if (kPro & kProNorm) {
@@ -716,6 +748,10 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                                 ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * DIN))
                                 : make_float2(0.f, 0.f);
             }
+            // kGate: this chunk's b_t, one per thread of the first 64, for the table below
+            const __nv_bfloat16 bt = (kGate && etid < 64 && etid < L)
+                                         ? p.b[((size_t)bos + (size_t)ci * C + etid) * p.H + hh]
+                                         : __float2bfloat16_rn(0.f);
             if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
 #pragma unroll
@@ -726,6 +762,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 gv[i] = make_float2(a0, kGScalar ? a0 : __expf(gv[i].y));  // alpha
             }
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
+            if (kGate && etid < 64) s_bsc[buf][etid] = bt;
             named_sync(2, kGroup);
             if (s_abort_e) break;
             float sqq[16], sqk[16];  // prologue: this thread's share of |q|^2, |k|^2 per token
@@ -766,7 +803,13 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     const float m0 = mv[i].x, m1 = mv[i].y;
                     uint32_t qw = *reinterpret_cast<const uint32_t *>(pq + off);
                     uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
-                    uint32_t bw = *reinterpret_cast<const uint32_t *>(pe + off);
+                    uint32_t bw;
+                    if (kGate) {
+                        const uint32_t b16 = (uint32_t)__bfloat16_as_ushort(s_bsc[buf][t]);
+                        bw = b16 | (b16 << 16);
+                    } else {
+                        bw = *reinterpret_cast<const uint32_t *>(pe + off);
+                    }
                     if (t >= L) { qw = 0u; kw = 0u; bw = 0u; }
                     if (kPro & kProNorm) {
                         const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
@@ -944,16 +987,17 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     memset(&maps, 0, sizeof(maps));
     const int rows = (int)token_rows(pr);  // the maps view every tensor as [rows, H, din]
     if (!make_map(&maps.q, pr.q, false, 1, rows, pr.H, din) || !make_map(&maps.k, pr.k, false, 1, rows, pr.H, din) ||
-        !make_map(&maps.v, pr.v, false, 1, rows, pr.H, din) || !make_map(&maps.b, pr.b, false, 1, rows, pr.H, din) ||
-        !make_map(&maps.w, pr.w, false, 1, rows, pr.H, din) ||
+        !make_map(&maps.v, pr.v, false, 1, rows, pr.H, din) ||
+        (!pr.bw_scalar && !make_map(&maps.b, pr.b, false, 1, rows, pr.H, din)) ||
+        (!pr.bw_scalar && !make_map(&maps.w, pr.w, false, 1, rows, pr.H, din)) ||
         (!pr.g_scalar && !make_map(&maps.g, pr.g, true, 1, rows, pr.H, din)) ||
         (o && !make_map(&maps.o, o, false, 1, rows, pr.H, din, true)))
         return cudaErrorInvalidValue;
     TcParams prm{pr.B, pr.T, pr.H, (const __nv_bfloat16 *)pr.q, (const __nv_bfloat16 *)pr.k, (const __nv_bfloat16 *)pr.b,
-                 pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
+                 (const __nv_bfloat16 *)pr.w, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
                  pr.g_scalar ? 1 : 0, ScanArgs{}, BwdFactors{}};
-    if (bw) {  // the backward's factors: states runs with per-channel decay and no prologue only
-        if (!states || pr.g_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
+    if (bw) {  // the backward's factors: states runs with per-channel gates and no prologue only
+        if (!states || pr.g_scalar || pr.bw_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
         prm.bw = *bw;
         const uint64_t nchunk = (uint64_t)pr.H * chunk_bound(pr);
         if (!make_map_2d(&maps.kh, bw->Kh, D, nchunk * C, 64, C) || !make_map_2d(&maps.wt, bw->W, C, nchunk * D, 64, 64) ||
@@ -963,7 +1007,7 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     }
     int grid = pr.B * pr.H;
     if (scan) {  // plain gates, fixed length, no prologue; one CTA per (segment task, head)
-        if (pr.g_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C ||
+        if (pr.g_scalar || pr.bw_scalar || pr.prologue || pr.cu_seqlens || states || scan->nseg < 3 || scan->seg_len % C ||
             scan->seg0_len % C)
             return cudaErrorInvalidValue;
         prm.scan = *scan;
@@ -981,6 +1025,14 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     auto by_pro = [&](auto gs, auto dn) -> cudaError_t {
         constexpr bool kGS = decltype(gs)::value;
         constexpr int kDin = decltype(dn)::value;
+        if (pr.bw_scalar) {
+            switch (pr.prologue) {
+            case kProNorm: return run(fwd_tc_kernel<kGS, kDin, kProNorm, false, false, true>);
+            case kProSigmoid: return run(fwd_tc_kernel<kGS, kDin, kProSigmoid, false, false, true>);
+            case kProNorm | kProSigmoid: return run(fwd_tc_kernel<kGS, kDin, kProNorm | kProSigmoid, false, false, true>);
+            default: return run(fwd_tc_kernel<kGS, kDin, 0, false, false, true>);
+            }
+        }
         switch (pr.prologue) {
         case kProNorm: return run(fwd_tc_kernel<kGS, kDin, kProNorm>);
         case kProSigmoid: return run(fwd_tc_kernel<kGS, kDin, kProSigmoid>);

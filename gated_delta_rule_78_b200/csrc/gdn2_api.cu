@@ -134,7 +134,12 @@ size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 // present) as logits.  The bf16 forward with per-channel b and w applies it inside the
 // tensor-core kernel; every other call runs it as a pass into the workspace first.
 bool pro_any(int flags) { return flags & (GDN2_QK_L2NORM | GDN2_BW_LOGITS); }
-bool pro_fused(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_full(flags, 1) && gate_full(flags, 2); }
+// b and w both one value per (token, head): the bf16 forward reads them as they are
+bool bw_native(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_scalar(flags, 1) && gate_scalar(flags, 2); }
+bool pro_fused(int flags, gdn2_dtype dt)
+{
+    return dt == GDN2_BF16 && ((gate_full(flags, 1) && gate_full(flags, 2)) || bw_native(flags, dt));
+}
 // prologue mode of gate i (1 = b, 2 = w): 0 none, 1 per channel, 2 per token
 int pro_gate_mode(int flags, int i)
 {
@@ -147,7 +152,10 @@ int pro_gate_mode(int flags, int i)
 struct GatedWs {
     size_t pro[4], off[3], grad[3], core, total;
 };
-GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes, bool pro_pass)
+// The chunk forward keeps some scalar gates as they are, which then need no broadcast copy:
+// bw_kept (scalar b and w together) and decay_kept (a scalar decay, bf16).
+GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes, bool pro_pass,
+                 bool bw_kept = false, bool decay_kept = false)
 {
     GatedWs l;
     const size_t n = rows * H * D;
@@ -164,7 +172,7 @@ GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, 
     }
     for (int i = 0; i < 3; ++i) {
         l.off[i] = off;
-        if (!gate_full(flags, i)) off += round256(n * es[i]);
+        if (!gate_full(flags, i) && !(bw_kept && i > 0) && !(decay_kept && i == 0)) off += round256(n * es[i]);
     }
     for (int i = 0; i < 3; ++i) {
         l.grad[i] = off;
@@ -440,7 +448,9 @@ size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int
                                                                                 nullptr, nullptr, nullptr, nullptr))
                                    : 0;
     const bool pro_pass = pro_any(flags) && (which == 1 || !pro_fused(flags, dt));
-    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass).total;
+    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass, which == 0 && bw_native(flags, dt),
+                    which == 0 && dt == GDN2_BF16 && gate_scalar(flags, 0))
+        .total;
 }
 
 gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, int Dk, int Dv, const void *q,
@@ -454,7 +464,9 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if ((st = check_ptrs({q, k, v, o}, {S0, S_T})) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
     const bool fused = pro_any(flags) && pro_fused(flags, dt);
-    const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0, pro_any(flags) && !fused);
+    const bool native_bw = bw_native(flags, dt);
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0, pro_any(flags) && !fused, native_bw,
+                               dt == GDN2_BF16 && gate_scalar(flags, 0));
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
@@ -463,14 +475,17 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if (pro_any(flags) && !fused &&
         (st = prologue_pass(flags, dt, l, ws, (size_t)B * T, H, Dk, qq, kk, bq, wq, s)) != GDN2_OK)
         return st;
-    // a scalar decay goes to the tensor-core forward as it is (one exponential per token)
+    // a scalar decay, and scalar b and w together, go to the tensor-core forward as they are
+    // (one exponential per token; one gate value per token)
     const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16;
-    const int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
+    int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
+    if (native_bw) expand_flags &= ~(GDN2_ERASE_SCALAR | GDN2_WRITE_SCALAR);
     const void *gp[3] = {log_alpha, bq, wq};
     if ((st = expand_gates(expand_flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s)) != GDN2_OK) return st;
     gdn2::Problem p = make_problem(B, T, H, Dk, qq, kk, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S0);
-    if (native_decay || fused) {
+    if (native_decay || native_bw || fused) {
         p.g_scalar = native_decay;
+        p.bw_scalar = native_bw;
         if (fused)
             p.prologue = ((flags & GDN2_QK_L2NORM) ? gdn2::kProNorm : 0) | ((flags & GDN2_BW_LOGITS) ? gdn2::kProSigmoid : 0);
         int *status = gdn2::status_word();

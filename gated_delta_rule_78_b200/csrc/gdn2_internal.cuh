@@ -41,6 +41,7 @@ struct Problem {
     const int *cu_seqlens = nullptr;
     const int *chunk_off = nullptr;
     bool g_scalar = false;  // tensor-core forward only: log alpha is [rows, H] (one decay per head)
+    bool bw_scalar = false; // tensor-core forward only: b and w are [rows, H] (one gate value each per head)
     int prologue = 0;       // tensor-core forward only: kProNorm | kProSigmoid, applied inside the kernel
 };
 

@@ -114,6 +114,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                  ::"l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1)
                  : "memory");
 }
+// L2 prefetch of a global range (address 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Untiled bulk copy global -> shared (both addresses 16-byte aligned, bytes a multiple of 16),
 // completing `bytes` on the mbarrier.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)

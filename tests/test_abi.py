@@ -184,18 +184,23 @@ def test_prologue_arguments(lib):
 
 
 def test_forward_workspace_for_the_scan(lib):
-    # few long chains (at most 48 (batch, head) pairs, at least 48 chunks): the chunk-parallel scan
+    # few long chains: the chunk-parallel scan, (3 nseg - 4) states per chain for nseg segments,
+    # the plan chosen by the wave model of the 148 SMs
     st = 128 * 128 * 4
-    assert lib.gdn2_workspace_size(0, BF16, 2, 32768, 16, 128, 128) == 32 * st * 5
+    # 32 chains: segment 0 of twice the length, then four more (5 segments, 11 states)
+    assert lib.gdn2_workspace_size(0, BF16, 2, 32768, 16, 128, 128) == 32 * st * 11
+    # 2 chains of 48 chunks: 3 equal segments (the minimum of 16 chunks each)
     assert lib.gdn2_workspace_size(0, BF16, 1, 3072, 2, 64, 64) == 2 * 64 * 64 * 4 * 5
     assert lib.gdn2_workspace_size(0, BF16, 1, 3008, 2, 128, 128) == 0   # 47 chunks: serial
-    # 49 to 74 chains: 3 segments, the first twice as long
+    # 64 chains: 3 segments, the first twice as long (a short last one at 63 chunks)
     assert lib.gdn2_workspace_size(0, BF16, 4, 16384, 16, 128, 128) == 64 * st * 5
-    assert lib.gdn2_workspace_size(0, BF16, 4, 4032, 16, 128, 128) == 0  # 63 chunks: too short for that plan
+    assert lib.gdn2_workspace_size(0, BF16, 4, 4032, 16, 128, 128) == 64 * st * 5
     assert lib.gdn2_workspace_size(0, BF16, 5, 16384, 15, 128, 128) == 0  # 75 chains: serial
+    assert lib.gdn2_workspace_size(0, BF16, 8, 4096, 16, 128, 128) == 0   # 128 chains: serial
     assert lib.gdn2_workspace_size(0, F32, 2, 32768, 16, 128, 128) == 0   # fp32 path: serial
-    # fewer chains get more segments: 16 chains fill 148 slots with 6 segments (9 CTAs each)
-    assert lib.gdn2_workspace_size(0, BF16, 1, 32768, 16, 128, 128) == 16 * st * (3 * 6 - 4)
+    # fewer chains get more segments: 16 chains, segment 0 of twice the length and seven more
+    # (8 segments; the model gives 171 chunk steps against 172 for six equal ones and 512 serial)
+    assert lib.gdn2_workspace_size(0, BF16, 1, 32768, 16, 128, 128) == 16 * st * (3 * 8 - 4)
 
 
 def test_training_pair_arguments(lib):
