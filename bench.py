@@ -107,24 +107,34 @@ def device_code_sha(text: str, kernel_def: str):
     return hashlib.sha256(text[:j].encode()).hexdigest()
 
 
+def _code_matches(src_name: str, kernel_def: str, sha: str) -> bool:
+    src = os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", src_name)
+    if not os.path.exists(src):
+        return False
+    try:
+        return device_code_sha(open(src).read(), kernel_def) == sha
+    except ValueError:
+        return False
+
+
 def kernel_traffic(kernel_src: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the kernel's
-    current device code (same SHA-256 of the file up to the kernel's end), else None."""
+    """DRAM bytes per launch (or per call, for a record that spans several kernels) from the
+    committed ncu summary, if it was taken on the current device code of every kernel it covers
+    (same SHA-256 of each file up to the kernel's end), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    src = os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", kernel_src)
-    e = d.get(kernel_src)
-    if not e or not os.path.exists(src):
+    e = json.load(open(p)).get(kernel_src)
+    if not e:
         return None
+    if "kernels" in e:  # several kernels: every one must still be the captured code
+        ok = all(_code_matches(k["file"], k["kernel_def"], k["sha256_device"]) for k in e["kernels"])
+        return e.get("bytes_per_call") if ok else None
     try:
-        h = device_code_sha(open(src).read(), e["kernel_def"])
-    except (KeyError, ValueError):
+        ok = _code_matches(kernel_src, e["kernel_def"], e["sha256_device"])
+    except KeyError:
         return None
-    if e.get("sha256_device") != h:
-        return None
-    return e.get("bytes_per_launch")
+    return e.get("bytes_per_launch") if ok else None
 
 
 # ------------------------------------------------------------------ clocks
@@ -352,10 +362,11 @@ def run_ours(args):
         assert g.gdn2_sync_status() == 0
         bb = bwd_bytes(B, T, H, D)
         extras["fwd_bwd"] = {"bwd_ms": round(ms_bwd, 4), "steps": ksteps,
-                             "bwd_roofline": roofline(bb, ms_bwd, pk), "bwd_launches": 1 + 3}
+                             "bwd_roofline": roofline(bb, ms_bwd, pk, kernel_traffic("backward") if args.workload == "layer_4k" else None),
+                             "bwd_launches": 1 + 3}
         if ms_fwd is not None:
-            # a training step: the forward records the chunk-boundary states into the backward's
-            # workspace, and the backward skips its own states pass
+            # a training step: the forward records the chunk-boundary states and chunk factors into
+            # the backward's workspace, and the backward skips its own states pass
             o_tr = torch.empty_like(x["v"])
             S_tr = torch.empty_like(x["S0"])
 

@@ -23,11 +23,11 @@
 // products used and gamma dgamma from the state-update part of dK~ (its own accumulator): the
 // cancelling pairs then cancel exactly, and dlog alpha keeps its accuracy at any decay.
 //
-// The only serial dependence is the dS chain.  With W = T E~ and K^ = K~ Diag(gamma):
-//   dS = (Diag(gamma) - W^T K^) dS_n + R,   R = Q~^T dO - W^T (P^T dO) = M^T dO,  M = Q~ - P W,
+// The only serial dependence is the dS chain.  With W = T E~ and Gm = Diag(gamma):
+//   dS = Gm dS_n - W^T K~ (Gm dS_n) + R,   R = Q~^T dO - W^T (P^T dO) = M^T dO,  M = Q~ - P W,
 // so the work splits into three launches:
 //   1. the tensor-core forward in states mode: S^T (bf16) at every chunk boundary, and from
-//      its M group the state-independent factors W^T, K^, gamma, M^T, T and P of every chunk
+//      its M group the state-independent factors W^T, K~, gamma, M^T, T and P of every chunk
 //      (BwdFactors), formed where the chunk's Q~, E~, K~, T and P already are;
 //   2. bwd_chain_tc_kernel, one CTA per (batch, head): the reverse dS chain with dS^T
 //      kept in TMEM, R^T = dO^T M formed on the tensor pipe beside it; stores dS_n per chunk;
@@ -57,15 +57,16 @@ constexpr int GSTR = kGamStride;  // per-chunk record of gamma: D floats, then t
 
 // ------------------------------------------------------------------ workspace
 struct BwdTcLayout {
-    size_t coff, states, flist, W, Kh, gam, Mc, Tm, Pm, dSn, scratch, total;
+    size_t coff, states, flist, W, Kt, gam, Mc, Tm, Pm, dSn, scratch, total;
     int tok_blocks;  // blocks of the token-level gradient kernel
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Per (batch, head) and chunk: states S^T bf16 (nchunks + 1 entries), W^T bf16 [D][C],
-// K^ bf16 [C][D], gamma and the chunk's token-mode flag [GSTR] fp32, M^T bf16 [D][C], T and P
-// bf16 [C][C], dS_n^T bf16 [D][D].  flist: the count and the list of the chunk tasks that run
+// K~ bf16 [C][D], gamma and the chunk's token-mode flag [GSTR] fp32, M^T bf16 [D][C], T and P
+// bf16 [C][C], (Diag(gamma) dS_n)^T bf16 [D][D] (dS_n^T as is for chunks stepped token by
+// token).  flist: the count and the list of the chunk tasks that run
 // token by token.  Variable length puts chunk_off first; chunk lists are sized by the chunk
 // bound.  The token-level gradient kernel's scratch reuses W .. M^T, which only the chain reads
 // (one block's scratch at least; past the end of the workspace when that region is smaller).
@@ -78,7 +79,7 @@ BwdTcLayout tc_layout(const Problem &p)
     l.states = off; off += H * nbound * D * D * 2;
     l.flist = off;  off += round256((1 + H * nchunk) * 4);
     l.W = off;      off += H * nchunk * C * D * 2;
-    l.Kh = off;     off += H * nchunk * C * D * 2;
+    l.Kt = off;     off += H * nchunk * C * D * 2;
     l.gam = off;    off += round256(H * nchunk * GSTR * 4);
     l.Mc = off;     off += H * nchunk * D * C * 2;
     l.Tm = off;     off += H * nchunk * C * C * 2;
@@ -105,7 +106,7 @@ struct BwdTcArgs {
     const __nv_bfloat16 *q, *k, *v, *b, *w, *dO;
     const float *g;
     const float *dS_T;  // may be null
-    __nv_bfloat16 *states, *W, *Kh, *Tm, *Pm, *dSn;
+    __nv_bfloat16 *states, *W, *Kt, *Tm, *Pm, *dSn;
     float *gam;          // [chunk][GSTR]: gamma, then the chunk's token-mode flag
     int *flist;          // flist[0]: count of the chunks that run token by token, then their tasks
     __nv_bfloat16 *Mc;  // M^T per chunk, bf16 (R^T = dO^T M)
@@ -196,13 +197,14 @@ __device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, in
 // ================================================================== 3. chain on the tensor cores
 // One CTA per (batch, head).  dS^T (d_v x d_k, fp32) lives in TMEM as an MMA accumulator, one
 // row per lane.  Per chunk, newest first:
-//   read dS_n^T: bf16 copy to global (the gradient kernel's dS_n) and to TMEM (A operand);
-//     dS_n^T Diag(gamma) + R^T back into the accumulator;
-//   Z^T = dS_n^T K^^T                    M d_v, N 64, K d_k   (A from TMEM)
+//   read dS_n^T and scale its d_k columns: (Gm dS_n)^T to global in bf16 (the gradient kernel
+//     takes it as it is) and to TMEM (A operand); (Gm dS_n)^T + R^T back into the accumulator;
+//   Z^T = (Gm dS_n)^T K~^T               M d_v, N 64, K d_k   (A from TMEM)
 //   dS^T += (-Z^T) W                     M d_v, N d_k, K 64   (A = -Z^T bf16 from TMEM)
-// K^, W^T, R^T and gamma arrive by TMA in a three-stage ring, two chunks ahead.
+// with R^T = dO^T M formed a chunk ahead on the tensor pipe.  K~, W^T, dO, M^T and gamma arrive
+// by TMA in a three-stage ring, two chunks ahead.
 namespace chain_tc {
-constexpr uint32_t ST_K = 0;          // K^ [64][128] (two 8 KiB atoms)
+constexpr uint32_t ST_K = 0;          // K~ [64][128] (two 8 KiB atoms)
 constexpr uint32_t ST_W = 16384;      // W^T [128 d_k][64 tokens] (one 16 KiB atom)
 constexpr uint32_t ST_DO = 32768;     // dO [64 tokens][128 d_v] (two 8 KiB atoms)
 constexpr uint32_t ST_M = 49152;      // M^T [128 d_k][64 tokens] (one 16 KiB atom)
@@ -219,7 +221,7 @@ constexpr int kThreads = 256;
 }  // namespace chain_tc
 
 struct ChainMaps {
-    CUtensorMap kh, wt, mt, dO;
+    CUtensorMap kt, wt, mt, dO;
 };
 
 __global__ void __launch_bounds__(chain_tc::kThreads, 1)
@@ -257,13 +259,13 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    // chunk ci's K^, W^T, dO, M^T, gamma into stage s
+    // chunk ci's K~, W^T, dO, M^T, gamma into stage s
     auto load = [&](int ci, int s) {
         const size_t cidx = chunk_slot(a.pr, n, hh, nc, ci);
         uint8_t *st = sm + s * STAGE;
         mbar_expect_tx(&bar_full[s], STAGE_BYTES);
         for (int at = 0; at < 2; ++at) {
-            tma_load_2d(st + ST_K + at * 8192, &maps.kh, at * 64, (int)(cidx * C), &bar_full[s]);
+            tma_load_2d(st + ST_K + at * 8192, &maps.kt, at * 64, (int)(cidx * C), &bar_full[s]);
             tma_load_3d(st + ST_DO + at * 8192, &maps.dO, at * 64, hh, sp.bos + ci * C, &bar_full[s]);
         }
         tma_load_2d(st + ST_W, &maps.wt, 0, (int)(cidx * D), &bar_full[s]);
@@ -381,7 +383,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
             issue_next_r();
             continue;
         }
-        // ---- dS_n^T: bf16 to global and to TMEM; dS_n^T Diag(gamma) + R^T back into the accumulator
+        // ---- (Gm dS_n)^T: bf16 to global and to TMEM; (Gm dS_n)^T + R^T back into the accumulator
         {
             const float *gam = reinterpret_cast<const float *>(st + ST_G) + 64 * half;
             __nv_bfloat16 *dsn = a.dSn + cidx * D * D + (size_t)row * D + 64 * half;
@@ -389,30 +391,29 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
             for (int h2 = 0; h2 < 2; ++h2) {
                 uint32_t r[32], pk[16];
                 tmem_ld32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-                tmem_st16(tmem + TM_SB + 32 * half + 16 * h2 + lane_off, pk);
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4 *>(dsn + 32 * h2 + 8 * m) =
-                        make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                 uint32_t rr[32];  // R^T row `row`, columns 64 half + 32 h2 ..
                 tmem_ld32(tmem + TM_R + 64 * half + 32 * h2 + lane_off, rr);
                 tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 32; u += 2) {
                     const float2 g2 = *reinterpret_cast<const float2 *>(gam + 32 * h2 + u);
-                    r[u] = __float_as_uint(fmaf(__uint_as_float(r[u]), g2.x, __uint_as_float(rr[u])));
-                    r[u + 1] = __float_as_uint(fmaf(__uint_as_float(r[u + 1]), g2.y, __uint_as_float(rr[u + 1])));
+                    const float s0 = __uint_as_float(r[u]) * g2.x, s1 = __uint_as_float(r[u + 1]) * g2.y;
+                    pk[u >> 1] = pack_bf16x2(s0, s1);
+                    r[u] = __float_as_uint(s0 + __uint_as_float(rr[u]));
+                    r[u + 1] = __float_as_uint(s1 + __uint_as_float(rr[u + 1]));
                 }
+                tmem_st16(tmem + TM_SB + 32 * half + 16 * h2 + lane_off, pk);
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(dsn + 32 * h2 + 8 * m) =
+                        make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                 tmem_st32(tmem + TM_S + 64 * half + 32 * h2 + lane_off, r);
             }
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
-        // ---- Z^T = dS_n^T K^^T
+        // ---- Z^T = (Gm dS_n)^T K~^T
         if (tid == 0) {
             tc_fence_after();
             const uint32_t kb = smem_u32(st + ST_K);
@@ -492,7 +493,7 @@ constexpr uint32_t RK = 16384;    // k -> K~
 constexpr uint32_t RB = 32768;    // b -> E~
 constexpr uint32_t GG = 49152;    // log alpha fp32 [64][128]: four 8 KiB boxes of 32 channels
 constexpr uint32_t SS = 81920;    // S^T [128][128] (atoms 16 KiB apart); after the S products: raw q, k
-constexpr uint32_t DS = 114688;   // dS_n^T -> (Gm dS_n)^T; after its products: raw b
+constexpr uint32_t DS = 114688;   // (Gm dS_n)^T, as the chain stored it; after its products: raw b
 constexpr uint32_t DY = 147456;   // [dO; -dY] [128][128]: atom a = dO rows 0-63 then -dY rows 64-127
 constexpr uint32_t TT = 180224;   // T [64][64]; after dY: U~ [64][128] over T and P; after U~'s
 constexpr uint32_t PP = 188416;   //   products: [dP; dA] [128][64]
@@ -506,7 +507,6 @@ constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
 // scratch inside the -dY rows (free until dY is read back), and in DS's second half (free once
 // (Gm dS_n)^T's products are done) for the factor chain
 constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
-constexpr uint32_t SC_GAM = DY + 8192 + 4096;    // gamma [D]
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
 constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [8][D], then [4][D] twice
 // full chunks stage dq, dk, db over the reloaded raw q, k, b and dg over v, w for the TMA stores
@@ -636,7 +636,6 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     // ---- decay folding in place: thread (channel pair cp, token group g8 of 8)
     const int cp = tid & 63, g8 = tid >> 6;
     float *sTot = reinterpret_cast<float *>(sm + SC_TOT);
-    float *sGam = reinterpret_cast<float *>(sm + SC_GAM);
     wait_or_abort(&bar_in0, ph, a.status, &s_abort);
     {
         const bool ch_ok = 2 * cp < a.din;
@@ -649,7 +648,6 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                         : make_float2(0.f, 0.f);
         }
         decay_pair8(gl, eG, emG, tot, cp, g8, sTot);
-        if (g8 == 0) *reinterpret_cast<float2 *>(sGam + 2 * cp) = make_float2(__expf(tot.x), __expf(tot.y));
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int t = 8 * g8 + i;
@@ -677,28 +675,21 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             mma_ss(tmem + TM_Y, sdesc_sw128(sb + SS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                    sdesc_sw128(sb + RB + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), IDESC_KK, ks > 0);
     }
-    // ---- dS_n^T -> (Gm dS_n)^T in place; gamma dgamma's part gamma rowsum(dS_n . S) from the column
-    //      sums of dS_n^T . S^T
+    // ---- gamma dgamma's part gamma rowsum(dS_n . S) = rowsum((Gm dS_n) . S), from the column sums
+    //      of (Gm dS_n)^T . S^T (the chain stored dS_n already scaled by gamma)
     {
         float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float gm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gm[e] = sGam[8 * dch + e];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int j = (tid >> 4) + 32 * u;
-            uint4 *p = reinterpret_cast<uint4 *>(sm + DS + (dch >> 3) * 16384 + sw128(j, (dch & 7) * 16));
-            const uint4 dv4 = *p, sv4 = ssv[u];
+            const uint4 dv4 = *reinterpret_cast<const uint4 *>(sm + DS + (dch >> 3) * 16384 + sw128(j, (dch & 7) * 16));
+            const uint4 sv4 = ssv[u];
             const uint32_t dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w}, sw[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
-            uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float d0 = bf_lo(dw[e]), d1 = bf_hi(dw[e]);
-                part[2 * e] += d0 * bf_lo(sw[e]);
-                part[2 * e + 1] += d1 * bf_hi(sw[e]);
-                o[e] = pack_bf16x2(d0 * gm[2 * e], d1 * gm[2 * e + 1]);
+                part[2 * e] += bf_lo(dw[e]) * bf_lo(sw[e]);
+                part[2 * e + 1] += bf_hi(dw[e]) * bf_hi(sw[e]);
             }
-            *p = make_uint4(o[0], o[1], o[2], o[3]);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) part[e] += __shfl_xor_sync(0xffffffffu, part[e], 16);
@@ -721,7 +712,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         float s = 0.f;
 #pragma unroll
         for (int u = 0; u < 16; ++u) s += sDgp[u * D + tid];
-        reinterpret_cast<float *>(sm + DGF)[tid] = sGam[tid] * s;
+        reinterpret_cast<float *>(sm + DGF)[tid] = s;
     }
     // ---- dU~^T = dO^T P + (Gm dS_n)^T K~^T
     if (tid == 0) {
@@ -1025,7 +1016,7 @@ static BwdFactors bwd_factors(const Problem &p, const BwdTcLayout &l, char *base
 {
     BwdFactors f;
     f.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
-    f.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
+    f.Kt = reinterpret_cast<__nv_bfloat16 *>(base + l.Kt);
     f.Mc = reinterpret_cast<__nv_bfloat16 *>(base + l.Mc);
     f.Tm = reinterpret_cast<__nv_bfloat16 *>(base + l.Tm);
     f.Pm = reinterpret_cast<__nv_bfloat16 *>(base + l.Pm);
@@ -1077,7 +1068,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
     a.dS_T = dS_T;
     a.states = reinterpret_cast<__nv_bfloat16 *>(base + l.states);
     a.W = reinterpret_cast<__nv_bfloat16 *>(base + l.W);
-    a.Kh = reinterpret_cast<__nv_bfloat16 *>(base + l.Kh);
+    a.Kt = reinterpret_cast<__nv_bfloat16 *>(base + l.Kt);
     a.gam = reinterpret_cast<float *>(base + l.gam);
     a.flist = reinterpret_cast<int *>(base + l.flist);
     a.Mc = reinterpret_cast<__nv_bfloat16 *>(base + l.Mc);
@@ -1106,7 +1097,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         ChainMaps cm;
         memset(&cm, 0, sizeof(cm));
         const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p);
-        if (!make_map_2d(&cm.kh, a.Kh, D, nchunk * C, 64, C) || !make_map_2d(&cm.wt, a.W, C, nchunk * D, 64, D) ||
+        if (!make_map_2d(&cm.kt, a.Kt, D, nchunk * C, 64, C) || !make_map_2d(&cm.wt, a.W, C, nchunk * D, 64, D) ||
             !make_map_2d(&cm.mt, a.Mc, C, nchunk * D, 64, D) ||
             !make_map(&cm.dO, d_o, false, 1, (int)token_rows(p), p.H, p.D))
             return cudaErrorInvalidValue;

@@ -38,6 +38,7 @@
 // M owns TMEM lanes 32 (m & 3) .. +31 and column half (m >> 2) of every
 // readback and holds its 64 columns of S^T in fp32 registers.  The output tile
 // is staged in shared memory and written by a TMA store.
+#include <climits>
 #include <cuda.h>
 #include <string.h>
 
@@ -72,7 +73,8 @@ constexpr uint32_t OFF_TOT = OFF_ST + 64 * LDA * 4;  // per-group decay totals [
 constexpr uint32_t OFF_GAM = OFF_TOT + 4 * 128 * 4;  // gamma [2][128] fp32
 constexpr uint32_t OFF_NRM = OFF_GAM + 2 * 128 * 4;  // prologue: sum of squares [q|k][channel half][64] fp32
 constexpr uint32_t OFF_RN = OFF_NRM + 2 * 2 * 64 * 4;  // prologue: 1/|q|, 1/|k| [2][q|k][64] fp32
-constexpr uint32_t SMEM_USED = OFF_RN + 2 * 2 * 64 * 4;
+constexpr uint32_t OFF_ID = (OFF_RN + 2 * 2 * 64 * 4 + 1023) / 1024 * 1024;  // kBw: identity [64][64] bf16
+constexpr uint32_t SMEM_USED = OFF_ID + 8192;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for the 1024-byte alignment
 
 // TMEM columns
@@ -117,7 +119,8 @@ struct TcParams {
 
 struct TcMaps {
     CUtensorMap q, k, v, b, w, g, o;
-    CUtensorMap kh, wt, mt, tm, pm;  // kBw: stores of the backward's factors (2-D, 128-byte swizzle)
+    CUtensorMap kt, wt, mt, tm, pm;  // kBw: stores of the backward's factors (2-D, 128-byte swizzle)
+    CUtensorMap st;                  // kBw: stores of the chunk-boundary states, 64 columns x 128 rows
 };
 
 // barrier over `count` threads (id 0 is __syncthreads)
@@ -371,8 +374,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 dst[u] = make_uint4(pack_bf16x2(Sv[8 * u], Sv[8 * u + 1]), pack_bf16x2(Sv[8 * u + 2], Sv[8 * u + 3]),
                                     pack_bf16x2(Sv[8 * u + 4], Sv[8 * u + 5]), pack_bf16x2(Sv[8 * u + 6], Sv[8 * u + 7]));
         };
+        // kBw: this thread's row of the bf16 S^T into a [128 rows][64 columns] staging tile (128-byte
+        // swizzle, as the TMA store of maps.st reads it); the two column halves go out one after
+        // the other through the same tile
+        auto stage_state = [&](const float *Sv, uint8_t *tile) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4 *>(tile + sw128(jrow, 16 * u)) =
+                    make_uint4(pack_bf16x2(Sv[8 * u], Sv[8 * u + 1]), pack_bf16x2(Sv[8 * u + 2], Sv[8 * u + 3]),
+                               pack_bf16x2(Sv[8 * u + 4], Sv[8 * u + 5]), pack_bf16x2(Sv[8 * u + 6], Sv[8 * u + 7]));
+        };
         // first chunk of this sequence over all sequences (the backward's per-chunk slots)
         const size_t bw_first = p.chunk_off ? (size_t)p.chunk_off[bb] : (size_t)bb * nchunks;
+        // row of maps.st where the state at chunk boundary idx starts
+        auto state_row = [&](int idx) { return (int)(((bw_first + bb) * p.H + (size_t)hh * (nchunks + 1) + idx) * D); };
         float Sf[64];  // S^T[jrow][64 half + i]
 #pragma unroll
         for (int i = 0; i < 64; ++i)
@@ -387,6 +402,15 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
         }
         tmem_wait_st();
+        if (kBw) {  // the 64 x 64 identity (B operand, 128-byte swizzle) of M^T = Q~^T I - W^T P^T
+            for (int c = tid; c < 64 * 8; c += kGroup) {
+                const int r = c >> 3, k8 = c & 7;
+                const uint32_t one = (r >> 3) != k8 ? 0u : (r & 1) ? 0x3f800000u : 0x00003f80u, wi = (r & 7) >> 1;
+                *reinterpret_cast<uint4 *>(sm + OFF_ID + sw128(r, 16 * k8)) =
+                    make_uint4(wi == 0 ? one : 0u, wi == 1 ? one : 0u, wi == 2 ? one : 0u, wi == 3 ? one : 0u);
+            }
+            fence_proxy_async_smem();
+        }
         tc_fence_before();
         named_sync(1, kGroup);
         uint32_t mma_phase = 0;
@@ -559,17 +583,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(Sf[32 * h2 + 2 * e], Sf[32 * h2 + 2 * e + 1]);
                     tmem_st16(tmem + TM_SBF + 32 * half + 16 * h2 + lane_off, pk);
                 }
-                if (p.states) store_state(Sf, ci + 1);
+                // the chunk-end state (kBw): column half 0 through the consumed X tile now, half 1
+                // once that store has read it
+                if (kBw && half == 0) stage_state(Sf, sm + ov);
             }
             if (kBw) {
                 // ---- the backward's per-chunk factors, state-independent: W^T, M^T = Q~^T - W^T P^T
-                //      (the chain forms R^T = dO^T M from them), K^ = K~ Diag(gamma), T, P, gamma and
-                //      the token-mode flag.  W^T goes over the consumed E~ tile, K^ over K~ and M^T over
-                //      Q~ (128-byte swizzled, as TMA stores read them), and TMA stores take them and the
-                //      T, P tiles to global.  TMEM lanes are d_k channels here (jrow), columns tokens.
+                //      (the chain forms R^T = dO^T M from them), K~, T, P, gamma and the token-mode
+                //      flag.  W^T goes over the consumed E~ tile and M^T over Q~ (128-byte swizzled, as
+                //      TMA stores read them), and TMA stores take them and the K~, T, P tiles to global.
+                //      TMEM lanes are d_k channels here (jrow), columns tokens.
                 const BwdFactors &bw = p.bw;
                 const size_t cidx = bw_first * p.H + (size_t)hh * nchunks + ci;
                 uint8_t *const pe = sm + oqe, *const pq = sm + oqe + 8192, *const pkt = sm + ok;
+                const int srow = state_row(ci + 1);
                 const uint32_t arow = (jrow & 63), aoff = (jrow >> 6) * 16384;  // this row in a [128][64] E~ / Q~ tile
                 {  // W^T -> bf16 into the E~ tile, and -W^T as the A operand of M's product
                     uint32_t r[32], pk[16], nk[16];
@@ -588,38 +615,26 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     tmem_st16(tmem + TM_YB + 16 * half + lane_off, nk);
                     tmem_wait_st();
                 }
-                {  // K^ = K~ gamma in place: thread (token t, 32 channels)
-                    const int t = tid >> 2, cq = tid & 3;
-                    const float *gm = sGam + buf * 128 + 32 * cq;
-                    uint8_t *kt = pkt + (cq >> 1) * 8192;
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        uint4 *pv = reinterpret_cast<uint4 *>(kt + sw128(t, 64 * (cq & 1) + 16 * m));
-                        const uint4 v = *pv;
-                        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t o4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float k0 = __uint_as_float(vw[e] << 16), k1 = __uint_as_float(vw[e] & 0xffff0000u);
-                            o4[e] = pack_bf16x2(k0 * gm[8 * m + 2 * e], k1 * gm[8 * m + 2 * e + 1]);
-                        }
-                        *pv = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                    }
-                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 named_sync(1, kGroup);
-                if (tid == 0) {  // (-W^T) P^T into TM_YO's first half (free since the Y read-back); the stores
+                if (tid == 0) {  // M^T = Q~^T I + (-W^T) P^T into TM_YO's first half (free since the Y read-back)
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_ts(tmem + TM_YO, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64,
-                               ks > 0);
+                        mma_ss(tmem + TM_YO, sdesc_sw128(sbase + oqe + 8192 + ks * 2048, 16384, 1024),
+                               sdesc_sw128(sbase + OFF_ID + ks * 32, 16, 1024), IDESC_W, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ts(tmem + TM_YO, tmem + TM_YB + 8 * ks, sdesc_sw128(sbase + opt + ks * 32, 16, 1024), IDESC_N64, 1);
                     mma_commit(&bar_mma);
+                    // the stores: state columns 0-63 as a group of its own (its tile is refilled first)
+                    tma_store_2d(&maps.st, sm + ov, 0, srow);
+                    bulk_commit();
                     const int wrow = (int)(cidx * D), trow = (int)(cidx * C);
                     for (int a = 0; a < 2; ++a) {
                         tma_store_2d(&maps.wt, pe + a * 16384, 0, wrow + 64 * a);
-                        tma_store_2d(&maps.kh, pkt + a * 8192, 64 * a, trow);
+                        tma_store_2d(&maps.kt, pkt + a * 8192, 64 * a, trow);
                     }
                     tma_store_2d(&maps.tm, sm + ott, 0, trow);
                     tma_store_2d(&maps.pm, sm + opt, 0, trow);
@@ -634,25 +649,18 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 if (!mbar_wait(&bar_mma, mma_phase)) fail();
                 mma_phase ^= 1;
                 tc_fence_after();
-                {  // M^T = Q~^T + (-W^T P^T) -> bf16 over the Q~ tile, once every thread has read it
+                {  // M^T -> bf16 over the Q~ tile (the product has read it)
                     uint32_t r[32], pk[16];
                     tmem_ld32(tmem + TM_YO + 32 * half + lane_off, r);
                     tmem_wait_ld();
-                    const uint8_t *qt = pq + (jrow >> 6) * 16384;
-                    const uint32_t cb2 = (jrow & 63) * 2;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int t0 = 32 * half + 2 * e;
-                        const float q0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qt + sw128(t0, cb2)));
-                        const float q1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qt + sw128(t0 + 1, cb2)));
-                        pk[e] = pack_bf16x2(q0 + __uint_as_float(r[2 * e]), q1 + __uint_as_float(r[2 * e + 1]));
-                    }
-                    named_sync(1, kGroup);
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
 #pragma unroll
                     for (int m = 0; m < 4; ++m)
                         *reinterpret_cast<uint4 *>(pq + aoff + sw128(arow, 64 * half + 16 * m)) =
                             make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
                 }
+                if (tid == 0) bulk_wait_read1();  // state columns 0-63 have left their tile
                 fence_proxy_async_smem();
                 tc_fence_before();
                 named_sync(1, kGroup);
@@ -660,6 +668,15 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     for (int a = 0; a < 2; ++a) tma_store_2d(&maps.mt, pq + a * 16384, 0, (int)(cidx * D) + 64 * a);
                     bulk_commit();
                     if (o_on) bulk_wait_read0();  // T and P are read before the output tile goes over them
+                }
+                if (half == 1) {  // state columns 64-127 through the same tile; thread 128 owns their store
+                    stage_state(Sf, sm + ov);
+                    fence_proxy_async_smem();
+                    named_sync(4, kGroup / 2);
+                    if (tid == kGroup / 2) {
+                        tma_store_2d(&maps.st, sm + ov, 64, srow);
+                        bulk_commit();
+                    }
                 }
                 if (o_on) named_sync(1, kGroup);
             }
@@ -699,6 +716,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 if (!mbar_wait(&bar_in[buf ^ 1], ((ci + 1) >> 1) & 1)) fail();
                 fold_value(ci + 1);
             }
+            if (kBw && tid == kGroup / 2) bulk_wait_read0();  // the state columns 64-127 have left their tile
             fence_proxy_async_smem();
             named_sync(1, kGroup);
             if (tid == 0) {
@@ -712,7 +730,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             for (int i = 0; i < 64; ++i)
                 if (64 * half + i < DIN && jrow < DIN) st_dst[(64 * half + i) * DIN + jrow] = Sf[i];
         }
-        if (tid == 0) bulk_wait0();
+        if (tid == 0 || (kBw && tid == kGroup / 2)) bulk_wait0();
     } else {
         // =========== E group: decay folding, [A; P] and T = (I+A)^-1, one chunk ahead of M ===========
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegE) : "memory");
@@ -1000,9 +1018,11 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         if (!states || pr.g_scalar || pr.bw_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
         prm.bw = *bw;
         const uint64_t nchunk = (uint64_t)pr.H * chunk_bound(pr);
-        if (!make_map_2d(&maps.kh, bw->Kh, D, nchunk * C, 64, C) || !make_map_2d(&maps.wt, bw->W, C, nchunk * D, 64, 64) ||
+        const uint64_t state_rows = (uint64_t)pr.H * (chunk_bound(pr) + pr.B) * D;  // TMA coordinates are 32-bit
+        if (state_rows > (uint64_t)INT_MAX ||
+            !make_map_2d(&maps.kt, bw->Kt, D, nchunk * C, 64, C) || !make_map_2d(&maps.wt, bw->W, C, nchunk * D, 64, 64) ||
             !make_map_2d(&maps.mt, bw->Mc, C, nchunk * D, 64, 64) || !make_map_2d(&maps.tm, bw->Tm, C, nchunk * C, 64, C) ||
-            !make_map_2d(&maps.pm, bw->Pm, C, nchunk * C, 64, C))
+            !make_map_2d(&maps.pm, bw->Pm, C, nchunk * C, 64, C) || !make_map_2d(&maps.st, states, D, state_rows, 64, D))
             return cudaErrorInvalidValue;
     }
     int grid = pr.B * pr.H;

@@ -172,14 +172,14 @@ struct ScanArgs {
 };
 
 // The backward's per-chunk factors, written by the tensor-core forward in states mode for the
-// dS chain and the gradient kernel (chunk slots of chunk_slot): W^T [D][C], K^ = K~ Diag(gamma)
-// [C][D], M^T [D][C] with M = Q~ - P W (so that R = Q~^T dO - W^T P^T dO = M^T dO), T = (I + A)^-1
-// and P [C][C], all bf16 with D = 128; gamma [kGamStride] fp32 with the chunk's token-mode flag
+// dS chain and the gradient kernel (chunk slots of chunk_slot): W^T [D][C], K~ [C][D], M^T [D][C]
+// with M = Q~ - P W (so that R = Q~^T dO - W^T P^T dO = M^T dO), T = (I + A)^-1 and P [C][C], all
+// bf16 with D = 128; gamma [kGamStride] fp32 with the chunk's token-mode flag
 // (an int) after the D values; flist[0] counts the chunks that run token by token and flist[1 ..]
 // lists them as tasks gc + nchb h (gc the chunk over all sequences).
 constexpr int kGamStride = 128 + 4;
 struct BwdFactors {
-    __nv_bfloat16 *W = nullptr, *Kh = nullptr, *Mc = nullptr, *Tm = nullptr, *Pm = nullptr;
+    __nv_bfloat16 *W = nullptr, *Kt = nullptr, *Mc = nullptr, *Tm = nullptr, *Pm = nullptr;
     float *gam = nullptr;
     int *flist = nullptr;
     int nchb = 0;

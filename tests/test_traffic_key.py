@@ -46,6 +46,29 @@ def test_committed_records_name_a_kernel_definition_present_in_their_file():
     for name, e in d.items():
         if name.startswith("_"):
             continue
-        text = open(os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", name)).read()
-        assert e["kernel_def"] in text, name
-        assert e["bytes_per_launch"] > 0
+        # a record for one kernel is named for its file; one for a call of several kernels
+        # lists them
+        kernels = e["kernels"] if "kernels" in e else [dict(e, file=name)]
+        for k in kernels:
+            text = open(os.path.join(ROOT, "gated_delta_rule_78_b200", "csrc", k["file"])).read()
+            assert k["kernel_def"] in text, (name, k["file"])
+        assert e.get("bytes_per_launch", e.get("bytes_per_call", 0)) > 0
+
+
+def test_a_record_over_several_kernels_needs_all_of_them_unchanged(tmp_path, monkeypatch):
+    import json
+    b = load_bench()
+    csrc = tmp_path / "gated_delta_rule_78_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "a.cu").write_text(SRC)
+    (csrc / "b.cu").write_text(SRC.replace("my_kernel", "other_kernel"))
+    rec = {"bytes_per_call": 123, "kernels": [
+        {"file": "a.cu", "kernel_def": DEF, "sha256_device": b.device_code_sha(SRC, DEF)},
+        {"file": "b.cu", "kernel_def": "\nother_kernel(int *p)\n",
+         "sha256_device": b.device_code_sha(SRC.replace("my_kernel", "other_kernel"), "\nother_kernel(int *p)\n")}]}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"call": rec}))
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    assert b.kernel_traffic("call") == 123
+    (csrc / "b.cu").write_text(SRC.replace("my_kernel", "other_kernel").replace("kTile = 64", "kTile = 32"))
+    assert b.kernel_traffic("call") is None
