@@ -195,9 +195,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     // Offset (not integer-cast) so that the compiler keeps the shared address space and
     // emits shared-memory instructions for every access through `sm`.
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    // bar_in[2]: a chunk's k, b, q, v, w have landed     bar_emma / bar_mma: E's / M's tcgen05 batches
-    // bar_fact[2]: E -> M, factors, P and T of a chunk   bar_mdone[2]: M -> E, a chunk's buffers are free
-    __shared__ __align__(8) uint64_t bar_in[2], bar_emma, bar_mma, bar_fact[2], bar_mdone[2];
+    // bar_in[2]: a chunk's k, b, q have landed (E)       bar_vw[2]: its v, w have landed (M)
+    // bar_emma / bar_mma: E's / M's tcgen05 batches      bar_fact[2]: E -> M, factors, P and T of a chunk
+    // bar_qk[2]: M -> E, M no longer reads a chunk's E~, Q~, K~ tiles
+    // bar_mdone[2]: M -> E, M is done with a chunk (its X, T / P tiles, w and per-parity values are free)
+    __shared__ __align__(8) uint64_t bar_in[2], bar_vw[2], bar_emma, bar_mma, bar_fact[2], bar_qk[2], bar_mdone[2];
+    __shared__ __align__(8) uint64_t bar_tfree;  // M -> E: M has read T (fp32) of the last chunk
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort_m, s_abort_e;
     // E -> M with a chunk's factors: [parity][channel half] some channel of the chunk decays past
@@ -263,8 +266,11 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         s_stp = STp;
         mbar_init(&bar_emma, 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_tfree, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_in[i], 1);
+            mbar_init(&bar_vw[i], 1);
+            mbar_init(&bar_qk[i], 1);
             mbar_init(&bar_fact[i], 1);
             mbar_init(&bar_mdone[i], 1);
         }
@@ -285,18 +291,29 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    // TMA loads of chunk ci's k, b, q, v, w into the buffers of parity ci & 1, log alpha into L2.
-    // The issuing thread may block while the TMA engine drains earlier boxes, so the loads are
-    // issued from an E warp that is idle during the solve.
-    auto issue = [&](int ci) {
+    // TMA loads of chunk ci into the buffers of parity ci & 1 as they free up: k, b, q (E's inputs,
+    // bar_in) once M's products no longer read the chunk two back (bar_qk: at its state update in
+    // the plain forward), and v, w (M's, bar_vw) with log alpha into L2 once M is done with the
+    // chunk before (bar_mdone; w is single-buffered and folded into X at the end of a chunk).  The
+    // issuing thread may block while the TMA engine drains earlier boxes, so after the first two
+    // chunks the loads go out from an E warp that is idle during the solve.
+    auto issue_qbk = [&](int ci) {
         const int y = bos + ci * C, bf = ci & 1;
-        mbar_expect_tx(&bar_in[bf], (kGate ? 6 : 10) * 8192);
+        fence_proxy_async_smem();
+        mbar_expect_tx(&bar_in[bf], (kGate ? 4 : 6) * 8192);
         for (int a = 0; a < 2; ++a) {
             tma_load_3d(sm + OFF_K + bf * 16384 + a * 8192, &maps.k, a * 64, hh, y, &bar_in[bf]);
             if (!kGate) tma_load_3d(sm + OFF_QE + bf * 32768 + a * 16384, &maps.b, a * 64, hh, y, &bar_in[bf]);
             tma_load_3d(sm + OFF_QE + bf * 32768 + 8192 + a * 16384, &maps.q, a * 64, hh, y, &bar_in[bf]);
-            tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_in[bf]);
-            if (!kGate) tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_in[bf]);
+        }
+    };
+    auto issue_vw = [&](int ci) {
+        const int y = bos + ci * C, bf = ci & 1;
+        fence_proxy_async_smem();
+        mbar_expect_tx(&bar_vw[bf], (kGate ? 2 : 4) * 8192);
+        for (int a = 0; a < 2; ++a) {
+            tma_load_3d(sm + OFF_V + bf * 16384 + a * 8192, &maps.v, a * 64, hh, y, &bar_vw[bf]);
+            if (!kGate) tma_load_3d(sm + OFF_W + a * 8192, &maps.w, a * 64, hh, y, &bar_vw[bf]);
         }
         if (!kGScalar)
             for (int a = 0; a < DIN / 32; ++a) tma_prefetch_3d(&maps.g, a * 32, hh, y);
@@ -356,14 +373,18 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             }
         };
         if (kGate) load_w(0);
-        if (tid == 0 && nchunks > 0) issue(0);
+        if (tid == 0 && nchunks > 0) {
+            issue_qbk(0);
+            issue_vw(0);
+            if (nchunks > 1) issue_qbk(1);
+        }
         if (nchunks > 0) {
-            if (!mbar_wait(&bar_in[0], 0)) fail();
+            if (!mbar_wait(&bar_vw[0], 0)) fail();
             fold_value(0);
         }
         fence_proxy_async_smem();
         named_sync(1, kGroup);
-        if (tid == 0 && nchunks > 1) issue(1);  // w(1) may only land after w(0) was folded
+        if (tid == 0 && nchunks > 1) issue_vw(1);  // w(1) may only land after w(0) was folded
         // bf16 copy of this thread's 64 entries of S^T at chunk boundary `idx`
         auto store_state = [&](const float *Sv, int idx) {
             const size_t first = p.chunk_off ? (size_t)p.chunk_off[bb] : (size_t)bb * nchunks;
@@ -414,6 +435,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
         tc_fence_before();
         named_sync(1, kGroup);
         uint32_t mma_phase = 0;
+        bool qk_sent = false;  // thread 0: bar_qk of this chunk already signalled
         for (int ci = 0; ci < nchunks; ++ci) {
             const int buf = ci & 1;
             const int L = min(C, T - ci * C);
@@ -423,6 +445,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             // ---- factors, P and T of chunk ci are ready
             if (!mbar_wait(&bar_fact[buf], (ci >> 1) & 1)) fail();
             if (s_tok[buf][0] | s_tok[buf][1]) {
+                if (tid == 0) mbar_arrive(&bar_tfree);  // T is not needed
                 // ---- the chunk token by token (its decay is too strong for the factors, whose
                 //      products E formed all the same): q, k, b from global memory (E folded the
                 //      tiles in place), X = w.v from its tile; records and exchange buffers over this
@@ -490,6 +513,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                            sdesc_sw128(sbase + oqe + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), IDESC_N128, ks > 0);
                 mma_commit(&bar_mma);
             }
+            {  // while MMA 1 runs: T (fp32, from E's solve) -> bf16 rows i of 64 j, zero above the diagonal
+                const int i = tid >> 2, q4 = tid & 3;
+                uint32_t w8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j0 = 16 * q4 + 2 * e;
+                    const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
+                    const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
+                    w8[e] = pack_bf16x2(lo, hi);
+                }
+                *reinterpret_cast<uint4 *>(sm + ott + sw128(i, 32 * q4)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                *reinterpret_cast<uint4 *>(sm + ott + sw128(i, 32 * q4 + 16)) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                fence_proxy_async_smem();
+            }
             if (!mbar_wait(&bar_mma, mma_phase)) fail();
             mma_phase ^= 1;
             tc_fence_after();
@@ -520,6 +557,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             }
             tc_fence_before();
             named_sync(1, kGroup);
+            if (tid == 0) mbar_arrive(&bar_tfree);  // every M thread has read T
             if (s_abort_m) break;
             // ---- MMA 2: U~^T = Y^T T^T
             if (tid == 0) {
@@ -586,6 +624,12 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 // the chunk-end state (kBw): column half 0 through the consumed X tile now, half 1
                 // once that store has read it
                 if (kBw && half == 0) stage_state(Sf, sm + ov);
+            }
+            // the plain forward's products are done with this parity's E~, Q~ and K~ tiles (the
+            // states run still stores factors from them): chunk ci+2's k, b, q may come in
+            if (!kBw && tid == 0) {
+                mbar_arrive(&bar_qk[buf]);
+                qk_sent = true;
             }
             if (kBw) {
                 // ---- the backward's per-chunk factors, state-independent: W^T, M^T = Q~^T - W^T P^T
@@ -713,16 +757,18 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             }  // the chunkwise products
             // ---- next chunk's values (w is single-buffered), then chunk ci+2's loads into this parity
             if (ci + 1 < nchunks) {
-                if (!mbar_wait(&bar_in[buf ^ 1], ((ci + 1) >> 1) & 1)) fail();
+                if (!mbar_wait(&bar_vw[buf ^ 1], ((ci + 1) >> 1) & 1)) fail();
                 fold_value(ci + 1);
             }
             if (kBw && tid == kGroup / 2) bulk_wait_read0();  // the state columns 64-127 have left their tile
+            if (tid == 0) bulk_wait_read0();                  // the output and factor stores have read their tiles
             fence_proxy_async_smem();
             named_sync(1, kGroup);
             if (tid == 0) {
-                bulk_wait_read0();                 // the output store has read its tile
-                mbar_arrive(&bar_mdone[buf]);      // this parity's buffers and w are free
+                if (!qk_sent) mbar_arrive(&bar_qk[buf]);
+                mbar_arrive(&bar_mdone[buf]);  // this chunk's tiles, w and per-parity values are free
             }
+            qk_sent = false;
         }
         float *const st_dst = s_stp;
         if (!s_abort_m && st_dst) {
@@ -771,6 +817,8 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                                          ? p.b[((size_t)bos + (size_t)ci * C + etid) * p.H + hh]
                                          : __float2bfloat16_rn(0.f);
             if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
+            // M is done with chunk ci-2, whose T / P tiles and per-parity values this chunk reuses
+            if (ci >= 2 && !mbar_wait(&bar_mdone[buf], ((ci - 2) >> 1) & 1)) fail();
             float run0 = 0.f, run1 = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -904,31 +952,17 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             named_sync(2, kGroup);
             if (s_abort_e) break;
             // ---- T = (I + A)^-1 on warps 8-11: diagonal 16x16 blocks, then the doubling levels on
-            //      warp-level TF32 MMAs; meanwhile warp 12 issues the next chunk's loads
+            //      warp-level TF32 MMAs
             if (ew < 4) {
+                // M converts the last chunk's T to bf16 from sT: wait until it has
+                if (ci >= 1 && !mbar_wait(&bar_tfree, (ci - 1) & 1)) fail();
                 wm::solve_unit_lower64<LDA>(sA, sT, ew, lane, [] { named_sync(3, 128); });
-                {  // T -> bf16 rows (i) of 64 j, zero above the diagonal
-                    const int i = etid >> 1, hf = etid & 1;
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j0 = 32 * hf + 8 * m + 2 * e;
-                            const float lo = (j0 <= i) ? sT[i * LDA + j0] : 0.f;
-                            const float hi = (j0 + 1 <= i) ? sT[i * LDA + j0 + 1] : 0.f;
-                            w4[e] = pack_bf16x2(lo, hi);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + ott + sw128(i, 64 * hf + 16 * m)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                }
-                fence_proxy_async_smem();
             } else if (ew == 4 && lane == 0 && ci >= 1 && ci + 1 < nchunks) {
-                // chunk ci+1's loads go to the buffers chunk ci-1 used; M frees them with bar_mdone
+                // chunk ci+1's loads go to the buffers chunk ci-1 used
+                if (!mbar_wait(&bar_qk[buf ^ 1], ((ci - 1) >> 1) & 1)) fail();
+                issue_qbk(ci + 1);
                 if (!mbar_wait(&bar_mdone[buf ^ 1], ((ci - 1) >> 1) & 1)) fail();
-                fence_proxy_async_smem();
-                issue(ci + 1);
+                issue_vw(ci + 1);
             }
             named_sync(2, kGroup);
             if (etid == 0) mbar_arrive(&bar_fact[buf]);
