@@ -207,7 +207,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
     // kChunkDecayLimit, so the chunk runs token by token
     __shared__ int s_tok[2][2];
     __shared__ float *s_stp;  // this CTA's end-state destination (read once, at the end)
-    __shared__ __nv_bfloat16 s_bsc[2][kGate ? 64 : 1];  // kGate: b_t of the chunk, by chunk parity
+    __shared__ uint32_t s_bsc[2][kGate ? 64 : 1];  // kGate: (b_t, b_t) bf16x2 of the chunk, by chunk parity
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool is_m = warp < 8;
@@ -789,11 +789,20 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
             s_abort_e = 1;
             atomicExch(p.status, kStatusTimeout);
         };
+        // kGate: b_t of chunk c, one per thread of the first 64, loaded a chunk ahead of its table
+        auto load_bt = [&](int c) -> __nv_bfloat16 {
+            return (kGate && etid < 64 && c < nchunks && c * C + etid < T)
+                       ? p.b[((size_t)bos + (size_t)c * C + etid) * p.H + hh]
+                       : __float2bfloat16_rn(0.f);
+        };
+        __nv_bfloat16 bt_next = load_bt(0);
         for (int ci = 0; ci < nchunks; ++ci) {
             const int buf = ci & 1;
             const int L = min(C, T - ci * C);
             const uint32_t oqe = OFF_QE + buf * 32768, ok = OFF_K + buf * 16384;
             const uint32_t ott = OFF_TP + buf * 16384, opt = ott + 8192;
+            const __nv_bfloat16 bt = bt_next;
+            bt_next = load_bt(ci + 1);
             // log alpha of this warp's 16 tokens x 2 channels, straight from L2
             float2 gv[16];
             if (kGScalar) {  // one decay per (token, head), the same for both channels
@@ -812,10 +821,6 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                                 ? __ldg(reinterpret_cast<const float2 *>(gsrc + (size_t)i * p.H * DIN))
                                 : make_float2(0.f, 0.f);
             }
-            // kGate: this chunk's b_t, one per thread of the first 64, for the table below
-            const __nv_bfloat16 bt = (kGate && etid < 64 && etid < L)
-                                         ? p.b[((size_t)bos + (size_t)ci * C + etid) * p.H + hh]
-                                         : __float2bfloat16_rn(0.f);
             if (!mbar_wait(&bar_in[buf], (ci >> 1) & 1)) fail();
             // M is done with chunk ci-2, whose T / P tiles and per-parity values this chunk reuses
             if (ci >= 2 && !mbar_wait(&bar_mdone[buf], ((ci - 2) >> 1) & 1)) fail();
@@ -828,7 +833,10 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                 gv[i] = make_float2(a0, kGScalar ? a0 : __expf(gv[i].y));  // alpha
             }
             *reinterpret_cast<float2 *>(sTot + tg * 128 + ch) = make_float2(run0, run1);
-            if (kGate && etid < 64) s_bsc[buf][etid] = bt;
+            if (kGate && etid < 64) {
+                const uint32_t b16 = (uint32_t)__bfloat16_as_ushort(bt);
+                s_bsc[buf][etid] = b16 | (b16 << 16);
+            }
             named_sync(2, kGroup);
             if (s_abort_e) break;
             float sqq[16], sqk[16];  // prologue: this thread's share of |q|^2, |k|^2 per token
@@ -871,8 +879,7 @@ fwd_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p)
                     uint32_t kw = *reinterpret_cast<const uint32_t *>(pk + off);
                     uint32_t bw;
                     if (kGate) {
-                        const uint32_t b16 = (uint32_t)__bfloat16_as_ushort(s_bsc[buf][t]);
-                        bw = b16 | (b16 << 16);
+                        bw = s_bsc[buf][t];
                     } else {
                         bw = *reinterpret_cast<const uint32_t *>(pe + off);
                     }
