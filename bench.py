@@ -507,7 +507,8 @@ def run_ours(args):
                               "unfused_extra_bytes": 8 * B * T * H * D * xr["q"].element_size()}
         del xr, pro_out
         # ---- head size 64 (same model width: H = 32), bf16, on the tensor-core forward
-        x64 = make_inputs(B, T, 2 * H, D // 2, D // 2, dtype=w["dtype"], seed=rank_seed(rank) + 29, device=str(dev))
+        x64 = make_inputs(B, T, 2 * H, D // 2, D // 2, dtype=w["dtype"], seed=rank_seed(rank) + 29, device=str(dev),
+                          with_do=True)
         o64 = torch.empty_like(x64["v"])
         S64 = torch.empty_like(x64["S0"])
 
@@ -518,10 +519,26 @@ def run_ours(args):
         ms_64 = time_region(fwd_64, 10, 3, stream) / 10
         assert g.gdn2_sync_status() == 0
         b64 = fwd_bytes(B, T, 2 * H, D // 2)
+        # its backward, with the same workspace rules as the headline one
+        ws64 = torch.empty(g.gdn2_workspace_size(1, x64["q"].dtype, B, T, 2 * H, D // 2, D // 2), dtype=torch.uint8,
+                           device=dev)
+        gr64 = {"dq": torch.empty_like(x64["q"]), "dk": torch.empty_like(x64["k"]), "dv": torch.empty_like(x64["v"]),
+                "dlog_alpha": torch.empty_like(x64["log_alpha"]), "db": torch.empty_like(x64["b"]),
+                "dw": torch.empty_like(x64["w"]), "dS0": torch.empty_like(x64["S0"])}
+
+        def bwd_64():
+            g.gdn2_chunk_bwd(x64["q"], x64["k"], x64["v"], x64["log_alpha"], x64["b"], x64["w"], x64["S0"], x64["do"],
+                             None, workspace=ws64, out=gr64)
+
+        ms_64b = time_region(bwd_64, 5, 3, stream) / 5
+        assert g.gdn2_sync_status() == 0
+        bb64 = bwd_bytes(B, T, 2 * H, D // 2)
         extras["d64"] = {"workload": f"B={B}, T={T}, H={2 * H}, d={D // 2}, bf16", "ms": round(ms_64, 4),
                          "tokens_per_s": round(job_rate(tokens, world, ms_64), 1), "algorithmic_bytes": b64,
-                         "hbm_frac": round(b64 / (ms_64 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-        del x64, o64, S64
+                         "hbm_frac": round(b64 / (ms_64 * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                         "bwd_ms": round(ms_64b, 4), "bwd_algorithmic_bytes": bb64,
+                         "bwd_hbm_frac": round(bb64 / (ms_64b * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del x64, o64, S64, ws64, gr64
         extras["varlen"] = {"sequences": len(lens), "lengths": [int(v) for v in lens], "tokens": tokens,
                             "fwd_ms": round(ms_v, 4), "fwd_tokens_per_s": round(job_rate(tokens, world, ms_v), 1),
                             "fwd_hbm_frac": round(fwd_bytes(1, tokens, H, D) / (ms_v * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
