@@ -542,7 +542,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_in0, bar_in1, bar_in2, bar_a, bar_b, bar_c, bar_d;
+    __shared__ __align__(8) uint64_t bar_in0, bar_in1, bar_in2, bar_in3, bar_a, bar_b, bar_c, bar_d;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -562,6 +562,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         mbar_init(&bar_in0, 1);
         mbar_init(&bar_in1, 1);
         mbar_init(&bar_in2, 1);
+        mbar_init(&bar_in3, 1);
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_init(&bar_c, 1);
@@ -577,15 +578,17 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    // A task's tile loads, issued by warp 0 in three parts as their regions free up during the
-    // task before: part 0 q, k, b, dO, T, P (and both input barriers' byte counts); part 1 log
-    // alpha; part 2 S^T, dS_n^T, v, w.
+    // A task's tile loads, in four parts as their regions free up: part 0 q, k, b, dO, T, P (and
+    // the byte counts of bar_in0 and bar_in1) and part 1 log alpha, from warp 0 during the task
+    // before; part 2 S^T and dS_n^T from warp 1 at the end of the task before, once the staged
+    // dq, dk, db have left their tiles; part 3 v and w (bar_in3) from warp 1 during this task's
+    // decay folding, once the staged dg has left its tiles.
     auto issue = [&](int part, const ChunkRef &r) {
         const int yy = r.sp.bos + r.ci * C, h = r.h, at = lane & 1;
         if (part == 0) {
             if (lane == 0) {
                 mbar_expect_tx(&bar_in0, 10 * 8192);
-                mbar_expect_tx(&bar_in1, 4 * 16384 + 8 * 8192);
+                mbar_expect_tx(&bar_in1, 6 * 16384);
             }
             __syncwarp();
             if (lane < 6) {
@@ -599,12 +602,15 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             }
         } else if (part == 1) {
             if (lane < 4) tma_load_3d(sm + GG + lane * 8192, &maps.g, lane * 32, h, yy, &bar_in0);
-        } else {
+        } else if (part == 2) {
             const int sl = (int)(bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D);
             if (lane < 2) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, sl, &bar_in1);
             else if (lane < 4) tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(r.cidx * D), &bar_in1);
-            else if (lane < 6) tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, h, yy, &bar_in1);
-            else if (lane < 8) tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, h, yy, &bar_in1);
+        } else {
+            if (lane == 0) mbar_expect_tx(&bar_in3, 4 * 8192);
+            __syncwarp();
+            if (lane < 2) tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, h, yy, &bar_in3);
+            else if (lane < 4) tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, h, yy, &bar_in3);
         }
     };
     ChunkRef cr;
@@ -613,8 +619,10 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         issue(0, cr);
         issue(1, cr);
         issue(2, cr);
+        issue(3, cr);
     }
     uint32_t ph = 0;  // parity of this task's barrier phases
+    bool pend3 = false;  // warp 1: this task's v, w are still to be loaded
     while (task >= 0) {
     ChunkRef nx;
     const int next = find_task(task + gridDim.x, nx);
@@ -648,6 +656,12 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                         : make_float2(0.f, 0.f);
         }
         decay_pair8(gl, eG, emG, tot, cp, g8, sTot);
+        if (warp == 1 && pend3) {  // the last task's dg has left v, w's tiles by now: this task's v, w
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+            issue(3, cr);
+            pend3 = false;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int t = 8 * g8 + i;
@@ -729,6 +743,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     }
     // ---- read back: Y^T = X^T - acc and dU~^T, as bf16 A operands (lane = d_v, 16 tokens per warp)
     wait_or_abort(&bar_a, ph, a.status, &s_abort);
+    wait_or_abort(&bar_in3, ph, a.status, &s_abort);  // v, w
     tc_fence_after();
     {
         uint32_t r[16], pk[8];
@@ -988,17 +1003,22 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                 tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
                 tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
             }
+            bulk_commit();
             for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + VV + bx * 8192, bx * 32, hh, y);
             bulk_commit();
         }
-        if (lane == 0) bulk_wait_read0();  // the staged gradients are read before their tiles are refilled
+        if (lane == 0) bulk_wait_read1();  // dq, dk and db are read before S^T and dS_n^T come in
         __syncwarp();
-        if (next >= 0) issue(2, nx);  // S^T, dS_n^T, v, w into the freed tiles
+        if (next >= 0) {
+            issue(2, nx);  // S^T, dS_n^T into the freed tiles; v, w wait for dg (next task's folding)
+            pend3 = true;
+        }
     }
     task = next;
     cr = nx;
     ph ^= 1;
     }
+    if (warp == 1 && lane == 0) bulk_wait0();  // the last task's gradients have been written
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
