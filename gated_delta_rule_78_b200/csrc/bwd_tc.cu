@@ -962,6 +962,16 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                 a.dk[go] = __float2bfloat16_rn(de * b0 + dK * emG[i]);
             }
         }
+        fence_proxy_async_smem();
+        __syncthreads();  // dq, dk, db are staged: their stores go out while dg is formed
+        if (tid == 32 && full) {
+            for (int at = 0; at < a.din / 64; ++at) {
+                tma_store_3d(&maps.dq, sm + SS + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
+                tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
+            }
+            bulk_commit();
+        }
         if (cg == 3) dG[15] += reinterpret_cast<const float *>(sm + DGF)[row];  // gamma dgamma, last row
         float rs = 0.f;
 #pragma unroll
@@ -997,13 +1007,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {  // lane 0 owns every bulk store of the block
-        if (lane == 0 && full) {
-            for (int at = 0; at < a.din / 64; ++at) {
-                tma_store_3d(&maps.dq, sm + SS + at * 8192, at * 64, hh, y);
-                tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
-                tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
-            }
-            bulk_commit();
+        if (lane == 0 && full) {  // dq, dk, db went out before dg was formed
             for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + VV + bx * 8192, bx * 32, hh, y);
             bulk_commit();
         }
