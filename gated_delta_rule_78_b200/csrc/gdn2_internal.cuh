@@ -241,13 +241,14 @@ cudaError_t launch_tok_grad_tc(const Problem &p, const void *d_o, const __nv_bfl
                                const __nv_bfloat16 *dSn, const int *list, float *scratch, int nblocks,
                                const BwdOut &out, cudaStream_t s);
 
-// tensor-core backward (bf16, D = 128): the forward in states mode, then the prep,
-// chain and gradient kernels
+// tensor-core backward (bf16, D = 128): the forward in states mode (which also stores the
+// chunk factors), then the chain and gradient kernels, then the token-form gradients of the
+// chunks past the factors' range
 size_t bwd_tc_workspace_bytes(const Problem &p);
 cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, const BwdOut &out, void *ws,
                           int *status, cudaStream_t s, bool states_saved = false);
-// the bf16 forward (o, S_T) that also records the chunk-boundary states into the backward's
-// workspace ws, for launch_bwd_tc(..., states_saved = true); fixed-length batches
+// the bf16 forward (o, S_T) that also records the chunk-boundary states and factors into the
+// backward's workspace ws, for launch_bwd_tc(..., states_saved = true); fixed-length batches
 cudaError_t launch_fwd_save(const Problem &p, void *o, float *S_T, void *ws, int *status, cudaStream_t s);
 
 // Gate layouts (gates.cu): fill dst ([n_rows, D]) with src[row] (a per-row scalar) or,

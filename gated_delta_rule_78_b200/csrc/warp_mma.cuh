@@ -1,7 +1,7 @@
-// Warp-level tensor-core building block shared by the forward and the backward prep
-// kernels: the 64 x 64 unit lower-triangular inverse T = (I + A)^-1 that every chunk
-// needs (closed-form 4x4 blocks, in-warp doubling to 16x16, then two doubling levels
-// on TF32 warp MMAs).
+// Warp-level tensor-core building block of the forward kernel (and so of the backward's
+// states pass): the 64 x 64 unit lower-triangular inverse T = (I + A)^-1 that every chunk
+// needs (closed-form 4x4 blocks, in-warp doubling to 16x16, then two doubling levels on
+// TF32 warp MMAs).
 #pragma once
 
 #include <stdint.h>
