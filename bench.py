@@ -474,11 +474,26 @@ def run_ours(args):
             ms_k = time_region(fwd_k, 20, 3, stream) / 20
             assert g.gdn2_sync_status() == 0
             kb = fwd_bytes(B, T, H, D) - B * T * H * 2 * (2 * D - 2) - (B * T * H * (4 * D - 4) if gdec is gsc else 0)
+            # its backward: scalar b and w run natively, a scalar decay is broadcast
+            wsb = torch.empty(g.gdn2_workspace_size_gated(1, fl, x["q"].dtype, B, T, H, D, D), dtype=torch.uint8,
+                              device=dev)
+            grk = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
+                   "dlog_alpha": torch.empty_like(gdec), "db": torch.empty_like(beta), "dw": torch.empty_like(beta),
+                   "dS0": torch.empty_like(x["S0"])}
+
+            def bwd_k():
+                g.gdn2_chunk_bwd_gated(x["q"], x["k"], x["v"], gdec, beta, beta, x["S0"], x["do"], flags=fl,
+                                       workspace=wsb, out=grk)
+
+            ms_kb = time_region(bwd_k, 5, 3, stream) / 5
+            assert g.gdn2_sync_status() == 0
+            del wsb, grk
             gate_pts[name] = {"workload": f"B={B}, T={T}, H={H}, d={D}; b = w = beta [B,T,H]" +
                               ("; log alpha [B,T,H]" if gdec is gsc else "; log alpha per channel"),
                               "ms": round(ms_k, 4), "tokens_per_s": round(job_rate(tokens, world, ms_k), 1),
                               "algorithmic_bytes": kb, "hbm_frac": round(kb / (ms_k * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                              "workspace_bytes": int(wsk.numel()) if wsk.numel() > 16 else 0}
+                              "workspace_bytes": int(wsk.numel()) if wsk.numel() > 16 else 0,
+                              "bwd_ms": round(ms_kb, 4)}
             del wsk
         extras.update(gate_pts)
         # ---- input prologue fused in the chunk kernel, against a separate pass + the plain forward

@@ -355,7 +355,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                         const size_t off = ((row0 + t) * a.H + hh) * a.din + c;
                         qv = __bfloat162float(a.q[off]);
                         kv = __bfloat162float(a.k[off]);
-                        bv = __bfloat162float(a.b[off]);
+                        bv = __bfloat162float(a.pr.bw_scalar ? a.b[(row0 + t) * a.H + hh] : a.b[off]);
                         gv = a.g[off];
                     }
                     rc.q[c] = qv;
@@ -502,7 +502,11 @@ constexpr uint32_t PA = TT;
 constexpr uint32_t VV = 196608;   // v, then dw (full chunks: stored from here by TMA)
 constexpr uint32_t WW = 212992;   // w, then dv
 constexpr uint32_t DGF = 229376;  // gamma dgamma [D] fp32
-constexpr uint32_t USED = DGF + D * 4;
+// scalar erase and write gates: b_t and w_t of the chunk [2][64] bf16, and the four lane quarters'
+// partial sums of dw_t [4][64] fp32 (those of db_t go to the first half of DS, unused then)
+constexpr uint32_t SBW = DGF + D * 4;
+constexpr uint32_t SDW = SBW + 256;
+constexpr uint32_t USED = SDW + 1024;
 constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
 // scratch inside the -dY rows (free until dY is read back), and in DS's second half (free once
 // (Gm dS_n)^T's products are done) for the factor chain
@@ -527,6 +531,22 @@ struct GradMaps {
 };
 
 
+// Sums of 16 per-lane values over the 32 lanes of a warp, by halving exchanges: on return lane
+// 2 i (and 2 i + 1) holds the total of value i in v[0].
+__device__ __forceinline__ void warp_sum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int m = 16, n = 8; m >= 2; m >>= 1, n >>= 1) {
+        const bool hi = lane & m;
+#pragma unroll
+        for (int j = 0; j < n; ++j) {
+            const float give = hi ? v[j] : v[j + n];
+            v[j] = (hi ? v[j + n] : v[j]) + __shfl_xor_sync(0xffffffffu, give, m);
+        }
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 // bf16 element (t, c) of a [rows][128] tile whose two column atoms are `astride` bytes apart
 __device__ __forceinline__ uint32_t tile_off(int t, int c, uint32_t astride)
 {
@@ -535,6 +555,10 @@ __device__ __forceinline__ uint32_t tile_off(int t, int c, uint32_t astride)
 __device__ __forceinline__ float ld_bf(const uint8_t *p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p)); }
 __device__ __forceinline__ void st_bf(uint8_t *p, float x) { *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x); }
 
+// kSG: the erase and write gates are one value per (token, head) ([rows, H]): per-token tables
+// replace the b and w tiles, and db_t, dw_t are the per-channel gradients summed over the
+// channels (over the 32 lanes of a warp, then over the four lane quarters).
+template <bool kSG>
 __global__ void __launch_bounds__(grad_tc::kThreads, 1)
 bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 {
@@ -587,11 +611,12 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         const int yy = r.sp.bos + r.ci * C, h = r.h, at = lane & 1;
         if (part == 0) {
             if (lane == 0) {
-                mbar_expect_tx(&bar_in0, 10 * 8192);
+                mbar_expect_tx(&bar_in0, (kSG ? 8 : 10) * 8192);
                 mbar_expect_tx(&bar_in1, 6 * 16384);
             }
             __syncwarp();
-            if (lane < 6) {
+            if (kSG && (lane == 4 || lane == 5)) {  // b comes from the per-token table
+            } else if (lane < 6) {
                 const int which = lane >> 1;
                 const CUtensorMap *mp = which == 0 ? &maps.q : which == 1 ? &maps.k : &maps.b;
                 tma_load_3d(sm + RQ + which * 16384 + at * 8192, mp, at * 64, h, yy, &bar_in0);
@@ -607,10 +632,10 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             if (lane < 2) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, sl, &bar_in1);
             else if (lane < 4) tma_load_2d(sm + DS + at * 16384, &maps.dsn, at * 64, (int)(r.cidx * D), &bar_in1);
         } else {
-            if (lane == 0) mbar_expect_tx(&bar_in3, 4 * 8192);
+            if (lane == 0) mbar_expect_tx(&bar_in3, (kSG ? 2 : 4) * 8192);
             __syncwarp();
             if (lane < 2) tma_load_3d(sm + VV + at * 8192, &maps.v, at * 64, h, yy, &bar_in3);
-            else if (lane < 4) tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, h, yy, &bar_in3);
+            else if (!kSG && lane < 4) tma_load_3d(sm + WW + at * 8192, &maps.w, at * 64, h, yy, &bar_in3);
         }
     };
     ChunkRef cr;
@@ -639,6 +664,12 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
+    }
+    __nv_bfloat16 *const sBt = reinterpret_cast<__nv_bfloat16 *>(sm + SBW), *const sWt = sBt + 64;
+    if (kSG && tid < 128) {  // this chunk's b_t (threads 0-63) and w_t (64-127); seen after the folding's first barrier
+        const int t = tid & 63;
+        const __nv_bfloat16 *src = tid < 64 ? a.b : a.w;
+        (tid < 64 ? sBt : sWt)[t] = t < L ? src[((size_t)y + t) * a.H + hh] : __float2bfloat16_rn(0.f);
     }
 
     // ---- decay folding in place: thread (channel pair cp, token group g8 of 8)
@@ -669,7 +700,13 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             uint32_t *pq = reinterpret_cast<uint32_t *>(sm + RQ + off);
             uint32_t *pk = reinterpret_cast<uint32_t *>(sm + RK + off);
             uint32_t *pe = reinterpret_cast<uint32_t *>(sm + RB + off);
-            uint32_t q2 = *pq, k2 = *pk, b2 = *pe;
+            uint32_t q2 = *pq, k2 = *pk, b2;
+            if (kSG) {
+                const uint32_t b16 = (uint32_t)__bfloat16_as_ushort(sBt[t]);
+                b2 = b16 | (b16 << 16);
+            } else {
+                b2 = *pe;
+            }
             if (t >= L) { q2 = 0u; k2 = 0u; b2 = 0u; }
             const float k0 = bf_lo(k2), k1 = bf_hi(k2);
             *pq = pack_bf16x2(bf_lo(q2) * eG[i].x, bf_hi(q2) * eG[i].y);
@@ -756,7 +793,8 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             for (int h = 0; h < 2; ++h) {
                 const int t = 16 * cg + 2 * e + h;
                 const uint32_t so = tile_off(t, row, 8192);
-                const float x = (t < L) ? ld_bf(sm + VV + so) * ld_bf(sm + WW + so) : 0.f;
+                const float wt = kSG ? __bfloat162float(sWt[t]) : ld_bf(sm + WW + so);
+                const float x = (t < L) ? ld_bf(sm + VV + so) * wt : 0.f;
                 y2[h] = x - __uint_as_float(r[2 * e + h]);
             }
             pk[e] = pack_bf16x2(y2[0], y2[1]);
@@ -795,21 +833,27 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         tmem_ld16(tmem + TM_DY + 16 * cg + lane_off, r);
         tmem_wait_ld();
         const bool ch_ok = row < a.din;
+        float pdw[16];  // kSG: this channel's share of dw_t
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * cg + i;
             const float d = __uint_as_float(r[i]);
             st_bf(sm + DY + tile_off(64 + t, row, 16384), -d);
             const uint32_t so = tile_off(t, row, 8192);
-            const float wv = ld_bf(sm + WW + so), vv = ld_bf(sm + VV + so);
+            const float wv = kSG ? __bfloat162float(sWt[t]) : ld_bf(sm + WW + so), vv = ld_bf(sm + VV + so);
+            pdw[i] = t < L ? d * vv : 0.f;
             if (full) {
                 st_bf(sm + WW + so, d * wv);
-                st_bf(sm + VV + so, d * vv);
+                if (!kSG) st_bf(sm + VV + so, d * vv);
             } else if (t < L && ch_ok) {
                 const size_t go = tok_off(a, bb, hh, ci, t) + row;
                 a.dv[go] = __float2bfloat16_rn(d * wv);
-                a.dw[go] = __float2bfloat16_rn(d * vv);
+                if (!kSG) a.dw[go] = __float2bfloat16_rn(d * vv);
             }
+        }
+        if (kSG) {  // sum over this lane quarter's 32 channels; the quarters add up below
+            warp_sum16(pdw, lane);
+            if (!(lane & 1)) reinterpret_cast<float *>(sm + SDW)[quarter * 64 + 16 * cg + (lane >> 1)] = pdw[0];
         }
     }
     fence_proxy_async_smem();
@@ -835,18 +879,22 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     if (tid == 32 && full) {  // dv, dw by TMA (thread 32 owns every bulk store of the block)
         for (int at = 0; at < a.din / 64; ++at) {
             tma_store_3d(&maps.dv, sm + WW + at * 8192, at * 64, hh, y);
-            tma_store_3d(&maps.dw, sm + VV + at * 8192, at * 64, hh, y);
+            if (!kSG) tma_store_3d(&maps.dw, sm + VV + at * 8192, at * 64, hh, y);
         }
         bulk_commit();
+    }
+    if (kSG && tid < 64 && tid < L) {  // dw_t: the four lane quarters' sums
+        const float *p4 = reinterpret_cast<const float *>(sm + SDW);
+        a.dw[((size_t)y + tid) * a.H + hh] = __float2bfloat16_rn(p4[tid] + p4[64 + tid] + p4[128 + tid] + p4[192 + tid]);
     }
     wait_or_abort(&bar_c, ph, a.status, &s_abort);
     tc_fence_after();
     if (tid == 0) {  // S^T and (Gm dS_n)^T are consumed: the raw q, k, b for the factor chain
-        mbar_expect_tx(&bar_in2, 6 * 8192);
+        mbar_expect_tx(&bar_in2, (kSG ? 4 : 6) * 8192);
         for (int at = 0; at < 2; ++at) {
             tma_load_3d(sm + SS + at * 8192, &maps.q, at * 64, hh, y, &bar_in2);
             tma_load_3d(sm + SS + 16384 + at * 8192, &maps.k, at * 64, hh, y, &bar_in2);
-            tma_load_3d(sm + DS + at * 8192, &maps.b, at * 64, hh, y, &bar_in2);
+            if (!kSG) tma_load_3d(sm + DS + at * 8192, &maps.b, at * 64, hh, y, &bar_in2);
         }
     }
     {  // [dP; dA] -> bf16 tile [128][64] (over U~): dP lower incl., dA strictly lower
@@ -933,7 +981,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         tmem_wait_ld();
         wait_or_abort(&bar_in2, ph, a.status, &s_abort);
         float e = 0.f, kup = 0.f;  // kup: this thread's share of sum_s K~_s . dK~_s (state-update part)
-        float dG[16];
+        float dG[16], pdb[16];     // pdb (kSG): this channel's share of db_t
         const size_t base = tok_off(a, bb, hh, ci, 16 * cg) + row, stride = (size_t)a.H * a.din;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -943,7 +991,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             const uint32_t so = tile_off(t, row, 8192);
             const bool ok = t < L;
             const float q0 = ok ? ld_bf(sm + SS + so) : 0.f, k0 = ok ? ld_bf(sm + SS + 16384 + so) : 0.f;
-            const float b0 = ok ? ld_bf(sm + DS + so) : 0.f;
+            const float b0 = ok ? (kSG ? __bfloat162float(sBt[t]) : ld_bf(sm + DS + so)) : 0.f;
             const float dQ = __uint_as_float(rq[i]), dE = __uint_as_float(re[i]), dKu = __uint_as_float(ru[i]);
             const float dK = __uint_as_float(rk[i]) + dKu;
             const float de = dE * e;
@@ -951,16 +999,21 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             const float kt = __bfloat162float(__float2bfloat16_rn(k0 * emG[i]));  // K~, likewise
             dG[i] = dQ * bf_lo(qe) + dE * bf_hi(qe) - dK * kt;
             kup = fmaf(kt, dKu, kup);
+            pdb[i] = ok ? de * k0 : 0.f;
             if (full) {  // over the raw q, k, b just read
                 st_bf(sm + SS + so, dQ * e);
-                st_bf(sm + DS + so, de * k0);
+                if (!kSG) st_bf(sm + DS + so, de * k0);
                 st_bf(sm + SS + 16384 + so, de * b0 + dK * emG[i]);
             } else if (ok && ch_ok) {
                 const size_t go = base + (size_t)i * stride;
                 a.dq[go] = __float2bfloat16_rn(dQ * e);
-                a.db[go] = __float2bfloat16_rn(de * k0);
+                if (!kSG) a.db[go] = __float2bfloat16_rn(de * k0);
                 a.dk[go] = __float2bfloat16_rn(de * b0 + dK * emG[i]);
             }
+        }
+        if (kSG) {  // db_t: sum over this lane quarter's 32 channels into the unused first half of DS
+            warp_sum16(pdb, lane);
+            if (!(lane & 1)) reinterpret_cast<float *>(sm + DS)[quarter * 64 + 16 * cg + (lane >> 1)] = pdb[0];
         }
         fence_proxy_async_smem();
         __syncthreads();  // dq, dk, db are staged: their stores go out while dg is formed
@@ -968,9 +1021,13 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             for (int at = 0; at < a.din / 64; ++at) {
                 tma_store_3d(&maps.dq, sm + SS + at * 8192, at * 64, hh, y);
                 tma_store_3d(&maps.dk, sm + SS + 16384 + at * 8192, at * 64, hh, y);
-                tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
+                if (!kSG) tma_store_3d(&maps.db, sm + DS + at * 8192, at * 64, hh, y);
             }
             bulk_commit();
+        }
+        if (kSG && tid < 64 && tid < L) {  // db_t: the four lane quarters' sums
+            const float *p4 = reinterpret_cast<const float *>(sm + DS);
+            a.db[((size_t)y + tid) * a.H + hh] = __float2bfloat16_rn(p4[tid] + p4[64 + tid] + p4[128 + tid] + p4[192 + tid]);
         }
         if (cg == 3) dG[15] += reinterpret_cast<const float *>(sm + DGF)[row];  // gamma dgamma, last row
         float rs = 0.f;
@@ -1135,23 +1192,26 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         memset(&maps, 0, sizeof(maps));
         const int rows = (int)token_rows(p);
         const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p), nbound = (uint64_t)p.H * (chunk_bound(p) + p.B);
+        const bool sg = p.bw_scalar;  // scalar b and w ([rows, H]): no tiles of theirs, db and dw written per token
         if (!make_map(&maps.q, p.q, false, 1, rows, p.H, p.D) || !make_map(&maps.k, p.k, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D) || !make_map(&maps.v, p.v, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.w, p.w, false, 1, rows, p.H, p.D) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
+            (!sg && !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D)) || !make_map(&maps.v, p.v, false, 1, rows, p.H, p.D) ||
+            (!sg && !make_map(&maps.w, p.w, false, 1, rows, p.H, p.D)) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
             !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D) ||
             !make_map_2d(&maps.st, a.states, D, nbound * D, 64, D) ||
             !make_map_2d(&maps.dsn, a.dSn, D, nchunk * D, 64, D) ||
             !make_map_2d(&maps.tm, a.Tm, C, nchunk * C, 64, C) || !make_map_2d(&maps.pm, a.Pm, C, nchunk * C, 64, C) ||
             !make_map(&maps.dq, out.dq, false, 1, rows, p.H, p.D) || !make_map(&maps.dk, out.dk, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.db, out.db, false, 1, rows, p.H, p.D) || !make_map(&maps.dv, out.dv, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.dw, out.dw, false, 1, rows, p.H, p.D) || !make_map(&maps.dg, out.dg, true, 1, rows, p.H, p.D))
+            (!sg && !make_map(&maps.db, out.db, false, 1, rows, p.H, p.D)) || !make_map(&maps.dv, out.dv, false, 1, rows, p.H, p.D) ||
+            (!sg && !make_map(&maps.dw, out.dw, false, 1, rows, p.H, p.D)) || !make_map(&maps.dg, out.dg, true, 1, rows, p.H, p.D))
             return cudaErrorInvalidValue;
-        if ((e = set_smem_attr(reinterpret_cast<const void *>(bwd_grad_kernel), (int)grad_tc::SMEM)) != cudaSuccess)
-            return e;
+        const void *kern = sg ? reinterpret_cast<const void *>(bwd_grad_kernel<true>)
+                              : reinterpret_cast<const void *>(bwd_grad_kernel<false>);
+        if ((e = set_smem_attr(kern, (int)grad_tc::SMEM)) != cudaSuccess) return e;
         int dev = 0, n_sm = 148;  // persistent: one block per multiprocessor
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
         const int ntask = (int)chunk_bound(p) * p.H;
-        bwd_grad_kernel<<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+        if (sg) bwd_grad_kernel<true><<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+        else bwd_grad_kernel<false><<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the chunks that run token by token: their gradients, exact, over what the gradient kernel wrote

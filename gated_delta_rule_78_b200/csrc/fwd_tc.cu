@@ -1055,8 +1055,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     TcParams prm{pr.B, pr.T, pr.H, (const __nv_bfloat16 *)pr.q, (const __nv_bfloat16 *)pr.k, (const __nv_bfloat16 *)pr.b,
                  (const __nv_bfloat16 *)pr.w, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
                  pr.g_scalar ? 1 : 0, ScanArgs{}, BwdFactors{}};
-    if (bw) {  // the backward's factors: states runs with per-channel gates and no prologue only
-        if (!states || pr.g_scalar || pr.bw_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
+    if (bw) {  // the backward's factors: states runs with a per-channel decay and no prologue only
+        if (!states || pr.g_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
         prm.bw = *bw;
         const uint64_t nchunk = (uint64_t)pr.H * chunk_bound(pr);
         const uint64_t state_rows = (uint64_t)pr.H * (chunk_bound(pr) + pr.B) * D;  // TMA coordinates are 32-bit
@@ -1081,6 +1081,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         return cudaGetLastError();
     };
     if (scan) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, true>) : run(fwd_tc_kernel<false, 64, 0, true>);
+    if (bw && pr.bw_scalar)  // scalar erase and write gates
+        return din == 128 ? run(fwd_tc_kernel<false, 128, 0, false, true, true>) : run(fwd_tc_kernel<false, 64, 0, false, true, true>);
     if (bw) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, false, true>) : run(fwd_tc_kernel<false, 64, 0, false, true>);
     if (pr.prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
     auto by_pro = [&](auto gs, auto dn) -> cudaError_t {

@@ -136,6 +136,8 @@ size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 bool pro_any(int flags) { return flags & (GDN2_QK_L2NORM | GDN2_BW_LOGITS); }
 // b and w both one value per (token, head): the bf16 forward reads them as they are
 bool bw_native(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_scalar(flags, 1) && gate_scalar(flags, 2); }
+// ... and the bf16 backward, without the prologue (whose backward pass wants per-channel gates)
+bool bw_native_bwd(int flags, gdn2_dtype dt) { return bw_native(flags, dt) && !pro_any(flags); }
 bool pro_fused(int flags, gdn2_dtype dt)
 {
     return dt == GDN2_BF16 && ((gate_full(flags, 1) && gate_full(flags, 2)) || bw_native(flags, dt));
@@ -153,7 +155,8 @@ struct GatedWs {
     size_t pro[4], off[3], grad[3], core, total;
 };
 // The chunk forward keeps some scalar gates as they are, which then need no broadcast copy:
-// bw_kept (scalar b and w together) and decay_kept (a scalar decay, bf16).
+// bw_kept (scalar b and w together; in the backward also no full-size gradients of theirs)
+// and decay_kept (a scalar decay, bf16).
 GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes, bool pro_pass,
                  bool bw_kept = false, bool decay_kept = false)
 {
@@ -176,7 +179,7 @@ GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, 
     }
     for (int i = 0; i < 3; ++i) {
         l.grad[i] = off;
-        if (bwd && !gate_full(flags, i)) off += round256(n * es[i]);
+        if (bwd && !gate_full(flags, i) && !(bw_kept && i > 0)) off += round256(n * es[i]);
     }
     l.core = off;
     l.total = off + core_bytes;
@@ -186,10 +189,10 @@ GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, 
 // Broadcast the non-per-channel gates into the workspace; gp[i] is replaced by the full
 // tensor's address.  Absent gates are 0 (log decay) or 1 (b, w).
 gdn2_status expand_gates(int flags, gdn2_dtype dt, const GatedWs &l, char *ws, size_t rows, int H, int D,
-                         const void *gp[3], cudaStream_t s)
+                         const void *gp[3], cudaStream_t s, bool bw_kept = false)
 {
     for (int i = 0; i < 3; ++i) {
-        if (gate_full(flags, i)) continue;
+        if (gate_full(flags, i) || (bw_kept && i > 0)) continue;
         void *dst = ws + l.off[i];
         const bool fp32 = (i == 0) || dt == GDN2_F32;
         cudaError_t e = gdn2::launch_expand_gate(fp32, gate_none(flags, i) ? nullptr : gp[i], dst, rows * H, D,
@@ -448,7 +451,8 @@ size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int
                                                                                 nullptr, nullptr, nullptr, nullptr))
                                    : 0;
     const bool pro_pass = pro_any(flags) && (which == 1 || !pro_fused(flags, dt));
-    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass, which == 0 && bw_native(flags, dt),
+    return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass,
+                    which == 0 ? bw_native(flags, dt) : bw_native_bwd(flags, dt),
                     which == 0 && dt == GDN2_BF16 && gate_scalar(flags, 0))
         .total;
 }
@@ -511,7 +515,11 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, dlog_alpha, db, dw)) != GDN2_OK) return st;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
-    const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p), pro_any(flags));
+    // scalar b and w (KDA-shaped) run natively: the kernels read them per token and write db, dw
+    // per token; only a scalar decay is still broadcast
+    const bool nat = bw_native_bwd(flags, dt);
+    const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p), pro_any(flags),
+                               nat);
     if (!workspace || ws_bytes < l.total) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
@@ -522,18 +530,19 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     p.q = qq;
     p.k = kk;
     const void *gp[3] = {log_alpha, bq, wq};
-    if ((st = expand_gates(flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s)) != GDN2_OK) return st;
+    if ((st = expand_gates(flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s, nat)) != GDN2_OK) return st;
     p.g = static_cast<const float *>(gp[0]);
     p.b = gp[1];
     p.w = gp[2];
+    p.bw_scalar = nat;
     void *grads[3] = {dlog_alpha, db, dw};
     for (int i = 0; i < 3; ++i)
-        if (!gate_full(flags, i)) grads[i] = ws + l.grad[i];  // full-size gradient, reduced below
+        if (!gate_full(flags, i) && !(nat && i > 0)) grads[i] = ws + l.grad[i];  // full-size gradient, reduced below
     gdn2::BwdOut out{dq, dk, dv, grads[1], grads[2], static_cast<float *>(grads[0]), dS0};
     if (gdn2::launch_bwd(dt, p, d_o, dS_T, out, ws + l.core, s) != cudaSuccess) return GDN2_ERR_CUDA;
     void *user[3] = {dlog_alpha, db, dw};
     for (int i = 0; i < 3; ++i) {
-        if (!gate_scalar(flags, i)) continue;
+        if (!gate_scalar(flags, i) || (nat && i > 0)) continue;
         const bool fp32 = (i == 0) || dt == GDN2_F32;
         if (gdn2::launch_channel_sum(fp32, grads[i], user[i], (size_t)B * T * H, Dk, s) != cudaSuccess)
             return GDN2_ERR_CUDA;

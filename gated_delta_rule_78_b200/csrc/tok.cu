@@ -161,7 +161,7 @@ __device__ __forceinline__ void lane_reduce(float (&v)[N], int lane)
 template <int D>
 struct TokGradSmem {
     static constexpr int NW = D / 32;  // warps per column quarter (32 rows each)
-    static constexpr size_t floats = 4 * (size_t)C * D + (size_t)NW * D + D + 16 * (size_t)D;
+    static constexpr size_t floats = 4 * (size_t)C * D + (size_t)NW * D + D + 16 * (size_t)D + 2 * NW;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -182,12 +182,21 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
     float *sRed = sU + C * D;        // [NW][D] partial sums over d_k
     float *sVec = sRed + NW * D;     // [D]     du of the current token
     float *sRow = sVec + D;          // [4 quantities][4 quarters][D]
+    float *sScal = sRow + 16 * D;    // [dw | db][NW] per-warp sums (scalar gates)
     const Problem &p = a.p;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c = tid % D, jq = tid / D, j0 = jq * NJ, cw = warp % NW;
     const Tin *q = (const Tin *)p.q, *k = (const Tin *)p.k, *v = (const Tin *)p.v;
     const Tin *bg = (const Tin *)p.b, *wg = (const Tin *)p.w, *dOg = (const Tin *)a.dO;
     Tin *dq = (Tin *)a.dq, *dk = (Tin *)a.dk, *dv = (Tin *)a.dv, *db = (Tin *)a.db, *dw = (Tin *)a.dw;
+    // scalar erase and write gates ([rows, H]): b_t, w_t read per token, db_t, dw_t summed over
+    // the channels (the first D threads: a warp shuffle, then the NW warps in shared memory)
+    const bool sg = p.bw_scalar;
+    auto warp_total = [&](float x) {
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+        return x;
+    };
     float *Sp = a.scratch + (size_t)blockIdx.x * C * D * D;
     const int nchb = (int)chunk_bound(p);
     const int ntask = a.list ? a.list[0] : a.ntask;
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
                 const size_t off = tok_row(p, r.sp, h, ci * C + t) + jj;
                 dov = to_f(dOg[off]);
                 vv = to_f(v[off]);
-                wv = to_f(wg[off]);
+                wv = to_f(sg ? wg[off / p.D] : wg[off]);
             }
             sDo[idx] = dov;
             sV[idx] = vv;
@@ -248,7 +257,7 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
             const size_t off = tok_row(p, r.sp, h, ci * C + t) + c;
             qc = to_f(q[off]);
             kc = to_f(k[off]);
-            bc = to_f(bg[off]);
+            bc = to_f(sg ? bg[off / p.D] : bg[off]);
             ac = expf(p.g[off]);
         };
         // ---- forward: S'_t into the scratch, u_t into sU
@@ -302,9 +311,19 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
                 sVec[tid] = du;
                 const size_t off = tok_row(p, r.sp, h, ci * C + t) + tid;
                 dv[off] = from_f<Tin>(du * sW[t * D + tid]);
-                dw[off] = from_f<Tin>(du * sV[t * D + tid]);
+                if (!sg) dw[off] = from_f<Tin>(du * sV[t * D + tid]);
+                else {
+                    const float x = warp_total(du * sV[t * D + tid]);
+                    if (lane == 0) sScal[warp] = x;
+                }
             }
             __syncthreads();
+            if (sg && tid == 0) {
+                float x = 0.f;
+#pragma unroll
+                for (int u = 0; u < NW; ++u) x += sScal[u];
+                dw[tok_row(p, r.sp, h, ci * C + t) / p.D] = from_f<Tin>(x);
+            }
             float pde = 0.f, pdg = 0.f;
 #pragma unroll
             for (int jj = 0; jj < NJ; ++jj) {
@@ -329,8 +348,21 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
                 const size_t off = tok_row(p, r.sp, h, ci * C + t) + c;
                 dq[off] = from_f<Tin>(s4[0]);
                 dk[off] = from_f<Tin>(fmaf(de, bc, s4[1]));
-                db[off] = from_f<Tin>(de * kc);
+                if (!sg) db[off] = from_f<Tin>(de * kc);
+                else {
+                    const float x = warp_total(de * kc);
+                    if (lane == 0) sScal[NW + warp] = x;
+                }
                 a.dg[off] = s4[3];
+            }
+            if (sg) {
+                __syncthreads();
+                if (tid == 0) {
+                    float x = 0.f;
+#pragma unroll
+                    for (int u = 0; u < NW; ++u) x += sScal[NW + u];
+                    db[tok_row(p, r.sp, h, ci * C + t) / p.D] = from_f<Tin>(x);
+                }
             }
         }
     }

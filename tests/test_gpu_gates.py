@@ -119,3 +119,26 @@ def test_kda_and_gated_deltanet_match_their_own_recurrences(cuda_lib):
     assert g.gdn2_sync_status() == 0
     assert_close(o, ro, "f32", "gdn o")
     assert_close(ST, rS, "f32", "gdn S_T")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("x_mean", [-3.0, 2.0])
+def test_native_scalar_gate_backward(cuda_lib, D, x_mean):
+    """bf16 backward with scalar b and w (KDA shape), which the kernels read per token: the same
+    q, k, v, log alpha and S0 gradients as the plain call on the broadcast gates, and db, dw equal
+    to its per-channel gradients summed over the channels.  With x ~ N(+2, 1) every chunk's decay
+    is past the chunk factors' range, so the chain and the gradients run token by token."""
+    B, T, H = 2, 200, 2
+    x = make_inputs(B, T, H, D, D, dtype="bf16", seed=23, with_do=True, x_mean=x_mean)
+    gen = torch.Generator().manual_seed(29)
+    beta = torch.sigmoid(torch.randn(B, T, H, generator=gen)).to(torch.bfloat16)
+    full = beta[..., None].expand(B, T, H, D).contiguous()
+    common = (dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["log_alpha"]))
+    gr = g.gdn2_chunk_bwd_gated(*common, dev(beta), dev(beta), dev(x["S0"]), dev(x["do"]), flags=KDA)
+    pr = g.gdn2_chunk_bwd(*common, dev(full), dev(full), dev(x["S0"]), dev(x["do"]))
+    assert g.gdn2_sync_status() == 0
+    for k in ("dq", "dk", "dv", "dlog_alpha", "dS0"):
+        assert torch.equal(gr[k], pr[k]), k
+    for k in ("db", "dw"):
+        assert gr[k].shape == (B, T, H)
+        assert_close(gr[k].float(), pr[k].float().sum(-1), "bf16", k)
