@@ -474,7 +474,7 @@ def run_ours(args):
             ms_k = time_region(fwd_k, 20, 3, stream) / 20
             assert g.gdn2_sync_status() == 0
             kb = fwd_bytes(B, T, H, D) - B * T * H * 2 * (2 * D - 2) - (B * T * H * (4 * D - 4) if gdec is gsc else 0)
-            # its backward: scalar b and w run natively, a scalar decay is broadcast
+            # its backward: the scalar gates (b, w and, for Gated DeltaNet, the decay) run natively
             wsb = torch.empty(g.gdn2_workspace_size_gated(1, fl, x["q"].dtype, B, T, H, D, D), dtype=torch.uint8,
                               device=dev)
             grk = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),

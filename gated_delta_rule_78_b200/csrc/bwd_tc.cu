@@ -356,7 +356,7 @@ bwd_chain_tc_kernel(const __grid_constant__ ChainMaps maps, const BwdTcArgs a)
                         qv = __bfloat162float(a.q[off]);
                         kv = __bfloat162float(a.k[off]);
                         bv = __bfloat162float(a.pr.bw_scalar ? a.b[(row0 + t) * a.H + hh] : a.b[off]);
-                        gv = a.g[off];
+                        gv = a.pr.g_scalar ? a.g[(row0 + t) * a.H + hh] : a.g[off];
                     }
                     rc.q[c] = qv;
                     rc.k[c] = kv;
@@ -513,6 +513,10 @@ constexpr uint32_t SMEM = USED + 1024;  // slack for the 1024-byte alignment
 constexpr uint32_t SC_TOT = DY + 8192;           // decay group totals [8][D] fp32
 constexpr uint32_t SC_DGP = DY + 16384 + 8192;   // gamma dgamma partials [16][D]
 constexpr uint32_t SC_FIN = DS + 16384;          // factor chain: group sums [8][D], then [4][D] twice
+// scalar decay: no log alpha tile; its region holds g_t of the chunk [64] fp32 and the four lane
+// quarters' partial sums of dlog alpha_t [4][64] fp32
+constexpr uint32_t SGT = GG;
+constexpr uint32_t SDG = GG + 256;
 // full chunks stage dq, dk, db over the reloaded raw q, k, b and dg over v, w for the TMA stores
 // TMEM columns
 constexpr uint32_t TM_Y = 0, TM_DU = 64, TM_YB = 128, TM_DUB = 160, TM_U = 192, TM_DY = 256, TM_PA = 320;
@@ -558,7 +562,10 @@ __device__ __forceinline__ void st_bf(uint8_t *p, float x) { *reinterpret_cast<_
 // kSG: the erase and write gates are one value per (token, head) ([rows, H]): per-token tables
 // replace the b and w tiles, and db_t, dw_t are the per-channel gradients summed over the
 // channels (over the 32 lanes of a warp, then over the four lane quarters).
-template <bool kSG>
+// kGS: the decay is one value per (token, head): g_t is read per token (registers for the
+// folding, a table for the factor chain) instead of as a tile, and dlog alpha_t is the
+// per-channel gradient summed over the channels in the same way.
+template <bool kSG, bool kGS>
 __global__ void __launch_bounds__(grad_tc::kThreads, 1)
 bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 {
@@ -603,7 +610,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     // A task's tile loads, in four parts as their regions free up: part 0 q, k, b, dO, T, P (and
-    // the byte counts of bar_in0 and bar_in1) and part 1 log alpha, from warp 0 during the task
+    // the byte counts of bar_in0 and bar_in1) and part 1 log alpha (per channel), from warp 0 during the task
     // before; part 2 S^T and dS_n^T from warp 1 at the end of the task before, once the staged
     // dq, dk, db have left their tiles; part 3 v and w (bar_in3) from warp 1 during this task's
     // decay folding, once the staged dg has left its tiles.
@@ -611,7 +618,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         const int yy = r.sp.bos + r.ci * C, h = r.h, at = lane & 1;
         if (part == 0) {
             if (lane == 0) {
-                mbar_expect_tx(&bar_in0, (kSG ? 8 : 10) * 8192);
+                mbar_expect_tx(&bar_in0, ((kSG ? 4 : 6) + (kGS ? 0 : 4)) * 8192);
                 mbar_expect_tx(&bar_in1, 6 * 16384);
             }
             __syncwarp();
@@ -626,7 +633,7 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
                 tma_load_2d(sm + (lane == 8 ? TT : PP), lane == 8 ? &maps.tm : &maps.pm, 0, (int)(r.cidx * C), &bar_in1);
             }
         } else if (part == 1) {
-            if (lane < 4) tma_load_3d(sm + GG + lane * 8192, &maps.g, lane * 32, h, yy, &bar_in0);
+            if (!kGS && lane < 4) tma_load_3d(sm + GG + lane * 8192, &maps.g, lane * 32, h, yy, &bar_in0);
         } else if (part == 2) {
             const int sl = (int)(bound_slot(a.pr, r.n, r.h, r.nch, r.ci) * D);
             if (lane < 2) tma_load_2d(sm + SS + at * 16384, &maps.st, at * 64, sl, &bar_in1);
@@ -665,6 +672,14 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
         for (int u = 0; u < 4; ++u)
             ssv[u] = __ldg(reinterpret_cast<const uint4 *>(st_n + (size_t)((tid >> 4) + 32 * u) * D + 8 * dch));
     }
+    float gsv[8];  // kGS: g_t of the folding's 8 tokens (tokens 8 (tid >> 6) ..), in flight likewise
+    if (kGS) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * (tid >> 6) + i;
+            gsv[i] = t < L ? __ldg(a.g + ((size_t)y + t) * a.H + hh) : 0.f;
+        }
+    }
     __nv_bfloat16 *const sBt = reinterpret_cast<__nv_bfloat16 *>(sm + SBW), *const sWt = sBt + 64;
     if (kSG && tid < 128) {  // this chunk's b_t (threads 0-63) and w_t (64-127); seen after the folding's first barrier
         const int t = tid & 63;
@@ -682,9 +697,16 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int t = 8 * g8 + i;
-            gl[i] = (t < L && ch_ok)
-                        ? *reinterpret_cast<const float2 *>(sm + GG + (cp >> 4) * 8192 + sw128(t, (cp & 15) * 8))
-                        : make_float2(0.f, 0.f);
+            if (kGS)
+                gl[i] = (t < L && ch_ok) ? make_float2(gsv[i], gsv[i]) : make_float2(0.f, 0.f);
+            else
+                gl[i] = (t < L && ch_ok)
+                            ? *reinterpret_cast<const float2 *>(sm + GG + (cp >> 4) * 8192 + sw128(t, (cp & 15) * 8))
+                            : make_float2(0.f, 0.f);
+        }
+        if (kGS && cp == 0) {  // the factor chain's table of g_t (the last task read it before its end)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) reinterpret_cast<float *>(sm + SGT)[8 * g8 + i] = gsv[i];
         }
         decay_pair8(gl, eG, emG, tot, cp, g8, sTot);
         if (warp == 1 && pend3) {  // the last task's dg has left v, w's tiles by now: this task's v, w
@@ -944,9 +966,9 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * cg + i;
-            const float gv = (t < L && ch_ok) ? *reinterpret_cast<const float *>(sm + GG + (row >> 5) * 8192 +
-                                                                                  sw128(t, (row & 31) * 4))
-                                              : 0.f;
+            const float gv = !(t < L && ch_ok) ? 0.f
+                             : kGS ? reinterpret_cast<const float *>(sm + SGT)[t]
+                                   : *reinterpret_cast<const float *>(sm + GG + (row >> 5) * 8192 + sw128(t, (row & 31) * 4));
             run2[i >> 3] += gv;
             al[i] = __expf(gv);
         }
@@ -1047,7 +1069,13 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
             if (u > cg) after += sFin[8 * D + u * D + row];
             after += sFin[12 * D + u * D + row];
         }
-        if (full) {
+        if (kGS) {  // dlog alpha_t: sum over this lane quarter's 32 channels; the quarters add up below
+            float pdg[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pdg[i] = (ch_ok && 16 * cg + i < L) ? dG[i] + after : 0.f;
+            warp_sum16(pdg, lane);
+            if (!(lane & 1)) reinterpret_cast<float *>(sm + SDG)[quarter * 64 + 16 * cg + (lane >> 1)] = pdg[0];
+        } else if (full) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 *reinterpret_cast<float *>(sm + VV + (row >> 5) * 8192 + sw128(16 * cg + i, (row & 31) * 4)) =
@@ -1063,12 +1091,21 @@ bwd_grad_kernel(const __grid_constant__ GradMaps maps, const BwdTcArgs a)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (kGS && tid >= 64 && tid < 64 + L) {  // dlog alpha_t: the four lane quarters' sums (warps 2, 3)
+        const float *p4 = reinterpret_cast<const float *>(sm + SDG);
+        const int t = tid - 64;
+        a.dg[((size_t)y + t) * a.H + hh] = p4[t] + p4[64 + t] + p4[128 + t] + p4[192 + t];
+    }
     if (warp == 1) {  // lane 0 owns every bulk store of the block
-        if (lane == 0 && full) {  // dq, dk, db went out before dg was formed
+        if (!kGS && lane == 0 && full) {  // dq, dk, db went out before dg was formed
             for (int bx = 0; bx < a.din / 32; ++bx) tma_store_3d(&maps.dg, sm + VV + bx * 8192, bx * 32, hh, y);
             bulk_commit();
         }
-        if (lane == 0) bulk_wait_read1();  // dq, dk and db are read before S^T and dS_n^T come in
+        // dq, dk and db are read before S^T and dS_n^T come in (kGS: theirs is the last group)
+        if (lane == 0) {
+            if (kGS) bulk_wait_read0();
+            else bulk_wait_read1();
+        }
         __syncwarp();
         if (next >= 0) {
             issue(2, nx);  // S^T, dS_n^T into the freed tiles; v, w wait for dg (next task's folding)
@@ -1193,25 +1230,31 @@ cudaError_t launch_bwd_tc(const Problem &p, const void *d_o, const float *dS_T, 
         const int rows = (int)token_rows(p);
         const uint64_t nchunk = (uint64_t)p.H * chunk_bound(p), nbound = (uint64_t)p.H * (chunk_bound(p) + p.B);
         const bool sg = p.bw_scalar;  // scalar b and w ([rows, H]): no tiles of theirs, db and dw written per token
+        const bool gs = p.g_scalar;   // scalar decay ([rows, H]): likewise log alpha and dlog alpha
         if (!make_map(&maps.q, p.q, false, 1, rows, p.H, p.D) || !make_map(&maps.k, p.k, false, 1, rows, p.H, p.D) ||
             (!sg && !make_map(&maps.b, p.b, false, 1, rows, p.H, p.D)) || !make_map(&maps.v, p.v, false, 1, rows, p.H, p.D) ||
             (!sg && !make_map(&maps.w, p.w, false, 1, rows, p.H, p.D)) || !make_map(&maps.dO, d_o, false, 1, rows, p.H, p.D) ||
-            !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D) ||
+            (!gs && !make_map(&maps.g, p.g, true, 1, rows, p.H, p.D)) ||
             !make_map_2d(&maps.st, a.states, D, nbound * D, 64, D) ||
             !make_map_2d(&maps.dsn, a.dSn, D, nchunk * D, 64, D) ||
             !make_map_2d(&maps.tm, a.Tm, C, nchunk * C, 64, C) || !make_map_2d(&maps.pm, a.Pm, C, nchunk * C, 64, C) ||
             !make_map(&maps.dq, out.dq, false, 1, rows, p.H, p.D) || !make_map(&maps.dk, out.dk, false, 1, rows, p.H, p.D) ||
             (!sg && !make_map(&maps.db, out.db, false, 1, rows, p.H, p.D)) || !make_map(&maps.dv, out.dv, false, 1, rows, p.H, p.D) ||
-            (!sg && !make_map(&maps.dw, out.dw, false, 1, rows, p.H, p.D)) || !make_map(&maps.dg, out.dg, true, 1, rows, p.H, p.D))
+            (!sg && !make_map(&maps.dw, out.dw, false, 1, rows, p.H, p.D)) ||
+            (!gs && !make_map(&maps.dg, out.dg, true, 1, rows, p.H, p.D)))
             return cudaErrorInvalidValue;
-        const void *kern = sg ? reinterpret_cast<const void *>(bwd_grad_kernel<true>)
-                              : reinterpret_cast<const void *>(bwd_grad_kernel<false>);
-        if ((e = set_smem_attr(kern, (int)grad_tc::SMEM)) != cudaSuccess) return e;
         int dev = 0, n_sm = 148;  // persistent: one block per multiprocessor
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
         const int ntask = (int)chunk_bound(p) * p.H;
-        if (sg) bwd_grad_kernel<true><<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
-        else bwd_grad_kernel<false><<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+        auto run = [&](auto kernel) -> cudaError_t {
+            cudaError_t er = set_smem_attr(reinterpret_cast<const void *>(kernel), (int)grad_tc::SMEM);
+            if (er != cudaSuccess) return er;
+            kernel<<<max(1, min(ntask, n_sm)), grad_tc::kThreads, grad_tc::SMEM, s>>>(maps, a);
+            return cudaSuccess;
+        };
+        e = sg ? (gs ? run(bwd_grad_kernel<true, true>) : run(bwd_grad_kernel<true, false>))
+               : (gs ? run(bwd_grad_kernel<false, true>) : run(bwd_grad_kernel<false, false>));
+        if (e != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the chunks that run token by token: their gradients, exact, over what the gradient kernel wrote

@@ -1055,8 +1055,8 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
     TcParams prm{pr.B, pr.T, pr.H, (const __nv_bfloat16 *)pr.q, (const __nv_bfloat16 *)pr.k, (const __nv_bfloat16 *)pr.b,
                  (const __nv_bfloat16 *)pr.w, pr.S0, pr.g, (__nv_bfloat16 *)o, S_T, states, status, pr.cu_seqlens, pr.chunk_off,
                  pr.g_scalar ? 1 : 0, ScanArgs{}, BwdFactors{}};
-    if (bw) {  // the backward's factors: states runs with a per-channel decay and no prologue only
-        if (!states || pr.g_scalar || pr.prologue || scan) return cudaErrorInvalidValue;
+    if (bw) {  // the backward's factors: states runs without the prologue only
+        if (!states || pr.prologue || scan) return cudaErrorInvalidValue;
         prm.bw = *bw;
         const uint64_t nchunk = (uint64_t)pr.H * chunk_bound(pr);
         const uint64_t state_rows = (uint64_t)pr.H * (chunk_bound(pr) + pr.B) * D;  // TMA coordinates are 32-bit
@@ -1080,10 +1080,21 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         kernel<<<grid, kThreads, SMEM_BYTES, s>>>(maps, prm);
         return cudaGetLastError();
     };
+    using T1 = std::true_type;
+    using F1 = std::false_type;
+    using D128 = std::integral_constant<int, 128>;
+    using D64 = std::integral_constant<int, 64>;
     if (scan) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, true>) : run(fwd_tc_kernel<false, 64, 0, true>);
-    if (bw && pr.bw_scalar)  // scalar erase and write gates
-        return din == 128 ? run(fwd_tc_kernel<false, 128, 0, false, true, true>) : run(fwd_tc_kernel<false, 64, 0, false, true, true>);
-    if (bw) return din == 128 ? run(fwd_tc_kernel<false, 128, 0, false, true>) : run(fwd_tc_kernel<false, 64, 0, false, true>);
+    if (bw) {  // a scalar decay, and scalar erase and write gates, read as they are
+        auto by_gate = [&](auto gs, auto dn) -> cudaError_t {
+            constexpr bool kGS = decltype(gs)::value;
+            constexpr int kDin = decltype(dn)::value;
+            if (pr.bw_scalar) return run(fwd_tc_kernel<kGS, kDin, 0, false, true, true>);
+            return run(fwd_tc_kernel<kGS, kDin, 0, false, true>);
+        };
+        if (din == 128) return pr.g_scalar ? by_gate(T1{}, D128{}) : by_gate(F1{}, D128{});
+        return pr.g_scalar ? by_gate(T1{}, D64{}) : by_gate(F1{}, D64{});
+    }
     if (pr.prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
     auto by_pro = [&](auto gs, auto dn) -> cudaError_t {
         constexpr bool kGS = decltype(gs)::value;
@@ -1103,10 +1114,6 @@ cudaError_t launch_fwd_tc(const Problem &pr, void *o, float *S_T, __nv_bfloat16 
         default: return run(fwd_tc_kernel<kGS, kDin, 0>);
         }
     };
-    using T1 = std::true_type;
-    using F1 = std::false_type;
-    using D128 = std::integral_constant<int, 128>;
-    using D64 = std::integral_constant<int, 64>;
     if (din == 128) return pr.g_scalar ? by_pro(T1{}, D128{}) : by_pro(F1{}, D128{});
     return pr.g_scalar ? by_pro(T1{}, D64{}) : by_pro(F1{}, D64{});
 }

@@ -138,6 +138,8 @@ bool pro_any(int flags) { return flags & (GDN2_QK_L2NORM | GDN2_BW_LOGITS); }
 bool bw_native(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_scalar(flags, 1) && gate_scalar(flags, 2); }
 // ... and the bf16 backward, without the prologue (whose backward pass wants per-channel gates)
 bool bw_native_bwd(int flags, gdn2_dtype dt) { return bw_native(flags, dt) && !pro_any(flags); }
+// a scalar decay: the bf16 forward and backward read it as it is (the prologue leaves log alpha alone)
+bool decay_native(int flags, gdn2_dtype dt) { return dt == GDN2_BF16 && gate_scalar(flags, 0); }
 bool pro_fused(int flags, gdn2_dtype dt)
 {
     return dt == GDN2_BF16 && ((gate_full(flags, 1) && gate_full(flags, 2)) || bw_native(flags, dt));
@@ -154,9 +156,9 @@ int pro_gate_mode(int flags, int i)
 struct GatedWs {
     size_t pro[4], off[3], grad[3], core, total;
 };
-// The chunk forward keeps some scalar gates as they are, which then need no broadcast copy:
-// bw_kept (scalar b and w together; in the backward also no full-size gradients of theirs)
-// and decay_kept (a scalar decay, bf16).
+// The chunk kernels keep some scalar gates as they are, which then need no broadcast copy and,
+// in the backward, no full-size gradient: bw_kept (scalar b and w together) and decay_kept (a
+// scalar decay, bf16).
 GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, size_t core_bytes, bool pro_pass,
                  bool bw_kept = false, bool decay_kept = false)
 {
@@ -179,7 +181,7 @@ GatedWs gated_ws(bool bwd, int flags, gdn2_dtype dt, size_t rows, int H, int D, 
     }
     for (int i = 0; i < 3; ++i) {
         l.grad[i] = off;
-        if (bwd && !gate_full(flags, i) && !(bw_kept && i > 0)) off += round256(n * es[i]);
+        if (bwd && !gate_full(flags, i) && !(bw_kept && i > 0) && !(decay_kept && i == 0)) off += round256(n * es[i]);
     }
     l.core = off;
     l.total = off + core_bytes;
@@ -452,8 +454,7 @@ size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int
                                    : 0;
     const bool pro_pass = pro_any(flags) && (which == 1 || !pro_fused(flags, dt));
     return gated_ws(which == 1, flags, dt, (size_t)B * T, H, Dk, core, pro_pass,
-                    which == 0 ? bw_native(flags, dt) : bw_native_bwd(flags, dt),
-                    which == 0 && dt == GDN2_BF16 && gate_scalar(flags, 0))
+                    which == 0 ? bw_native(flags, dt) : bw_native_bwd(flags, dt), decay_native(flags, dt))
         .total;
 }
 
@@ -469,8 +470,9 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
     const bool fused = pro_any(flags) && pro_fused(flags, dt);
     const bool native_bw = bw_native(flags, dt);
+    const bool native_decay = decay_native(flags, dt);
     const GatedWs l = gated_ws(false, flags, dt, (size_t)B * T, H, Dk, 0, pro_any(flags) && !fused, native_bw,
-                               dt == GDN2_BF16 && gate_scalar(flags, 0));
+                               native_decay);
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
@@ -481,7 +483,6 @@ gdn2_status gdn2_chunk_fwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
         return st;
     // a scalar decay, and scalar b and w together, go to the tensor-core forward as they are
     // (one exponential per token; one gate value per token)
-    const bool native_decay = gate_scalar(flags, 0) && dt == GDN2_BF16;
     int expand_flags = native_decay ? (flags & ~GDN2_DECAY_SCALAR) : flags;
     if (native_bw) expand_flags &= ~(GDN2_ERASE_SCALAR | GDN2_WRITE_SCALAR);
     const void *gp[3] = {log_alpha, bq, wq};
@@ -515,11 +516,11 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, dlog_alpha, db, dw)) != GDN2_OK) return st;
     gdn2::Problem p = make_problem(B, T, H, Dk, q, k, v, log_alpha, b, w, S0);
-    // scalar b and w (KDA-shaped) run natively: the kernels read them per token and write db, dw
-    // per token; only a scalar decay is still broadcast
-    const bool nat = bw_native_bwd(flags, dt);
+    // scalar b and w together (KDA-shaped), and a scalar decay, run natively: the kernels read them
+    // per token and write their gradients per token
+    const bool nat = bw_native_bwd(flags, dt), nat_g = decay_native(flags, dt);
     const GatedWs l = gated_ws(true, flags, dt, (size_t)B * T, H, Dk, gdn2::bwd_workspace_bytes(dt, p), pro_any(flags),
-                               nat);
+                               nat, nat_g);
     if (!workspace || ws_bytes < l.total) return GDN2_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
@@ -530,19 +531,22 @@ gdn2_status gdn2_chunk_bwd_gated(int flags, gdn2_dtype dt, int B, int T, int H, 
     p.q = qq;
     p.k = kk;
     const void *gp[3] = {log_alpha, bq, wq};
-    if ((st = expand_gates(flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s, nat)) != GDN2_OK) return st;
+    if ((st = expand_gates(nat_g ? (flags & ~GDN2_DECAY_SCALAR) : flags, dt, l, ws, (size_t)B * T, H, Dk, gp, s,
+                           nat)) != GDN2_OK)
+        return st;
     p.g = static_cast<const float *>(gp[0]);
     p.b = gp[1];
     p.w = gp[2];
     p.bw_scalar = nat;
+    p.g_scalar = nat_g;
     void *grads[3] = {dlog_alpha, db, dw};
-    for (int i = 0; i < 3; ++i)
-        if (!gate_full(flags, i) && !(nat && i > 0)) grads[i] = ws + l.grad[i];  // full-size gradient, reduced below
+    for (int i = 0; i < 3; ++i)  // full-size gradients, reduced below
+        if (!gate_full(flags, i) && !(nat && i > 0) && !(nat_g && i == 0)) grads[i] = ws + l.grad[i];
     gdn2::BwdOut out{dq, dk, dv, grads[1], grads[2], static_cast<float *>(grads[0]), dS0};
     if (gdn2::launch_bwd(dt, p, d_o, dS_T, out, ws + l.core, s) != cudaSuccess) return GDN2_ERR_CUDA;
     void *user[3] = {dlog_alpha, db, dw};
     for (int i = 0; i < 3; ++i) {
-        if (!gate_scalar(flags, i) || (nat && i > 0)) continue;
+        if (!gate_scalar(flags, i) || (nat && i > 0) || (nat_g && i == 0)) continue;
         const bool fp32 = (i == 0) || dt == GDN2_F32;
         if (gdn2::launch_channel_sum(fp32, grads[i], user[i], (size_t)B * T * H, Dk, s) != cudaSuccess)
             return GDN2_ERR_CUDA;

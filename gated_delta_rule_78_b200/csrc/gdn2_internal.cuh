@@ -40,8 +40,10 @@ struct Problem {
     const float *S0;  // may be null
     const int *cu_seqlens = nullptr;
     const int *chunk_off = nullptr;
-    bool g_scalar = false;  // tensor-core forward only: log alpha is [rows, H] (one decay per head)
-    bool bw_scalar = false; // tensor-core forward only: b and w are [rows, H] (one gate value each per head)
+    bool g_scalar = false;  // bf16 tensor-core paths only: log alpha is [rows, H] (one decay per head),
+                            // and in the backward so is dlog alpha
+    bool bw_scalar = false; // bf16 tensor-core paths only: b and w are [rows, H] (one gate value each per
+                            // head), and in the backward so are db and dw
     int prologue = 0;       // tensor-core forward only: kProNorm | kProSigmoid, applied inside the kernel
 };
 

@@ -161,7 +161,7 @@ __device__ __forceinline__ void lane_reduce(float (&v)[N], int lane)
 template <int D>
 struct TokGradSmem {
     static constexpr int NW = D / 32;  // warps per column quarter (32 rows each)
-    static constexpr size_t floats = 4 * (size_t)C * D + (size_t)NW * D + D + 16 * (size_t)D + 2 * NW;
+    static constexpr size_t floats = 4 * (size_t)C * D + (size_t)NW * D + D + 16 * (size_t)D + 3 * NW;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
     float *sRed = sU + C * D;        // [NW][D] partial sums over d_k
     float *sVec = sRed + NW * D;     // [D]     du of the current token
     float *sRow = sVec + D;          // [4 quantities][4 quarters][D]
-    float *sScal = sRow + 16 * D;    // [dw | db][NW] per-warp sums (scalar gates)
+    float *sScal = sRow + 16 * D;    // [dw | db | dlog alpha][NW] per-warp sums (scalar gates)
     const Problem &p = a.p;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c = tid % D, jq = tid / D, j0 = jq * NJ, cw = warp % NW;
@@ -190,8 +190,9 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
     const Tin *bg = (const Tin *)p.b, *wg = (const Tin *)p.w, *dOg = (const Tin *)a.dO;
     Tin *dq = (Tin *)a.dq, *dk = (Tin *)a.dk, *dv = (Tin *)a.dv, *db = (Tin *)a.db, *dw = (Tin *)a.dw;
     // scalar erase and write gates ([rows, H]): b_t, w_t read per token, db_t, dw_t summed over
-    // the channels (the first D threads: a warp shuffle, then the NW warps in shared memory)
-    const bool sg = p.bw_scalar;
+    // the channels (the first D threads: a warp shuffle, then the NW warps in shared memory); a
+    // scalar decay likewise (g_t per token, dlog alpha_t summed over the channels)
+    const bool sg = p.bw_scalar, gs = p.g_scalar;
     auto warp_total = [&](float x) {
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
             qc = to_f(q[off]);
             kc = to_f(k[off]);
             bc = to_f(sg ? bg[off / p.D] : bg[off]);
-            ac = expf(p.g[off]);
+            ac = expf(gs ? p.g[off / p.D] : p.g[off]);
         };
         // ---- forward: S'_t into the scratch, u_t into sU
         for (int t = 0; t < L; ++t) {
@@ -353,15 +354,24 @@ __global__ void __launch_bounds__(4 * D, 1) tok_grad_kernel(const TokGradArgs a)
                     const float x = warp_total(de * kc);
                     if (lane == 0) sScal[NW + warp] = x;
                 }
-                a.dg[off] = s4[3];
+                if (!gs) a.dg[off] = s4[3];
+                else {
+                    const float x = warp_total(s4[3]);
+                    if (lane == 0) sScal[2 * NW + warp] = x;
+                }
             }
-            if (sg) {
+            if (sg || gs) {
                 __syncthreads();
                 if (tid == 0) {
-                    float x = 0.f;
+                    const size_t tr = tok_row(p, r.sp, h, ci * C + t) / p.D;
+                    float x = 0.f, xg = 0.f;
 #pragma unroll
-                    for (int u = 0; u < NW; ++u) x += sScal[NW + u];
-                    db[tok_row(p, r.sp, h, ci * C + t) / p.D] = from_f<Tin>(x);
+                    for (int u = 0; u < NW; ++u) {
+                        x += sScal[NW + u];
+                        xg += sScal[2 * NW + u];
+                    }
+                    if (sg) db[tr] = from_f<Tin>(x);
+                    if (gs) a.dg[tr] = xg;
                 }
             }
         }

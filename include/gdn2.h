@@ -241,9 +241,12 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
  * needhelp.icu write-up's generalisation hierarchy).  Absent b or w gives the
  * write-only and erase-only ablations of the aixai.ru post ("Абляции").
  * The results are identical to the plain calls made with the gates broadcast to
- * per-channel tensors: the library broadcasts them into the workspace and runs the
- * same kernels.  In the backward the gradient of a scalar gate is the sum of the
- * per-channel gradients over the channels.  An absent gate's gradient pointer is
+ * per-channel tensors.  In the bf16 calls the chunk kernels read a scalar decay, and
+ * scalar b and w together (without the prologue flags, in the backward), as they are, one
+ * value per token; every other scalar or absent gate is broadcast into the workspace
+ * first.  In the backward the gradient of a scalar gate is the sum of the per-channel
+ * gradients over the channels (the order of that sum, so its last bits, depends on which
+ * of the two routes ran); the other gradients are identical.  An absent gate's gradient pointer is
  * ignored (NULL allowed).  Flags outside the eight below, or scalar and absent set
  * for one gate, give GDN2_ERR_UNSUPPORTED.
  * Workspace: gdn2_workspace_size_gated(which, flags, ...) with which = 0 (forward),

@@ -125,10 +125,16 @@ def test_gated_flags_and_workspace(lib):
     assert lib.gdn2_workspace_size_gated(0, g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == one
     assert lib.gdn2_workspace_size_gated(0, g.DECAY_NONE, BF16, 2, 128, 4, 128, 128) == 2 * one
     plain = lib.gdn2_workspace_size(1, BF16, 2, 128, 4, 128, 128)
-    # scalar b and w together run natively in the bf16 backward (no broadcast gates, no full-size
-    # gate gradients); a scalar b alone, or fp32, is broadcast and its gradient summed back
+    # scalar b and w together, and a scalar decay, run natively in the bf16 backward (no broadcast
+    # gates, no full-size gate gradients); a scalar b alone, or fp32, is broadcast and its
+    # gradient summed back
     assert lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR | g.WRITE_SCALAR, BF16, 2, 128, 4, 128, 128) == plain
     assert lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == plain + 2 * one
+    assert lib.gdn2_workspace_size_gated(1, g.DECAY_SCALAR, BF16, 2, 128, 4, 128, 128) == plain
+    gdn = g.DECAY_SCALAR | g.ERASE_SCALAR | g.WRITE_SCALAR
+    assert lib.gdn2_workspace_size_gated(1, gdn, BF16, 2, 128, 4, 128, 128) == plain
+    assert lib.gdn2_workspace_size_gated(1, g.DECAY_SCALAR, F32, 2, 128, 4, 128, 128) == \
+        lib.gdn2_workspace_size(1, F32, 2, 128, 4, 128, 128) + 2 * 2 * one  # fp32: g and dg, 4 bytes each
     plain32 = lib.gdn2_workspace_size(1, F32, 2, 128, 4, 128, 128)
     assert (lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR | g.WRITE_SCALAR, F32, 2, 128, 4, 128, 128)
             == plain32 + 4 * 2 * one)

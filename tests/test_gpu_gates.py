@@ -142,3 +142,39 @@ def test_native_scalar_gate_backward(cuda_lib, D, x_mean):
     for k in ("db", "dw"):
         assert gr[k].shape == (B, T, H)
         assert_close(gr[k].float(), pr[k].float().sum(-1), "bf16", k)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("shift", [-3.0, 2.0])
+@pytest.mark.parametrize("bw", ["channel", "scalar"])
+def test_native_scalar_decay_backward(cuda_lib, D, shift, bw):
+    """bf16 backward with a scalar decay, which the kernels read per token: the same q, k, v and
+    S0 gradients (and b, w gradients where those are per channel) as the plain call on the
+    broadcast decay, and dlog alpha equal to its per-channel gradient summed over the channels.
+    log alpha_t = -softplus(x), x ~ N(shift, 1): at shift +2 every chunk's decay (about -135) is
+    past the chunk factors' range, so the chain and the gradients run token by token."""
+    B, T, H = 2, 200, 2
+    x = make_inputs(B, T, H, D, D, dtype="bf16", seed=31, with_do=True)
+    gen = torch.Generator().manual_seed(37)
+    la = -torch.nn.functional.softplus(torch.randn(B, T, H, generator=gen) + shift)
+    la_full = la[..., None].expand(B, T, H, D).contiguous()
+    flags = g.DECAY_SCALAR
+    b, w, b_full, w_full = x["b"], x["w"], x["b"], x["w"]
+    if bw == "scalar":  # Gated DeltaNet: scalar beta for both gates too
+        flags |= g.ERASE_SCALAR | g.WRITE_SCALAR
+        b = w = torch.sigmoid(torch.randn(B, T, H, generator=gen)).to(torch.bfloat16)
+        b_full = w_full = b[..., None].expand(B, T, H, D).contiguous()
+    common = (dev(x["q"]), dev(x["k"]), dev(x["v"]))
+    gr = g.gdn2_chunk_bwd_gated(*common, dev(la), dev(b), dev(w), dev(x["S0"]), dev(x["do"]), flags=flags)
+    pr = g.gdn2_chunk_bwd(*common, dev(la_full), dev(b_full), dev(w_full), dev(x["S0"]), dev(x["do"]))
+    assert g.gdn2_sync_status() == 0
+    for k in ("dq", "dk", "dv", "dS0"):
+        assert torch.equal(gr[k], pr[k]), k
+    assert gr["dlog_alpha"].shape == (B, T, H)
+    assert_close(gr["dlog_alpha"], pr["dlog_alpha"].sum(-1), "f32", "dlog_alpha")
+    for k in ("db", "dw"):
+        if bw == "scalar":
+            assert gr[k].shape == (B, T, H)
+            assert_close(gr[k].float(), pr[k].float().sum(-1), "bf16", k)
+        else:
+            assert torch.equal(gr[k], pr[k]), k
