@@ -29,12 +29,14 @@ __device__ __forceinline__ void scale_fma(float2 &s, float a) { s.x *= a; s.y *=
 __device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
 
 // kPro: the fused input prologue (kProNorm | kProSigmoid of gdn2_internal.cuh): q and k are
-// L2-normalised in the block before use, b and w pass through the sigmoid.
+// L2-normalised in the block before use, b and w pass through the sigmoid.  `modes` gives each
+// gate's layout (two bits each, kGate* of gdn2_internal.cuh): a scalar gate is read once per
+// (sequence, head) and used for every channel, an absent one is not read.
 template <int D, typename Tin, int kPro>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const Tin *__restrict__ b, const Tin *__restrict__ w,
-              float *__restrict__ S, Tin *__restrict__ o)
+              float *__restrict__ S, Tin *__restrict__ o, int modes)
 {
     constexpr int CPT = D / 32;      // columns per lane
     constexpr int RPW = D / kWarps;  // rows per warp
@@ -48,6 +50,10 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
     const size_t nh = blockIdx.x;
     const size_t vec = nh * D;
     float *Sp = S + nh * D * D;
+    const int mg = modes & 3, mb = (modes >> 2) & 3, mw = (modes >> 4) & 3;
+    // element of each gate this thread reads (tid < D): its channel, or the (sequence, head) scalar
+    const size_t g_at = mg == kGateScalar ? nh : vec + tid, b_at = mb == kGateScalar ? nh : vec + tid,
+                 w_at = mw == kGateScalar ? nh : vec + tid;
 
     // issue the state loads first: they are the long pole
     V sv[RPW];
@@ -70,7 +76,7 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
                 s_nrm[warp][1] = sk;
             }
         }
-        s_a[tid] = expf(g[vec + tid]);
+        s_a[tid] = expf(mg == kGateAbsent ? 0.f : g[g_at]);
         s_q[tid] = qv;
         s_k[tid] = kv;
     }
@@ -86,7 +92,7 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
             s_q[tid] = qv;
             s_k[tid] = kv;
         }
-        const float bv = to_f(b[vec + tid]);
+        const float bv = mb == kGateAbsent ? 1.f : to_f(b[b_at]);
         s_e[tid] = ((kPro & kProSigmoid) ? sigmoid(bv) : bv) * kv;
     }
     __syncthreads();
@@ -116,7 +122,7 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
         float r = 0.f, pq = 0.f;
 #pragma unroll
         for (int wi = 0; wi < kWarps; ++wi) { r += s_r[wi][tid]; pq += s_p[wi][tid]; }
-        const float wv = to_f(w[vec + tid]);
+        const float wv = mw == kGateAbsent ? 1.f : to_f(w[w_at]);
         const float u = ((kPro & kProSigmoid) ? sigmoid(wv) : wv) * to_f(v[vec + tid]) - r;
         s_u[tid] = u;
         o[vec + tid] = from_f<Tin>(pq + s_kq * u);
@@ -138,11 +144,11 @@ decode_kernel(int H, const Tin *__restrict__ q, const Tin *__restrict__ k, const
 
 template <int D, typename Tin>
 cudaError_t launch_t(int N, int H, const void *q, const void *k, const void *v, const float *g,
-                     const void *b, const void *w, float *S, void *o, int pro, cudaStream_t s)
+                     const void *b, const void *w, float *S, void *o, int pro, int modes, cudaStream_t s)
 {
     auto go = [&](auto kernel) {
         kernel<<<N * H, kWarps * 32, 0, s>>>(H, (const Tin *)q, (const Tin *)k, (const Tin *)v, g, (const Tin *)b,
-                                             (const Tin *)w, S, (Tin *)o);
+                                             (const Tin *)w, S, (Tin *)o, modes);
         return cudaGetLastError();
     };
     switch (pro) {
@@ -157,14 +163,17 @@ cudaError_t launch_t(int N, int H, const void *q, const void *k, const void *v, 
 
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
-                          void *o, cudaStream_t s, int prologue)
+                          void *o, cudaStream_t s, int prologue, int gate_modes)
 {
     if (prologue & ~(kProNorm | kProSigmoid)) return cudaErrorInvalidValue;
+    for (int i = 0; i < 3; ++i)
+        if (((gate_modes >> (2 * i)) & 3) > kGateAbsent) return cudaErrorInvalidValue;
+    if (gate_modes >> 6) return cudaErrorInvalidValue;
     if (dt == GDN2_F32)
-        return D == 64 ? launch_t<64, float>(N, H, q, k, v, g, b, w, S, o, prologue, s)
-                       : launch_t<128, float>(N, H, q, k, v, g, b, w, S, o, prologue, s);
-    return D == 64 ? launch_t<64, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, s)
-                   : launch_t<128, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, s);
+        return D == 64 ? launch_t<64, float>(N, H, q, k, v, g, b, w, S, o, prologue, gate_modes, s)
+                       : launch_t<128, float>(N, H, q, k, v, g, b, w, S, o, prologue, gate_modes, s);
+    return D == 64 ? launch_t<64, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, gate_modes, s)
+                   : launch_t<128, __nv_bfloat16>(N, H, q, k, v, g, b, w, S, o, prologue, gate_modes, s);
 }
 
 }  // namespace gdn2

@@ -446,7 +446,7 @@ size_t gdn2_workspace_size_gated(int which, int flags, gdn2_dtype dt, int B, int
     if (which == 2) {  // decode: B sequences of one token (the prologue is fused for per-channel b and w)
         if (check_sizes(dt, B, 1, H, Dk, Dv) != GDN2_OK) return 0;
         const bool fused = gate_full(flags, 1) && gate_full(flags, 2);
-        return gated_ws(false, flags, dt, (size_t)B, H, Dk, 0, pro_any(flags) && !fused).total;
+        return gated_ws(false, flags, dt, (size_t)B, H, Dk, 0, pro_any(flags) && !fused, true, true).total;
     }
     if (check_sizes(dt, B, T, H, Dk, Dv) != GDN2_OK || T == 0 || (which != 0 && which != 1)) return 0;
     const size_t core = which == 1 ? gdn2::bwd_workspace_bytes(dt, make_problem(B, T, H, Dk, nullptr, nullptr, nullptr,
@@ -567,9 +567,10 @@ gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int H, int D
     if ((st = check_sizes(dt, N, 1, H, Dk, Dv)) != GDN2_OK) return st;
     if ((st = check_ptrs({q, k, v, S, o}, {})) != GDN2_OK) return st;
     if ((st = check_gate_ptrs(flags, log_alpha, b, w)) != GDN2_OK) return st;
-    // the prologue runs inside the decode kernel when b and w are per channel
+    // the prologue runs inside the decode kernel when b and w are per channel; the kernel reads
+    // every gate layout as it is (nothing is broadcast)
     const bool fused = pro_any(flags) && gate_full(flags, 1) && gate_full(flags, 2);
-    const GatedWs l = gated_ws(false, flags, dt, (size_t)N, H, Dk, 0, pro_any(flags) && !fused);
+    const GatedWs l = gated_ws(false, flags, dt, (size_t)N, H, Dk, 0, pro_any(flags) && !fused, true, true);
     if (l.total > 0 && (!workspace || ws_bytes < l.total)) return GDN2_ERR_WORKSPACE;
     if (l.total > 0 && !aligned16(workspace)) return GDN2_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
@@ -578,12 +579,13 @@ gdn2_status gdn2_decode_step_gated(int flags, gdn2_dtype dt, int N, int H, int D
     if (pro_any(flags) && !fused &&
         (st = prologue_pass(flags, dt, l, ws, (size_t)N, H, Dk, qq, kk, bq, wq, s)) != GDN2_OK)
         return st;
-    const void *gp[3] = {log_alpha, bq, wq};
-    if ((st = expand_gates(flags, dt, l, ws, (size_t)N, H, Dk, gp, s)) != GDN2_OK) return st;
+    int modes = 0;
+    for (int i = 0; i < 3; ++i)
+        modes |= (gate_scalar(flags, i) ? gdn2::kGateScalar : gate_none(flags, i) ? gdn2::kGateAbsent : gdn2::kGateChannel)
+                 << (2 * i);
     const int pro = fused ? ((flags & GDN2_QK_L2NORM) ? gdn2::kProNorm : 0) | ((flags & GDN2_BW_LOGITS) ? gdn2::kProSigmoid : 0)
                           : 0;
-    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, qq, kk, v, static_cast<const float *>(gp[0]), gp[1], gp[2], S, o,
-                                         s, pro));
+    return from_cuda(gdn2::launch_decode(dt, N, H, Dk, qq, kk, v, log_alpha, bq, wq, S, o, s, pro, modes));
 }
 
 gdn2_status gdn2_prologue(int flags, gdn2_dtype dt, int N, int H, int D, const void *q, const void *k, const void *b,

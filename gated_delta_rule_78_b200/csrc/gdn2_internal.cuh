@@ -213,9 +213,12 @@ cudaError_t launch_fwd_tc(const Problem &p, void *o, float *S_T, __nv_bfloat16 *
                           cudaStream_t s,
                           const ScanArgs *scan = nullptr, const BwdFactors *bw = nullptr);
 
+// gate_modes: two bits per gate (log alpha, b, w from bit 0 up): kGateChannel (one value per
+// channel), kGateScalar (one per sequence and head), kGateAbsent (log alpha 0, b and w 1)
+constexpr int kGateChannel = 0, kGateScalar = 1, kGateAbsent = 2;
 cudaError_t launch_decode(gdn2_dtype dt, int N, int H, int D, const void *q, const void *k,
                           const void *v, const float *g, const void *b, const void *w, float *S,
-                          void *o, cudaStream_t s, int prologue = 0);
+                          void *o, cudaStream_t s, int prologue = 0, int gate_modes = 0);
 
 struct BwdOut {
     void *dq, *dk, *dv, *db, *dw;

@@ -241,10 +241,10 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
  * needhelp.icu write-up's generalisation hierarchy).  Absent b or w gives the
  * write-only and erase-only ablations of the aixai.ru post ("Абляции").
  * The results are identical to the plain calls made with the gates broadcast to
- * per-channel tensors.  In the bf16 calls the chunk kernels read a scalar decay, and
- * scalar b and w together (without the prologue flags, in the backward), as they are, one
- * value per token; every other scalar or absent gate is broadcast into the workspace
- * first.  In the backward the gradient of a scalar gate is the sum of the per-channel
+ * per-channel tensors.  The decode step reads every layout as it is.  In the bf16 chunk
+ * calls the kernels read a scalar decay, and scalar b and w together (without the prologue
+ * flags, in the backward), as they are, one value per token; every other scalar or absent
+ * gate of the chunk calls is broadcast into the workspace first.  In the backward the gradient of a scalar gate is the sum of the per-channel
  * gradients over the channels (the order of that sum, so its last bits, depends on which
  * of the two routes ran); the other gradients are identical.  An absent gate's gradient pointer is
  * ignored (NULL allowed).  Flags outside the eight below, or scalar and absent set

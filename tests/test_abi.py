@@ -138,7 +138,9 @@ def test_gated_flags_and_workspace(lib):
     plain32 = lib.gdn2_workspace_size(1, F32, 2, 128, 4, 128, 128)
     assert (lib.gdn2_workspace_size_gated(1, g.ERASE_SCALAR | g.WRITE_SCALAR, F32, 2, 128, 4, 128, 128)
             == plain32 + 4 * 2 * one)
-    assert lib.gdn2_workspace_size_gated(2, g.ERASE_SCALAR, BF16, 8, 0, 4, 128, 128) == 8 * 4 * 128 * 2
+    # the decode kernel reads every gate layout as it is: no workspace without the prologue
+    for fl in (g.ERASE_SCALAR, g.DECAY_SCALAR | g.ERASE_SCALAR | g.WRITE_SCALAR, g.DECAY_NONE | g.WRITE_NONE):
+        assert lib.gdn2_workspace_size_gated(2, fl, BF16, 8, 0, 4, 128, 128) == 0
     # input prologue: fused in the bf16 forward with per-channel gates (no workspace); a pass
     # into the workspace (q_n, k_n, b_s, w_s) everywhere else
     pro = g.QK_L2NORM | g.BW_LOGITS
@@ -149,10 +151,10 @@ def test_gated_flags_and_workspace(lib):
     # scalar b logits: q_n, k_n, per-token b_s, w_s, then the broadcast b
     assert lib.gdn2_workspace_size_gated(0, pro | g.ERASE_SCALAR, BF16, 2, 128, 4, 128, 128) == 4 * one + 2 * 128 * 4 * 2
     # decode: fused for per-channel b and w; a scalar b logit goes through the pass
-    # (q_n, k_n, w_s per channel, b_s per token, then the broadcast b)
+    # (q_n, k_n, w_s per channel, b_s per token, which the kernel then reads as it is)
     assert lib.gdn2_workspace_size_gated(2, g.QK_L2NORM, BF16, 8, 0, 4, 128, 128) == 0
     assert lib.gdn2_workspace_size_gated(2, pro | g.ERASE_SCALAR, BF16, 8, 0, 4, 128, 128) == \
-        3 * 8 * 4 * 128 * 2 + 256 + 8 * 4 * 128 * 2
+        3 * 8 * 4 * 128 * 2 + 256
 
 
 def test_workspace_size(lib):

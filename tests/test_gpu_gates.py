@@ -87,10 +87,13 @@ def test_gated_backward_equals_broadcast_plain_backward(cuda_lib, dtype, D, name
             assert torch.equal(gr[gk], pr[gk]), (name, gk)
 
 
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
 @pytest.mark.parametrize("name,flags", CASES)
-def test_gated_decode_equals_broadcast_plain_decode(cuda_lib, name, flags):
-    N, H, D = 8, 2, 128
-    x, gates, full = gated_inputs(N, 1, H, D, "bf16", flags, seed=17)
+def test_gated_decode_equals_broadcast_plain_decode(cuda_lib, dtype, D, name, flags):
+    """The decode kernel reads scalar and absent gates as they are (no broadcast): bit for bit
+    the plain step on the broadcast gates."""
+    N, H = 8, 2
+    x, gates, full = gated_inputs(N, 1, H, D, dtype, flags, seed=17)
     sq = lambda t: None if t is None else t[:, 0].contiguous().cuda()
     S1 = x["S0"].clone().cuda()
     S2 = x["S0"].clone().cuda()
