@@ -114,6 +114,22 @@ def fwd_g(lib, flags, g=P, b=P, w=P, ws=P, ws_bytes=1 << 40):
     return lib.gdn2_chunk_fwd_gated(flags, BF16, 1, 64, 1, 128, 128, P, P, P, g, b, w, NUL, P, NUL, ws, ws_bytes, S)
 
 
+def dec_g(lib, flags, g=P, b=P, w=P, ws=NUL, ws_bytes=0):
+    return lib.gdn2_decode_step_gated(flags, BF16, 1, 1, 128, 128, P, P, P, g, b, w, P, P, ws, ws_bytes, S)
+
+
+def test_gated_decode_invalid_arguments_return_status(lib):
+    """Every case returns before a launch (the pointers are stand-ins)."""
+    assert dec_g(lib, 256) == -8                              # unknown flag bit
+    assert dec_g(lib, g.DECAY_SCALAR | g.DECAY_NONE) == -8    # scalar and absent for one gate
+    assert dec_g(lib, g.ERASE_SCALAR, b=NUL) == -1            # a scalar gate needs its tensor
+    assert dec_g(lib, g.DECAY_SCALAR, g=MIS) == -4
+    assert dec_g(lib, 0, w=NUL) == -1                         # so does a per-channel one
+    # the prologue as a pass (scalar b logits) needs a workspace; per-channel b, w fuse it
+    assert dec_g(lib, g.BW_LOGITS | g.ERASE_SCALAR) == -5
+    assert dec_g(lib, g.BW_LOGITS | g.ERASE_SCALAR, ws=MIS, ws_bytes=1 << 20) == -4
+
+
 def test_gated_flags_and_workspace(lib):
     assert fwd_g(lib, 256) == -8                      # unknown flag bit
     assert fwd_g(lib, g.ERASE_SCALAR | g.ERASE_NONE) == -8  # scalar and absent for one gate
