@@ -250,7 +250,9 @@ GDN2_API gdn2_status gdn2_chunk_bwd_varlen(gdn2_dtype dt, int N, int total_T, in
  * ignored (NULL allowed).  Flags outside the eight below, or scalar and absent set
  * for one gate, give GDN2_ERR_UNSUPPORTED.
  * Workspace: gdn2_workspace_size_gated(which, flags, ...) with which = 0 (forward),
- * 1 (backward), 2 (decode; B = N, T ignored).  Fixed-length batches only.
+ * 1 (backward), 2 (decode; B = N, T ignored).  Where it returns 0 the call needs no
+ * workspace (NULL allowed): the decode step without the prologue pass, and the bf16
+ * forward whose gates the kernels read as they are.  Fixed-length batches only.
  *
  * Input prologue (two more flags, combinable with the layouts above).  The aixai.ru
  * post's architecture paragraph normalises queries and keys before the recurrent update
