@@ -199,3 +199,20 @@ def test_decode_prologue_variants(cuda_lib, dtype, flags):
         assert_close(o, ro, dtype, "o")
     assert g.gdn2_sync_status() == 0
     assert_close(S, Sr, dtype, "S")
+
+
+def test_backward_scalar_decay_with_prologue(cuda_lib):
+    """Raw q, k and gate logits with a scalar decay: the prologue runs as a pass, the kernels read
+    log alpha per token, and dlog alpha is the per-channel gradient summed over the channels."""
+    B, T, H, D = 1, 130, 2, 128
+    x = raw_inputs(B, T, H, D, "bf16", seed=43)
+    la = -torch.nn.functional.softplus(torch.randn(B, T, H, generator=torch.Generator().manual_seed(13)) - 3.0)
+    gr = g.gdn2_chunk_bwd_gated(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(la), dev(x["b"]), dev(x["w"]),
+                                dev(x["S0"]), dev(x["do"]), flags=PRO | g.DECAY_SCALAR)
+    assert g.gdn2_sync_status() == 0
+    ref = oracle.ref_bwd_prologue(x["q"], x["k"], x["v"], la[..., None].expand(B, T, H, D), x["b"], x["w"],
+                                  x["S0"], x["do"])
+    for gk, rk in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("db", "db"), ("dw", "dw"), ("dS0", "dS0")):
+        assert_close(gr[gk], ref[rk], "bf16", gk)
+    assert gr["dlog_alpha"].shape == (B, T, H)
+    assert_close(gr["dlog_alpha"], ref["dg"].sum(-1), "bf16", "dlog_alpha (scalar)")
