@@ -24,7 +24,10 @@ steps) and the roofline fraction of each, plus:
   (256 ... 8192, seeded), through gdn2_chunk_fwd_varlen / gdn2_chunk_bwd_varlen;
 * `scalar_decay`: the headline batch with one log decay per (token, head) through
   gdn2_chunk_fwd_gated (the tensor-core forward's scalar-decay path);
-* `d64`: the same model width with head size 64 (H = 32);
+* `kda`, `gated_deltanet`: the headline batch with scalar b = w = beta (and, for Gated
+  DeltaNet, a scalar decay) through the gated forward and backward, whose kernels read the
+  scalar gates as they are;
+* `d64`: the same model width with head size 64 (H = 32), forward and backward;
 * `prologue`: raw q, k and gate logits, with the input prologue (L2-normalised q, k;
   sigmoid b, w) fused into the tensor-core forward, against the same prologue run as a
   separate pass (gdn2_prologue) before the plain forward.
